@@ -1,0 +1,189 @@
+/*
+ * tern.h -- C ABI of libterngemv.so: packed-ternary linear layers and the int8 output head on
+ * NVIDIA B200 (sm_100a).
+ *
+ * Sources, cited by page and section heading:
+ *   [R] PyTorchKR review "Fermion Research, 3진 계열 포맷으로 직접 학습한 Neutrino-1 모델군 3종 공개"
+ *       (discuss.pytorch.kr/t/11456);
+ *   [A] aiatolah.com, "Neutrino-1 8B: modelo ternario de 3,88 GB roda em GPU e laptop";
+ *   [O] origotech.dev, "더 적은 비트로 계산하기" (lowbit explainer).
+ *
+ * What the library computes
+ *   A linear layer's output feature is a sum of weight x activation terms, y_j = sum_i w_ij x_i
+ *   ([R] "학습 중에 포맷이 있어야 하는 이유", displayed equation). Here w_ij = scale_j * t_ij with a
+ *   trit t in {-1, 0, +1}, so each term is an add, a skip or a subtract ([O] Figure I). Weights stay
+ *   packed at rest and are decoded inside the matrix kernels; no fp16/fp32 weight copy is ever
+ *   made ([A] second paragraph and "Formato unico, tres portas"). The transport form of the
+ *   ternary lane expands bit-exactly into the packed container ([R] "3진 계열이라는 이름의 실체";
+ *   [A] "Formato unico"); embeddings and the output head stay int8 ([R] same section).
+ *
+ * Conventions (every entry point)
+ *   - Every pointer named *_dev is device memory owned by the caller; the library keeps no
+ *     reference after the call returns and allocates no device memory.
+ *   - Work is enqueued asynchronously on `stream` (NULL = the legacy default stream); nothing
+ *     synchronises except tern_read_flag.
+ *   - Argument errors are returned before anything is enqueued. A launch error is returned as
+ *     TERN_ECUDA (the CUDA error is left to cudaGetLastError-style inspection by the caller).
+ *   - Data errors that only the device can see (a trit outside {-1,0,+1}, a transport byte above
+ *     242) set *err_flag_dev to a nonzero value; read it with tern_read_flag. Kernels never trap and
+ *     never wait without a bound.
+ *   - Outputs are deterministic: the same inputs give the same bits on every run.
+ *
+ * Packed layout (this library's own; the pages' FV5 bit-planes are only partly described)
+ *   Matrix N x K, K a multiple of 128. Row n occupies K/16 uint32 words at word offset n*K/16:
+ *     words [0, K/32)     nonzero-mask plane, bit = (t != 0)
+ *     words [K/32, K/16)  sign plane,         bit = (t == -1)   (0 wherever the mask bit is 0)
+ *   Trit k of the row sits in word k/32 of each plane. With j = k % 32:
+ *     mask bit position  p(j) = 16*(j % 2) + (j / 16) + 2*((j % 16) / 2)
+ *     sign bit position  (p(j) + 1) % 32
+ *   i.e. the sign plane is the mask plane's bit order rotated by one. This order lets a kernel
+ *   merge one mask word and one sign word into two words of sixteen 2-bit two's-complement
+ *   fields (m in the low bit, s in the high bit) and read a field placed in the top two bits of
+ *   a byte as the int8 value 64*t, or in the top two bits of a half-word as the bf16 value
+ *   2.0*t, with one shift and one AND. Per-row scales are a separate fp16[N] array.
+ *   Packed size: N*K/4 bytes of planes + 2*N bytes of scales.
+ *
+ * Transport layout (base 3, fixed rate)
+ *   Row n occupies ceil(K/5) bytes at byte offset n*ceil(K/5). Byte j of a row holds trits
+ *   5j..5j+4 as b = d0 + 3*d1 + 9*d2 + 27*d3 + 81*d4 with d_i = t_(5j+i) + 1. Trits past the end of
+ *   the row are written as t = 0 (d = 1) and ignored on reading; bytes 243..255 are invalid.
+ */
+#ifndef TERN_H_
+#define TERN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; declared here so that this header needs no CUDA header. */
+typedef struct CUstream_st* tern_stream_t;
+
+typedef enum {
+  TERN_OK = 0,
+  TERN_EINVAL = 1,    /* null pointer, unknown enum value, misaligned pointer, bad flags      */
+  TERN_ESHAPE = 2,    /* N <= 0, K <= 0, K % 128 != 0, M out of range, size overflow          */
+  TERN_EBADCODE = 3,  /* device saw an invalid trit / transport byte (via the error flag)     */
+  TERN_ECUDA = 4,     /* a CUDA runtime call or kernel launch failed                          */
+  TERN_ETIMEOUT = 5   /* a bounded device-side wait gave up (reserved: no kernel here waits)  */
+} tern_status;
+
+typedef enum { TERN_ACT_BF16 = 0, TERN_ACT_INT8 = 1 } tern_act;
+typedef enum { TERN_SRC_INT8_TRITS = 0, TERN_SRC_BASE3 = 1 } tern_src;
+
+/* Launch flags for the *_ex entry points.
+ * TERN_FLAG_PDL: launch with programmatic dependent launch. The kernel may start while the
+ *   previous kernel on the stream is still running; it reads weights before waiting for that
+ *   kernel, and reads activations / writes outputs only after. Only valid when the weight
+ *   buffers are not written by work still in flight on the stream (true in a decode loop). */
+#define TERN_FLAG_PDL 1u
+
+/* A packed ternary matrix: views of caller-owned device memory. */
+typedef struct {
+  int32_t N;                  /* rows (output features), > 0                                */
+  int32_t K;                  /* columns (input features), > 0, multiple of 128             */
+  const uint32_t* planes;     /* device, N*K/16 words in the packed layout, 16-byte aligned */
+  const uint16_t* scale_f16;  /* device, N fp16 bit patterns (per-row scale)                */
+} tern_matrix;
+
+/* Human-readable name of a status code (static string). */
+const char* tern_status_string(tern_status s);
+
+/* Bytes of packed planes for an N x K matrix (N*K/4); 0 if the shape is invalid. */
+size_t tern_packed_bytes(int32_t N, int32_t K);
+
+/* Bytes of the base-3 transport for an N x K matrix (N*ceil(K/5)); 0 if the shape is invalid. */
+size_t tern_base3_bytes(int32_t N, int32_t K);
+
+/* Pack a ternary matrix into the planes layout (the loader step: weights packed at rest, [A]).
+ *   src = TERN_SRC_INT8_TRITS: src_dev is int8[N][K] row-major with values in {-1, 0, +1}.
+ *   src = TERN_SRC_BASE3:      src_dev is the transport, uint8[N][ceil(K/5)] (layout above); it is
+ *                              expanded bit-exactly ([R] "3진 계열이라는 이름의 실체").
+ *   planes_dev: output, N*K/16 uint32 words, 16-byte aligned.
+ *   err_flag_dev: int32 on the device; cleared by this call on the stream, then set nonzero if
+ *   any input value is invalid (the planes are then unspecified). Required. */
+tern_status tern_pack(tern_src src, const void* src_dev, int32_t N, int32_t K, uint32_t* planes_dev,
+                      int32_t* err_flag_dev, tern_stream_t stream);
+
+/* Encode dense trits int8[N][K] into the base-3 transport uint8[N][ceil(K/5)] (the inverse of
+ * tern_pack with TERN_SRC_BASE3). err_flag_dev as for tern_pack. */
+tern_status tern_base3_encode(const int8_t* trits_dev, int32_t N, int32_t K, uint8_t* out_dev,
+                              int32_t* err_flag_dev, tern_stream_t stream);
+
+/* Per-row occupancy of a packed matrix ([R] "출하된 컨테이너를 직접 읽기": zero / +1 / -1
+ * fractions of each tensor). counts_dev: int64[N][3] = {zeros, plus_ones, minus_ones}. */
+tern_status tern_occupancy(const tern_matrix* W, int64_t* counts_dev, tern_stream_t stream);
+
+/* Per-token absmax int8 quantisation of bf16 activations (the int8-activation runtime of
+ * [R] "토큰 동일성의 경계"): for each of the M rows of x (bf16 bits, M x K row-major),
+ *   s_x = absmax / 127 (fp32 division),  q = clamp(rint(x / s_x), -127, 127)  (fp32 division,
+ *   round half to even); an all-zero row gives s_x = 0 and q = 0. Finite inputs.
+ * q_dev: int8[M][K]; s_x_dev: float[M]. 1 <= M <= 4096, K % 128 == 0. */
+tern_status tern_quantize_act(const uint16_t* x_bf16_dev, int32_t M, int32_t K, int8_t* q_dev,
+                              float* s_x_dev, tern_stream_t stream);
+
+/* M = 1 ternary GEMV: y[n] = scale[n] * sum_k t[n][k] * x[k]  ([R] "학습 중에 포맷이 있어야 하는
+ * 이유"; [O] Figure I).
+ *   act = TERN_ACT_BF16: x_dev = bf16[K] (bit patterns); x_scale_dev ignored (may be NULL).
+ *                        Products are exact, accumulation is fp32 on the tensor cores.
+ *   act = TERN_ACT_INT8: x_dev = int8[K] from tern_quantize_act, x_scale_dev = &s_x (device).
+ *                        acc = sum t*q in int32 (exact), y = ((float)acc * s_x) * scale with two
+ *                        fp32 round-to-nearest multiplies.
+ *   y_dev: float[N]. x_dev 16-byte aligned. */
+tern_status tern_gemv(const tern_matrix* W, tern_act act, const void* x_dev, const float* x_scale_dev,
+                      float* y_dev, tern_stream_t stream);
+tern_status tern_gemv_ex(const tern_matrix* W, tern_act act, const void* x_dev, const float* x_scale_dev,
+                         float* y_dev, uint32_t flags, tern_stream_t stream);
+
+/* Small-M GEMM for the draft-verify pass of speculative decoding ([R] "검증된 추측 디코딩": the
+ * 8B scores up to seven drafted positions in one batched forward pass):
+ *   Y[m][n] = scale[n] * sum_k t[n][k] * X[m][k],  0 <= m < M, 1 <= M <= 16.
+ * Each decoded weight word is reused for all M rows. X_dev: bf16[M][K] or int8[M][K];
+ * x_scale_dev: float[M] (int8 only); Y_dev: float[M][N]. Arithmetic as for tern_gemv. */
+tern_status tern_gemm_small_m(const tern_matrix* W, int32_t M, tern_act act, const void* X_dev,
+                              const float* x_scale_dev, float* Y_dev, tern_stream_t stream);
+tern_status tern_gemm_small_m_ex(const tern_matrix* W, int32_t M, tern_act act, const void* X_dev,
+                                 const float* x_scale_dev, float* Y_dev, uint32_t flags,
+                                 tern_stream_t stream);
+
+/* Prefill dense contraction ([R] "실행해보기": batched prefill):
+ *   Y[m][n] = scale[n] * sum_k t[n][k] * X[m][k] for M up to 65536 rows of bf16 activations,
+ * computed as a genuine dense matrix product on the tensor cores (trits expanded to bf16 in
+ * shared memory, fp32 accumulation). X_bf16_dev: bf16[M][K]; Y_dev: float[M][N]. */
+tern_status tern_gemm_prefill(const tern_matrix* W, int32_t M, const uint16_t* X_bf16_dev, float* Y_dev,
+                              tern_stream_t stream);
+
+/* Scratch bytes i8_head_gemv_argmax needs for V rows and M activation rows. */
+size_t i8_head_workspace_bytes(int32_t V, int32_t M);
+
+/* int8 output head with fused per-row scale and greedy argmax ([R] "3진 계열이라는 이름의 실체":
+ * the head stays int8; [R] "뉴트리노 엔진": the unembedding streams at the DRAM roofline):
+ *   logits[m][v] = s_h[v] * sum_k W[v][k] * x[m][k],   argmax[m] = argmax_v logits[m][v]
+ * with the lowest index winning an exact tie, maxval[m] = logits[m][argmax[m]].
+ *   W_dev: int8[V][K] row-major, 16-byte aligned; scale_f16_dev: fp16[V]; K % 128 == 0;
+ *   1 <= M <= 16; act/X_dev/x_scale_dev as for tern_gemm_small_m (int8 mode: logits =
+ *   ((float)acc * s_x) * s_h, bit-exact; bf16 mode: exact products, fp32-rounded logits).
+ *   logits_dev: optional float[M][V] (NULL to skip writing the logits).
+ *   workspace_dev: at least i8_head_workspace_bytes(V, M) bytes, 16-byte aligned, zero-filled
+ *   before its first use; every call leaves it zero-filled again, so one buffer serves any
+ *   number of calls in stream order (two calls that overlap in time need two buffers). */
+tern_status i8_head_gemv_argmax(const int8_t* W_dev, const uint16_t* scale_f16_dev, int32_t V, int32_t K,
+                                int32_t M, tern_act act, const void* X_dev, const float* x_scale_dev,
+                                int32_t* argmax_dev, float* maxval_dev, float* logits_dev,
+                                void* workspace_dev, size_t workspace_bytes, tern_stream_t stream);
+tern_status i8_head_gemv_argmax_ex(const int8_t* W_dev, const uint16_t* scale_f16_dev, int32_t V,
+                                   int32_t K, int32_t M, tern_act act, const void* X_dev,
+                                   const float* x_scale_dev, int32_t* argmax_dev, float* maxval_dev,
+                                   float* logits_dev, void* workspace_dev, size_t workspace_bytes,
+                                   uint32_t flags, tern_stream_t stream);
+
+/* Synchronise `stream`, read *err_flag_dev and map it: 0 -> TERN_OK, nonzero -> TERN_EBADCODE. */
+tern_status tern_read_flag(const int32_t* err_flag_dev, tern_stream_t stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* TERN_H_ */

@@ -1,0 +1,361 @@
+/*
+ * tern_oracle.c -- plain CPU reference for the packed-ternary linear path.
+ *
+ * TEST INFRASTRUCTURE. Only the tests, the smoke check and the bench's CPU-baseline leg may load
+ * or run this code. The product path (the CUDA library) never calls it, and this file shares no
+ * code, header, table or constant generator with it.
+ *
+ * Everything here is the plain definition written out: nested loops, fp64 sums for bf16
+ * activations, int64 sums for int8 activations, no blocking and no reordering beyond the
+ * definition. Rows may be split across threads (each output is computed by one thread, start to
+ * finish), which changes nothing in the arithmetic.
+ *
+ * What is computed. Sources are three of the pages about the Neutrino-1 ternary models, cited by
+ * page and section heading:
+ *   [R] the PyTorchKR review "Fermion Research, 3진 계열 포맷으로 직접 학습한 Neutrino-1 모델군
+ *       3종 공개" (discuss.pytorch.kr/t/11456);
+ *   [A] the aiatolah.com article "Neutrino-1 8B: modelo ternario de 3,88 GB roda em GPU e laptop";
+ *   [O] the origotech.dev explainer "더 적은 비트로 계산하기" (lowbit).
+ *   - the linear-layer contraction y_j = sum_i w_ij x_i ([R] "학습 중에 포맷이 있어야 하는 이유",
+ *     displayed equation), with w in {-1, 0, +1} times a per-row scale;
+ *   - ternary weights mean add / skip / subtract, no multiplies ([O] Figure I caption);
+ *   - weights packed at rest and decoded inside the matrix kernels ([A] second paragraph and
+ *     "Formato unico, tres portas");
+ *   - the transport form of the ternary lane expands bit-exactly into the container ([R] "3진
+ *     계열이라는 이름의 실체"; [A] "Formato unico"); the pages do not give its coder, so this
+ *     library uses fixed-rate base 3, five trits per byte;
+ *   - int8 activations (the 0.6B C runtime) and bf16 activations (the CLI default), fp32 output
+ *     ([R] "토큰 동일성의 경계: 그리디, float32, 그리고 두 개의 근접 동점");
+ *   - the int8 output head with greedy argmax ([R] "3진 계열이라는 이름의 실체": embeddings and
+ *     head stay int8; [R] "토큰 동일성의 경계": near ties between implementations); the lowest
+ *     index wins an exact tie.
+ *
+ * Packed layout (this library's own definition; the pages' FV5 planes are only partly described):
+ *   row n of an N x K matrix (K % 128 == 0) occupies K/16 uint32 words starting at word n*K/16;
+ *   words [0, K/32) are the nonzero-mask plane, words [K/32, K/16) the sign plane;
+ *   trit k is in word k/32 of each plane; with j = k % 32 its mask bit is at position
+ *   p(j) = 16*(j%2) + j/16 + 2*((j%16)/2) and its sign bit at position (p(j) + 1) % 32;
+ *   mask bit = (t != 0), sign bit = (t == -1), so the sign bit is 0 wherever the mask bit is 0.
+ * Transport layout: row n occupies ceil(K/5) bytes; byte j holds trits 5j..5j+4 as
+ *   b = d0 + 3 d1 + 9 d2 + 27 d3 + 81 d4 with d_i = t_{5j+i} + 1; trits past K are t = 0 (d = 1)
+ *   when encoding and are ignored when decoding; a byte above 242 is an error.
+ *
+ * Parity pins: every function here is checked against something other than itself in the CPU
+ * test-suite (numpy brute force, closed forms, exhaustive small cases, hand-worked fixtures).
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ----------------------------------------------------------------------------------------- */
+/* number formats                                                                              */
+
+/* IEEE binary16 -> double, from the format definition (sign, 5-bit exponent, 10-bit fraction). */
+double orc_half_to_double(uint16_t h) {
+  const int sign = h >> 15, e = (h >> 10) & 31, m = h & 1023;
+  double v;
+  if (e == 0) v = ldexp((double)m, -24);            /* subnormal: m * 2^-24            */
+  else if (e == 31) v = m ? NAN : INFINITY;
+  else v = ldexp(1024.0 + (double)m, e - 25);       /* (1 + m/1024) * 2^(e-15)         */
+  return sign ? -v : v;
+}
+
+/* bfloat16 -> float: the upper half of an IEEE binary32. */
+float orc_bf16_to_float(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+}
+
+/* ----------------------------------------------------------------------------------------- */
+/* packed layout                                                                               */
+
+static int mask_bit(int k) { const int j = k % 32; return 16 * (j % 2) + j / 16 + 2 * ((j % 16) / 2); }
+static int sign_bit(int k) { return (mask_bit(k) + 1) % 32; }
+
+int64_t orc_packed_words(int32_t N, int32_t K) { return (int64_t)N * (K / 16); }
+
+/* Dense trits (int8, N x K, row-major) -> planes. Returns -1 on success, else the flat index of
+ * the first trit outside {-1, 0, +1} (planes then hold an unspecified partial result). */
+int64_t orc_pack(const int8_t* trits, int32_t N, int32_t K, uint32_t* planes) {
+  const int kw = K / 32;
+  memset(planes, 0, sizeof(uint32_t) * (size_t)orc_packed_words(N, K));
+  for (int n = 0; n < N; ++n) {
+    uint32_t* mask = planes + (size_t)n * (K / 16);
+    uint32_t* sign = mask + kw;
+    for (int k = 0; k < K; ++k) {
+      const int8_t t = trits[(size_t)n * K + k];
+      if (t != -1 && t != 0 && t != 1) return (int64_t)n * K + k;
+      if (t != 0) mask[k / 32] |= 1u << mask_bit(k);
+      if (t == -1) sign[k / 32] |= 1u << sign_bit(k);
+    }
+  }
+  return -1;
+}
+
+/* One row of planes -> dense trits. A sign bit without its mask bit reads as 0 (never produced by
+ * orc_pack). */
+void orc_unpack_row(const uint32_t* planes, int32_t K, int32_t n, int8_t* out) {
+  const uint32_t* mask = planes + (size_t)n * (K / 16);
+  const uint32_t* sign = mask + K / 32;
+  for (int k = 0; k < K; ++k) {
+    const int m = (mask[k / 32] >> mask_bit(k)) & 1, s = (sign[k / 32] >> sign_bit(k)) & 1;
+    out[k] = (int8_t)(m ? (s ? -1 : 1) : 0);
+  }
+}
+
+void orc_unpack(const uint32_t* planes, int32_t N, int32_t K, int8_t* trits) {
+  for (int n = 0; n < N; ++n) orc_unpack_row(planes, K, n, trits + (size_t)n * K);
+}
+
+/* Per-row occupancy: counts[3n+0] = zeros, [3n+1] = +1s, [3n+2] = -1s. */
+void orc_occupancy(const uint32_t* planes, int32_t N, int32_t K, int64_t* counts) {
+  int8_t* row = (int8_t*)malloc((size_t)K);
+  for (int n = 0; n < N; ++n) {
+    orc_unpack_row(planes, K, n, row);
+    int64_t z = 0, p = 0, q = 0;
+    for (int k = 0; k < K; ++k) { if (row[k] == 0) ++z; else if (row[k] == 1) ++p; else ++q; }
+    counts[3 * n] = z; counts[3 * n + 1] = p; counts[3 * n + 2] = q;
+  }
+  free(row);
+}
+
+/* ----------------------------------------------------------------------------------------- */
+/* base-3 transport                                                                            */
+
+int32_t orc_base3_row_bytes(int32_t K) { return (K + 4) / 5; }
+
+/* Returns -1 on success, else the flat index of the first trit outside {-1, 0, +1}. */
+int64_t orc_base3_encode(const int8_t* trits, int32_t N, int32_t K, uint8_t* bytes) {
+  const int nb = orc_base3_row_bytes(K);
+  for (int n = 0; n < N; ++n) {
+    for (int j = 0; j < nb; ++j) {
+      int b = 0, w = 1;
+      for (int i = 0; i < 5; ++i) {
+        const int k = 5 * j + i;
+        int d = 1;                                   /* padding past K: t = 0 */
+        if (k < K) {
+          const int8_t t = trits[(size_t)n * K + k];
+          if (t != -1 && t != 0 && t != 1) return (int64_t)n * K + k;
+          d = t + 1;
+        }
+        b += d * w;
+        w *= 3;
+      }
+      bytes[(size_t)n * nb + j] = (uint8_t)b;
+    }
+  }
+  return -1;
+}
+
+/* Returns -1 on success, else the flat index of the first byte above 242. */
+int64_t orc_base3_decode(const uint8_t* bytes, int32_t N, int32_t K, int8_t* trits) {
+  const int nb = orc_base3_row_bytes(K);
+  for (int n = 0; n < N; ++n) {
+    for (int j = 0; j < nb; ++j) {
+      int b = bytes[(size_t)n * nb + j];
+      if (b > 242) return (int64_t)n * nb + j;
+      for (int i = 0; i < 5; ++i) {
+        const int d = b % 3;
+        b /= 3;
+        const int k = 5 * j + i;
+        if (k < K) trits[(size_t)n * K + k] = (int8_t)(d - 1);
+      }
+    }
+  }
+  return -1;
+}
+
+/* ----------------------------------------------------------------------------------------- */
+/* threads: outputs split into contiguous ranges, one thread per range                         */
+
+typedef void (*range_fn)(void* ctx, int64_t begin, int64_t end);
+typedef struct { range_fn fn; void* ctx; int64_t b, e; } range_job;
+
+static void* run_range(void* p) {
+  range_job* j = (range_job*)p;
+  j->fn(j->ctx, j->b, j->e);
+  return NULL;
+}
+
+static void parallel_for(int64_t n, int nthreads, range_fn fn, void* ctx) {
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > 256) nthreads = 256;
+  if ((int64_t)nthreads > n) nthreads = n > 0 ? (int)n : 1;
+  if (nthreads == 1) { fn(ctx, 0, n); return; }
+  pthread_t th[256];
+  range_job jobs[256];
+  for (int i = 0; i < nthreads; ++i) {
+    jobs[i].fn = fn; jobs[i].ctx = ctx;
+    jobs[i].b = n * i / nthreads; jobs[i].e = n * (i + 1) / nthreads;
+    pthread_create(&th[i], NULL, run_range, &jobs[i]);
+  }
+  for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+}
+
+/* ----------------------------------------------------------------------------------------- */
+/* bf16 activations: Y[m][n] = scale[n] * sum_k t[n][k] * X[m][k], all in fp64                  */
+
+typedef struct {
+  const uint32_t* planes; const uint16_t* scale; int32_t N, K, M; const uint16_t* X; double* Y;
+} gemm_bf16_ctx;
+
+static void gemm_bf16_rows(void* p, int64_t b, int64_t e) {
+  gemm_bf16_ctx* c = (gemm_bf16_ctx*)p;
+  int8_t* t = (int8_t*)malloc((size_t)c->K);
+  for (int64_t n = b; n < e; ++n) {
+    orc_unpack_row(c->planes, c->K, (int32_t)n, t);
+    const double s = orc_half_to_double(c->scale[n]);
+    for (int m = 0; m < c->M; ++m) {
+      const uint16_t* x = c->X + (size_t)m * c->K;
+      double acc = 0.0;
+      for (int k = 0; k < c->K; ++k)
+        if (t[k] != 0) acc += (double)t[k] * (double)orc_bf16_to_float(x[k]);   /* add / skip / subtract */
+      c->Y[(size_t)m * c->N + n] = s * acc;
+    }
+  }
+  free(t);
+}
+
+void orc_gemm_bf16(const uint32_t* planes, const uint16_t* scale, int32_t N, int32_t K, int32_t M,
+                   const uint16_t* X, double* Y, int32_t nthreads) {
+  gemm_bf16_ctx c = {planes, scale, N, K, M, X, Y};
+  parallel_for(N, nthreads, gemm_bf16_rows, &c);
+}
+
+/* ----------------------------------------------------------------------------------------- */
+/* int8 activations: per-token absmax quantisation, int64 accumulation, fp32 epilogue           */
+
+/* s_x = absmax/127 (fp32 division); q = clamp(rint(x / s_x), -127, 127) with fp32 division and
+ * round-half-to-even; an all-zero row gives s_x = 0 and q = 0. Finite inputs. */
+void orc_quantize_act(const uint16_t* X, int32_t M, int32_t K, int8_t* Q, float* SX) {
+  for (int m = 0; m < M; ++m) {
+    const uint16_t* x = X + (size_t)m * K;
+    float amax = 0.0f;
+    for (int k = 0; k < K; ++k) {
+      const float v = fabsf(orc_bf16_to_float(x[k]));
+      if (v > amax) amax = v;
+    }
+    const float s = amax / 127.0f;
+    SX[m] = s;
+    for (int k = 0; k < K; ++k) {
+      float r = 0.0f;
+      if (s != 0.0f) {
+        const float xs = orc_bf16_to_float(x[k]) / s;
+        r = rintf(xs);
+        if (r > 127.0f) r = 127.0f;
+        if (r < -127.0f) r = -127.0f;
+      }
+      Q[(size_t)m * K + k] = (int8_t)r;
+    }
+  }
+}
+
+typedef struct {
+  const uint32_t* planes; const uint16_t* scale; int32_t N, K, M; const int8_t* Q; const float* SX;
+  int64_t* ACC; float* Y;
+} gemm_i8_ctx;
+
+static void gemm_i8_rows(void* p, int64_t b, int64_t e) {
+  gemm_i8_ctx* c = (gemm_i8_ctx*)p;
+  int8_t* t = (int8_t*)malloc((size_t)c->K);
+  for (int64_t n = b; n < e; ++n) {
+    orc_unpack_row(c->planes, c->K, (int32_t)n, t);
+    const float sw = (float)orc_half_to_double(c->scale[n]);          /* exact */
+    for (int m = 0; m < c->M; ++m) {
+      const int8_t* q = c->Q + (size_t)m * c->K;
+      int64_t acc = 0;
+      for (int k = 0; k < c->K; ++k)
+        if (t[k] == 1) acc += q[k]; else if (t[k] == -1) acc -= q[k];
+      if (c->ACC) c->ACC[(size_t)m * c->N + n] = acc;
+      float y = (float)acc;            /* round to nearest */
+      y = y * c->SX[m];                /* fp32 multiply #1 */
+      y = y * sw;                      /* fp32 multiply #2 */
+      c->Y[(size_t)m * c->N + n] = y;
+    }
+  }
+  free(t);
+}
+
+void orc_gemm_i8(const uint32_t* planes, const uint16_t* scale, int32_t N, int32_t K, int32_t M,
+                 const int8_t* Q, const float* SX, int64_t* ACC, float* Y, int32_t nthreads) {
+  gemm_i8_ctx c = {planes, scale, N, K, M, Q, SX, ACC, Y};
+  parallel_for(N, nthreads, gemm_i8_rows, &c);
+}
+
+/* ----------------------------------------------------------------------------------------- */
+/* int8 output head with greedy argmax                                                         */
+
+typedef struct {
+  const int8_t* W; const uint16_t* SH; int32_t V, K, M; const uint16_t* X; double* L;
+} head_bf16_ctx;
+
+static void head_bf16_rows(void* p, int64_t b, int64_t e) {
+  head_bf16_ctx* c = (head_bf16_ctx*)p;
+  for (int64_t v = b; v < e; ++v) {
+    const int8_t* w = c->W + (size_t)v * c->K;
+    const double s = orc_half_to_double(c->SH[v]);
+    for (int m = 0; m < c->M; ++m) {
+      const uint16_t* x = c->X + (size_t)m * c->K;
+      double acc = 0.0;
+      for (int k = 0; k < c->K; ++k) acc += (double)w[k] * (double)orc_bf16_to_float(x[k]);
+      c->L[(size_t)m * c->V + v] = s * acc;
+    }
+  }
+}
+
+/* logits[m][v] = s_h[v] * sum_k W[v][k] x[m][k] (fp64); argmax over v, lowest index on ties. */
+void orc_head_bf16(const int8_t* W, const uint16_t* SH, int32_t V, int32_t K, int32_t M,
+                   const uint16_t* X, double* LOGITS, int32_t* ARGMAX, double* MAXV, int32_t nthreads) {
+  double* L = LOGITS ? LOGITS : (double*)malloc(sizeof(double) * (size_t)M * V);
+  head_bf16_ctx c = {W, SH, V, K, M, X, L};
+  parallel_for(V, nthreads, head_bf16_rows, &c);
+  for (int m = 0; m < M; ++m) {
+    int32_t best = 0;
+    for (int32_t v = 1; v < V; ++v)
+      if (L[(size_t)m * V + v] > L[(size_t)m * V + best]) best = v;
+    ARGMAX[m] = best;
+    MAXV[m] = L[(size_t)m * V + best];
+  }
+  if (!LOGITS) free(L);
+}
+
+typedef struct {
+  const int8_t* W; const uint16_t* SH; int32_t V, K, M; const int8_t* Q; const float* SX; float* L;
+} head_i8_ctx;
+
+static void head_i8_rows(void* p, int64_t b, int64_t e) {
+  head_i8_ctx* c = (head_i8_ctx*)p;
+  for (int64_t v = b; v < e; ++v) {
+    const int8_t* w = c->W + (size_t)v * c->K;
+    const float sh = (float)orc_half_to_double(c->SH[v]);
+    for (int m = 0; m < c->M; ++m) {
+      const int8_t* q = c->Q + (size_t)m * c->K;
+      int64_t acc = 0;
+      for (int k = 0; k < c->K; ++k) acc += (int64_t)w[k] * q[k];
+      float y = (float)acc;
+      y = y * c->SX[m];
+      y = y * sh;
+      c->L[(size_t)m * c->V + v] = y;
+    }
+  }
+}
+
+void orc_head_i8(const int8_t* W, const uint16_t* SH, int32_t V, int32_t K, int32_t M,
+                 const int8_t* Q, const float* SX, float* LOGITS, int32_t* ARGMAX, float* MAXV,
+                 int32_t nthreads) {
+  float* L = LOGITS ? LOGITS : (float*)malloc(sizeof(float) * (size_t)M * V);
+  head_i8_ctx c = {W, SH, V, K, M, Q, SX, L};
+  parallel_for(V, nthreads, head_i8_rows, &c);
+  for (int m = 0; m < M; ++m) {
+    int32_t best = 0;
+    for (int32_t v = 1; v < V; ++v)
+      if (L[(size_t)m * V + v] > L[(size_t)m * V + best]) best = v;
+    ARGMAX[m] = best;
+    MAXV[m] = L[(size_t)m * V + best];
+  }
+  if (!LOGITS) free(L);
+}
