@@ -1,0 +1,177 @@
+"""bit_gemv_tern_b200: packed-ternary linear layers and the int8 output head on NVIDIA B200.
+
+A thin ctypes binding over libterngemv.so, whose C ABI is declared in include/tern.h. Every
+function here only marshals arguments: device memory comes from torch tensors (data_ptr), the
+stream from torch's current stream, and every step of the computation runs in the library's
+sm_100a kernels. There is no CPU path; if the shared library is missing, importing the functions
+raises.
+
+The functions keep the C names (tern_pack, tern_gemv, tern_gemm_small_m, tern_gemm_prefill,
+i8_head_gemv_argmax, ...), take torch tensors, check the returned tern_status and raise
+TernError on anything but TERN_OK.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "TernError", "TernMatrix", "lib", "library_path",
+    "TERN_ACT_BF16", "TERN_ACT_INT8", "TERN_SRC_INT8_TRITS", "TERN_SRC_BASE3", "TERN_FLAG_PDL",
+    "tern_packed_bytes", "tern_base3_bytes", "tern_pack", "tern_base3_encode", "tern_occupancy",
+    "tern_quantize_act", "tern_gemv", "tern_gemm_small_m", "tern_gemm_prefill",
+    "i8_head_workspace_bytes", "i8_head_gemv_argmax", "tern_read_flag", "tern_status_string",
+]
+
+TERN_OK, TERN_EINVAL, TERN_ESHAPE, TERN_EBADCODE, TERN_ECUDA, TERN_ETIMEOUT = range(6)
+TERN_ACT_BF16, TERN_ACT_INT8 = 0, 1
+TERN_SRC_INT8_TRITS, TERN_SRC_BASE3 = 0, 1
+TERN_FLAG_PDL = 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libterngemv.so")
+_LIB = None
+
+
+class TernError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {tern_status_string(status)}")
+
+
+class _Matrix(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int32), ("K", ctypes.c_int32),
+                ("planes", ctypes.c_void_p), ("scale_f16", ctypes.c_void_p)]
+
+
+def lib() -> ctypes.CDLL:
+    """Load libterngemv.so (raises if it has not been built)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(library_path):
+            raise RuntimeError(f"{library_path} is missing: build it with `python bit_gemv_tern_b200/build.py`")
+        L = ctypes.CDLL(library_path)
+        vp, i32, u32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint32, ctypes.c_size_t
+        mp = ctypes.POINTER(_Matrix)
+        sig = {
+            "tern_status_string": ([i32], ctypes.c_char_p),
+            "tern_packed_bytes": ([i32, i32], sz),
+            "tern_base3_bytes": ([i32, i32], sz),
+            "tern_pack": ([i32, vp, i32, i32, vp, vp, vp], i32),
+            "tern_base3_encode": ([vp, i32, i32, vp, vp, vp], i32),
+            "tern_occupancy": ([mp, vp, vp], i32),
+            "tern_quantize_act": ([vp, i32, i32, vp, vp, vp], i32),
+            "tern_gemv": ([mp, i32, vp, vp, vp, vp], i32),
+            "tern_gemv_ex": ([mp, i32, vp, vp, vp, u32, vp], i32),
+            "tern_gemm_small_m": ([mp, i32, i32, vp, vp, vp, vp], i32),
+            "tern_gemm_small_m_ex": ([mp, i32, i32, vp, vp, vp, u32, vp], i32),
+            "tern_gemm_prefill": ([mp, i32, vp, vp, vp], i32),
+            "i8_head_workspace_bytes": ([i32, i32], sz),
+            "i8_head_gemv_argmax": ([vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+            "i8_head_gemv_argmax_ex": ([vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, sz, u32, vp], i32),
+            "tern_read_flag": ([vp, vp], i32),
+        }
+        for name, (args, res) in sig.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _LIB = L
+    return _LIB
+
+
+def tern_status_string(status: int) -> str:
+    return lib().tern_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != TERN_OK:
+        raise TernError(status, what)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else int(t.data_ptr())
+
+
+def _stream(stream) -> int:
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+class TernMatrix:
+    """A packed ternary matrix: planes (int32/uint32 tensor of N*K/16 words) and fp16 scales."""
+
+    def __init__(self, planes, scale_f16, N: int, K: int):
+        self.planes, self.scale, self.N, self.K = planes, scale_f16, int(N), int(K)
+        self._c = _Matrix(self.N, self.K, _ptr(planes), _ptr(scale_f16))
+
+    def ref(self):
+        return ctypes.byref(self._c)
+
+    @staticmethod
+    def empty(N: int, K: int, device="cuda"):
+        import torch
+        planes = torch.empty(N * K // 16, dtype=torch.int32, device=device)
+        scale = torch.empty(N, dtype=torch.float16, device=device)
+        return TernMatrix(planes, scale, N, K)
+
+
+def tern_packed_bytes(N: int, K: int) -> int:
+    return int(lib().tern_packed_bytes(N, K))
+
+
+def tern_base3_bytes(N: int, K: int) -> int:
+    return int(lib().tern_base3_bytes(N, K))
+
+
+def tern_pack(src_kind: int, src, N: int, K: int, planes, err_flag, stream=None) -> None:
+    """Pack dense int8 trits (src_kind=TERN_SRC_INT8_TRITS) or the base-3 transport
+    (TERN_SRC_BASE3) into planes; invalid input values set err_flag (see tern_read_flag)."""
+    _check(lib().tern_pack(src_kind, _ptr(src), N, K, _ptr(planes), _ptr(err_flag), _stream(stream)), "tern_pack")
+
+
+def tern_base3_encode(trits, N: int, K: int, out, err_flag, stream=None) -> None:
+    _check(lib().tern_base3_encode(_ptr(trits), N, K, _ptr(out), _ptr(err_flag), _stream(stream)),
+           "tern_base3_encode")
+
+
+def tern_occupancy(W: TernMatrix, counts, stream=None) -> None:
+    _check(lib().tern_occupancy(W.ref(), _ptr(counts), _stream(stream)), "tern_occupancy")
+
+
+def tern_quantize_act(x_bf16, M: int, K: int, q, s_x, stream=None) -> None:
+    _check(lib().tern_quantize_act(_ptr(x_bf16), M, K, _ptr(q), _ptr(s_x), _stream(stream)), "tern_quantize_act")
+
+
+def tern_gemv(W: TernMatrix, act: int, x, x_scale, y, flags: int = 0, stream=None) -> None:
+    _check(lib().tern_gemv_ex(W.ref(), act, _ptr(x), _ptr(x_scale), _ptr(y), flags, _stream(stream)), "tern_gemv")
+
+
+def tern_gemm_small_m(W: TernMatrix, M: int, act: int, X, x_scale, Y, flags: int = 0, stream=None) -> None:
+    _check(lib().tern_gemm_small_m_ex(W.ref(), M, act, _ptr(X), _ptr(x_scale), _ptr(Y), flags, _stream(stream)),
+           "tern_gemm_small_m")
+
+
+def tern_gemm_prefill(W: TernMatrix, M: int, X_bf16, Y, stream=None) -> None:
+    _check(lib().tern_gemm_prefill(W.ref(), M, _ptr(X_bf16), _ptr(Y), _stream(stream)), "tern_gemm_prefill")
+
+
+def i8_head_workspace_bytes(V: int, M: int) -> int:
+    return int(lib().i8_head_workspace_bytes(V, M))
+
+
+def i8_head_gemv_argmax(W, scale_f16, V: int, K: int, M: int, act: int, X, x_scale, argmax, maxval,
+                        logits, workspace, flags: int = 0, stream=None) -> None:
+    """workspace: a zero-filled uint8 CUDA tensor of at least i8_head_workspace_bytes(V, M) bytes."""
+    _check(lib().i8_head_gemv_argmax_ex(_ptr(W), _ptr(scale_f16), V, K, M, act, _ptr(X), _ptr(x_scale),
+                                        _ptr(argmax), _ptr(maxval), _ptr(logits), _ptr(workspace),
+                                        int(workspace.numel() * workspace.element_size()), flags,
+                                        _stream(stream)), "i8_head_gemv_argmax")
+
+
+def tern_read_flag(err_flag, stream=None) -> int:
+    """Synchronise the stream and return TERN_OK or TERN_EBADCODE from a device error flag."""
+    st = lib().tern_read_flag(_ptr(err_flag), _stream(stream))
+    if st not in (TERN_OK, TERN_EBADCODE):
+        raise TernError(st, "tern_read_flag")
+    return st

@@ -1,0 +1,213 @@
+// C ABI of libterngemv.so (declared and documented in include/tern.h): argument validation,
+// launch planning and kernel launches. No entry point allocates device memory or keeps state.
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/tern.h"
+#include "tern_kernels.h"
+
+namespace {
+
+constexpr int kSMs = 148;
+constexpr size_t kGemmSmemCap = 160 * 1024;
+constexpr size_t kHeadSmemCap = 100 * 1024;
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+inline cudaStream_t cs(tern_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+inline tern_status from_cuda(cudaError_t e) { return e == cudaSuccess ? TERN_OK : TERN_ECUDA; }
+
+bool valid_shape(int32_t N, int32_t K) { return N > 0 && K > 0 && (K % 128) == 0; }
+
+tern_status check_matrix(const tern_matrix* W) {
+  if (!W || !W->planes || !W->scale_f16) return TERN_EINVAL;
+  if (!valid_shape(W->N, W->K)) return TERN_ESHAPE;
+  if (!aligned(W->planes, 16) || !aligned(W->scale_f16, 2)) return TERN_EINVAL;
+  return TERN_OK;
+}
+
+// Split K over a cluster of up to 8 CTAs so that small matrices still cover every SM.
+bool plan_gemm(int N, int K, int M, int mode, int& ksplit) {
+  const int row_blocks = (N + tern::gemm_rows_per_cta() - 1) / tern::gemm_rows_per_cta();
+  const int units = K / 128;
+  int ks = 1;
+  while (ks < 8 && row_blocks * ks < 2 * kSMs && units % (2 * ks) == 0) ks *= 2;
+  while (tern::gemm_smem_bytes(mode, M, K / ks) > kGemmSmemCap && ks < 8 && units % (2 * ks) == 0) ks *= 2;
+  if (tern::gemm_smem_bytes(mode, M, K / ks) > kGemmSmemCap) return false;
+  ksplit = ks;
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* tern_status_string(tern_status s) {
+  switch (s) {
+    case TERN_OK: return "TERN_OK";
+    case TERN_EINVAL: return "TERN_EINVAL: invalid argument";
+    case TERN_ESHAPE: return "TERN_ESHAPE: invalid shape";
+    case TERN_EBADCODE: return "TERN_EBADCODE: invalid trit or transport byte in the input";
+    case TERN_ECUDA: return "TERN_ECUDA: CUDA error";
+    case TERN_ETIMEOUT: return "TERN_ETIMEOUT: bounded device wait gave up";
+  }
+  return "unknown tern_status";
+}
+
+size_t tern_packed_bytes(int32_t N, int32_t K) {
+  return valid_shape(N, K) ? (size_t)N * (size_t)K / 4 : 0;
+}
+
+size_t tern_base3_bytes(int32_t N, int32_t K) {
+  return valid_shape(N, K) ? (size_t)N * (size_t)((K + 4) / 5) : 0;
+}
+
+tern_status tern_pack(tern_src src, const void* src_dev, int32_t N, int32_t K, uint32_t* planes_dev,
+                      int32_t* err_flag_dev, tern_stream_t stream) {
+  if (!src_dev || !planes_dev || !err_flag_dev) return TERN_EINVAL;
+  if (src != TERN_SRC_INT8_TRITS && src != TERN_SRC_BASE3) return TERN_EINVAL;
+  if (!valid_shape(N, K)) return TERN_ESHAPE;
+  if (!aligned(planes_dev, 16) || !aligned(err_flag_dev, 4)) return TERN_EINVAL;
+  if (src == TERN_SRC_INT8_TRITS && !aligned(src_dev, 16)) return TERN_EINVAL;
+  cudaError_t e = cudaMemsetAsync(err_flag_dev, 0, sizeof(int32_t), cs(stream));
+  if (e != cudaSuccess) return TERN_ECUDA;
+  if (src == TERN_SRC_INT8_TRITS)
+    e = tern::launch_pack_trits(static_cast<const int8_t*>(src_dev), N, K, planes_dev, err_flag_dev, cs(stream));
+  else
+    e = tern::launch_unpack_base3(static_cast<const uint8_t*>(src_dev), N, K, planes_dev, err_flag_dev, cs(stream));
+  return from_cuda(e);
+}
+
+tern_status tern_base3_encode(const int8_t* trits_dev, int32_t N, int32_t K, uint8_t* out_dev,
+                              int32_t* err_flag_dev, tern_stream_t stream) {
+  if (!trits_dev || !out_dev || !err_flag_dev) return TERN_EINVAL;
+  if (!valid_shape(N, K)) return TERN_ESHAPE;
+  if (!aligned(err_flag_dev, 4)) return TERN_EINVAL;
+  if (cudaMemsetAsync(err_flag_dev, 0, sizeof(int32_t), cs(stream)) != cudaSuccess) return TERN_ECUDA;
+  return from_cuda(tern::launch_encode_base3(trits_dev, N, K, out_dev, err_flag_dev, cs(stream)));
+}
+
+tern_status tern_occupancy(const tern_matrix* W, int64_t* counts_dev, tern_stream_t stream) {
+  if (!W || !W->planes || !counts_dev) return TERN_EINVAL;
+  if (!valid_shape(W->N, W->K)) return TERN_ESHAPE;
+  if (!aligned(W->planes, 16) || !aligned(counts_dev, 8)) return TERN_EINVAL;
+  return from_cuda(tern::launch_occupancy(W->planes, W->N, W->K, counts_dev, cs(stream)));
+}
+
+tern_status tern_quantize_act(const uint16_t* x_bf16_dev, int32_t M, int32_t K, int8_t* q_dev, float* s_x_dev,
+                              tern_stream_t stream) {
+  if (!x_bf16_dev || !q_dev || !s_x_dev) return TERN_EINVAL;
+  if (M < 1 || M > 4096 || !valid_shape(1, K)) return TERN_ESHAPE;
+  if (!aligned(x_bf16_dev, 16) || !aligned(q_dev, 8) || !aligned(s_x_dev, 4)) return TERN_EINVAL;
+  return from_cuda(tern::launch_quantize(x_bf16_dev, M, K, q_dev, s_x_dev, cs(stream)));
+}
+
+tern_status tern_gemm_small_m_ex(const tern_matrix* W, int32_t M, tern_act act, const void* X_dev,
+                                 const float* x_scale_dev, float* Y_dev, uint32_t flags, tern_stream_t stream) {
+  tern_status st = check_matrix(W);
+  if (st != TERN_OK) return st;
+  if (act != TERN_ACT_BF16 && act != TERN_ACT_INT8) return TERN_EINVAL;
+  if (flags & ~TERN_FLAG_PDL) return TERN_EINVAL;
+  if (M < 1 || M > 16) return TERN_ESHAPE;
+  if (!X_dev || !Y_dev || !aligned(X_dev, 16) || !aligned(Y_dev, 4)) return TERN_EINVAL;
+  if (act == TERN_ACT_INT8 && (!x_scale_dev || !aligned(x_scale_dev, 4))) return TERN_EINVAL;
+  tern::GemmParams p = {};
+  p.planes = W->planes;
+  p.scale = W->scale_f16;
+  p.N = W->N;
+  p.K = W->K;
+  p.x = X_dev;
+  p.sx = x_scale_dev;
+  p.y = Y_dev;
+  p.M = M;
+  p.mode = act == TERN_ACT_BF16 ? 0 : 1;
+  if (!plan_gemm(p.N, p.K, M, p.mode, p.ksplit)) return TERN_ESHAPE;
+  p.kr = p.K / p.ksplit;
+  return from_cuda(tern::launch_tern_gemm(p, (flags & TERN_FLAG_PDL) != 0, cs(stream)));
+}
+
+tern_status tern_gemm_small_m(const tern_matrix* W, int32_t M, tern_act act, const void* X_dev,
+                              const float* x_scale_dev, float* Y_dev, tern_stream_t stream) {
+  return tern_gemm_small_m_ex(W, M, act, X_dev, x_scale_dev, Y_dev, 0u, stream);
+}
+
+tern_status tern_gemv_ex(const tern_matrix* W, tern_act act, const void* x_dev, const float* x_scale_dev,
+                         float* y_dev, uint32_t flags, tern_stream_t stream) {
+  return tern_gemm_small_m_ex(W, 1, act, x_dev, x_scale_dev, y_dev, flags, stream);
+}
+
+tern_status tern_gemv(const tern_matrix* W, tern_act act, const void* x_dev, const float* x_scale_dev,
+                      float* y_dev, tern_stream_t stream) {
+  return tern_gemm_small_m_ex(W, 1, act, x_dev, x_scale_dev, y_dev, 0u, stream);
+}
+
+size_t i8_head_workspace_bytes(int32_t V, int32_t M) {
+  if (V <= 0 || M < 1 || M > 16) return 0;
+  return tern::head_workspace_bytes(M);
+}
+
+tern_status i8_head_gemv_argmax_ex(const int8_t* W_dev, const uint16_t* scale_f16_dev, int32_t V, int32_t K,
+                                   int32_t M, tern_act act, const void* X_dev, const float* x_scale_dev,
+                                   int32_t* argmax_dev, float* maxval_dev, float* logits_dev,
+                                   void* workspace_dev, size_t workspace_bytes, uint32_t flags,
+                                   tern_stream_t stream) {
+  if (!W_dev || !scale_f16_dev || !X_dev || !argmax_dev || !maxval_dev || !workspace_dev) return TERN_EINVAL;
+  if (act != TERN_ACT_BF16 && act != TERN_ACT_INT8) return TERN_EINVAL;
+  if (flags & ~TERN_FLAG_PDL) return TERN_EINVAL;
+  if (!valid_shape(V, K) || M < 1 || M > 16) return TERN_ESHAPE;
+  if (!aligned(W_dev, 16) || !aligned(X_dev, 16) || !aligned(workspace_dev, 16) || !aligned(scale_f16_dev, 2))
+    return TERN_EINVAL;
+  if (!aligned(argmax_dev, 4) || !aligned(maxval_dev, 4) || (logits_dev && !aligned(logits_dev, 4)))
+    return TERN_EINVAL;
+  if (act == TERN_ACT_INT8 && (!x_scale_dev || !aligned(x_scale_dev, 4))) return TERN_EINVAL;
+  if (workspace_bytes < tern::head_workspace_bytes(M)) return TERN_EINVAL;
+  tern::HeadParams p = {};
+  p.W = W_dev;
+  p.sh = scale_f16_dev;
+  p.V = V;
+  p.K = K;
+  p.M = M;
+  p.mode = act == TERN_ACT_BF16 ? 0 : 1;
+  p.x = X_dev;
+  p.sx = x_scale_dev;
+  p.argmax = argmax_dev;
+  p.maxval = maxval_dev;
+  p.logits = logits_dev;
+  p.counter = static_cast<unsigned int*>(workspace_dev);
+  p.keys = reinterpret_cast<unsigned long long*>(static_cast<char*>(workspace_dev) + 16);
+  const int units = K / 128;
+  int ks = 1;
+  while (tern::head_smem_bytes(p.mode, M, K / ks) > kHeadSmemCap && ks < 8 && units % (2 * ks) == 0) ks *= 2;
+  if (tern::head_smem_bytes(p.mode, M, K / ks) > kHeadSmemCap) return TERN_ESHAPE;
+  p.ksplit = ks;
+  p.kr = K / ks;
+  p.nrb = (V + 127) / 128;
+  int nby = (2 * kSMs) / ks;
+  if (nby > p.nrb) nby = p.nrb;
+  if (nby < 1) nby = 1;
+  p.nby = nby;
+  return from_cuda(tern::launch_head(p, (flags & TERN_FLAG_PDL) != 0, cs(stream)));
+}
+
+tern_status i8_head_gemv_argmax(const int8_t* W_dev, const uint16_t* scale_f16_dev, int32_t V, int32_t K, int32_t M,
+                                tern_act act, const void* X_dev, const float* x_scale_dev, int32_t* argmax_dev,
+                                float* maxval_dev, float* logits_dev, void* workspace_dev, size_t workspace_bytes,
+                                tern_stream_t stream) {
+  return i8_head_gemv_argmax_ex(W_dev, scale_f16_dev, V, K, M, act, X_dev, x_scale_dev, argmax_dev, maxval_dev,
+                                logits_dev, workspace_dev, workspace_bytes, 0u, stream);
+}
+
+tern_status tern_read_flag(const int32_t* err_flag_dev, tern_stream_t stream) {
+  if (!err_flag_dev) return TERN_EINVAL;
+  if (cudaStreamSynchronize(cs(stream)) != cudaSuccess) return TERN_ECUDA;
+  int32_t v = 0;
+  if (cudaMemcpy(&v, err_flag_dev, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return TERN_ECUDA;
+  return v == 0 ? TERN_OK : TERN_EBADCODE;
+}
+
+tern_status tern_gemm_prefill(const tern_matrix* W, int32_t M, const uint16_t* X_bf16_dev, float* Y_dev,
+                              tern_stream_t stream) {
+  (void)W; (void)M; (void)X_bf16_dev; (void)Y_dev; (void)stream;
+  return TERN_EINVAL;
+}
+
+}  // extern "C"

@@ -1,0 +1,113 @@
+// Device helpers shared by the sm_100a kernels of libterngemv.so.
+//
+// Decode of the packed layout (include/tern.h): a row stores, per 32 trits, one mask word m
+// (bit = t != 0) and one sign word s (bit = t == -1) whose bit order is the mask order rotated by
+// one. Merging the two words gives two words of sixteen 2-bit fields (mask bit low, sign bit high):
+//   wa = (m & 0x55555555) | (s & 0xAAAAAAAA)          fields of the trits on even mask bits
+//   wb = rotr((m & 0xAAAAAAAA) | (s & 0x55555555), 1) fields of the trits on odd mask bits
+// A field (m, s) read as a 2-bit two's-complement number is exactly t (00 = 0, 01 = +1,
+// 11 = -1), so a field moved to the top two bits of a byte is the int8 value 64*t, and a field in
+// the top two bits of a 16-bit half is the bf16 (or fp16) value 2.0*t. One shift and one AND
+// produce a whole tensor-core operand register: this is the add / skip / subtract rule of the
+// ternary weights (origotech.dev "더 적은 비트로 계산하기", Figure I) carried out by the tensor
+// cores with exact +-1 products.
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+namespace tern {
+
+constexpr int kThreads = 256;  // 8 warps per CTA for the matrix kernels
+
+// ---- programmatic dependent launch -----------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---- global loads ------------------------------------------------------------------------------
+// Streaming 128-bit load for data read exactly once (weights): bypasses L1 allocation.
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint4 ld_nc(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+
+// ---- warp-level tensor-core products -------------------------------------------------------------
+// D(16x8) += A(16x32, s8, row) * B(32x8, s8, col), s32 accumulate.
+__device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                       uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// D(16x8) += A(16x16, bf16, row) * B(16x8, bf16, col), f32 accumulate.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// ---- decode ------------------------------------------------------------------------------------
+__device__ __forceinline__ void merge_planes(uint32_t m, uint32_t s, uint32_t& wa, uint32_t& wb) {
+  wa = (m & 0x55555555u) | (s & 0xAAAAAAAAu);
+  const uint32_t v = (m & 0xAAAAAAAAu) | (s & 0x55555555u);
+  wb = __funnelshift_r(v, v, 1);
+}
+
+// int8 operand register R (0..7) of a 32-trit word: bytes hold 64*t for the four trits
+//   R < 4: fields R, R+4, R+8, R+12 of wa;  R >= 4: the same fields (R-4, ...) of wb.
+// In-word trit offsets of bytes 0..3: R < 4: {2R, 2R+8, 2R+1, 2R+9}; R >= 4: 16 + the same.
+template <int R>
+__device__ __forceinline__ uint32_t dec_i8(uint32_t wa, uint32_t wb) {
+  constexpr int i = R & 3;
+  return ((R < 4 ? wa : wb) << (6 - 2 * i)) & 0xC0C0C0C0u;
+}
+
+// bf16 operand register A (0..15) of a 32-trit word: low half = trit 2A, high half = trit 2A+1
+// (in-word offsets), each as the bf16 value 2.0*t.
+//   A < 8: fields A and A+8 of wa;  A >= 8: fields A-8 and A of wb.
+template <int A>
+__device__ __forceinline__ uint32_t dec_bf16(uint32_t wa, uint32_t wb) {
+  constexpr int f = A & 7;
+  return ((A < 8 ? wa : wb) << (14 - 2 * f)) & 0xC000C000u;
+}
+
+// int8 activations, permuted once per CTA so that activation word R of each 32-byte block holds
+// the four bytes that dec_i8<R> pairs with. `lo` holds bytes 0..15 (or 16..31) of the block.
+__device__ __forceinline__ uint4 permute_i8_half(uint4 lo) {
+  uint4 o;
+  o.x = __byte_perm(lo.x, lo.z, 0x5140);
+  o.y = __byte_perm(lo.x, lo.z, 0x7362);
+  o.z = __byte_perm(lo.y, lo.w, 0x5140);
+  o.w = __byte_perm(lo.y, lo.w, 0x7362);
+  return o;
+}
+
+// fp16 bit pattern -> float (exact).
+__device__ __forceinline__ float f16_bits_to_float(uint16_t h) {
+  return __half2float(__ushort_as_half(h));
+}
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t b) { return __uint_as_float(b << 16); }
+
+// Monotone 32-bit key of a float (larger float -> larger key; -0 and +0 give the same key).
+__device__ __forceinline__ uint32_t float_order_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float float_from_order_key(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+}  // namespace tern

@@ -1,0 +1,290 @@
+// int8 output head with fused per-row scale and greedy argmax.
+//
+//   logits[m][v] = s_h[v] * sum_k W[v][k] * x[m][k],   argmax[m] = argmax_v logits[m][v]
+//
+// The head stays int8 (PyTorchKR review "Fermion Research, 3진 계열 포맷으로 직접 학습한
+// Neutrino-1 모델군 3종 공개", section "3진 계열이라는 이름의 실체"), and the unembedding is the
+// single step that runs at the DRAM roofline, 43% of a decode step's DRAM traffic (same review,
+// section "뉴트리노 엔진"). Greedy decoding takes the argmax; independent implementations may differ
+// on near ties (section "토큰 동일성의 경계"); here an exact tie goes to the lowest index.
+//
+// Design: int8 W rows feed mma.sync directly as the A operand (no decode at all); the activation
+// is the B operand. int8 mode uses q from the per-token quantiser and is bit-exact. bf16 mode
+// splits each bf16 x exactly into three int8 limbs of a 22-bit fixed-point value relative to
+// 2^E, E from the absmax of this CTA's K slice (exact for every x within 2^-15 of that absmax,
+// rounding below it), so the products and the int32 sums stay exact; limbs and K slices are
+// combined in fp64 before the single rounding to fp32. Limbs (and the M rows) occupy the eight
+// columns of each tensor-core n-group, which for M = 1 come for free. CTAs splitting K form a
+// cluster and add partial sums through distributed shared memory. The running maximum per row is
+// kept as a packed (order-preserving value key, inverted index) 64-bit word, reduced with
+// shared-memory and then global atomicMax; the last CTA to finish publishes the result and
+// zero-fills the workspace again.
+#include <cooperative_groups.h>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "tern_device.cuh"
+#include "tern_kernels.h"
+
+namespace cg = cooperative_groups;
+
+namespace tern {
+namespace {
+
+constexpr int kHeadRows = 128;   // rows per row block: 8 warps x 16 rows
+constexpr int kLimbFrac = 22;    // bf16 mode: x ~= X * 2^(E - 22), |X| < 2^22
+
+template <int MODE, int NG>
+__global__ void __launch_bounds__(kThreads) k_head(const HeadParams p) {
+  extern __shared__ __align__(16) uint32_t smem[];
+  __shared__ unsigned long long best[16];
+  __shared__ int expo[16];
+  __shared__ int is_last;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int ks = blockIdx.x;
+  const int k0 = ks * p.kr;
+  const int ncols = MODE == 0 ? 3 * p.M : p.M;
+  const int RS = p.kr / 4 + 4;             // words per staged activation column (+4: banks)
+  const int nch = p.kr / 128;              // 128-byte chunks per row in this slice
+  if (threadIdx.x < 16) best[threadIdx.x] = 0ull;
+
+  // chunk c of a row block: 32 bytes of rows ra, rb at k0 + 128c + 32t
+  const int8_t* pa = nullptr;
+  const int8_t* pb = nullptr;
+  bool warp_live = false;
+  auto set_rows = [&](int rb) {
+    const int row0 = rb * kHeadRows + warp * 16;
+    warp_live = row0 < p.V;
+    const int ra = min(row0 + g, p.V - 1), rbb = min(row0 + g + 8, p.V - 1);
+    pa = p.W + (size_t)ra * p.K + k0 + 32 * t;
+    pb = p.W + (size_t)rbb * p.K + k0 + 32 * t;
+  };
+  auto load_chunk = [&](int c, uint4 (&w)[4]) {
+    if (warp_live && c < nch) {
+      w[0] = ld_stream(pa + 128 * c);
+      w[1] = ld_stream(pa + 128 * c + 16);
+      w[2] = ld_stream(pb + 128 * c);
+      w[3] = ld_stream(pb + 128 * c + 16);
+    } else {
+      w[0] = w[1] = w[2] = w[3] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+
+  int rb = blockIdx.y;
+  uint4 cur[4], nxt[4];
+  set_rows(rb);
+  load_chunk(0, cur);
+  load_chunk(1, nxt);
+  pdl_wait();
+
+  // ---- stage activations: column c of the B operand holds K-slice bytes -------------------------
+  if (MODE == 1) {
+    const int8_t* xq = static_cast<const int8_t*>(p.x);
+    const int per_row = p.kr / 16;
+    for (int i = threadIdx.x; i < p.M * per_row; i += kThreads) {
+      const int m = i / per_row, v = i - m * per_row;
+      *reinterpret_cast<uint4*>(smem + m * RS + 4 * v) = ld_nc(xq + (size_t)m * p.K + k0 + 16 * v);
+    }
+  } else {
+    const uint16_t* xb = static_cast<const uint16_t*>(p.x);
+    for (int m = warp; m < p.M; m += kThreads / 32) {
+      float amax = 0.0f;
+      for (int k = lane * 8; k < p.kr; k += 256) {
+        const uint4 v = ld_nc(xb + (size_t)m * p.K + k0 + k);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          amax = fmaxf(amax, fmaxf(fabsf(bf16_bits_to_float(w[e] & 0xFFFFu)), fabsf(bf16_bits_to_float(w[e] >> 16))));
+      }
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+      int E = 0;
+      if (amax > 0.0f) {
+        frexpf(amax, &E);                  // amax < 2^E
+        E = max(E, -100);
+      }
+      if (lane == 0) expo[m] = E;
+    }
+    __syncthreads();
+    const int per_row = p.kr / 8;
+    for (int i = threadIdx.x; i < p.M * per_row; i += kThreads) {
+      const int m = i / per_row, v = i - m * per_row;
+      const float f = ldexpf(1.0f, kLimbFrac - expo[m]);
+      const uint4 val = ld_nc(xb + (size_t)m * p.K + k0 + 8 * v);
+      const uint32_t w[4] = {val.x, val.y, val.z, val.w};
+      uint32_t l2[2] = {0u, 0u}, l1[2] = {0u, 0u}, l0[2] = {0u, 0u};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint32_t bits = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
+        const int X = __float2int_rn(bf16_bits_to_float(bits) * f);   // exact power-of-two scaling
+        const int L0 = (int)(int8_t)(X & 0xFF);
+        const int X1 = (X - L0) >> 8;
+        const int L1 = (int)(int8_t)(X1 & 0xFF);
+        const int L2 = (X1 - L1) >> 8;                                 // |L2| <= 64
+        const int sh = 8 * (e & 3);
+        l0[e >> 2] |= (uint32_t)(uint8_t)L0 << sh;
+        l1[e >> 2] |= (uint32_t)(uint8_t)L1 << sh;
+        l2[e >> 2] |= (uint32_t)(uint8_t)L2 << sh;
+      }
+      *reinterpret_cast<uint2*>(smem + (3 * m) * RS + 2 * v) = make_uint2(l2[0], l2[1]);
+      *reinterpret_cast<uint2*>(smem + (3 * m + 1) * RS + 2 * v) = make_uint2(l1[0], l1[1]);
+      *reinterpret_cast<uint2*>(smem + (3 * m + 2) * RS + 2 * v) = make_uint2(l0[0], l0[1]);
+    }
+  }
+  __syncthreads();
+
+  constexpr int kCols = 8 * NG;
+  int* part = reinterpret_cast<int*>(smem + ncols * RS);
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rows_per_rank = kHeadRows / p.ksplit;
+  bool first = true;
+
+  for (; rb < p.nrb; rb += p.nby) {
+    if (!first) {
+      set_rows(rb);
+      load_chunk(0, cur);
+      load_chunk(1, nxt);
+    }
+    first = false;
+    int acc[NG][4];
+#pragma unroll
+    for (int n = 0; n < NG; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0;
+
+    for (int c = 0; c < nch; ++c) {
+#pragma unroll
+      for (int n = 0; n < NG; ++n) {
+        const int col = 8 * n + g;
+        uint4 b0 = make_uint4(0u, 0u, 0u, 0u), b1 = b0;
+        if (col < ncols) {
+          const uint32_t* cp = smem + col * RS + 32 * c + 8 * t;
+          b0 = *reinterpret_cast<const uint4*>(cp);
+          b1 = *reinterpret_cast<const uint4*>(cp + 4);
+        }
+        // k-slots: lane t owns bytes [32t, 32t + 32) of the 128-byte chunk, four MMAs of 32.
+        mma_s8(acc[n], cur[0].x, cur[2].x, cur[0].y, cur[2].y, b0.x, b0.y);
+        mma_s8(acc[n], cur[0].z, cur[2].z, cur[0].w, cur[2].w, b0.z, b0.w);
+        mma_s8(acc[n], cur[1].x, cur[3].x, cur[1].y, cur[3].y, b1.x, b1.y);
+        mma_s8(acc[n], cur[1].z, cur[3].z, cur[1].w, cur[3].w, b1.z, b1.w);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) cur[i] = nxt[i];
+      load_chunk(c + 2, nxt);
+    }
+
+    // partial sums of this K slice: part[local row][column]
+#pragma unroll
+    for (int n = 0; n < NG; ++n)
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        part[(warp * 16 + g + 8 * (i >> 1)) * kCols + 8 * n + 2 * t + (i & 1)] = acc[n][i];
+    if (p.ksplit > 1) cluster.sync(); else __syncthreads();
+
+    for (int i = threadIdx.x; i < rows_per_rank * p.M; i += kThreads) {
+      const int lrow = ks * rows_per_rank + i / p.M, m = i % p.M;
+      const int row = rb * kHeadRows + lrow;
+      if (row >= p.V) continue;
+      const float shv = f16_bits_to_float(p.sh[row]);
+      float logit;
+      if (MODE == 1) {
+        int a = 0;
+        for (int r = 0; r < p.ksplit; ++r)
+          a += (p.ksplit > 1 ? cluster.map_shared_rank(part, r) : part)[lrow * kCols + m];
+        logit = __fmul_rn(__fmul_rn(__int2float_rn(a), p.sx[m]), shv);
+      } else {
+        double tot = 0.0;
+        for (int r = 0; r < p.ksplit; ++r) {
+          const int* rp = (p.ksplit > 1 ? cluster.map_shared_rank(part, r) : part) + lrow * kCols + 3 * m;
+          const int E = (p.ksplit > 1 ? cluster.map_shared_rank(expo, r) : expo)[m];
+          const long long D = (long long)rp[0] * 65536 + (long long)rp[1] * 256 + rp[2];
+          tot += ldexp((double)D, E - kLimbFrac);
+        }
+        logit = (float)(tot * (double)shv);
+      }
+      if (p.logits) p.logits[(size_t)m * p.V + row] = logit;
+      const unsigned long long key =
+          ((unsigned long long)float_order_key(logit) << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)row);
+      atomicMax(&best[m], key);
+    }
+    if (p.ksplit > 1) cluster.sync(); else __syncthreads();
+  }
+  pdl_launch_dependents();
+
+  // ---- grid-wide argmax: global atomicMax, then the last CTA publishes and resets ----------------
+  __syncthreads();
+  if (threadIdx.x < p.M && best[threadIdx.x] != 0ull) atomicMax(&p.keys[threadIdx.x], best[threadIdx.x]);
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned int total = gridDim.x * gridDim.y;
+    is_last = (atomicAdd(p.counter, 1u) == total - 1u);
+  }
+  __syncthreads();
+  if (is_last) {
+    __threadfence();
+    if (threadIdx.x < p.M) {
+      const unsigned long long key = atomicExch(&p.keys[threadIdx.x], 0ull);
+      p.argmax[threadIdx.x] = (int32_t)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull));
+      p.maxval[threadIdx.x] = float_from_order_key((uint32_t)(key >> 32));
+    }
+    if (threadIdx.x == 0) atomicExch(p.counter, 0u);
+  }
+}
+
+template <int MODE, int NG>
+cudaError_t launch_ng(const HeadParams& p, size_t smem, bool pdl, cudaStream_t st) {
+  auto kern = k_head<MODE, NG>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.ksplit, p.nby, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (p.ksplit > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = p.ksplit;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+template <int MODE>
+cudaError_t launch_mode(const HeadParams& p, int ng, size_t smem, bool pdl, cudaStream_t st) {
+  switch (ng) {
+    case 1: return launch_ng<MODE, 1>(p, smem, pdl, st);
+    case 2: return launch_ng<MODE, 2>(p, smem, pdl, st);
+    case 3: return launch_ng<MODE, 3>(p, smem, pdl, st);
+    case 4: return launch_ng<MODE, 4>(p, smem, pdl, st);
+    case 5: return launch_ng<MODE, 5>(p, smem, pdl, st);
+    default: return launch_ng<MODE, 6>(p, smem, pdl, st);
+  }
+}
+
+}  // namespace
+
+size_t head_workspace_bytes(int M) { return 16 + 8 * (size_t)M; }
+
+size_t head_smem_bytes(int mode, int M, int kr) {
+  const int ncols = mode == 0 ? 3 * M : M;
+  const int ng = (ncols + 7) / 8;
+  return (size_t)ncols * (kr / 4 + 4) * 4 + (size_t)kHeadRows * 8 * ng * 4;
+}
+
+cudaError_t launch_head(const HeadParams& p, bool pdl, cudaStream_t st) {
+  const int ncols = p.mode == 0 ? 3 * p.M : p.M;
+  const int ng = (ncols + 7) / 8;
+  const size_t smem = head_smem_bytes(p.mode, p.M, p.kr);
+  return p.mode == 0 ? launch_mode<0>(p, ng, smem, pdl, st) : launch_mode<1>(p, ng, smem, pdl, st);
+}
+
+}  // namespace tern

@@ -1,0 +1,188 @@
+// Loader-side kernels: packing trits into the two-plane layout, the base-3 transport in both
+// directions, and per-row occupancy counts. All are streaming, HBM-bound integer kernels.
+//
+// Sources: weights packed at rest and decoded inside the matrix kernels (aiatolah.com,
+// "Neutrino-1 8B: modelo ternario de 3,88 GB roda em GPU e laptop", second paragraph); the
+// transport form of the ternary lane expands bit-exactly into the container (PyTorchKR review
+// "Fermion Research, 3진 계열 포맷으로 직접 학습한 Neutrino-1 모델군 3종 공개", section
+// "3진 계열이라는 이름의 실체"); per-tensor zero / +1 / -1 occupancy (same review, section
+// "출하된 컨테이너를 직접 읽기: 62.63%의 침묵"). The packed layout is defined in include/tern.h.
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "tern_device.cuh"
+#include "tern_kernels.h"
+
+namespace tern {
+namespace {
+
+// Mask-bit position of in-word trit offset j (0..31); the sign bit sits one position higher
+// (mod 32).
+__device__ __forceinline__ int mask_pos(int j) { return 16 * (j & 1) + (j >> 4) + 2 * ((j & 15) >> 1); }
+
+__device__ __forceinline__ void set_flag(int32_t* flag) { atomicExch(flag, 1); }
+
+// One thread per 32-trit word: reads 32 trit bytes, writes one mask word and one sign word.
+__global__ void k_pack_trits(const int8_t* __restrict__ src, int64_t n_words, int32_t KM,
+                             uint32_t* __restrict__ planes, int32_t* __restrict__ flag) {
+  bool bad = false;
+  for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < n_words;
+       w += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = w / KM, col = w % KM;
+    const uint4* p = reinterpret_cast<const uint4*>(src + w * 32);
+    const uint4 v0 = ld_stream(p), v1 = ld_stream(p + 1);
+    const uint32_t b[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    uint32_t m = 0, s = 0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const uint32_t t = (b[j >> 2] >> (8 * (j & 3))) & 0xFFu;
+      const int p_m = mask_pos(j);
+      m |= (uint32_t)(t != 0u) << p_m;
+      s |= (uint32_t)(t == 0xFFu) << ((p_m + 1) & 31);
+      bad |= (t > 1u && t != 0xFFu);
+    }
+    uint32_t* row_p = planes + row * (2 * (int64_t)KM);
+    row_p[col] = m;
+    row_p[KM + col] = s;
+  }
+  if (__any_sync(0xFFFFFFFFu, bad) && (threadIdx.x & 31) == 0) set_flag(flag);
+}
+
+// Byte -> five trits as (mask5 | sign5 << 5); 0xFFFF marks an invalid byte (> 242).
+__device__ __forceinline__ void build_base3_lut(uint16_t* lut) {
+  for (int b = threadIdx.x; b < 256; b += blockDim.x) {
+    uint16_t e = 0xFFFFu;
+    if (b < 243) {
+      int v = b;
+      uint32_t m = 0, s = 0;
+      for (int i = 0; i < 5; ++i) {
+        const int d = v % 3;
+        v /= 3;
+        m |= (uint32_t)(d != 1) << i;
+        s |= (uint32_t)(d == 0) << i;
+      }
+      e = (uint16_t)(m | (s << 5));
+    }
+    lut[b] = e;
+  }
+}
+
+// One thread per 32-trit word of the output: decodes the 7 or 8 transport bytes that cover it.
+__global__ void k_unpack_base3(const uint8_t* __restrict__ src, int64_t n_words, int32_t KM, int32_t row_bytes,
+                               uint32_t* __restrict__ planes, int32_t* __restrict__ flag) {
+  __shared__ uint16_t lut[256];
+  build_base3_lut(lut);
+  __syncthreads();
+  bool bad = false;
+  for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < n_words;
+       w += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = w / KM;
+    const int col = (int)(w % KM);
+    const uint8_t* rp = src + row * (int64_t)row_bytes;
+    const int k_begin = col * 32;
+    uint32_t m = 0, s = 0;
+    for (int j = k_begin / 5; j <= (k_begin + 31) / 5; ++j) {
+      const uint32_t e = lut[__ldg(rp + j)];
+      bad |= (e == 0xFFFFu);
+#pragma unroll
+      for (int i = 0; i < 5; ++i) {
+        const int k = 5 * j + i - k_begin;
+        if (k >= 0 && k < 32) {
+          const int p_m = mask_pos(k);
+          m |= ((e >> i) & 1u) << p_m;
+          s |= ((e >> (5 + i)) & 1u) << ((p_m + 1) & 31);
+        }
+      }
+    }
+    uint32_t* row_p = planes + row * (2 * (int64_t)KM);
+    row_p[col] = m;
+    row_p[KM + col] = s;
+  }
+  if (__any_sync(0xFFFFFFFFu, bad) && (threadIdx.x & 31) == 0) set_flag(flag);
+}
+
+// One thread per transport byte.
+__global__ void k_encode_base3(const int8_t* __restrict__ src, int64_t n_bytes, int32_t K, int32_t row_bytes,
+                               uint8_t* __restrict__ out, int32_t* __restrict__ flag) {
+  bool bad = false;
+  for (int64_t o = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; o < n_bytes;
+       o += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = o / row_bytes;
+    const int j = (int)(o % row_bytes);
+    const int8_t* rp = src + row * (int64_t)K;
+    int b = 0, p3 = 1;
+#pragma unroll
+    for (int i = 0; i < 5; ++i) {
+      const int k = 5 * j + i;
+      int d = 1;
+      if (k < K) {
+        const int t = rp[k];
+        bad |= (t < -1 || t > 1);
+        d = t + 1;
+      }
+      b += d * p3;
+      p3 *= 3;
+    }
+    out[o] = (uint8_t)(b > 242 ? 121 : b);
+  }
+  if (__any_sync(0xFFFFFFFFu, bad) && (threadIdx.x & 31) == 0) set_flag(flag);
+}
+
+// One warp per row: popcounts of the two planes.
+__global__ void k_occupancy(const uint32_t* __restrict__ planes, int32_t N, int32_t K, int64_t* __restrict__ counts) {
+  const int KM = K / 32;
+  const int warps = blockDim.x / 32;
+  for (int row = blockIdx.x * warps + threadIdx.x / 32; row < N; row += gridDim.x * warps) {
+    const uint32_t* rp = planes + (int64_t)row * 2 * KM;
+    int nz = 0, neg = 0;
+    for (int c = threadIdx.x & 31; c < KM; c += 32) {
+      const uint32_t m = rp[c], s = rp[KM + c];
+      nz += __popc(m);
+      neg += __popc(s & __funnelshift_l(m, m, 1));
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+      nz += __shfl_xor_sync(0xFFFFFFFFu, nz, o);
+      neg += __shfl_xor_sync(0xFFFFFFFFu, neg, o);
+    }
+    if ((threadIdx.x & 31) == 0) {
+      counts[3 * (int64_t)row] = K - nz;
+      counts[3 * (int64_t)row + 1] = nz - neg;
+      counts[3 * (int64_t)row + 2] = neg;
+    }
+  }
+}
+
+int grid_for(int64_t work, int threads) {
+  int64_t g = (work + threads - 1) / threads;
+  return (int)(g < 1 ? 1 : (g > 148 * 32 ? 148 * 32 : g));
+}
+
+}  // namespace
+
+cudaError_t launch_pack_trits(const int8_t* src, int32_t N, int32_t K, uint32_t* planes, int32_t* flag,
+                              cudaStream_t st) {
+  const int64_t n_words = (int64_t)N * (K / 32);
+  k_pack_trits<<<grid_for(n_words, 256), 256, 0, st>>>(src, n_words, K / 32, planes, flag);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpack_base3(const uint8_t* src, int32_t N, int32_t K, uint32_t* planes, int32_t* flag,
+                                cudaStream_t st) {
+  const int64_t n_words = (int64_t)N * (K / 32);
+  k_unpack_base3<<<grid_for(n_words, 256), 256, 0, st>>>(src, n_words, K / 32, (K + 4) / 5, planes, flag);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_encode_base3(const int8_t* src, int32_t N, int32_t K, uint8_t* out, int32_t* flag,
+                                cudaStream_t st) {
+  const int64_t n_bytes = (int64_t)N * ((K + 4) / 5);
+  k_encode_base3<<<grid_for(n_bytes, 256), 256, 0, st>>>(src, n_bytes, K, (K + 4) / 5, out, flag);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_occupancy(const uint32_t* planes, int32_t N, int32_t K, int64_t* counts, cudaStream_t st) {
+  k_occupancy<<<grid_for((int64_t)N * 32, 256), 256, 0, st>>>(planes, N, K, counts);
+  return cudaGetLastError();
+}
+
+}  // namespace tern

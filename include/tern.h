@@ -58,6 +58,12 @@
 extern "C" {
 #endif
 
+/* Everything declared below is exported from libterngemv.so, which is otherwise built with
+ * hidden symbol visibility. */
+#if defined(__GNUC__)
+#pragma GCC visibility push(default)
+#endif
+
 /* Same object as cudaStream_t; declared here so that this header needs no CUDA header. */
 typedef struct CUstream_st* tern_stream_t;
 
@@ -181,6 +187,10 @@ tern_status i8_head_gemv_argmax_ex(const int8_t* W_dev, const uint16_t* scale_f1
 
 /* Synchronise `stream`, read *err_flag_dev and map it: 0 -> TERN_OK, nonzero -> TERN_EBADCODE. */
 tern_status tern_read_flag(const int32_t* err_flag_dev, tern_stream_t stream);
+
+#if defined(__GNUC__)
+#pragma GCC visibility pop
+#endif
 
 #ifdef __cplusplus
 }  /* extern "C" */
