@@ -1,0 +1,636 @@
+"""Benchmark of the packed-ternary decode path on B200.
+
+One step = one decode token at M = 1 through the synthetic 8B-geometry linear stack (36 layers,
+each as four fused launches: q|k|v 6144x4096, o 4096x4096, gate|up 24576x4096, down 4096x12288,
+i.e. all 252 ternary linears) plus the int8 output head 151936x4096 with fused argmax, bf16
+activations. Weights are packed on the device from the seeded generator (synth), activations
+are N(0,1) bf16; every input of a step (2.37 GB) is far larger than the 126 MB L2, so each step
+streams its weights from HBM.
+
+Prints one JSON line (rank 0). --impl reference times the CPU oracle instead (the same workload,
+a bounded sample per step, extrapolated to a token).
+
+The timed region replays CUDA graphs of captured steps (kernels launched with programmatic
+dependent launch); each kernel reads its activations only after the previous kernel finished,
+as in a real decode chain. Extra rows measure the other scope rows (single GEMV, int8 mode,
+0.6B stack, small-M sweep, base-3 unpack).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ternary GEMV HBM GB/s & 8B linear-stack tok/s at M=1 (fraction of HBM peak)"
+SEED = 0x7E2A2026
+L2_BYTES = 126 * 1024 * 1024
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------------------------------------
+# synthetic model on the device
+class Linear:
+    """A fused packed-ternary launch: rows of several projections stacked (same input)."""
+
+    def __init__(self, W, N, K, parts):
+        self.W, self.N, self.K, self.parts = W, N, K, parts
+
+    @property
+    def bytes(self):
+        # algorithmic bytes of one M=1 launch: planes + scales + activation in + output out
+        return self.N * self.K // 4 + 2 * self.N + 2 * self.K + 4 * self.N
+
+
+def build_linear(model, layer, projs, seed=SEED):
+    import torch
+    import bit_gemv_tern_b200 as tg
+    import synth
+    import synth.cuda as sc
+    shapes = {p: (N, K) for p, N, K in synth.linear_shapes(model)}
+    K = shapes[projs[0]][1]
+    N = sum(shapes[p][0] for p in projs)
+    tr = torch.empty(N * K, dtype=torch.int8, device="cuda")
+    scales, r = [], 0
+    for p in projs:
+        n = shapes[p][0]
+        tid = synth.tensor_id(layer, p)
+        sc.trits_into(tr[r * K:(r + n) * K], seed, tid, K, synth.trit_probs(model, layer, p))
+        scales.append(synth.row_scales(seed, tid, n))
+        r += n
+    W = tg.TernMatrix.empty(N, K)
+    W.scale.copy_(torch.from_numpy(np.concatenate(scales).view(np.float16)))
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tg.tern_pack(tg.TERN_SRC_INT8_TRITS, tr, N, K, W.planes, flag)
+    assert tg.tern_read_flag(flag) == 0
+    del tr
+    return Linear(W, N, K, projs)
+
+
+class Stack:
+    """A model's fused linears + int8 head with activations for M rows, on the device."""
+
+    def __init__(self, model, M=1, seed=SEED, layers=None):
+        import torch
+        import synth
+        import synth.cuda as sc
+        g = synth.GEOMETRY[model]
+        self.model, self.M = model, M
+        self.L = g["layers"] if layers is None else layers
+        self.V, self.d = g["vocab"], g["d"]
+        self.linears, self.x_tid = [], []
+        for layer in range(self.L):
+            for grp, projs in synth.FUSED_GROUPS:
+                self.linears.append(build_linear(model, layer, projs, seed))
+                self.x_tid.append(synth.act_tensor_id(model, layer, grp))
+        htid = synth.head_tensor_id(model)
+        self.head_W = torch.empty(self.V * self.d, dtype=torch.int8, device="cuda")
+        sc.head_into(self.head_W, seed, htid, self.d)
+        self.head_s = torch.from_numpy(synth.head_scales(seed, htid, self.V).view(np.float16)).cuda()
+        # activations: one bf16 [M, K] per fused launch + the head input, in one contiguous buffer
+        xs = [synth.activations(seed, tid, M, lin.K) for tid, lin in zip(self.x_tid, self.linears)]
+        xs.append(synth.activations(seed, synth.head_act_tensor_id(model), M, self.d))
+        self.x_offsets, off = [], 0
+        for a in xs:
+            self.x_offsets.append(off)
+            off += a.size
+        self.x_host = torch.empty(off, dtype=torch.int16, pin_memory=True)
+        flat = np.concatenate([a.reshape(-1) for a in xs]).view(np.int16)
+        self.x_host.numpy()[:] = flat
+        self.x = self.x_host.cuda()
+        self.y = [torch.empty(M * lin.N, dtype=torch.float32, device="cuda") for lin in self.linears]
+        # int8 mode inputs (quantised once; a full model fuses this into the producing kernel)
+        self.q = torch.empty(off, dtype=torch.int8, device="cuda")
+        self.sx = torch.empty(len(xs) * M, dtype=torch.float32, device="cuda")
+        self.argmax = torch.empty(M, dtype=torch.int32, device="cuda")
+        self.maxval = torch.empty(M, dtype=torch.float32, device="cuda")
+        import bit_gemv_tern_b200 as tg
+        self.ws = torch.zeros(tg.i8_head_workspace_bytes(self.V, M), dtype=torch.uint8, device="cuda")
+        self.result_host = torch.empty(2 * M, dtype=torch.int32, pin_memory=True)
+        self._batches = {}
+        for i, (o, a) in enumerate(zip(self.x_offsets, xs)):
+            K = a.shape[1]
+            tg.tern_quantize_act(self.x[o:o + M * K], M, K, self.q[o:o + M * K], self.sx[i * M:(i + 1) * M])
+        torch.cuda.synchronize()
+
+    def xs(self, i):
+        K = self.linears[i].K if i < len(self.linears) else self.d
+        o = self.x_offsets[i]
+        return self.x[o:o + self.M * K], self.q[o:o + self.M * K], self.sx[i * self.M:(i + 1) * self.M]
+
+    @property
+    def stack_bytes(self):
+        return sum(l.bytes + (self.M - 1) * (2 * l.K + 4 * l.N) for l in self.linears)
+
+    @property
+    def head_bytes(self):
+        return self.V * self.d + 2 * self.V + 2 * self.M * self.d + 8 * self.M
+
+    def batch(self, mode):
+        """The stack's M = 1 GEMVs as one tern_gemv_batch (independent activations)."""
+        import bit_gemv_tern_b200 as tg
+        if mode not in self._batches:
+            act = tg.TERN_ACT_BF16 if mode == "bf16" else tg.TERN_ACT_INT8
+            entries = []
+            for i, lin in enumerate(self.linears):
+                xb, q, sx = self.xs(i)
+                entries.append((lin.W, xb if mode == "bf16" else q, None if mode == "bf16" else sx, self.y[i]))
+            self._batches[mode] = tg.GemvBatch(entries, act)
+        return self._batches[mode]
+
+    def launch_stack(self, mode="bf16", pdl=True, chained=False):
+        """M = 1: one batched launch pair for all linears (their activations are independent
+        inputs); chained=True launches one GEMV per linear instead, each waiting for the previous
+        kernel before reading its activation (a decode chain)."""
+        import bit_gemv_tern_b200 as tg
+        act = tg.TERN_ACT_BF16 if mode == "bf16" else tg.TERN_ACT_INT8
+        fl = tg.TERN_FLAG_PDL if pdl else 0
+        if self.M == 1 and not chained:
+            self.batch(mode)(flags=fl)
+            return
+        for i, lin in enumerate(self.linears):
+            xb, q, sx = self.xs(i)
+            if self.M == 1:
+                tg.tern_gemv(lin.W, act, xb if act == tg.TERN_ACT_BF16 else q, None if act == tg.TERN_ACT_BF16 else sx,
+                             self.y[i], flags=fl)
+            else:
+                tg.tern_gemm_small_m(lin.W, self.M, act, xb if act == tg.TERN_ACT_BF16 else q,
+                                     None if act == tg.TERN_ACT_BF16 else sx, self.y[i], flags=fl)
+
+    def launch_head(self, mode="bf16", pdl=True):
+        import bit_gemv_tern_b200 as tg
+        act = tg.TERN_ACT_BF16 if mode == "bf16" else tg.TERN_ACT_INT8
+        xb, q, sx = self.xs(len(self.linears))
+        tg.i8_head_gemv_argmax(self.head_W, self.head_s, self.V, self.d, self.M, act,
+                               xb if act == tg.TERN_ACT_BF16 else q, None if act == tg.TERN_ACT_BF16 else sx,
+                               self.argmax, self.maxval, None, self.ws, flags=tg.TERN_FLAG_PDL if pdl else 0)
+
+    @property
+    def launches_per_step(self):
+        return 3 if self.M == 1 else len(self.linears) + 1
+
+
+def capture(fn, steps, events=None):
+    """CUDA graph of `steps` repetitions of fn(step_index, events)."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(g, stream=s):
+        for i in range(steps):
+            fn(i)
+    torch.cuda.current_stream().wait_stream(s)
+    return g
+
+
+def timed_replays(graphs_and_counts):
+    """Replay graphs back to back between two events; returns elapsed ms."""
+    import torch
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record()
+    for g, n in graphs_and_counts:
+        for _ in range(n):
+            g.replay()
+    b.record()
+    b.synchronize()
+    return a.elapsed_time(b)
+
+
+# ---------------------------------------------------------------------------------------------
+# clocks during the timed region
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu, self.proc, self.path = gpu_index, None, None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        out = {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        try:
+            rows = [l.split(",") for l in open(self.path).read().strip().splitlines() if l.strip()]
+            os.unlink(self.path)
+        except Exception:
+            return out
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [c.strip() for c in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1])); mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if sm:
+            out = {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                   "samples": len(sm)}
+        return out
+
+
+# ---------------------------------------------------------------------------------------------
+def _oracle_sample(rows=256):
+    """Inputs for the CPU oracle: `rows` rows of each fused 8B launch and 4x as many head rows."""
+    import oracle
+    import synth
+    shapes = {p: (N, K) for p, N, K in synth.linear_shapes("8b")}
+    fused = [(grp, sum(shapes[p][0] for p in projs), shapes[projs[0]][1]) for grp, projs in synth.FUSED_GROUPS]
+    mats = []
+    for grp, N, K in fused:
+        t = synth.trits(SEED, 9000 + K, rows, K)
+        mats.append((grp, N, K, oracle.pack(t), synth.row_scales(SEED, 9000 + K, rows),
+                     synth.activations(SEED, 9000 + K, 1, K)))
+    d = synth.GEOMETRY["8b"]["d"]
+    head = (synth.head_weights(SEED, 9999, 4 * rows, d), synth.head_scales(SEED, 9999, 4 * rows),
+            synth.activations(SEED, 9999, 1, d))
+    return mats, head, rows
+
+
+def _oracle_token_seconds(sample, threads, budget_s):
+    """Time the oracle on the sample (repeating calls until budget_s is spent) and scale by rows to
+    one 8B token: 36 layers x 4 fused launches + the 151936-row head. Returns (s/token, s measured)."""
+    import oracle
+    import synth
+    mats, head, rows = sample
+    L, V = synth.GEOMETRY["8b"]["layers"], synth.GEOMETRY["8b"]["vocab"]
+    per_row = {}
+    spent, reps = 0.0, 0
+    tot = {}
+    while True:
+        for grp, N, K, pl, s, x in mats:
+            t0 = time.perf_counter()
+            oracle.gemm_bf16(pl, s, K, x, nthreads=threads)
+            dt = time.perf_counter() - t0
+            tot[grp] = tot.get(grp, 0.0) + dt
+            spent += dt
+        t0 = time.perf_counter()
+        oracle.head_bf16(head[0], head[1], head[2], nthreads=threads)
+        dt = time.perf_counter() - t0
+        tot["head"] = tot.get("head", 0.0) + dt
+        spent += dt
+        reps += 1
+        if spent >= budget_s:
+            break
+    t_token = sum(tot[grp] / (reps * rows) * N * L for grp, N, K, _, _, _ in mats)
+    t_token += tot["head"] / (reps * 4 * rows) * V
+    return t_token, spent
+
+
+def cpu_baseline(budget_s=12.0):
+    """The oracle on this host's cores on a bounded sample of the 8B token, scaled to tok/s."""
+    threads = os.cpu_count() or 1
+    sample = _oracle_sample()
+    t_token, spent = _oracle_token_seconds(sample, threads, budget_s)
+    return {"value": 1.0 / t_token, "unit": "tok/s", "cores": threads, "kind": "oracle",
+            "sample": f"{sample[2]} rows of each fused 8B launch (q|k|v, o, gate|up, down; full K) and "
+                      f"{4 * sample[2]} head rows (K=4096), fp64 oracle, calls repeated for {spent:.1f} s, "
+                      f"per-row time scaled to 36 layers + the 151936-row head"}
+
+
+# ---------------------------------------------------------------------------------------------
+def run_reference(args, rank, world):
+    """The CPU oracle as the reference arm: each step times the oracle on a bounded sample of the
+    token (sized so that warm-up + steps take about a minute), extrapolated to tok/s."""
+    if rank != 0:
+        return 0
+    threads = os.cpu_count() or 1
+    sample = _oracle_sample()
+    per_step = max(0.002, 60.0 / (args.steps + args.warmup))
+    for _ in range(args.warmup):
+        _oracle_token_seconds(sample, threads, per_step)
+    toks, spent = [], 0.0
+    for _ in range(args.steps):
+        t, sp = _oracle_token_seconds(sample, threads, per_step)
+        toks.append(t)
+        spent += sp
+    t_token = statistics.median(toks)
+    cb = {"value": 1.0 / t_token, "unit": "tok/s", "cores": threads, "kind": "oracle",
+          "sample": f"per step: {sample[2]} rows of each fused 8B launch and {4 * sample[2]} head rows, "
+                    f"oracle calls repeated for >= {per_step * 1000:.0f} ms, per-row time scaled to a token; "
+                    f"median over {args.steps} steps ({spent:.1f} s measured)"}
+    line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "tok/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * t_token,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": "8b_linear_stack_m1_bf16_plus_int8_head", "model": "neutrino-1-8b-geometry",
+                       "global_batch": 1, "seq_len": 1, "parallelism": "none (host cores)"},
+            "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-rows", action="store_true", help="skip the extra scope rows")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    import bit_gemv_tern_b200 as tg
+    from bit_gemv_tern_b200 import build as _b
+    _b.build()
+    hbm_peak, bf16_peak, bf16_sust, peak_kind = peaks()
+
+    stack = Stack("8b", M=1)
+    n_linear = len(stack.linears)
+    S = min(args.steps, 100)
+    R, rem = divmod(args.steps, S)
+    ev = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True),
+           torch.cuda.Event(enable_timing=True, external=True)) for _ in range(S)]
+
+    def step(i):
+        if i < len(ev):
+            ev[i][0].record()
+        stack.launch_stack("bf16")
+        if i < len(ev):
+            ev[i][1].record()
+        stack.launch_head("bf16")
+        if i < len(ev):
+            ev[i][2].record()
+
+    g_main = capture(step, S)
+    g_rem = capture(lambda i: (stack.launch_stack("bf16"), stack.launch_head("bf16")), rem) if rem else None
+    g_warm = capture(lambda i: (stack.launch_stack("bf16"), stack.launch_head("bf16")), args.warmup)
+    g_warm.replay()
+    torch.cuda.synchronize()
+
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ms = timed_replays([(g_main, R)] + ([(g_rem, 1)] if g_rem else []))
+    barrier()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(ms)
+    clocks = clk.summary()
+    ms_step = ms / args.steps
+    value = world * args.steps / (ms / 1000.0)
+
+    # dominant kernel: the ternary GEMV launches of the last replay's steps
+    stack_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(S)]
+    head_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(S)]
+    gemv_s = statistics.median(stack_ms) / 1000.0
+    gemv_gbs = stack.stack_bytes / gemv_s / 1e9
+    head_gbs = stack.head_bytes / (statistics.median(head_ms) / 1000.0) / 1e9
+    step_bytes = stack.stack_bytes + stack.head_bytes
+
+    # end to end through the C ABI: H2D of the step's activations, the step, D2H of the argmax
+    g_one = capture(lambda i: (stack.launch_stack("bf16"), stack.launch_head("bf16")), 1)
+    n_e2e = min(args.steps, 300)
+    res = torch.empty(2, dtype=torch.int32, device="cuda")
+    barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(n_e2e):
+        stack.x.copy_(stack.x_host, non_blocking=True)
+        g_one.replay()
+        res[0:1].copy_(stack.argmax)
+        res[1:2].copy_(stack.maxval.view(torch.int32))
+        stack.result_host.copy_(res, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+    e2e_s = max_over_ranks(time.perf_counter() - t0)
+    e2e = {"value": world * n_e2e / e2e_s, "unit": "tok/s",
+           "h2d_bytes_per_step": int(stack.x_host.numel() * 2), "d2h_bytes_per_step": 8, "steps": n_e2e,
+           "note": "per step: pinned-host activations -> device, graph of the step's launches, argmax + max logit -> host, stream sync"}
+
+    rows = {}
+    if not args.no_rows:
+        rows = extra_rows(stack, torch, tg, hbm_peak, bf16_peak)
+    cb = None
+    if rank == 0 and not args.no_cpu:
+        cb = cpu_baseline()
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "8b_linear_stack_m1_bf16_plus_int8_head",
+                       "model": "neutrino-1-8b-geometry (36 x 7 ternary linears as 144 fused launches + int8 head 151936x4096)",
+                       "global_batch": world, "seq_len": 1, "parallelism": f"replicas x{world}" if world > 1 else "none",
+                       "step_bytes": step_bytes, "l2": "inputs larger than L2: every step streams 2.37 GB of weights from HBM",
+                       "graph": f"{S}-step CUDA graph x {R}" + (f" + {rem}-step graph" if rem else "") + ", PDL launches"},
+            "gbs": step_bytes / (ms_step / 1000.0) / 1e9,
+            "hbm_frac_step": step_bytes / (ms_step / 1000.0) / 1e9 / hbm_peak,
+            "roofline": {"bound": "hbm", "kernel": "k_batch_prep + k_batch_stream<bf16> (all 144 fused GEMVs of the step in one persistent launch)",
+                         "achieved": gemv_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gemv_gbs / hbm_peak,
+                         "peak_kind": f"{peak_kind} hbm_gbs (copy)", "traffic": None,
+                         "algorithmic_bytes_per_step": stack.stack_bytes, "launches": n_linear,
+                         "head": {"kernel": "k_head<bf16,1>", "achieved": head_gbs, "frac": head_gbs / hbm_peak}},
+            "cpu_baseline": cb,
+            "e2e": e2e,
+            "clocks": clocks,
+            "gpu_launches": stack.launches_per_step * args.steps,
+            "rows": rows,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def extra_rows(stack, torch, tg, hbm_peak, bf16_peak):
+    """The other scope rows, each timed with CUDA events over graph replays."""
+    out = {}
+
+    def gbs_of(nbytes, ms):
+        return nbytes / (ms / 1000.0) / 1e9
+
+    # int8-activation mode on the same 8B stack
+    reps = 50
+    g = capture(lambda i: (stack.launch_stack("int8"), stack.launch_head("int8")), 10)
+    g.replay()
+    ms = timed_replays([(g, reps // 10)]) / reps
+    nb = stack.stack_bytes - sum(l.K for l in stack.linears) + stack.head_bytes - stack.d
+    out["8b_stack_m1_int8"] = {"tok_s": 1000.0 / ms, "ms": ms, "gbs": gbs_of(nb, ms), "frac": gbs_of(nb, ms) / hbm_peak}
+    # decode-chain variant: one launch per fused linear, each waiting for its predecessor (PDL)
+    g = capture(lambda i: (stack.launch_stack("bf16", chained=True), stack.launch_head("bf16")), 10)
+    g.replay()
+    ms = timed_replays([(g, 5)]) / 50
+    nb = stack.stack_bytes + stack.head_bytes
+    out["8b_stack_m1_bf16_chained"] = {"tok_s": 1000.0 / ms, "ms": ms, "gbs": gbs_of(nb, ms), "frac": gbs_of(nb, ms) / hbm_peak,
+                                      "launches_per_step": len(stack.linears) + 1}
+    # stack only (no head), bf16
+    g = capture(lambda i: stack.launch_stack("bf16"), 10)
+    g.replay()
+    ms = timed_replays([(g, 5)]) / 50
+    out["8b_stack_only_m1_bf16"] = {"tok_s": 1000.0 / ms, "ms": ms, "gbs": gbs_of(stack.stack_bytes, ms),
+                                    "frac": gbs_of(stack.stack_bytes, ms) / hbm_peak}
+
+    # single GEMV 3072 x 1024 (the small configuration), L2 defeated by rotating replicas
+    import synth
+    reps_w = int(math.ceil(3 * L2_BYTES / (3072 * 1024 // 4)))
+    lin = build_linear("0.6b", 0, ("gate",))
+    planes = torch.empty(reps_w * lin.W.planes.numel(), dtype=torch.int32, device="cuda")
+    for r in range(reps_w):
+        planes[r * lin.W.planes.numel():(r + 1) * lin.W.planes.numel()].copy_(lin.W.planes)
+    mats = [tg.TernMatrix(planes[r * lin.W.planes.numel():(r + 1) * lin.W.planes.numel()], lin.W.scale, 3072, 1024)
+            for r in range(reps_w)]
+    x = torch.from_numpy(synth.activations(SEED, 7, 1, 1024).view(np.int16)).cuda()
+    y = torch.empty(3072, dtype=torch.float32, device="cuda")
+    g = capture(lambda i: tg.tern_gemv(mats[i], tg.TERN_ACT_BF16, x, None, y, flags=tg.TERN_FLAG_PDL), reps_w)
+    g.replay()
+    ms = timed_replays([(g, 4)]) / (4 * reps_w)
+    out["gemv_3072x1024_bf16"] = {"us": ms * 1000.0, "gbs": gbs_of(lin.bytes, ms), "frac": gbs_of(lin.bytes, ms) / hbm_peak,
+                                  "replicas": reps_w}
+    del planes, mats
+
+    # 0.6B stack + tied head (the second configuration)
+    s06 = Stack("0.6b", M=1)
+    g = capture(lambda i: (s06.launch_stack("bf16"), s06.launch_head("bf16")), 20)
+    g.replay()
+    ms = timed_replays([(g, 10)]) / 200
+    nb = s06.stack_bytes + s06.head_bytes
+    out["0.6b_stack_m1_bf16"] = {"tok_s": 1000.0 / ms, "ms": ms, "gbs": gbs_of(nb, ms), "frac": gbs_of(nb, ms) / hbm_peak,
+                                 "launches_per_step": s06.launches_per_step}
+    del s06
+
+    # small-M sweep on the 8B stack + head (speculative verify)
+    sweep = {}
+    for M in (1, 2, 4, 7, 8, 16):
+        sm = stack if M == 1 else StackView(stack, M)
+        g = capture(lambda i: (sm.launch_stack("bf16"), sm.launch_head("bf16")), 5)
+        g.replay()
+        ms = timed_replays([(g, 4)]) / 20
+        nb = sm.stack_bytes + sm.head_bytes
+        sweep[str(M)] = {"pass_us": ms * 1000.0, "tokens_per_s": M * 1000.0 / ms, "gbs": gbs_of(nb, ms),
+                         "frac": gbs_of(nb, ms) / hbm_peak}
+        del g
+    out["small_m_8b_bf16"] = sweep
+
+    # base-3 transport unpack of all 8B trits (bit-exact expansion into the planes)
+    out["base3_unpack_8b"] = base3_row(stack, torch, tg, hbm_peak)
+    return out
+
+
+class StackView:
+    """The 8B stack's weights with M activation rows (for the small-M sweep)."""
+
+    def __init__(self, base, M):
+        import torch
+        import synth
+        self.base, self.M, self.linears, self.V, self.d = base, M, base.linears, base.V, base.d
+        self.x = torch.from_numpy(synth.activations(SEED, 5000 + M, M, 12288).view(np.int16)).cuda()
+        self.y = [torch.empty(M * l.N, dtype=torch.float32, device="cuda") for l in base.linears]
+        self.argmax = torch.empty(M, dtype=torch.int32, device="cuda")
+        self.maxval = torch.empty(M, dtype=torch.float32, device="cuda")
+        import bit_gemv_tern_b200 as tg
+        self.ws = torch.zeros(tg.i8_head_workspace_bytes(self.V, M), dtype=torch.uint8, device="cuda")
+
+    stack_bytes = Stack.stack_bytes
+    head_bytes = Stack.head_bytes
+
+    def launch_stack(self, mode="bf16", pdl=True):
+        import bit_gemv_tern_b200 as tg
+        for i, lin in enumerate(self.linears):
+            tg.tern_gemm_small_m(lin.W, self.M, tg.TERN_ACT_BF16, self.x[:self.M * lin.K], None, self.y[i],
+                                 flags=tg.TERN_FLAG_PDL if pdl else 0)
+
+    def launch_head(self, mode="bf16", pdl=True):
+        import bit_gemv_tern_b200 as tg
+        tg.i8_head_gemv_argmax(self.base.head_W, self.base.head_s, self.V, self.d, self.M, tg.TERN_ACT_BF16,
+                               self.x[:self.M * self.d], None, self.argmax, self.maxval, None, self.ws,
+                               flags=tg.TERN_FLAG_PDL if pdl else 0)
+
+
+def base3_row(stack, torch, tg, hbm_peak):
+    import synth
+    import synth.cuda as sc
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    encs, outs, shapes = [], [], []
+    for p, N, K in synth.linear_shapes("8b"):
+        t = torch.empty(N * K, dtype=torch.int8, device="cuda")
+        sc.trits_into(t, SEED, synth.tensor_id(0, p), K)
+        e = torch.empty(tg.tern_base3_bytes(N, K), dtype=torch.uint8, device="cuda")
+        tg.tern_base3_encode(t, N, K, e, flag)
+        encs.append(e)
+        outs.append(torch.empty(N * K // 16, dtype=torch.int32, device="cuda"))
+        shapes.append((N, K))
+        del t
+    # one layer's seven tensors stand for each of the 36 identical-shape layers
+    g = capture(lambda i: [tg.tern_pack(tg.TERN_SRC_BASE3, e, N, K, o, flag) for e, o, (N, K) in zip(encs, outs, shapes)], 36)
+    g.replay()
+    ms = timed_replays([(g, 3)]) / 3
+    nb = 36 * sum(e.numel() + o.numel() * 4 for e, o in zip(encs, outs))
+    assert tg.tern_read_flag(flag) == 0
+    return {"ms": ms, "gbs": nb / (ms / 1000.0) / 1e9, "frac": nb / (ms / 1000.0) / 1e9 / hbm_peak,
+            "trits": 36 * sum(N * K for N, K in shapes), "bytes": nb}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -20,7 +20,9 @@ __all__ = [
     "TERN_ACT_BF16", "TERN_ACT_INT8", "TERN_SRC_INT8_TRITS", "TERN_SRC_BASE3", "TERN_FLAG_PDL",
     "tern_packed_bytes", "tern_base3_bytes", "tern_pack", "tern_base3_encode", "tern_occupancy",
     "tern_quantize_act", "tern_gemv", "tern_gemm_small_m", "tern_gemm_prefill",
-    "i8_head_workspace_bytes", "i8_head_gemv_argmax", "tern_read_flag", "tern_status_string",
+    "i8_head_workspace_bytes", "i8_head_gemv_argmax", "tern_read_flag", "tern_device_status",
+    "GemvBatch", "tern_gemv_batch", "tern_gemv_batch_workspace_bytes",
+    "tern_status_string",
 ]
 
 TERN_OK, TERN_EINVAL, TERN_ESHAPE, TERN_EBADCODE, TERN_ECUDA, TERN_ETIMEOUT = range(6)
@@ -70,6 +72,9 @@ def lib() -> ctypes.CDLL:
             "i8_head_gemv_argmax": ([vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp], i32),
             "i8_head_gemv_argmax_ex": ([vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, sz, u32, vp], i32),
             "tern_read_flag": ([vp, vp], i32),
+            "tern_device_status": ([vp], i32),
+            "tern_gemv_batch_workspace_bytes": ([vp, i32, i32], sz),
+            "tern_gemv_batch": ([vp, i32, i32, vp, sz, u32, vp], i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -96,6 +101,11 @@ def _stream(stream) -> int:
     import torch
     s = stream if stream is not None else torch.cuda.current_stream()
     return int(s.cuda_stream)
+
+
+class _Item(ctypes.Structure):
+    _fields_ = [("W", _Matrix), ("x_dev", ctypes.c_void_p), ("x_scale_dev", ctypes.c_void_p),
+                ("y_dev", ctypes.c_void_p)]
 
 
 class TernMatrix:
@@ -175,3 +185,49 @@ def tern_read_flag(err_flag, stream=None) -> int:
     if st not in (TERN_OK, TERN_EBADCODE):
         raise TernError(st, "tern_read_flag")
     return st
+
+
+def tern_device_status(stream=None) -> int:
+    """Synchronise and return TERN_OK, or TERN_ETIMEOUT if a kernel gave up a bounded wait."""
+    return int(lib().tern_device_status(_stream(stream)))
+
+
+def _items(entries):
+    arr = (_Item * len(entries))()
+    for i, (W, x, x_scale, y) in enumerate(entries):
+        arr[i].W = W._c
+        arr[i].x_dev = _ptr(x)
+        arr[i].x_scale_dev = _ptr(x_scale)
+        arr[i].y_dev = _ptr(y)
+    return arr
+
+
+def tern_gemv_batch_workspace_bytes(entries, act: int) -> int:
+    """entries: list of (TernMatrix, x, x_scale or None, y)."""
+    arr = _items(entries)
+    return int(lib().tern_gemv_batch_workspace_bytes(arr, len(entries), act))
+
+
+def tern_gemv_batch(entries, act: int, workspace, flags: int = 0, stream=None) -> None:
+    arr = _items(entries)
+    _check(lib().tern_gemv_batch(arr, len(entries), act, _ptr(workspace),
+                                 int(workspace.numel() * workspace.element_size()), flags, _stream(stream)),
+           "tern_gemv_batch")
+
+
+class GemvBatch:
+    """A fixed list of M = 1 GEMVs with its descriptor array and workspace, launched repeatedly
+    (e.g. inside a captured CUDA graph). entries: list of (TernMatrix, x, x_scale or None, y)."""
+
+    def __init__(self, entries, act: int, device="cuda"):
+        import torch
+        self.entries, self.act = list(entries), act
+        self._arr = _items(self.entries)
+        nbytes = int(lib().tern_gemv_batch_workspace_bytes(self._arr, len(self.entries), act))
+        if nbytes == 0:
+            raise TernError(TERN_ESHAPE, "tern_gemv_batch_workspace_bytes")
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+    def __call__(self, flags: int = 0, stream=None) -> None:
+        _check(lib().tern_gemv_batch(self._arr, len(self.entries), self.act, _ptr(self.workspace),
+                                     int(self.workspace.numel()), flags, _stream(stream)), "tern_gemv_batch")

@@ -2,6 +2,7 @@
 // launch planning and kernel launches. No entry point allocates device memory or keeps state.
 #include <cstdint>
 #include <cuda_runtime.h>
+#include <new>
 
 #include "../../include/tern.h"
 #include "tern_kernels.h"
@@ -9,6 +10,11 @@
 namespace {
 
 constexpr int kSMs = 148;
+
+// Consumer warps of the M = 1 streaming kernel (8: two CTAs per SM; 16: one CTA per SM).
+#ifndef TERN_STREAM_CW
+#define TERN_STREAM_CW 16
+#endif
 constexpr size_t kGemmSmemCap = 160 * 1024;
 constexpr size_t kHeadSmemCap = 100 * 1024;
 
@@ -110,6 +116,19 @@ tern_status tern_gemm_small_m_ex(const tern_matrix* W, int32_t M, tern_act act, 
   if (M < 1 || M > 16) return TERN_ESHAPE;
   if (!X_dev || !Y_dev || !aligned(X_dev, 16) || !aligned(Y_dev, 4)) return TERN_EINVAL;
   if (act == TERN_ACT_INT8 && (!x_scale_dev || !aligned(x_scale_dev, 4))) return TERN_EINVAL;
+  if (M == 1) {
+    tern::StreamParams sp = {};
+    sp.cw = TERN_STREAM_CW;
+    size_t smem = 0;
+    if (tern::plan_stream(W->N, W->K, act == TERN_ACT_BF16 ? 0 : 1, sp, smem)) {
+      sp.planes = W->planes;
+      sp.scale = W->scale_f16;
+      sp.x = X_dev;
+      sp.sx = x_scale_dev;
+      sp.y = Y_dev;
+      return from_cuda(tern::launch_stream(sp, smem, (flags & TERN_FLAG_PDL) != 0, cs(stream)));
+    }
+  }
   tern::GemmParams p = {};
   p.planes = W->planes;
   p.scale = W->scale_f16;
@@ -138,6 +157,61 @@ tern_status tern_gemv_ex(const tern_matrix* W, tern_act act, const void* x_dev, 
 tern_status tern_gemv(const tern_matrix* W, tern_act act, const void* x_dev, const float* x_scale_dev,
                       float* y_dev, tern_stream_t stream) {
   return tern_gemm_small_m_ex(W, 1, act, x_dev, x_scale_dev, y_dev, 0u, stream);
+}
+
+namespace {
+
+tern_status fill_batch(const tern_gemv_item* items, int32_t count, tern_act act, tern::BatchParams& bp,
+                       size_t& smem, size_t& ws) {
+  if (!items) return TERN_EINVAL;
+  if (act != TERN_ACT_BF16 && act != TERN_ACT_INT8) return TERN_EINVAL;
+  if (count < 1 || count > TERN_BATCH_MAX_ITEMS) return TERN_ESHAPE;
+  bp.count = count;
+  bp.mode = act == TERN_ACT_BF16 ? 0 : 1;
+  for (int i = 0; i < count; ++i) {
+    const tern_gemv_item& in = items[i];
+    tern_status st = check_matrix(&in.W);
+    if (st != TERN_OK) return st;
+    if (in.W.K > 12288) return TERN_ESHAPE;
+    if (!in.x_dev || !in.y_dev || !aligned(in.x_dev, 16) || !aligned(in.y_dev, 4)) return TERN_EINVAL;
+    if (act == TERN_ACT_INT8 && (!in.x_scale_dev || !aligned(in.x_scale_dev, 4))) return TERN_EINVAL;
+    tern::BatchItem& it = bp.items[i];
+    it.planes = in.W.planes;
+    it.scale = in.W.scale_f16;
+    it.y = in.y_dev;
+    it.x = in.x_dev;
+    it.sx = in.x_scale_dev;
+    it.N = in.W.N;
+    it.K = in.W.K;
+  }
+  if (!tern::plan_batch(bp, smem, ws)) return TERN_ESHAPE;
+  return TERN_OK;
+}
+
+}  // namespace
+
+size_t tern_gemv_batch_workspace_bytes(const tern_gemv_item* items, int32_t count, tern_act act) {
+  static tern::BatchParams bp;   // large; host-side planning only
+  size_t smem = 0, ws = 0;
+  if (fill_batch(items, count, act, bp, smem, ws) != TERN_OK) return 0;
+  return ws;
+}
+
+tern_status tern_gemv_batch(const tern_gemv_item* items, int32_t count, tern_act act, void* workspace_dev,
+                            size_t workspace_bytes, uint32_t flags, tern_stream_t stream) {
+  if (flags & ~TERN_FLAG_PDL) return TERN_EINVAL;
+  if (!workspace_dev || !aligned(workspace_dev, 16)) return TERN_EINVAL;
+  tern::BatchParams* bp = new (std::nothrow) tern::BatchParams();
+  if (!bp) return TERN_EINVAL;
+  size_t smem = 0, ws = 0;
+  tern_status st = fill_batch(items, count, act, *bp, smem, ws);
+  if (st == TERN_OK && workspace_bytes < ws) st = TERN_EINVAL;
+  if (st == TERN_OK) {
+    bp->xprep = static_cast<uint8_t*>(workspace_dev);
+    st = from_cuda(tern::launch_batch(*bp, smem, (flags & TERN_FLAG_PDL) != 0, cs(stream)));
+  }
+  delete bp;
+  return st;
 }
 
 size_t i8_head_workspace_bytes(int32_t V, int32_t M) {
@@ -202,6 +276,13 @@ tern_status tern_read_flag(const int32_t* err_flag_dev, tern_stream_t stream) {
   int32_t v = 0;
   if (cudaMemcpy(&v, err_flag_dev, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return TERN_ECUDA;
   return v == 0 ? TERN_OK : TERN_EBADCODE;
+}
+
+tern_status tern_device_status(tern_stream_t stream) {
+  int v = 0, w = 0;
+  if (tern::read_and_clear_error_latch(&v, cs(stream)) != cudaSuccess) return TERN_ECUDA;
+  if (tern::read_and_clear_batch_latch(&w) != cudaSuccess) return TERN_ECUDA;
+  return (v == 0 && w == 0) ? TERN_OK : TERN_ETIMEOUT;
 }
 
 tern_status tern_gemm_prefill(const tern_matrix* W, int32_t M, const uint16_t* X_bf16_dev, float* Y_dev,

@@ -58,7 +58,25 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// D(16x8) += A(16x32, u8, row) * B(32x8, s8, col), s32 accumulate.
+__device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // ---- decode ------------------------------------------------------------------------------------
+// Offset-binary merge: fields (m, NOT s) read as an unsigned 2-bit number equal t + 2
+// (t = 0 -> 2, t = +1 -> 3, t = -1 -> 1). A field left in place at bit 2i of a byte and masked is
+// the u8 value 4^i * (t + 2): one AND per tensor-core register, no shift. Sums then carry a known
+// offset 2 * sum(x) that is removed exactly.
+__device__ __forceinline__ void merge_planes_offset(uint32_t m, uint32_t s, uint32_t& wa, uint32_t& wb) {
+  wa = (m & 0x55555555u) | (~s & 0xAAAAAAAAu);
+  const uint32_t v = (m & 0xAAAAAAAAu) | (~s & 0x55555555u);
+  wb = __funnelshift_r(v, v, 1);
+}
+
 __device__ __forceinline__ void merge_planes(uint32_t m, uint32_t s, uint32_t& wa, uint32_t& wb) {
   wa = (m & 0x55555555u) | (s & 0xAAAAAAAAu);
   const uint32_t v = (m & 0xAAAAAAAAu) | (s & 0x55555555u);

@@ -219,11 +219,13 @@ __global__ void __launch_bounds__(kThreads) k_tern_gemm(const GemmParams p) {
 template <int MODE, int NG>
 cudaError_t launch_one(const GemmParams& p, size_t smem, bool pdl, cudaStream_t st) {
   auto kern = k_tern_gemm<MODE, NG>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  if (p.ksplit > 1) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+  // Raise the kernel's dynamic shared-memory limit once per size increase (not on every launch).
+  static int smem_set = 0;
+  cudaError_t e = cudaSuccess;
+  if ((int)smem > smem_set) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    smem_set = (int)smem;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.ksplit, (p.N + kRows - 1) / kRows, 1);

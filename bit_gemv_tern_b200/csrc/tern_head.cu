@@ -132,6 +132,8 @@ __global__ void __launch_bounds__(kThreads) k_head(const HeadParams p) {
   }
   __syncthreads();
 
+  // Let the next kernel of the chain get resident and start its own weight prefetch.
+  pdl_launch_dependents();
   constexpr int kCols = 8 * NG;
   int* part = reinterpret_cast<int*>(smem + ncols * RS);
   cg::cluster_group cluster = cg::this_cluster();
@@ -206,7 +208,6 @@ __global__ void __launch_bounds__(kThreads) k_head(const HeadParams p) {
     }
     if (p.ksplit > 1) cluster.sync(); else __syncthreads();
   }
-  pdl_launch_dependents();
 
   // ---- grid-wide argmax: global atomicMax, then the last CTA publishes and resets ----------------
   __syncthreads();
@@ -232,8 +233,14 @@ __global__ void __launch_bounds__(kThreads) k_head(const HeadParams p) {
 template <int MODE, int NG>
 cudaError_t launch_ng(const HeadParams& p, size_t smem, bool pdl, cudaStream_t st) {
   auto kern = k_head<MODE, NG>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
+  // Raise the kernel's dynamic shared-memory limit once per size increase (not on every launch).
+  static int smem_set = 0;
+  cudaError_t e = cudaSuccess;
+  if ((int)smem > smem_set) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    smem_set = (int)smem;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.ksplit, p.nby, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);

@@ -24,6 +24,62 @@ size_t gemm_smem_bytes(int mode, int M, int kr);
 int gemm_rows_per_cta();
 cudaError_t launch_tern_gemm(const GemmParams& p, bool pdl, cudaStream_t st);
 
+// Persistent TMA-fed M = 1 GEMV (tern_stream.cu).
+struct StreamParams {
+  const uint32_t* planes;
+  const uint16_t* scale;
+  int32_t N, K;
+  const void* x;          // bf16 bits [K] (mode 0) or int8 [K] (mode 1)
+  const float* sx;        // [1], int8 mode only
+  float* y;               // [N]
+  int32_t mode;
+  int32_t ks;             // trits of K per stage (divides K)
+  int32_t ts;             // tiles of 16 rows per stage (1, 2, 4 or 8)
+  int32_t pitch;          // shared-memory bytes per staged row
+  int32_t stage_bytes;
+  int32_t stages;         // ring depth
+  int32_t tiles;          // ceil(N / 16)
+  int32_t x_words;        // shared-memory words per staged activation column
+  int32_t cw;             // consumer warps: 8 (two CTAs per SM) or 16 (one CTA per SM)
+};
+bool plan_stream(int N, int K, int mode, StreamParams& p, size_t& smem);
+cudaError_t launch_stream(const StreamParams& p, size_t smem, bool pdl, cudaStream_t st);
+// Reads and clears the device word that kernels set when a bounded wait gives up.
+cudaError_t read_and_clear_error_latch(int* out, cudaStream_t st);
+
+// Batched M = 1 GEMV over a list of matrices (tern_batch.cu).
+struct BatchItem {
+  const uint32_t* planes;
+  const uint16_t* scale;
+  float* y;
+  const void* x;          // bf16 bits [K] or int8 [K]
+  const float* sx;        // int8 mode: [1]
+  int32_t N, K;
+  int32_t ts;             // tiles of 16 rows per stage
+  int32_t kp;             // 512-trit K parts (last may be partial)
+  int32_t unit0;          // first global unit (stage) of the item
+  int32_t units;          // stages of the item
+  uint32_t xoff;          // byte offset of the item's operand block in the workspace
+  int32_t xbytes;         // bytes of that block
+};
+constexpr int kBatchMaxItems = 160;
+struct BatchParams {
+  BatchItem items[kBatchMaxItems];
+  int32_t count;
+  int32_t mode;           // 0 = bf16 activations (three int8 limbs), 1 = int8
+  int32_t nc;             // operand columns: 3 or 1
+  int32_t total_units;
+  int32_t grid;
+  int32_t stages;
+  int32_t stage_slot_bytes;
+  int32_t x_slot_bytes;
+  uint8_t* xprep;         // workspace: operand blocks
+  int32_t cta_unit[149];  // CTA c handles units [cta_unit[c], cta_unit[c + 1])
+};
+bool plan_batch(BatchParams& p, size_t& smem, size_t& workspace);
+cudaError_t launch_batch(const BatchParams& p, size_t smem, bool pdl, cudaStream_t st);
+cudaError_t read_and_clear_batch_latch(int* out);
+
 // int8 output head with argmax (tern_head.cu).
 struct HeadParams {
   const int8_t* W;

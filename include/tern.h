@@ -73,7 +73,7 @@ typedef enum {
   TERN_ESHAPE = 2,    /* N <= 0, K <= 0, K % 128 != 0, M out of range, size overflow          */
   TERN_EBADCODE = 3,  /* device saw an invalid trit / transport byte (via the error flag)     */
   TERN_ECUDA = 4,     /* a CUDA runtime call or kernel launch failed                          */
-  TERN_ETIMEOUT = 5   /* a bounded device-side wait gave up (reserved: no kernel here waits)  */
+  TERN_ETIMEOUT = 5   /* a bounded device-side wait gave up (see tern_device_status)          */
 } tern_status;
 
 typedef enum { TERN_ACT_BF16 = 0, TERN_ACT_INT8 = 1 } tern_act;
@@ -143,6 +143,36 @@ tern_status tern_gemv(const tern_matrix* W, tern_act act, const void* x_dev, con
 tern_status tern_gemv_ex(const tern_matrix* W, tern_act act, const void* x_dev, const float* x_scale_dev,
                          float* y_dev, uint32_t flags, tern_stream_t stream);
 
+/* One M = 1 GEMV of a batch: y[n] = scale[n] * sum_k t[n][k] * x[k] for matrix W. */
+typedef struct {
+  tern_matrix W;              /* packed matrix, K a multiple of 128 and at most 12288           */
+  const void* x_dev;          /* bf16[K] or int8[K] (16-byte aligned)                          */
+  const float* x_scale_dev;   /* int8 mode: &s_x from tern_quantize_act; bf16 mode: ignored     */
+  float* y_dev;               /* float[N]                                                      */
+} tern_gemv_item;
+
+#define TERN_BATCH_MAX_ITEMS 160
+
+/* Workspace bytes tern_gemv_batch needs for these items (0 if the list is invalid). */
+size_t tern_gemv_batch_workspace_bytes(const tern_gemv_item* items, int32_t count, tern_act act);
+
+/* A list of independent M = 1 GEMVs -- e.g. every linear layer of a decode step whose inputs are
+ * ready -- computed by two launches: one that turns every activation into tensor-core operand
+ * blocks in the workspace, and one persistent kernel (one CTA per SM) that streams all the
+ * matrices' packed weights back to back through shared memory, so the weight stream never stops
+ * at a layer boundary (the pages place the time above a decode step's DRAM floor at its kernel
+ * boundaries: [R] "뉴트리노 엔진"). Arithmetic as for tern_gemv; results are deterministic and,
+ * in int8 mode, bit-identical to tern_gemv's. Items must not alias: no y_dev may overlap another
+ * item's weights, activations or outputs.
+ *   items: host array of `count` descriptors (1 <= count <= TERN_BATCH_MAX_ITEMS), read during
+ *          the call only.
+ *   workspace_dev: device scratch of at least tern_gemv_batch_workspace_bytes(...) bytes,
+ *          16-byte aligned; its contents need no initialisation and are overwritten.
+ *   flags: TERN_FLAG_PDL as for tern_gemv_ex (the first launch waits for the preceding kernel
+ *          before reading activations; weights are read only after that launch started). */
+tern_status tern_gemv_batch(const tern_gemv_item* items, int32_t count, tern_act act, void* workspace_dev,
+                            size_t workspace_bytes, uint32_t flags, tern_stream_t stream);
+
 /* Small-M GEMM for the draft-verify pass of speculative decoding ([R] "검증된 추측 디코딩": the
  * 8B scores up to seven drafted positions in one batched forward pass):
  *   Y[m][n] = scale[n] * sum_k t[n][k] * X[m][k],  0 <= m < M, 1 <= M <= 16.
@@ -187,6 +217,12 @@ tern_status i8_head_gemv_argmax_ex(const int8_t* W_dev, const uint16_t* scale_f1
 
 /* Synchronise `stream`, read *err_flag_dev and map it: 0 -> TERN_OK, nonzero -> TERN_EBADCODE. */
 tern_status tern_read_flag(const int32_t* err_flag_dev, tern_stream_t stream);
+
+/* Synchronise `stream` and report whether any kernel of this library on the current device gave
+ * up a bounded wait (an mbarrier that did not complete within seconds) since the last call:
+ * TERN_ETIMEOUT if so, else TERN_OK. Reading clears the device's latch. Kernels that give up
+ * stop early and leave their outputs incomplete; they never hang or trap. */
+tern_status tern_device_status(tern_stream_t stream);
 
 #if defined(__GNUC__)
 #pragma GCC visibility pop

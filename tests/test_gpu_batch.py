@@ -1,0 +1,116 @@
+"""GPU parity of the batched M = 1 GEMV (one prep launch + one persistent streaming launch for a
+whole list of matrices) against the CPU oracle, and its agreement with the single-GEMV path."""
+import numpy as np
+import pytest
+import torch
+
+import bit_gemv_tern_b200 as tg
+import oracle
+import synth
+from gpu_util import check_bf16, dev, host, make_matrix
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [(37, 384), (200, 640), (1, 128), (3072, 1024), (2048, 1024), (1024, 3072), (6144, 4096),
+          (4096, 4096), (129, 12288), (4096, 12288), (24576, 4096)]
+
+
+def _build(seed, shapes, act):
+    items, refs = [], []
+    for i, (N, K) in enumerate(shapes):
+        W, t, s = make_matrix(seed, 100 + i, N, K, host_trits=N * K <= 4096 * 4096)
+        x = synth.activations(seed, 200 + i, 1, K)
+        xd = dev(x.view(np.int16))
+        if act == tg.TERN_ACT_INT8:
+            q = torch.empty(K, dtype=torch.int8, device="cuda")
+            sx = torch.empty(1, dtype=torch.float32, device="cuda")
+            tg.tern_quantize_act(xd, 1, K, q, sx)
+            xin, sxin = q, sx
+        else:
+            xin, sxin = xd, None
+        y = torch.full((N,), float("nan"), dtype=torch.float32, device="cuda")
+        items.append((W, xin, sxin, y))
+        refs.append((t, s, x, i))
+    return items, refs
+
+
+def _rows(N, seed):
+    if N <= 4096:
+        return np.arange(N)
+    r = np.sort(np.random.default_rng(seed).choice(N, 64, replace=False))
+    r[0], r[-1] = 0, N - 1
+    return r
+
+
+@pytest.mark.parametrize("mode", ["bf16", "int8"])
+def test_batch_matches_oracle(mode):
+    act = tg.TERN_ACT_BF16 if mode == "bf16" else tg.TERN_ACT_INT8
+    items, refs = _build(71, SHAPES, act)
+    batch = tg.GemvBatch(items, act)
+    batch()
+    torch.cuda.synchronize()
+    assert tg.tern_device_status() == tg.TERN_OK
+    for (W, xin, sxin, y), (t, s, x, i) in zip(items, refs):
+        N, K = W.N, W.K
+        rows = _rows(N, i)
+        tr = t[rows] if t is not None else synth.trits(71, 100 + i, N, K, rows=rows)
+        yy = host(y)[rows]
+        if mode == "bf16":
+            check_bf16(yy[None, :], oracle.gemm_bf16(oracle.pack(tr), s[rows], K, x), x, s[rows])
+        else:
+            q, sx = host(xin), host(sxin)
+            _, y_ref = oracle.gemm_i8(oracle.pack(tr), s[rows], K, q[None, :], sx)
+            assert (yy == y_ref[0]).all(), (N, K)
+
+
+def test_batch_int8_equals_single_and_is_deterministic():
+    items, _ = _build(72, [(6144, 4096), (4096, 12288), (1000, 1024)], tg.TERN_ACT_INT8)
+    batch = tg.GemvBatch(items, tg.TERN_ACT_INT8)
+    batch()
+    first = [host(y).copy() for (_, _, _, y) in items]
+    batch(flags=tg.TERN_FLAG_PDL)
+    for (W, q, sx, y), a in zip(items, first):
+        b = host(y)
+        assert (a.view(np.uint32) == b.view(np.uint32)).all()
+        y1 = torch.empty_like(y)
+        tg.tern_gemv(W, tg.TERN_ACT_INT8, q, sx, y1)
+        assert (host(y1).view(np.uint32) == b.view(np.uint32)).all()
+
+
+def test_batch_full_8b_layer_sampled():
+    """One 8B layer as its four fused launches (q|k|v, o, gate|up, down) in one batch, bf16."""
+    import bench
+    lins = [bench.build_linear("8b", 2, projs) for _, projs in synth.FUSED_GROUPS]
+    items, xs = [], []
+    for i, lin in enumerate(lins):
+        x = synth.activations(73, i, 1, lin.K)
+        xs.append(x)
+        items.append((lin.W, dev(x.view(np.int16)), None, torch.empty(lin.N, dtype=torch.float32, device="cuda")))
+    tg.GemvBatch(items, tg.TERN_ACT_BF16)()
+    shapes = {p: (N, K) for p, N, K in synth.linear_shapes("8b")}
+    for (grp, projs), lin, (W, xd, _, y), x in zip(synth.FUSED_GROUPS, lins, items, xs):
+        r0 = 0
+        for pj in projs:
+            n = shapes[pj][0]
+            rows = np.sort(np.random.default_rng(n).choice(n, 24, replace=False))
+            tid = synth.tensor_id(2, pj)
+            p = synth.trit_probs("8b", 2, pj)
+            t = synth.trits(synth.DEFAULT_SEED, tid, n, lin.K, p, rows=rows)
+            s = synth.row_scales(synth.DEFAULT_SEED, tid, n)[rows]
+            ref = oracle.gemm_bf16(oracle.pack(t), s, lin.K, x)
+            check_bf16(host(y)[r0 + rows][None, :], ref, x, s)
+            r0 += n
+
+
+def test_batch_argument_errors():
+    W = tg.TernMatrix.empty(64, 128)
+    x = torch.zeros(128, dtype=torch.int16, device="cuda")
+    y = torch.zeros(64, dtype=torch.float32, device="cuda")
+    assert tg.tern_gemv_batch_workspace_bytes([(W, x, None, y)], tg.TERN_ACT_BF16) > 0
+    big = tg.TernMatrix.empty(16, 12288 + 128)
+    assert tg.tern_gemv_batch_workspace_bytes([(big, x, None, y)], tg.TERN_ACT_BF16) == 0
+    ws = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(tg.TernError):
+        tg.tern_gemv_batch([(W, x, None, y)], tg.TERN_ACT_BF16, ws)        # workspace too small
+    with pytest.raises(tg.TernError):
+        tg.tern_gemv_batch([(W, x, None, y)], tg.TERN_ACT_INT8, ws)        # int8 needs s_x
