@@ -168,6 +168,7 @@ tern_status fill_batch(const tern_gemv_item* items, int32_t count, tern_act act,
   if (count < 1 || count > TERN_BATCH_MAX_ITEMS) return TERN_ESHAPE;
   bp.count = count;
   bp.mode = act == TERN_ACT_BF16 ? 0 : 1;
+  const uint32_t* planes[TERN_BATCH_MAX_ITEMS];
   for (int i = 0; i < count; ++i) {
     const tern_gemv_item& in = items[i];
     tern_status st = check_matrix(&in.W);
@@ -176,7 +177,7 @@ tern_status fill_batch(const tern_gemv_item* items, int32_t count, tern_act act,
     if (!in.x_dev || !in.y_dev || !aligned(in.x_dev, 16) || !aligned(in.y_dev, 4)) return TERN_EINVAL;
     if (act == TERN_ACT_INT8 && (!in.x_scale_dev || !aligned(in.x_scale_dev, 4))) return TERN_EINVAL;
     tern::BatchItem& it = bp.items[i];
-    it.planes = in.W.planes;
+    planes[i] = in.W.planes;
     it.scale = in.W.scale_f16;
     it.y = in.y_dev;
     it.x = in.x_dev;
@@ -184,7 +185,7 @@ tern_status fill_batch(const tern_gemv_item* items, int32_t count, tern_act act,
     it.N = in.W.N;
     it.K = in.W.K;
   }
-  if (!tern::plan_batch(bp, smem, ws)) return TERN_ESHAPE;
+  if (!tern::plan_batch(bp, planes, smem, ws)) return TERN_ESHAPE;
   return TERN_OK;
 }
 

@@ -1,4 +1,4 @@
-// Batched M = 1 ternary GEMV: a whole list of linear layers in two launches.
+// Batched M = 1 GEMV: a whole list of linear layers in two launches.
 //
 //   for every item i:  y_i[n] = scale_i[n] * sum_k t_i[n][k] * x_i[k]
 //
@@ -9,20 +9,24 @@
 // launch walks all items, so the weight stream never pauses between layers.
 //
 //   1. k_batch_prep (one CTA per item) turns each activation into ready-to-load tensor-core operand
-//      blocks: int8 q permuted to the decode's byte order (int8 mode), or three exact int8 limbs of
-//      a 22-bit fixed-point value relative to 2^E with E from the item's absmax (bf16 mode), plus
-//      the per-part column sums that remove the decode offset.
-//   2. k_batch_stream (one CTA per SM) splits the list's tile groups evenly by bytes. Its producer
-//      warp streams, in order, each item's operand block into a double buffer and each stage of
-//      weights (TS whole tiles of 16 rows x K, one contiguous cp.async.bulk) into a ring of S
-//      stages. 12 consumer warps walk the stages in order; each warp handles 2 of the stage's 24
-//      (tile, 512-trit K part) pairs: decode (one AND per operand register, see
-//      tern_device.cuh), mma.sync u8 x s8, add the part into the tile's shared-memory accumulator
-//      with integer atomics; the warp that completes a tile writes its outputs.
+//      segments, one per 512-trit K part: int8 q permuted to the decode's byte order (int8 mode),
+//      or three exact int8 limbs of a 22-bit fixed-point value relative to 2^E with E from the
+//      item's absmax (bf16 mode), followed by the item's column sums (which remove the decode
+//      offset) and E.
+//   2. k_batch_stream (one CTA per SM) splits the list's row blocks (kStageRows rows x all of K)
+//      evenly by bytes. Its producer lane walks the CTA's row blocks part by part: each stage of
+//      the ring receives, by tensor TMA, the mask and sign words of the block's rows for one K part
+//      (the packed planes seen as a [plane][row][word] tensor, so the row-major layout is read in
+//      place) plus that part's operand segment. The consumer warps walk the stages in order; warp
+//      w owns kTPW tiles of 16 rows of the block, decodes them (one AND per operand register, see
+//      tern_device.cuh) into mma.sync u8 x s8 products, and keeps the sums in registers across all
+//      parts of the block, so a tile's outputs are written once, at its end.
 // All sums are exact integers; int8 mode ends with y = ((float)acc * s_x) * scale (two fp32
 // round-to-nearest multiplies), bf16 mode with one fp64 -> fp32 rounding. Every mbarrier wait is
 // bounded and latches TERN_ETIMEOUT on give-up.
 #include <cstdint>
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include "tern_device.cuh"
@@ -35,8 +39,15 @@ __device__ int g_batch_latch = 0;
 
 namespace {
 
-constexpr int kCW = 12;                               // consumer warps (one group, in unit order)
+constexpr int kCW = 12;                               // consumer warps
+constexpr int kTPW = 2;                               // tiles of 16 rows per consumer warp
 constexpr int kBatchThreads = (kCW + 1) * 32;
+constexpr int kBoxRows = kCW * 16;                    // rows of one TMA box: tile slot a of every warp
+constexpr int kStageRows = kBoxRows * kTPW;           // rows of a row block
+constexpr int kPartWords = 16;                        // words per plane and row in a 512-trit part
+constexpr int kBoxBytes = 2 * kBoxRows * kPartWords * 4;
+constexpr int kWStageBytes = kTPW * kBoxBytes;
+constexpr int kColWords = 132;                        // operand words per column and part (128 + bank skew)
 constexpr uint32_t kWaitTries = 1u << 13;
 constexpr int kLimbFrac = 22;
 
@@ -66,29 +77,45 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
 }
+// Tiled 3-d tensor load (no multicast): the box at coordinates (word c0, row c1, plane c2).
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
 __device__ __forceinline__ uint32_t u4get(const uint4& v, int e) {
   return e == 0 ? v.x : (e == 1 ? v.y : (e == 2 ? v.z : v.w));
 }
 __device__ __forceinline__ int bsum(uint32_t w) { return __dp4a((int)w, 0x01010101, 0); }
+// 2^e as a double for |e| < 1000 (built from the exponent field: exact).
+__device__ __forceinline__ double exp2_i(int e) { return __longlong_as_double((long long)(e + 1023) << 52); }
 
 // Operand slot of 16-byte half h of word w (0..15) of a 512-trit part: lane t = w / 4 reads the
 // eight words of its word e = w % 4 at ((e * 4) + t) * 8, so a quarter-warp's loads hit distinct banks.
 __device__ __forceinline__ int part_slot(int w, int h) { return ((w & 3) * 4 + (w >> 2)) * 8 + 4 * h; }
 
 // ---------------------------------------------------------------------------------------------
-// prep: one CTA per item
-__global__ void __launch_bounds__(256) k_batch_prep(const BatchParams p) {
+// prep: one CTA per item. Block layout: kp segments of seg_bytes =
+//   [nc columns x kColWords words][nc column sums over all of K][E][padding to 16 bytes].
+__global__ void __launch_bounds__(256) k_batch_prep(const __grid_constant__ BatchParams p) {
   const BatchItem& it = p.items[blockIdx.x];
   uint32_t* blk = reinterpret_cast<uint32_t*>(p.xprep + it.xoff);
   const int K = it.K, KP = it.kp, NC = p.nc;
-  const int xcw = KP * 128 + 4;                      // words per column
-  int* meta = reinterpret_cast<int*>(blk + NC * xcw);  // [KP][NC] sums, then E
+  const int segw = p.seg_bytes / 4;
   __shared__ float red[8];
-  __shared__ int sums[24 * 3];
+  __shared__ int sums[3];
   __shared__ int Esh;
   pdl_wait();
-  for (int i = threadIdx.x; i < NC * xcw; i += blockDim.x) blk[i] = 0u;
-  for (int i = threadIdx.x; i < KP * NC; i += blockDim.x) sums[i] = 0;
+  for (int i = threadIdx.x; i < KP * segw; i += blockDim.x) blk[i] = 0u;
+  if (threadIdx.x < 3) sums[threadIdx.x] = 0;
+  if (threadIdx.x == 0) Esh = 0;
   float f = 1.0f;
   if (p.mode == 0) {
     const uint16_t* xb = static_cast<const uint16_t*>(it.x);
@@ -118,14 +145,15 @@ __global__ void __launch_bounds__(256) k_batch_prep(const BatchParams p) {
   }
   __syncthreads();
   // one 16-element half of a 32-trit word per thread iteration
+  int ls[3] = {0, 0, 0};
   for (int v = threadIdx.x; v < K / 16; v += blockDim.x) {
     const int word = v >> 1, h = v & 1;              // global word index and half
     const int part = word >> 4, w = word & 15;
-    const int slot = part * 128 + part_slot(w, h);
+    uint32_t* seg = blk + part * segw + part_slot(w, h);
     if (p.mode == 1) {
       const uint4 q = ld_nc(static_cast<const int8_t*>(it.x) + 16 * v);
-      atomicAdd(&sums[part], bsum(q.x) + bsum(q.y) + bsum(q.z) + bsum(q.w));
-      *reinterpret_cast<uint4*>(blk + slot) = permute_i8_half(q);
+      ls[0] += bsum(q.x) + bsum(q.y) + bsum(q.z) + bsum(q.w);
+      *reinterpret_cast<uint4*>(seg) = permute_i8_half(q);
     } else {
       const uint16_t* xb = static_cast<const uint16_t*>(it.x) + 16 * v;
       const uint4 a = ld_nc(xb), b = ld_nc(xb + 8);
@@ -146,55 +174,55 @@ __global__ void __launch_bounds__(256) k_batch_prep(const BatchParams p) {
       }
 #pragma unroll
       for (int c = 0; c < 3; ++c) {
-        atomicAdd(&sums[part * 3 + c], bsum(l[c][0]) + bsum(l[c][1]) + bsum(l[c][2]) + bsum(l[c][3]));
-        *reinterpret_cast<uint4*>(blk + c * xcw + slot) = permute_i8_half(make_uint4(l[c][0], l[c][1], l[c][2], l[c][3]));
+        ls[c] += bsum(l[c][0]) + bsum(l[c][1]) + bsum(l[c][2]) + bsum(l[c][3]);
+        *reinterpret_cast<uint4*>(seg + c * kColWords) =
+            permute_i8_half(make_uint4(l[c][0], l[c][1], l[c][2], l[c][3]));
       }
     }
   }
+  for (int c = 0; c < NC; ++c) {
+    int v = ls[c];
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    if ((threadIdx.x & 31) == 0) atomicAdd(&sums[c], v);
+  }
   __syncthreads();
-  for (int i = threadIdx.x; i < KP * NC; i += blockDim.x) meta[i] = sums[i];
-  if (threadIdx.x == 0) meta[KP * NC] = p.mode == 0 ? Esh : 0;
+  // every segment carries the sums over all of K and E, so the consumer reads them from a stage
+  for (int part = threadIdx.x; part < KP; part += blockDim.x) {
+    int* meta = reinterpret_cast<int*>(blk + part * segw + NC * kColWords);
+    for (int c = 0; c < NC; ++c) meta[c] = sums[c];
+    meta[NC] = Esh;
+  }
   pdl_launch_dependents();
 }
 
 // ---------------------------------------------------------------------------------------------
 template <int MODE>
-__global__ void __launch_bounds__(kBatchThreads, 1) k_batch_stream(const BatchParams p) {
-  extern __shared__ __align__(128) uint8_t smem[];
+__global__ void __launch_bounds__(kBatchThreads, 1) k_batch_stream(const __grid_constant__ BatchParams p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
   constexpr int NC = MODE == 0 ? 3 : 1;
   const int S = p.stages;
-  // layout: [bars 512 B][tile counters 512 B][ring S x slot][x buffers 2 x xslot][tile acc S x 12 x 16 x NC]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
-  const uint32_t full0 = smem_u32(bars);                  // [S]
-  const uint32_t empty0 = full0 + 8 * S;                  // [S]
-  const uint32_t xfull0 = empty0 + 8 * S;                 // [2]
-  const uint32_t xempty0 = xfull0 + 16;                   // [2]
-  int* cnt = reinterpret_cast<int*>(smem + 512);          // [S][12]
-  uint8_t* ring = smem + 1024;
-  uint8_t* xbuf = ring + (size_t)S * p.stage_slot_bytes;
-  int* tacc = reinterpret_cast<int*>(xbuf + 2 * (size_t)p.x_slot_bytes);   // [S][12][16][NC]
+  // layout: [full[S], empty[S] mbarriers; 1 KB][ring: S slots of stage_slot_bytes]
+  //   slot: [tile slot 0 box][tile slot 1 box]...[operand segment]
+  //   box:  [plane 0: kBoxRows rows x 64 B][plane 1: kBoxRows rows x 64 B]
+  const uint32_t full0 = smem_u32(smem);
+  const uint32_t empty0 = full0 + 8 * S;
+  const uint32_t ring = smem_u32(smem + 1024);
+  const uint32_t slot_bytes = (uint32_t)p.stage_slot_bytes;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int u0 = p.cta_unit[blockIdx.x], u1 = p.cta_unit[blockIdx.x + 1];
-  const int n = u1 - u0;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(full0 + 8 * i, 1);
       mbar_init(empty0 + 8 * i, kCW);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(xfull0 + 8 * b, 1);
-      mbar_init(xempty0 + 8 * b, kCW);
-    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-  for (int i = threadIdx.x; i < S * 12; i += blockDim.x) cnt[i] = 0;
-  for (int i = threadIdx.x; i < S * 12 * 16 * NC; i += blockDim.x) tacc[i] = 0;
   __syncthreads();
   pdl_launch_dependents();
-  if (n <= 0) return;
+  if (u1 <= u0) return;
 
   // item of the first unit
   int first_item = 0;
@@ -203,206 +231,220 @@ __global__ void __launch_bounds__(kBatchThreads, 1) k_batch_stream(const BatchPa
   if (warp == kCW) {
     // ====================== producer (lane 0) ======================
     if (lane != 0) return;
+    // stages of this CTA in order: (item, row block, part)
+    int n = 0;
+    {
+      int it = first_item;
+      for (int u = u0; u < u1; ++u) {
+        while (it + 1 < p.count && p.items[it + 1].unit0 <= u) ++it;
+        n += p.items[it].kp;
+      }
+    }
     bool ok = true;
-    auto issue_weights = [&](int lu, int it) -> bool {
-      const int s = lu % S;
-      if (lu >= S && !mbar_wait(empty0 + 8 * s, ((lu / S) - 1) & 1)) return false;
-      const BatchItem& b = p.items[it];
-      const int grp = (u0 + lu) - b.unit0;
-      const int r0 = grp * b.ts * 16;
-      const uint32_t row_bytes = (uint32_t)b.K / 4;
-      const uint32_t bytes = (uint32_t)min(b.ts * 16, b.N - r0) * row_bytes;
-      mbar_arrive_expect_tx(full0 + 8 * s, bytes);
-      bulk_g2s(smem_u32(ring + (size_t)s * p.stage_slot_bytes), b.planes + (size_t)r0 * (b.K / 16), bytes, full0 + 8 * s);
-      return true;
-    };
-    // weights of the first stages do not depend on earlier kernels: start them before the wait
-    int it = first_item;
+    // 1. weights of the first stages: they do not depend on earlier kernels
     const int pre = n < S ? n : S;
-    for (int lu = 0; lu < pre && ok; ++lu) {
-      while (it + 1 < p.count && p.items[it + 1].unit0 <= u0 + lu) ++it;
-      ok = issue_weights(lu, it);
+    int it = first_item, rb = u0 - p.items[first_item].unit0, part = 0;
+    for (int q = 0; q < pre; ++q) {
+      const BatchItem& B = p.items[it];
+      const uint32_t bar = full0 + 8 * q;
+      const uint32_t dst = ring + (uint32_t)q * slot_bytes;
+      int boxes = 0;
+      for (int b = 0; b < kTPW; ++b) boxes += (rb * kStageRows + b * kBoxRows < B.N) ? 1 : 0;
+      mbar_arrive_expect_tx(bar, (uint32_t)(boxes * kBoxBytes + p.seg_bytes));
+      for (int b = 0; b < boxes; ++b)
+        tma_load_3d(dst + b * kBoxBytes, &p.tmap[it], part * kPartWords, rb * kStageRows + b * kBoxRows, 0, bar);
+      if (++part == B.kp) {
+        part = 0;
+        if (++rb == B.units) { rb = 0; ++it; }
+      }
     }
     pdl_wait();
-    it = first_item;
-    int seq = -1;                                         // item sequence number in this CTA
-    for (int lu = 0; lu < n && ok; ++lu) {
-      int it_new = it;
-      while (it_new + 1 < p.count && p.items[it_new + 1].unit0 <= u0 + lu) ++it_new;
-      if (lu == 0 || it_new != it) {
-        it = it_new;
-        ++seq;
-        const int b = seq & 1;
-        if (seq >= 2 && !(ok = mbar_wait(xempty0 + 8 * b, ((seq >> 1) - 1) & 1))) break;
-        const uint32_t bytes = (uint32_t)p.items[it].xbytes;
-        mbar_arrive_expect_tx(xfull0 + 8 * b, bytes);
-        bulk_g2s(smem_u32(xbuf + (size_t)b * p.x_slot_bytes), p.xprep + p.items[it].xoff, bytes, xfull0 + 8 * b);
+    // 2. every stage: its operand segment and, past the first S, its weights once the slot is free
+    it = first_item; rb = u0 - p.items[first_item].unit0; part = 0;
+    int s = 0;
+    uint32_t ph = 0;
+    for (int q = 0; q < n && ok; ++q) {
+      const BatchItem& B = p.items[it];
+      const uint32_t bar = full0 + 8 * s;
+      const uint32_t dst = ring + (uint32_t)s * slot_bytes;
+      if (q >= S) {
+        if (!(ok = mbar_wait(empty0 + 8 * s, ph ^ 1u))) break;
+        int boxes = 0;
+        for (int b = 0; b < kTPW; ++b) boxes += (rb * kStageRows + b * kBoxRows < B.N) ? 1 : 0;
+        mbar_arrive_expect_tx(bar, (uint32_t)(boxes * kBoxBytes + p.seg_bytes));
+        for (int b = 0; b < boxes; ++b)
+          tma_load_3d(dst + b * kBoxBytes, &p.tmap[it], part * kPartWords, rb * kStageRows + b * kBoxRows, 0, bar);
       }
-      if (lu >= pre) ok = issue_weights(lu, it);
+      bulk_g2s(dst + kWStageBytes, p.xprep + B.xoff + (size_t)part * p.seg_bytes, (uint32_t)p.seg_bytes, bar);
+      if (++part == B.kp) {
+        part = 0;
+        if (++rb == B.units) { rb = 0; ++it; }
+      }
+      if (++s == S) { s = 0; ph ^= 1u; }
     }
     if (!ok) atomicExch(&g_batch_latch, 5);
-    // do not exit with copies in flight
-    for (int lu = n > S ? n - S : 0; lu < n; ++lu)
-      if (!mbar_wait(full0 + 8 * (lu % S), (lu / S) & 1)) break;
+    // do not exit with copies in flight: wait for the last min(n, S) stages to land
+    if (ok) {
+      for (int q = n > S ? n - S : 0; q < n; ++q) {
+        if (!mbar_wait(full0 + 8 * (q % S), (uint32_t)((q / S) & 1))) {
+          atomicExch(&g_batch_latch, 5);
+          break;
+        }
+      }
+    }
     return;
   }
 
   // ====================== consumers ======================
   const int g = lane >> 2, t = lane & 3;
-  const int j = warp;
+  const int col = g < NC ? g : 0;                           // operand column this lane feeds
+  // byte offsets inside a slot
+  const uint32_t wofs = (uint32_t)((warp * 16 + g) * kPartWords * 4 + t * 16);   // plane 0, row g
+  const uint32_t xofs = (uint32_t)(kWStageBytes + (col * kColWords + t * 8) * 4);
+  const uint32_t mofs = (uint32_t)(kWStageBytes + NC * kColWords * 4);
   bool ok = true;
-  int it = first_item, seq = 0, released = 0, acquired = -1;
-  // Release of an item's operand buffer: every warp arrives once per item, in item order (all warps
-  // see every unit), so item q's arrivals never mix with item q - 2's on the same barrier.
-  for (int lu = 0; lu < n && ok; ++lu) {
-    // item of this unit and its sequence number
-    while (it + 1 < p.count && p.items[it + 1].unit0 <= u0 + lu) {
-      ++it;
-      ++seq;
-    }
-    for (; released < seq; ++released) {                 // items this warp has passed
-      __syncwarp();
-      if (lane == 0) mbar_arrive(xempty0 + 8 * (released & 1));
-    }
-    if (acquired != seq) {
-      if (!(ok = mbar_wait(xfull0 + 8 * (seq & 1), (seq >> 1) & 1))) break;
-      acquired = seq;
-    }
-    const int s = lu % S;
-    if (!(ok = mbar_wait(full0 + 8 * s, (lu / S) & 1))) break;
+  int it = first_item, rb = u0 - p.items[first_item].unit0;
+  int s = 0;
+  uint32_t ph = 0;
+  for (int u = u0; u < u1 && ok; ++u) {
     const BatchItem& B = p.items[it];
-    const int KM = B.K >> 5, KP = B.kp, TS = B.ts;
-    const int grp_idx = (u0 + lu) - B.unit0;
-    const int xcw = KP * 128 + 4;
-    const uint32_t* xb_base = reinterpret_cast<const uint32_t*>(xbuf + (size_t)(seq & 1) * p.x_slot_bytes);
-    const int* meta = reinterpret_cast<const int*>(xb_base + NC * xcw);
-    const uint32_t* st = reinterpret_cast<const uint32_t*>(ring + (size_t)s * p.stage_slot_bytes);
-    const int row_w = 2 * KM;
-    const int pairs = TS * KP;
-    int* acc_s = tacc + s * 12 * 16 * NC;
-    int* cnt_s = cnt + s * 12;
-    for (int pr = j; pr < pairs; pr += kCW) {
-      const int tile = pr / KP, part = pr - tile * KP;
-      const int wbase = part * 16 + 4 * t;                // first word of this lane in the part
-      const bool live = wbase < KM;
-      const uint32_t* ra = st + (tile * 16 + g) * row_w + wbase;
-      const uint32_t* rb = ra + 8 * row_w;
-      const uint32_t* xl = xb_base + (g < NC ? g : 0) * xcw + part * 128 + t * 8;
-      int acc[4][4];
+    const int KP = B.kp;
+    const int row_base = rb * kStageRows + warp * 16;          // first row of this warp's tile slot 0
+    int acc[kTPW][4][4];
 #pragma unroll
-      for (int a = 0; a < 4; ++a) acc[a][0] = acc[a][1] = acc[a][2] = acc[a][3] = 0;
-      uint4 ma = make_uint4(0u, 0u, 0u, 0u), mb = ma, sa = ma, sb = ma;
-      if (live) {
-        ma = *reinterpret_cast<const uint4*>(ra);
-        mb = *reinterpret_cast<const uint4*>(rb);
-        sa = *reinterpret_cast<const uint4*>(ra + KM);
-        sb = *reinterpret_cast<const uint4*>(rb + KM);
+    for (int a = 0; a < kTPW; ++a)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[a][i][0] = acc[a][i][1] = acc[a][i][2] = acc[a][i][3] = 0;
+    int tot[3] = {0, 0, 0};
+    int E = 0;
+    for (int part = 0; part < KP; ++part) {
+      if (!(ok = mbar_wait(full0 + 8 * s, ph))) break;
+      const uint32_t st = ring + (uint32_t)s * slot_bytes;
+      uint4 ma[kTPW], mb[kTPW], sa[kTPW], sb[kTPW];
+#pragma unroll
+      for (int a = 0; a < kTPW; ++a) {
+        const uint32_t r = st + a * kBoxBytes + wofs;
+        ma[a] = lds128(r);
+        mb[a] = lds128(r + 8 * kPartWords * 4);
+        sa[a] = lds128(r + kBoxRows * kPartWords * 4);
+        sb[a] = lds128(r + (kBoxRows + 8) * kPartWords * 4);
       }
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const uint4 x0 = *reinterpret_cast<const uint4*>(xl + e * 32);
-        const uint4 x1 = *reinterpret_cast<const uint4*>(xl + e * 32 + 4);
-        uint32_t wa0, wb0, wa1, wb1;
-        merge_planes_offset(u4get(ma, e), u4get(sa, e), wa0, wb0);
-        merge_planes_offset(u4get(mb, e), u4get(sb, e), wa1, wb1);
-        if (!live) wa0 = wb0 = wa1 = wb1 = 0u;
-        mma_u8s8(acc[0], wa0 & 0x03030303u, wa1 & 0x03030303u, wb0 & 0x03030303u, wb1 & 0x03030303u, x0.x, x1.x);
-        mma_u8s8(acc[1], wa0 & 0x0C0C0C0Cu, wa1 & 0x0C0C0C0Cu, wb0 & 0x0C0C0C0Cu, wb1 & 0x0C0C0C0Cu, x0.y, x1.y);
-        mma_u8s8(acc[2], wa0 & 0x30303030u, wa1 & 0x30303030u, wb0 & 0x30303030u, wb1 & 0x30303030u, x0.z, x1.z);
-        mma_u8s8(acc[3], wa0 & 0xC0C0C0C0u, wa1 & 0xC0C0C0C0u, wb0 & 0xC0C0C0C0u, wb1 & 0xC0C0C0C0u, x0.w, x1.w);
-      }
-      // this part's exact sums for the lane's rows and columns (offset 2 * sum x removed)
-      if (t < (NC + 1) / 2) {
+        const uint4 x0 = lds128(st + xofs + e * 128);
+        const uint4 x1 = lds128(st + xofs + e * 128 + 16);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int col = 2 * t + (q & 1);
-          if (col < NC) {
-            const int v = acc[0][q] + (acc[1][q] >> 2) + (acc[2][q] >> 4) + (acc[3][q] >> 6) - 2 * meta[part * NC + col];
-            atomicAdd(&acc_s[(tile * 16 + g + 8 * (q >> 1)) * NC + col], v);
-          }
+        for (int a = 0; a < kTPW; ++a) {
+          uint32_t wa0, wb0, wa1, wb1;
+          merge_planes_offset(u4get(ma[a], e), u4get(sa[a], e), wa0, wb0);
+          merge_planes_offset(u4get(mb[a], e), u4get(sb[a], e), wa1, wb1);
+          mma_u8s8(acc[a][0], wa0 & 0x03030303u, wa1 & 0x03030303u, wb0 & 0x03030303u, wb1 & 0x03030303u, x0.x, x1.x);
+          mma_u8s8(acc[a][1], wa0 & 0x0C0C0C0Cu, wa1 & 0x0C0C0C0Cu, wb0 & 0x0C0C0C0Cu, wb1 & 0x0C0C0C0Cu, x0.y, x1.y);
+          mma_u8s8(acc[a][2], wa0 & 0x30303030u, wa1 & 0x30303030u, wb0 & 0x30303030u, wb1 & 0x30303030u, x0.z, x1.z);
+          mma_u8s8(acc[a][3], wa0 & 0xC0C0C0C0u, wa1 & 0xC0C0C0C0u, wb0 & 0xC0C0C0C0u, wb1 & 0xC0C0C0C0u, x0.w, x1.w);
         }
       }
-      __syncwarp();
-      int done = 0;
-      if (lane == 0) {
-        __threadfence_block();
-        done = atomicAdd(&cnt_s[tile], 1) == KP - 1;
+      if (part == KP - 1) {                                  // sums over all of K and E ride in every segment
+        const uint4 m4 = lds128(st + mofs);
+        tot[0] = (int)m4.x;
+        tot[1] = (int)m4.y;
+        tot[2] = (int)m4.z;
+        E = (int)m4.w;
       }
-      done = __shfl_sync(0xFFFFFFFFu, done, 0);
-      if (done) {                                          // all K parts of the tile are in
-        __threadfence_block();
-        const int row = (grp_idx * TS + tile) * 16 + lane;
-        if (lane < 16) {
-          int* ta = acc_s + (tile * 16 + lane) * NC;
-          if (row < B.N) {
-            const float sc = f16_bits_to_float(B.scale[row]);
-            float y;
-            if (MODE == 1) {
-              y = __fmul_rn(__fmul_rn(__int2float_rn(ta[0]), B.sx[0]), sc);
-            } else {
-              const long long D = (long long)ta[0] * 65536 + (long long)ta[1] * 256 + (long long)ta[2];
-              y = (float)(ldexp((double)D, meta[KP * NC] - kLimbFrac) * (double)sc);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty0 + 8 * s);
+      if (++s == S) { s = 0; ph ^= 1u; }
+    }
+    if (!ok) break;
+    // ---- outputs of this warp's tiles: exact integer sums, one rounding ----------------------------
+    float sxv = 0.0f;
+    if (MODE == 1) sxv = B.sx[0];
+#pragma unroll
+    for (int a = 0; a < kTPW; ++a) {
+      int v[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        v[q] = acc[a][0][q] + (acc[a][1][q] >> 2) + (acc[a][2][q] >> 4) + (acc[a][3][q] >> 6);
+      const int r0 = row_base + a * kBoxRows + g;            // rows r0 (q = 0, 1) and r0 + 8 (q = 2, 3)
+      if (MODE == 1) {
+        if (t == 0) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int row = r0 + 8 * h;
+            if (row < B.N) {
+              const int S1 = v[2 * h] - 2 * tot[0];
+              B.y[row] = __fmul_rn(__fmul_rn(__int2float_rn(S1), sxv), f16_bits_to_float(B.scale[row]));
             }
-            B.y[row] = y;
           }
-#pragma unroll
-          for (int c = 0; c < NC; ++c) ta[c] = 0;
         }
-        __syncwarp();
-        if (lane == 0) cnt_s[tile] = 0;
+      } else {
+        // lane t = 0 holds columns 0 (L2) and 1 (L1), lane t = 1 column 2 (L0)
+        const int l0a = __shfl_down_sync(0xFFFFFFFFu, v[0], 1);
+        const int l0b = __shfl_down_sync(0xFFFFFFFFu, v[2], 1);
+        if (t == 0) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int row = r0 + 8 * h;
+            if (row < B.N) {
+              const long long S2 = v[2 * h] - 2LL * tot[0];
+              const long long S1 = v[2 * h + 1] - 2LL * tot[1];
+              const long long S0 = (h ? l0b : l0a) - 2LL * tot[2];
+              const long long D = S2 * 65536 + S1 * 256 + S0;
+              B.y[row] = (float)((double)D * exp2_i(E - kLimbFrac) * (double)f16_bits_to_float(B.scale[row]));
+            }
+          }
+        }
       }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(empty0 + 8 * s);
+    if (++rb == B.units) { rb = 0; ++it; }
   }
-  // release the last item of this CTA (every earlier one was released on leaving it)
-  if (ok) {
-    for (; released <= seq; ++released) {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(xempty0 + 8 * (released & 1));
-    }
-  } else if (lane == 0) {
-    atomicExch(&g_batch_latch, 5);
+  if (!ok && lane == 0) atomicExch(&g_batch_latch, 5);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
   }
+  return fn;
 }
 
 }  // namespace
 
-bool plan_batch(BatchParams& p, size_t& smem, size_t& workspace) {
+bool plan_batch(BatchParams& p, const uint32_t* const* planes, size_t& smem, size_t& workspace) {
   const int nc = p.mode == 0 ? 3 : 1;
   p.nc = nc;
-  // stage: TS whole tiles, at most 48 KB and 12 tiles; K parts of 512 trits (the last one partial)
-  const int kSlot = 48 * 1024;
+  p.seg_bytes = ((nc * kColWords + 4) * 4 + 15) & ~15;
+  PFN_cuTensorMapEncodeTiled_v12000 encode = encode_fn();
+  if (!encode) return false;
   long long total_bytes = 0;
-  int units = 0, max_x = 0, max_slot = 0;
+  int units = 0;
   size_t xoff = 0;
   for (int i = 0; i < p.count; ++i) {
     BatchItem& it = p.items[i];
     if (it.K % 128 || it.K <= 0 || it.N <= 0) return false;
-    const int tile_bytes = 16 * it.K / 4;
-    int ts = kSlot / tile_bytes;
-    if (ts > 12) ts = 12;
-    if (ts < 1) return false;                              // a tile larger than a stage slot
-    it.ts = ts;
     it.kp = (it.K + 511) / 512;
-    if (it.kp > 24) return false;
     it.unit0 = units;
-    const int tiles = (it.N + 15) / 16;
-    it.units = (tiles + ts - 1) / ts;
+    it.units = (it.N + kStageRows - 1) / kStageRows;
     units += it.units;
-    const int xcw = it.kp * 128 + 4;
-    int xb = nc * xcw * 4 + (it.kp * nc + 1) * 4;
-    xb = (xb + 15) & ~15;
-    it.xbytes = xb;
     it.xoff = (uint32_t)xoff;
-    xoff += (size_t)xb;
-    if (xb > max_x) max_x = xb;
-    if (ts * tile_bytes > max_slot) max_slot = ts * tile_bytes;
+    xoff += (size_t)it.kp * p.seg_bytes;
     total_bytes += (long long)it.N * it.K / 4;
+    // planes of row n: mask words [n * K/16, n * K/16 + K/32), its sign words right after
+    const cuuint64_t dims[3] = {(cuuint64_t)(it.K / 32), (cuuint64_t)it.N, 2};
+    const cuuint64_t strides[2] = {(cuuint64_t)it.K / 4, (cuuint64_t)it.K / 8};   // bytes: row, plane
+    const cuuint32_t box[3] = {(cuuint32_t)kPartWords, (cuuint32_t)kBoxRows, 2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (encode(&p.tmap[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t*>(planes[i]), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
   }
   p.total_units = units;
-  p.stage_slot_bytes = max_slot;
-  p.x_slot_bytes = max_x;
   workspace = xoff;
   // balanced by weight bytes: CTA c starts at the first unit whose start byte reaches c/G of the total
   const int grid = units < 148 ? units : 148;
@@ -412,23 +454,21 @@ bool plan_batch(BatchParams& p, size_t& smem, size_t& workspace) {
   p.cta_unit[0] = 0;
   for (int i = 0; i < p.count; ++i) {
     const BatchItem& it = p.items[i];
-    const long long unit_bytes = (long long)it.ts * 16 * it.K / 4;
     for (int u = 0; u < it.units; ++u) {
       while (c + 1 < grid && acc >= total_bytes * (c + 1) / grid) p.cta_unit[++c] = it.unit0 + u;
-      acc += unit_bytes;
+      const int rows = it.N - u * kStageRows < kStageRows ? it.N - u * kStageRows : kStageRows;
+      acc += (long long)rows * it.K / 4;
     }
   }
   while (c + 1 <= grid) p.cta_unit[++c] = units;
   p.cta_unit[grid] = units;
-  const size_t fixed = 1024 + 2 * (size_t)max_x;
-  int stages = 0;
-  for (int s = 6; s >= 2; --s) {
-    const size_t need = fixed + (size_t)s * max_slot + (size_t)s * 12 * 16 * nc * 4;
-    if (need <= 226 * 1024) { stages = s; break; }
-  }
-  if (!stages) return false;
+  p.stage_slot_bytes = (kWStageBytes + p.seg_bytes + 1023) & ~1023;
+  const size_t budget = 227 * 1024;
+  int stages = (int)((budget - 1024) / (size_t)p.stage_slot_bytes);
+  if (stages > 8) stages = 8;
+  if (stages < 2) return false;
   p.stages = stages;
-  smem = fixed + (size_t)stages * max_slot + (size_t)stages * 12 * 16 * nc * 4;
+  smem = 1024 + (size_t)stages * p.stage_slot_bytes;
   return true;
 }
 
@@ -451,7 +491,7 @@ cudaError_t launch_batch(const BatchParams& p, size_t smem, bool pdl, cudaStream
   cfg.attrs = attr;
   cfg.numAttrs = na;
   cfg.stream = st;
-  // 1. operand blocks
+  // 1. operand segments
   cfg.gridDim = dim3(p.count, 1, 1);
   cfg.blockDim = dim3(256, 1, 1);
   cfg.dynamicSmemBytes = 0;

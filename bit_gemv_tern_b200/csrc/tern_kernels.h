@@ -3,6 +3,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace tern {
@@ -49,21 +50,19 @@ cudaError_t read_and_clear_error_latch(int* out, cudaStream_t st);
 
 // Batched M = 1 GEMV over a list of matrices (tern_batch.cu).
 struct BatchItem {
-  const uint32_t* planes;
   const uint16_t* scale;
   float* y;
   const void* x;          // bf16 bits [K] or int8 [K]
   const float* sx;        // int8 mode: [1]
   int32_t N, K;
-  int32_t ts;             // tiles of 16 rows per stage
-  int32_t kp;             // 512-trit K parts (last may be partial)
-  int32_t unit0;          // first global unit (stage) of the item
-  int32_t units;          // stages of the item
+  int32_t kp;             // 512-trit K parts (the last may be partial): stages per row block
+  int32_t unit0;          // first global unit (row block) of the item
+  int32_t units;          // row blocks of the item
   uint32_t xoff;          // byte offset of the item's operand block in the workspace
-  int32_t xbytes;         // bytes of that block
 };
 constexpr int kBatchMaxItems = 160;
 struct BatchParams {
+  CUtensorMap tmap[kBatchMaxItems];  // per item: planes viewed as [2 planes][N rows][K/32 words]
   BatchItem items[kBatchMaxItems];
   int32_t count;
   int32_t mode;           // 0 = bf16 activations (three int8 limbs), 1 = int8
@@ -72,11 +71,13 @@ struct BatchParams {
   int32_t grid;
   int32_t stages;
   int32_t stage_slot_bytes;
-  int32_t x_slot_bytes;
+  int32_t seg_bytes;      // operand bytes of one 512-trit part (all columns + sums + exponent)
   uint8_t* xprep;         // workspace: operand blocks
   int32_t cta_unit[149];  // CTA c handles units [cta_unit[c], cta_unit[c + 1])
 };
-bool plan_batch(BatchParams& p, size_t& smem, size_t& workspace);
+static_assert(sizeof(BatchParams) <= 32764, "kernel parameter limit");
+// Host: fills tmap/kp/units/xoff, the stage ring and the CTA split; fails on unsupported shapes.
+bool plan_batch(BatchParams& p, const uint32_t* const* planes, size_t& smem, size_t& workspace);
 cudaError_t launch_batch(const BatchParams& p, size_t smem, bool pdl, cudaStream_t st);
 cudaError_t read_and_clear_batch_latch(int* out);
 
