@@ -20,7 +20,8 @@ __all__ = [
     "TERN_ACT_BF16", "TERN_ACT_INT8", "TERN_SRC_INT8_TRITS", "TERN_SRC_BASE3", "TERN_FLAG_PDL",
     "tern_packed_bytes", "tern_base3_bytes", "tern_pack", "tern_base3_encode", "tern_occupancy",
     "tern_quantize_act", "tern_gemv", "tern_gemm_small_m", "tern_gemm_prefill",
-    "i8_head_workspace_bytes", "i8_head_gemv_argmax", "tern_read_flag", "tern_device_status",
+    "i8_head_workspace_bytes", "i8_head_gemv_argmax", "i8_head_gemv_argmax_noalloc",
+    "TERN_HEAD_NOALLOC_MAX_M", "tern_read_flag", "tern_device_status",
     "GemvBatch", "tern_gemv_batch", "tern_gemv_batch_workspace_bytes",
     "tern_status_string",
 ]
@@ -29,6 +30,7 @@ TERN_OK, TERN_EINVAL, TERN_ESHAPE, TERN_EBADCODE, TERN_ECUDA, TERN_ETIMEOUT = ra
 TERN_ACT_BF16, TERN_ACT_INT8 = 0, 1
 TERN_SRC_INT8_TRITS, TERN_SRC_BASE3 = 0, 1
 TERN_FLAG_PDL = 1
+TERN_HEAD_NOALLOC_MAX_M = 16
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libterngemv.so")
@@ -71,6 +73,7 @@ def lib() -> ctypes.CDLL:
             "i8_head_workspace_bytes": ([i32, i32], sz),
             "i8_head_gemv_argmax": ([vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp], i32),
             "i8_head_gemv_argmax_ex": ([vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, sz, u32, vp], i32),
+            "i8_head_gemv_argmax_noalloc": ([vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp], i32),
             "tern_read_flag": ([vp, vp], i32),
             "tern_device_status": ([vp], i32),
             "tern_gemv_batch_workspace_bytes": ([vp, i32, i32], sz),
@@ -177,6 +180,15 @@ def i8_head_gemv_argmax(W, scale_f16, V: int, K: int, M: int, act: int, X, x_sca
                                         _ptr(argmax), _ptr(maxval), _ptr(logits), _ptr(workspace),
                                         int(workspace.numel() * workspace.element_size()), flags,
                                         _stream(stream)), "i8_head_gemv_argmax")
+
+
+def i8_head_gemv_argmax_noalloc(W, scale_f16, V: int, K: int, M: int, act: int, X, x_scale, argmax, maxval,
+                                logits, stream=None) -> None:
+    """i8_head_gemv_argmax with the library's internal per-device scratch instead of a caller
+    workspace (M <= TERN_HEAD_NOALLOC_MAX_M; calls that overlap in time race)."""
+    _check(lib().i8_head_gemv_argmax_noalloc(_ptr(W), _ptr(scale_f16), V, K, M, act, _ptr(X), _ptr(x_scale),
+                                             _ptr(argmax), _ptr(maxval), _ptr(logits), _stream(stream)),
+           "i8_head_gemv_argmax_noalloc")
 
 
 def tern_read_flag(err_flag, stream=None) -> int:

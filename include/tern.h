@@ -215,6 +215,25 @@ tern_status i8_head_gemv_argmax_ex(const int8_t* W_dev, const uint16_t* scale_f1
                                    float* logits_dev, void* workspace_dev, size_t workspace_bytes,
                                    uint32_t flags, tern_stream_t stream);
 
+/* No-allocation variant of i8_head_gemv_argmax. The source pages describe no counterpart: it is
+ * an interface convenience of this library. Same arguments, results and error codes as
+ * i8_head_gemv_argmax, minus the workspace: the scratch is one library-internal device array of
+ * TERN_HEAD_NOALLOC_SCRATCH_BYTES bytes per device, enough for M <= TERN_HEAD_NOALLOC_MAX_M.
+ *   - M outside 1..TERN_HEAD_NOALLOC_MAX_M (scratch need above the array's size): TERN_ESHAPE,
+ *     nothing launched.
+ *   - The first call on a device looks up the array's address (cudaGetSymbolAddress, with that
+ *     device current) and keeps it; that first call must come before any stream capture.
+ *   - Each call clears the scratch bytes it uses (cudaMemsetAsync on `stream`) before the launch;
+ *     no call allocates or frees device memory.
+ *   - All calls on one device share the array: calls that overlap in time (different streams,
+ *     host threads) race and may return wrong results. Order them on one stream. */
+#define TERN_HEAD_NOALLOC_MAX_M 16
+#define TERN_HEAD_NOALLOC_SCRATCH_BYTES 256
+tern_status i8_head_gemv_argmax_noalloc(const int8_t* W_dev, const uint16_t* scale_f16_dev, int32_t V,
+                                        int32_t K, int32_t M, tern_act act, const void* X_dev,
+                                        const float* x_scale_dev, int32_t* argmax_dev, float* maxval_dev,
+                                        float* logits_dev, tern_stream_t stream);
+
 /* Synchronise `stream`, read *err_flag_dev and map it: 0 -> TERN_OK, nonzero -> TERN_EBADCODE. */
 tern_status tern_read_flag(const int32_t* err_flag_dev, tern_stream_t stream);
 
