@@ -373,6 +373,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-rows", action="store_true", help="skip the extra scope rows")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    ap.add_argument("--profile", default=None, choices=sorted(PROFILE_CASES),
+                    help="run one small case 4 times (3 warm-up launches + 1) for an ncu capture, then exit")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -405,6 +407,8 @@ def main():
     from bit_gemv_tern_b200 import build as _b
     _b.build()
     hbm_peak, bf16_peak, bf16_sust, peak_kind = peaks()
+    if args.profile:
+        return run_profile_case(args.profile)
 
     stack = Stack("8b", M=1)
     n_linear = len(stack.linears)
@@ -502,6 +506,42 @@ def main():
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def _profile_batch(mode):
+    def run():
+        st = Stack("8b", M=1, layers=4)
+        return lambda: st.launch_stack(mode)
+    return run
+
+
+def _profile_head(mode):
+    def run():
+        st = Stack("8b", M=1, layers=0)
+        return lambda: st.launch_head(mode)
+    return run
+
+
+# Small cases for ncu captures (inputs > L2, a few hundred MB on the device):
+#   batch-8b-4layers-*: 4 layers of the 8B stack (16 fused GEMVs, 193 MB of planes) as one batch
+#   head-8b-*:          the int8 head 151936 x 4096 (622 MB)
+PROFILE_CASES = {
+    "batch-8b-4layers-bf16": _profile_batch("bf16"),
+    "batch-8b-4layers-int8": _profile_batch("int8"),
+    "head-8b-bf16": _profile_head("bf16"),
+}
+
+
+def run_profile_case(name):
+    import torch
+    import bit_gemv_tern_b200 as tg
+    fn = PROFILE_CASES[name]()
+    for _ in range(4):
+        fn()
+    torch.cuda.synchronize()
+    st = tg.tern_device_status()
+    print(f"profile case {name}: status {st}", flush=True)
+    return 0 if st == tg.TERN_OK else 1
 
 
 def extra_rows(stack, torch, tg, hbm_peak, bf16_peak):

@@ -39,8 +39,15 @@ __device__ int g_batch_latch = 0;
 
 namespace {
 
-constexpr int kCW = 12;                               // consumer warps
-constexpr int kTPW = 2;                               // tiles of 16 rows per consumer warp
+#ifndef TERN_BATCH_CW
+#define TERN_BATCH_CW 12
+#endif
+#ifndef TERN_BATCH_TPW
+#define TERN_BATCH_TPW 2
+#endif
+constexpr int kCW = TERN_BATCH_CW;                    // consumer warps (kBoxRows <= 256: at most 16)
+constexpr int kTPW = TERN_BATCH_TPW;                  // tiles of 16 rows per consumer warp
+static_assert(kCW >= 1 && kCW <= 16 && kTPW >= 1 && kTPW <= 4, "batch kernel shape");
 constexpr int kBatchThreads = (kCW + 1) * 32;
 constexpr int kBoxRows = kCW * 16;                    // rows of one TMA box: tile slot a of every warp
 constexpr int kStageRows = kBoxRows * kTPW;           // rows of a row block
@@ -317,8 +324,22 @@ __global__ void __launch_bounds__(kBatchThreads, 1) k_batch_stream(const __grid_
       for (int i = 0; i < 4; ++i) acc[a][i][0] = acc[a][i][1] = acc[a][i][2] = acc[a][i][3] = 0;
     int tot[3] = {0, 0, 0};
     int E = 0;
+    // the epilogue's reads of the row scales (weights: written before any launch of this list),
+    // issued now so that they land while the block streams
+    float sxv = 0.0f;
+    uint16_t sc_bits[kTPW][2];
+#pragma unroll
+    for (int a = 0; a < kTPW; ++a)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int row = row_base + a * kBoxRows + g + 8 * h;
+        sc_bits[a][h] = (t == 0 && row < B.N) ? B.scale[row] : (uint16_t)0;
+      }
     for (int part = 0; part < KP; ++part) {
       if (!(ok = mbar_wait(full0 + 8 * s, ph))) break;
+      // s_x comes from an earlier kernel: read only after a stage has landed (the producer issues
+      // every copy after its grid-dependency wait)
+      if (MODE == 1 && part == 0) sxv = B.sx[0];
       const uint32_t st = ring + (uint32_t)s * slot_bytes;
       uint4 ma[kTPW], mb[kTPW], sa[kTPW], sb[kTPW];
 #pragma unroll
@@ -357,8 +378,6 @@ __global__ void __launch_bounds__(kBatchThreads, 1) k_batch_stream(const __grid_
     }
     if (!ok) break;
     // ---- outputs of this warp's tiles: exact integer sums, one rounding ----------------------------
-    float sxv = 0.0f;
-    if (MODE == 1) sxv = B.sx[0];
 #pragma unroll
     for (int a = 0; a < kTPW; ++a) {
       int v[4];
@@ -373,7 +392,7 @@ __global__ void __launch_bounds__(kBatchThreads, 1) k_batch_stream(const __grid_
             const int row = r0 + 8 * h;
             if (row < B.N) {
               const int S1 = v[2 * h] - 2 * tot[0];
-              B.y[row] = __fmul_rn(__fmul_rn(__int2float_rn(S1), sxv), f16_bits_to_float(B.scale[row]));
+              B.y[row] = __fmul_rn(__fmul_rn(__int2float_rn(S1), sxv), f16_bits_to_float(sc_bits[a][h]));
             }
           }
         }
@@ -390,7 +409,7 @@ __global__ void __launch_bounds__(kBatchThreads, 1) k_batch_stream(const __grid_
               const long long S1 = v[2 * h + 1] - 2LL * tot[1];
               const long long S0 = (h ? l0b : l0a) - 2LL * tot[2];
               const long long D = S2 * 65536 + S1 * 256 + S0;
-              B.y[row] = (float)((double)D * exp2_i(E - kLimbFrac) * (double)f16_bits_to_float(B.scale[row]));
+              B.y[row] = (float)((double)D * exp2_i(E - kLimbFrac) * (double)f16_bits_to_float(sc_bits[a][h]));
             }
           }
         }
@@ -440,7 +459,7 @@ bool plan_batch(BatchParams& p, const uint32_t* const* planes, size_t& smem, siz
     const cuuint32_t box[3] = {(cuuint32_t)kPartWords, (cuuint32_t)kBoxRows, 2};
     const cuuint32_t estr[3] = {1, 1, 1};
     if (encode(&p.tmap[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t*>(planes[i]), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return false;
   }
