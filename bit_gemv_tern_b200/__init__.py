@@ -22,7 +22,8 @@ __all__ = [
     "tern_quantize_act", "tern_gemv", "tern_gemm_small_m", "tern_gemm_prefill",
     "i8_head_workspace_bytes", "i8_head_gemv_argmax", "i8_head_gemv_argmax_noalloc",
     "TERN_HEAD_NOALLOC_MAX_M", "tern_read_flag", "tern_device_status",
-    "GemvBatch", "tern_gemv_batch", "tern_gemv_batch_workspace_bytes",
+    "GemvBatch", "tern_gemv_batch", "tern_gemv_batch_workspace_bytes", "tern_gemm_batch",
+    "tern_gemm_batch_workspace_bytes",
     "tern_status_string",
 ]
 
@@ -78,6 +79,8 @@ def lib() -> ctypes.CDLL:
             "tern_device_status": ([vp], i32),
             "tern_gemv_batch_workspace_bytes": ([vp, i32, i32], sz),
             "tern_gemv_batch": ([vp, i32, i32, vp, sz, u32, vp], i32),
+            "tern_gemm_batch_workspace_bytes": ([vp, i32, i32, i32], sz),
+            "tern_gemm_batch": ([vp, i32, i32, i32, vp, sz, u32, vp], i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -227,19 +230,33 @@ def tern_gemv_batch(entries, act: int, workspace, flags: int = 0, stream=None) -
            "tern_gemv_batch")
 
 
-class GemvBatch:
-    """A fixed list of M = 1 GEMVs with its descriptor array and workspace, launched repeatedly
-    (e.g. inside a captured CUDA graph). entries: list of (TernMatrix, x, x_scale or None, y)."""
+def tern_gemm_batch_workspace_bytes(entries, M: int, act: int) -> int:
+    """entries: list of (TernMatrix, X [M][K], x_scale [M] or None, Y [M][N])."""
+    arr = _items(entries)
+    return int(lib().tern_gemm_batch_workspace_bytes(arr, len(entries), M, act))
 
-    def __init__(self, entries, act: int, device="cuda"):
+
+def tern_gemm_batch(entries, M: int, act: int, workspace, flags: int = 0, stream=None) -> None:
+    arr = _items(entries)
+    _check(lib().tern_gemm_batch(arr, len(entries), M, act, _ptr(workspace),
+                                 int(workspace.numel() * workspace.element_size()), flags, _stream(stream)),
+           "tern_gemm_batch")
+
+
+class GemvBatch:
+    """A fixed list of GEMVs (M = 1) or small-M GEMMs with its descriptor array and workspace,
+    launched repeatedly (e.g. inside a captured CUDA graph). entries: list of (TernMatrix, X,
+    x_scale or None, Y) with X [M][K] and Y [M][N]."""
+
+    def __init__(self, entries, act: int, M: int = 1, device="cuda"):
         import torch
-        self.entries, self.act = list(entries), act
+        self.entries, self.act, self.M = list(entries), act, int(M)
         self._arr = _items(self.entries)
-        nbytes = int(lib().tern_gemv_batch_workspace_bytes(self._arr, len(self.entries), act))
+        nbytes = int(lib().tern_gemm_batch_workspace_bytes(self._arr, len(self.entries), self.M, act))
         if nbytes == 0:
-            raise TernError(TERN_ESHAPE, "tern_gemv_batch_workspace_bytes")
+            raise TernError(TERN_ESHAPE, "tern_gemm_batch_workspace_bytes")
         self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
 
     def __call__(self, flags: int = 0, stream=None) -> None:
-        _check(lib().tern_gemv_batch(self._arr, len(self.entries), self.act, _ptr(self.workspace),
-                                     int(self.workspace.numel()), flags, _stream(stream)), "tern_gemv_batch")
+        _check(lib().tern_gemm_batch(self._arr, len(self.entries), self.M, self.act, _ptr(self.workspace),
+                                     int(self.workspace.numel()), flags, _stream(stream)), "tern_gemm_batch")

@@ -161,12 +161,13 @@ tern_status tern_gemv(const tern_matrix* W, tern_act act, const void* x_dev, con
 
 namespace {
 
-tern_status fill_batch(const tern_gemv_item* items, int32_t count, tern_act act, tern::BatchParams& bp,
-                       size_t& smem, size_t& ws) {
+tern_status fill_batch(const tern_gemv_item* items, int32_t count, int32_t M, tern_act act,
+                       tern::BatchParams& bp, size_t& smem, size_t& ws) {
   if (!items) return TERN_EINVAL;
   if (act != TERN_ACT_BF16 && act != TERN_ACT_INT8) return TERN_EINVAL;
-  if (count < 1 || count > TERN_BATCH_MAX_ITEMS) return TERN_ESHAPE;
+  if (count < 1 || count > TERN_BATCH_MAX_ITEMS || M < 1 || M > 16) return TERN_ESHAPE;
   bp.count = count;
+  bp.M = M;
   bp.mode = act == TERN_ACT_BF16 ? 0 : 1;
   const uint32_t* planes[TERN_BATCH_MAX_ITEMS];
   for (int i = 0; i < count; ++i) {
@@ -191,21 +192,27 @@ tern_status fill_batch(const tern_gemv_item* items, int32_t count, tern_act act,
 
 }  // namespace
 
-size_t tern_gemv_batch_workspace_bytes(const tern_gemv_item* items, int32_t count, tern_act act) {
-  static tern::BatchParams bp;   // large; host-side planning only
+size_t tern_gemm_batch_workspace_bytes(const tern_gemv_item* items, int32_t count, int32_t M, tern_act act) {
+  tern::BatchParams* bp = new (std::nothrow) tern::BatchParams();
+  if (!bp) return 0;
   size_t smem = 0, ws = 0;
-  if (fill_batch(items, count, act, bp, smem, ws) != TERN_OK) return 0;
-  return ws;
+  const tern_status st = fill_batch(items, count, M, act, *bp, smem, ws);
+  delete bp;
+  return st == TERN_OK ? ws : 0;
 }
 
-tern_status tern_gemv_batch(const tern_gemv_item* items, int32_t count, tern_act act, void* workspace_dev,
-                            size_t workspace_bytes, uint32_t flags, tern_stream_t stream) {
+size_t tern_gemv_batch_workspace_bytes(const tern_gemv_item* items, int32_t count, tern_act act) {
+  return tern_gemm_batch_workspace_bytes(items, count, 1, act);
+}
+
+tern_status tern_gemm_batch(const tern_gemv_item* items, int32_t count, int32_t M, tern_act act,
+                            void* workspace_dev, size_t workspace_bytes, uint32_t flags, tern_stream_t stream) {
   if (flags & ~TERN_FLAG_PDL) return TERN_EINVAL;
   if (!workspace_dev || !aligned(workspace_dev, 16)) return TERN_EINVAL;
   tern::BatchParams* bp = new (std::nothrow) tern::BatchParams();
   if (!bp) return TERN_EINVAL;
   size_t smem = 0, ws = 0;
-  tern_status st = fill_batch(items, count, act, *bp, smem, ws);
+  tern_status st = fill_batch(items, count, M, act, *bp, smem, ws);
   if (st == TERN_OK && workspace_bytes < ws) st = TERN_EINVAL;
   if (st == TERN_OK) {
     bp->xprep = static_cast<uint8_t*>(workspace_dev);
@@ -213,6 +220,11 @@ tern_status tern_gemv_batch(const tern_gemv_item* items, int32_t count, tern_act
   }
   delete bp;
   return st;
+}
+
+tern_status tern_gemv_batch(const tern_gemv_item* items, int32_t count, tern_act act, void* workspace_dev,
+                            size_t workspace_bytes, uint32_t flags, tern_stream_t stream) {
+  return tern_gemm_batch(items, count, 1, act, workspace_dev, workspace_bytes, flags, stream);
 }
 
 size_t i8_head_workspace_bytes(int32_t V, int32_t M) {
@@ -280,16 +292,31 @@ tern_status tern_read_flag(const int32_t* err_flag_dev, tern_stream_t stream) {
 }
 
 tern_status tern_device_status(tern_stream_t stream) {
-  int v = 0, w = 0;
+  int v = 0, w = 0, x = 0;
   if (tern::read_and_clear_error_latch(&v, cs(stream)) != cudaSuccess) return TERN_ECUDA;
   if (tern::read_and_clear_batch_latch(&w) != cudaSuccess) return TERN_ECUDA;
-  return (v == 0 && w == 0) ? TERN_OK : TERN_ETIMEOUT;
+  if (tern::read_and_clear_prefill_latch(&x) != cudaSuccess) return TERN_ECUDA;
+  return (v == 0 && w == 0 && x == 0) ? TERN_OK : TERN_ETIMEOUT;
 }
 
 tern_status tern_gemm_prefill(const tern_matrix* W, int32_t M, const uint16_t* X_bf16_dev, float* Y_dev,
                               tern_stream_t stream) {
-  (void)W; (void)M; (void)X_bf16_dev; (void)Y_dev; (void)stream;
-  return TERN_EINVAL;
+  tern_status st = check_matrix(W);
+  if (st != TERN_OK) return st;
+  if (!X_bf16_dev || !Y_dev || !aligned(X_bf16_dev, 16) || !aligned(Y_dev, 4)) return TERN_EINVAL;
+  if (M < 1 || M > 65536) return TERN_ESHAPE;
+  tern::PrefillParams p = {};
+  p.planes = W->planes;
+  p.scale = W->scale_f16;
+  p.Y = Y_dev;
+  p.M = M;
+  p.N = W->N;
+  p.K = W->K;
+  p.vec_store = (W->N % 4 == 0 && aligned(Y_dev, 16)) ? 1 : 0;
+  int grid = 0;
+  size_t smem = 0;
+  if (!tern::plan_prefill(p, X_bf16_dev, grid, smem)) return TERN_ESHAPE;
+  return from_cuda(tern::launch_prefill(p, grid, smem, cs(stream)));
 }
 
 }  // extern "C"

@@ -39,21 +39,13 @@ __device__ int g_batch_latch = 0;
 
 namespace {
 
-#ifndef TERN_BATCH_CW
-#define TERN_BATCH_CW 12
-#endif
-#ifndef TERN_BATCH_TPW
-#define TERN_BATCH_TPW 2
-#endif
-constexpr int kCW = TERN_BATCH_CW;                    // consumer warps (kBoxRows <= 256: at most 16)
-constexpr int kTPW = TERN_BATCH_TPW;                  // tiles of 16 rows per consumer warp
-static_assert(kCW >= 1 && kCW <= 16 && kTPW >= 1 && kTPW <= 4, "batch kernel shape");
-constexpr int kBatchThreads = (kCW + 1) * 32;
-constexpr int kBoxRows = kCW * 16;                    // rows of one TMA box: tile slot a of every warp
-constexpr int kStageRows = kBoxRows * kTPW;           // rows of a row block
 constexpr int kPartWords = 16;                        // words per plane and row in a 512-trit part
-constexpr int kBoxBytes = 2 * kBoxRows * kPartWords * 4;
-constexpr int kWStageBytes = kTPW * kBoxBytes;
+// Consumer warps of a kernel shape, and the rows / bytes of one TMA box (tile slot a of every
+// consumer warp). A CTA's warps are spread over the SM's four sub-partitions, each with 16K
+// registers: 12 consumers + 1 producer put 4 warps on one sub-partition (<= 128 registers per
+// thread), 11 + 1 put 3 (<= 168).
+__host__ __device__ constexpr int box_rows(int cw) { return cw * 16; }
+__host__ __device__ constexpr int box_bytes(int cw) { return 2 * box_rows(cw) * kPartWords * 4; }
 constexpr int kColWords = 132;                        // operand words per column and part (128 + bank skew)
 constexpr uint32_t kWaitTries = 1u << 13;
 constexpr int kLimbFrac = 22;
@@ -109,23 +101,42 @@ __device__ __forceinline__ double exp2_i(int e) { return __longlong_as_double((l
 __device__ __forceinline__ int part_slot(int w, int h) { return ((w & 3) * 4 + (w >> 2)) * 8 + 4 * h; }
 
 // ---------------------------------------------------------------------------------------------
-// prep: one CTA per item. Block layout: kp segments of seg_bytes =
-//   [nc columns x kColWords words][nc column sums over all of K][E][padding to 16 bytes].
+// Operand columns of a segment. M = 1 (mp == 1): the nc columns are the limbs L2, L1, L0 (bf16
+// mode) or q (int8 mode). M >= 2 (mp = 8 or 16 token slots): int8 mode column m = token m; bf16
+// mode column l * mp + m = limb l of token m, so each MMA group of 8 columns holds one limb of
+// eight tokens and a lane ends up with all three limbs of the tokens it owns.
+__host__ __device__ constexpr int seg_cols(int mode, int mp) { return mp == 1 ? (mode == 0 ? 3 : 1) : (mode == 0 ? 3 * mp : mp); }
+// Segment words: columns, then the column sums over all of K, then E per token slot, padded to 16 B.
+__host__ __device__ constexpr int seg_words(int mode, int mp) {
+  return (seg_cols(mode, mp) * kColWords + seg_cols(mode, mp) + mp + 3) & ~3;
+}
+
+// prep: one CTA per (item, token slot). Block layout: kp segments of seg_bytes.
 __global__ void __launch_bounds__(256) k_batch_prep(const __grid_constant__ BatchParams p) {
   const BatchItem& it = p.items[blockIdx.x];
+  const int m = blockIdx.y;                          // token slot (< mp)
   uint32_t* blk = reinterpret_cast<uint32_t*>(p.xprep + it.xoff);
-  const int K = it.K, KP = it.kp, NC = p.nc;
+  const int K = it.K, KP = it.kp, mp = p.mp;
+  const int ncols = seg_cols(p.mode, mp);
   const int segw = p.seg_bytes / 4;
+  const int nl = p.mode == 0 ? 3 : 1;                // columns of this token
+  int colof[3];
+  for (int l = 0; l < 3; ++l) colof[l] = mp == 1 ? l : l * mp + m;
+  const bool live = m < p.M;
   __shared__ float red[8];
   __shared__ int sums[3];
   __shared__ int Esh;
   pdl_wait();
-  for (int i = threadIdx.x; i < KP * segw; i += blockDim.x) blk[i] = 0u;
+  // this token's columns (and its meta words) start at zero: the K tail of the last part stays so
+  for (int i = threadIdx.x; i < KP * nl * kColWords; i += blockDim.x) {
+    const int part = i / (nl * kColWords), r = i % (nl * kColWords);
+    blk[part * segw + colof[r / kColWords] * kColWords + r % kColWords] = 0u;
+  }
   if (threadIdx.x < 3) sums[threadIdx.x] = 0;
   if (threadIdx.x == 0) Esh = 0;
   float f = 1.0f;
-  if (p.mode == 0) {
-    const uint16_t* xb = static_cast<const uint16_t*>(it.x);
+  if (p.mode == 0 && live) {
+    const uint16_t* xb = static_cast<const uint16_t*>(it.x) + (size_t)m * K;
     float amax = 0.0f;
     for (int k = threadIdx.x * 8; k < K; k += blockDim.x * 8) {
       const uint4 v = ld_nc(xb + k);
@@ -138,11 +149,11 @@ __global__ void __launch_bounds__(256) k_batch_prep(const __grid_constant__ Batc
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
     __syncthreads();
     if (threadIdx.x == 0) {
-      float m = red[0];
-      for (int i = 1; i < 8; ++i) m = fmaxf(m, red[i]);
+      float mx = red[0];
+      for (int i = 1; i < 8; ++i) mx = fmaxf(mx, red[i]);
       int E = 0;
-      if (m > 0.0f) {
-        frexpf(m, &E);                               // m < 2^E
+      if (mx > 0.0f) {
+        frexpf(mx, &E);                              // mx < 2^E
         E = max(E, -100);
       }
       Esh = E;
@@ -153,16 +164,16 @@ __global__ void __launch_bounds__(256) k_batch_prep(const __grid_constant__ Batc
   __syncthreads();
   // one 16-element half of a 32-trit word per thread iteration
   int ls[3] = {0, 0, 0};
-  for (int v = threadIdx.x; v < K / 16; v += blockDim.x) {
+  for (int v = threadIdx.x; live && v < K / 16; v += blockDim.x) {
     const int word = v >> 1, h = v & 1;              // global word index and half
     const int part = word >> 4, w = word & 15;
     uint32_t* seg = blk + part * segw + part_slot(w, h);
     if (p.mode == 1) {
-      const uint4 q = ld_nc(static_cast<const int8_t*>(it.x) + 16 * v);
+      const uint4 q = ld_nc(static_cast<const int8_t*>(it.x) + (size_t)m * K + 16 * v);
       ls[0] += bsum(q.x) + bsum(q.y) + bsum(q.z) + bsum(q.w);
-      *reinterpret_cast<uint4*>(seg) = permute_i8_half(q);
+      *reinterpret_cast<uint4*>(seg + colof[0] * kColWords) = permute_i8_half(q);
     } else {
-      const uint16_t* xb = static_cast<const uint16_t*>(it.x) + 16 * v;
+      const uint16_t* xb = static_cast<const uint16_t*>(it.x) + (size_t)m * K + 16 * v;
       const uint4 a = ld_nc(xb), b = ld_nc(xb + 8);
       const uint32_t wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
       uint32_t l[3][4] = {};
@@ -182,12 +193,12 @@ __global__ void __launch_bounds__(256) k_batch_prep(const __grid_constant__ Batc
 #pragma unroll
       for (int c = 0; c < 3; ++c) {
         ls[c] += bsum(l[c][0]) + bsum(l[c][1]) + bsum(l[c][2]) + bsum(l[c][3]);
-        *reinterpret_cast<uint4*>(seg + c * kColWords) =
+        *reinterpret_cast<uint4*>(seg + colof[c] * kColWords) =
             permute_i8_half(make_uint4(l[c][0], l[c][1], l[c][2], l[c][3]));
       }
     }
   }
-  for (int c = 0; c < NC; ++c) {
+  for (int c = 0; c < nl; ++c) {
     int v = ls[c];
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
     if ((threadIdx.x & 31) == 0) atomicAdd(&sums[c], v);
@@ -195,18 +206,27 @@ __global__ void __launch_bounds__(256) k_batch_prep(const __grid_constant__ Batc
   __syncthreads();
   // every segment carries the sums over all of K and E, so the consumer reads them from a stage
   for (int part = threadIdx.x; part < KP; part += blockDim.x) {
-    int* meta = reinterpret_cast<int*>(blk + part * segw + NC * kColWords);
-    for (int c = 0; c < NC; ++c) meta[c] = sums[c];
-    meta[NC] = Esh;
+    int* meta = reinterpret_cast<int*>(blk + part * segw + ncols * kColWords);
+    for (int c = 0; c < nl; ++c) meta[colof[c]] = sums[c];
+    meta[ncols + m] = Esh;
   }
   pdl_launch_dependents();
 }
 
 // ---------------------------------------------------------------------------------------------
-template <int MODE>
-__global__ void __launch_bounds__(kBatchThreads, 1) k_batch_stream(const __grid_constant__ BatchParams p) {
+// MODE: 0 bf16 / 1 int8 activations; MP: token slots (1, 8 or 16); TPW: tiles per consumer warp;
+// CW: consumer warps.
+template <int MODE, int MP, int TPW, int CW>
+__global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_constant__ BatchParams p) {
+  constexpr int kCW = CW;
+  constexpr int kBoxRows = box_rows(CW);
+  constexpr int kBoxBytes = box_bytes(CW);
   extern __shared__ __align__(1024) uint8_t smem[];
-  constexpr int NC = MODE == 0 ? 3 : 1;
+  constexpr int NCOL = seg_cols(MODE, MP);
+  constexpr int G = MP == 1 ? 1 : NCOL / 8;                 // MMA column groups
+  constexpr int JJ = MP == 1 ? 1 : MP / 8;                  // groups per limb (token octets)
+  constexpr int kStageRowsT = kBoxRows * TPW;
+  constexpr int kWStageBytesT = TPW * kBoxBytes;
   const int S = p.stages;
   // layout: [full[S], empty[S] mbarriers; 1 KB][ring: S slots of stage_slot_bytes]
   //   slot: [tile slot 0 box][tile slot 1 box]...[operand segment]
@@ -256,10 +276,10 @@ __global__ void __launch_bounds__(kBatchThreads, 1) k_batch_stream(const __grid_
       const uint32_t bar = full0 + 8 * q;
       const uint32_t dst = ring + (uint32_t)q * slot_bytes;
       int boxes = 0;
-      for (int b = 0; b < kTPW; ++b) boxes += (rb * kStageRows + b * kBoxRows < B.N) ? 1 : 0;
+      for (int b = 0; b < TPW; ++b) boxes += (rb * kStageRowsT + b * kBoxRows < B.N) ? 1 : 0;
       mbar_arrive_expect_tx(bar, (uint32_t)(boxes * kBoxBytes + p.seg_bytes));
       for (int b = 0; b < boxes; ++b)
-        tma_load_3d(dst + b * kBoxBytes, &p.tmap[it], part * kPartWords, rb * kStageRows + b * kBoxRows, 0, bar);
+        tma_load_3d(dst + b * kBoxBytes, &p.tmap[it], part * kPartWords, rb * kStageRowsT + b * kBoxRows, 0, bar);
       if (++part == B.kp) {
         part = 0;
         if (++rb == B.units) { rb = 0; ++it; }
@@ -277,12 +297,12 @@ __global__ void __launch_bounds__(kBatchThreads, 1) k_batch_stream(const __grid_
       if (q >= S) {
         if (!(ok = mbar_wait(empty0 + 8 * s, ph ^ 1u))) break;
         int boxes = 0;
-        for (int b = 0; b < kTPW; ++b) boxes += (rb * kStageRows + b * kBoxRows < B.N) ? 1 : 0;
+        for (int b = 0; b < TPW; ++b) boxes += (rb * kStageRowsT + b * kBoxRows < B.N) ? 1 : 0;
         mbar_arrive_expect_tx(bar, (uint32_t)(boxes * kBoxBytes + p.seg_bytes));
         for (int b = 0; b < boxes; ++b)
-          tma_load_3d(dst + b * kBoxBytes, &p.tmap[it], part * kPartWords, rb * kStageRows + b * kBoxRows, 0, bar);
+          tma_load_3d(dst + b * kBoxBytes, &p.tmap[it], part * kPartWords, rb * kStageRowsT + b * kBoxRows, 0, bar);
       }
-      bulk_g2s(dst + kWStageBytes, p.xprep + B.xoff + (size_t)part * p.seg_bytes, (uint32_t)p.seg_bytes, bar);
+      bulk_g2s(dst + kWStageBytesT, p.xprep + B.xoff + (size_t)part * p.seg_bytes, (uint32_t)p.seg_bytes, bar);
       if (++part == B.kp) {
         part = 0;
         if (++rb == B.units) { rb = 0; ++it; }
@@ -304,11 +324,13 @@ __global__ void __launch_bounds__(kBatchThreads, 1) k_batch_stream(const __grid_
 
   // ====================== consumers ======================
   const int g = lane >> 2, t = lane & 3;
-  const int col = g < NC ? g : 0;                           // operand column this lane feeds
+  // operand column of group j this lane feeds: M = 1: the lane's limb (rows g >= nc repeat column 0)
+  const int col0 = MP == 1 ? (g < NCOL ? g : 0) : g;
   // byte offsets inside a slot
   const uint32_t wofs = (uint32_t)((warp * 16 + g) * kPartWords * 4 + t * 16);   // plane 0, row g
-  const uint32_t xofs = (uint32_t)(kWStageBytes + (col * kColWords + t * 8) * 4);
-  const uint32_t mofs = (uint32_t)(kWStageBytes + NC * kColWords * 4);
+  const uint32_t xofs = (uint32_t)(kWStageBytesT + (col0 * kColWords + t * 8) * 4);
+  const uint32_t mofs = (uint32_t)(kWStageBytesT + NCOL * kColWords * 4);
+  const int M = p.M;
   bool ok = true;
   int it = first_item, rb = u0 - p.items[first_item].unit0;
   int s = 0;
@@ -316,34 +338,46 @@ __global__ void __launch_bounds__(kBatchThreads, 1) k_batch_stream(const __grid_
   for (int u = u0; u < u1 && ok; ++u) {
     const BatchItem& B = p.items[it];
     const int KP = B.kp;
-    const int row_base = rb * kStageRows + warp * 16;          // first row of this warp's tile slot 0
-    int acc[kTPW][4][4];
+    const int row_base = rb * kStageRowsT + warp * 16;         // first row of this warp's tile slot 0
+    int acc[TPW][G][4][4];
 #pragma unroll
-    for (int a = 0; a < kTPW; ++a)
+    for (int a = 0; a < TPW; ++a)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[a][i][0] = acc[a][i][1] = acc[a][i][2] = acc[a][i][3] = 0;
-    int tot[3] = {0, 0, 0};
-    int E = 0;
+      for (int j = 0; j < G; ++j)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[a][j][i][0] = acc[a][j][i][1] = acc[a][j][i][2] = acc[a][j][i][3] = 0;
+    // column sums (over all of K) and exponents of the columns this lane owns
+    //   M = 1: tot[c] for c < nc, E; M >= 2: [jj][limb][token parity], E per [jj][parity]
+    int tot[JJ][3][2];
+    int Etok[JJ][2];
+    float sxv[JJ][2];
     // the epilogue's reads of the row scales (weights: written before any launch of this list),
     // issued now so that they land while the block streams
-    float sxv = 0.0f;
-    uint16_t sc_bits[kTPW][2];
+    uint16_t sc_bits[TPW][2];
 #pragma unroll
-    for (int a = 0; a < kTPW; ++a)
+    for (int a = 0; a < TPW; ++a)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int row = row_base + a * kBoxRows + g + 8 * h;
-        sc_bits[a][h] = (t == 0 && row < B.N) ? B.scale[row] : (uint16_t)0;
+        sc_bits[a][h] = ((MP > 1 || t == 0) && row < B.N) ? B.scale[row] : (uint16_t)0;
       }
     for (int part = 0; part < KP; ++part) {
       if (!(ok = mbar_wait(full0 + 8 * s, ph))) break;
       // s_x comes from an earlier kernel: read only after a stage has landed (the producer issues
       // every copy after its grid-dependency wait)
-      if (MODE == 1 && part == 0) sxv = B.sx[0];
-      const uint32_t st = ring + (uint32_t)s * slot_bytes;
-      uint4 ma[kTPW], mb[kTPW], sa[kTPW], sb[kTPW];
+      if (MODE == 1 && part == 0) {
 #pragma unroll
-      for (int a = 0; a < kTPW; ++a) {
+        for (int jj = 0; jj < JJ; ++jj)
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            const int m = MP == 1 ? 0 : 8 * jj + 2 * t + b;
+            sxv[jj][b] = m < M ? B.sx[m] : 0.0f;
+          }
+      }
+      const uint32_t st = ring + (uint32_t)s * slot_bytes;
+      uint4 ma[TPW], mb[TPW], sa[TPW], sb[TPW];
+#pragma unroll
+      for (int a = 0; a < TPW; ++a) {
         const uint32_t r = st + a * kBoxBytes + wofs;
         ma[a] = lds128(r);
         mb[a] = lds128(r + 8 * kPartWords * 4);
@@ -352,25 +386,62 @@ __global__ void __launch_bounds__(kBatchThreads, 1) k_batch_stream(const __grid_
       }
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const uint4 x0 = lds128(st + xofs + e * 128);
-        const uint4 x1 = lds128(st + xofs + e * 128 + 16);
+        // the word's operand registers for every tile (4 fields x 4 registers), then one group of
+        // activation columns at a time
+        uint32_t A[TPW][4][4];
 #pragma unroll
-        for (int a = 0; a < kTPW; ++a) {
+        for (int a = 0; a < TPW; ++a) {
           uint32_t wa0, wb0, wa1, wb1;
           merge_planes_offset(u4get(ma[a], e), u4get(sa[a], e), wa0, wb0);
           merge_planes_offset(u4get(mb[a], e), u4get(sb[a], e), wa1, wb1);
-          mma_u8s8(acc[a][0], wa0 & 0x03030303u, wa1 & 0x03030303u, wb0 & 0x03030303u, wb1 & 0x03030303u, x0.x, x1.x);
-          mma_u8s8(acc[a][1], wa0 & 0x0C0C0C0Cu, wa1 & 0x0C0C0C0Cu, wb0 & 0x0C0C0C0Cu, wb1 & 0x0C0C0C0Cu, x0.y, x1.y);
-          mma_u8s8(acc[a][2], wa0 & 0x30303030u, wa1 & 0x30303030u, wb0 & 0x30303030u, wb1 & 0x30303030u, x0.z, x1.z);
-          mma_u8s8(acc[a][3], wa0 & 0xC0C0C0C0u, wa1 & 0xC0C0C0C0u, wb0 & 0xC0C0C0C0u, wb1 & 0xC0C0C0C0u, x0.w, x1.w);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t msk = 0x03030303u << (2 * i);
+            A[a][i][0] = wa0 & msk;
+            A[a][i][1] = wa1 & msk;
+            A[a][i][2] = wb0 & msk;
+            A[a][i][3] = wb1 & msk;
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+          const uint4 x0 = lds128(st + xofs + (j * 8 * kColWords) * 4 + e * 128);
+          const uint4 x1 = lds128(st + xofs + (j * 8 * kColWords) * 4 + e * 128 + 16);
+#pragma unroll
+          for (int a = 0; a < TPW; ++a)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              mma_u8s8(acc[a][j][i], A[a][i][0], A[a][i][1], A[a][i][2], A[a][i][3], u4get(x0, i), u4get(x1, i));
         }
       }
       if (part == KP - 1) {                                  // sums over all of K and E ride in every segment
-        const uint4 m4 = lds128(st + mofs);
-        tot[0] = (int)m4.x;
-        tot[1] = (int)m4.y;
-        tot[2] = (int)m4.z;
-        E = (int)m4.w;
+#pragma unroll
+        for (int jj = 0; jj < JJ; ++jj)
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            if (MP == 1) {
+              if (jj == 0 && b == 0) {
+                const uint4 m4 = lds128(st + mofs);
+                tot[0][0][0] = (int)m4.x;
+                tot[0][1][0] = (int)m4.y;
+                tot[0][2][0] = (int)m4.z;
+                Etok[0][0] = MODE == 0 ? (int)m4.w : 0;
+              }
+            } else {
+              const int m = 8 * jj + 2 * t + b;
+#pragma unroll
+              for (int l = 0; l < 3; ++l) {
+                if (MODE == 0 || l == 0) {
+                  uint32_t v;
+                  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(st + mofs + 4u * (uint32_t)(l * MP + m)));
+                  tot[jj][l][b] = (int)v;
+                }
+              }
+              uint32_t ev;
+              asm volatile("ld.shared.u32 %0, [%1];" : "=r"(ev) : "r"(st + mofs + 4u * (uint32_t)(NCOL + m)));
+              Etok[jj][b] = (int)ev;
+            }
+          }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(empty0 + 8 * s);
@@ -379,40 +450,71 @@ __global__ void __launch_bounds__(kBatchThreads, 1) k_batch_stream(const __grid_
     if (!ok) break;
     // ---- outputs of this warp's tiles: exact integer sums, one rounding ----------------------------
 #pragma unroll
-    for (int a = 0; a < kTPW; ++a) {
-      int v[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        v[q] = acc[a][0][q] + (acc[a][1][q] >> 2) + (acc[a][2][q] >> 4) + (acc[a][3][q] >> 6);
+    for (int a = 0; a < TPW; ++a) {
       const int r0 = row_base + a * kBoxRows + g;            // rows r0 (q = 0, 1) and r0 + 8 (q = 2, 3)
-      if (MODE == 1) {
-        if (t == 0) {
+      if (MP == 1) {
+        int v[4];
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int row = r0 + 8 * h;
-            if (row < B.N) {
-              const int S1 = v[2 * h] - 2 * tot[0];
-              B.y[row] = __fmul_rn(__fmul_rn(__int2float_rn(S1), sxv), f16_bits_to_float(sc_bits[a][h]));
+        for (int q = 0; q < 4; ++q)
+          v[q] = acc[a][0][0][q] + (acc[a][0][1][q] >> 2) + (acc[a][0][2][q] >> 4) + (acc[a][0][3][q] >> 6);
+        if (MODE == 1) {
+          if (t == 0) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int row = r0 + 8 * h;
+              if (row < B.N) {
+                const int S1 = v[2 * h] - 2 * tot[0][0][0];
+                B.y[row] = __fmul_rn(__fmul_rn(__int2float_rn(S1), sxv[0][0]), f16_bits_to_float(sc_bits[a][h]));
+              }
+            }
+          }
+        } else {
+          // lane t = 0 holds columns 0 (L2) and 1 (L1), lane t = 1 column 2 (L0)
+          const int l0a = __shfl_down_sync(0xFFFFFFFFu, v[0], 1);
+          const int l0b = __shfl_down_sync(0xFFFFFFFFu, v[2], 1);
+          if (t == 0) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int row = r0 + 8 * h;
+              if (row < B.N) {
+                const long long S2 = v[2 * h] - 2LL * tot[0][0][0];
+                const long long S1 = v[2 * h + 1] - 2LL * tot[0][1][0];
+                const long long S0 = (h ? l0b : l0a) - 2LL * tot[0][2][0];
+                const long long D = S2 * 65536 + S1 * 256 + S0;
+                B.y[row] = (float)((double)D * exp2_i(Etok[0][0] - kLimbFrac) * (double)f16_bits_to_float(sc_bits[a][h]));
+              }
             }
           }
         }
       } else {
-        // lane t = 0 holds columns 0 (L2) and 1 (L1), lane t = 1 column 2 (L0)
-        const int l0a = __shfl_down_sync(0xFFFFFFFFu, v[0], 1);
-        const int l0b = __shfl_down_sync(0xFFFFFFFFu, v[2], 1);
-        if (t == 0) {
+        // lane (g, t) holds, for rows r0 and r0 + 8, the columns 2t and 2t + 1 of every group:
+        // tokens m = 8 jj + 2t + b, with all of their limbs (groups l * JJ + jj)
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
+        for (int jj = 0; jj < JJ; ++jj)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int b = q & 1, h = q >> 1;
+            const int m = 8 * jj + 2 * t + b;
             const int row = r0 + 8 * h;
-            if (row < B.N) {
-              const long long S2 = v[2 * h] - 2LL * tot[0];
-              const long long S1 = v[2 * h + 1] - 2LL * tot[1];
-              const long long S0 = (h ? l0b : l0a) - 2LL * tot[2];
-              const long long D = S2 * 65536 + S1 * 256 + S0;
-              B.y[row] = (float)((double)D * exp2_i(E - kLimbFrac) * (double)f16_bits_to_float(sc_bits[a][h]));
+            if (m < M && row < B.N) {
+              const float sc = f16_bits_to_float(sc_bits[a][h]);
+              if (MODE == 1) {
+                const int v = acc[a][jj][0][q] + (acc[a][jj][1][q] >> 2) + (acc[a][jj][2][q] >> 4) + (acc[a][jj][3][q] >> 6);
+                const int S1 = v - 2 * tot[jj][0][b];
+                B.y[(size_t)m * B.N + row] = __fmul_rn(__fmul_rn(__int2float_rn(S1), sxv[jj][b]), sc);
+              } else {
+                long long Sl[3];
+#pragma unroll
+                for (int l = 0; l < 3; ++l) {
+                  const int j = l * JJ + jj;
+                  const int v = acc[a][j][0][q] + (acc[a][j][1][q] >> 2) + (acc[a][j][2][q] >> 4) + (acc[a][j][3][q] >> 6);
+                  Sl[l] = (long long)v - 2LL * tot[jj][l][b];
+                }
+                const long long D = Sl[0] * 65536 + Sl[1] * 256 + Sl[2];
+                B.y[(size_t)m * B.N + row] = (float)((double)D * exp2_i(Etok[jj][b] - kLimbFrac) * (double)sc);
+              }
             }
           }
-        }
       }
     }
     if (++rb == B.units) { rb = 0; ++it; }
@@ -432,12 +534,39 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+// Token slots, tiles per warp and consumer warps for M rows: the accumulators (tiles x groups x
+// 16 registers) stay at or under 96 registers.
+void batch_shape(int mode, int M, int& mp, int& tpw, int& cw) {
+  mp = M == 1 ? 1 : (M <= 8 ? 8 : 16);
+  tpw = (mode == 0 && M > 1) ? 1 : 2;
+  cw = M == 1 ? 12 : 11;
+}
+
+template <int MODE, int MP, int TPW, int CW>
+cudaError_t launch_stream_kernel(cudaLaunchConfig_t& cfg, const BatchParams& p, size_t smem) {
+  static int set = 0;
+  if ((int)smem > set) {
+    cudaError_t e = cudaFuncSetAttribute(k_batch_stream<MODE, MP, TPW, CW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    set = (int)smem;
+  }
+  cfg.blockDim = dim3((CW + 1) * 32, 1, 1);
+  return cudaLaunchKernelEx(&cfg, k_batch_stream<MODE, MP, TPW, CW>, p);
+}
+
 }  // namespace
 
 bool plan_batch(BatchParams& p, const uint32_t* const* planes, size_t& smem, size_t& workspace) {
-  const int nc = p.mode == 0 ? 3 : 1;
-  p.nc = nc;
-  p.seg_bytes = ((nc * kColWords + 4) * 4 + 15) & ~15;
+  if (p.M < 1 || p.M > 16) return false;
+  int mp = 1, tpw = 2, cw = 12;
+  batch_shape(p.mode, p.M, mp, tpw, cw);
+  p.mp = mp;
+  p.tpw = tpw;
+  p.cw = cw;
+  const int kBoxRows = box_rows(cw), kBoxBytes = box_bytes(cw);
+  p.nc = seg_cols(p.mode, mp);
+  p.seg_bytes = seg_words(p.mode, mp) * 4;
+  const int stage_rows = kBoxRows * tpw;
   PFN_cuTensorMapEncodeTiled_v12000 encode = encode_fn();
   if (!encode) return false;
   long long total_bytes = 0;
@@ -448,7 +577,7 @@ bool plan_batch(BatchParams& p, const uint32_t* const* planes, size_t& smem, siz
     if (it.K % 128 || it.K <= 0 || it.N <= 0) return false;
     it.kp = (it.K + 511) / 512;
     it.unit0 = units;
-    it.units = (it.N + kStageRows - 1) / kStageRows;
+    it.units = (it.N + stage_rows - 1) / stage_rows;
     units += it.units;
     it.xoff = (uint32_t)xoff;
     xoff += (size_t)it.kp * p.seg_bytes;
@@ -475,13 +604,13 @@ bool plan_batch(BatchParams& p, const uint32_t* const* planes, size_t& smem, siz
     const BatchItem& it = p.items[i];
     for (int u = 0; u < it.units; ++u) {
       while (c + 1 < grid && acc >= total_bytes * (c + 1) / grid) p.cta_unit[++c] = it.unit0 + u;
-      const int rows = it.N - u * kStageRows < kStageRows ? it.N - u * kStageRows : kStageRows;
+      const int rows = it.N - u * stage_rows < stage_rows ? it.N - u * stage_rows : stage_rows;
       acc += (long long)rows * it.K / 4;
     }
   }
   while (c + 1 <= grid) p.cta_unit[++c] = units;
   p.cta_unit[grid] = units;
-  p.stage_slot_bytes = (kWStageBytes + p.seg_bytes + 1023) & ~1023;
+  p.stage_slot_bytes = (tpw * kBoxBytes + p.seg_bytes + 1023) & ~1023;
   const size_t budget = 227 * 1024;
   int stages = (int)((budget - 1024) / (size_t)p.stage_slot_bytes);
   if (stages > 8) stages = 8;
@@ -510,8 +639,8 @@ cudaError_t launch_batch(const BatchParams& p, size_t smem, bool pdl, cudaStream
   cfg.attrs = attr;
   cfg.numAttrs = na;
   cfg.stream = st;
-  // 1. operand segments
-  cfg.gridDim = dim3(p.count, 1, 1);
+  // 1. operand segments: one CTA per (item, token slot)
+  cfg.gridDim = dim3(p.count, p.mp, 1);
   cfg.blockDim = dim3(256, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cudaError_t e = cudaLaunchKernelEx(&cfg, k_batch_prep, p);
@@ -523,24 +652,15 @@ cudaError_t launch_batch(const BatchParams& p, size_t smem, bool pdl, cudaStream
   cfg.attrs = attr2;
   cfg.numAttrs = 1;
   cfg.gridDim = dim3(p.grid, 1, 1);
-  cfg.blockDim = dim3(kBatchThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   if (p.mode == 0) {
-    static int set0 = 0;
-    if ((int)smem > set0) {
-      e = cudaFuncSetAttribute(k_batch_stream<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      set0 = (int)smem;
-    }
-    return cudaLaunchKernelEx(&cfg, k_batch_stream<0>, p);
+    if (p.mp == 1) return launch_stream_kernel<0, 1, 2, 12>(cfg, p, smem);
+    if (p.mp == 8) return launch_stream_kernel<0, 8, 1, 11>(cfg, p, smem);
+    return launch_stream_kernel<0, 16, 1, 11>(cfg, p, smem);
   }
-  static int set1 = 0;
-  if ((int)smem > set1) {
-    e = cudaFuncSetAttribute(k_batch_stream<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    set1 = (int)smem;
-  }
-  return cudaLaunchKernelEx(&cfg, k_batch_stream<1>, p);
+  if (p.mp == 1) return launch_stream_kernel<1, 1, 2, 12>(cfg, p, smem);
+  if (p.mp == 8) return launch_stream_kernel<1, 8, 2, 11>(cfg, p, smem);
+  return launch_stream_kernel<1, 16, 2, 11>(cfg, p, smem);
 }
 
 }  // namespace tern

@@ -48,12 +48,12 @@ cudaError_t launch_stream(const StreamParams& p, size_t smem, bool pdl, cudaStre
 // Reads and clears the device word that kernels set when a bounded wait gives up.
 cudaError_t read_and_clear_error_latch(int* out, cudaStream_t st);
 
-// Batched M = 1 GEMV over a list of matrices (tern_batch.cu).
+// Batched GEMV / small-M GEMM over a list of matrices (tern_batch.cu).
 struct BatchItem {
   const uint16_t* scale;
-  float* y;
-  const void* x;          // bf16 bits [K] or int8 [K]
-  const float* sx;        // int8 mode: [1]
+  float* y;               // [M][N]
+  const void* x;          // bf16 bits [M][K] or int8 [M][K]
+  const float* sx;        // int8 mode: [M]
   int32_t N, K;
   int32_t kp;             // 512-trit K parts (the last may be partial): stages per row block
   int32_t unit0;          // first global unit (row block) of the item
@@ -66,7 +66,11 @@ struct BatchParams {
   BatchItem items[kBatchMaxItems];
   int32_t count;
   int32_t mode;           // 0 = bf16 activations (three int8 limbs), 1 = int8
-  int32_t nc;             // operand columns: 3 or 1
+  int32_t nc;             // operand columns of a segment
+  int32_t M;              // activation rows (tokens), 1..16
+  int32_t mp;             // token slots: 1, 8 or 16
+  int32_t tpw;            // tiles of 16 rows per consumer warp
+  int32_t cw;             // consumer warps
   int32_t total_units;
   int32_t grid;
   int32_t stages;
@@ -80,6 +84,19 @@ static_assert(sizeof(BatchParams) <= 32764, "kernel parameter limit");
 bool plan_batch(BatchParams& p, const uint32_t* const* planes, size_t& smem, size_t& workspace);
 cudaError_t launch_batch(const BatchParams& p, size_t smem, bool pdl, cudaStream_t st);
 cudaError_t read_and_clear_batch_latch(int* out);
+
+// Prefill dense contraction on tcgen05 (tern_prefill.cu).
+struct PrefillParams {
+  CUtensorMap xmap;       // X bf16 [M][K], boxes of 64 x 128, 128-byte swizzle
+  const uint32_t* planes;
+  const uint16_t* scale;
+  float* Y;               // [M][N]
+  int32_t M, N, K;
+  int32_t vec_store;      // Y rows 16-byte aligned (N % 4 == 0 and Y aligned): 128-bit stores
+};
+bool plan_prefill(PrefillParams& p, const uint16_t* X, int& grid, size_t& smem);
+cudaError_t launch_prefill(const PrefillParams& p, int grid, size_t smem, cudaStream_t st);
+cudaError_t read_and_clear_prefill_latch(int* out);
 
 // int8 output head with argmax (tern_head.cu).
 struct HeadParams {

@@ -1,0 +1,379 @@
+// Prefill dense contraction on the 5th-generation tensor cores (tcgen05 + TMEM).
+//
+//   Y[m][n] = scale[n] * sum_k t[n][k] * X[m][k],   X bf16 [M][K], t packed ternary, Y fp32 [M][N]
+//
+// Prefill runs the same linear layers at M = prompt length ("batched prefill" of the PyTorchKR
+// review "Fermion Research, 3진 계열 포맷으로 직접 학습한 Neutrino-1 모델군 3종 공개", section
+// "실행해보기"), which makes the product a genuine dense contraction. The ternary weights stay
+// packed in HBM and are expanded only inside the kernel, in shared memory, right before the
+// tensor cores read them (weights packed at rest, aiatolah.com "Neutrino-1 8B: modelo ternario
+// ...", second paragraph); the products by +-1 / 0 are exact (origotech.dev Figure I).
+//
+// One persistent CTA per SM walks output tiles of BM = 128 tokens x BN = 256 weight rows:
+//   warp 0      TMA producer: X tile (128 x 64 bf16, 128-byte swizzle) per K stage;
+//   warp 1      allocates 512 TMEM columns (two fp32 accumulators of 128 x 256) and one lane
+//               issues tcgen05.mma kind::f16 (A = X tile, B = expanded weights, both K-major);
+//               tcgen05.commit frees a stage when the MMAs reading it are done;
+//   warps 2..5  expand the tile's 256 weight rows x 64 trits to bf16 (2.0 * t, the field decode
+//               of tern_device.cuh) in the same swizzled layout the tensor core reads;
+//   warps 6..9  epilogue: tcgen05.ld of the accumulator their TMEM lane quarter owns, times
+//               0.5 * scale[n], stored to Y; the second accumulator lets the next tile's MMAs run
+//               meanwhile.
+// Every mbarrier wait is bounded; a kernel that gives up latches TERN_ETIMEOUT, drains what it
+// issued (bounded), frees its TMEM and returns.
+#include <cstdint>
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include "tern_device.cuh"
+#include "tern_kernels.h"
+
+namespace tern {
+
+__device__ int g_prefill_latch = 0;
+
+namespace {
+
+constexpr int BM = 128;                          // tokens per tile: UMMA M, TMEM lanes
+constexpr int BN = 256;                          // weight rows per tile: UMMA N, accumulator columns
+constexpr int BK = 64;                           // K per stage: one 128-byte swizzle span of bf16
+constexpr int kStages = 4;
+constexpr int kABytes = BM * BK * 2;             // 16 KB
+constexpr int kBBytes = BN * BK * 2;             // 32 KB
+constexpr int kDecWarps = 4, kEpiWarps = 4;
+constexpr int kPrefillThreads = (2 + kDecWarps + kEpiWarps) * 32;
+constexpr int kTmemCols = 2 * BN;                // two accumulators
+constexpr uint32_t kWaitTries = 1u << 13;
+// smem: [A stages][B stages][barriers + TMEM address], stages 1024-byte aligned
+constexpr int kSmemA = 0;
+constexpr int kSmemB = kStages * kABytes;
+constexpr int kSmemBar = kSmemB + kStages * kBBytes;
+constexpr int kSmemBytes = kSmemBar + 256 + 1024;  // + barriers, + slack for 1024-byte alignment
+
+// Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator, A and B bf16, both
+// K-major, N = 256, M = 128.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                            ((uint32_t)(BM >> 4) << 24);
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kWaitTries; ++i) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(bar), "r"(parity), "r"(500000u)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+// Tiled 2-d tensor load (no multicast): box at (c0 = k, c1 = token).
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+}
+__device__ __forceinline__ uint2 ldg64(const void* p) {
+  uint2 v;
+  asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
+}
+// K-major, 128-byte-swizzled operand descriptor (sm_100 layout): start address, leading byte
+// offset 16 (unused for swizzled K-major), stride byte offset 1024 (8 rows x 128 B), version 1,
+// swizzle mode 2 (128 B).
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)(16u >> 4) << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accum) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
+      ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 32 consecutive fp32 accumulator columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// bf16 register A (0..15) of a merged word pair: trits 2A, 2A+1 of the 32-trit word as 2.0 * t.
+template <int A>
+__device__ __forceinline__ uint32_t dec2(uint32_t wa, uint32_t wb) {
+  return dec_bf16<A>(wa, wb);
+}
+
+__global__ void __launch_bounds__(kPrefillThreads, 1) k_prefill(const __grid_constant__ PrefillParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte alignment for the swizzled tiles
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  const uint32_t sA = base + kSmemA, sB = base + kSmemB, sBar = base + kSmemBar;
+  const uint32_t a_full = sBar, b_full = sBar + 8 * kStages, empty = sBar + 16 * kStages;
+  const uint32_t acc_full = sBar + 24 * kStages, acc_empty = acc_full + 16, done_bar = acc_empty + 16;
+  const uint32_t tmem_slot = done_bar + 8;
+  uint32_t* tmem_slot_ptr = reinterpret_cast<uint32_t*>(smem_raw + (tmem_slot - raw));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles_n = (p.N + BN - 1) / BN, tiles_m = (p.M + BM - 1) / BM;
+  const int tiles = tiles_m * tiles_n;
+  const int KT = p.K / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(a_full + 8 * s, 1);
+      mbar_init(b_full + 8 * s, kDecWarps);
+      mbar_init(empty + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(acc_full + 8 * a, 1);
+      mbar_init(acc_empty + 8 * a, kEpiWarps);
+    }
+    mbar_init(done_bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(tmem_slot), "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot_ptr;
+  bool ok = true;
+
+  if (warp == 0) {
+    // ---------------- TMA producer: X tiles ----------------
+    if (lane == 0) {
+      int q = 0;
+      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+        const int mt = tile / tiles_n;
+        for (int kt = 0; kt < KT; ++kt, ++q) {
+          const int s = q % kStages;
+          if (q >= kStages && !(ok = mbar_wait(empty + 8 * s, ((q / kStages) - 1) & 1))) break;
+          mbar_arrive_expect_tx(a_full + 8 * s, kABytes);
+          tma_load_2d(sA + s * kABytes, &p.xmap, kt * BK, mt * BM, a_full + 8 * s);
+        }
+      }
+      // do not leave with copies in flight (bounded, also after a give-up)
+      for (int r = q > kStages ? q - kStages : 0; r < q; ++r)
+        if (!mbar_wait(a_full + 8 * (r % kStages), (r / kStages) & 1)) { ok = false; break; }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issue (one lane) ----------------
+    if (lane == 0) {
+      int q = 0, tl = 0;
+      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++tl) {
+        const int acc = tl & 1;
+        if (tl >= 2 && !(ok = mbar_wait(acc_empty + 8 * acc, ((tl >> 1) - 1) & 1))) break;
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(acc * BN);
+        for (int kt = 0; kt < KT; ++kt, ++q) {
+          const int s = q % kStages;
+          const uint32_t ph = (q / kStages) & 1;
+          if (!(ok = mbar_wait(a_full + 8 * s, ph))) break;
+          if (!(ok = mbar_wait(b_full + 8 * s, ph))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            umma_bf16(d, umma_desc(sA + s * kABytes + 32 * k), umma_desc(sB + s * kBBytes + 32 * k), kIdesc,
+                      (kt > 0 || k > 0) ? 1u : 0u);
+          umma_commit(empty + 8 * s);                 // the stage is free once these MMAs are done
+        }
+        if (!ok) break;
+        umma_commit(acc_full + 8 * acc);              // the accumulator is complete
+      }
+      // every MMA this thread issued has completed once done_bar flips
+      umma_commit(done_bar);
+      if (!mbar_wait(done_bar, 0)) ok = false;
+    }
+  } else if (warp < 2 + kDecWarps) {
+    // ---------------- weight expansion: 256 rows x 64 trits -> bf16, swizzled ----------------
+    const int d = threadIdx.x - 64;                   // 0..127: rows d and d + 128 of the tile
+    const int KW = p.K / 16;                          // words per row (both planes)
+    int q = 0;
+    for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+      const int nt = tile % tiles_n;
+      const uint32_t* rowp[2];
+      bool live[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int n = nt * BN + d + 128 * h;
+        live[h] = n < p.N;
+        rowp[h] = p.planes + (size_t)(live[h] ? n : 0) * KW;
+      }
+      // words of the next stage, loaded one stage ahead
+      uint2 nm[2], ns[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        nm[h] = live[h] ? ldg64(rowp[h]) : make_uint2(0u, 0u);
+        ns[h] = live[h] ? ldg64(rowp[h] + KW / 2) : make_uint2(0u, 0u);
+      }
+      for (int kt = 0; kt < KT; ++kt, ++q) {
+        const int s = q % kStages;
+        uint2 cm[2] = {nm[0], nm[1]}, cs[2] = {ns[0], ns[1]};
+        if (kt + 1 < KT) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            nm[h] = live[h] ? ldg64(rowp[h] + 2 * (kt + 1)) : make_uint2(0u, 0u);
+            ns[h] = live[h] ? ldg64(rowp[h] + KW / 2 + 2 * (kt + 1)) : make_uint2(0u, 0u);
+          }
+        }
+        if (q >= kStages && !(ok = mbar_wait(empty + 8 * s, ((q / kStages) - 1) & 1))) break;
+        const uint32_t tileB = sB + s * kBBytes;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int r = d + 128 * h;
+          const uint32_t rowa = tileB + r * 128;
+          const int sw = r & 7;
+#pragma unroll
+          for (int w = 0; w < 2; ++w) {
+            uint32_t wa, wb;
+            merge_planes(w ? cm[h].y : cm[h].x, w ? cs[h].y : cs[h].x, wa, wb);
+            // 16-byte chunk c holds trits 8c .. 8c+7 of the stage: word w, registers 4(c%4) ..
+            sts128(rowa + (((4 * w + 0) ^ sw) << 4), dec2<0>(wa, wb), dec2<1>(wa, wb), dec2<2>(wa, wb), dec2<3>(wa, wb));
+            sts128(rowa + (((4 * w + 1) ^ sw) << 4), dec2<4>(wa, wb), dec2<5>(wa, wb), dec2<6>(wa, wb), dec2<7>(wa, wb));
+            sts128(rowa + (((4 * w + 2) ^ sw) << 4), dec2<8>(wa, wb), dec2<9>(wa, wb), dec2<10>(wa, wb), dec2<11>(wa, wb));
+            sts128(rowa + (((4 * w + 3) ^ sw) << 4), dec2<12>(wa, wb), dec2<13>(wa, wb), dec2<14>(wa, wb), dec2<15>(wa, wb));
+          }
+        }
+        // generic-proxy writes -> visible to the tensor core (async proxy), then signal
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(b_full + 8 * s);
+      }
+    }
+  } else {
+    // ---------------- epilogue: TMEM -> registers -> 0.5 * scale -> Y ----------------
+    const int quarter = warp & 3;                     // TMEM lanes 32*quarter .. +31
+    int tl = 0;
+    for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++tl) {
+      const int mt = tile / tiles_n, nt = tile % tiles_n;
+      const int acc = tl & 1;
+      if (!(ok = mbar_wait(acc_full + 8 * acc, (tl >> 1) & 1))) break;
+      tc_fence_after();
+      const int m = mt * BM + quarter * 32 + lane;
+      float* yrow = p.Y + (size_t)(m < p.M ? m : 0) * p.N;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN + 32 * c), r);
+        const int n0 = nt * BN + 32 * c;
+        if (m < p.M) {
+          if (p.vec_store && n0 + 32 <= p.N) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              float4 v;
+              v.x = __uint_as_float(r[j + 0]) * (0.5f * f16_bits_to_float(p.scale[n0 + j + 0]));
+              v.y = __uint_as_float(r[j + 1]) * (0.5f * f16_bits_to_float(p.scale[n0 + j + 1]));
+              v.z = __uint_as_float(r[j + 2]) * (0.5f * f16_bits_to_float(p.scale[n0 + j + 2]));
+              v.w = __uint_as_float(r[j + 3]) * (0.5f * f16_bits_to_float(p.scale[n0 + j + 3]));
+              *reinterpret_cast<float4*>(yrow + n0 + j) = v;
+            }
+          } else {
+            for (int j = 0; j < 32 && n0 + j < p.N; ++j)
+              yrow[n0 + j] = __uint_as_float(r[j]) * (0.5f * f16_bits_to_float(p.scale[n0 + j]));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty + 8 * acc);
+    }
+  }
+
+  if (!ok) atomicExch(&g_prefill_latch, 5);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+}  // namespace
+
+bool plan_prefill(PrefillParams& p, const uint16_t* X, int& grid, size_t& smem) {
+  if (p.M < 1 || p.N < 1 || p.K < BK || p.K % 128) return false;
+  PFN_cuTensorMapEncodeTiled_v12000 encode = encode_fn();
+  if (!encode) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)p.K, (cuuint64_t)p.M};
+  const cuuint64_t strides[1] = {(cuuint64_t)p.K * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)BM};
+  const cuuint32_t estr[2] = {1, 1};
+  if (encode(&p.xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  const int tiles = ((p.M + BM - 1) / BM) * ((p.N + BN - 1) / BN);
+  grid = tiles < 148 ? tiles : 148;
+  smem = kSmemBytes;
+  return true;
+}
+
+cudaError_t launch_prefill(const PrefillParams& p, int grid, size_t smem, cudaStream_t st) {
+  static int set = 0;
+  if (!set) {
+    cudaError_t e = cudaFuncSetAttribute(k_prefill, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    set = 1;
+  }
+  k_prefill<<<grid, kPrefillThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t read_and_clear_prefill_latch(int* out) {
+  cudaError_t e = cudaMemcpyFromSymbol(out, g_prefill_latch, sizeof(int));
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_prefill_latch, &zero, sizeof(int));
+}
+
+}  // namespace tern

@@ -173,6 +173,19 @@ size_t tern_gemv_batch_workspace_bytes(const tern_gemv_item* items, int32_t coun
 tern_status tern_gemv_batch(const tern_gemv_item* items, int32_t count, tern_act act, void* workspace_dev,
                             size_t workspace_bytes, uint32_t flags, tern_stream_t stream);
 
+/* Workspace bytes tern_gemm_batch needs for these items and M activation rows (0 if invalid). */
+size_t tern_gemm_batch_workspace_bytes(const tern_gemv_item* items, int32_t count, int32_t M, tern_act act);
+
+/* tern_gemv_batch for M activation rows per item (the draft-verify pass of speculative decoding
+ * over a whole layer list, [R] "검증된 추측 디코딩"): for every item,
+ *   Y[m][n] = scale[n] * sum_k t[n][k] * X[m][k],  0 <= m < M, 1 <= M <= 16,
+ * with each item's x_dev = X: bf16[M][K] or int8[M][K] row-major, x_scale_dev = float[M] (int8
+ * mode), y_dev = Y: float[M][N]. Each decoded weight word feeds all M rows; the weights stream
+ * once. Arithmetic, determinism, aliasing rule, workspace and flags as for tern_gemv_batch (whose
+ * call equals this one with M = 1). */
+tern_status tern_gemm_batch(const tern_gemv_item* items, int32_t count, int32_t M, tern_act act,
+                            void* workspace_dev, size_t workspace_bytes, uint32_t flags, tern_stream_t stream);
+
 /* Small-M GEMM for the draft-verify pass of speculative decoding ([R] "검증된 추측 디코딩": the
  * 8B scores up to seven drafted positions in one batched forward pass):
  *   Y[m][n] = scale[n] * sum_k t[n][k] * X[m][k],  0 <= m < M, 1 <= M <= 16.
@@ -185,9 +198,12 @@ tern_status tern_gemm_small_m_ex(const tern_matrix* W, int32_t M, tern_act act, 
                                  tern_stream_t stream);
 
 /* Prefill dense contraction ([R] "실행해보기": batched prefill):
- *   Y[m][n] = scale[n] * sum_k t[n][k] * X[m][k] for M up to 65536 rows of bf16 activations,
- * computed as a genuine dense matrix product on the tensor cores (trits expanded to bf16 in
- * shared memory, fp32 accumulation). X_bf16_dev: bf16[M][K]; Y_dev: float[M][N]. */
+ *   Y[m][n] = scale[n] * sum_k t[n][k] * X[m][k] for 1 <= M <= 65536 rows of bf16 activations,
+ * computed as a genuine dense matrix product on the 5th-generation tensor cores: trits expanded
+ * to bf16 (2.0 * t) in shared memory, tcgen05 MMA with the fp32 accumulator in tensor memory,
+ * times 0.5 * scale[n] at the end (one fp32 rounding of the accumulated sum, which the tensor
+ * core forms in fp32). X_bf16_dev: bf16[M][K] row-major, 16-byte aligned; Y_dev: float[M][N],
+ * 4-byte aligned (16-byte aligned with N % 4 == 0 for the fastest stores). */
 tern_status tern_gemm_prefill(const tern_matrix* W, int32_t M, const uint16_t* X_bf16_dev, float* Y_dev,
                               tern_stream_t stream);
 

@@ -114,3 +114,59 @@ def test_batch_argument_errors():
         tg.tern_gemv_batch([(W, x, None, y)], tg.TERN_ACT_BF16, ws)        # workspace too small
     with pytest.raises(tg.TernError):
         tg.tern_gemv_batch([(W, x, None, y)], tg.TERN_ACT_INT8, ws)        # int8 needs s_x
+
+
+def _build_m(seed, shapes, M, act):
+    items, refs = [], []
+    for i, (N, K) in enumerate(shapes):
+        W, t, s = make_matrix(seed, 300 + i, N, K, host_trits=N * K <= 4096 * 4096)
+        X = synth.activations(seed, 400 + i, M, K)
+        Xd = dev(X.view(np.int16))
+        if act == tg.TERN_ACT_INT8:
+            q = torch.empty(M * K, dtype=torch.int8, device="cuda")
+            sx = torch.empty(M, dtype=torch.float32, device="cuda")
+            tg.tern_quantize_act(Xd, M, K, q, sx)
+            xin, sxin = q, sx
+        else:
+            xin, sxin = Xd, None
+        Y = torch.full((M * N,), float("nan"), dtype=torch.float32, device="cuda")
+        items.append((W, xin, sxin, Y))
+        refs.append((t, s, X, i))
+    return items, refs
+
+
+SHAPES_M = [(37, 384), (200, 640), (3072, 1024), (1024, 3072), (4096, 12288), (24576, 4096)]
+
+
+@pytest.mark.parametrize("M", [2, 4, 7, 8, 9, 16])
+@pytest.mark.parametrize("mode", ["bf16", "int8"])
+def test_gemm_batch_small_m_matches_oracle(mode, M):
+    """Every token row of every item: int8 bit-exact, bf16 within the tolerance (sampled rows of
+    the large matrices); rows of Y beyond N and tokens beyond M are never written."""
+    act = tg.TERN_ACT_BF16 if mode == "bf16" else tg.TERN_ACT_INT8
+    items, refs = _build_m(81 + M, SHAPES_M, M, act)
+    tg.GemvBatch(items, act, M=M)()
+    torch.cuda.synchronize()
+    assert tg.tern_device_status() == tg.TERN_OK
+    for (W, xin, sxin, Y), (t, s, X, i) in zip(items, refs):
+        N, K = W.N, W.K
+        rows = _rows(N, i)
+        tr = t[rows] if t is not None else synth.trits(81 + M, 300 + i, N, K, rows=rows)
+        yy = host(Y).reshape(M, N)[:, rows]
+        if mode == "bf16":
+            check_bf16(yy, oracle.gemm_bf16(oracle.pack(tr), s[rows], K, X), X, s[rows])
+        else:
+            q, sx = host(xin).reshape(M, K), host(sxin)
+            _, y_ref = oracle.gemm_i8(oracle.pack(tr), s[rows], K, q, sx)
+            assert (yy == y_ref).all(), (N, K, M)
+
+
+def test_gemm_batch_int8_equals_small_m_entry():
+    """The batched small-M path and tern_gemm_small_m agree bit for bit in int8 mode."""
+    M = 7
+    items, _ = _build_m(90, [(6144, 4096), (4096, 12288)], M, tg.TERN_ACT_INT8)
+    tg.GemvBatch(items, tg.TERN_ACT_INT8, M=M)()
+    for W, q, sx, Y in items:
+        Y1 = torch.empty_like(Y)
+        tg.tern_gemm_small_m(W, M, tg.TERN_ACT_INT8, q, sx, Y1)
+        assert (host(Y1).view(np.uint32) == host(Y).view(np.uint32)).all()
