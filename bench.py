@@ -522,13 +522,22 @@ def _profile_head(mode):
     return run
 
 
+def _profile_prefill(proj):
+    def run():
+        ps = PrefillSet(M=4096, projs=(proj,))
+        return ps.launch
+    return run
+
+
 # Small cases for ncu captures (inputs > L2, a few hundred MB on the device):
 #   batch-8b-4layers-*: 4 layers of the 8B stack (16 fused GEMVs, 193 MB of planes) as one batch
 #   head-8b-*:          the int8 head 151936 x 4096 (622 MB)
+#   prefill-8b-gate-*:  one 12288 x 4096 linear at M = 4096 tokens (tcgen05 prefill)
 PROFILE_CASES = {
     "batch-8b-4layers-bf16": _profile_batch("bf16"),
     "batch-8b-4layers-int8": _profile_batch("int8"),
     "head-8b-bf16": _profile_head("bf16"),
+    "prefill-8b-gate-m4096": _profile_prefill("gate"),
 }
 
 
@@ -613,9 +622,57 @@ def extra_rows(stack, torch, tg, hbm_peak, bf16_peak):
         del g
     out["small_m_8b_bf16"] = sweep
 
+    # prefill: M = 4096 tokens through each of the 7 distinct 8B linear shapes (tcgen05)
+    out["prefill_8b_m4096"] = prefill_row(torch, tg, bf16_peak)
+
     # base-3 transport unpack of all 8B trits (bit-exact expansion into the planes)
     out["base3_unpack_8b"] = base3_row(stack, torch, tg, hbm_peak)
     return out
+
+
+class PrefillSet:
+    """The seven distinct 8B linear shapes (layer 0 weights) with M bf16 activation rows each."""
+
+    def __init__(self, M=4096, projs=("q", "k", "v", "o", "gate", "up", "down")):
+        import torch
+        import synth
+        self.M = M
+        self.lins = [build_linear("8b", 0, (p,)) for p in projs]
+        self.X = {}
+        for lin in self.lins:
+            if lin.K not in self.X:
+                self.X[lin.K] = torch.from_numpy(synth.activations(SEED, 6000 + lin.K, M, lin.K).view(np.int16)).cuda()
+        self.Y = [torch.empty(M * lin.N, dtype=torch.float32, device="cuda") for lin in self.lins]
+
+    @property
+    def flops(self):
+        return sum(2.0 * self.M * lin.N * lin.K for lin in self.lins)
+
+    def launch(self):
+        import bit_gemv_tern_b200 as tg
+        for lin, y in zip(self.lins, self.Y):
+            tg.tern_gemm_prefill(lin.W, self.M, self.X[lin.K], y)
+
+
+def prefill_row(torch, tg, bf16_peak):
+    ps = PrefillSet()
+    g = capture(lambda i: ps.launch(), 1)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    reps = 10
+    ms = timed_replays([(g, reps)]) / reps
+    tf = ps.flops / (ms / 1000.0) / 1e12
+    st = tg.tern_device_status()
+    per = {}
+    for lin, y in zip(ps.lins, ps.Y):
+        g1 = capture(lambda i, lin=lin, y=y: tg.tern_gemm_prefill(lin.W, ps.M, ps.X[lin.K], y), 1)
+        g1.replay()
+        m1 = timed_replays([(g1, reps)]) / reps
+        per["x".join(map(str, (lin.N, lin.K)))] = {"ms": m1, "tflops": 2.0 * ps.M * lin.N * lin.K / (m1 / 1000.0) / 1e12}
+    del ps
+    return {"ms_per_set": ms, "tflops": tf, "frac": tf / bf16_peak, "peak": "measured bf16 dense (burst)",
+            "flops_per_set": 1.5805e12, "status": st, "shapes": per}
 
 
 class StackView:

@@ -49,7 +49,7 @@ constexpr uint32_t kWaitTries = 1u << 13;
 constexpr int kSmemA = 0;
 constexpr int kSmemB = kStages * kABytes;
 constexpr int kSmemBar = kSmemB + kStages * kBBytes;
-constexpr int kSmemBytes = kSmemBar + 256 + 1024;  // + barriers, + slack for 1024-byte alignment
+constexpr int kSmemBytes = kSmemBar + 256 + kEpiWarps * BN * 4 + 1024;  // + barriers, scales, alignment slack
 
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator, A and B bf16, both
 // K-major, N = 256, M = 128.
@@ -88,9 +88,9 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 __device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
 }
-__device__ __forceinline__ uint2 ldg64(const void* p) {
-  uint2 v;
-  asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+__device__ __forceinline__ uint4 ldg128(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
   return v;
 }
 // K-major, 128-byte-swizzled operand descriptor (sm_100 layout): start address, leading byte
@@ -145,6 +145,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) k_prefill(const __grid_con
   const uint32_t a_full = sBar, b_full = sBar + 8 * kStages, empty = sBar + 16 * kStages;
   const uint32_t acc_full = sBar + 24 * kStages, acc_empty = acc_full + 16, done_bar = acc_empty + 16;
   const uint32_t tmem_slot = done_bar + 8;
+  const uint32_t sScale = sBar + 256;                 // [4 epilogue warps][BN] floats
   uint32_t* tmem_slot_ptr = reinterpret_cast<uint32_t*>(smem_raw + (tmem_slot - raw));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -237,21 +238,34 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) k_prefill(const __grid_con
         live[h] = n < p.N;
         rowp[h] = p.planes + (size_t)(live[h] ? n : 0) * KW;
       }
-      // words of the next stage, loaded one stage ahead
-      uint2 nm[2], ns[2];
+      // 16-byte loads of each plane cover two stages (a pair); pairs are loaded two pairs ahead
+      //   p0 = the pair being decoded, p1, p2 = the next two
+      uint4 pm[3][2], ps[3][2];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        nm[h] = live[h] ? ldg64(rowp[h]) : make_uint2(0u, 0u);
-        ns[h] = live[h] ? ldg64(rowp[h] + KW / 2) : make_uint2(0u, 0u);
-      }
+      for (int j = 0; j < 3; ++j)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const bool in = live[h] && 2 * j < KT;
+          pm[j][h] = in ? ldg128(rowp[h] + 4 * j) : make_uint4(0u, 0u, 0u, 0u);
+          ps[j][h] = in ? ldg128(rowp[h] + KW / 2 + 4 * j) : make_uint4(0u, 0u, 0u, 0u);
+        }
       for (int kt = 0; kt < KT; ++kt, ++q) {
         const int s = q % kStages;
-        uint2 cm[2] = {nm[0], nm[1]}, cs[2] = {ns[0], ns[1]};
-        if (kt + 1 < KT) {
+        uint2 cm[2], cs[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          cm[h] = (kt & 1) ? make_uint2(pm[0][h].z, pm[0][h].w) : make_uint2(pm[0][h].x, pm[0][h].y);
+          cs[h] = (kt & 1) ? make_uint2(ps[0][h].z, ps[0][h].w) : make_uint2(ps[0][h].x, ps[0][h].y);
+        }
+        if (kt & 1) {                                    // pair done: shift the queue, fetch pair + 3
+          const int j3 = (kt >> 1) + 3;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            nm[h] = live[h] ? ldg64(rowp[h] + 2 * (kt + 1)) : make_uint2(0u, 0u);
-            ns[h] = live[h] ? ldg64(rowp[h] + KW / 2 + 2 * (kt + 1)) : make_uint2(0u, 0u);
+            pm[0][h] = pm[1][h]; pm[1][h] = pm[2][h];
+            ps[0][h] = ps[1][h]; ps[1][h] = ps[2][h];
+            const bool in = live[h] && 2 * j3 < KT;
+            pm[2][h] = in ? ldg128(rowp[h] + 4 * j3) : make_uint4(0u, 0u, 0u, 0u);
+            ps[2][h] = in ? ldg128(rowp[h] + KW / 2 + 4 * j3) : make_uint4(0u, 0u, 0u, 0u);
           }
         }
         if (q >= kStages && !(ok = mbar_wait(empty + 8 * s, ((q / kStages) - 1) & 1))) break;
@@ -281,10 +295,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) k_prefill(const __grid_con
   } else {
     // ---------------- epilogue: TMEM -> registers -> 0.5 * scale -> Y ----------------
     const int quarter = warp & 3;                     // TMEM lanes 32*quarter .. +31
+    // this warp's copy of 0.5 * scale[n] for the tile's columns (no cross-warp barrier)
+    float* hs = reinterpret_cast<float*>(smem_raw + (sScale - raw)) + quarter * BN;
     int tl = 0;
     for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++tl) {
       const int mt = tile / tiles_n, nt = tile % tiles_n;
       const int acc = tl & 1;
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < BN / 32; ++i) {
+        const int n = nt * BN + lane + 32 * i;
+        hs[lane + 32 * i] = n < p.N ? 0.5f * f16_bits_to_float(p.scale[n]) : 0.0f;
+      }
+      __syncwarp();
       if (!(ok = mbar_wait(acc_full + 8 * acc, (tl >> 1) & 1))) break;
       tc_fence_after();
       const int m = mt * BM + quarter * 32 + lane;
@@ -294,20 +317,23 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) k_prefill(const __grid_con
         uint32_t r[32];
         tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN + 32 * c), r);
         const int n0 = nt * BN + 32 * c;
+        const float* sc = hs + 32 * c;
         if (m < p.M) {
           if (p.vec_store && n0 + 32 <= p.N) {
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
+              const float4 s4 = *reinterpret_cast<const float4*>(sc + j);
               float4 v;
-              v.x = __uint_as_float(r[j + 0]) * (0.5f * f16_bits_to_float(p.scale[n0 + j + 0]));
-              v.y = __uint_as_float(r[j + 1]) * (0.5f * f16_bits_to_float(p.scale[n0 + j + 1]));
-              v.z = __uint_as_float(r[j + 2]) * (0.5f * f16_bits_to_float(p.scale[n0 + j + 2]));
-              v.w = __uint_as_float(r[j + 3]) * (0.5f * f16_bits_to_float(p.scale[n0 + j + 3]));
+              v.x = __uint_as_float(r[j + 0]) * s4.x;
+              v.y = __uint_as_float(r[j + 1]) * s4.y;
+              v.z = __uint_as_float(r[j + 2]) * s4.z;
+              v.w = __uint_as_float(r[j + 3]) * s4.w;
               *reinterpret_cast<float4*>(yrow + n0 + j) = v;
             }
           } else {
-            for (int j = 0; j < 32 && n0 + j < p.N; ++j)
-              yrow[n0 + j] = __uint_as_float(r[j]) * (0.5f * f16_bits_to_float(p.scale[n0 + j]));
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (n0 + j < p.N) yrow[n0 + j] = __uint_as_float(r[j]) * sc[j];
           }
         }
       }
