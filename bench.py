@@ -33,6 +33,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "ternary GEMV HBM GB/s & 8B linear-stack tok/s at M=1 (fraction of HBM peak)"
+# DRAM bytes (read + write) of the stream kernel per full 8B step, from the ncu capture summarised
+# in profiles/k_batch_stream_8b_4layers_bf16.md (4 layers: 193.69 MB read + 4.74 MB written),
+# scaled by the units processed (36 / 4 layers). Set to None whenever that kernel changes.
+STREAM_TRAFFIC_PER_STEP = 9 * (193.69e6 + 4.74e6)
 SEED = 0x7E2A2026
 L2_BYTES = 126 * 1024 * 1024
 
@@ -492,7 +496,8 @@ def main():
             "hbm_frac_step": step_bytes / (ms_step / 1000.0) / 1e9 / hbm_peak,
             "roofline": {"bound": "hbm", "kernel": "k_batch_prep + k_batch_stream<bf16> (all 144 fused GEMVs of the step in one persistent launch)",
                          "achieved": gemv_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gemv_gbs / hbm_peak,
-                         "peak_kind": f"{peak_kind} hbm_gbs (copy)", "traffic": None,
+                         "peak_kind": f"{peak_kind} hbm_gbs (copy)", "traffic": STREAM_TRAFFIC_PER_STEP,
+                         "traffic_note": "dram read+write bytes per step, ncu capture of 4 layers x 9",
                          "algorithmic_bytes_per_step": stack.stack_bytes, "launches": n_linear,
                          "head": {"kernel": "k_head<bf16,1>", "achieved": head_gbs, "frac": head_gbs / hbm_peak}},
             "cpu_baseline": cb,
