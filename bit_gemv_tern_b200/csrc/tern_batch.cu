@@ -96,9 +96,17 @@ __device__ __forceinline__ int bsum(uint32_t w) { return __dp4a((int)w, 0x010101
 // 2^e as a double for |e| < 1000 (built from the exponent field: exact).
 __device__ __forceinline__ double exp2_i(int e) { return __longlong_as_double((long long)(e + 1023) << 52); }
 
-// Operand slot of 16-byte half h of word w (0..15) of a 512-trit part: lane t = w / 4 reads the
-// eight words of its word e = w % 4 at ((e * 4) + t) * 8, so a quarter-warp's loads hit distinct banks.
-__device__ __forceinline__ int part_slot(int w, int h) { return ((w & 3) * 4 + (w >> 2)) * 8 + 4 * h; }
+// Operand words of word w (0..15) of a 512-trit part: lane t = w / 4 reads the eight words of its
+// word e = w % 4 at ((e * 4) + t) * 8 (so a quarter-warp's loads hit distinct banks), ordered
+// (field 0: b0, b1), (field 1: b0, b1), ...: each tensor-core B register pair is two adjacent
+// words of one 128-bit load. b0 / b1 come from 16-byte half h = 0 / 1 of the permuted activation.
+__device__ __forceinline__ int part_slot(int w) { return ((w & 3) * 4 + (w >> 2)) * 8; }
+__device__ __forceinline__ void store_operand_half(uint32_t* slot, int h, uint4 v) {
+  slot[0 + h] = v.x;
+  slot[2 + h] = v.y;
+  slot[4 + h] = v.z;
+  slot[6 + h] = v.w;
+}
 
 // ---------------------------------------------------------------------------------------------
 // Operand columns of a segment. M = 1 (mp == 1): the nc columns are the limbs L2, L1, L0 (bf16
@@ -167,11 +175,11 @@ __global__ void __launch_bounds__(256) k_batch_prep(const __grid_constant__ Batc
   for (int v = threadIdx.x; live && v < K / 16; v += blockDim.x) {
     const int word = v >> 1, h = v & 1;              // global word index and half
     const int part = word >> 4, w = word & 15;
-    uint32_t* seg = blk + part * segw + part_slot(w, h);
+    uint32_t* seg = blk + part * segw + part_slot(w);
     if (p.mode == 1) {
       const uint4 q = ld_nc(static_cast<const int8_t*>(it.x) + (size_t)m * K + 16 * v);
       ls[0] += bsum(q.x) + bsum(q.y) + bsum(q.z) + bsum(q.w);
-      *reinterpret_cast<uint4*>(seg + colof[0] * kColWords) = permute_i8_half(q);
+      store_operand_half(seg + colof[0] * kColWords, h, permute_i8_half(q));
     } else {
       const uint16_t* xb = static_cast<const uint16_t*>(it.x) + (size_t)m * K + 16 * v;
       const uint4 a = ld_nc(xb), b = ld_nc(xb + 8);
@@ -193,8 +201,7 @@ __global__ void __launch_bounds__(256) k_batch_prep(const __grid_constant__ Batc
 #pragma unroll
       for (int c = 0; c < 3; ++c) {
         ls[c] += bsum(l[c][0]) + bsum(l[c][1]) + bsum(l[c][2]) + bsum(l[c][3]);
-        *reinterpret_cast<uint4*>(seg + colof[c] * kColWords) =
-            permute_i8_half(make_uint4(l[c][0], l[c][1], l[c][2], l[c][3]));
+        store_operand_half(seg + colof[c] * kColWords, h, permute_i8_half(make_uint4(l[c][0], l[c][1], l[c][2], l[c][3])));
       }
     }
   }
@@ -405,13 +412,16 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
         }
 #pragma unroll
         for (int j = 0; j < G; ++j) {
-          const uint4 x0 = lds128(st + xofs + (j * 8 * kColWords) * 4 + e * 128);
-          const uint4 x1 = lds128(st + xofs + (j * 8 * kColWords) * 4 + e * 128 + 16);
+          // (b0, b1) of fields 0, 1 and of fields 2, 3
+          const uint4 x01 = lds128(st + xofs + (j * 8 * kColWords) * 4 + e * 128);
+          const uint4 x23 = lds128(st + xofs + (j * 8 * kColWords) * 4 + e * 128 + 16);
 #pragma unroll
           for (int a = 0; a < TPW; ++a)
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-              mma_u8s8(acc[a][j][i], A[a][i][0], A[a][i][1], A[a][i][2], A[a][i][3], u4get(x0, i), u4get(x1, i));
+              mma_u8s8(acc[a][j][i], A[a][i][0], A[a][i][1], A[a][i][2], A[a][i][3],
+                       i < 2 ? u4get(x01, 2 * i) : u4get(x23, 2 * i - 4),
+                       i < 2 ? u4get(x01, 2 * i + 1) : u4get(x23, 2 * i - 3));
         }
       }
       if (part == KP - 1) {                                  // sums over all of K and E ride in every segment

@@ -67,36 +67,84 @@ __device__ __forceinline__ void build_base3_lut(uint16_t* lut) {
   }
 }
 
-// One thread per 32-trit word of the output: decodes the 7 or 8 transport bytes that cover it.
-__global__ void k_unpack_base3(const uint8_t* __restrict__ src, int64_t n_words, int32_t KM, int32_t row_bytes,
-                               uint32_t* __restrict__ planes, int32_t* __restrict__ flag) {
-  __shared__ uint16_t lut[256];
+// Natural-order bits -> the layout's order: bit j moves to p(j), which swaps bits 0 and 4 of
+// the index j (one delta swap: positions with j0 = 1, j4 = 0 trade places with j + 15).
+__device__ __forceinline__ uint32_t to_mask_order(uint32_t x) {
+  const uint32_t t = ((x >> 15) ^ x) & 0x0000AAAAu;
+  return x ^ t ^ (t << 15);
+}
+
+constexpr int kB3Threads = 256;
+constexpr int kB3StageBytes = 8 * 1024;           // transport bytes staged per CTA (whole rows)
+constexpr int kB3Slack = 64;                      // read slack after the staged bytes
+
+// A CTA stages a block of whole transport rows (contiguous bytes) in shared memory with 16-byte
+// loads, then each thread decodes runs of 32 bytes = 160 trits = 5 output words: a table turns
+// each byte into its five mask and five sign bits in natural order, the bits are gathered per
+// 32-trit word and moved to the layout's bit order.
+__global__ void __launch_bounds__(kB3Threads) k_unpack_base3(const uint8_t* __restrict__ src, int32_t N, int32_t KW,
+                                                             int32_t rb, int32_t rows_per_cta, int32_t aligned16,
+                                                             uint32_t* __restrict__ planes, int32_t* __restrict__ flag) {
+  extern __shared__ uint4 b3_smem[];
+  uint16_t* lut = reinterpret_cast<uint16_t*>(b3_smem);
+  uint8_t* bytes = reinterpret_cast<uint8_t*>(b3_smem) + 512;
   build_base3_lut(lut);
+  const int r0 = blockIdx.x * rows_per_cta;
+  const int r1 = min(N, r0 + rows_per_cta);
+  const int64_t g0 = (int64_t)r0 * rb, g1 = (int64_t)r1 * rb;   // this block's bytes
+  const int64_t total = (int64_t)N * rb;
+  const int64_t a0 = aligned16 ? (g0 & ~(int64_t)15) : g0;
+  int64_t a1 = aligned16 ? min((g1 + 15) & ~(int64_t)15, total & ~(int64_t)15) : g0;
+  if (a1 < a0) a1 = a0;
+  for (int64_t o = a0 + 16 * (int64_t)threadIdx.x; o + 16 <= a1; o += 16 * (int64_t)blockDim.x)
+    *reinterpret_cast<uint4*>(bytes + (o - a0)) = ld_stream(src + o);
+  for (int64_t o = max(a1, g0) + threadIdx.x; o < g1; o += blockDim.x) bytes[o - a0] = src[o];
   __syncthreads();
+  const int rpr = (KW + 4) / 5;                    // runs per row
+  const int nruns = (r1 - r0) * rpr;
   bool bad = false;
-  for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < n_words;
-       w += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t row = w / KM;
-    const int col = (int)(w % KM);
-    const uint8_t* rp = src + row * (int64_t)row_bytes;
-    const int k_begin = col * 32;
-    uint32_t m = 0, s = 0;
-    for (int j = k_begin / 5; j <= (k_begin + 31) / 5; ++j) {
-      const uint32_t e = lut[__ldg(rp + j)];
-      bad |= (e == 0xFFFFu);
+  for (int g = threadIdx.x; g < nruns; g += blockDim.x) {
+    const int rr = g / rpr, i = g - rr * rpr;
+    const int row = r0 + rr;
+    const int off = (int)((int64_t)row * rb - a0) + 32 * i;     // run start in the staged bytes
+    const int nb = min(32, rb - 32 * i);                        // bytes of the run inside the row
+    const uint32_t* wp = reinterpret_cast<const uint32_t*>(bytes + (off & ~3));
+    const uint32_t sh = 8u * (uint32_t)(off & 3);
+    uint32_t by[8];
+    {
+      uint32_t prev = wp[0];
 #pragma unroll
-      for (int i = 0; i < 5; ++i) {
-        const int k = 5 * j + i - k_begin;
-        if (k >= 0 && k < 32) {
-          const int p_m = mask_pos(k);
-          m |= ((e >> i) & 1u) << p_m;
-          s |= ((e >> (5 + i)) & 1u) << ((p_m + 1) & 31);
-        }
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t next = wp[k + 1];
+        by[k] = __funnelshift_r(prev, next, sh);
+        prev = next;
       }
     }
-    uint32_t* row_p = planes + row * (2 * (int64_t)KM);
-    row_p[col] = m;
-    row_p[KM + col] = s;
+    uint32_t m[6] = {0u, 0u, 0u, 0u, 0u, 0u}, s[6] = {0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const uint32_t e = lut[(by[j >> 2] >> (8 * (j & 3))) & 0xFFu];
+      const bool in = j < nb;
+      bad |= in && e == 0xFFFFu;
+      const uint32_t mm = in ? (e & 31u) : 0u, ss = in ? ((e >> 5) & 31u) : 0u;
+      const int w = (5 * j) >> 5, o = (5 * j) & 31;
+      m[w] |= mm << o;
+      s[w] |= ss << o;
+      if (o > 27) {
+        m[w + 1] |= mm >> (32 - o);
+        s[w + 1] |= ss >> (32 - o);
+      }
+    }
+    uint32_t* rowp = planes + (size_t)row * 2 * KW;
+#pragma unroll
+    for (int u = 0; u < 5; ++u) {
+      const int w = 5 * i + u;
+      if (w < KW) {
+        rowp[w] = to_mask_order(m[u]);
+        const uint32_t sp = to_mask_order(s[u]);
+        rowp[KW + w] = (sp << 1) | (sp >> 31);                 // sign bit sits one above its mask bit
+      }
+    }
   }
   if (__any_sync(0xFFFFFFFFu, bad) && (threadIdx.x & 31) == 0) set_flag(flag);
 }
@@ -168,8 +216,19 @@ cudaError_t launch_pack_trits(const int8_t* src, int32_t N, int32_t K, uint32_t*
 
 cudaError_t launch_unpack_base3(const uint8_t* src, int32_t N, int32_t K, uint32_t* planes, int32_t* flag,
                                 cudaStream_t st) {
-  const int64_t n_words = (int64_t)N * (K / 32);
-  k_unpack_base3<<<grid_for(n_words, 256), 256, 0, st>>>(src, n_words, K / 32, (K + 4) / 5, planes, flag);
+  const int rb = (K + 4) / 5;
+  int rows = kB3StageBytes / rb;
+  if (rows < 1) rows = 1;
+  const int grid = (N + rows - 1) / rows;
+  const size_t smem = 512 + (size_t)rows * rb + 16 + kB3Slack;
+  static size_t set = 0;
+  if (smem > 48 * 1024 && smem > set) {
+    cudaError_t e = cudaFuncSetAttribute(k_unpack_base3, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    set = smem;
+  }
+  const int al = (reinterpret_cast<uintptr_t>(src) & 15) == 0 ? 1 : 0;
+  k_unpack_base3<<<grid, kB3Threads, smem, st>>>(src, N, K / 32, rb, rows, al, planes, flag);
   return cudaGetLastError();
 }
 
