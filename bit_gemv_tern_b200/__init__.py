@@ -18,7 +18,7 @@ import os
 __all__ = [
     "TernError", "TernMatrix", "lib", "library_path",
     "TERN_ACT_BF16", "TERN_ACT_INT8", "TERN_SRC_INT8_TRITS", "TERN_SRC_BASE3", "TERN_FLAG_PDL",
-    "tern_packed_bytes", "tern_base3_bytes", "tern_pack", "tern_base3_encode", "tern_occupancy",
+    "tern_packed_bytes", "tern_base3_bytes", "tern_pack", "tern_pack_batch", "tern_base3_encode", "tern_occupancy",
     "tern_quantize_act", "tern_gemv", "tern_gemm_small_m", "tern_gemm_prefill",
     "i8_head_workspace_bytes", "i8_head_gemv_argmax", "i8_head_gemv_argmax_noalloc",
     "TERN_HEAD_NOALLOC_MAX_M", "tern_read_flag", "tern_device_status",
@@ -64,6 +64,7 @@ def lib() -> ctypes.CDLL:
             "tern_base3_bytes": ([i32, i32], sz),
             "tern_pack": ([i32, vp, i32, i32, vp, vp, vp], i32),
             "tern_base3_encode": ([vp, i32, i32, vp, vp, vp], i32),
+            "tern_pack_batch": ([i32, vp, i32, vp, vp], i32),
             "tern_occupancy": ([mp, vp, vp], i32),
             "tern_quantize_act": ([vp, i32, i32, vp, vp, vp], i32),
             "tern_gemv": ([mp, i32, vp, vp, vp, vp], i32),
@@ -144,6 +145,19 @@ def tern_pack(src_kind: int, src, N: int, K: int, planes, err_flag, stream=None)
     """Pack dense int8 trits (src_kind=TERN_SRC_INT8_TRITS) or the base-3 transport
     (TERN_SRC_BASE3) into planes; invalid input values set err_flag (see tern_read_flag)."""
     _check(lib().tern_pack(src_kind, _ptr(src), N, K, _ptr(planes), _ptr(err_flag), _stream(stream)), "tern_pack")
+
+
+class _PackItem(ctypes.Structure):
+    _fields_ = [("src_dev", ctypes.c_void_p), ("N", ctypes.c_int32), ("K", ctypes.c_int32),
+                ("planes_dev", ctypes.c_void_p)]
+
+
+def tern_pack_batch(src_kind: int, entries, err_flag, stream=None) -> None:
+    """tern_pack over a list of (src, N, K, planes) in one call (one flag clear; one launch for base-3)."""
+    arr = (_PackItem * len(entries))()
+    for i, (src, N, K, planes) in enumerate(entries):
+        arr[i].src_dev, arr[i].N, arr[i].K, arr[i].planes_dev = _ptr(src), int(N), int(K), _ptr(planes)
+    _check(lib().tern_pack_batch(src_kind, arr, len(entries), _ptr(err_flag), _stream(stream)), "tern_pack_batch")
 
 
 def tern_base3_encode(trits, N: int, K: int, out, err_flag, stream=None) -> None:

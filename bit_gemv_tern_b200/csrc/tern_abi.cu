@@ -74,12 +74,47 @@ tern_status tern_pack(tern_src src, const void* src_dev, int32_t N, int32_t K, u
   if (!valid_shape(N, K)) return TERN_ESHAPE;
   if (!aligned(planes_dev, 16) || !aligned(err_flag_dev, 4)) return TERN_EINVAL;
   if (src == TERN_SRC_INT8_TRITS && !aligned(src_dev, 16)) return TERN_EINVAL;
+  if (src == TERN_SRC_BASE3 && !aligned(src_dev, 4)) return TERN_EINVAL;
   cudaError_t e = cudaMemsetAsync(err_flag_dev, 0, sizeof(int32_t), cs(stream));
   if (e != cudaSuccess) return TERN_ECUDA;
   if (src == TERN_SRC_INT8_TRITS)
     e = tern::launch_pack_trits(static_cast<const int8_t*>(src_dev), N, K, planes_dev, err_flag_dev, cs(stream));
   else
     e = tern::launch_unpack_base3(static_cast<const uint8_t*>(src_dev), N, K, planes_dev, err_flag_dev, cs(stream));
+  return from_cuda(e);
+}
+
+tern_status tern_pack_batch(tern_src src, const tern_pack_item* items, int32_t count, int32_t* err_flag_dev,
+                            tern_stream_t stream) {
+  if (!items || !err_flag_dev) return TERN_EINVAL;
+  if (src != TERN_SRC_INT8_TRITS && src != TERN_SRC_BASE3) return TERN_EINVAL;
+  if (count < 1 || count > TERN_PACK_MAX_ITEMS) return TERN_ESHAPE;
+  if (!aligned(err_flag_dev, 4)) return TERN_EINVAL;
+  for (int i = 0; i < count; ++i) {
+    const tern_pack_item& it = items[i];
+    if (!it.src_dev || !it.planes_dev) return TERN_EINVAL;
+    if (!valid_shape(it.N, it.K)) return TERN_ESHAPE;
+    if (!aligned(it.planes_dev, 16) || !aligned(it.src_dev, src == TERN_SRC_BASE3 ? 4 : 16)) return TERN_EINVAL;
+  }
+  cudaError_t e = cudaMemsetAsync(err_flag_dev, 0, sizeof(int32_t), cs(stream));
+  if (e != cudaSuccess) return TERN_ECUDA;
+  if (src == TERN_SRC_INT8_TRITS) {
+    for (int i = 0; i < count && e == cudaSuccess; ++i)
+      e = tern::launch_pack_trits(static_cast<const int8_t*>(items[i].src_dev), items[i].N, items[i].K,
+                                  items[i].planes_dev, err_flag_dev, cs(stream));
+    return from_cuda(e);
+  }
+  tern::Base3Batch* b = new (std::nothrow) tern::Base3Batch();
+  if (!b) return TERN_EINVAL;
+  b->count = count;
+  for (int i = 0; i < count; ++i) {
+    b->src[i] = static_cast<const uint8_t*>(items[i].src_dev);
+    b->planes[i] = items[i].planes_dev;
+    b->N[i] = items[i].N;
+    b->K[i] = items[i].K;
+  }
+  e = tern::launch_unpack_base3_batch(*b, err_flag_dev, cs(stream));
+  delete b;
   return from_cuda(e);
 }
 

@@ -120,6 +120,16 @@ size_t head_smem_bytes(int mode, int M, int kr);
 cudaError_t launch_head(const HeadParams& p, bool pdl, cudaStream_t st);
 
 // Loader kernels (tern_pack.cu).
+constexpr int kPackMaxItems = 256;
+struct Base3Batch {
+  const uint8_t* src[kPackMaxItems];
+  uint32_t* planes[kPackMaxItems];
+  int32_t N[kPackMaxItems], K[kPackMaxItems];
+  int32_t rows[kPackMaxItems];     // rows per CTA (set by the launcher)
+  int32_t block0[kPackMaxItems];   // first CTA of each item (set by the launcher)
+  int32_t count;
+};
+cudaError_t launch_unpack_base3_batch(Base3Batch& p, int32_t* flag, cudaStream_t st);
 cudaError_t launch_pack_trits(const int8_t* src, int32_t N, int32_t K, uint32_t* planes, int32_t* flag,
                               cudaStream_t st);
 cudaError_t launch_unpack_base3(const uint8_t* src, int32_t N, int32_t K, uint32_t* planes, int32_t* flag,

@@ -75,59 +75,74 @@ __device__ __forceinline__ uint32_t to_mask_order(uint32_t x) {
 }
 
 constexpr int kB3Threads = 256;
-constexpr int kB3StageBytes = 8 * 1024;           // transport bytes staged per CTA (whole rows)
-constexpr int kB3Slack = 64;                      // read slack after the staged bytes
+constexpr int kB3StageBytes = 8 * 1024;           // transport bytes per CTA (whole rows)
+constexpr int kB3Slot = 48;                       // shared-memory bytes per 32-byte run
 
-// A CTA stages a block of whole transport rows (contiguous bytes) in shared memory with 16-byte
-// loads, then each thread decodes runs of 32 bytes = 160 trits = 5 output words: a table turns
-// each byte into its five mask and five sign bits in natural order, the bits are gathered per
-// 32-trit word and moved to the layout's bit order.
-__global__ void __launch_bounds__(kB3Threads) k_unpack_base3(const uint8_t* __restrict__ src, int32_t N, int32_t KW,
-                                                             int32_t rb, int32_t rows_per_cta, int32_t aligned16,
-                                                             uint32_t* __restrict__ planes, int32_t* __restrict__ flag) {
-  extern __shared__ uint4 b3_smem[];
-  uint16_t* lut = reinterpret_cast<uint16_t*>(b3_smem);
-  uint8_t* bytes = reinterpret_cast<uint8_t*>(b3_smem) + 512;
-  build_base3_lut(lut);
-  const int r0 = blockIdx.x * rows_per_cta;
-  const int r1 = min(N, r0 + rows_per_cta);
-  const int64_t g0 = (int64_t)r0 * rb, g1 = (int64_t)r1 * rb;   // this block's bytes
-  const int64_t total = (int64_t)N * rb;
-  const int64_t a0 = aligned16 ? (g0 & ~(int64_t)15) : g0;
-  int64_t a1 = aligned16 ? min((g1 + 15) & ~(int64_t)15, total & ~(int64_t)15) : g0;
-  if (a1 < a0) a1 = a0;
-  for (int64_t o = a0 + 16 * (int64_t)threadIdx.x; o + 16 <= a1; o += 16 * (int64_t)blockDim.x)
-    *reinterpret_cast<uint4*>(bytes + (o - a0)) = ld_stream(src + o);
-  for (int64_t o = max(a1, g0) + threadIdx.x; o < g1; o += blockDim.x) bytes[o - a0] = src[o];
-  __syncthreads();
+// One CTA per block of whole transport rows, three phases:
+//   1. copy: run j (32 bytes = 160 trits = 5 output words) of the block goes to its own 48-byte
+//      slot, so that phase 2's two 16-byte reads per lane hit distinct banks;
+//   2. decode: a table turns each byte into its five mask and five sign bits in natural order;
+//      the bits are gathered per 32-trit word, moved to the layout's bit order and written to a
+//      shared-memory copy of the block's output rows;
+//   3. write-out: the block's rows are contiguous in the planes, copied with 16-byte stores.
+__device__ __forceinline__ void unpack_base3_block(const uint8_t* __restrict__ src, int32_t N, int32_t KW, int32_t rb,
+                                                   int32_t rows_per_cta, int32_t block, uint32_t* __restrict__ planes,
+                                                   int32_t* __restrict__ flag, uint4* b3_smem) {
+  const int r0 = block * rows_per_cta;
+  const int nrow = min(N - r0, rows_per_cta);
   const int rpr = (KW + 4) / 5;                    // runs per row
-  const int nruns = (r1 - r0) * rpr;
-  bool bad = false;
-  for (int g = threadIdx.x; g < nruns; g += blockDim.x) {
-    const int rr = g / rpr, i = g - rr * rpr;
-    const int row = r0 + rr;
-    const int off = (int)((int64_t)row * rb - a0) + 32 * i;     // run start in the staged bytes
-    const int nb = min(32, rb - 32 * i);                        // bytes of the run inside the row
-    const uint32_t* wp = reinterpret_cast<const uint32_t*>(bytes + (off & ~3));
-    const uint32_t sh = 8u * (uint32_t)(off & 3);
-    uint32_t by[8];
-    {
-      uint32_t prev = wp[0];
+  const int nruns = nrow * rpr;
+  uint16_t* lut = reinterpret_cast<uint16_t*>(b3_smem);
+  uint8_t* runs = reinterpret_cast<uint8_t*>(b3_smem) + 512;
+  uint32_t* outw = reinterpret_cast<uint32_t*>(runs + (size_t)rows_per_cta * rpr * kB3Slot);
+  build_base3_lut(lut);
+  const int64_t total = (int64_t)N * rb;
+  // 1. copy: half-runs of 16 bytes, each from five aligned words of the transport
+  for (int hr = threadIdx.x; hr < 2 * nruns; hr += blockDim.x) {
+    const int j = hr >> 1, h = hr & 1;
+    const int rr = j / rpr, i = j - rr * rpr;
+    const int pos = 32 * i + 16 * h;              // byte position in the row
+    const int64_t g = (int64_t)(r0 + rr) * rb + pos;
+    const int64_t ga = g & ~(int64_t)3;
+    const uint32_t sh = 8u * (uint32_t)(g & 3);
+    uint32_t w[5];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const uint32_t next = wp[k + 1];
-        by[k] = __funnelshift_r(prev, next, sh);
-        prev = next;
+    for (int k = 0; k < 5; ++k) {
+      const int64_t a = ga + 4 * k;
+      if (a + 4 <= total) {
+        w[k] = __ldg(reinterpret_cast<const uint32_t*>(src + a));
+      } else {                                    // the buffer's last, partial word: byte by byte
+        uint32_t x = 0u;
+        for (int t = 0; t < 4; ++t)
+          if (a + t < total) x |= (uint32_t)__ldg(src + a + t) << (8 * t);
+        w[k] = x;
       }
     }
+    // bytes past the row's end belong to the next row: never decoded into an output word
+    uint4 v;
+    v.x = __funnelshift_r(w[0], w[1], sh);
+    v.y = __funnelshift_r(w[1], w[2], sh);
+    v.z = __funnelshift_r(w[2], w[3], sh);
+    v.w = __funnelshift_r(w[3], w[4], sh);
+    *reinterpret_cast<uint4*>(runs + (size_t)j * kB3Slot + 16 * h) = v;
+  }
+  __syncthreads();
+  // 2. decode
+  bool bad = false;
+  for (int j = threadIdx.x; j < nruns; j += blockDim.x) {
+    const int rr = j / rpr, i = j - rr * rpr;
+    const int nb = min(32, rb - 32 * i);          // bytes of the run inside the row
+    const uint4 lo = *reinterpret_cast<const uint4*>(runs + (size_t)j * kB3Slot);
+    const uint4 hi = *reinterpret_cast<const uint4*>(runs + (size_t)j * kB3Slot + 16);
+    const uint32_t by[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
     uint32_t m[6] = {0u, 0u, 0u, 0u, 0u, 0u}, s[6] = {0u, 0u, 0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const uint32_t e = lut[(by[j >> 2] >> (8 * (j & 3))) & 0xFFu];
-      const bool in = j < nb;
+    for (int b = 0; b < 32; ++b) {
+      const uint32_t e = lut[(by[b >> 2] >> (8 * (b & 3))) & 0xFFu];
+      const bool in = b < nb;
       bad |= in && e == 0xFFFFu;
       const uint32_t mm = in ? (e & 31u) : 0u, ss = in ? ((e >> 5) & 31u) : 0u;
-      const int w = (5 * j) >> 5, o = (5 * j) & 31;
+      const int w = (5 * b) >> 5, o = (5 * b) & 31;
       m[w] |= mm << o;
       s[w] |= ss << o;
       if (o > 27) {
@@ -135,18 +150,45 @@ __global__ void __launch_bounds__(kB3Threads) k_unpack_base3(const uint8_t* __re
         s[w + 1] |= ss >> (32 - o);
       }
     }
-    uint32_t* rowp = planes + (size_t)row * 2 * KW;
+    uint32_t* rowo = outw + (size_t)rr * 2 * KW;
 #pragma unroll
     for (int u = 0; u < 5; ++u) {
       const int w = 5 * i + u;
       if (w < KW) {
-        rowp[w] = to_mask_order(m[u]);
+        rowo[w] = to_mask_order(m[u]);
         const uint32_t sp = to_mask_order(s[u]);
-        rowp[KW + w] = (sp << 1) | (sp >> 31);                 // sign bit sits one above its mask bit
+        rowo[KW + w] = (sp << 1) | (sp >> 31);     // the sign bit sits one above its mask bit
       }
     }
   }
   if (__any_sync(0xFFFFFFFFu, bad) && (threadIdx.x & 31) == 0) set_flag(flag);
+  __syncthreads();
+  // 3. write-out: nrow rows x 2*KW words, contiguous in the planes (KW % 4 == 0)
+  const int nvec = nrow * 2 * KW / 4;
+  uint4* dst = reinterpret_cast<uint4*>(planes + (size_t)r0 * 2 * KW);
+  const uint4* from = reinterpret_cast<const uint4*>(outw);
+  for (int v = threadIdx.x; v < nvec; v += blockDim.x) dst[v] = from[v];
+}
+
+__global__ void __launch_bounds__(kB3Threads) k_unpack_base3(const uint8_t* __restrict__ src, int32_t N, int32_t KW,
+                                                             int32_t rb, int32_t rows_per_cta,
+                                                             uint32_t* __restrict__ planes, int32_t* __restrict__ flag) {
+  extern __shared__ uint4 b3_smem[];
+  unpack_base3_block(src, N, KW, rb, rows_per_cta, blockIdx.x, planes, flag, b3_smem);
+}
+
+// Many tensors in one launch: CTA b belongs to the item whose block range holds b.
+__global__ void __launch_bounds__(kB3Threads) k_unpack_base3_batch(const __grid_constant__ Base3Batch p,
+                                                                   int32_t* __restrict__ flag) {
+  extern __shared__ uint4 b3_smem[];
+  int lo = 0, hi = p.count - 1;
+  while (lo < hi) {                                // last item with block0 <= blockIdx.x
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.block0[mid] <= (int)blockIdx.x) lo = mid; else hi = mid - 1;
+  }
+  const int K = p.K[lo];
+  unpack_base3_block(p.src[lo], p.N[lo], K / 32, (K + 4) / 5, p.rows[lo], (int)blockIdx.x - p.block0[lo], p.planes[lo],
+                     flag, b3_smem);
 }
 
 // One thread per transport byte.
@@ -214,21 +256,52 @@ cudaError_t launch_pack_trits(const int8_t* src, int32_t N, int32_t K, uint32_t*
   return cudaGetLastError();
 }
 
-cudaError_t launch_unpack_base3(const uint8_t* src, int32_t N, int32_t K, uint32_t* planes, int32_t* flag,
-                                cudaStream_t st) {
-  const int rb = (K + 4) / 5;
-  int rows = kB3StageBytes / rb;
+void base3_plan(int32_t K, int& rows, size_t& smem) {
+  const int rb = (K + 4) / 5, KW = K / 32, rpr = (KW + 4) / 5;
+  rows = kB3StageBytes / rb;
   if (rows < 1) rows = 1;
-  const int grid = (N + rows - 1) / rows;
-  const size_t smem = 512 + (size_t)rows * rb + 16 + kB3Slack;
-  static size_t set = 0;
+  smem = 512 + (size_t)rows * rpr * kB3Slot + (size_t)rows * K / 4;
+}
+
+cudaError_t base3_smem_attr(const void* fn, size_t smem, size_t& set) {
   if (smem > 48 * 1024 && smem > set) {
-    cudaError_t e = cudaFuncSetAttribute(k_unpack_base3, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     set = smem;
   }
-  const int al = (reinterpret_cast<uintptr_t>(src) & 15) == 0 ? 1 : 0;
-  k_unpack_base3<<<grid, kB3Threads, smem, st>>>(src, N, K / 32, rb, rows, al, planes, flag);
+  return cudaSuccess;
+}
+
+cudaError_t launch_unpack_base3(const uint8_t* src, int32_t N, int32_t K, uint32_t* planes, int32_t* flag,
+                                cudaStream_t st) {
+  int rows = 1;
+  size_t smem = 0;
+  base3_plan(K, rows, smem);
+  const int grid = (N + rows - 1) / rows;
+  static size_t set = 0;
+  cudaError_t e = base3_smem_attr(reinterpret_cast<const void*>(k_unpack_base3), smem, set);
+  if (e != cudaSuccess) return e;
+  k_unpack_base3<<<grid, kB3Threads, smem, st>>>(src, N, K / 32, (K + 4) / 5, rows, planes, flag);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpack_base3_batch(Base3Batch& p, int32_t* flag, cudaStream_t st) {
+  size_t smem = 0;
+  int64_t blocks = 0;
+  for (int i = 0; i < p.count; ++i) {
+    int rows = 1;
+    size_t sm = 0;
+    base3_plan(p.K[i], rows, sm);
+    p.rows[i] = rows;
+    p.block0[i] = (int32_t)blocks;
+    blocks += (p.N[i] + rows - 1) / rows;
+    if (sm > smem) smem = sm;
+  }
+  if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  static size_t set = 0;
+  cudaError_t e = base3_smem_attr(reinterpret_cast<const void*>(k_unpack_base3_batch), smem, set);
+  if (e != cudaSuccess) return e;
+  k_unpack_base3_batch<<<(unsigned)blocks, kB3Threads, smem, st>>>(p, flag);
   return cudaGetLastError();
 }
 

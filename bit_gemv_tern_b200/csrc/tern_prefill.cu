@@ -14,9 +14,9 @@
 //   warp 1      allocates 512 TMEM columns (two fp32 accumulators of 128 x 256) and one lane
 //               issues tcgen05.mma kind::f16 (A = X tile, B = expanded weights, both K-major);
 //               tcgen05.commit frees a stage when the MMAs reading it are done;
-//   warps 2..5  expand the tile's 256 weight rows x 64 trits to bf16 (2.0 * t, the field decode
+//   warps 2..9  expand the tile's 256 weight rows x 64 trits to bf16 (2.0 * t, the field decode
 //               of tern_device.cuh) in the same swizzled layout the tensor core reads;
-//   warps 6..9  epilogue: tcgen05.ld of the accumulator their TMEM lane quarter owns, times
+//   warps 10..13 epilogue: tcgen05.ld of the accumulator their TMEM lane quarter owns, times
 //               0.5 * scale[n], stored to Y; the second accumulator lets the next tile's MMAs run
 //               meanwhile.
 // Every mbarrier wait is bounded; a kernel that gives up latches TERN_ETIMEOUT, drains what it
@@ -41,7 +41,12 @@ constexpr int BK = 64;                           // K per stage: one 128-byte sw
 constexpr int kStages = 4;
 constexpr int kABytes = BM * BK * 2;             // 16 KB
 constexpr int kBBytes = BN * BK * 2;             // 32 KB
-constexpr int kDecWarps = 4, kEpiWarps = 4;
+#ifndef TERN_PREFILL_DEC_WARPS
+#define TERN_PREFILL_DEC_WARPS 8
+#endif
+constexpr int kDecWarps = TERN_PREFILL_DEC_WARPS, kEpiWarps = 4;
+constexpr int kRowsPerDec = BN / (kDecWarps * 32);   // weight rows expanded per decoder thread
+static_assert(kRowsPerDec * kDecWarps * 32 == BN, "decoder rows");
 constexpr int kPrefillThreads = (2 + kDecWarps + kEpiWarps) * 32;
 constexpr int kTmemCols = 2 * BN;                // two accumulators
 constexpr uint32_t kWaitTries = 1u << 13;
@@ -225,42 +230,42 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) k_prefill(const __grid_con
     }
   } else if (warp < 2 + kDecWarps) {
     // ---------------- weight expansion: 256 rows x 64 trits -> bf16, swizzled ----------------
-    const int d = threadIdx.x - 64;                   // 0..127: rows d and d + 128 of the tile
+    const int d = threadIdx.x - 64;                   // rows d, d + 32 * kDecWarps, ... of the tile
     const int KW = p.K / 16;                          // words per row (both planes)
     int q = 0;
     for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
       const int nt = tile % tiles_n;
-      const uint32_t* rowp[2];
-      bool live[2];
+      const uint32_t* rowp[kRowsPerDec];
+      bool live[kRowsPerDec];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int n = nt * BN + d + 128 * h;
+      for (int h = 0; h < kRowsPerDec; ++h) {
+        const int n = nt * BN + d + 32 * kDecWarps * h;
         live[h] = n < p.N;
         rowp[h] = p.planes + (size_t)(live[h] ? n : 0) * KW;
       }
       // 16-byte loads of each plane cover two stages (a pair); pairs are loaded two pairs ahead
       //   p0 = the pair being decoded, p1, p2 = the next two
-      uint4 pm[3][2], ps[3][2];
+      uint4 pm[3][kRowsPerDec], ps[3][kRowsPerDec];
 #pragma unroll
       for (int j = 0; j < 3; ++j)
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < kRowsPerDec; ++h) {
           const bool in = live[h] && 2 * j < KT;
           pm[j][h] = in ? ldg128(rowp[h] + 4 * j) : make_uint4(0u, 0u, 0u, 0u);
           ps[j][h] = in ? ldg128(rowp[h] + KW / 2 + 4 * j) : make_uint4(0u, 0u, 0u, 0u);
         }
       for (int kt = 0; kt < KT; ++kt, ++q) {
         const int s = q % kStages;
-        uint2 cm[2], cs[2];
+        uint2 cm[kRowsPerDec], cs[kRowsPerDec];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < kRowsPerDec; ++h) {
           cm[h] = (kt & 1) ? make_uint2(pm[0][h].z, pm[0][h].w) : make_uint2(pm[0][h].x, pm[0][h].y);
           cs[h] = (kt & 1) ? make_uint2(ps[0][h].z, ps[0][h].w) : make_uint2(ps[0][h].x, ps[0][h].y);
         }
         if (kt & 1) {                                    // pair done: shift the queue, fetch pair + 3
           const int j3 = (kt >> 1) + 3;
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
+          for (int h = 0; h < kRowsPerDec; ++h) {
             pm[0][h] = pm[1][h]; pm[1][h] = pm[2][h];
             ps[0][h] = ps[1][h]; ps[1][h] = ps[2][h];
             const bool in = live[h] && 2 * j3 < KT;
@@ -271,8 +276,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) k_prefill(const __grid_con
         if (q >= kStages && !(ok = mbar_wait(empty + 8 * s, ((q / kStages) - 1) & 1))) break;
         const uint32_t tileB = sB + s * kBBytes;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int r = d + 128 * h;
+        for (int h = 0; h < kRowsPerDec; ++h) {
+          const int r = d + 32 * kDecWarps * h;
           const uint32_t rowa = tileB + r * 128;
           const int sw = r & 7;
 #pragma unroll

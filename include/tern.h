@@ -105,13 +105,30 @@ size_t tern_base3_bytes(int32_t N, int32_t K);
 
 /* Pack a ternary matrix into the planes layout (the loader step: weights packed at rest, [A]).
  *   src = TERN_SRC_INT8_TRITS: src_dev is int8[N][K] row-major with values in {-1, 0, +1}.
- *   src = TERN_SRC_BASE3:      src_dev is the transport, uint8[N][ceil(K/5)] (layout above); it is
- *                              expanded bit-exactly ([R] "3진 계열이라는 이름의 실체").
+ *   src = TERN_SRC_BASE3:      src_dev is the transport, uint8[N][ceil(K/5)] (layout above), 4-byte
+ *                              aligned; it is expanded bit-exactly ([R] "3진 계열이라는 이름의 실체").
  *   planes_dev: output, N*K/16 uint32 words, 16-byte aligned.
  *   err_flag_dev: int32 on the device; cleared by this call on the stream, then set nonzero if
  *   any input value is invalid (the planes are then unspecified). Required. */
 tern_status tern_pack(tern_src src, const void* src_dev, int32_t N, int32_t K, uint32_t* planes_dev,
                       int32_t* err_flag_dev, tern_stream_t stream);
+
+/* One tensor of a tern_pack_batch call: views of caller-owned device memory. */
+typedef struct {
+  const void* src_dev;        /* as tern_pack's src_dev for the call's src kind        */
+  int32_t N, K;               /* shape, as for tern_pack                               */
+  uint32_t* planes_dev;       /* output planes, N*K/16 words, 16-byte aligned          */
+} tern_pack_item;
+
+#define TERN_PACK_MAX_ITEMS 256
+
+/* tern_pack over a list of tensors (a whole model's transport at load time): one clear of
+ * err_flag_dev, then one launch for all base-3 items (TERN_SRC_BASE3), or one launch per item
+ * for TERN_SRC_INT8_TRITS. Results are bit-identical to tern_pack per item; the flag is set if
+ * any item holds an invalid value. items: host array of 1..TERN_PACK_MAX_ITEMS descriptors,
+ * read during the call only. No output may overlap another item's input or output. */
+tern_status tern_pack_batch(tern_src src, const tern_pack_item* items, int32_t count, int32_t* err_flag_dev,
+                            tern_stream_t stream);
 
 /* Encode dense trits int8[N][K] into the base-3 transport uint8[N][ceil(K/5)] (the inverse of
  * tern_pack with TERN_SRC_BASE3). err_flag_dev as for tern_pack. */

@@ -120,3 +120,26 @@ def test_8b_transport_full_size():
             del t, enc, a, b
     assert tg.tern_read_flag(flag) == 0
     assert total == 6_945_767_424
+
+
+def test_base3_batch_bit_exact_and_flag():
+    """tern_pack_batch over ragged base-3 items equals the oracle per item (odd byte counts, so the
+    transport buffers end inside a word); a bad byte in one item sets the flag."""
+    shapes = [(1, 128), (37, 384), (20, 4096), (5, 12288), (9, 1024), (3, 640)]
+    items, refs, flag = [], [], torch.zeros(1, dtype=torch.int32, device="cuda")
+    for i, (N, K) in enumerate(shapes):
+        t = synth.trits(34, 50 + i, N, K)
+        enc = dev(oracle.base3_encode(t).reshape(-1))
+        planes = torch.full((N * K // 16,), -1, dtype=torch.int32, device="cuda")
+        items.append((enc, N, K, planes))
+        refs.append(oracle.pack(t))
+    tg.tern_pack_batch(tg.TERN_SRC_BASE3, items, flag)
+    assert tg.tern_read_flag(flag) == 0
+    for (enc, N, K, planes), ref in zip(items, refs):
+        assert (host(planes).view(np.uint32).reshape(N, K // 16) == ref).all(), (N, K)
+    bad = items[3][0].clone()
+    bad[7] = 243
+    tg.tern_pack_batch(tg.TERN_SRC_BASE3, [items[0], (bad, 5, 12288, items[3][3])], flag)
+    assert tg.tern_read_flag(flag) == tg.TERN_EBADCODE
+    tg.tern_pack_batch(tg.TERN_SRC_BASE3, items[:2], flag)          # the next call clears the flag
+    assert tg.tern_read_flag(flag) == 0
