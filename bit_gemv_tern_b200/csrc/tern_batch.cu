@@ -135,6 +135,12 @@ __global__ void __launch_bounds__(256) k_batch_prep(const __grid_constant__ Batc
   __shared__ int sums[3];
   __shared__ int Esh;
   pdl_wait();
+  {
+    // the split-block sums and counters of the stream start at zero
+    uint32_t* scr = reinterpret_cast<uint32_t*>(p.xprep + p.scratch_off);
+    const int nct = gridDim.x * gridDim.y, ct = blockIdx.y * gridDim.x + blockIdx.x;
+    for (int i = ct * blockDim.x + threadIdx.x; i < p.scratch_words; i += nct * blockDim.x) scr[i] = 0u;
+  }
   // this token's columns (and its meta words) start at zero: the K tail of the last part stays so
   for (int i = threadIdx.x; i < KP * nl * kColWords; i += blockDim.x) {
     const int part = i / (nl * kColWords), r = i % (nl * kColWords);
@@ -244,7 +250,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
   const uint32_t slot_bytes = (uint32_t)p.stage_slot_bytes;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int u0 = p.cta_unit[blockIdx.x], u1 = p.cta_unit[blockIdx.x + 1];
+  const int g0 = p.cta_part[blockIdx.x], g1 = p.cta_part[blockIdx.x + 1];
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
@@ -256,28 +262,23 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
   }
   __syncthreads();
   pdl_launch_dependents();
-  if (u1 <= u0) return;
+  if (g1 <= g0) return;
 
-  // item of the first unit
+  // item, row block and part of the first stage
   int first_item = 0;
-  while (first_item + 1 < p.count && p.items[first_item + 1].unit0 <= u0) ++first_item;
+  while (first_item + 1 < p.count && p.items[first_item + 1].part0 <= g0) ++first_item;
+  const int first_rb = (g0 - p.items[first_item].part0) / p.items[first_item].kp;
+  const int first_part = (g0 - p.items[first_item].part0) - first_rb * p.items[first_item].kp;
 
   if (warp == kCW) {
     // ====================== producer (lane 0) ======================
     if (lane != 0) return;
     // stages of this CTA in order: (item, row block, part)
-    int n = 0;
-    {
-      int it = first_item;
-      for (int u = u0; u < u1; ++u) {
-        while (it + 1 < p.count && p.items[it + 1].unit0 <= u) ++it;
-        n += p.items[it].kp;
-      }
-    }
+    const int n = g1 - g0;
     bool ok = true;
     // 1. weights of the first stages: they do not depend on earlier kernels
     const int pre = n < S ? n : S;
-    int it = first_item, rb = u0 - p.items[first_item].unit0, part = 0;
+    int it = first_item, rb = first_rb, part = first_part;
     for (int q = 0; q < pre; ++q) {
       const BatchItem& B = p.items[it];
       const uint32_t bar = full0 + 8 * q;
@@ -294,7 +295,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
     }
     pdl_wait();
     // 2. every stage: its operand segment and, past the first S, its weights once the slot is free
-    it = first_item; rb = u0 - p.items[first_item].unit0; part = 0;
+    it = first_item; rb = first_rb; part = first_part;
     int s = 0;
     uint32_t ph = 0;
     for (int q = 0; q < n && ok; ++q) {
@@ -338,13 +339,21 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
   const uint32_t xofs = (uint32_t)(kWStageBytesT + (col0 * kColWords + t * 8) * 4);
   const uint32_t mofs = (uint32_t)(kWStageBytesT + NCOL * kColWords * 4);
   const int M = p.M;
+  constexpr int NCOLP = 8 * G;                              // scratch columns per row
+  const uint32_t split = p.cta_split[blockIdx.x];
+  const int slot_first = (int)(split & 0xFFu) - 1, need_first = (int)((split >> 8) & 0xFFu);
+  const int slot_last = (int)((split >> 16) & 0xFFu) - 1, need_last = (int)(split >> 24);
   bool ok = true;
-  int it = first_item, rb = u0 - p.items[first_item].unit0;
+  int it = first_item, rb = first_rb, pstart = first_part;
   int s = 0;
   uint32_t ph = 0;
-  for (int u = u0; u < u1 && ok; ++u) {
+  for (int gq = g0; gq < g1 && ok;) {
     const BatchItem& B = p.items[it];
     const int KP = B.kp;
+    const int pend = min(KP, pstart + (g1 - gq));           // this CTA's parts of the block: [pstart, pend)
+    int slot = -1, need = 0;                                // block shared with other CTAs
+    if (gq == g0) { slot = slot_first; need = need_first; }
+    if (gq + (pend - pstart) == g1 && slot_last >= 0) { slot = slot_last; need = need_last; }
     const int row_base = rb * kStageRowsT + warp * 16;         // first row of this warp's tile slot 0
     int acc[TPW][G][4][4];
 #pragma unroll
@@ -368,11 +377,11 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
         const int row = row_base + a * kBoxRows + g + 8 * h;
         sc_bits[a][h] = ((MP > 1 || t == 0) && row < B.N) ? B.scale[row] : (uint16_t)0;
       }
-    for (int part = 0; part < KP; ++part) {
+    for (int part = pstart; part < pend; ++part) {
       if (!(ok = mbar_wait(full0 + 8 * s, ph))) break;
       // s_x comes from an earlier kernel: read only after a stage has landed (the producer issues
       // every copy after its grid-dependency wait)
-      if (MODE == 1 && part == 0) {
+      if (MODE == 1 && part == pstart) {
 #pragma unroll
         for (int jj = 0; jj < JJ; ++jj)
 #pragma unroll
@@ -424,7 +433,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
                        i < 2 ? u4get(x01, 2 * i + 1) : u4get(x23, 2 * i - 3));
         }
       }
-      if (part == KP - 1) {                                  // sums over all of K and E ride in every segment
+      if (part == pend - 1) {                                // sums over all of K and E ride in every segment
 #pragma unroll
         for (int jj = 0; jj < JJ; ++jj)
 #pragma unroll
@@ -459,14 +468,60 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
     }
     if (!ok) break;
     // ---- outputs of this warp's tiles: exact integer sums, one rounding ----------------------------
+    // the four field accumulators of each (row, column) combined exactly
+    int V[TPW][G][4];
 #pragma unroll
-    for (int a = 0; a < TPW; ++a) {
+    for (int a = 0; a < TPW; ++a)
+#pragma unroll
+      for (int j = 0; j < G; ++j)
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          V[a][j][q] = acc[a][j][0][q] + (acc[a][j][1][q] >> 2) + (acc[a][j][2][q] >> 4) + (acc[a][j][3][q] >> 6);
+    bool emit = true;
+    if (slot >= 0) {
+      // a block split between CTAs: add this CTA's part sums; the last contributor (per warp)
+      // reads the totals back and writes the outputs
+      int* sums = reinterpret_cast<int*>(p.xprep + p.scratch_off) + (size_t)slot * kStageRowsT * NCOLP;
+      int* counter = reinterpret_cast<int*>(p.xprep + p.scratch_off) + (size_t)p.nslots * kStageRowsT * NCOLP +
+                     slot * kCW + warp;
+#pragma unroll
+      for (int a = 0; a < TPW; ++a)
+#pragma unroll
+        for (int j = 0; j < G; ++j)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int col = 8 * j + 2 * t + (q & 1);
+            if (MP > 1 || col < NCOL)
+              atomicAdd(&sums[(a * kBoxRows + warp * 16 + g + 8 * (q >> 1)) * NCOLP + col], V[a][j][q]);
+          }
+      __threadfence();
+      __syncwarp();
+      int last = 0;
+      if (lane == 0) last = atomicAdd(counter, 1) == need - 1;
+      last = __shfl_sync(0xFFFFFFFFu, last, 0);
+      if (last) {
+        __threadfence();
+#pragma unroll
+        for (int a = 0; a < TPW; ++a)
+#pragma unroll
+          for (int j = 0; j < G; ++j)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int col = 8 * j + 2 * t + (q & 1);
+              if (MP > 1 || col < NCOL)
+                V[a][j][q] = __ldcg(&sums[(a * kBoxRows + warp * 16 + g + 8 * (q >> 1)) * NCOLP + col]);
+            }
+      } else {
+        emit = false;
+      }
+    }
+#pragma unroll
+    for (int a = 0; a < TPW && emit; ++a) {
       const int r0 = row_base + a * kBoxRows + g;            // rows r0 (q = 0, 1) and r0 + 8 (q = 2, 3)
       if (MP == 1) {
         int v[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          v[q] = acc[a][0][0][q] + (acc[a][0][1][q] >> 2) + (acc[a][0][2][q] >> 4) + (acc[a][0][3][q] >> 6);
+        for (int q = 0; q < 4; ++q) v[q] = V[a][0][q];
         if (MODE == 1) {
           if (t == 0) {
 #pragma unroll
@@ -509,16 +564,13 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
             if (m < M && row < B.N) {
               const float sc = f16_bits_to_float(sc_bits[a][h]);
               if (MODE == 1) {
-                const int v = acc[a][jj][0][q] + (acc[a][jj][1][q] >> 2) + (acc[a][jj][2][q] >> 4) + (acc[a][jj][3][q] >> 6);
-                const int S1 = v - 2 * tot[jj][0][b];
+                const int S1 = V[a][jj][q] - 2 * tot[jj][0][b];
                 B.y[(size_t)m * B.N + row] = __fmul_rn(__fmul_rn(__int2float_rn(S1), sxv[jj][b]), sc);
               } else {
                 long long Sl[3];
 #pragma unroll
                 for (int l = 0; l < 3; ++l) {
-                  const int j = l * JJ + jj;
-                  const int v = acc[a][j][0][q] + (acc[a][j][1][q] >> 2) + (acc[a][j][2][q] >> 4) + (acc[a][j][3][q] >> 6);
-                  Sl[l] = (long long)v - 2LL * tot[jj][l][b];
+                  Sl[l] = (long long)V[a][l * JJ + jj][q] - 2LL * tot[jj][l][b];
                 }
                 const long long D = Sl[0] * 65536 + Sl[1] * 256 + Sl[2];
                 B.y[(size_t)m * B.N + row] = (float)((double)D * exp2_i(Etok[jj][b] - kLimbFrac) * (double)sc);
@@ -527,6 +579,8 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
           }
       }
     }
+    gq += pend - pstart;
+    pstart = 0;
     if (++rb == B.units) { rb = 0; ++it; }
   }
   if (!ok && lane == 0) atomicExch(&g_batch_latch, 5);
@@ -577,10 +631,11 @@ bool plan_batch(BatchParams& p, const uint32_t* const* planes, size_t& smem, siz
   p.nc = seg_cols(p.mode, mp);
   p.seg_bytes = seg_words(p.mode, mp) * 4;
   const int stage_rows = kBoxRows * tpw;
+  const int ncolp = mp == 1 ? 8 : seg_cols(p.mode, mp);   // scratch columns: 8 per MMA group
   PFN_cuTensorMapEncodeTiled_v12000 encode = encode_fn();
   if (!encode) return false;
-  long long total_bytes = 0;
-  int units = 0;
+  long long total_cost = 0;
+  int units = 0, parts = 0;
   size_t xoff = 0;
   for (int i = 0; i < p.count; ++i) {
     BatchItem& it = p.items[i];
@@ -588,10 +643,14 @@ bool plan_batch(BatchParams& p, const uint32_t* const* planes, size_t& smem, siz
     it.kp = (it.K + 511) / 512;
     it.unit0 = units;
     it.units = (it.N + stage_rows - 1) / stage_rows;
+    it.part0 = parts;
     units += it.units;
+    if ((long long)parts + (long long)it.units * it.kp > 0x3FFFFFFF) return false;
+    parts += it.units * it.kp;
     it.xoff = (uint32_t)xoff;
     xoff += (size_t)it.kp * p.seg_bytes;
-    total_bytes += (long long)it.N * it.K / 4;
+    // cost of the item's parts: rows x 128 bytes of planes each
+    total_cost += (long long)it.N * it.kp * 128;
     // planes of row n: mask words [n * K/16, n * K/16 + K/32), its sign words right after
     const cuuint64_t dims[3] = {(cuuint64_t)(it.K / 32), (cuuint64_t)it.N, 2};
     const cuuint64_t strides[2] = {(cuuint64_t)it.K / 4, (cuuint64_t)it.K / 8};   // bytes: row, plane
@@ -603,23 +662,76 @@ bool plan_batch(BatchParams& p, const uint32_t* const* planes, size_t& smem, siz
       return false;
   }
   p.total_units = units;
-  workspace = xoff;
-  // balanced by weight bytes: CTA c starts at the first unit whose start byte reaches c/G of the total
-  const int grid = units < 148 ? units : 148;
+  // CTA c starts at the first part whose cost prefix reaches c/G of the total: the split is
+  // balanced to one 512-trit part, and a row block may be shared by neighbouring CTAs
+  const int grid = parts < 148 ? parts : 148;
   p.grid = grid;
-  long long acc = 0;
-  int c = 0;
-  p.cta_unit[0] = 0;
-  for (int i = 0; i < p.count; ++i) {
-    const BatchItem& it = p.items[i];
-    for (int u = 0; u < it.units; ++u) {
-      while (c + 1 < grid && acc >= total_bytes * (c + 1) / grid) p.cta_unit[++c] = it.unit0 + u;
-      const int rows = it.N - u * stage_rows < stage_rows ? it.N - u * stage_rows : stage_rows;
-      acc += (long long)rows * it.K / 4;
+  {
+    int c = 1;
+    long long acc = 0;
+    p.cta_part[0] = 0;
+    for (int i = 0; i < p.count && c < grid; ++i) {
+      const BatchItem& it = p.items[i];
+      for (int u = 0; u < it.units && c < grid; ++u) {
+        const int rows = it.N - u * stage_rows < stage_rows ? it.N - u * stage_rows : stage_rows;
+        const long long cu = (long long)rows * 128;
+        const int ustart = it.part0 + u * it.kp;
+        while (c < grid && total_cost * c / grid < acc + cu * it.kp) {
+          long long off = (total_cost * c / grid - acc + cu - 1) / cu;   // parts of this block before c
+          if (off < 0) off = 0;
+          p.cta_part[c++] = ustart + (int)off;
+        }
+        acc += cu * it.kp;
+      }
     }
+    for (; c <= grid; ++c) p.cta_part[c] = parts;
+    p.cta_part[grid] = parts;
   }
-  while (c + 1 <= grid) p.cta_unit[++c] = units;
-  p.cta_unit[grid] = units;
+  // blocks shared by several CTAs: one scratch slot each, with its contributor count
+  auto unit_of = [&](int gpart, int& ustart, int& uend) {
+    int i = 0;
+    while (i + 1 < p.count && p.items[i + 1].part0 <= gpart) ++i;
+    const BatchItem& it = p.items[i];
+    const int u = (gpart - it.part0) / it.kp;
+    ustart = it.part0 + u * it.kp;
+    uend = ustart + it.kp;
+    return it.unit0 + u;
+  };
+  int nslots = 0;
+  int slot_unit[160], slot_need[160];
+  for (int c = 0; c < grid; ++c) {
+    p.cta_split[c] = 0;
+    const int lo = p.cta_part[c], hi = p.cta_part[c + 1];
+    if (lo >= hi) continue;
+    int ends[2] = {lo, hi - 1};
+    uint32_t code = 0;
+    for (int e = 0; e < 2; ++e) {
+      int us, ue;
+      const int u = unit_of(ends[e], us, ue);
+      if (us >= lo && ue <= hi) continue;               // the block is this CTA's alone
+      int sl = -1;
+      for (int k = 0; k < nslots; ++k)
+        if (slot_unit[k] == u) sl = k;
+      if (sl < 0) {
+        if (nslots >= 160 || nslots >= 254) return false;
+        sl = nslots++;
+        slot_unit[sl] = u;
+        int need = 0;                                   // CTAs whose range meets [us, ue)
+        for (int d = 0; d < grid; ++d)
+          if (p.cta_part[d] < p.cta_part[d + 1] && p.cta_part[d] < ue && p.cta_part[d + 1] > us) ++need;
+        if (need > 255) return false;
+        slot_need[sl] = need;
+      }
+      code |= ((uint32_t)(sl + 1) | ((uint32_t)slot_need[sl] << 8)) << (16 * e);
+    }
+    p.cta_split[c] = code;
+  }
+  p.nslots = nslots;
+  // workspace: operand segments, then the split sums [slot][rows][ncolp] and counters [slot][cw]
+  xoff = (xoff + 15) & ~(size_t)15;
+  p.scratch_off = (uint32_t)xoff;
+  p.scratch_words = nslots * (stage_rows * ncolp + cw);
+  workspace = xoff + (size_t)p.scratch_words * 4 + 16;
   p.stage_slot_bytes = (tpw * kBoxBytes + p.seg_bytes + 1023) & ~1023;
   const size_t budget = 227 * 1024;
   int stages = (int)((budget - 1024) / (size_t)p.stage_slot_bytes);

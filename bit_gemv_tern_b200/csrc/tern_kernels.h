@@ -58,6 +58,7 @@ struct BatchItem {
   int32_t kp;             // 512-trit K parts (the last may be partial): stages per row block
   int32_t unit0;          // first global unit (row block) of the item
   int32_t units;          // row blocks of the item
+  int32_t part0;          // first global part (unit x 512-trit K part) of the item
   uint32_t xoff;          // byte offset of the item's operand block in the workspace
 };
 constexpr int kBatchMaxItems = 160;
@@ -77,7 +78,15 @@ struct BatchParams {
   int32_t stage_slot_bytes;
   int32_t seg_bytes;      // operand bytes of one 512-trit part (all columns + sums + exponent)
   uint8_t* xprep;         // workspace: operand blocks
-  int32_t cta_unit[149];  // CTA c handles units [cta_unit[c], cta_unit[c + 1])
+  int32_t cta_part[149];  // CTA c handles global parts [cta_part[c], cta_part[c + 1])
+  // Row blocks split between CTAs: each contributor adds exact partial sums into a workspace
+  // slot; the last one (per warp, by counter) writes the outputs.
+  // per CTA, 8 bits each: slot of its first block + 1, that block's contributors, slot of its
+  // last block + 1, that block's contributors (slot + 1 = 0: the block is this CTA's alone)
+  uint32_t cta_split[148];
+  int32_t nslots;
+  uint32_t scratch_off;   // workspace byte offset: [nslots][rows][8 * groups] int32, then counters
+  int32_t scratch_words;  // words to zero before the stream (sums and counters)
 };
 static_assert(sizeof(BatchParams) <= 32764, "kernel parameter limit");
 // Host: fills tmap/kp/units/xoff, the stage ring and the CTA split; fails on unsupported shapes.
