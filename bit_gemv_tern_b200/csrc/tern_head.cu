@@ -35,7 +35,7 @@ constexpr int kHeadRows = 128;   // rows per row block: 8 warps x 16 rows
 constexpr int kLimbFrac = 22;    // bf16 mode: x ~= X * 2^(E - 22), |X| < 2^22
 
 template <int MODE, int NG>
-__global__ void __launch_bounds__(kThreads) k_head(const HeadParams p) {
+__global__ void __launch_bounds__(kThreads, 2) k_head(const HeadParams p) {
   extern __shared__ __align__(16) uint32_t smem[];
   __shared__ unsigned long long best[16];
   __shared__ int expo[16];
@@ -71,10 +71,11 @@ __global__ void __launch_bounds__(kThreads) k_head(const HeadParams p) {
   };
 
   int rb = blockIdx.y;
-  uint4 cur[4], nxt[4];
+  uint4 cur[4], nxt[4], nx2[4];                // three chunks of the warp's rows in flight
   set_rows(rb);
   load_chunk(0, cur);
   load_chunk(1, nxt);
+  load_chunk(2, nx2);
   pdl_wait();
 
   // ---- stage activations: column c of the B operand holds K-slice bytes -------------------------
@@ -138,15 +139,7 @@ __global__ void __launch_bounds__(kThreads) k_head(const HeadParams p) {
   int* part = reinterpret_cast<int*>(smem + ncols * RS);
   cg::cluster_group cluster = cg::this_cluster();
   const int rows_per_rank = kHeadRows / p.ksplit;
-  bool first = true;
-
   for (; rb < p.nrb; rb += p.nby) {
-    if (!first) {
-      set_rows(rb);
-      load_chunk(0, cur);
-      load_chunk(1, nxt);
-    }
-    first = false;
     int acc[NG][4];
 #pragma unroll
     for (int n = 0; n < NG; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0;
@@ -168,8 +161,18 @@ __global__ void __launch_bounds__(kThreads) k_head(const HeadParams p) {
         mma_s8(acc[n], cur[1].z, cur[3].z, cur[1].w, cur[3].w, b1.z, b1.w);
       }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) cur[i] = nxt[i];
-      load_chunk(c + 2, nxt);
+      for (int i = 0; i < 4; ++i) {
+        cur[i] = nxt[i];
+        nxt[i] = nx2[i];
+      }
+      load_chunk(c + 3, nx2);
+    }
+    // the next row block's first chunks stream in while this block's outputs are formed
+    if (rb + p.nby < p.nrb) {
+      set_rows(rb + p.nby);
+      load_chunk(0, cur);
+      load_chunk(1, nxt);
+      load_chunk(2, nx2);
     }
 
     // partial sums of this K slice: part[local row][column]
