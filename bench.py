@@ -369,6 +369,27 @@ def run_reference(args, rank, world):
     return 0
 
 
+def rank_barrier(dist):
+    """Barrier over the replica ranks (no-op on one GPU)."""
+    if dist is not None:
+        dist.barrier()
+
+
+def max_over(dist, v, device):
+    """The maximum of a per-rank time over all replica ranks (the slowest rank sets the clock)."""
+    if dist is None:
+        return v
+    import torch
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(world, steps, ms):
+    """Whole-job units per second: every rank processed `steps` units in `ms` (the max over ranks)."""
+    return world * steps / (ms / 1000.0)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -397,15 +418,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
     def barrier():
-        if dist is not None:
-            dist.barrier()
+        rank_barrier(dist)
 
     def max_over_ranks(v):
-        if dist is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return max_over(dist, v, "cuda")
 
     import bit_gemv_tern_b200 as tg
     from bit_gemv_tern_b200 import build as _b
@@ -446,7 +462,7 @@ def main():
     ms = max_over_ranks(ms)
     clocks = clk.summary()
     ms_step = ms / args.steps
-    value = world * args.steps / (ms / 1000.0)
+    value = replica_throughput(world, args.steps, ms)
 
     # dominant kernel: the ternary GEMV launches of the last replay's steps
     stack_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(S)]
@@ -534,15 +550,36 @@ def _profile_prefill(proj):
     return run
 
 
+def _profile_base3():
+    def run():
+        import torch
+        import synth
+        import synth.cuda as sc
+        import bit_gemv_tern_b200 as tg
+        flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+        items = []
+        for p, N, K in synth.linear_shapes("8b"):
+            t = torch.empty(N * K, dtype=torch.int8, device="cuda")
+            sc.trits_into(t, SEED, synth.tensor_id(0, p), K)
+            e = torch.empty(tg.tern_base3_bytes(N, K), dtype=torch.uint8, device="cuda")
+            tg.tern_base3_encode(t, N, K, e, flag)
+            del t
+            items.append((e, N, K, torch.empty(N * K // 16, dtype=torch.int32, device="cuda")))
+        return lambda: tg.tern_pack_batch(tg.TERN_SRC_BASE3, items, flag)
+    return run
+
+
 # Small cases for ncu captures (inputs > L2, a few hundred MB on the device):
 #   batch-8b-4layers-*: 4 layers of the 8B stack (16 fused GEMVs, 193 MB of planes) as one batch
 #   head-8b-*:          the int8 head 151936 x 4096 (622 MB)
 #   prefill-8b-gate-*:  one 12288 x 4096 linear at M = 4096 tokens (tcgen05 prefill)
+#   base3-8b-1layer:    the transport of one 8B layer's seven tensors (86.9 MB) in one batched call
 PROFILE_CASES = {
     "batch-8b-4layers-bf16": _profile_batch("bf16"),
     "batch-8b-4layers-int8": _profile_batch("int8"),
     "head-8b-bf16": _profile_head("bf16"),
     "prefill-8b-gate-m4096": _profile_prefill("gate"),
+    "base3-8b-1layer": _profile_base3(),
 }
 
 

@@ -48,10 +48,11 @@ __global__ void k_pack_trits(const int8_t* __restrict__ src, int64_t n_words, in
   if (__any_sync(0xFFFFFFFFu, bad) && (threadIdx.x & 31) == 0) set_flag(flag);
 }
 
-// Byte -> five trits as (mask5 | sign5 << 5); 0xFFFF marks an invalid byte (> 242).
-__device__ __forceinline__ void build_base3_lut(uint16_t* lut) {
+// Byte -> five trits as (mask5 | sign5 << 16), in natural order; all ones marks an invalid byte
+// (> 242), which also sets bit 31 of the OR of a run's entries.
+__device__ __forceinline__ void build_base3_lut(uint32_t* lut) {
   for (int b = threadIdx.x; b < 256; b += blockDim.x) {
-    uint16_t e = 0xFFFFu;
+    uint32_t e = 0xFFFFFFFFu;
     if (b < 243) {
       int v = b;
       uint32_t m = 0, s = 0;
@@ -61,7 +62,7 @@ __device__ __forceinline__ void build_base3_lut(uint16_t* lut) {
         m |= (uint32_t)(d != 1) << i;
         s |= (uint32_t)(d == 0) << i;
       }
-      e = (uint16_t)(m | (s << 5));
+      e = m | (s << 16);
     }
     lut[b] = e;
   }
@@ -92,73 +93,99 @@ __device__ __forceinline__ void unpack_base3_block(const uint8_t* __restrict__ s
   const int nrow = min(N - r0, rows_per_cta);
   const int rpr = (KW + 4) / 5;                    // runs per row
   const int nruns = nrow * rpr;
-  uint16_t* lut = reinterpret_cast<uint16_t*>(b3_smem);
-  uint8_t* runs = reinterpret_cast<uint8_t*>(b3_smem) + 512;
+  uint32_t* lut = reinterpret_cast<uint32_t*>(b3_smem);
+  uint8_t* runs = reinterpret_cast<uint8_t*>(b3_smem) + 1024;
   uint32_t* outw = reinterpret_cast<uint32_t*>(runs + (size_t)rows_per_cta * rpr * kB3Slot);
   build_base3_lut(lut);
   const int64_t total = (int64_t)N * rb;
+  // run index j -> (row rr, run i) advanced without divisions: j steps by `step`
+  const int step = blockDim.x / 2;                 // copy phase: two half-runs per run
+  const int dq = step / rpr, dr = step - (step / rpr) * rpr;
   // 1. copy: half-runs of 16 bytes, each from five aligned words of the transport
-  for (int hr = threadIdx.x; hr < 2 * nruns; hr += blockDim.x) {
-    const int j = hr >> 1, h = hr & 1;
-    const int rr = j / rpr, i = j - rr * rpr;
-    const int pos = 32 * i + 16 * h;              // byte position in the row
-    const int64_t g = (int64_t)(r0 + rr) * rb + pos;
-    const int64_t ga = g & ~(int64_t)3;
-    const uint32_t sh = 8u * (uint32_t)(g & 3);
-    uint32_t w[5];
+  {
+    int j = threadIdx.x >> 1, rr = j / rpr, i = j - rr * rpr;
+    const int h = threadIdx.x & 1;
+    for (; j < nruns; j += step) {
+      const int pos = 32 * i + 16 * h;              // byte position in the row
+      const int64_t g = (int64_t)(r0 + rr) * rb + pos;
+      const int64_t ga = g & ~(int64_t)3;
+      const uint32_t sh = 8u * (uint32_t)(g & 3);
+      uint32_t w[5];
 #pragma unroll
-    for (int k = 0; k < 5; ++k) {
-      const int64_t a = ga + 4 * k;
-      if (a + 4 <= total) {
-        w[k] = __ldg(reinterpret_cast<const uint32_t*>(src + a));
-      } else {                                    // the buffer's last, partial word: byte by byte
-        uint32_t x = 0u;
-        for (int t = 0; t < 4; ++t)
-          if (a + t < total) x |= (uint32_t)__ldg(src + a + t) << (8 * t);
-        w[k] = x;
+      for (int k = 0; k < 5; ++k) {
+        const int64_t a = ga + 4 * k;
+        if (a + 4 <= total) {
+          w[k] = __ldg(reinterpret_cast<const uint32_t*>(src + a));
+        } else {                                    // the buffer's last, partial word: byte by byte
+          uint32_t x = 0u;
+          for (int t = 0; t < 4; ++t)
+            if (a + t < total) x |= (uint32_t)__ldg(src + a + t) << (8 * t);
+          w[k] = x;
+        }
       }
+      // bytes past the row's end belong to the next row: they only reach trits past K, never written
+      uint4 v;
+      v.x = __funnelshift_r(w[0], w[1], sh);
+      v.y = __funnelshift_r(w[1], w[2], sh);
+      v.z = __funnelshift_r(w[2], w[3], sh);
+      v.w = __funnelshift_r(w[3], w[4], sh);
+      *reinterpret_cast<uint4*>(runs + (size_t)j * kB3Slot + 16 * h) = v;
+      rr += dq;
+      i += dr;
+      if (i >= rpr) { i -= rpr; ++rr; }
     }
-    // bytes past the row's end belong to the next row: never decoded into an output word
-    uint4 v;
-    v.x = __funnelshift_r(w[0], w[1], sh);
-    v.y = __funnelshift_r(w[1], w[2], sh);
-    v.z = __funnelshift_r(w[2], w[3], sh);
-    v.w = __funnelshift_r(w[3], w[4], sh);
-    *reinterpret_cast<uint4*>(runs + (size_t)j * kB3Slot + 16 * h) = v;
   }
   __syncthreads();
   // 2. decode
   bool bad = false;
-  for (int j = threadIdx.x; j < nruns; j += blockDim.x) {
-    const int rr = j / rpr, i = j - rr * rpr;
-    const int nb = min(32, rb - 32 * i);          // bytes of the run inside the row
-    const uint4 lo = *reinterpret_cast<const uint4*>(runs + (size_t)j * kB3Slot);
-    const uint4 hi = *reinterpret_cast<const uint4*>(runs + (size_t)j * kB3Slot + 16);
-    const uint32_t by[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-    uint32_t m[6] = {0u, 0u, 0u, 0u, 0u, 0u}, s[6] = {0u, 0u, 0u, 0u, 0u, 0u};
+  {
+    const int step2 = blockDim.x;
+    const int eq = step2 / rpr, er = step2 - eq * rpr;
+    int j = threadIdx.x, rr = j / rpr, i = j - rr * rpr;
+    for (; j < nruns; j += step2) {
+      const int nb = min(32, rb - 32 * i);        // bytes of the run inside the row
+      const uint4 lo = *reinterpret_cast<const uint4*>(runs + (size_t)j * kB3Slot);
+      const uint4 hi = *reinterpret_cast<const uint4*>(runs + (size_t)j * kB3Slot + 16);
+      const uint32_t by[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+      // groups of 16 trits: W[k] holds the group's 16 mask bits low and 16 sign bits high, so one
+      // shifted table entry (mask5 | sign5 << 16) lands both fields of a byte with one add; the
+      // bytes whose five trits cross a group boundary are added in two parts
+      uint32_t W[10] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+      uint32_t eor = 0u;
+      const bool full = nb == 32;                 // every run but a row's last
 #pragma unroll
-    for (int b = 0; b < 32; ++b) {
-      const uint32_t e = lut[(by[b >> 2] >> (8 * (b & 3))) & 0xFFu];
-      const bool in = b < nb;
-      bad |= in && e == 0xFFFFu;
-      const uint32_t mm = in ? (e & 31u) : 0u, ss = in ? ((e >> 5) & 31u) : 0u;
-      const int w = (5 * b) >> 5, o = (5 * b) & 31;
-      m[w] |= mm << o;
-      s[w] |= ss << o;
-      if (o > 27) {
-        m[w + 1] |= mm >> (32 - o);
-        s[w + 1] |= ss >> (32 - o);
+      for (int b = 0; b < 32; ++b) {
+        const uint32_t e = lut[(by[b >> 2] >> (8 * (b & 3))) & 0xFFu];
+        eor |= (full || b < nb) ? e : 0u;
+        const int k = (5 * b) >> 4, o = (5 * b) & 15;
+        if (o <= 11) {
+          W[k] += e << o;
+        } else {
+          // low parts stay in group k (mask bits o..15, sign bits 16+o..31), high parts open k+1
+          W[k] += (e << o) & (0x0000FFFFu | (0xFFFFFFFFu << (16 + o)));
+          W[k + 1] += ((e & 31u) >> (16 - o)) | ((((e >> 16) & 31u) >> (16 - o)) << 16);
+        }
       }
-    }
-    uint32_t* rowo = outw + (size_t)rr * 2 * KW;
+      uint32_t m[5], s[5];
 #pragma unroll
-    for (int u = 0; u < 5; ++u) {
-      const int w = 5 * i + u;
-      if (w < KW) {
-        rowo[w] = to_mask_order(m[u]);
-        const uint32_t sp = to_mask_order(s[u]);
-        rowo[KW + w] = (sp << 1) | (sp >> 31);     // the sign bit sits one above its mask bit
+      for (int u = 0; u < 5; ++u) {
+        m[u] = __byte_perm(W[2 * u], W[2 * u + 1], 0x5410);   // low halves: mask bits of trits 32u ..
+        s[u] = __byte_perm(W[2 * u], W[2 * u + 1], 0x7632);   // high halves: their sign bits
       }
+      bad |= (eor >> 31) != 0u;
+      uint32_t* rowo = outw + (size_t)rr * 2 * KW;
+#pragma unroll
+      for (int u = 0; u < 5; ++u) {
+        const int w = 5 * i + u;
+        if (w < KW) {
+          rowo[w] = to_mask_order(m[u]);
+          const uint32_t sp = to_mask_order(s[u]);
+          rowo[KW + w] = (sp << 1) | (sp >> 31);     // the sign bit sits one above its mask bit
+        }
+      }
+      rr += eq;
+      i += er;
+      if (i >= rpr) { i -= rpr; ++rr; }
     }
   }
   if (__any_sync(0xFFFFFFFFu, bad) && (threadIdx.x & 31) == 0) set_flag(flag);
@@ -260,7 +287,7 @@ void base3_plan(int32_t K, int& rows, size_t& smem) {
   const int rb = (K + 4) / 5, KW = K / 32, rpr = (KW + 4) / 5;
   rows = kB3StageBytes / rb;
   if (rows < 1) rows = 1;
-  smem = 512 + (size_t)rows * rpr * kB3Slot + (size_t)rows * K / 4;
+  smem = 1024 + (size_t)rows * rpr * kB3Slot + (size_t)rows * K / 4;
 }
 
 cudaError_t base3_smem_attr(const void* fn, size_t smem, size_t& set) {
