@@ -110,9 +110,10 @@ __device__ __forceinline__ void store_operand_half(uint32_t* slot, int h, uint4 
 
 // ---------------------------------------------------------------------------------------------
 // Operand columns of a segment. M = 1 (mp == 1): the nc columns are the limbs L2, L1, L0 (bf16
-// mode) or q (int8 mode). M >= 2 (mp = 8 or 16 token slots): int8 mode column m = token m; bf16
-// mode column l * mp + m = limb l of token m, so each MMA group of 8 columns holds one limb of
-// eight tokens and a lane ends up with all three limbs of the tokens it owns.
+// mode) or q (int8 mode). M >= 2: int8 mode (mp = 8 or 16 token slots) column m = token m; bf16
+// mode column l * mp + m = limb l of token m. With mp = 8 or 16 each MMA group of 8 columns holds
+// one limb of eight tokens and a lane ends up with all three limbs of the tokens it owns; with
+// mp = 2 or 4 the 6 or 12 columns fill one or two groups and the epilogue gathers the limbs.
 __host__ __device__ constexpr int seg_cols(int mode, int mp) { return mp == 1 ? (mode == 0 ? 3 : 1) : (mode == 0 ? 3 * mp : mp); }
 // Segment words: columns, then the column sums over all of K, then E per token slot, padded to 16 B.
 __host__ __device__ constexpr int seg_words(int mode, int mp) {
@@ -227,17 +228,21 @@ __global__ void __launch_bounds__(256) k_batch_prep(const __grid_constant__ Batc
 }
 
 // ---------------------------------------------------------------------------------------------
-// MODE: 0 bf16 / 1 int8 activations; MP: token slots (1, 8 or 16); TPW: tiles per consumer warp;
-// CW: consumer warps.
+// MODE: 0 bf16 / 1 int8 activations; MP: token slots (1, 2, 4, 8 or 16; 2 and 4 in bf16 mode
+// only); TPW: tiles per consumer warp; CW: consumer warps.
 template <int MODE, int MP, int TPW, int CW>
 __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_constant__ BatchParams p) {
   constexpr int kCW = CW;
   constexpr int kBoxRows = box_rows(CW);
   constexpr int kBoxBytes = box_bytes(CW);
   extern __shared__ __align__(1024) uint8_t smem[];
+  // PACK: bf16 mode with 2 or 4 token slots, whose 3 * MP limb columns share one or two MMA
+  // groups (a lane then holds limbs of several tokens; the epilogue gathers them by shuffles)
+  constexpr bool PACK = MP == 2 || MP == 4;
+  static_assert(!PACK || MODE == 0, "packed token slots are a bf16-mode shape");
   constexpr int NCOL = seg_cols(MODE, MP);
-  constexpr int G = MP == 1 ? 1 : NCOL / 8;                 // MMA column groups
-  constexpr int JJ = MP == 1 ? 1 : MP / 8;                  // groups per limb (token octets)
+  constexpr int G = MP == 1 ? 1 : (NCOL + 7) / 8;           // MMA column groups
+  constexpr int JJ = (MP == 1 || PACK) ? 1 : MP / 8;        // groups per limb (token octets)
   constexpr int kStageRowsT = kBoxRows * TPW;
   constexpr int kWStageBytesT = TPW * kBoxBytes;
   const int S = p.stages;
@@ -296,7 +301,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
     pdl_wait();
     // 2. every stage: its operand segment and, past the first S, its weights once the slot is free
     it = first_item; rb = first_rb; part = first_part;
-    int s = 0;
+    int s = 0, nq = 0;
     uint32_t ph = 0;
     for (int q = 0; q < n && ok; ++q) {
       const BatchItem& B = p.items[it];
@@ -311,6 +316,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
           tma_load_3d(dst + b * kBoxBytes, &p.tmap[it], part * kPartWords, rb * kStageRowsT + b * kBoxRows, 0, bar);
       }
       bulk_g2s(dst + kWStageBytesT, p.xprep + B.xoff + (size_t)part * p.seg_bytes, (uint32_t)p.seg_bytes, bar);
+      ++nq;
       if (++part == B.kp) {
         part = 0;
         if (++rb == B.units) { rb = 0; ++it; }
@@ -318,13 +324,13 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
       if (++s == S) { s = 0; ph ^= 1u; }
     }
     if (!ok) atomicExch(&g_batch_latch, 5);
-    // do not exit with copies in flight: wait for the last min(n, S) stages to land
-    if (ok) {
-      for (int q = n > S ? n - S : 0; q < n; ++q) {
-        if (!mbar_wait(full0 + 8 * (q % S), (uint32_t)((q / S) & 1))) {
-          atomicExch(&g_batch_latch, 5);
-          break;
-        }
+    // do not exit with copies in flight (on the error path too): wait for the last nq stages to
+    // land. A wait gives up only at some q >= S, before that stage's weights are issued, so every
+    // copy in flight belongs to one of the stages [0, nq) issued in full.
+    for (int q = nq > S ? nq - S : 0; q < nq; ++q) {
+      if (!mbar_wait(full0 + 8 * (q % S), (uint32_t)((q / S) & 1))) {
+        atomicExch(&g_batch_latch, 5);
+        break;
       }
     }
     return;
@@ -333,10 +339,13 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
   // ====================== consumers ======================
   const int g = lane >> 2, t = lane & 3;
   // operand column of group j this lane feeds: M = 1: the lane's limb (rows g >= nc repeat column 0)
-  const int col0 = MP == 1 ? (g < NCOL ? g : 0) : g;
+  // columns past NCOL (M = 1, PACK) repeat a real column; their sums are never read
+  const int col0 = (MP == 1 || PACK) ? (g < NCOL ? g : 0) : g;
+  const int col1 = 8 + g < NCOL ? 8 + g : 8;                // PACK, MP = 4: group 1
   // byte offsets inside a slot
   const uint32_t wofs = (uint32_t)((warp * 16 + g) * kPartWords * 4 + t * 16);   // plane 0, row g
   const uint32_t xofs = (uint32_t)(kWStageBytesT + (col0 * kColWords + t * 8) * 4);
+  const uint32_t xofs1 = (uint32_t)(kWStageBytesT + (col1 * kColWords + t * 8) * 4);
   const uint32_t mofs = (uint32_t)(kWStageBytesT + NCOL * kColWords * 4);
   const int M = p.M;
   constexpr int NCOLP = 8 * G;                              // scratch columns per row
@@ -422,8 +431,9 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
 #pragma unroll
         for (int j = 0; j < G; ++j) {
           // (b0, b1) of fields 0, 1 and of fields 2, 3
-          const uint4 x01 = lds128(st + xofs + (j * 8 * kColWords) * 4 + e * 128);
-          const uint4 x23 = lds128(st + xofs + (j * 8 * kColWords) * 4 + e * 128 + 16);
+          const uint32_t xo = (PACK && j == 1) ? xofs1 : xofs + (uint32_t)(j * 8 * kColWords) * 4;
+          const uint4 x01 = lds128(st + xo + e * 128);
+          const uint4 x23 = lds128(st + xo + e * 128 + 16);
 #pragma unroll
           for (int a = 0; a < TPW; ++a)
 #pragma unroll
@@ -445,6 +455,20 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
                 tot[0][1][0] = (int)m4.y;
                 tot[0][2][0] = (int)m4.z;
                 Etok[0][0] = MODE == 0 ? (int)m4.w : 0;
+              }
+            } else if (PACK) {
+              // lane t writes token t: its three column sums and E
+              if (jj == 0 && b == 0) {
+                const int m = t < MP ? t : 0;
+#pragma unroll
+                for (int l = 0; l < 3; ++l) {
+                  uint32_t v;
+                  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(st + mofs + 4u * (uint32_t)(l * MP + m)));
+                  tot[0][l][0] = (int)v;
+                }
+                uint32_t ev;
+                asm volatile("ld.shared.u32 %0, [%1];" : "=r"(ev) : "r"(st + mofs + 4u * (uint32_t)(NCOL + m)));
+                Etok[0][0] = (int)ev;
               }
             } else {
               const int m = 8 * jj + 2 * t + b;
@@ -491,7 +515,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const int col = 8 * j + 2 * t + (q & 1);
-            if (MP > 1 || col < NCOL)
+            if (col < NCOL)
               atomicAdd(&sums[(a * kBoxRows + warp * 16 + g + 8 * (q >> 1)) * NCOLP + col], V[a][j][q]);
           }
       __threadfence();
@@ -508,7 +532,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               const int col = 8 * j + 2 * t + (q & 1);
-              if (MP > 1 || col < NCOL)
+              if (col < NCOL)
                 V[a][j][q] = __ldcg(&sums[(a * kBoxRows + warp * 16 + g + 8 * (q >> 1)) * NCOLP + col]);
             }
       } else {
@@ -548,6 +572,30 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
                 const long long D = S2 * 65536 + S1 * 256 + S0;
                 B.y[row] = (float)((double)D * exp2_i(Etok[0][0] - kLimbFrac) * (double)f16_bits_to_float(sc_bits[a][h]));
               }
+            }
+          }
+        }
+      } else if (PACK) {
+        // limb l of token m sits in column c = l * MP + m: group c / 8, held by quad lane
+        // (c % 8) / 2 as half c % 2 of its row pair; lane t = m gathers its token's limbs
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int row = r0 + 8 * h;
+#pragma unroll
+          for (int m = 0; m < MP; ++m) {
+            int L[3];
+#pragma unroll
+            for (int l = 0; l < 3; ++l) {
+              const int c = l * MP + m;
+              L[l] = __shfl_sync(0xFFFFFFFFu, V[a][c >> 3][2 * h + (c & 1)], (lane & ~3) | ((c & 7) >> 1));
+            }
+            if (t == m && m < M && row < B.N) {
+              const long long S2 = L[0] - 2LL * tot[0][0][0];
+              const long long S1 = L[1] - 2LL * tot[0][1][0];
+              const long long S0 = L[2] - 2LL * tot[0][2][0];
+              const long long D = S2 * 65536 + S1 * 256 + S0;
+              B.y[(size_t)m * B.N + row] =
+                  (float)((double)D * exp2_i(Etok[0][0] - kLimbFrac) * (double)f16_bits_to_float(sc_bits[a][h]));
             }
           }
         }
@@ -601,9 +649,21 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // Token slots, tiles per warp and consumer warps for M rows: the accumulators (tiles x groups x
 // 16 registers) stay at or under 96 registers.
 void batch_shape(int mode, int M, int& mp, int& tpw, int& cw) {
-  mp = M == 1 ? 1 : (M <= 8 ? 8 : 16);
-  tpw = (mode == 0 && M > 1) ? 1 : 2;
-  cw = M == 1 ? 12 : 11;
+  if (M == 1 || (mode == 0 && M == 2)) {       // one MMA group: 1 or 3 columns, or 2 x 3 limbs
+    mp = M;
+    tpw = 2;
+    cw = 12;
+    return;
+  }
+  if (mode == 0 && M <= 4) {                    // 4 x 3 limbs in two groups
+    mp = 4;
+    tpw = 2;
+    cw = 11;
+    return;
+  }
+  mp = M <= 8 ? 8 : 16;
+  tpw = mode == 0 ? 1 : 2;
+  cw = 11;
 }
 
 template <int MODE, int MP, int TPW, int CW>
@@ -631,7 +691,7 @@ bool plan_batch(BatchParams& p, const uint32_t* const* planes, size_t& smem, siz
   p.nc = seg_cols(p.mode, mp);
   p.seg_bytes = seg_words(p.mode, mp) * 4;
   const int stage_rows = kBoxRows * tpw;
-  const int ncolp = mp == 1 ? 8 : seg_cols(p.mode, mp);   // scratch columns: 8 per MMA group
+  const int ncolp = 8 * ((seg_cols(p.mode, mp) + 7) / 8); // scratch columns: 8 per MMA group
   PFN_cuTensorMapEncodeTiled_v12000 encode = encode_fn();
   if (!encode) return false;
   long long total_cost = 0;
@@ -777,6 +837,8 @@ cudaError_t launch_batch(const BatchParams& p, size_t smem, bool pdl, cudaStream
   cfg.dynamicSmemBytes = smem;
   if (p.mode == 0) {
     if (p.mp == 1) return launch_stream_kernel<0, 1, 2, 12>(cfg, p, smem);
+    if (p.mp == 2) return launch_stream_kernel<0, 2, 2, 12>(cfg, p, smem);
+    if (p.mp == 4) return launch_stream_kernel<0, 4, 2, 11>(cfg, p, smem);
     if (p.mp == 8) return launch_stream_kernel<0, 8, 1, 11>(cfg, p, smem);
     return launch_stream_kernel<0, 16, 1, 11>(cfg, p, smem);
   }

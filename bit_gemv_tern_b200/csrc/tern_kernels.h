@@ -69,7 +69,7 @@ struct BatchParams {
   int32_t mode;           // 0 = bf16 activations (three int8 limbs), 1 = int8
   int32_t nc;             // operand columns of a segment
   int32_t M;              // activation rows (tokens), 1..16
-  int32_t mp;             // token slots: 1, 8 or 16
+  int32_t mp;             // token slots: 1, 2 / 4 (bf16 mode), 8 or 16
   int32_t tpw;            // tiles of 16 rows per consumer warp
   int32_t cw;             // consumer warps
   int32_t total_units;

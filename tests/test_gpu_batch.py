@@ -138,7 +138,7 @@ def _build_m(seed, shapes, M, act):
 SHAPES_M = [(37, 384), (200, 640), (3072, 1024), (1024, 3072), (4096, 12288), (24576, 4096)]
 
 
-@pytest.mark.parametrize("M", [2, 4, 7, 8, 9, 16])
+@pytest.mark.parametrize("M", [2, 3, 4, 5, 7, 8, 9, 16])
 @pytest.mark.parametrize("mode", ["bf16", "int8"])
 def test_gemm_batch_small_m_matches_oracle(mode, M):
     """Every token row of every item: int8 bit-exact, bf16 within the tolerance (sampled rows of
