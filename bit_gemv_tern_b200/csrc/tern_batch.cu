@@ -120,8 +120,11 @@ __host__ __device__ constexpr int seg_words(int mode, int mp) {
   return (seg_cols(mode, mp) * kColWords + seg_cols(mode, mp) + mp + 3) & ~3;
 }
 
-// prep: one CTA per (item, token slot). Block layout: kp segments of seg_bytes.
-__global__ void __launch_bounds__(256) k_batch_prep(const __grid_constant__ BatchParams p) {
+// prep: one CTA of kPrepThreads per (item, token slot), wide enough that each pass over an
+// activation of up to 8192 (int8: 16384) elements is a single round of loads. Block layout: kp
+// segments of seg_bytes.
+constexpr int kPrepThreads = 1024;
+__global__ void __launch_bounds__(kPrepThreads) k_batch_prep(const __grid_constant__ BatchParams p) {
   const BatchItem& it = p.items[blockIdx.x];
   const int m = blockIdx.y;                          // token slot (< mp)
   uint32_t* blk = reinterpret_cast<uint32_t*>(p.xprep + it.xoff);
@@ -132,7 +135,7 @@ __global__ void __launch_bounds__(256) k_batch_prep(const __grid_constant__ Batc
   int colof[3];
   for (int l = 0; l < 3; ++l) colof[l] = mp == 1 ? l : l * mp + m;
   const bool live = m < p.M;
-  __shared__ float red[8];
+  __shared__ float red[kPrepThreads / 32];
   __shared__ int sums[3];
   __shared__ int Esh;
   pdl_wait();
@@ -142,10 +145,17 @@ __global__ void __launch_bounds__(256) k_batch_prep(const __grid_constant__ Batc
     const int nct = gridDim.x * gridDim.y, ct = blockIdx.y * gridDim.x + blockIdx.x;
     for (int i = ct * blockDim.x + threadIdx.x; i < p.scratch_words; i += nct * blockDim.x) scr[i] = 0u;
   }
-  // this token's columns (and its meta words) start at zero: the K tail of the last part stays so
-  for (int i = threadIdx.x; i < KP * nl * kColWords; i += blockDim.x) {
-    const int part = i / (nl * kColWords), r = i % (nl * kColWords);
-    blk[part * segw + colof[r / kColWords] * kColWords + r % kColWords] = 0u;
+  // words of this token's columns that the loop below does not write read as zero: all of them
+  // for an empty token slot, else the words of the last part past K (K % 512 != 0)
+  {
+    const int wl = live ? K / 32 - 16 * (KP - 1) : 0;      // words written in the last part
+    const int p0 = live ? KP - 1 : 0;                       // first part with unwritten words
+    const int per_part = (16 - wl) * 8;                     // unwritten operand words per column
+    for (int i = threadIdx.x; i < (KP - p0) * nl * per_part; i += blockDim.x) {
+      const int part = p0 + i / (nl * per_part), r = i % (nl * per_part);
+      const int c = r / per_part, j = r % per_part;
+      blk[part * segw + colof[c] * kColWords + part_slot(wl + j / 8) + j % 8] = 0u;
+    }
   }
   if (threadIdx.x < 3) sums[threadIdx.x] = 0;
   if (threadIdx.x == 0) Esh = 0;
@@ -165,7 +175,7 @@ __global__ void __launch_bounds__(256) k_batch_prep(const __grid_constant__ Batc
     __syncthreads();
     if (threadIdx.x == 0) {
       float mx = red[0];
-      for (int i = 1; i < 8; ++i) mx = fmaxf(mx, red[i]);
+      for (int i = 1; i < kPrepThreads / 32; ++i) mx = fmaxf(mx, red[i]);
       int E = 0;
       if (mx > 0.0f) {
         frexpf(mx, &E);                              // mx < 2^E
@@ -823,7 +833,7 @@ cudaError_t launch_batch(const BatchParams& p, size_t smem, bool pdl, cudaStream
   cfg.stream = st;
   // 1. operand segments: one CTA per (item, token slot)
   cfg.gridDim = dim3(p.count, p.mp, 1);
-  cfg.blockDim = dim3(256, 1, 1);
+  cfg.blockDim = dim3(kPrepThreads, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cudaError_t e = cudaLaunchKernelEx(&cfg, k_batch_prep, p);
   if (e != cudaSuccess) return e;
