@@ -96,12 +96,13 @@ cudaError_t read_and_clear_batch_latch(int* out);
 
 // Prefill dense contraction on tcgen05 (tern_prefill.cu).
 struct PrefillParams {
-  CUtensorMap xmap;       // X bf16 [M][K], boxes of 64 x 128, 128-byte swizzle
+  CUtensorMap xmap;       // X bf16 [M][K], boxes of 64 x (128 * halves), 128-byte swizzle
   const uint32_t* planes;
   const uint16_t* scale;
   float* Y;               // [M][N]
   int32_t M, N, K;
   int32_t vec_store;      // Y rows 16-byte aligned (N % 4 == 0 and Y aligned): 128-bit stores
+  int32_t halves;         // 128-token halves per tile (1 or 2), set by plan_prefill
 };
 bool plan_prefill(PrefillParams& p, const uint16_t* X, int& grid, size_t& smem);
 cudaError_t launch_prefill(const PrefillParams& p, int grid, size_t smem, cudaStream_t st);

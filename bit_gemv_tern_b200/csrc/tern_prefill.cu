@@ -9,16 +9,20 @@
 // tensor cores read them (weights packed at rest, aiatolah.com "Neutrino-1 8B: modelo ternario
 // ...", second paragraph); the products by +-1 / 0 are exact (origotech.dev Figure I).
 //
-// One persistent CTA per SM walks output tiles of BM = 128 tokens x BN = 256 weight rows:
-//   warp 0      TMA producer: X tile (128 x 64 bf16, 128-byte swizzle) per K stage;
-//   warp 1      allocates 512 TMEM columns (two fp32 accumulators of 128 x 256) and one lane
-//               issues tcgen05.mma kind::f16 (A = X tile, B = expanded weights, both K-major);
-//               tcgen05.commit frees a stage when the MMAs reading it are done;
+// One persistent CTA per SM walks output tiles of H x 128 tokens x BN = 256 weight rows:
+//   warp 0      TMA producer: X tile (H x 128 x 64 bf16, 128-byte swizzle) per K stage;
+//   warp 1      allocates 512 TMEM columns and one lane issues tcgen05.mma kind::f16 (A = X,
+//               B = expanded weights, both K-major; M = 128 per instruction, one instruction per
+//               128-token half); tcgen05.commit frees a stage when the MMAs reading it are done;
 //   warps 2..9  expand the tile's 256 weight rows x 64 trits to bf16 (2.0 * t, the field decode
 //               of tern_device.cuh) in the same swizzled layout the tensor core reads;
 //   warps 10..13 epilogue: tcgen05.ld of the accumulator their TMEM lane quarter owns, times
-//               0.5 * scale[n], stored to Y; the second accumulator lets the next tile's MMAs run
-//               meanwhile.
+//               0.5 * scale[n], stored to Y.
+// H = 1: two 128 x 256 fp32 accumulators, so the next tile's MMAs run during the epilogue.
+// H = 2: both halves of a 256-token tile read every expanded weight stage, which halves the
+//        expansion work and cuts shared-memory traffic per flop by a sixth; the two halves' 128 x
+//        256 accumulators fill TMEM, so the tensor core waits for each tile's epilogue. The host
+//        takes H = 2 when its tiles still fill the GPU.
 // Every mbarrier wait is bounded; a kernel that gives up latches TERN_ETIMEOUT, drains what it
 // issued (bounded), frees its TMEM and returns.
 #include <cstdint>
@@ -35,11 +39,10 @@ __device__ int g_prefill_latch = 0;
 
 namespace {
 
-constexpr int BM = 128;                          // tokens per tile: UMMA M, TMEM lanes
+constexpr int BM = 128;                          // tokens per MMA (tile half): UMMA M, TMEM lanes
 constexpr int BN = 256;                          // weight rows per tile: UMMA N, accumulator columns
 constexpr int BK = 64;                           // K per stage: one 128-byte swizzle span of bf16
-constexpr int kStages = 4;
-constexpr int kABytes = BM * BK * 2;             // 16 KB
+constexpr int kHalfBytes = BM * BK * 2;          // 16 KB: one 128-token X tile of a stage
 constexpr int kBBytes = BN * BK * 2;             // 32 KB
 #ifndef TERN_PREFILL_DEC_WARPS
 #define TERN_PREFILL_DEC_WARPS 8
@@ -48,13 +51,22 @@ constexpr int kDecWarps = TERN_PREFILL_DEC_WARPS, kEpiWarps = 4;
 constexpr int kRowsPerDec = BN / (kDecWarps * 32);   // weight rows expanded per decoder thread
 static_assert(kRowsPerDec * kDecWarps * 32 == BN, "decoder rows");
 constexpr int kPrefillThreads = (2 + kDecWarps + kEpiWarps) * 32;
-constexpr int kTmemCols = 2 * BN;                // two accumulators
+constexpr int kTmemCols = 2 * BN;                // two 128 x 256 fp32 accumulators
 constexpr uint32_t kWaitTries = 1u << 13;
-// smem: [A stages][B stages][barriers + TMEM address], stages 1024-byte aligned
-constexpr int kSmemA = 0;
-constexpr int kSmemB = kStages * kABytes;
-constexpr int kSmemBar = kSmemB + kStages * kBBytes;
-constexpr int kSmemBytes = kSmemBar + 256 + kEpiWarps * BN * 4 + 1024;  // + barriers, scales, alignment slack
+// Shape of the kernel for H 128-token halves per tile.
+//   smem: [A stages][B stages][barriers + TMEM address][epilogue scales], stages 1024-byte aligned
+template <int H>
+struct Shape {
+  static constexpr int kTileM = BM * H;                    // tokens per tile
+  static constexpr int kStages = H == 1 ? 4 : 3;
+  static constexpr int kABytes = H * kHalfBytes;
+  static constexpr int kAccBufs = H == 1 ? 2 : 1;          // accumulator buffers (tiles in flight)
+  static constexpr int kSmemA = 0;
+  static constexpr int kSmemB = kStages * kABytes;
+  static constexpr int kSmemBar = kSmemB + kStages * kBBytes;
+  static constexpr int kSmemBytes = kSmemBar + 256 + kEpiWarps * BN * 4 + 1024;  // + barriers, scales, slack
+  static_assert(kAccBufs * H * BN == kTmemCols, "TMEM columns");
+};
 
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator, A and B bf16, both
 // K-major, N = 256, M = 128.
@@ -141,7 +153,11 @@ __device__ __forceinline__ uint32_t dec2(uint32_t wa, uint32_t wb) {
   return dec_bf16<A>(wa, wb);
 }
 
+template <int H>
 __global__ void __launch_bounds__(kPrefillThreads, 1) k_prefill(const __grid_constant__ PrefillParams p) {
+  using SH = Shape<H>;
+  constexpr int kStages = SH::kStages, kABytes = SH::kABytes, kTileM = SH::kTileM, kAccBufs = SH::kAccBufs;
+  constexpr int kSmemA = SH::kSmemA, kSmemB = SH::kSmemB, kSmemBar = SH::kSmemBar;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the swizzled tiles
   const uint32_t raw = smem_u32(smem_raw);
@@ -154,7 +170,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) k_prefill(const __grid_con
   uint32_t* tmem_slot_ptr = reinterpret_cast<uint32_t*>(smem_raw + (tmem_slot - raw));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tiles_n = (p.N + BN - 1) / BN, tiles_m = (p.M + BM - 1) / BM;
+  const int tiles_n = (p.N + BN - 1) / BN, tiles_m = (p.M + kTileM - 1) / kTileM;
   const int tiles = tiles_m * tiles_n;
   const int KT = p.K / BK;
 
@@ -193,7 +209,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) k_prefill(const __grid_con
           const int s = q % kStages;
           if (q >= kStages && !(ok = mbar_wait(empty + 8 * s, ((q / kStages) - 1) & 1))) break;
           mbar_arrive_expect_tx(a_full + 8 * s, kABytes);
-          tma_load_2d(sA + s * kABytes, &p.xmap, kt * BK, mt * BM, a_full + 8 * s);
+          tma_load_2d(sA + s * kABytes, &p.xmap, kt * BK, mt * kTileM, a_full + 8 * s);
         }
       }
       // do not leave with copies in flight (bounded, also after a give-up)
@@ -205,10 +221,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) k_prefill(const __grid_con
     if (lane == 0) {
       int q = 0, tl = 0;
       for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++tl) {
-        const int acc = tl & 1;
-        if (tl >= 2 && !(ok = mbar_wait(acc_empty + 8 * acc, ((tl >> 1) - 1) & 1))) break;
+        const int acc = tl % kAccBufs, use = tl / kAccBufs;
+        if (use >= 1 && !(ok = mbar_wait(acc_empty + 8 * acc, (use - 1) & 1))) break;
         tc_fence_after();
-        const uint32_t d = tmem + (uint32_t)(acc * BN);
+        const uint32_t d = tmem + (uint32_t)(acc * H * BN);
         for (int kt = 0; kt < KT; ++kt, ++q) {
           const int s = q % kStages;
           const uint32_t ph = (q / kStages) & 1;
@@ -217,8 +233,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) k_prefill(const __grid_con
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
-            umma_bf16(d, umma_desc(sA + s * kABytes + 32 * k), umma_desc(sB + s * kBBytes + 32 * k), kIdesc,
-                      (kt > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+            for (int h = 0; h < H; ++h)                 // every half reads the same weight stage
+              umma_bf16(d + (uint32_t)(h * BN), umma_desc(sA + s * kABytes + h * kHalfBytes + 32 * k),
+                        umma_desc(sB + s * kBBytes + 32 * k), kIdesc, (kt > 0 || k > 0) ? 1u : 0u);
           umma_commit(empty + 8 * s);                 // the stage is free once these MMAs are done
         }
         if (!ok) break;
@@ -305,7 +323,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) k_prefill(const __grid_con
     int tl = 0;
     for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++tl) {
       const int mt = tile / tiles_n, nt = tile % tiles_n;
-      const int acc = tl & 1;
+      const int acc = tl % kAccBufs, use = tl / kAccBufs;
       __syncwarp();
 #pragma unroll
       for (int i = 0; i < BN / 32; ++i) {
@@ -313,32 +331,35 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) k_prefill(const __grid_con
         hs[lane + 32 * i] = n < p.N ? 0.5f * f16_bits_to_float(p.scale[n]) : 0.0f;
       }
       __syncwarp();
-      if (!(ok = mbar_wait(acc_full + 8 * acc, (tl >> 1) & 1))) break;
+      if (!(ok = mbar_wait(acc_full + 8 * acc, use & 1))) break;
       tc_fence_after();
-      const int m = mt * BM + quarter * 32 + lane;
-      float* yrow = p.Y + (size_t)(m < p.M ? m : 0) * p.N;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN + 32 * c), r);
-        const int n0 = nt * BN + 32 * c;
-        const float* sc = hs + 32 * c;
-        if (m < p.M) {
-          if (p.vec_store && n0 + 32 <= p.N) {
+      for (int h = 0; h < H; ++h) {
+        const int m = mt * kTileM + h * BM + quarter * 32 + lane;
+        float* yrow = p.Y + (size_t)(m < p.M ? m : 0) * p.N;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)((acc * H + h) * BN + 32 * c), r);
+          const int n0 = nt * BN + 32 * c;
+          const float* sc = hs + 32 * c;
+          if (m < p.M) {
+            if (p.vec_store && n0 + 32 <= p.N) {
 #pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-              const float4 s4 = *reinterpret_cast<const float4*>(sc + j);
-              float4 v;
-              v.x = __uint_as_float(r[j + 0]) * s4.x;
-              v.y = __uint_as_float(r[j + 1]) * s4.y;
-              v.z = __uint_as_float(r[j + 2]) * s4.z;
-              v.w = __uint_as_float(r[j + 3]) * s4.w;
-              *reinterpret_cast<float4*>(yrow + n0 + j) = v;
+              for (int j = 0; j < 32; j += 4) {
+                const float4 s4 = *reinterpret_cast<const float4*>(sc + j);
+                float4 v;
+                v.x = __uint_as_float(r[j + 0]) * s4.x;
+                v.y = __uint_as_float(r[j + 1]) * s4.y;
+                v.z = __uint_as_float(r[j + 2]) * s4.z;
+                v.w = __uint_as_float(r[j + 3]) * s4.w;
+                *reinterpret_cast<float4*>(yrow + n0 + j) = v;
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (n0 + j < p.N) yrow[n0 + j] = __uint_as_float(r[j]) * sc[j];
             }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (n0 + j < p.N) yrow[n0 + j] = __uint_as_float(r[j]) * sc[j];
           }
         }
       }
@@ -375,29 +396,39 @@ bool plan_prefill(PrefillParams& p, const uint16_t* X, int& grid, size_t& smem) 
   if (p.M < 1 || p.N < 1 || p.K < BK || p.K % 128) return false;
   PFN_cuTensorMapEncodeTiled_v12000 encode = encode_fn();
   if (!encode) return false;
+  // two 128-token halves per tile while such tiles still give every SM one (they halve the weight
+  // expansion per flop); 128-token tiles otherwise
+  const int tiles_n = (p.N + BN - 1) / BN;
+  p.halves = (long long)((p.M + 2 * BM - 1) / (2 * BM)) * tiles_n >= 148 ? 2 : 1;
+  const int tile_m = BM * p.halves;
   const cuuint64_t dims[2] = {(cuuint64_t)p.K, (cuuint64_t)p.M};
   const cuuint64_t strides[1] = {(cuuint64_t)p.K * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)BM};
+  const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)tile_m};
   const cuuint32_t estr[2] = {1, 1};
   if (encode(&p.xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return false;
-  const int tiles = ((p.M + BM - 1) / BM) * ((p.N + BN - 1) / BN);
-  grid = tiles < 148 ? tiles : 148;
-  smem = kSmemBytes;
+  const long long tiles = (long long)((p.M + tile_m - 1) / tile_m) * tiles_n;
+  grid = tiles < 148 ? (int)tiles : 148;
+  smem = p.halves == 2 ? Shape<2>::kSmemBytes : Shape<1>::kSmemBytes;
   return true;
 }
 
-cudaError_t launch_prefill(const PrefillParams& p, int grid, size_t smem, cudaStream_t st) {
+template <int H>
+cudaError_t launch_prefill_h(const PrefillParams& p, int grid, size_t smem, cudaStream_t st) {
   static int set = 0;
   if (!set) {
-    cudaError_t e = cudaFuncSetAttribute(k_prefill, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(k_prefill<H>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     set = 1;
   }
-  k_prefill<<<grid, kPrefillThreads, smem, st>>>(p);
+  k_prefill<H><<<grid, kPrefillThreads, smem, st>>>(p);
   return cudaGetLastError();
+}
+
+cudaError_t launch_prefill(const PrefillParams& p, int grid, size_t smem, cudaStream_t st) {
+  return p.halves == 2 ? launch_prefill_h<2>(p, grid, smem, st) : launch_prefill_h<1>(p, grid, smem, st);
 }
 
 cudaError_t read_and_clear_prefill_latch(int* out) {

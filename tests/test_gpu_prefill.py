@@ -23,8 +23,10 @@ def _prefill(W, X):
     return host(Y).reshape(M, W.N)
 
 
+# The last two shapes give at least 148 tiles of 256 tokens x 256 rows, so they run the two-halves
+# kernel (both 128-token halves of a tile share each expanded weight stage) with a ragged M and N.
 @pytest.mark.parametrize("N,K,M", [(256, 128, 128), (512, 1024, 200), (300, 640, 130), (1024, 4096, 256),
-                                   (256, 12288, 64), (4096, 128, 1)])
+                                   (256, 12288, 64), (4096, 128, 1), (18944, 128, 300), (18901, 256, 257)])
 def test_prefill_full(N, K, M):
     W, t, s = make_matrix(51, N + K, N, K)
     X = synth.activations(51, M + K, M, K)
