@@ -52,6 +52,7 @@ constexpr int kRowsPerDec = BN / (kDecWarps * 32);   // weight rows expanded per
 static_assert(kRowsPerDec * kDecWarps * 32 == BN, "decoder rows");
 constexpr int kPrefillThreads = (2 + kDecWarps + kEpiWarps) * 32;
 constexpr int kTmemCols = 2 * BN;                // two 128 x 256 fp32 accumulators
+constexpr int kStageTile = 32 * 32 * 4;          // epilogue staging: 32 rows x 32 fp32 columns per warp
 constexpr uint32_t kWaitTries = 1u << 13;
 // Shape of the kernel for H 128-token halves per tile.
 //   smem: [A stages][B stages][barriers + TMEM address][epilogue scales], stages 1024-byte aligned
@@ -64,7 +65,8 @@ struct Shape {
   static constexpr int kSmemA = 0;
   static constexpr int kSmemB = kStages * kABytes;
   static constexpr int kSmemBar = kSmemB + kStages * kBBytes;
-  static constexpr int kSmemBytes = kSmemBar + 256 + kEpiWarps * BN * 4 + 1024;  // + barriers, scales, slack
+  // + barriers, epilogue scales, epilogue staging tiles, alignment slack
+  static constexpr int kSmemBytes = kSmemBar + 256 + kEpiWarps * BN * 4 + kEpiWarps * kStageTile + 1024;
   static_assert(kAccBufs * H * BN == kTmemCols, "TMEM columns");
 };
 
@@ -104,6 +106,11 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 }
 __device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a) : "memory");
+  return v;
 }
 __device__ __forceinline__ uint4 ldg128(const void* p) {
   uint4 v;
@@ -167,6 +174,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) k_prefill(const __grid_con
   const uint32_t acc_full = sBar + 24 * kStages, acc_empty = acc_full + 16, done_bar = acc_empty + 16;
   const uint32_t tmem_slot = done_bar + 8;
   const uint32_t sScale = sBar + 256;                 // [4 epilogue warps][BN] floats
+  const uint32_t sStage = sScale + kEpiWarps * BN * 4;  // [4 epilogue warps][32 rows][128 B]
   uint32_t* tmem_slot_ptr = reinterpret_cast<uint32_t*>(smem_raw + (tmem_slot - raw));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -343,23 +351,31 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) k_prefill(const __grid_con
           tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)((acc * H + h) * BN + 32 * c), r);
           const int n0 = nt * BN + 32 * c;
           const float* sc = hs + 32 * c;
-          if (m < p.M) {
-            if (p.vec_store && n0 + 32 <= p.N) {
+          if (p.vec_store && n0 + 32 <= p.N) {
+            // through this warp's staging tile (16-byte chunks swizzled by row, conflict-free both
+            // ways), so that every store instruction writes four whole 128-byte rows of Y
+            const uint32_t stg = sStage + (uint32_t)(quarter * kStageTile);
 #pragma unroll
-              for (int j = 0; j < 32; j += 4) {
-                const float4 s4 = *reinterpret_cast<const float4*>(sc + j);
-                float4 v;
-                v.x = __uint_as_float(r[j + 0]) * s4.x;
-                v.y = __uint_as_float(r[j + 1]) * s4.y;
-                v.z = __uint_as_float(r[j + 2]) * s4.z;
-                v.w = __uint_as_float(r[j + 3]) * s4.w;
-                *reinterpret_cast<float4*>(yrow + n0 + j) = v;
-              }
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (n0 + j < p.N) yrow[n0 + j] = __uint_as_float(r[j]) * sc[j];
+            for (int j = 0; j < 8; ++j) {
+              const float4 s4 = *reinterpret_cast<const float4*>(sc + 4 * j);
+              sts128(stg + lane * 128 + ((j ^ (lane & 7)) << 4), __float_as_uint(__uint_as_float(r[4 * j + 0]) * s4.x),
+                     __float_as_uint(__uint_as_float(r[4 * j + 1]) * s4.y),
+                     __float_as_uint(__uint_as_float(r[4 * j + 2]) * s4.z),
+                     __float_as_uint(__uint_as_float(r[4 * j + 3]) * s4.w));
             }
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int rr = 4 * i + (lane >> 3), cj = lane & 7;
+              const uint4 v = lds128(stg + rr * 128 + ((cj ^ (rr & 7)) << 4));
+              const int mm = m - lane + rr;
+              if (mm < p.M) *reinterpret_cast<uint4*>(p.Y + (size_t)mm * p.N + n0 + 4 * cj) = v;
+            }
+            __syncwarp();
+          } else if (m < p.M) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (n0 + j < p.N) yrow[n0 + j] = __uint_as_float(r[j]) * sc[j];
           }
         }
       }
