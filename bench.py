@@ -679,6 +679,9 @@ def extra_rows(stack, torch, tg, hbm_peak, bf16_peak):
     # prefill: M = 4096 tokens through each of the 7 distinct 8B linear shapes (tcgen05)
     out["prefill_8b_m4096"] = prefill_row(torch, tg, bf16_peak)
 
+    # pack of int8 trits into the planes: the seven tensors of one 8B layer per call
+    out["pack_8b_layer"] = pack_row(torch, tg, hbm_peak)
+
     # base-3 transport unpack of all 8B trits (bit-exact expansion into the planes)
     out["base3_unpack_8b"] = base3_row(stack, torch, tg, hbm_peak)
     return out
@@ -759,6 +762,30 @@ class StackView:
         tg.i8_head_gemv_argmax(self.base.head_W, self.base.head_s, self.V, self.d, self.M, tg.TERN_ACT_BF16,
                                self.x[:self.M * self.d], None, self.argmax, self.maxval, None, self.ws,
                                flags=tg.TERN_FLAG_PDL if pdl else 0)
+
+
+def pack_row(torch, tg, hbm_peak):
+    """int8 trits of the seven tensors of one 8B layer (193 MB, > L2) packed into their planes by
+    one tern_pack_batch call; bytes = N*K in + N*K/4 out per tensor."""
+    import synth
+    import synth.cuda as sc
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    items, nb, trits = [], 0, 0
+    for p, N, K in synth.linear_shapes("8b"):
+        t = torch.empty(N * K, dtype=torch.int8, device="cuda")
+        sc.trits_into(t, SEED, synth.tensor_id(1, p), K, synth.trit_probs("8b", 1, p))
+        items.append((t, N, K, torch.empty(N * K // 16, dtype=torch.int32, device="cuda")))
+        nb += N * K + N * K // 4
+        trits += N * K
+    g = capture(lambda i: tg.tern_pack_batch(tg.TERN_SRC_INT8_TRITS, items, flag), 1)
+    g.replay()
+    reps = 10
+    ms = timed_replays([(g, reps)]) / reps
+    assert tg.tern_read_flag(flag) == 0
+    gbs = nb / (ms / 1000.0) / 1e9
+    layers = synth.GEOMETRY["8b"]["layers"]
+    return {"ms": ms, "gbs": gbs, "frac": gbs / hbm_peak, "trits": trits, "bytes": nb, "tensors": len(items),
+            "launches": len(items), "ms_8b_equivalent": ms * layers}
 
 
 def base3_row(stack, torch, tg, hbm_peak):

@@ -16,37 +16,7 @@
 namespace tern {
 namespace {
 
-// Mask-bit position of in-word trit offset j (0..31); the sign bit sits one position higher
-// (mod 32).
-__device__ __forceinline__ int mask_pos(int j) { return 16 * (j & 1) + (j >> 4) + 2 * ((j & 15) >> 1); }
-
 __device__ __forceinline__ void set_flag(int32_t* flag) { atomicExch(flag, 1); }
-
-// One thread per 32-trit word: reads 32 trit bytes, writes one mask word and one sign word.
-__global__ void k_pack_trits(const int8_t* __restrict__ src, int64_t n_words, int32_t KM,
-                             uint32_t* __restrict__ planes, int32_t* __restrict__ flag) {
-  bool bad = false;
-  for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < n_words;
-       w += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t row = w / KM, col = w % KM;
-    const uint4* p = reinterpret_cast<const uint4*>(src + w * 32);
-    const uint4 v0 = ld_stream(p), v1 = ld_stream(p + 1);
-    const uint32_t b[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    uint32_t m = 0, s = 0;
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const uint32_t t = (b[j >> 2] >> (8 * (j & 3))) & 0xFFu;
-      const int p_m = mask_pos(j);
-      m |= (uint32_t)(t != 0u) << p_m;
-      s |= (uint32_t)(t == 0xFFu) << ((p_m + 1) & 31);
-      bad |= (t > 1u && t != 0xFFu);
-    }
-    uint32_t* row_p = planes + row * (2 * (int64_t)KM);
-    row_p[col] = m;
-    row_p[KM + col] = s;
-  }
-  if (__any_sync(0xFFFFFFFFu, bad) && (threadIdx.x & 31) == 0) set_flag(flag);
-}
 
 // Byte -> five trits as (mask5 | sign5 << 16), in natural order; all ones marks an invalid byte
 // (> 242), which also sets bit 31 of the OR of a run's entries.
@@ -73,6 +43,40 @@ __device__ __forceinline__ void build_base3_lut(uint32_t* lut) {
 __device__ __forceinline__ uint32_t to_mask_order(uint32_t x) {
   const uint32_t t = ((x >> 15) ^ x) & 0x0000AAAAu;
   return x ^ t ^ (t << 15);
+}
+
+// int8 trits -> planes: one thread per 32-trit word (32 bytes in, one mask and one sign word
+// out), the rows on the grid's y axis so that no index needs a division. In a valid trit byte
+// (0x00, 0x01 or 0xFF) bit 0 is the mask bit and bit 7 the sign bit; one multiply by
+// 1 + 2^7 + 2^14 + 2^21 gathers those bits of a word's four bytes into four adjacent bits (the
+// partial products never overlap, so there are no carries): mask bits of bytes 0..3 land at
+// bits 21..24, sign bits at 28..31. A byte is valid iff its bits 1..7 are all equal and bit 1
+// set implies bit 0 set.
+constexpr int kPackThreads = 128;
+__global__ void __launch_bounds__(kPackThreads) k_pack_trits(const int8_t* __restrict__ src, int32_t N, int32_t KM,
+                                                             uint32_t* __restrict__ planes, int32_t* __restrict__ flag) {
+  const int col = blockIdx.x * kPackThreads + threadIdx.x;
+  uint32_t bad = 0u;
+  if (col < KM) {
+    for (int row = blockIdx.y; row < N; row += gridDim.y) {
+      const uint4* p = reinterpret_cast<const uint4*>(src + ((int64_t)row * KM + col) * 32);
+      const uint4 v0 = ld_stream(p), v1 = ld_stream(p + 1);
+      const uint32_t b[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+      uint32_t m = 0u, s = 0u;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {                    // trits 4k .. 4k+3 in natural order
+        const uint32_t x = b[k];
+        m |= ((((x & 0x01010101u) * 0x00204081u) >> 21) & 0xFu) << (4 * k);
+        s |= (((x & 0x80808080u) * 0x00204081u) >> 28) << (4 * k);
+        bad |= ((x ^ (x >> 1)) & 0x7E7E7E7Eu) | ((x >> 1) & ~x & 0x01010101u);
+      }
+      const uint32_t sp = to_mask_order(s);
+      uint32_t* row_p = planes + (int64_t)row * (2 * (int64_t)KM);
+      row_p[col] = to_mask_order(m);
+      row_p[KM + col] = (sp << 1) | (sp >> 31);       // the sign bit sits one above its mask bit
+    }
+  }
+  if (__any_sync(0xFFFFFFFFu, bad != 0u) && (threadIdx.x & 31) == 0) set_flag(flag);
 }
 
 constexpr int kB3Threads = 256;
@@ -278,8 +282,12 @@ int grid_for(int64_t work, int threads) {
 
 cudaError_t launch_pack_trits(const int8_t* src, int32_t N, int32_t K, uint32_t* planes, int32_t* flag,
                               cudaStream_t st) {
-  const int64_t n_words = (int64_t)N * (K / 32);
-  k_pack_trits<<<grid_for(n_words, 256), 256, 0, st>>>(src, n_words, K / 32, planes, flag);
+  const int KM = K / 32;
+  const int gx = (KM + kPackThreads - 1) / kPackThreads;
+  int gy = (148 * 16 + gx - 1) / gx;                     // ~16 CTAs per SM over all columns
+  if (gy > N) gy = N;
+  if (gy > 65535) gy = 65535;
+  k_pack_trits<<<dim3(gx, gy), kPackThreads, 0, st>>>(src, N, KM, planes, flag);
   return cudaGetLastError();
 }
 
