@@ -83,7 +83,7 @@ constexpr int kB3Threads = 256;
 constexpr int kB3StageBytes = 8 * 1024;           // transport bytes per CTA (whole rows)
 constexpr int kB3Slot = 48;                       // shared-memory bytes per 32-byte run
 
-// One CTA per block of whole transport rows, three phases:
+// One block of whole transport rows, three phases (the CTA has built the byte table first):
 //   1. copy: run j (32 bytes = 160 trits = 5 output words) of the block goes to its own 48-byte
 //      slot, so that phase 2's two 16-byte reads per lane hit distinct banks;
 //   2. decode: a table turns each byte into its five mask and five sign bits in natural order;
@@ -97,10 +97,9 @@ __device__ __forceinline__ void unpack_base3_block(const uint8_t* __restrict__ s
   const int nrow = min(N - r0, rows_per_cta);
   const int rpr = (KW + 4) / 5;                    // runs per row
   const int nruns = nrow * rpr;
-  uint32_t* lut = reinterpret_cast<uint32_t*>(b3_smem);
+  const uint32_t* lut = reinterpret_cast<const uint32_t*>(b3_smem);
   uint8_t* runs = reinterpret_cast<uint8_t*>(b3_smem) + 1024;
   uint32_t* outw = reinterpret_cast<uint32_t*>(runs + (size_t)rows_per_cta * rpr * kB3Slot);
-  build_base3_lut(lut);
   const int64_t total = (int64_t)N * rb;
   // run index j -> (row rr, run i) advanced without divisions: j steps by `step`
   const int step = blockDim.x / 2;                 // copy phase: two half-runs per run
@@ -147,20 +146,20 @@ __device__ __forceinline__ void unpack_base3_block(const uint8_t* __restrict__ s
     const int eq = step2 / rpr, er = step2 - eq * rpr;
     int j = threadIdx.x, rr = j / rpr, i = j - rr * rpr;
     for (; j < nruns; j += step2) {
-      const int nb = min(32, rb - 32 * i);        // bytes of the run inside the row
       const uint4 lo = *reinterpret_cast<const uint4*>(runs + (size_t)j * kB3Slot);
       const uint4 hi = *reinterpret_cast<const uint4*>(runs + (size_t)j * kB3Slot + 16);
       const uint32_t by[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
       // groups of 16 trits: W[k] holds the group's 16 mask bits low and 16 sign bits high, so one
       // shifted table entry (mask5 | sign5 << 16) lands both fields of a byte with one add; the
       // bytes whose five trits cross a group boundary are added in two parts
+      // A row's last run also holds bytes past the row: the next row's own bytes, or zeros past
+      // the buffer, so an invalid byte among them is an invalid byte of the transport too.
       uint32_t W[10] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
       uint32_t eor = 0u;
-      const bool full = nb == 32;                 // every run but a row's last
 #pragma unroll
       for (int b = 0; b < 32; ++b) {
-        const uint32_t e = lut[(by[b >> 2] >> (8 * (b & 3))) & 0xFFu];
-        eor |= (full || b < nb) ? e : 0u;
+        const uint32_t e = lut[__byte_perm(by[b >> 2], 0u, 0x4440u | (uint32_t)(b & 3))];
+        eor |= e;
         const int k = (5 * b) >> 4, o = (5 * b) & 15;
         if (o <= 11) {
           W[k] += e << o;
@@ -201,25 +200,30 @@ __device__ __forceinline__ void unpack_base3_block(const uint8_t* __restrict__ s
   for (int v = threadIdx.x; v < nvec; v += blockDim.x) dst[v] = from[v];
 }
 
+// Persistent: each CTA builds the byte table once, then walks blocks of rows grid-strided.
 __global__ void __launch_bounds__(kB3Threads) k_unpack_base3(const uint8_t* __restrict__ src, int32_t N, int32_t KW,
-                                                             int32_t rb, int32_t rows_per_cta,
-                                                             uint32_t* __restrict__ planes, int32_t* __restrict__ flag) {
+                                                              int32_t rb, int32_t rows_per_cta, int32_t nblocks,
+                                                              uint32_t* __restrict__ planes, int32_t* __restrict__ flag) {
   extern __shared__ uint4 b3_smem[];
-  unpack_base3_block(src, N, KW, rb, rows_per_cta, blockIdx.x, planes, flag, b3_smem);
+  build_base3_lut(reinterpret_cast<uint32_t*>(b3_smem));
+  __syncthreads();
+  for (int block = blockIdx.x; block < nblocks; block += gridDim.x)
+    unpack_base3_block(src, N, KW, rb, rows_per_cta, block, planes, flag, b3_smem);
 }
 
-// Many tensors in one launch: CTA b belongs to the item whose block range holds b.
+// Persistent over the blocks of all items in order; a CTA's item index only moves forward.
 __global__ void __launch_bounds__(kB3Threads) k_unpack_base3_batch(const __grid_constant__ Base3Batch p,
-                                                                   int32_t* __restrict__ flag) {
+                                                                    int32_t nblocks, int32_t* __restrict__ flag) {
   extern __shared__ uint4 b3_smem[];
-  int lo = 0, hi = p.count - 1;
-  while (lo < hi) {                                // last item with block0 <= blockIdx.x
-    const int mid = (lo + hi + 1) >> 1;
-    if (p.block0[mid] <= (int)blockIdx.x) lo = mid; else hi = mid - 1;
+  build_base3_lut(reinterpret_cast<uint32_t*>(b3_smem));
+  __syncthreads();
+  int lo = 0;
+  for (int block = blockIdx.x; block < nblocks; block += gridDim.x) {
+    while (lo + 1 < p.count && p.block0[lo + 1] <= block) ++lo;   // last item with block0 <= block
+    const int K = p.K[lo];
+    unpack_base3_block(p.src[lo], p.N[lo], K / 32, (K + 4) / 5, p.rows[lo], block - p.block0[lo], p.planes[lo],
+                       flag, b3_smem);
   }
-  const int K = p.K[lo];
-  unpack_base3_block(p.src[lo], p.N[lo], K / 32, (K + 4) / 5, p.rows[lo], (int)blockIdx.x - p.block0[lo], p.planes[lo],
-                     flag, b3_smem);
 }
 
 // One thread per transport byte.
@@ -298,6 +302,17 @@ void base3_plan(int32_t K, int& rows, size_t& smem) {
   smem = 1024 + (size_t)rows * rpr * kB3Slot + (size_t)rows * K / 4;
 }
 
+// Resident CTAs of a persistent unpack kernel (at least one), capped by the blocks there are.
+int base3_grid(const void* fn, size_t smem, int nblocks) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kB3Threads, smem) != cudaSuccess || per_sm < 1)
+    per_sm = 1;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long g = (long long)per_sm * sms;
+  return (int)(g < nblocks ? g : (nblocks < 1 ? 1 : nblocks));
+}
+
 cudaError_t base3_smem_attr(const void* fn, size_t smem, size_t& set) {
   if (smem > 48 * 1024 && smem > set) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -312,11 +327,12 @@ cudaError_t launch_unpack_base3(const uint8_t* src, int32_t N, int32_t K, uint32
   int rows = 1;
   size_t smem = 0;
   base3_plan(K, rows, smem);
-  const int grid = (N + rows - 1) / rows;
+  const int nblocks = (N + rows - 1) / rows;
   static size_t set = 0;
   cudaError_t e = base3_smem_attr(reinterpret_cast<const void*>(k_unpack_base3), smem, set);
   if (e != cudaSuccess) return e;
-  k_unpack_base3<<<grid, kB3Threads, smem, st>>>(src, N, K / 32, (K + 4) / 5, rows, planes, flag);
+  const int grid = base3_grid(reinterpret_cast<const void*>(k_unpack_base3), smem, nblocks);
+  k_unpack_base3<<<grid, kB3Threads, smem, st>>>(src, N, K / 32, (K + 4) / 5, rows, nblocks, planes, flag);
   return cudaGetLastError();
 }
 
@@ -336,7 +352,8 @@ cudaError_t launch_unpack_base3_batch(Base3Batch& p, int32_t* flag, cudaStream_t
   static size_t set = 0;
   cudaError_t e = base3_smem_attr(reinterpret_cast<const void*>(k_unpack_base3_batch), smem, set);
   if (e != cudaSuccess) return e;
-  k_unpack_base3_batch<<<(unsigned)blocks, kB3Threads, smem, st>>>(p, flag);
+  const int grid = base3_grid(reinterpret_cast<const void*>(k_unpack_base3_batch), smem, (int)blocks);
+  k_unpack_base3_batch<<<grid, kB3Threads, smem, st>>>(p, (int32_t)blocks, flag);
   return cudaGetLastError();
 }
 
