@@ -80,8 +80,63 @@ __global__ void __launch_bounds__(kPackThreads) k_pack_trits(const int8_t* __res
 }
 
 constexpr int kB3Threads = 256;
-constexpr int kB3StageBytes = 8 * 1024;           // transport bytes per CTA (whole rows)
+constexpr int kB3StageBytes = 16 * 1024;          // transport bytes per block (whole rows)
 constexpr int kB3Slot = 48;                       // shared-memory bytes per 32-byte run
+
+// The five words of a copy window that reaches the end of the transport buffer: the words wholly
+// inside it as words, the last partial one byte by byte, zeros past the end (n = bytes left).
+struct Words5 {
+  uint32_t w0, w1, w2, w3, w4;
+};
+__device__ __noinline__ uint32_t load_tail_word(const uint8_t* p, int n) {
+  uint32_t x = 0u;
+  if (n >= 4) return __ldg(reinterpret_cast<const uint32_t*>(p));
+  for (int t = 0; t < 4; ++t)
+    if (t < n) x |= (uint32_t)__ldg(p + t) << (8 * t);
+  return x;
+}
+__device__ __noinline__ Words5 load_tail_words(const uint8_t* p, int n) {
+  Words5 r;
+  r.w0 = load_tail_word(p, n);
+  r.w1 = load_tail_word(p + 4, n - 4);
+  r.w2 = load_tail_word(p + 8, n - 8);
+  r.w3 = load_tail_word(p + 12, n - 12);
+  r.w4 = load_tail_word(p + 16, n - 16);
+  return r;
+}
+
+// A tensor's constants for the unpack walks, computed once per tensor and thread: run j of a
+// block (32 transport bytes = 160 trits) is run i of block row rr, and each walk advances j by a
+// fixed step, so (rr, i) advance by (step / rpr, step % rpr) without a division per block.
+struct B3Shape {
+  const uint8_t* src;
+  uint32_t* planes;
+  int N, KW, rb, rows, rpr;
+  int64_t total;                                   // transport bytes of the tensor
+  int c_rr, c_i, c_dq, c_dr;                       // copy walk: j = tid / 2, step blockDim / 2
+  int d_rr, d_i, d_dq, d_dr;                       // decode walk: j = tid, step blockDim
+};
+__device__ __forceinline__ B3Shape b3_shape(const uint8_t* src, uint32_t* planes, int N, int K, int rows) {
+  B3Shape s;
+  s.src = src;
+  s.planes = planes;
+  s.N = N;
+  s.KW = K / 32;
+  s.rb = (K + 4) / 5;
+  s.rows = rows;
+  s.rpr = (s.KW + 4) / 5;
+  s.total = (int64_t)N * s.rb;
+  const int jc = threadIdx.x >> 1, sc = blockDim.x >> 1, jd = threadIdx.x, sd = blockDim.x;
+  s.c_rr = jc / s.rpr;
+  s.c_i = jc - s.c_rr * s.rpr;
+  s.c_dq = sc / s.rpr;
+  s.c_dr = sc - s.c_dq * s.rpr;
+  s.d_rr = jd / s.rpr;
+  s.d_i = jd - s.d_rr * s.rpr;
+  s.d_dq = sd / s.rpr;
+  s.d_dr = sd - s.d_dq * s.rpr;
+  return s;
+}
 
 // One block of whole transport rows, three phases (the CTA has built the byte table first):
 //   1. copy: run j (32 bytes = 160 trits = 5 output words) of the block goes to its own 48-byte
@@ -90,41 +145,41 @@ constexpr int kB3Slot = 48;                       // shared-memory bytes per 32-
 //      the bits are gathered per 32-trit word, moved to the layout's bit order and written to a
 //      shared-memory copy of the block's output rows;
 //   3. write-out: the block's rows are contiguous in the planes, copied with 16-byte stores.
-__device__ __forceinline__ void unpack_base3_block(const uint8_t* __restrict__ src, int32_t N, int32_t KW, int32_t rb,
-                                                   int32_t rows_per_cta, int32_t block, uint32_t* __restrict__ planes,
-                                                   int32_t* __restrict__ flag, uint4* b3_smem) {
+__device__ __forceinline__ void unpack_base3_block(const B3Shape& S, int32_t block, int32_t* __restrict__ flag,
+                                                   uint4* b3_smem) {
+  const uint8_t* __restrict__ src = S.src;
+  const int N = S.N, KW = S.KW, rb = S.rb, rows_per_cta = S.rows, rpr = S.rpr;
   const int r0 = block * rows_per_cta;
   const int nrow = min(N - r0, rows_per_cta);
-  const int rpr = (KW + 4) / 5;                    // runs per row
   const int nruns = nrow * rpr;
   const uint32_t* lut = reinterpret_cast<const uint32_t*>(b3_smem);
   uint8_t* runs = reinterpret_cast<uint8_t*>(b3_smem) + 1024;
   uint32_t* outw = reinterpret_cast<uint32_t*>(runs + (size_t)rows_per_cta * rpr * kB3Slot);
-  const int64_t total = (int64_t)N * rb;
-  // run index j -> (row rr, run i) advanced without divisions: j steps by `step`
+  const int64_t total = S.total;
   const int step = blockDim.x / 2;                 // copy phase: two half-runs per run
-  const int dq = step / rpr, dr = step - (step / rpr) * rpr;
-  // 1. copy: half-runs of 16 bytes, each from five aligned words of the transport
+  const int dq = S.c_dq, dr = S.c_dr;
+  // 1. copy: half-runs of 16 bytes, each from five aligned words of the transport. Offsets are
+  // 32-bit, relative to the aligned word at or below the block's first byte; only a window that
+  // reaches the buffer's end takes the byte-wise path.
   {
-    int j = threadIdx.x >> 1, rr = j / rpr, i = j - rr * rpr;
+    const int64_t b0 = (int64_t)r0 * rb;             // the block's first transport byte
+    const uint8_t* base = src + (b0 & ~(int64_t)3);
+    const int lead = (int)(b0 & 3);
+    const int64_t rem64 = total - (b0 & ~(int64_t)3);
+    const int remain = rem64 > 0x7FFFFFFF ? 0x7FFFFFFF : (int)rem64;   // bytes from base to the end
+    int j = threadIdx.x >> 1, rr = S.c_rr, i = S.c_i;
     const int h = threadIdx.x & 1;
     for (; j < nruns; j += step) {
-      const int pos = 32 * i + 16 * h;              // byte position in the row
-      const int64_t g = (int64_t)(r0 + rr) * rb + pos;
-      const int64_t ga = g & ~(int64_t)3;
-      const uint32_t sh = 8u * (uint32_t)(g & 3);
+      const int off = lead + rr * rb + 32 * i + 16 * h; // byte offset of the half-run from base
+      const int oa = off & ~3;
+      const uint32_t sh = 8u * (uint32_t)(off & 3);
       uint32_t w[5];
+      if (oa + 20 <= remain) {
 #pragma unroll
-      for (int k = 0; k < 5; ++k) {
-        const int64_t a = ga + 4 * k;
-        if (a + 4 <= total) {
-          w[k] = __ldg(reinterpret_cast<const uint32_t*>(src + a));
-        } else {                                    // the buffer's last, partial word: byte by byte
-          uint32_t x = 0u;
-          for (int t = 0; t < 4; ++t)
-            if (a + t < total) x |= (uint32_t)__ldg(src + a + t) << (8 * t);
-          w[k] = x;
-        }
+        for (int k = 0; k < 5; ++k) w[k] = __ldg(reinterpret_cast<const uint32_t*>(base + oa + 4 * k));
+      } else {
+        const Words5 t = load_tail_words(base + oa, remain - oa);
+        w[0] = t.w0; w[1] = t.w1; w[2] = t.w2; w[3] = t.w3; w[4] = t.w4;
       }
       // bytes past the row's end belong to the next row: they only reach trits past K, never written
       uint4 v;
@@ -143,8 +198,8 @@ __device__ __forceinline__ void unpack_base3_block(const uint8_t* __restrict__ s
   bool bad = false;
   {
     const int step2 = blockDim.x;
-    const int eq = step2 / rpr, er = step2 - eq * rpr;
-    int j = threadIdx.x, rr = j / rpr, i = j - rr * rpr;
+    const int eq = S.d_dq, er = S.d_dr;
+    int j = threadIdx.x, rr = S.d_rr, i = S.d_i;
     for (; j < nruns; j += step2) {
       const uint4 lo = *reinterpret_cast<const uint4*>(runs + (size_t)j * kB3Slot);
       const uint4 hi = *reinterpret_cast<const uint4*>(runs + (size_t)j * kB3Slot + 16);
@@ -195,34 +250,37 @@ __device__ __forceinline__ void unpack_base3_block(const uint8_t* __restrict__ s
   __syncthreads();
   // 3. write-out: nrow rows x 2*KW words, contiguous in the planes (KW % 4 == 0)
   const int nvec = nrow * 2 * KW / 4;
-  uint4* dst = reinterpret_cast<uint4*>(planes + (size_t)r0 * 2 * KW);
+  uint4* dst = reinterpret_cast<uint4*>(S.planes + (size_t)r0 * 2 * KW);
   const uint4* from = reinterpret_cast<const uint4*>(outw);
   for (int v = threadIdx.x; v < nvec; v += blockDim.x) dst[v] = from[v];
 }
 
 // Persistent: each CTA builds the byte table once, then walks blocks of rows grid-strided.
-__global__ void __launch_bounds__(kB3Threads) k_unpack_base3(const uint8_t* __restrict__ src, int32_t N, int32_t KW,
+__global__ void __launch_bounds__(kB3Threads, 5) k_unpack_base3(const uint8_t* __restrict__ src, int32_t N, int32_t KW,
                                                               int32_t rb, int32_t rows_per_cta, int32_t nblocks,
                                                               uint32_t* __restrict__ planes, int32_t* __restrict__ flag) {
   extern __shared__ uint4 b3_smem[];
   build_base3_lut(reinterpret_cast<uint32_t*>(b3_smem));
   __syncthreads();
-  for (int block = blockIdx.x; block < nblocks; block += gridDim.x)
-    unpack_base3_block(src, N, KW, rb, rows_per_cta, block, planes, flag, b3_smem);
+  const B3Shape S = b3_shape(src, planes, N, KW * 32, rows_per_cta);
+  for (int block = blockIdx.x; block < nblocks; block += gridDim.x) unpack_base3_block(S, block, flag, b3_smem);
 }
 
 // Persistent over the blocks of all items in order; a CTA's item index only moves forward.
-__global__ void __launch_bounds__(kB3Threads) k_unpack_base3_batch(const __grid_constant__ Base3Batch p,
+__global__ void __launch_bounds__(kB3Threads, 5) k_unpack_base3_batch(const __grid_constant__ Base3Batch p,
                                                                     int32_t nblocks, int32_t* __restrict__ flag) {
   extern __shared__ uint4 b3_smem[];
   build_base3_lut(reinterpret_cast<uint32_t*>(b3_smem));
   __syncthreads();
-  int lo = 0;
+  int lo = 0, cur = -1;
+  B3Shape S;
   for (int block = blockIdx.x; block < nblocks; block += gridDim.x) {
     while (lo + 1 < p.count && p.block0[lo + 1] <= block) ++lo;   // last item with block0 <= block
-    const int K = p.K[lo];
-    unpack_base3_block(p.src[lo], p.N[lo], K / 32, (K + 4) / 5, p.rows[lo], block - p.block0[lo], p.planes[lo],
-                       flag, b3_smem);
+    if (lo != cur) {
+      S = b3_shape(p.src[lo], p.planes[lo], p.N[lo], p.K[lo], p.rows[lo]);
+      cur = lo;
+    }
+    unpack_base3_block(S, block - p.block0[lo], flag, b3_smem);
   }
 }
 
