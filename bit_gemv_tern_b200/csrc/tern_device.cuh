@@ -67,19 +67,31 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, 
 }
 
 // ---- decode ------------------------------------------------------------------------------------
+// One three-input logic operation with an immediate truth table (lut bit (a<<2 | b<<1 | c) is the
+// result for those input bits). Written out because the compiler does not always fold a merge of
+// two planes under two complementary constants into a single operation.
+template <uint32_t LUT>
+__device__ __forceinline__ uint32_t lop3(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, %4;" : "=r"(d) : "r"(a), "r"(b), "r"(c), "n"(LUT));
+  return d;
+}
+
 // Offset-binary merge: fields (m, NOT s) read as an unsigned 2-bit number equal t + 2
 // (t = 0 -> 2, t = +1 -> 3, t = -1 -> 1). A field left in place at bit 2i of a byte and masked is
 // the u8 value 4^i * (t + 2): one AND per tensor-core register, no shift. Sums then carry a known
 // offset 2 * sum(x) that is removed exactly.
+//   wa = (m & C) | (~s & ~C),  v = (m & ~C) | (~s & C),  C = 0x55555555:  one LOP3 each
 __device__ __forceinline__ void merge_planes_offset(uint32_t m, uint32_t s, uint32_t& wa, uint32_t& wb) {
-  wa = (m & 0x55555555u) | (~s & 0xAAAAAAAAu);
-  const uint32_t v = (m & 0xAAAAAAAAu) | (~s & 0x55555555u);
+  wa = lop3<0xB1u>(m, s, 0x55555555u);
+  const uint32_t v = lop3<0x72u>(m, s, 0x55555555u);
   wb = __funnelshift_r(v, v, 1);
 }
 
+//   wa = (m & C) | (s & ~C),  v = (m & ~C) | (s & C),  C = 0x55555555:  one LOP3 each
 __device__ __forceinline__ void merge_planes(uint32_t m, uint32_t s, uint32_t& wa, uint32_t& wb) {
-  wa = (m & 0x55555555u) | (s & 0xAAAAAAAAu);
-  const uint32_t v = (m & 0xAAAAAAAAu) | (s & 0x55555555u);
+  wa = lop3<0xE4u>(m, s, 0x55555555u);
+  const uint32_t v = lop3<0xD8u>(m, s, 0x55555555u);
   wb = __funnelshift_r(v, v, 1);
 }
 
