@@ -766,7 +766,7 @@ class StackView:
 
 def pack_row(torch, tg, hbm_peak):
     """int8 trits of the seven tensors of one 8B layer (193 MB, > L2) packed into their planes by
-    one tern_pack_batch call; bytes = N*K in + N*K/4 out per tensor."""
+    one tern_pack_batch call (one launch); bytes = N*K in + N*K/4 out per tensor."""
     import synth
     import synth.cuda as sc
     flag = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -785,7 +785,7 @@ def pack_row(torch, tg, hbm_peak):
     gbs = nb / (ms / 1000.0) / 1e9
     layers = synth.GEOMETRY["8b"]["layers"]
     return {"ms": ms, "gbs": gbs, "frac": gbs / hbm_peak, "trits": trits, "bytes": nb, "tensors": len(items),
-            "launches": len(items), "ms_8b_equivalent": ms * layers}
+            "launches": 1, "ms_8b_equivalent": ms * layers}
 
 
 def base3_row(stack, torch, tg, hbm_peak):

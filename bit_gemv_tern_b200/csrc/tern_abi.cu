@@ -99,9 +99,17 @@ tern_status tern_pack_batch(tern_src src, const tern_pack_item* items, int32_t c
   cudaError_t e = cudaMemsetAsync(err_flag_dev, 0, sizeof(int32_t), cs(stream));
   if (e != cudaSuccess) return TERN_ECUDA;
   if (src == TERN_SRC_INT8_TRITS) {
-    for (int i = 0; i < count && e == cudaSuccess; ++i)
-      e = tern::launch_pack_trits(static_cast<const int8_t*>(items[i].src_dev), items[i].N, items[i].K,
-                                  items[i].planes_dev, err_flag_dev, cs(stream));
+    tern::PackBatch* pb = new (std::nothrow) tern::PackBatch();
+    if (!pb) return TERN_EINVAL;
+    pb->count = count;
+    for (int i = 0; i < count; ++i) {
+      pb->src[i] = static_cast<const int8_t*>(items[i].src_dev);
+      pb->planes[i] = items[i].planes_dev;
+      pb->N[i] = items[i].N;
+      pb->KM[i] = items[i].K / 32;
+    }
+    e = tern::launch_pack_trits_batch(*pb, err_flag_dev, cs(stream));
+    delete pb;
     return from_cuda(e);
   }
   tern::Base3Batch* b = new (std::nothrow) tern::Base3Batch();

@@ -140,6 +140,15 @@ struct Base3Batch {
   int32_t count;
 };
 cudaError_t launch_unpack_base3_batch(Base3Batch& p, int32_t* flag, cudaStream_t st);
+// int8 trits of several tensors packed in one launch: work units of 16 rows x 128 words.
+struct PackBatch {
+  const int8_t* src[kPackMaxItems];
+  uint32_t* planes[kPackMaxItems];
+  int32_t N[kPackMaxItems], KM[kPackMaxItems];     // rows, words per row and plane (K / 32)
+  int32_t unit0[kPackMaxItems];                    // first work unit of each item (set by the launcher)
+  int32_t count, units;
+};
+cudaError_t launch_pack_trits_batch(PackBatch& p, int32_t* flag, cudaStream_t st);
 cudaError_t launch_pack_trits(const int8_t* src, int32_t N, int32_t K, uint32_t* planes, int32_t* flag,
                               cudaStream_t st);
 cudaError_t launch_unpack_base3(const uint8_t* src, int32_t N, int32_t K, uint32_t* planes, int32_t* flag,

@@ -46,34 +46,64 @@ __device__ __forceinline__ uint32_t to_mask_order(uint32_t x) {
 }
 
 // int8 trits -> planes: one thread per 32-trit word (32 bytes in, one mask and one sign word
-// out), the rows on the grid's y axis so that no index needs a division. In a valid trit byte
+// out). A single tensor puts its rows on the grid's y axis, so no index needs a division; a
+// batch of tensors walks work units of 16 rows x 128 words in one persistent launch. In a valid
+// trit byte
 // (0x00, 0x01 or 0xFF) bit 0 is the mask bit and bit 7 the sign bit; one multiply by
 // 1 + 2^7 + 2^14 + 2^21 gathers those bits of a word's four bytes into four adjacent bits (the
 // partial products never overlap, so there are no carries): mask bits of bytes 0..3 land at
 // bits 21..24, sign bits at 28..31. A byte is valid iff its bits 1..7 are all equal and bit 1
 // set implies bit 0 set.
 constexpr int kPackThreads = 128;
+constexpr int kPackUnitRows = 16;                 // rows of one batched work unit
+// One 32-trit word: 32 bytes in, the mask and sign words out (bit order of the layout).
+__device__ __forceinline__ void pack_word(const int8_t* __restrict__ src, uint32_t* __restrict__ planes, int row,
+                                          int col, int KM, uint32_t& bad) {
+  const uint4* q = reinterpret_cast<const uint4*>(src + ((int64_t)row * KM + col) * 32);
+  const uint4 v0 = ld_stream(q), v1 = ld_stream(q + 1);
+  const uint32_t b[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+  uint32_t m = 0u, s = 0u;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {                      // trits 4k .. 4k+3 in natural order
+    const uint32_t x = b[k];
+    m |= ((((x & 0x01010101u) * 0x00204081u) >> 21) & 0xFu) << (4 * k);
+    s |= (((x & 0x80808080u) * 0x00204081u) >> 28) << (4 * k);
+    bad |= ((x ^ (x >> 1)) & 0x7E7E7E7Eu) | ((x >> 1) & ~x & 0x01010101u);
+  }
+  const uint32_t sp = to_mask_order(s);
+  uint32_t* row_p = planes + (int64_t)row * (2 * (int64_t)KM);
+  row_p[col] = to_mask_order(m);
+  row_p[KM + col] = (sp << 1) | (sp >> 31);          // the sign bit sits one above its mask bit
+}
+
 __global__ void __launch_bounds__(kPackThreads) k_pack_trits(const int8_t* __restrict__ src, int32_t N, int32_t KM,
                                                              uint32_t* __restrict__ planes, int32_t* __restrict__ flag) {
   const int col = blockIdx.x * kPackThreads + threadIdx.x;
   uint32_t bad = 0u;
-  if (col < KM) {
-    for (int row = blockIdx.y; row < N; row += gridDim.y) {
-      const uint4* p = reinterpret_cast<const uint4*>(src + ((int64_t)row * KM + col) * 32);
-      const uint4 v0 = ld_stream(p), v1 = ld_stream(p + 1);
-      const uint32_t b[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-      uint32_t m = 0u, s = 0u;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {                    // trits 4k .. 4k+3 in natural order
-        const uint32_t x = b[k];
-        m |= ((((x & 0x01010101u) * 0x00204081u) >> 21) & 0xFu) << (4 * k);
-        s |= (((x & 0x80808080u) * 0x00204081u) >> 28) << (4 * k);
-        bad |= ((x ^ (x >> 1)) & 0x7E7E7E7Eu) | ((x >> 1) & ~x & 0x01010101u);
-      }
-      const uint32_t sp = to_mask_order(s);
-      uint32_t* row_p = planes + (int64_t)row * (2 * (int64_t)KM);
-      row_p[col] = to_mask_order(m);
-      row_p[KM + col] = (sp << 1) | (sp >> 31);       // the sign bit sits one above its mask bit
+  if (col < KM)
+    for (int row = blockIdx.y; row < N; row += gridDim.y) pack_word(src, planes, row, col, KM, bad);
+  if (__any_sync(0xFFFFFFFFu, bad != 0u) && (threadIdx.x & 31) == 0) set_flag(flag);
+}
+
+// Several tensors in one persistent launch: unit u of item i covers rows [16r, 16r + 16) and words
+// [128c, 128c + 128) of each row, u - unit0[i] = r * (column blocks) + c.
+__global__ void __launch_bounds__(kPackThreads) k_pack_trits_batch(const __grid_constant__ PackBatch p,
+                                                                   int32_t* __restrict__ flag) {
+  uint32_t bad = 0u;
+  for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
+    int lo = 0, hi = p.count - 1;                   // last item with unit0 <= u
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (p.unit0[mid] <= u) lo = mid; else hi = mid - 1;
+    }
+    const int KM = p.KM[lo], N = p.N[lo];
+    const int gx = (KM + kPackThreads - 1) / kPackThreads;
+    const int lu = u - p.unit0[lo];
+    const int rg = lu / gx, col = (lu - rg * gx) * kPackThreads + threadIdx.x;
+    if (col < KM) {
+      const int r1 = min(N, (rg + 1) * kPackUnitRows);
+#pragma unroll 4
+      for (int row = rg * kPackUnitRows; row < r1; ++row) pack_word(p.src[lo], p.planes[lo], row, col, KM, bad);
     }
   }
   if (__any_sync(0xFFFFFFFFu, bad != 0u) && (threadIdx.x & 31) == 0) set_flag(flag);
@@ -391,6 +421,25 @@ cudaError_t launch_unpack_base3(const uint8_t* src, int32_t N, int32_t K, uint32
   if (e != cudaSuccess) return e;
   const int grid = base3_grid(reinterpret_cast<const void*>(k_unpack_base3), smem, nblocks);
   k_unpack_base3<<<grid, kB3Threads, smem, st>>>(src, N, K / 32, (K + 4) / 5, rows, nblocks, planes, flag);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_trits_batch(PackBatch& p, int32_t* flag, cudaStream_t st) {
+  int64_t units = 0;
+  for (int i = 0; i < p.count; ++i) {
+    p.unit0[i] = (int32_t)units;
+    units += (int64_t)((p.N[i] + kPackUnitRows - 1) / kPackUnitRows) * ((p.KM[i] + kPackThreads - 1) / kPackThreads);
+  }
+  if (units > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  p.units = (int32_t)units;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_pack_trits_batch, kPackThreads, 0) != cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t g = (int64_t)per_sm * sms;
+  k_pack_trits_batch<<<(unsigned)(g < units ? g : units), kPackThreads, 0, st>>>(p, flag);
   return cudaGetLastError();
 }
 

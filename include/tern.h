@@ -123,8 +123,8 @@ typedef struct {
 #define TERN_PACK_MAX_ITEMS 256
 
 /* tern_pack over a list of tensors (a whole model's transport at load time): one clear of
- * err_flag_dev, then one launch for all base-3 items (TERN_SRC_BASE3), or one launch per item
- * for TERN_SRC_INT8_TRITS. Results are bit-identical to tern_pack per item; the flag is set if
+ * err_flag_dev, then one launch for all items (for either source kind). Results are
+ * bit-identical to tern_pack per item; the flag is set if
  * any item holds an invalid value. items: host array of 1..TERN_PACK_MAX_ITEMS descriptors,
  * read during the call only. No output may overlap another item's input or output. */
 tern_status tern_pack_batch(tern_src src, const tern_pack_item* items, int32_t count, int32_t* err_flag_dev,

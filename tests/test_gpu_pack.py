@@ -143,3 +143,26 @@ def test_base3_batch_bit_exact_and_flag():
     assert tg.tern_read_flag(flag) == tg.TERN_EBADCODE
     tg.tern_pack_batch(tg.TERN_SRC_BASE3, items[:2], flag)          # the next call clears the flag
     assert tg.tern_read_flag(flag) == 0
+
+
+def test_int8_batch_bit_exact_and_flag():
+    """tern_pack_batch over ragged int8-trit items (one persistent launch; units of 16 rows x 128
+    words, so N % 16 != 0 and K / 32 % 128 != 0 leave partial units) equals the oracle per item;
+    a byte outside {0, 1, 0xFF} in one item sets the flag, and the next call clears it."""
+    shapes = [(1, 128), (37, 384), (20, 4096), (5, 12288), (17, 1024), (300, 640), (33, 8192)]
+    items, refs, flag = [], [], torch.zeros(1, dtype=torch.int32, device="cuda")
+    for i, (N, K) in enumerate(shapes):
+        t = synth.trits(35, 60 + i, N, K)
+        planes = torch.full((N * K // 16,), -1, dtype=torch.int32, device="cuda")
+        items.append((dev(t.reshape(-1)), N, K, planes))
+        refs.append(oracle.pack(t))
+    tg.tern_pack_batch(tg.TERN_SRC_INT8_TRITS, items, flag)
+    assert tg.tern_read_flag(flag) == 0
+    for (src, N, K, planes), ref in zip(items, refs):
+        assert (host(planes).view(np.uint32).reshape(N, K // 16) == ref).all(), (N, K)
+    bad = items[5][0].clone()
+    bad[300 * 640 - 1] = 2                                          # the last byte of the last row
+    tg.tern_pack_batch(tg.TERN_SRC_INT8_TRITS, [items[0], (bad, 300, 640, items[5][3])], flag)
+    assert tg.tern_read_flag(flag) == tg.TERN_EBADCODE
+    tg.tern_pack_batch(tg.TERN_SRC_INT8_TRITS, items[:2], flag)     # the next call clears the flag
+    assert tg.tern_read_flag(flag) == 0
