@@ -581,17 +581,35 @@ def _profile_base3():
     return run
 
 
+def _profile_pack():
+    def run():
+        import torch
+        import synth
+        import synth.cuda as sc
+        import bit_gemv_tern_b200 as tg
+        flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+        items = []
+        for p, N, K in synth.linear_shapes("8b"):
+            t = torch.empty(N * K, dtype=torch.int8, device="cuda")
+            sc.trits_into(t, SEED, synth.tensor_id(0, p), K)
+            items.append((t, N, K, torch.empty(N * K // 16, dtype=torch.int32, device="cuda")))
+        return lambda: tg.tern_pack_batch(tg.TERN_SRC_INT8_TRITS, items, flag)
+    return run
+
+
 # Small cases for ncu captures (inputs > L2, a few hundred MB on the device):
 #   batch-8b-4layers-*: 4 layers of the 8B stack (16 fused GEMVs, 193 MB of planes) as one batch
 #   head-8b-*:          the int8 head 151936 x 4096 (622 MB)
 #   prefill-8b-gate-*:  one 12288 x 4096 linear at M = 4096 tokens (tcgen05 prefill)
 #   base3-8b-1layer:    the transport of one 8B layer's seven tensors (86.9 MB) in one batched call
+#   pack-8b-1layer:     the int8 trits of one 8B layer's seven tensors (193 MB) in one batched call
 PROFILE_CASES = {
     "batch-8b-4layers-bf16": _profile_batch("bf16"),
     "batch-8b-4layers-int8": _profile_batch("int8"),
     "head-8b-bf16": _profile_head("bf16"),
     "prefill-8b-gate-m4096": _profile_prefill("gate"),
     "base3-8b-1layer": _profile_base3(),
+    "pack-8b-1layer": _profile_pack(),
 }
 
 
