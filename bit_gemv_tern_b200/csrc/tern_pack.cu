@@ -41,8 +41,8 @@ __device__ __forceinline__ void build_base3_lut(uint32_t* lut) {
 // Natural-order bits -> the layout's order: bit j moves to p(j), which swaps bits 0 and 4 of
 // the index j (one delta swap: positions with j0 = 1, j4 = 0 trade places with j + 15).
 __device__ __forceinline__ uint32_t to_mask_order(uint32_t x) {
-  const uint32_t t = ((x >> 15) ^ x) & 0x0000AAAAu;
-  return x ^ t ^ (t << 15);
+  const uint32_t t = lop3<0x28u>(x >> 15, x, 0x0000AAAAu);    // ((x >> 15) ^ x) & 0xAAAA
+  return lop3<0x96u>(x, t, t << 15);                         // x ^ t ^ (t << 15)
 }
 
 // int8 trits -> planes: one thread per 32-trit word (32 bytes in, one mask and one sign word
@@ -65,10 +65,15 @@ __device__ __forceinline__ void pack_word(const int8_t* __restrict__ src, uint32
   uint32_t m = 0u, s = 0u;
 #pragma unroll
   for (int k = 0; k < 8; ++k) {                      // trits 4k .. 4k+3 in natural order
-    const uint32_t x = b[k];
-    m |= ((((x & 0x01010101u) * 0x00204081u) >> 21) & 0xFu) << (4 * k);
-    s |= (((x & 0x80808080u) * 0x00204081u) >> 28) << (4 * k);
-    bad |= ((x ^ (x >> 1)) & 0x7E7E7E7Eu) | ((x >> 1) & ~x & 0x01010101u);
+    const uint32_t x = b[k], y = x >> 1;
+    // gathered nibble at bits 21..24 (mask) / 28..31 (sign), moved to bits 4k..4k+3; the other
+    // partial products land outside the nibble's place and are masked off
+    const uint32_t gm = (x & 0x01010101u) * 0x00204081u, gs = (x & 0x80808080u) * 0x00204081u;
+    const uint32_t um = 4 * k <= 21 ? gm >> (21 - 4 * k) : gm << (4 * k - 21);
+    const uint32_t us = gs >> (28 - 4 * k);
+    m = lop3<0xEAu>(um, 0xFu << (4 * k), m);         // m | (um & nibble)
+    s = lop3<0xEAu>(us, 0xFu << (4 * k), s);
+    bad = lop3<0xFEu>(bad, lop3<0x28u>(x, y, 0x7E7E7E7Eu), lop3<0x20u>(y, x, 0x01010101u));
   }
   const uint32_t sp = to_mask_order(s);
   uint32_t* row_p = planes + (int64_t)row * (2 * (int64_t)KM);
