@@ -1,6 +1,7 @@
-// Batched M = 1 GEMV: a whole list of linear layers in two launches.
+// Batched GEMV (M = 1) and small-M GEMM (M = 2..16): a whole list of linear layers in two
+// launches.
 //
-//   for every item i:  y_i[n] = scale_i[n] * sum_k t_i[n][k] * x_i[k]
+//   for every item i:  y_i[m][n] = scale_i[n] * sum_k t_i[n][k] * x_i[m][k]
 //
 // A decode step streams every weight of the stack once per token (PyTorchKR review "Fermion
 // Research, 3진 계열 포맷으로 직접 학습한 Neutrino-1 모델군 3종 공개", section "뉴트리노 엔진":
@@ -8,13 +9,13 @@
 // that floor at the ~120 kernel boundaries of a step. Here the boundaries are gone: one persistent
 // launch walks all items, so the weight stream never pauses between layers.
 //
-//   1. k_batch_prep (one CTA per item) turns each activation into ready-to-load tensor-core operand
-//      segments, one per 512-trit K part: int8 q permuted to the decode's byte order (int8 mode),
+//   1. k_batch_prep (one CTA per item and token slot) turns each activation into ready-to-load
+//      tensor-core operand segments, one per 512-trit K part: int8 q permuted to the decode's byte order (int8 mode),
 //      or three exact int8 limbs of a 22-bit fixed-point value relative to 2^E with E from the
 //      item's absmax (bf16 mode), followed by the item's column sums (which remove the decode
-//      offset) and E.
-//   2. k_batch_stream (one CTA per SM) splits the list's row blocks (kStageRows rows x all of K)
-//      evenly by bytes. Its producer lane walks the CTA's row blocks part by part: each stage of
+//      offset) and E. Tokens occupy the MMA's n-columns (see seg_cols).
+//   2. k_batch_stream (one CTA per SM) splits the list's (row block, K part) sequence evenly by
+//      bytes, so a row block may be shared by neighbouring CTAs. Its producer lane walks the CTA's row blocks part by part: each stage of
 //      the ring receives, by tensor TMA, the mask and sign words of the block's rows for one K part
 //      (the packed planes seen as a [plane][row][word] tensor, so the row-major layout is read in
 //      place) plus that part's operand segment. The consumer warps walk the stages in order; warp
