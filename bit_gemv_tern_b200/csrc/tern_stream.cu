@@ -13,9 +13,10 @@
 //     while the previous kernel of the chain is still running, the ring already fills;
 //   * griddepcontrol.launch_dependents at entry, so the next kernel's CTA can become resident
 //     next to this one and prefetch its own weights (programmatic dependent launch);
-//   * eight consumer warps that wait for the previous kernel only when they need the activation,
-//     stage it once, then decode 2-bit fields to int8 tensor-core operands (64*t, see
-//     tern_device.cuh) and run mma.sync s8 with four independent accumulator chains;
+//   * 8 or 16 consumer warps that wait for the previous kernel only when they need the
+//     activation, stage it once, then decode the merged 2-bit fields into u8 tensor-core operands
+//     (one AND per register, see merge_planes_offset in tern_device.cuh) and run mma.sync u8 x s8
+//     with four field accumulators;
 //   * int8 mode: x = q (per-token int8), exact int32 sums; bf16 mode: x is split exactly into three
 //     int8 limbs of a 22-bit fixed-point value relative to 2^E (E from the absmax of x), which sit
 //     in three columns of the n = 8 operand for free at M = 1, so the products and sums stay
