@@ -1,5 +1,5 @@
 // Loader-side kernels: packing trits into the two-plane layout, the base-3 transport in both
-// directions, and per-row occupancy counts. All are streaming, HBM-bound integer kernels.
+// directions, and per-row occupancy counts: streaming integer kernels whose roofline is HBM.
 //
 // Sources: weights packed at rest and decoded inside the matrix kernels (aiatolah.com,
 // "Neutrino-1 8B: modelo ternario de 3,88 GB roda em GPU e laptop", second paragraph); the
