@@ -353,6 +353,10 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
   // columns past NCOL (M = 1, PACK) repeat a real column; their sums are never read
   const int col0 = (MP == 1 || PACK) ? (g < NCOL ? g : 0) : g;
   const int col1 = 8 + g < NCOL ? 8 + g : 8;                // PACK, MP = 4: group 1
+  // lanes whose column of group 0 / group 1 exists (M = 1, PACK); the others feed zeros, so the
+  // tensor cores multiply no real data into the accumulators that are never read
+  const bool live0 = (MP == 1 || PACK) ? g < NCOL : true;
+  const bool live1 = PACK ? 8 + g < NCOL : true;
   // byte offsets inside a slot
   const uint32_t wofs = (uint32_t)((warp * 16 + g) * kPartWords * 4 + t * 16);   // plane 0, row g
   const uint32_t xofs = (uint32_t)(kWStageBytesT + (col0 * kColWords + t * 8) * 4);
@@ -443,8 +447,10 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
         for (int j = 0; j < G; ++j) {
           // (b0, b1) of fields 0, 1 and of fields 2, 3
           const uint32_t xo = (PACK && j == 1) ? xofs1 : xofs + (uint32_t)(j * 8 * kColWords) * 4;
-          const uint4 x01 = lds128(st + xo + e * 128);
-          const uint4 x23 = lds128(st + xo + e * 128 + 16);
+          const bool live = (PACK && j == 1) ? live1 : (j == 0 ? live0 : true);
+          const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+          const uint4 x01 = live ? lds128(st + xo + e * 128) : zero;
+          const uint4 x23 = live ? lds128(st + xo + e * 128 + 16) : zero;
 #pragma unroll
           for (int a = 0; a < TPW; ++a)
 #pragma unroll
