@@ -34,9 +34,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "ternary GEMV HBM GB/s & 8B linear-stack tok/s at M=1 (fraction of HBM peak)"
 # DRAM bytes (read + write) of the stream kernel per full 8B step, from the ncu capture summarised
-# in profiles/k_batch_stream_8b_4layers_bf16.md (4 layers: 203.17 MB read + 5.58 MB written),
+# in profiles/k_batch_stream_8b_4layers_bf16.md (4 layers: 203.17 MB read + 6.00 MB written),
 # scaled by the units processed (36 / 4 layers). Set to None whenever that kernel changes.
-STREAM_TRAFFIC_PER_STEP = 9 * (203.17e6 + 5.58e6)
+STREAM_TRAFFIC_PER_STEP = 9 * (203.17e6 + 6.00e6)
 SEED = 0x7E2A2026
 L2_BYTES = 126 * 1024 * 1024
 
