@@ -153,7 +153,7 @@ class _PackItem(ctypes.Structure):
 
 
 def tern_pack_batch(src_kind: int, entries, err_flag, stream=None) -> None:
-    """tern_pack over a list of (src, N, K, planes) in one call (one flag clear; one launch for base-3)."""
+    """tern_pack over a list of (src, N, K, planes) in one call (one flag clear, one launch)."""
     arr = (_PackItem * len(entries))()
     for i, (src, N, K, planes) in enumerate(entries):
         arr[i].src_dev, arr[i].N, arr[i].K, arr[i].planes_dev = _ptr(src), int(N), int(K), _ptr(planes)

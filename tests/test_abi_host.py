@@ -64,3 +64,51 @@ def test_argument_errors_before_launch(L):
         == tg.TERN_ESHAPE
     assert L.tern_quantize_act(fake, 0, 128, fake, fake, None) == tg.TERN_ESHAPE
     assert "TERN_ESHAPE" in tg.tern_status_string(tg.TERN_ESHAPE)
+
+
+def test_list_and_prefill_argument_errors_before_launch(L):
+    """tern_gemm_batch, tern_pack_batch and tern_gemm_prefill reject bad arguments before they
+    encode a tensor map or launch anything."""
+    import bit_gemv_tern_b200 as tg
+    fake = 1 << 40
+    ws = fake                                           # 16-byte aligned, never dereferenced
+    m = tg._Matrix(256, 4096, fake, fake)
+    items = (tg._Item * 2)()
+    for it in items:
+        it.W, it.x_dev, it.x_scale_dev, it.y_dev = m, fake, None, fake
+    assert L.tern_gemm_batch(items, 2, 17, 0, ws, 1 << 20, 0, None) == tg.TERN_ESHAPE          # M > 16
+    assert L.tern_gemm_batch(items, 2, 0, 0, ws, 1 << 20, 0, None) == tg.TERN_ESHAPE           # M < 1
+    assert L.tern_gemm_batch(items, 0, 1, 0, ws, 1 << 20, 0, None) == tg.TERN_ESHAPE           # empty list
+    assert L.tern_gemm_batch(items, 161, 1, 0, ws, 1 << 20, 0, None) == tg.TERN_ESHAPE         # > 160 items
+    assert L.tern_gemm_batch(None, 2, 1, 0, ws, 1 << 20, 0, None) == tg.TERN_EINVAL
+    assert L.tern_gemm_batch(items, 2, 1, 9, ws, 1 << 20, 0, None) == tg.TERN_EINVAL           # bad act
+    assert L.tern_gemm_batch(items, 2, 1, 1, ws, 1 << 20, 0, None) == tg.TERN_EINVAL           # int8 needs s_x
+    assert L.tern_gemm_batch(items, 2, 1, 0, ws + 8, 1 << 20, 0, None) == tg.TERN_EINVAL       # misaligned ws
+    assert L.tern_gemm_batch(items, 2, 1, 0, ws, 1 << 20, 4, None) == tg.TERN_EINVAL           # unknown flag
+    items[1].W = tg._Matrix(256, 16384, fake, fake)                                          # K > 12288
+    assert L.tern_gemm_batch(items, 2, 1, 0, ws, 1 << 20, 0, None) == tg.TERN_ESHAPE
+    items[1].W = m
+    items[1].x_dev = fake + 4                                                                # misaligned x
+    assert L.tern_gemm_batch(items, 2, 1, 0, ws, 1 << 20, 0, None) == tg.TERN_EINVAL
+
+    packs = (tg._PackItem * 2)()
+    for p in packs:
+        p.src_dev, p.N, p.K, p.planes_dev = fake, 64, 128, fake
+    flag = fake
+    assert L.tern_pack_batch(0, packs, 0, flag, None) == tg.TERN_ESHAPE                         # empty list
+    assert L.tern_pack_batch(0, packs, 257, flag, None) == tg.TERN_ESHAPE                       # > 256 items
+    assert L.tern_pack_batch(4, packs, 2, flag, None) == tg.TERN_EINVAL                         # bad source kind
+    assert L.tern_pack_batch(0, packs, 2, None, None) == tg.TERN_EINVAL                         # no flag
+    assert L.tern_pack_batch(0, None, 2, flag, None) == tg.TERN_EINVAL
+    packs[1].K = 96                                                                          # K % 128 != 0
+    assert L.tern_pack_batch(0, packs, 2, flag, None) == tg.TERN_ESHAPE
+    packs[1].K, packs[1].planes_dev = 128, fake + 4                                           # misaligned planes
+    assert L.tern_pack_batch(0, packs, 2, flag, None) == tg.TERN_EINVAL
+    packs[1].planes_dev, packs[1].src_dev = fake, fake + 4                                    # base-3 src: 4-aligned is fine,
+    assert L.tern_pack_batch(0, packs, 2, flag, None) == tg.TERN_EINVAL                        # int8 src needs 16
+
+    assert L.tern_gemm_prefill(ctypes.byref(m), 0, fake, fake, None) == tg.TERN_ESHAPE          # M < 1
+    assert L.tern_gemm_prefill(ctypes.byref(m), 65537, fake, fake, None) == tg.TERN_ESHAPE      # M > 65536
+    assert L.tern_gemm_prefill(ctypes.byref(m), 128, fake + 8, fake, None) == tg.TERN_EINVAL    # misaligned X
+    assert L.tern_gemm_prefill(ctypes.byref(m), 128, fake, fake + 2, None) == tg.TERN_EINVAL    # misaligned Y
+    assert L.tern_gemm_prefill(ctypes.byref(m), 128, None, fake, None) == tg.TERN_EINVAL
