@@ -67,8 +67,8 @@ def lib() -> ctypes.CDLL:
             "tern_pack_batch": ([i32, vp, i32, vp, vp], i32),
             "tern_occupancy": ([mp, vp, vp], i32),
             "tern_quantize_act": ([vp, i32, i32, vp, vp, vp], i32),
-            "tern_gemv": ([mp, i32, vp, vp, vp, vp], i32),
-            "tern_gemv_ex": ([mp, i32, vp, vp, vp, u32, vp], i32),
+            "tern_gemv": ([mp, i32, vp, vp, vp, vp, vp], i32),
+            "tern_gemv_ex": ([mp, i32, vp, vp, vp, vp, u32, vp], i32),
             "tern_gemm_small_m": ([mp, i32, i32, vp, vp, vp, vp], i32),
             "tern_gemm_small_m_ex": ([mp, i32, i32, vp, vp, vp, u32, vp], i32),
             "tern_gemm_prefill": ([mp, i32, vp, vp, vp], i32),
@@ -173,8 +173,10 @@ def tern_quantize_act(x_bf16, M: int, K: int, q, s_x, stream=None) -> None:
     _check(lib().tern_quantize_act(_ptr(x_bf16), M, K, _ptr(q), _ptr(s_x), _stream(stream)), "tern_quantize_act")
 
 
-def tern_gemv(W: TernMatrix, act: int, x, x_scale, y, flags: int = 0, stream=None) -> None:
-    _check(lib().tern_gemv_ex(W.ref(), act, _ptr(x), _ptr(x_scale), _ptr(y), flags, _stream(stream)), "tern_gemv")
+def tern_gemv(W: TernMatrix, act: int, x, x_scale, y, flags: int = 0, stream=None, acc=None) -> None:
+    """acc: optional int32 tensor of N elements; int8 mode writes the exact sums sum_k t*q there."""
+    _check(lib().tern_gemv_ex(W.ref(), act, _ptr(x), _ptr(x_scale), _ptr(y), _ptr(acc), flags, _stream(stream)),
+           "tern_gemv")
 
 
 def tern_gemm_small_m(W: TernMatrix, M: int, act: int, X, x_scale, Y, flags: int = 0, stream=None) -> None:

@@ -9,8 +9,6 @@
 
 namespace {
 
-constexpr int kSMs = 148;
-
 // Consumer warps of the M = 1 streaming kernel (8: two CTAs per SM; 16: one CTA per SM).
 #ifndef TERN_STREAM_CW
 #define TERN_STREAM_CW 16
@@ -35,8 +33,9 @@ tern_status check_matrix(const tern_matrix* W) {
 bool plan_gemm(int N, int K, int M, int mode, int& ksplit) {
   const int row_blocks = (N + tern::gemm_rows_per_cta() - 1) / tern::gemm_rows_per_cta();
   const int units = K / 128;
+  const int sms = tern::device_sm_count();
   int ks = 1;
-  while (ks < 8 && row_blocks * ks < 2 * kSMs && units % (2 * ks) == 0) ks *= 2;
+  while (ks < 8 && row_blocks * ks < 2 * sms && units % (2 * ks) == 0) ks *= 2;
   while (tern::gemm_smem_bytes(mode, M, K / ks) > kGemmSmemCap && ks < 8 && units % (2 * ks) == 0) ks *= 2;
   if (tern::gemm_smem_bytes(mode, M, K / ks) > kGemmSmemCap) return false;
   ksplit = ks;
@@ -44,6 +43,53 @@ bool plan_gemm(int N, int K, int M, int mode, int& ksplit) {
 }
 
 }  // namespace
+
+namespace tern {
+
+// Every argument check of i8_head_gemv_argmax_ex and its launch plan, with nothing enqueued.
+tern_status plan_head_call(const int8_t* W_dev, const uint16_t* scale_f16_dev, int32_t V, int32_t K, int32_t M,
+                           tern_act act, const void* X_dev, const float* x_scale_dev, int32_t* argmax_dev,
+                           float* maxval_dev, float* logits_dev, void* workspace_dev, size_t workspace_bytes,
+                           uint32_t flags, HeadParams& p) {
+  if (!W_dev || !scale_f16_dev || !X_dev || !argmax_dev || !maxval_dev || !workspace_dev) return TERN_EINVAL;
+  if (act != TERN_ACT_BF16 && act != TERN_ACT_INT8) return TERN_EINVAL;
+  if (flags & ~TERN_FLAG_PDL) return TERN_EINVAL;
+  if (!valid_shape(V, K) || M < 1 || M > 16) return TERN_ESHAPE;
+  if (!aligned(W_dev, 16) || !aligned(X_dev, 16) || !aligned(workspace_dev, 16) || !aligned(scale_f16_dev, 2))
+    return TERN_EINVAL;
+  if (!aligned(argmax_dev, 4) || !aligned(maxval_dev, 4) || (logits_dev && !aligned(logits_dev, 4)))
+    return TERN_EINVAL;
+  if (act == TERN_ACT_INT8 && (!x_scale_dev || !aligned(x_scale_dev, 4))) return TERN_EINVAL;
+  if (workspace_bytes < head_workspace_bytes(M)) return TERN_EINVAL;
+  p = HeadParams{};
+  p.W = W_dev;
+  p.sh = scale_f16_dev;
+  p.V = V;
+  p.K = K;
+  p.M = M;
+  p.mode = act == TERN_ACT_BF16 ? 0 : 1;
+  p.x = X_dev;
+  p.sx = x_scale_dev;
+  p.argmax = argmax_dev;
+  p.maxval = maxval_dev;
+  p.logits = logits_dev;
+  p.counter = static_cast<unsigned int*>(workspace_dev);
+  p.keys = reinterpret_cast<unsigned long long*>(static_cast<char*>(workspace_dev) + 16);
+  const int units = K / 128;
+  int ks = 1;
+  while (head_smem_bytes(p.mode, M, K / ks) > kHeadSmemCap && ks < 8 && units % (2 * ks) == 0) ks *= 2;
+  if (head_smem_bytes(p.mode, M, K / ks) > kHeadSmemCap) return TERN_ESHAPE;
+  p.ksplit = ks;
+  p.kr = K / ks;
+  p.nrb = (V + 127) / 128;
+  int nby = (2 * device_sm_count()) / ks;
+  if (nby > p.nrb) nby = p.nrb;
+  if (nby < 1) nby = 1;
+  p.nby = nby;
+  return TERN_OK;
+}
+
+}  // namespace tern
 
 extern "C" {
 
@@ -150,8 +196,12 @@ tern_status tern_quantize_act(const uint16_t* x_bf16_dev, int32_t M, int32_t K, 
   return from_cuda(tern::launch_quantize(x_bf16_dev, M, K, q_dev, s_x_dev, cs(stream)));
 }
 
-tern_status tern_gemm_small_m_ex(const tern_matrix* W, int32_t M, tern_act act, const void* X_dev,
-                                 const float* x_scale_dev, float* Y_dev, uint32_t flags, tern_stream_t stream) {
+namespace {
+
+// The single-matrix product behind tern_gemv and tern_gemm_small_m: the persistent stream kernel
+// for M = 1 where its plan fits, the cluster split-K kernel otherwise.
+tern_status gemm_one(const tern_matrix* W, int32_t M, tern_act act, const void* X_dev, const float* x_scale_dev,
+                     float* Y_dev, int32_t* acc_dev, uint32_t flags, tern_stream_t stream) {
   tern_status st = check_matrix(W);
   if (st != TERN_OK) return st;
   if (act != TERN_ACT_BF16 && act != TERN_ACT_INT8) return TERN_EINVAL;
@@ -159,6 +209,7 @@ tern_status tern_gemm_small_m_ex(const tern_matrix* W, int32_t M, tern_act act, 
   if (M < 1 || M > 16) return TERN_ESHAPE;
   if (!X_dev || !Y_dev || !aligned(X_dev, 16) || !aligned(Y_dev, 4)) return TERN_EINVAL;
   if (act == TERN_ACT_INT8 && (!x_scale_dev || !aligned(x_scale_dev, 4))) return TERN_EINVAL;
+  if (acc_dev && (act != TERN_ACT_INT8 || !aligned(acc_dev, 4))) return TERN_EINVAL;
   if (M == 1) {
     tern::StreamParams sp = {};
     sp.cw = TERN_STREAM_CW;
@@ -169,6 +220,7 @@ tern_status tern_gemm_small_m_ex(const tern_matrix* W, int32_t M, tern_act act, 
       sp.x = X_dev;
       sp.sx = x_scale_dev;
       sp.y = Y_dev;
+      sp.acc = acc_dev;
       return from_cuda(tern::launch_stream(sp, smem, (flags & TERN_FLAG_PDL) != 0, cs(stream)));
     }
   }
@@ -180,6 +232,7 @@ tern_status tern_gemm_small_m_ex(const tern_matrix* W, int32_t M, tern_act act, 
   p.x = X_dev;
   p.sx = x_scale_dev;
   p.y = Y_dev;
+  p.acc = acc_dev;
   p.M = M;
   p.mode = act == TERN_ACT_BF16 ? 0 : 1;
   if (!plan_gemm(p.N, p.K, M, p.mode, p.ksplit)) return TERN_ESHAPE;
@@ -187,19 +240,26 @@ tern_status tern_gemm_small_m_ex(const tern_matrix* W, int32_t M, tern_act act, 
   return from_cuda(tern::launch_tern_gemm(p, (flags & TERN_FLAG_PDL) != 0, cs(stream)));
 }
 
+}  // namespace
+
+tern_status tern_gemm_small_m_ex(const tern_matrix* W, int32_t M, tern_act act, const void* X_dev,
+                                 const float* x_scale_dev, float* Y_dev, uint32_t flags, tern_stream_t stream) {
+  return gemm_one(W, M, act, X_dev, x_scale_dev, Y_dev, nullptr, flags, stream);
+}
+
 tern_status tern_gemm_small_m(const tern_matrix* W, int32_t M, tern_act act, const void* X_dev,
                               const float* x_scale_dev, float* Y_dev, tern_stream_t stream) {
-  return tern_gemm_small_m_ex(W, M, act, X_dev, x_scale_dev, Y_dev, 0u, stream);
+  return gemm_one(W, M, act, X_dev, x_scale_dev, Y_dev, nullptr, 0u, stream);
 }
 
 tern_status tern_gemv_ex(const tern_matrix* W, tern_act act, const void* x_dev, const float* x_scale_dev,
-                         float* y_dev, uint32_t flags, tern_stream_t stream) {
-  return tern_gemm_small_m_ex(W, 1, act, x_dev, x_scale_dev, y_dev, flags, stream);
+                         float* y_dev, int32_t* acc_i32_dev, uint32_t flags, tern_stream_t stream) {
+  return gemm_one(W, 1, act, x_dev, x_scale_dev, y_dev, acc_i32_dev, flags, stream);
 }
 
 tern_status tern_gemv(const tern_matrix* W, tern_act act, const void* x_dev, const float* x_scale_dev,
-                      float* y_dev, tern_stream_t stream) {
-  return tern_gemm_small_m_ex(W, 1, act, x_dev, x_scale_dev, y_dev, 0u, stream);
+                      float* y_dev, int32_t* acc_i32_dev, tern_stream_t stream) {
+  return gemm_one(W, 1, act, x_dev, x_scale_dev, y_dev, acc_i32_dev, 0u, stream);
 }
 
 namespace {
@@ -280,41 +340,10 @@ tern_status i8_head_gemv_argmax_ex(const int8_t* W_dev, const uint16_t* scale_f1
                                    int32_t* argmax_dev, float* maxval_dev, float* logits_dev,
                                    void* workspace_dev, size_t workspace_bytes, uint32_t flags,
                                    tern_stream_t stream) {
-  if (!W_dev || !scale_f16_dev || !X_dev || !argmax_dev || !maxval_dev || !workspace_dev) return TERN_EINVAL;
-  if (act != TERN_ACT_BF16 && act != TERN_ACT_INT8) return TERN_EINVAL;
-  if (flags & ~TERN_FLAG_PDL) return TERN_EINVAL;
-  if (!valid_shape(V, K) || M < 1 || M > 16) return TERN_ESHAPE;
-  if (!aligned(W_dev, 16) || !aligned(X_dev, 16) || !aligned(workspace_dev, 16) || !aligned(scale_f16_dev, 2))
-    return TERN_EINVAL;
-  if (!aligned(argmax_dev, 4) || !aligned(maxval_dev, 4) || (logits_dev && !aligned(logits_dev, 4)))
-    return TERN_EINVAL;
-  if (act == TERN_ACT_INT8 && (!x_scale_dev || !aligned(x_scale_dev, 4))) return TERN_EINVAL;
-  if (workspace_bytes < tern::head_workspace_bytes(M)) return TERN_EINVAL;
   tern::HeadParams p = {};
-  p.W = W_dev;
-  p.sh = scale_f16_dev;
-  p.V = V;
-  p.K = K;
-  p.M = M;
-  p.mode = act == TERN_ACT_BF16 ? 0 : 1;
-  p.x = X_dev;
-  p.sx = x_scale_dev;
-  p.argmax = argmax_dev;
-  p.maxval = maxval_dev;
-  p.logits = logits_dev;
-  p.counter = static_cast<unsigned int*>(workspace_dev);
-  p.keys = reinterpret_cast<unsigned long long*>(static_cast<char*>(workspace_dev) + 16);
-  const int units = K / 128;
-  int ks = 1;
-  while (tern::head_smem_bytes(p.mode, M, K / ks) > kHeadSmemCap && ks < 8 && units % (2 * ks) == 0) ks *= 2;
-  if (tern::head_smem_bytes(p.mode, M, K / ks) > kHeadSmemCap) return TERN_ESHAPE;
-  p.ksplit = ks;
-  p.kr = K / ks;
-  p.nrb = (V + 127) / 128;
-  int nby = (2 * kSMs) / ks;
-  if (nby > p.nrb) nby = p.nrb;
-  if (nby < 1) nby = 1;
-  p.nby = nby;
+  const tern_status st = tern::plan_head_call(W_dev, scale_f16_dev, V, K, M, act, X_dev, x_scale_dev, argmax_dev,
+                                              maxval_dev, logits_dev, workspace_dev, workspace_bytes, flags, p);
+  if (st != TERN_OK) return st;
   return from_cuda(tern::launch_head(p, (flags & TERN_FLAG_PDL) != 0, cs(stream)));
 }
 

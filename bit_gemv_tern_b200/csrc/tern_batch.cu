@@ -6,25 +6,29 @@
 // A decode step streams every weight of the stack once per token (PyTorchKR review "Fermion
 // Research, 3진 계열 포맷으로 직접 학습한 Neutrino-1 모델군 3종 공개", section "뉴트리노 엔진":
 // tok/s_max = memory bandwidth / bytes per token); the same section measures most of the time above
-// that floor at the ~120 kernel boundaries of a step. Here the boundaries are gone: one persistent
-// launch walks all items, so the weight stream never pauses between layers.
+// that floor at the ~120 kernel boundaries of a step. Here one persistent launch walks all items, so
+// the weight stream never pauses between layers.
 //
 //   1. k_batch_prep (one CTA per item and token slot) turns each activation into ready-to-load
-//      tensor-core operand segments, one per 512-trit K part: int8 q permuted to the decode's byte order (int8 mode),
-//      or three exact int8 limbs of a 22-bit fixed-point value relative to 2^E with E from the
-//      item's absmax (bf16 mode), followed by the item's column sums (which remove the decode
-//      offset) and E. Tokens occupy the MMA's n-columns (see seg_cols).
+//      tensor-core operand segments, one per 512-trit K part: int8 q permuted to the decode's byte
+//      order (int8 mode), or four exact int8 limbs of a 30-bit fixed-point value relative to 2^E with
+//      E from the item's absmax (bf16 mode, see tern_device.cuh), followed by the item's column sums
+//      (which remove the decode offset) and E. Tokens occupy the MMA's n-columns (see seg_cols).
 //   2. k_batch_stream (one CTA per SM) splits the list's (row block, K part) sequence evenly by
-//      bytes, so a row block may be shared by neighbouring CTAs. Its producer lane walks the CTA's row blocks part by part: each stage of
-//      the ring receives, by tensor TMA, the mask and sign words of the block's rows for one K part
-//      (the packed planes seen as a [plane][row][word] tensor, so the row-major layout is read in
-//      place) plus that part's operand segment. The consumer warps walk the stages in order; warp
-//      w owns kTPW tiles of 16 rows of the block, decodes them (one AND per operand register, see
-//      tern_device.cuh) into mma.sync u8 x s8 products, and keeps the sums in registers across all
-//      parts of the block, so a tile's outputs are written once, at its end.
+//      bytes, so a row block may be shared by neighbouring CTAs. Its producer lane walks the CTA's
+//      row blocks part by part: each stage of the ring receives, by tensor TMA, the mask and sign
+//      words of the block's rows for one K part (the packed planes seen as a [plane][row][word]
+//      tensor, so the row-major layout is read in place) plus that part's operand segment. The
+//      consumer warps walk the stages in order; warp w owns kTPW tiles of 16 rows of the block,
+//      decodes them (one AND per operand register, see tern_device.cuh) into mma.sync u8 x s8
+//      products, and keeps the sums in registers across all parts of the block, so a tile's
+//      outputs are written once, at its end. Shapes with many operand columns (bf16 mode, 8 or 16
+//      token slots) decode to signed 64 * t bytes instead (shift and AND) and keep one accumulator
+//      per column group rather than four.
 // All sums are exact integers; int8 mode ends with y = ((float)acc * s_x) * scale (two fp32
 // round-to-nearest multiplies), bf16 mode with one fp64 -> fp32 rounding. Every mbarrier wait is
 // bounded and latches TERN_ETIMEOUT on give-up.
+#include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -49,7 +53,6 @@ __host__ __device__ constexpr int box_rows(int cw) { return cw * 16; }
 __host__ __device__ constexpr int box_bytes(int cw) { return 2 * box_rows(cw) * kPartWords * 4; }
 constexpr int kColWords = 132;                        // operand words per column and part (128 + bank skew)
 constexpr uint32_t kWaitTries = 1u << 13;
-constexpr int kLimbFrac = 22;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -110,12 +113,16 @@ __device__ __forceinline__ void store_operand_half(uint32_t* slot, int h, uint4 
 }
 
 // ---------------------------------------------------------------------------------------------
-// Operand columns of a segment. M = 1 (mp == 1): the nc columns are the limbs L2, L1, L0 (bf16
-// mode) or q (int8 mode). M >= 2: int8 mode (mp = 8 or 16 token slots) column m = token m; bf16
-// mode column l * mp + m = limb l of token m. With mp = 8 or 16 each MMA group of 8 columns holds
-// one limb of eight tokens and a lane ends up with all three limbs of the tokens it owns; with
-// mp = 2 or 4 the 6 or 12 columns fill one or two groups and the epilogue gathers the limbs.
-__host__ __device__ constexpr int seg_cols(int mode, int mp) { return mp == 1 ? (mode == 0 ? 3 : 1) : (mode == 0 ? 3 * mp : mp); }
+// Operand columns of a segment. M = 1 (mp == 1): the nc columns are the limbs L3, L2, L1, L0
+// (bf16 mode, top limb first) or q (int8 mode). M >= 2: int8 mode (mp = 8 or 16 token slots)
+// column m = token m; bf16 mode column l * mp + m = limb l of token m. With mp = 8 or 16 each MMA
+// group of 8 columns holds one limb of eight tokens and a lane ends up with all four limbs of the
+// tokens it owns; with mp = 2 or 4 the 8 or 16 columns fill one or two groups and the epilogue
+// gathers the limbs.
+constexpr int kLimbs = 4;
+__host__ __device__ constexpr int seg_cols(int mode, int mp) {
+  return mp == 1 ? (mode == 0 ? kLimbs : 1) : (mode == 0 ? kLimbs * mp : mp);
+}
 // Segment words: columns, then the column sums over all of K, then E per token slot, padded to 16 B.
 __host__ __device__ constexpr int seg_words(int mode, int mp) {
   return (seg_cols(mode, mp) * kColWords + seg_cols(mode, mp) + mp + 3) & ~3;
@@ -132,12 +139,12 @@ __global__ void __launch_bounds__(kPrepThreads) k_batch_prep(const __grid_consta
   const int K = it.K, KP = it.kp, mp = p.mp;
   const int ncols = seg_cols(p.mode, mp);
   const int segw = p.seg_bytes / 4;
-  const int nl = p.mode == 0 ? 3 : 1;                // columns of this token
-  int colof[3];
-  for (int l = 0; l < 3; ++l) colof[l] = mp == 1 ? l : l * mp + m;
+  const int nl = p.mode == 0 ? kLimbs : 1;           // columns of this token
+  int colof[kLimbs];
+  for (int l = 0; l < kLimbs; ++l) colof[l] = mp == 1 ? l : l * mp + m;
   const bool live = m < p.M;
   __shared__ float red[kPrepThreads / 32];
-  __shared__ int sums[3];
+  __shared__ int sums[kLimbs];
   __shared__ int Esh;
   pdl_wait();
   {
@@ -158,9 +165,8 @@ __global__ void __launch_bounds__(kPrepThreads) k_batch_prep(const __grid_consta
       blk[part * segw + colof[c] * kColWords + part_slot(wl + j / 8) + j % 8] = 0u;
     }
   }
-  if (threadIdx.x < 3) sums[threadIdx.x] = 0;
+  if (threadIdx.x < kLimbs) sums[threadIdx.x] = 0;
   if (threadIdx.x == 0) Esh = 0;
-  float f = 1.0f;
   if (p.mode == 0 && live) {
     const uint16_t* xb = static_cast<const uint16_t*>(it.x) + (size_t)m * K;
     float amax = 0.0f;
@@ -177,19 +183,13 @@ __global__ void __launch_bounds__(kPrepThreads) k_batch_prep(const __grid_consta
     if (threadIdx.x == 0) {
       float mx = red[0];
       for (int i = 1; i < kPrepThreads / 32; ++i) mx = fmaxf(mx, red[i]);
-      int E = 0;
-      if (mx > 0.0f) {
-        frexpf(mx, &E);                              // mx < 2^E
-        E = max(E, -100);
-      }
-      Esh = E;
+      Esh = limb_exponent(mx);
     }
-    __syncthreads();
-    f = ldexpf(1.0f, kLimbFrac - Esh);
   }
   __syncthreads();
+  const int E = Esh;
   // one 16-element half of a 32-trit word per thread iteration
-  int ls[3] = {0, 0, 0};
+  int ls[kLimbs] = {0, 0, 0, 0};
   for (int v = threadIdx.x; live && v < K / 16; v += blockDim.x) {
     const int word = v >> 1, h = v & 1;              // global word index and half
     const int part = word >> 4, w = word & 15;
@@ -202,22 +202,18 @@ __global__ void __launch_bounds__(kPrepThreads) k_batch_prep(const __grid_consta
       const uint16_t* xb = static_cast<const uint16_t*>(it.x) + (size_t)m * K + 16 * v;
       const uint4 a = ld_nc(xb), b = ld_nc(xb + 8);
       const uint32_t wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-      uint32_t l[3][4] = {};
+      uint32_t l[kLimbs][4] = {};
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
         const uint32_t bits = (e & 1) ? (wv[e >> 1] >> 16) : (wv[e >> 1] & 0xFFFFu);
-        const int X = __float2int_rn(bf16_bits_to_float(bits) * f);   // exact power-of-two scaling
-        const int L0 = (int)(int8_t)(X & 0xFF);
-        const int X1 = (X - L0) >> 8;
-        const int L1 = (int)(int8_t)(X1 & 0xFF);
-        const int L2 = (X1 - L1) >> 8;                                 // |L2| <= 64
+        int L[kLimbs];
+        limbs_of(limb_fixed(bf16_bits_to_float(bits), E), L);
         const int sh = 8 * (e & 3);
-        l[0][e >> 2] |= (uint32_t)(uint8_t)L2 << sh;
-        l[1][e >> 2] |= (uint32_t)(uint8_t)L1 << sh;
-        l[2][e >> 2] |= (uint32_t)(uint8_t)L0 << sh;
+#pragma unroll
+        for (int c = 0; c < kLimbs; ++c) l[c][e >> 2] |= (uint32_t)(uint8_t)L[c] << sh;
       }
 #pragma unroll
-      for (int c = 0; c < 3; ++c) {
+      for (int c = 0; c < kLimbs; ++c) {
         ls[c] += bsum(l[c][0]) + bsum(l[c][1]) + bsum(l[c][2]) + bsum(l[c][3]);
         store_operand_half(seg + colof[c] * kColWords, h, permute_i8_half(make_uint4(l[c][0], l[c][1], l[c][2], l[c][3])));
       }
@@ -233,15 +229,17 @@ __global__ void __launch_bounds__(kPrepThreads) k_batch_prep(const __grid_consta
   for (int part = threadIdx.x; part < KP; part += blockDim.x) {
     int* meta = reinterpret_cast<int*>(blk + part * segw + ncols * kColWords);
     for (int c = 0; c < nl; ++c) meta[colof[c]] = sums[c];
-    meta[ncols + m] = Esh;
+    meta[ncols + m] = E;
   }
   pdl_launch_dependents();
 }
 
 // ---------------------------------------------------------------------------------------------
 // MODE: 0 bf16 / 1 int8 activations; MP: token slots (1, 2, 4, 8 or 16; 2 and 4 in bf16 mode
-// only); TPW: tiles per consumer warp; CW: consumer warps.
-template <int MODE, int MP, int TPW, int CW>
+// only); TPW: tiles per consumer warp; CW: consumer warps; SGN: signed decode (bytes 64 * t, one
+// accumulator per column group, no offset to remove) instead of the offset decode (bytes
+// 4^i * (t + 2), four field accumulators per group).
+template <int MODE, int MP, int TPW, int CW, bool SGN>
 __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_constant__ BatchParams p) {
   constexpr int kCW = CW;
   constexpr int kBoxRows = box_rows(CW);
@@ -348,6 +346,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
   }
 
   // ====================== consumers ======================
+  constexpr int NF = SGN ? 1 : 4;                           // accumulators per column group
   const int g = lane >> 2, t = lane & 3;
   // operand column of group j this lane feeds: M = 1: the lane's limb (rows g >= nc repeat column 0)
   // columns past NCOL (M = 1, PACK) repeat a real column; their sums are never read
@@ -364,9 +363,15 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
   const uint32_t mofs = (uint32_t)(kWStageBytesT + NCOL * kColWords * 4);
   const int M = p.M;
   constexpr int NCOLP = 8 * G;                              // scratch columns per row
+  constexpr int NL = MODE == 0 ? kLimbs : 1;                // columns per token
   const uint32_t split = p.cta_split[blockIdx.x];
   const int slot_first = (int)(split & 0xFFu) - 1, need_first = (int)((split >> 8) & 0xFFu);
   const int slot_last = (int)((split >> 16) & 0xFFu) - 1, need_last = (int)(split >> 24);
+  auto lds32 = [](uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return (int)v;
+  };
   bool ok = true;
   int it = first_item, rb = first_rb, pstart = first_part;
   int s = 0;
@@ -379,18 +384,27 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
     if (gq == g0) { slot = slot_first; need = need_first; }
     if (gq + (pend - pstart) == g1 && slot_last >= 0) { slot = slot_last; need = need_last; }
     const int row_base = rb * kStageRowsT + warp * 16;         // first row of this warp's tile slot 0
-    int acc[TPW][G][4][4];
+    int acc[TPW][G][NF][4];
 #pragma unroll
     for (int a = 0; a < TPW; ++a)
 #pragma unroll
       for (int j = 0; j < G; ++j)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[a][j][i][0] = acc[a][j][i][1] = acc[a][j][i][2] = acc[a][j][i][3] = 0;
-    // column sums (over all of K) and exponents of the columns this lane owns
-    //   M = 1: tot[c] for c < nc, E; M >= 2: [jj][limb][token parity], E per [jj][parity]
-    int tot[JJ][3][2];
+        for (int i = 0; i < NF; ++i) acc[a][j][i][0] = acc[a][j][i][1] = acc[a][j][i][2] = acc[a][j][i][3] = 0;
+    // column sums (over all of K; they remove the decode offset) and exponents of the columns this
+    // lane owns.  M = 1: tot[0][c][0] for every column c, E;  M >= 2: [jj][limb][token parity], E
+    // per [jj][parity]
+    int tot[JJ][kLimbs][2];
     int Etok[JJ][2];
     float sxv[JJ][2];
+#pragma unroll
+    for (int jj = 0; jj < JJ; ++jj)
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        Etok[jj][b] = 0;
+#pragma unroll
+        for (int l = 0; l < kLimbs; ++l) tot[jj][l][b] = 0;
+      }
     // the epilogue's reads of the row scales (weights: written before any launch of this list),
     // issued now so that they land while the block streams
     uint16_t sc_bits[TPW][2];
@@ -432,15 +446,27 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
 #pragma unroll
         for (int a = 0; a < TPW; ++a) {
           uint32_t wa0, wb0, wa1, wb1;
-          merge_planes_offset(u4get(ma[a], e), u4get(sa[a], e), wa0, wb0);
-          merge_planes_offset(u4get(mb[a], e), u4get(sb[a], e), wa1, wb1);
+          if (SGN) {
+            merge_planes(u4get(ma[a], e), u4get(sa[a], e), wa0, wb0);
+            merge_planes(u4get(mb[a], e), u4get(sb[a], e), wa1, wb1);
+          } else {
+            merge_planes_offset(u4get(ma[a], e), u4get(sa[a], e), wa0, wb0);
+            merge_planes_offset(u4get(mb[a], e), u4get(sb[a], e), wa1, wb1);
+          }
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const uint32_t msk = 0x03030303u << (2 * i);
-            A[a][i][0] = wa0 & msk;
-            A[a][i][1] = wa1 & msk;
-            A[a][i][2] = wb0 & msk;
-            A[a][i][3] = wb1 & msk;
+            if (SGN) {                                      // field i of every byte -> 64 * t
+              A[a][i][0] = (wa0 << (6 - 2 * i)) & 0xC0C0C0C0u;
+              A[a][i][1] = (wa1 << (6 - 2 * i)) & 0xC0C0C0C0u;
+              A[a][i][2] = (wb0 << (6 - 2 * i)) & 0xC0C0C0C0u;
+              A[a][i][3] = (wb1 << (6 - 2 * i)) & 0xC0C0C0C0u;
+            } else {                                        // field i in place -> 4^i * (t + 2)
+              const uint32_t msk = 0x03030303u << (2 * i);
+              A[a][i][0] = wa0 & msk;
+              A[a][i][1] = wa1 & msk;
+              A[a][i][2] = wb0 & msk;
+              A[a][i][3] = wb1 & msk;
+            }
           }
         }
 #pragma unroll
@@ -454,54 +480,42 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
 #pragma unroll
           for (int a = 0; a < TPW; ++a)
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              mma_u8s8(acc[a][j][i], A[a][i][0], A[a][i][1], A[a][i][2], A[a][i][3],
-                       i < 2 ? u4get(x01, 2 * i) : u4get(x23, 2 * i - 4),
-                       i < 2 ? u4get(x01, 2 * i + 1) : u4get(x23, 2 * i - 3));
+            for (int i = 0; i < 4; ++i) {
+              const uint32_t b0 = i < 2 ? u4get(x01, 2 * i) : u4get(x23, 2 * i - 4);
+              const uint32_t b1 = i < 2 ? u4get(x01, 2 * i + 1) : u4get(x23, 2 * i - 3);
+              if (SGN)
+                mma_s8(acc[a][j][0], A[a][i][0], A[a][i][1], A[a][i][2], A[a][i][3], b0, b1);
+              else
+                mma_u8s8(acc[a][j][i], A[a][i][0], A[a][i][1], A[a][i][2], A[a][i][3], b0, b1);
+            }
         }
       }
       if (part == pend - 1) {                                // sums over all of K and E ride in every segment
+        if (MP == 1) {
+          const uint4 m4 = lds128(st + mofs);               // the NCOL (<= 4) column sums
+          tot[0][0][0] = (int)m4.x;
+          tot[0][1][0] = (int)m4.y;
+          tot[0][2][0] = (int)m4.z;
+          tot[0][3][0] = (int)m4.w;
+          if (MODE == 0) Etok[0][0] = lds32(st + mofs + 4u * NCOL);
+        } else if (PACK) {
+          // lane t reads token t: its column sums and E
+          const int m = t < MP ? t : 0;
 #pragma unroll
-        for (int jj = 0; jj < JJ; ++jj)
+          for (int l = 0; l < kLimbs; ++l) tot[0][l][0] = lds32(st + mofs + 4u * (uint32_t)(l * MP + m));
+          Etok[0][0] = lds32(st + mofs + 4u * (uint32_t)(NCOL + m));
+        } else {
 #pragma unroll
-          for (int b = 0; b < 2; ++b) {
-            if (MP == 1) {
-              if (jj == 0 && b == 0) {
-                const uint4 m4 = lds128(st + mofs);
-                tot[0][0][0] = (int)m4.x;
-                tot[0][1][0] = (int)m4.y;
-                tot[0][2][0] = (int)m4.z;
-                Etok[0][0] = MODE == 0 ? (int)m4.w : 0;
-              }
-            } else if (PACK) {
-              // lane t writes token t: its three column sums and E
-              if (jj == 0 && b == 0) {
-                const int m = t < MP ? t : 0;
+          for (int jj = 0; jj < JJ; ++jj)
 #pragma unroll
-                for (int l = 0; l < 3; ++l) {
-                  uint32_t v;
-                  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(st + mofs + 4u * (uint32_t)(l * MP + m)));
-                  tot[0][l][0] = (int)v;
-                }
-                uint32_t ev;
-                asm volatile("ld.shared.u32 %0, [%1];" : "=r"(ev) : "r"(st + mofs + 4u * (uint32_t)(NCOL + m)));
-                Etok[0][0] = (int)ev;
-              }
-            } else {
+            for (int b = 0; b < 2; ++b) {
               const int m = 8 * jj + 2 * t + b;
+              if (!SGN)
 #pragma unroll
-              for (int l = 0; l < 3; ++l) {
-                if (MODE == 0 || l == 0) {
-                  uint32_t v;
-                  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(st + mofs + 4u * (uint32_t)(l * MP + m)));
-                  tot[jj][l][b] = (int)v;
-                }
-              }
-              uint32_t ev;
-              asm volatile("ld.shared.u32 %0, [%1];" : "=r"(ev) : "r"(st + mofs + 4u * (uint32_t)(NCOL + m)));
-              Etok[jj][b] = (int)ev;
+                for (int l = 0; l < NL; ++l) tot[jj][l][b] = lds32(st + mofs + 4u * (uint32_t)(l * MP + m));
+              if (MODE == 0) Etok[jj][b] = lds32(st + mofs + 4u * (uint32_t)(NCOL + m));
             }
-          }
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(empty0 + 8 * s);
@@ -509,7 +523,8 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
     }
     if (!ok) break;
     // ---- outputs of this warp's tiles: exact integer sums, one rounding ----------------------------
-    // the four field accumulators of each (row, column) combined exactly
+    // the field accumulators of each (row, column) combined exactly (the offset is removed below;
+    // the signed decode carries the factor 64)
     int V[TPW][G][4];
 #pragma unroll
     for (int a = 0; a < TPW; ++a)
@@ -517,7 +532,9 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
       for (int j = 0; j < G; ++j)
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          V[a][j][q] = acc[a][j][0][q] + (acc[a][j][1][q] >> 2) + (acc[a][j][2][q] >> 4) + (acc[a][j][3][q] >> 6);
+          V[a][j][q] = SGN ? (acc[a][j][0][q] >> 6)
+                           : acc[a][j][0][q] + (acc[a][j][NF > 1 ? 1 : 0][q] >> 2) +
+                                 (acc[a][j][NF > 2 ? 2 : 0][q] >> 4) + (acc[a][j][NF > 3 ? 3 : 0][q] >> 6);
     bool emit = true;
     if (slot >= 0) {
       // a block split between CTAs: add this CTA's part sums; the last contributor (per warp)
@@ -575,18 +592,17 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
             }
           }
         } else {
-          // lane t = 0 holds columns 0 (L2) and 1 (L1), lane t = 1 column 2 (L0)
-          const int l0a = __shfl_down_sync(0xFFFFFFFFu, v[0], 1);
-          const int l0b = __shfl_down_sync(0xFFFFFFFFu, v[2], 1);
+          // lane t = 0 holds columns 0 (L3) and 1 (L2), lane t = 1 columns 2 (L1) and 3 (L0)
+          int w[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) w[q] = __shfl_down_sync(0xFFFFFFFFu, v[q], 1);
           if (t == 0) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               const int row = r0 + 8 * h;
               if (row < B.N) {
-                const long long S2 = v[2 * h] - 2LL * tot[0][0][0];
-                const long long S1 = v[2 * h + 1] - 2LL * tot[0][1][0];
-                const long long S0 = (h ? l0b : l0a) - 2LL * tot[0][2][0];
-                const long long D = S2 * 65536 + S1 * 256 + S0;
+                const long long D = limb_combine(v[2 * h] - 2LL * tot[0][0][0], v[2 * h + 1] - 2LL * tot[0][1][0],
+                                                 w[2 * h] - 2LL * tot[0][2][0], w[2 * h + 1] - 2LL * tot[0][3][0]);
                 B.y[row] = (float)((double)D * exp2_i(Etok[0][0] - kLimbFrac) * (double)f16_bits_to_float(sc_bits[a][h]));
               }
             }
@@ -600,17 +616,15 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
           const int row = r0 + 8 * h;
 #pragma unroll
           for (int m = 0; m < MP; ++m) {
-            int L[3];
+            long long L[kLimbs];
 #pragma unroll
-            for (int l = 0; l < 3; ++l) {
+            for (int l = 0; l < kLimbs; ++l) {
               const int c = l * MP + m;
-              L[l] = __shfl_sync(0xFFFFFFFFu, V[a][c >> 3][2 * h + (c & 1)], (lane & ~3) | ((c & 7) >> 1));
+              L[l] = __shfl_sync(0xFFFFFFFFu, V[a][c >> 3][2 * h + (c & 1)], (lane & ~3) | ((c & 7) >> 1)) -
+                     2LL * tot[0][l][0];
             }
             if (t == m && m < M && row < B.N) {
-              const long long S2 = L[0] - 2LL * tot[0][0][0];
-              const long long S1 = L[1] - 2LL * tot[0][1][0];
-              const long long S0 = L[2] - 2LL * tot[0][2][0];
-              const long long D = S2 * 65536 + S1 * 256 + S0;
+              const long long D = limb_combine(L[0], L[1], L[2], L[3]);
               B.y[(size_t)m * B.N + row] =
                   (float)((double)D * exp2_i(Etok[0][0] - kLimbFrac) * (double)f16_bits_to_float(sc_bits[a][h]));
             }
@@ -632,12 +646,10 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
                 const int S1 = V[a][jj][q] - 2 * tot[jj][0][b];
                 B.y[(size_t)m * B.N + row] = __fmul_rn(__fmul_rn(__int2float_rn(S1), sxv[jj][b]), sc);
               } else {
-                long long Sl[3];
+                long long Sl[kLimbs];
 #pragma unroll
-                for (int l = 0; l < 3; ++l) {
-                  Sl[l] = (long long)V[a][l * JJ + jj][q] - 2LL * tot[jj][l][b];
-                }
-                const long long D = Sl[0] * 65536 + Sl[1] * 256 + Sl[2];
+                for (int l = 0; l < kLimbs; ++l) Sl[l] = (long long)V[a][l * JJ + jj][q] - 2LL * tot[jj][l][b];
+                const long long D = limb_combine(Sl[0], Sl[1], Sl[2], Sl[3]);
                 B.y[(size_t)m * B.N + row] = (float)((double)D * exp2_i(Etok[jj][b] - kLimbFrac) * (double)sc);
               }
             }
@@ -664,35 +676,32 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // Token slots, tiles per warp and consumer warps for M rows: the accumulators (tiles x groups x
-// 16 registers) stay at or under 96 registers.
+// fields x 4 registers) stay at or under 64 registers.
 void batch_shape(int mode, int M, int& mp, int& tpw, int& cw) {
-  if (M == 1 || (mode == 0 && M == 2)) {       // one MMA group: 1 or 3 columns, or 2 x 3 limbs
+  if (M == 1 || (mode == 0 && M == 2)) {       // one MMA group: 1 or 4 columns, or 2 x 4 limbs
     mp = M;
     tpw = 2;
     cw = 12;
     return;
   }
-  if (mode == 0 && M <= 4) {                    // 4 x 3 limbs in two groups
+  if (mode == 0 && M <= 4) {                    // 4 x 4 limbs in two groups
     mp = 4;
     tpw = 2;
     cw = 11;
     return;
   }
-  mp = M <= 8 ? 8 : 16;
+  mp = M <= 8 ? 8 : 16;                         // bf16: 4 or 8 groups, signed decode
   tpw = mode == 0 ? 1 : 2;
   cw = 11;
 }
 
-template <int MODE, int MP, int TPW, int CW>
-cudaError_t launch_stream_kernel(cudaLaunchConfig_t& cfg, const BatchParams& p, size_t smem) {
-  static int set = 0;
-  if ((int)smem > set) {
-    cudaError_t e = cudaFuncSetAttribute(k_batch_stream<MODE, MP, TPW, CW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    set = (int)smem;
-  }
+template <int MODE, int MP, int TPW, int CW, bool SGN = false>
+cudaError_t launch_stream_kernel(cudaLaunchConfig_t& cfg, const BatchParams& p) {
+  static std::atomic<unsigned long long> smem_raised{0};
+  cudaError_t e = allow_max_dynamic_smem(k_batch_stream<MODE, MP, TPW, CW, SGN>, smem_raised);
+  if (e != cudaSuccess) return e;
   cfg.blockDim = dim3((CW + 1) * 32, 1, 1);
-  return cudaLaunchKernelEx(&cfg, k_batch_stream<MODE, MP, TPW, CW>, p);
+  return cudaLaunchKernelEx(&cfg, k_batch_stream<MODE, MP, TPW, CW, SGN>, p);
 }
 
 }  // namespace
@@ -741,7 +750,7 @@ bool plan_batch(BatchParams& p, const uint32_t* const* planes, size_t& smem, siz
   p.total_units = units;
   // CTA c starts at the first part whose cost prefix reaches c/G of the total: the split is
   // balanced to one 512-trit part, and a row block may be shared by neighbouring CTAs
-  const int grid = parts < 148 ? parts : 148;
+  const int grid = persistent_grid(parts);
   p.grid = grid;
   {
     int c = 1;
@@ -853,15 +862,15 @@ cudaError_t launch_batch(const BatchParams& p, size_t smem, bool pdl, cudaStream
   cfg.gridDim = dim3(p.grid, 1, 1);
   cfg.dynamicSmemBytes = smem;
   if (p.mode == 0) {
-    if (p.mp == 1) return launch_stream_kernel<0, 1, 2, 12>(cfg, p, smem);
-    if (p.mp == 2) return launch_stream_kernel<0, 2, 2, 12>(cfg, p, smem);
-    if (p.mp == 4) return launch_stream_kernel<0, 4, 2, 11>(cfg, p, smem);
-    if (p.mp == 8) return launch_stream_kernel<0, 8, 1, 11>(cfg, p, smem);
-    return launch_stream_kernel<0, 16, 1, 11>(cfg, p, smem);
+    if (p.mp == 1) return launch_stream_kernel<0, 1, 2, 12>(cfg, p);
+    if (p.mp == 2) return launch_stream_kernel<0, 2, 2, 12>(cfg, p);
+    if (p.mp == 4) return launch_stream_kernel<0, 4, 2, 11>(cfg, p);
+    if (p.mp == 8) return launch_stream_kernel<0, 8, 1, 11, true>(cfg, p);
+    return launch_stream_kernel<0, 16, 1, 11, true>(cfg, p);
   }
-  if (p.mp == 1) return launch_stream_kernel<1, 1, 2, 12>(cfg, p, smem);
-  if (p.mp == 8) return launch_stream_kernel<1, 8, 2, 11>(cfg, p, smem);
-  return launch_stream_kernel<1, 16, 2, 11>(cfg, p, smem);
+  if (p.mp == 1) return launch_stream_kernel<1, 1, 2, 12>(cfg, p);
+  if (p.mp == 8) return launch_stream_kernel<1, 8, 2, 11>(cfg, p);
+  return launch_stream_kernel<1, 16, 2, 11>(cfg, p);
 }
 
 }  // namespace tern

@@ -130,6 +130,45 @@ __device__ __forceinline__ float f16_bits_to_float(uint16_t h) {
 }
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t b) { return __uint_as_float(b << 16); }
 
+// ---- bf16 activations as exact integer limbs ----------------------------------------------------
+// A group of bf16 activations with absmax < 2^E (E from frexp of the absmax; E = 0 for an all-zero
+// group) becomes X = rint(x * 2^(kLimbFrac - E)), |X| <= 2^30, split into four int8 limbs
+//   X = L3 * 2^24 + L2 * 2^16 + L1 * 2^8 + L0,   L0..L2 in [-128, 127], |L3| <= 64.
+// Every tensor-core product with a limb is exact and every sum is an exact integer, so the only
+// rounding of the bf16 paths is this encoding (|x - X * 2^(E - 30)| <= 2^(E - 31), zero for every x
+// with |x| >= 2^(E - 23)) and the final conversion to fp32. Per output the encoding error is at
+// most scale * K * 2^(E - 31) <= scale * K * 2^-30 * sum_k |x_k|, i.e. within 1e-4 * scale *
+// sum_k |x_k| for every K up to 107,000, whatever the inputs' dynamic range.
+constexpr int kLimbFrac = 30;
+// 2^s for -126 <= s <= 127, from the exponent field (exact).
+__device__ __forceinline__ float exp2f_i(int s) { return __int_as_float((s + 127) << 23); }
+// x * 2^(kLimbFrac - E) rounded half to even: one or two exact power-of-two multiplies (the
+// factor exceeds fp32's range only for E < -96, i.e. groups whose absmax is below 2^-97).
+__device__ __forceinline__ int limb_fixed(float x, int E) {
+  const int s = kLimbFrac - E;
+  const float v = s <= 126 ? __fmul_rn(x, exp2f_i(s)) : __fmul_rn(__fmul_rn(x, exp2f_i(64)), exp2f_i(s - 64));
+  return __float2int_rn(v);
+}
+// The group exponent E of an absmax a >= 0: a < 2^E, and 2^(E-1) <= a when a > 0.
+__device__ __forceinline__ int limb_exponent(float a) {
+  int E = 0;
+  if (a > 0.0f) frexpf(a, &E);
+  return E;
+}
+// Four limbs of X (top limb first) as bytes of the same position in four registers.
+__device__ __forceinline__ void limbs_of(int X, int (&L)[4]) {
+  L[3] = (int)(int8_t)(X & 0xFF);
+  X = (X - L[3]) >> 8;
+  L[2] = (int)(int8_t)(X & 0xFF);
+  X = (X - L[2]) >> 8;
+  L[1] = (int)(int8_t)(X & 0xFF);
+  L[0] = (X - L[1]) >> 8;                 // |L[0]| <= 64
+}
+// Exact recombination of the four limb sums S[0] (top) .. S[3]: fits int64 for K < 2^24.
+__device__ __forceinline__ long long limb_combine(long long s3, long long s2, long long s1, long long s0) {
+  return s3 * 16777216LL + s2 * 65536LL + s1 * 256LL + s0;
+}
+
 // Monotone 32-bit key of a float (larger float -> larger key; -0 and +0 give the same key).
 __device__ __forceinline__ uint32_t float_order_key(float f) {
   uint32_t u = __float_as_uint(f);

@@ -7,24 +7,26 @@
 // 이유", displayed equation), with ternary weights decoded inside the kernel (aiatolah.com,
 // "Neutrino-1 8B: modelo ternario ...", second paragraph). At decode batch sizes this is bound by
 // the bytes of weights streamed per token (same review, section "뉴트리노 엔진": tok/s_max =
-// memory bandwidth / bytes per token), so the kernel is built to stream the 2-bit planes at HBM
-// speed and to spend well under one instruction per trit on the decode:
+// memory bandwidth / bytes per token), so the kernel streams the 2-bit planes and spends well under
+// one instruction per trit on the decode:
 //   * each lane streams 128-bit words of both planes of two rows straight into registers, with
 //     the next 512-trit chunk in flight while the current one is decoded;
 //   * one LOP3 pair + rotate merges a mask/sign word pair into 2-bit fields, and one shift + AND
-//     per register turns them into tensor-core operands holding 64*t (int8) or 2.0*t (bf16)
-//     (see tern_device.cuh); the warp's 16 rows x 32 trits go through mma.sync, where the +-1
-//     products are exact (the add / skip / subtract rule, origotech.dev Figure I);
-//   * the activation slice of the CTA is staged once in shared memory (swizzled, conflict-free);
-//     for M > 1 every decoded weight register is reused for all M activation rows (n-groups);
+//     per register turns them into int8 tensor-core operands holding 64*t (see tern_device.cuh);
+//     the warp's 16 rows x 32 trits go through mma.sync s8 x s8, where the +-1 products are exact
+//     (the add / skip / subtract rule, origotech.dev Figure I);
+//   * the activation slice of the CTA is staged once in shared memory as int8 operand columns:
+//     q itself (int8 mode), or four exact int8 limbs per token of a 30-bit fixed-point value
+//     relative to 2^E, E from the absmax of the token's slice (bf16 mode; tern_device.cuh gives
+//     the error bound); every decoded weight register is reused for all columns (n-groups);
 //   * CTAs of one row block that split K form a thread-block cluster and add their partial sums
 //     through distributed shared memory in rank order: no global scratch, deterministic results.
-// int8 mode accumulates exactly in int32 (64 * sum t*q); bf16 mode accumulates 2 * sum t*x in
-// fp32 on the tensor cores.
+// All sums are exact integers: int8 mode ends with y = ((float)acc * s_x) * scale (two fp32
+// round-to-nearest multiplies), bf16 mode combines limbs and K slices in fp64 and rounds once.
+#include <atomic>
 #include <cooperative_groups.h>
 #include <cstdint>
 #include <cuda_runtime.h>
-#include <type_traits>
 
 #include "tern_device.cuh"
 #include "tern_kernels.h"
@@ -40,9 +42,18 @@ __device__ __forceinline__ uint32_t u4get(const uint4& v, int e) {
   return e == 0 ? v.x : (e == 1 ? v.y : (e == 2 ? v.z : v.w));
 }
 
+// Operand columns of the staged slice: q of each token (int8 mode) or four limbs per token, top
+// limb first (bf16 mode: column 4m + l).
+__host__ __device__ inline int gemm_cols(int mode, int M) { return mode == 0 ? 4 * M : M; }
+// Words per staged operand column: the slice's bytes plus 16 words of bank skew.
+__host__ __device__ inline int gemm_col_words(int kr) { return kr / 4 + 16; }
+// Word offset of 16-byte half v of a column (swizzled so that the quad's loads hit distinct banks).
+__device__ __forceinline__ int gemm_half_ofs(int v) { return 4 * (v ^ ((v >> 3) & 3)); }
+
 template <int MODE, int NG>
 __global__ void __launch_bounds__(kThreads) k_tern_gemm(const GemmParams p) {
   extern __shared__ __align__(16) uint32_t smem[];
+  __shared__ int expo[16];                         // bf16 mode: limb exponent of each token's slice
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int ks = blockIdx.x;                       // K slice = cluster rank
   const int k0 = ks * p.kr;
@@ -54,6 +65,8 @@ __global__ void __launch_bounds__(kThreads) k_tern_gemm(const GemmParams p) {
   const int ra = min(row0 + g, p.N - 1), rb = min(row0 + g + 8, p.N - 1);
   const uint32_t* pa = p.planes + (size_t)ra * (2 * KM) + (k0 >> 5);
   const uint32_t* pb = p.planes + (size_t)rb * (2 * KM) + (k0 >> 5);
+  const int ncols = gemm_cols(MODE, p.M);
+  const int RS = gemm_col_words(p.kr);
 
   // weight chunk c: words [16c + 4t, 16c + 4t + 4) of both planes of rows ra, rb
   auto load_chunk = [&](int c, uint4 (&w)[4]) {
@@ -73,31 +86,57 @@ __global__ void __launch_bounds__(kThreads) k_tern_gemm(const GemmParams p) {
   load_chunk(1, nxt);
   pdl_wait();
 
-  // ---- stage the activation slice X[:, k0 : k0 + kr) in shared memory --------------------------
-  const int RS = (MODE == 0 ? p.kr / 2 : p.kr / 4) + 16;   // words per activation row (+16: banks)
-  if (MODE == 0) {
-    const int per_row = p.kr >> 3;                          // 16-byte chunks of 8 bf16
-    const uint16_t* xs = static_cast<const uint16_t*>(p.x);
-    for (int i = threadIdx.x; i < p.M * per_row; i += kThreads) {
-      const int m = i / per_row, v = i - m * per_row;
-      const uint4 val = ld_nc(xs + (size_t)m * p.K + k0 + 8 * v);
-      *reinterpret_cast<uint4*>(smem + m * RS + 4 * (v ^ ((v >> 4) & 3))) = val;
-    }
-  } else {
-    const int per_row = p.kr >> 4;                          // 16-byte halves of 32-trit blocks
+  // ---- stage the activation slice X[:, k0 : k0 + kr) as int8 operand columns ---------------------
+  const int per_row = p.kr >> 4;                            // 16-element halves of 32-trit blocks
+  if (MODE == 1) {
     const int8_t* xs = static_cast<const int8_t*>(p.x);
     for (int i = threadIdx.x; i < p.M * per_row; i += kThreads) {
       const int m = i / per_row, v = i - m * per_row;
       const uint4 val = permute_i8_half(ld_nc(xs + (size_t)m * p.K + k0 + 16 * v));
-      *reinterpret_cast<uint4*>(smem + m * RS + 4 * (v ^ ((v >> 3) & 3))) = val;
+      *reinterpret_cast<uint4*>(smem + m * RS + gemm_half_ofs(v)) = val;
+    }
+  } else {
+    const uint16_t* xs = static_cast<const uint16_t*>(p.x);
+    for (int m = warp; m < p.M; m += kThreads / 32) {
+      float amax = 0.0f;
+      for (int k = lane * 8; k < p.kr; k += 256) {
+        const uint4 v = ld_nc(xs + (size_t)m * p.K + k0 + k);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          amax = fmaxf(amax, fmaxf(fabsf(bf16_bits_to_float(w[e] & 0xFFFFu)), fabsf(bf16_bits_to_float(w[e] >> 16))));
+      }
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+      if (lane == 0) expo[m] = limb_exponent(amax);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < p.M * per_row; i += kThreads) {
+      const int m = i / per_row, v = i - m * per_row;
+      const int E = expo[m];
+      const uint16_t* xb = xs + (size_t)m * p.K + k0 + 16 * v;
+      const uint4 a = ld_nc(xb), b = ld_nc(xb + 8);
+      const uint32_t wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      uint32_t l[4][4] = {};
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const uint32_t bits = (e & 1) ? (wv[e >> 1] >> 16) : (wv[e >> 1] & 0xFFFFu);
+        int L[4];
+        limbs_of(limb_fixed(bf16_bits_to_float(bits), E), L);
+        const int sh = 8 * (e & 3);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) l[c][e >> 2] |= (uint32_t)(uint8_t)L[c] << sh;
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        *reinterpret_cast<uint4*>(smem + (4 * m + c) * RS + gemm_half_ofs(v)) =
+            permute_i8_half(make_uint4(l[c][0], l[c][1], l[c][2], l[c][3]));
     }
   }
   __syncthreads();
 
-  using Acc = typename std::conditional<MODE == 0, float, int>::type;
-  Acc acc[NG][4];
+  int acc[NG][4];
 #pragma unroll
-  for (int n = 0; n < NG; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = Acc(0);
+  for (int n = 0; n < NG; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0;
 
   for (int c = 0; c < nchunks; ++c) {
     const bool live = (16 * c + 4 * t) < nw;
@@ -107,57 +146,28 @@ __global__ void __launch_bounds__(kThreads) k_tern_gemm(const GemmParams p) {
       uint32_t wa0, wb0, wa1, wb1;
       merge_planes(u4get(cur[0], e), u4get(cur[2], e), wa0, wb0);   // row ra
       merge_planes(u4get(cur[1], e), u4get(cur[3], e), wa1, wb1);   // row rb
-      if constexpr (MODE == 0) {
-        uint32_t xb[NG][16];
+      // the word's operand registers of both rows: 64 * t per byte
+      const uint32_t A[8][2] = {
+          {dec_i8<0>(wa0, wb0), dec_i8<0>(wa1, wb1)}, {dec_i8<1>(wa0, wb0), dec_i8<1>(wa1, wb1)},
+          {dec_i8<2>(wa0, wb0), dec_i8<2>(wa1, wb1)}, {dec_i8<3>(wa0, wb0), dec_i8<3>(wa1, wb1)},
+          {dec_i8<4>(wa0, wb0), dec_i8<4>(wa1, wb1)}, {dec_i8<5>(wa0, wb0), dec_i8<5>(wa1, wb1)},
+          {dec_i8<6>(wa0, wb0), dec_i8<6>(wa1, wb1)}, {dec_i8<7>(wa0, wb0), dec_i8<7>(wa1, wb1)}};
 #pragma unroll
-        for (int n = 0; n < NG; ++n) {
-          const int m = 8 * n + g;
-          if (live && m < p.M) {
+      for (int n = 0; n < NG; ++n) {
+        const int col = 8 * n + g;
+        uint32_t xb[8];
+        if (live && col < ncols) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int ch = 4 * w + q;
-              const uint4 v = *reinterpret_cast<const uint4*>(smem + m * RS + 4 * (ch ^ ((ch >> 4) & 3)));
-              xb[n][4 * q] = v.x; xb[n][4 * q + 1] = v.y; xb[n][4 * q + 2] = v.z; xb[n][4 * q + 3] = v.w;
-            }
-          } else {
-#pragma unroll
-            for (int q = 0; q < 16; ++q) xb[n][q] = 0u;
+          for (int q = 0; q < 2; ++q) {
+            const uint4 v = *reinterpret_cast<const uint4*>(smem + col * RS + gemm_half_ofs(2 * w + q));
+            xb[4 * q] = v.x; xb[4 * q + 1] = v.y; xb[4 * q + 2] = v.z; xb[4 * q + 3] = v.w;
           }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) xb[q] = 0u;
         }
-#define TERN_BF16_STEP(A0, A1)                                                                    \
-  {                                                                                              \
-    const uint32_t a0 = dec_bf16<A0>(wa0, wb0), a1 = dec_bf16<A0>(wa1, wb1);                     \
-    const uint32_t a2 = dec_bf16<A1>(wa0, wb0), a3 = dec_bf16<A1>(wa1, wb1);                     \
-    _Pragma("unroll") for (int n = 0; n < NG; ++n) mma_bf16(acc[n], a0, a1, a2, a3, xb[n][A0], xb[n][A1]); \
-  }
-        TERN_BF16_STEP(0, 1) TERN_BF16_STEP(2, 3) TERN_BF16_STEP(4, 5) TERN_BF16_STEP(6, 7)
-        TERN_BF16_STEP(8, 9) TERN_BF16_STEP(10, 11) TERN_BF16_STEP(12, 13) TERN_BF16_STEP(14, 15)
-#undef TERN_BF16_STEP
-      } else {
-        uint32_t xb[NG][8];
 #pragma unroll
-        for (int n = 0; n < NG; ++n) {
-          const int m = 8 * n + g;
-          if (live && m < p.M) {
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              const int ch = 2 * w + q;
-              const uint4 v = *reinterpret_cast<const uint4*>(smem + m * RS + 4 * (ch ^ ((ch >> 3) & 3)));
-              xb[n][4 * q] = v.x; xb[n][4 * q + 1] = v.y; xb[n][4 * q + 2] = v.z; xb[n][4 * q + 3] = v.w;
-            }
-          } else {
-#pragma unroll
-            for (int q = 0; q < 8; ++q) xb[n][q] = 0u;
-          }
-        }
-#define TERN_I8_STEP(R0, R1)                                                                      \
-  {                                                                                              \
-    const uint32_t a0 = dec_i8<R0>(wa0, wb0), a1 = dec_i8<R0>(wa1, wb1);                         \
-    const uint32_t a2 = dec_i8<R1>(wa0, wb0), a3 = dec_i8<R1>(wa1, wb1);                         \
-    _Pragma("unroll") for (int n = 0; n < NG; ++n) mma_s8(acc[n], a0, a1, a2, a3, xb[n][R0], xb[n][R1]); \
-  }
-        TERN_I8_STEP(0, 1) TERN_I8_STEP(2, 3) TERN_I8_STEP(4, 5) TERN_I8_STEP(6, 7)
-#undef TERN_I8_STEP
+        for (int r = 0; r < 8; r += 2) mma_s8(acc[n], A[r][0], A[r][1], A[r + 1][0], A[r + 1][1], xb[r], xb[r + 1]);
       }
     }
 #pragma unroll
@@ -166,67 +176,65 @@ __global__ void __launch_bounds__(kThreads) k_tern_gemm(const GemmParams p) {
   }
   pdl_launch_dependents();
 
-  // ---- epilogue ----------------------------------------------------------------------------------
-  // int8: y = ((float)(acc / 64) * s_x) * scale, two fp32 round-to-nearest multiplies.
-  // bf16: y = (acc * 0.5) * scale.
-  auto finish = [&](Acc v, int m, int row) -> float {
-    const float sc = f16_bits_to_float(p.scale[row]);
-    if constexpr (MODE == 0) {
-      return __fmul_rn(__fmul_rn(v, 0.5f), sc);
-    } else {
-      return __fmul_rn(__fmul_rn(__int2float_rn(v >> 6), p.sx[m]), sc);
-    }
-  };
-  if (p.ksplit == 1) {
+  // ---- epilogue: exact sums (acc = 64 * sum), one rounding ----------------------------------------
+  if (MODE == 1 && p.ksplit == 1) {
 #pragma unroll
     for (int n = 0; n < NG; ++n)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int m = 8 * n + 2 * t + (i & 1);
         const int row = row0 + g + 8 * (i >> 1);
-        if (m < p.M && row < p.N) p.y[(size_t)m * p.N + row] = finish(acc[n][i], m, row);
+        if (m < p.M && row < p.N) {
+          const int sum = acc[n][i] >> 6;
+          p.y[(size_t)m * p.N + row] = __fmul_rn(__fmul_rn(__int2float_rn(sum), p.sx[m]), f16_bits_to_float(p.scale[row]));
+          if (p.acc) p.acc[(size_t)m * p.N + row] = sum;
+        }
       }
     return;
   }
-  // Split K: partial tile [kRows][8*NG] in this CTA's shared memory, then a cluster-wide sum.
+  // partial tile [kRows][8 * NG] in this CTA's shared memory, then (split K) a cluster-wide sum
   constexpr int kCols = 8 * NG;
-  Acc* part = reinterpret_cast<Acc*>(smem + p.M * RS);
+  int* part = reinterpret_cast<int*>(smem + ncols * RS);
 #pragma unroll
   for (int n = 0; n < NG; ++n)
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int col = 8 * n + 2 * t + (i & 1);
       const int lrow = warp * 16 + g + 8 * (i >> 1);
-      part[lrow * kCols + col] = acc[n][i];
+      part[lrow * kCols + col] = acc[n][i] >> 6;
     }
   cg::cluster_group cluster = cg::this_cluster();
-  cluster.sync();
+  if (p.ksplit > 1) cluster.sync(); else __syncthreads();
   const int rows_per_rank = kRows / p.ksplit;
-  for (int i = threadIdx.x; i < rows_per_rank * kCols; i += kThreads) {
-    const int lrow = ks * rows_per_rank + i / kCols, col = i % kCols;
+  for (int i = threadIdx.x; i < rows_per_rank * p.M; i += kThreads) {
+    const int lrow = ks * rows_per_rank + i / p.M, m = i % p.M;
     const int row = blockIdx.y * kRows + lrow;
-    if (col >= p.M || row >= p.N) continue;
-    Acc sum = Acc(0);
-    for (int r = 0; r < p.ksplit; ++r) {
-      const Acc* rp = cluster.map_shared_rank(part, r);
-      sum += rp[lrow * kCols + col];
+    if (row >= p.N) continue;
+    const float sc = f16_bits_to_float(p.scale[row]);
+    if (MODE == 1) {
+      int sum = 0;
+      for (int r = 0; r < p.ksplit; ++r) sum += cluster.map_shared_rank(part, r)[lrow * kCols + m];
+      p.y[(size_t)m * p.N + row] = __fmul_rn(__fmul_rn(__int2float_rn(sum), p.sx[m]), sc);
+      if (p.acc) p.acc[(size_t)m * p.N + row] = sum;
+    } else {
+      double tot = 0.0;
+      for (int r = 0; r < p.ksplit; ++r) {
+        const int* rp = (p.ksplit > 1 ? cluster.map_shared_rank(part, r) : part) + lrow * kCols + 4 * m;
+        const int E = (p.ksplit > 1 ? cluster.map_shared_rank(expo, r) : expo)[m];
+        tot += ldexp((double)limb_combine(rp[0], rp[1], rp[2], rp[3]), E - kLimbFrac);
+      }
+      p.y[(size_t)m * p.N + row] = (float)(tot * (double)sc);
     }
-    p.y[(size_t)col * p.N + row] = finish(sum, col, row);
   }
-  cluster.sync();
+  if (p.ksplit > 1) cluster.sync();
 }
 
 template <int MODE, int NG>
 cudaError_t launch_one(const GemmParams& p, size_t smem, bool pdl, cudaStream_t st) {
   auto kern = k_tern_gemm<MODE, NG>;
-  // Raise the kernel's dynamic shared-memory limit once per size increase (not on every launch).
-  static int smem_set = 0;
-  cudaError_t e = cudaSuccess;
-  if ((int)smem > smem_set) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    smem_set = (int)smem;
-  }
+  static std::atomic<unsigned long long> smem_raised{0};
+  cudaError_t e = allow_max_dynamic_smem(kern, smem_raised);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.ksplit, (p.N + kRows - 1) / kRows, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -251,23 +259,35 @@ cudaError_t launch_one(const GemmParams& p, size_t smem, bool pdl, cudaStream_t 
   return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
+template <int MODE>
+cudaError_t launch_mode(const GemmParams& p, int ng, size_t smem, bool pdl, cudaStream_t st) {
+  switch (ng) {
+    case 1: return launch_one<MODE, 1>(p, smem, pdl, st);
+    case 2: return launch_one<MODE, 2>(p, smem, pdl, st);
+    case 3: return launch_one<MODE, 3>(p, smem, pdl, st);
+    case 4: return launch_one<MODE, 4>(p, smem, pdl, st);
+    case 5: return launch_one<MODE, 5>(p, smem, pdl, st);
+    case 6: return launch_one<MODE, 6>(p, smem, pdl, st);
+    case 7: return launch_one<MODE, 7>(p, smem, pdl, st);
+    default: return launch_one<MODE, 8>(p, smem, pdl, st);
+  }
+}
+
 }  // namespace
 
-// Shared-memory bytes of one CTA: activation slice (+ padding) and the split-K partial tile.
+// Shared-memory bytes of one CTA: the operand columns of the activation slice and the partial tile.
 size_t gemm_smem_bytes(int mode, int M, int kr) {
-  const int RS = (mode == 0 ? kr / 2 : kr / 4) + 16;
-  const int ng = (M + 7) / 8;
-  return (size_t)M * RS * 4 + (size_t)kRows * 8 * ng * 4;
+  const int ncols = gemm_cols(mode, M);
+  const int ng = (ncols + 7) / 8;
+  return (size_t)ncols * gemm_col_words(kr) * 4 + (size_t)kRows * 8 * ng * 4;
 }
 
 int gemm_rows_per_cta() { return kRows; }
 
 cudaError_t launch_tern_gemm(const GemmParams& p, bool pdl, cudaStream_t st) {
-  const int mode = p.mode;
-  const int ng = (p.M + 7) / 8;
-  const size_t smem = gemm_smem_bytes(mode, p.M, p.kr);
-  if (mode == 0) return ng == 1 ? launch_one<0, 1>(p, smem, pdl, st) : launch_one<0, 2>(p, smem, pdl, st);
-  return ng == 1 ? launch_one<1, 1>(p, smem, pdl, st) : launch_one<1, 2>(p, smem, pdl, st);
+  const int ng = (gemm_cols(p.mode, p.M) + 7) / 8;
+  const size_t smem = gemm_smem_bytes(p.mode, p.M, p.kr);
+  return p.mode == 0 ? launch_mode<0>(p, ng, smem, pdl, st) : launch_mode<1>(p, ng, smem, pdl, st);
 }
 
 }  // namespace tern

@@ -10,11 +10,11 @@
 //
 // Design: int8 W rows feed mma.sync directly as the A operand (no decode at all); the activation
 // is the B operand. int8 mode uses q from the per-token quantiser and is bit-exact. bf16 mode
-// splits each bf16 x exactly into three int8 limbs of a 22-bit fixed-point value relative to
-// 2^E, E from the absmax of this CTA's K slice (exact for every x within 2^-15 of that absmax,
-// rounding below it), so the products and the int32 sums stay exact; limbs and K slices are
-// combined in fp64 before the single rounding to fp32. Limbs (and the M rows) occupy the eight
-// columns of each tensor-core n-group, which for M = 1 come for free. CTAs splitting K form a
+// turns each bf16 x into four int8 limbs of a 30-bit fixed-point value relative to 2^E, E from the
+// absmax of this CTA's K slice (exact for every x within 2^-23 of that absmax, rounding by at most
+// 2^(E - 31) below it; see tern_device.cuh), so the products and the int32 sums stay exact; limbs
+// and K slices are combined in fp64 before the single rounding to fp32. Limbs (and the M rows)
+// occupy the eight columns of each tensor-core n-group, which for M = 1 come for free. CTAs splitting K form a
 // cluster and add partial sums through distributed shared memory. The running maximum per row is
 // kept as a packed (order-preserving value key, inverted index) 64-bit word, reduced with
 // shared-memory and then global atomicMax; the last CTA to finish publishes the result and
@@ -32,7 +32,6 @@ namespace tern {
 namespace {
 
 constexpr int kHeadRows = 128;   // rows per row block: 8 warps x 16 rows
-constexpr int kLimbFrac = 22;    // bf16 mode: x ~= X * 2^(E - 22), |X| < 2^22
 
 template <int MODE, int NG>
 __global__ void __launch_bounds__(kThreads, 2) k_head(const HeadParams p) {
@@ -43,7 +42,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_head(const HeadParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int ks = blockIdx.x;
   const int k0 = ks * p.kr;
-  const int ncols = MODE == 0 ? 3 * p.M : p.M;
+  const int ncols = MODE == 0 ? 4 * p.M : p.M;
   const int RS = p.kr / 4 + 4;             // words per staged activation column (+4: banks)
   const int nch = p.kr / 128;              // 128-byte chunks per row in this slice
   if (threadIdx.x < 16) best[threadIdx.x] = 0ull;
@@ -98,37 +97,27 @@ __global__ void __launch_bounds__(kThreads, 2) k_head(const HeadParams p) {
           amax = fmaxf(amax, fmaxf(fabsf(bf16_bits_to_float(w[e] & 0xFFFFu)), fabsf(bf16_bits_to_float(w[e] >> 16))));
       }
       for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-      int E = 0;
-      if (amax > 0.0f) {
-        frexpf(amax, &E);                  // amax < 2^E
-        E = max(E, -100);
-      }
-      if (lane == 0) expo[m] = E;
+      if (lane == 0) expo[m] = limb_exponent(amax);
     }
     __syncthreads();
     const int per_row = p.kr / 8;
     for (int i = threadIdx.x; i < p.M * per_row; i += kThreads) {
       const int m = i / per_row, v = i - m * per_row;
-      const float f = ldexpf(1.0f, kLimbFrac - expo[m]);
+      const int E = expo[m];
       const uint4 val = ld_nc(xb + (size_t)m * p.K + k0 + 8 * v);
       const uint32_t w[4] = {val.x, val.y, val.z, val.w};
-      uint32_t l2[2] = {0u, 0u}, l1[2] = {0u, 0u}, l0[2] = {0u, 0u};
+      uint32_t l[4][2] = {};
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const uint32_t bits = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
-        const int X = __float2int_rn(bf16_bits_to_float(bits) * f);   // exact power-of-two scaling
-        const int L0 = (int)(int8_t)(X & 0xFF);
-        const int X1 = (X - L0) >> 8;
-        const int L1 = (int)(int8_t)(X1 & 0xFF);
-        const int L2 = (X1 - L1) >> 8;                                 // |L2| <= 64
+        int L[4];
+        limbs_of(limb_fixed(bf16_bits_to_float(bits), E), L);
         const int sh = 8 * (e & 3);
-        l0[e >> 2] |= (uint32_t)(uint8_t)L0 << sh;
-        l1[e >> 2] |= (uint32_t)(uint8_t)L1 << sh;
-        l2[e >> 2] |= (uint32_t)(uint8_t)L2 << sh;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) l[c][e >> 2] |= (uint32_t)(uint8_t)L[c] << sh;
       }
-      *reinterpret_cast<uint2*>(smem + (3 * m) * RS + 2 * v) = make_uint2(l2[0], l2[1]);
-      *reinterpret_cast<uint2*>(smem + (3 * m + 1) * RS + 2 * v) = make_uint2(l1[0], l1[1]);
-      *reinterpret_cast<uint2*>(smem + (3 * m + 2) * RS + 2 * v) = make_uint2(l0[0], l0[1]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) *reinterpret_cast<uint2*>(smem + (4 * m + c) * RS + 2 * v) = make_uint2(l[c][0], l[c][1]);
     }
   }
   __syncthreads();
@@ -197,9 +186,9 @@ __global__ void __launch_bounds__(kThreads, 2) k_head(const HeadParams p) {
       } else {
         double tot = 0.0;
         for (int r = 0; r < p.ksplit; ++r) {
-          const int* rp = (p.ksplit > 1 ? cluster.map_shared_rank(part, r) : part) + lrow * kCols + 3 * m;
+          const int* rp = (p.ksplit > 1 ? cluster.map_shared_rank(part, r) : part) + lrow * kCols + 4 * m;
           const int E = (p.ksplit > 1 ? cluster.map_shared_rank(expo, r) : expo)[m];
-          const long long D = (long long)rp[0] * 65536 + (long long)rp[1] * 256 + rp[2];
+          const long long D = limb_combine(rp[0], rp[1], rp[2], rp[3]);
           tot += ldexp((double)D, E - kLimbFrac);
         }
         logit = (float)(tot * (double)shv);
@@ -236,14 +225,9 @@ __global__ void __launch_bounds__(kThreads, 2) k_head(const HeadParams p) {
 template <int MODE, int NG>
 cudaError_t launch_ng(const HeadParams& p, size_t smem, bool pdl, cudaStream_t st) {
   auto kern = k_head<MODE, NG>;
-  // Raise the kernel's dynamic shared-memory limit once per size increase (not on every launch).
-  static int smem_set = 0;
-  cudaError_t e = cudaSuccess;
-  if ((int)smem > smem_set) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    smem_set = (int)smem;
-  }
+  static std::atomic<unsigned long long> smem_raised{0};
+  cudaError_t e = allow_max_dynamic_smem(kern, smem_raised);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.ksplit, p.nby, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -276,7 +260,9 @@ cudaError_t launch_mode(const HeadParams& p, int ng, size_t smem, bool pdl, cuda
     case 3: return launch_ng<MODE, 3>(p, smem, pdl, st);
     case 4: return launch_ng<MODE, 4>(p, smem, pdl, st);
     case 5: return launch_ng<MODE, 5>(p, smem, pdl, st);
-    default: return launch_ng<MODE, 6>(p, smem, pdl, st);
+    case 6: return launch_ng<MODE, 6>(p, smem, pdl, st);
+    case 7: return launch_ng<MODE, 7>(p, smem, pdl, st);
+    default: return launch_ng<MODE, 8>(p, smem, pdl, st);
   }
 }
 
@@ -285,13 +271,13 @@ cudaError_t launch_mode(const HeadParams& p, int ng, size_t smem, bool pdl, cuda
 size_t head_workspace_bytes(int M) { return 16 + 8 * (size_t)M; }
 
 size_t head_smem_bytes(int mode, int M, int kr) {
-  const int ncols = mode == 0 ? 3 * M : M;
+  const int ncols = mode == 0 ? 4 * M : M;
   const int ng = (ncols + 7) / 8;
   return (size_t)ncols * (kr / 4 + 4) * 4 + (size_t)kHeadRows * 8 * ng * 4;
 }
 
 cudaError_t launch_head(const HeadParams& p, bool pdl, cudaStream_t st) {
-  const int ncols = p.mode == 0 ? 3 * p.M : p.M;
+  const int ncols = p.mode == 0 ? 4 * p.M : p.M;
   const int ng = (ncols + 7) / 8;
   const size_t smem = head_smem_bytes(p.mode, p.M, p.kr);
   return p.mode == 0 ? launch_mode<0>(p, ng, smem, pdl, st) : launch_mode<1>(p, ng, smem, pdl, st);

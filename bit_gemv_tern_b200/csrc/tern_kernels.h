@@ -1,12 +1,58 @@
 // Internal launch interface between the C ABI (tern_abi.cu) and the kernel files.
 #pragma once
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "../../include/tern.h"
+
 namespace tern {
+
+// Persistent kernels launch at most one CTA per SM and at most kMaxGridCTAs of them (the batch
+// plan keeps one split record per CTA in the kernel parameters); 148 = the SMs of a B200.
+constexpr int kMaxGridCTAs = 148;
+
+// SMs of the current device (148 on a B200; 148 if the query fails, which the launch then reports).
+inline int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      n <= 0)
+    return kMaxGridCTAs;
+  return n;
+}
+
+// CTAs of a persistent launch over `work` units: one per SM, at most kMaxGridCTAs and `work`.
+inline int persistent_grid(long long work) {
+  long long g = device_sm_count();
+  if (g > kMaxGridCTAs) g = kMaxGridCTAs;
+  if (work < g) g = work;
+  return g < 1 ? 1 : (int)g;
+}
+
+// Allow a kernel the device's whole opt-in dynamic shared memory (less its static shared memory).
+// The attribute belongs to one device, so each device is set up on its first launch there; `done`
+// holds one bit per device index below 64 (devices past that are set up on every launch). Two host
+// threads that race here both set the same value.
+template <typename F>
+cudaError_t allow_max_dynamic_smem(F* kern, std::atomic<unsigned long long>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = (dev >= 0 && dev < 64) ? 1ull << dev : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  int optin = 0;
+  e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return e;
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin - (int)fa.sharedSizeBytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 // Ternary GEMV / small-M GEMM (tern_gemv.cu).
 struct GemmParams {
@@ -16,6 +62,7 @@ struct GemmParams {
   const void* x;          // bf16 bits [M][K] (mode 0) or int8 [M][K] (mode 1)
   const float* sx;        // [M], int8 mode only
   float* y;               // [M][N]
+  int32_t* acc;           // int8 mode, optional: the exact sums sum_k t*q, [M][N]
   int32_t M;              // 1..16
   int32_t mode;           // 0 = bf16 activations, 1 = int8 activations
   int32_t kr;             // trits of K per CTA (multiple of 128); ksplit * kr == K
@@ -33,6 +80,7 @@ struct StreamParams {
   const void* x;          // bf16 bits [K] (mode 0) or int8 [K] (mode 1)
   const float* sx;        // [1], int8 mode only
   float* y;               // [N]
+  int32_t* acc;           // int8 mode, optional: the exact sums sum_k t*q, [N]
   int32_t mode;
   int32_t ks;             // trits of K per stage (divides K)
   int32_t ts;             // tiles of 16 rows per stage (1, 2, 4 or 8)
@@ -78,12 +126,12 @@ struct BatchParams {
   int32_t stage_slot_bytes;
   int32_t seg_bytes;      // operand bytes of one 512-trit part (all columns + sums + exponent)
   uint8_t* xprep;         // workspace: operand blocks
-  int32_t cta_part[149];  // CTA c handles global parts [cta_part[c], cta_part[c + 1])
+  int32_t cta_part[kMaxGridCTAs + 1];  // CTA c handles global parts [cta_part[c], cta_part[c + 1])
   // Row blocks split between CTAs: each contributor adds exact partial sums into a workspace
   // slot; the last one (per warp, by counter) writes the outputs.
   // per CTA, 8 bits each: slot of its first block + 1, that block's contributors, slot of its
   // last block + 1, that block's contributors (slot + 1 = 0: the block is this CTA's alone)
-  uint32_t cta_split[148];
+  uint32_t cta_split[kMaxGridCTAs];
   int32_t nslots;
   uint32_t scratch_off;   // workspace byte offset: [nslots][rows][8 * groups] int32, then counters
   int32_t scratch_words;  // words to zero before the stream (sums and counters)
@@ -128,6 +176,11 @@ struct HeadParams {
 size_t head_workspace_bytes(int M);
 size_t head_smem_bytes(int mode, int M, int kr);
 cudaError_t launch_head(const HeadParams& p, bool pdl, cudaStream_t st);
+// Every argument check of i8_head_gemv_argmax_ex and its launch plan (tern_abi.cu); enqueues nothing.
+tern_status plan_head_call(const int8_t* W_dev, const uint16_t* scale_f16_dev, int32_t V, int32_t K, int32_t M,
+                           tern_act act, const void* X_dev, const float* x_scale_dev, int32_t* argmax_dev,
+                           float* maxval_dev, float* logits_dev, void* workspace_dev, size_t workspace_bytes,
+                           uint32_t flags, HeadParams& p);
 
 // Loader kernels (tern_pack.cu).
 constexpr int kPackMaxItems = 256;

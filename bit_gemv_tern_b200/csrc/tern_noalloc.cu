@@ -4,15 +4,17 @@
 // maximum per activation row) from the caller. This entry point uses one library-internal device
 // array instead, so a caller needs no device buffer beyond the inputs and outputs. The array is
 // file-scope and sized for the largest M the head accepts (16 activation rows). Its address is
-// looked up once per device with cudaGetSymbolAddress, with that device current; each call clears
-// the bytes it uses with cudaMemsetAsync on its own stream and then runs exactly as
-// i8_head_gemv_argmax with that scratch. No call allocates or frees device memory. Every call on
-// a device shares the one array, so calls that overlap in time race.
+// looked up once per device with cudaGetSymbolAddress, with that device current. Each call checks
+// every argument and plans the launch first (an invalid call enqueues nothing), then clears the
+// bytes it uses with cudaMemsetAsync on its own stream and launches the head with that scratch. No
+// call allocates or frees device memory. Every call on a device shares the one array, so calls
+// that overlap in time race.
 #include <cstdint>
 #include <mutex>
 #include <cuda_runtime.h>
 
 #include "../../include/tern.h"
+#include "tern_kernels.h"
 
 namespace {
 
@@ -25,7 +27,7 @@ static __device__ __align__(256) unsigned char g_head_scratch[kScratchBytes];
 std::mutex g_mu;
 void* g_addr[kMaxDevices] = {};
 
-// Device address of g_head_scratch on the current device (set up on the first call there).
+// Device address of g_head_scratch on the current device (looked up on the first call there).
 tern_status scratch_address(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return TERN_ECUDA;
@@ -50,9 +52,13 @@ tern_status i8_head_gemv_argmax_noalloc(const int8_t* W_dev, const uint16_t* sca
   const size_t need = i8_head_workspace_bytes(V, M);
   if (need == 0 || need > kScratchBytes) return TERN_ESHAPE;
   void* ws = nullptr;
-  const tern_status st = scratch_address(&ws);
+  tern_status st = scratch_address(&ws);
   if (st != TERN_OK) return st;
-  if (cudaMemsetAsync(ws, 0, need, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return TERN_ECUDA;
-  return i8_head_gemv_argmax(W_dev, scale_f16_dev, V, K, M, act, X_dev, x_scale_dev, argmax_dev, maxval_dev,
-                             logits_dev, ws, kScratchBytes, stream);
+  tern::HeadParams p = {};
+  st = tern::plan_head_call(W_dev, scale_f16_dev, V, K, M, act, X_dev, x_scale_dev, argmax_dev, maxval_dev,
+                            logits_dev, ws, kScratchBytes, 0u, p);
+  if (st != TERN_OK) return st;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, need, s) != cudaSuccess) return TERN_ECUDA;
+  return tern::launch_head(p, false, s) == cudaSuccess ? TERN_OK : TERN_ECUDA;
 }

@@ -372,7 +372,8 @@ __global__ void k_occupancy(const uint32_t* __restrict__ planes, int32_t N, int3
 
 int grid_for(int64_t work, int threads) {
   int64_t g = (work + threads - 1) / threads;
-  return (int)(g < 1 ? 1 : (g > 148 * 32 ? 148 * 32 : g));
+  const int64_t cap = (int64_t)device_sm_count() * 32;
+  return (int)(g < 1 ? 1 : (g > cap ? cap : g));
 }
 
 }  // namespace
@@ -381,7 +382,7 @@ cudaError_t launch_pack_trits(const int8_t* src, int32_t N, int32_t K, uint32_t*
                               cudaStream_t st) {
   const int KM = K / 32;
   const int gx = (KM + kPackThreads - 1) / kPackThreads;
-  int gy = (148 * 16 + gx - 1) / gx;                     // ~16 CTAs per SM over all columns
+  int gy = (device_sm_count() * 16 + gx - 1) / gx;       // ~16 CTAs per SM over all columns
   if (gy > N) gy = N;
   if (gy > 65535) gy = 65535;
   k_pack_trits<<<dim3(gx, gy), kPackThreads, 0, st>>>(src, N, KM, planes, flag);
@@ -400,19 +401,8 @@ int base3_grid(const void* fn, size_t smem, int nblocks) {
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kB3Threads, smem) != cudaSuccess || per_sm < 1)
     per_sm = 1;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const long long g = (long long)per_sm * sms;
+  const long long g = (long long)per_sm * device_sm_count();
   return (int)(g < nblocks ? g : (nblocks < 1 ? 1 : nblocks));
-}
-
-cudaError_t base3_smem_attr(const void* fn, size_t smem, size_t& set) {
-  if (smem > 48 * 1024 && smem > set) {
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    set = smem;
-  }
-  return cudaSuccess;
 }
 
 cudaError_t launch_unpack_base3(const uint8_t* src, int32_t N, int32_t K, uint32_t* planes, int32_t* flag,
@@ -421,8 +411,8 @@ cudaError_t launch_unpack_base3(const uint8_t* src, int32_t N, int32_t K, uint32
   size_t smem = 0;
   base3_plan(K, rows, smem);
   const int nblocks = (N + rows - 1) / rows;
-  static size_t set = 0;
-  cudaError_t e = base3_smem_attr(reinterpret_cast<const void*>(k_unpack_base3), smem, set);
+  static std::atomic<unsigned long long> smem_raised{0};
+  cudaError_t e = allow_max_dynamic_smem(k_unpack_base3, smem_raised);
   if (e != cudaSuccess) return e;
   const int grid = base3_grid(reinterpret_cast<const void*>(k_unpack_base3), smem, nblocks);
   k_unpack_base3<<<grid, kB3Threads, smem, st>>>(src, N, K / 32, (K + 4) / 5, rows, nblocks, planes, flag);
@@ -441,9 +431,7 @@ cudaError_t launch_pack_trits_batch(PackBatch& p, int32_t* flag, cudaStream_t st
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_pack_trits_batch, kPackThreads, 0) != cudaSuccess ||
       per_sm < 1)
     per_sm = 1;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t g = (int64_t)per_sm * sms;
+  const int64_t g = (int64_t)per_sm * device_sm_count();
   k_pack_trits_batch<<<(unsigned)(g < units ? g : units), kPackThreads, 0, st>>>(p, flag);
   return cudaGetLastError();
 }
@@ -461,8 +449,8 @@ cudaError_t launch_unpack_base3_batch(Base3Batch& p, int32_t* flag, cudaStream_t
     if (sm > smem) smem = sm;
   }
   if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
-  static size_t set = 0;
-  cudaError_t e = base3_smem_attr(reinterpret_cast<const void*>(k_unpack_base3_batch), smem, set);
+  static std::atomic<unsigned long long> smem_raised{0};
+  cudaError_t e = allow_max_dynamic_smem(k_unpack_base3_batch, smem_raised);
   if (e != cudaSuccess) return e;
   const int grid = base3_grid(reinterpret_cast<const void*>(k_unpack_base3_batch), smem, (int)blocks);
   k_unpack_base3_batch<<<grid, kB3Threads, smem, st>>>(p, (int32_t)blocks, flag);

@@ -415,7 +415,8 @@ bool plan_prefill(PrefillParams& p, const uint16_t* X, int& grid, size_t& smem) 
   // two 128-token halves per tile while such tiles still give every SM one (they halve the weight
   // expansion per flop); 128-token tiles otherwise
   const int tiles_n = (p.N + BN - 1) / BN;
-  p.halves = (long long)((p.M + 2 * BM - 1) / (2 * BM)) * tiles_n >= 148 ? 2 : 1;
+  const int sms = device_sm_count();
+  p.halves = (long long)((p.M + 2 * BM - 1) / (2 * BM)) * tiles_n >= sms ? 2 : 1;
   const int tile_m = BM * p.halves;
   const cuuint64_t dims[2] = {(cuuint64_t)p.K, (cuuint64_t)p.M};
   const cuuint64_t strides[1] = {(cuuint64_t)p.K * 2};
@@ -426,19 +427,16 @@ bool plan_prefill(PrefillParams& p, const uint16_t* X, int& grid, size_t& smem) 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return false;
   const long long tiles = (long long)((p.M + tile_m - 1) / tile_m) * tiles_n;
-  grid = tiles < 148 ? (int)tiles : 148;
+  grid = tiles < sms ? (int)tiles : sms;
   smem = p.halves == 2 ? Shape<2>::kSmemBytes : Shape<1>::kSmemBytes;
   return true;
 }
 
 template <int H>
 cudaError_t launch_prefill_h(const PrefillParams& p, int grid, size_t smem, cudaStream_t st) {
-  static int set = 0;
-  if (!set) {
-    cudaError_t e = cudaFuncSetAttribute(k_prefill<H>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    set = 1;
-  }
+  static std::atomic<unsigned long long> smem_raised{0};
+  cudaError_t e = allow_max_dynamic_smem(k_prefill<H>, smem_raised);
+  if (e != cudaSuccess) return e;
   k_prefill<H><<<grid, kPrefillThreads, smem, st>>>(p);
   return cudaGetLastError();
 }

@@ -17,10 +17,11 @@
 //     activation, stage it once, then decode the merged 2-bit fields into u8 tensor-core operands
 //     (one AND per register, see merge_planes_offset in tern_device.cuh) and run mma.sync u8 x s8
 //     with four field accumulators;
-//   * int8 mode: x = q (per-token int8), exact int32 sums; bf16 mode: x is split exactly into three
-//     int8 limbs of a 22-bit fixed-point value relative to 2^E (E from the absmax of x), which sit
-//     in three columns of the n = 8 operand for free at M = 1, so the products and sums stay
-//     exact in int32 and only the final fp64 -> fp32 conversion rounds;
+//   * int8 mode: x = q (per-token int8), exact int32 sums; bf16 mode: x becomes four int8 limbs of
+//     a 30-bit fixed-point value relative to 2^E (E from the absmax of the warp's K part; see
+//     tern_device.cuh for the error bound), which sit in four columns of the n = 8 operand for free
+//     at M = 1, so the products and sums stay exact integers and only the encoding and the final
+//     fp64 -> fp32 conversion round;
 //   * every wait on an mbarrier is bounded; on timeout the kernel latches TERN_ETIMEOUT in a
 //     device word (read with tern_device_status), stops and returns.
 #include <cstdint>
@@ -37,7 +38,6 @@ namespace {
 
 constexpr int kConsumerWarps = 8;   // warps per consumer group
 constexpr uint32_t kWaitTries = 1u << 13;      // x ~0.5 ms suspend hint: seconds before giving up
-constexpr int kLimbFrac = 22;
 
 // ---- mbarrier / bulk-copy primitives ------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -94,7 +94,7 @@ __device__ __forceinline__ uint32_t u4get(const uint4& v, int e) {
 template <int MODE, int CW, bool XREG>
 __global__ void __launch_bounds__((CW + 1) * 32, 1) k_tern_stream(const StreamParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  constexpr int NC = MODE == 0 ? 3 : 1;                           // activation columns
+  constexpr int NC = MODE == 0 ? 4 : 1;                           // activation columns (limbs or q)
   constexpr int NGRP = CW / 8;                                    // consumer groups
   const int S = p.stages, TS = p.ts, WPT = 8 / TS;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem);          // full[S], empty[S]
@@ -189,34 +189,25 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_tern_stream(const StreamPa
         amax = fmaxf(amax, fmaxf(fabsf(bf16_bits_to_float(wv[e] & 0xFFFFu)), fabsf(bf16_bits_to_float(wv[e] >> 16))));
     }
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-    int E = 0;
-    if (amax > 0.0f) {
-      frexpf(amax, &E);                    // amax < 2^E
-      E = max(E, -100);
-    }
+    const int E = limb_exponent(amax);
     if (lane == 0) expo[warp] = E;
-    const float f = ldexpf(1.0f, kLimbFrac - E);
     for (int v = lane; v < nhalf; v += 32) {
       uint4 a2 = a, b2 = b;
       if (!(mine && v == lane)) { a2 = ld_nc(xb + 16 * v); b2 = ld_nc(xb + 16 * v + 8); }
       const uint32_t wv[8] = {a2.x, a2.y, a2.z, a2.w, b2.x, b2.y, b2.z, b2.w};
-      uint32_t l[3][4] = {};
+      uint32_t l[NC][4] = {};
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
         const uint32_t bits = (e & 1) ? (wv[e >> 1] >> 16) : (wv[e >> 1] & 0xFFFFu);
-        const int X = __float2int_rn(bf16_bits_to_float(bits) * f);   // exact power-of-two scaling
-        const int L0 = (int)(int8_t)(X & 0xFF);
-        const int X1 = (X - L0) >> 8;
-        const int L1 = (int)(int8_t)(X1 & 0xFF);
-        const int L2 = (X1 - L1) >> 8;                                 // |L2| <= 64
+        int L[4];
+        limbs_of(limb_fixed(bf16_bits_to_float(bits), E), L);
         const int sh = 8 * (e & 3);
-        l[0][e >> 2] |= (uint32_t)(uint8_t)L2 << sh;
-        l[1][e >> 2] |= (uint32_t)(uint8_t)L1 << sh;
-        l[2][e >> 2] |= (uint32_t)(uint8_t)L0 << sh;
+#pragma unroll
+        for (int c = 0; c < NC; ++c) l[c][e >> 2] |= (uint32_t)(uint8_t)L[c] << sh;
       }
       const int o = slot_of(v);
 #pragma unroll
-      for (int c = 0; c < 3; ++c) {
+      for (int c = 0; c < NC; ++c) {
         xsum[c] += bsum(l[c][0]) + bsum(l[c][1]) + bsum(l[c][2]) + bsum(l[c][3]);
         *reinterpret_cast<uint4*>(xw + c * p.x_words + o) = permute_i8_half(make_uint4(l[c][0], l[c][1], l[c][2], l[c][3]));
       }
@@ -327,11 +318,12 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_tern_stream(const StreamPa
           int sum = 0;
           for (int q = 0; q < WPT; ++q) sum += base[q * 16 * NC];
           y = __fmul_rn(__fmul_rn(__int2float_rn(sum), p.sx[0]), sc);
+          if (p.acc) p.acc[row] = sum;
         } else {
           double tot = 0.0;
           for (int q = 0; q < WPT; ++q) {
             const int* b = base + q * 16 * NC;
-            const long long D = (long long)b[0] * 65536 + (long long)b[1] * 256 + (long long)b[2];
+            const long long D = limb_combine(b[0], b[1], b[2], b[3]);
             tot += ldexp((double)D, expo[grp * 8 + tw * WPT + q] - kLimbFrac);
           }
           y = (float)(tot * (double)sc);
@@ -371,7 +363,7 @@ bool plan_stream(int N, int K, int mode, StreamParams& p, size_t& smem) {
   p.ts = best_ts;
   p.stage_bytes = best_ts * 16 * (K / 4);
   p.tiles = (N + 15) / 16;
-  const int nc = mode == 0 ? 3 : 1;
+  const int nc = mode == 0 ? 4 : 1;
   const int wpt = kConsumerWarps / best_ts;
   const int part_words = K / 32 / wpt;
   p.x_words = ((part_words + 15) / 16) * 128 + 4;  // whole chunks of one K part (+4 words: banks)
@@ -393,12 +385,9 @@ bool plan_stream(int N, int K, int mode, StreamParams& p, size_t& smem) {
 
 template <int MODE, int CW, bool XREG>
 cudaError_t launch_cw(const cudaLaunchConfig_t& cfg0, const StreamParams& p, size_t smem) {
-  static int set = 0;
-  if ((int)smem > set) {
-    cudaError_t e = cudaFuncSetAttribute(k_tern_stream<MODE, CW, XREG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    set = (int)smem;
-  }
+  static std::atomic<unsigned long long> smem_raised{0};
+  cudaError_t e = allow_max_dynamic_smem(k_tern_stream<MODE, CW, XREG>, smem_raised);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = cfg0;
   cfg.blockDim = dim3((CW + 1) * 32, 1, 1);
   return cudaLaunchKernelEx(&cfg, k_tern_stream<MODE, CW, XREG>, p);
@@ -411,7 +400,8 @@ cudaError_t launch_x(const cudaLaunchConfig_t& cfg, const StreamParams& p, size_
 
 cudaError_t launch_stream(const StreamParams& p, size_t smem, bool pdl, cudaStream_t st) {
   const int groups = (p.tiles + p.ts - 1) / p.ts;
-  const int grid = groups < 148 ? groups : 148;
+  const int sms = device_sm_count();
+  const int grid = groups < sms ? groups : sms;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
   cfg.dynamicSmemBytes = smem;

@@ -21,13 +21,32 @@
  *   - Every pointer named *_dev is device memory owned by the caller; the library keeps no
  *     reference after the call returns and allocates no device memory.
  *   - Work is enqueued asynchronously on `stream` (NULL = the legacy default stream); nothing
- *     synchronises except tern_read_flag.
+ *     synchronises except tern_read_flag and tern_device_status.
  *   - Argument errors are returned before anything is enqueued. A launch error is returned as
  *     TERN_ECUDA (the CUDA error is left to cudaGetLastError-style inspection by the caller).
  *   - Data errors that only the device can see (a trit outside {-1,0,+1}, a transport byte above
  *     242) set *err_flag_dev to a nonzero value; read it with tern_read_flag. Kernels never trap and
  *     never wait without a bound.
  *   - Outputs are deterministic: the same inputs give the same bits on every run.
+ *   - Precision of the bf16 mode: products with the ternary (or int8) weights are exact and sums
+ *     are exact integers; the only roundings are the activation encoding (a group of activations
+ *     with absmax below 2^E is held on a grid of 2^(E - 30), so an activation moves by at most
+ *     2^(E - 31)) and the final conversion to fp32. Every output y of a K-term product is
+ *     therefore within scale * K * 2^-30 * sum_k |x_k| (+ half an fp32 ulp of y) of the exact
+ *     value, whatever the inputs' dynamic range; for K <= 12288 that is under 1.2e-5 * scale *
+ *     sum_k |x_k|. tern_gemm_prefill instead accumulates exact bf16 products in fp32 on the
+ *     tensor cores.
+ *   - Global state, all of it: one device word per kernel family that latches TERN_ETIMEOUT when
+ *     a bounded wait gives up (shared by every stream and caller on a device; tern_device_status
+ *     reads and clears them), the scratch array of i8_head_gemv_argmax_noalloc, and host-side
+ *     records, per device, of the kernel attributes already set and of that array's address.
+ *
+ * Deliberate differences from the entry points sketched for this library's boundary
+ *   - tern_pack takes no scale argument: the per-row fp16 scales stay a separate caller array
+ *     that a tern_matrix points to; packing would only copy it.
+ *   - The launch flags of the *_ex entry points, the batched entry points (tern_pack_batch,
+ *     tern_gemv_batch, tern_gemm_batch), tern_base3_encode, tern_occupancy, tern_quantize_act and
+ *     i8_head_gemv_argmax_noalloc are additions.
  *
  * Packed layout (this library's own; the pages' FV5 bit-planes are only partly described)
  *   Matrix N x K, K a multiple of 128. Row n occupies K/16 uint32 words at word offset n*K/16:
@@ -150,15 +169,17 @@ tern_status tern_quantize_act(const uint16_t* x_bf16_dev, int32_t M, int32_t K, 
 /* M = 1 ternary GEMV: y[n] = scale[n] * sum_k t[n][k] * x[k]  ([R] "학습 중에 포맷이 있어야 하는
  * 이유"; [O] Figure I).
  *   act = TERN_ACT_BF16: x_dev = bf16[K] (bit patterns); x_scale_dev ignored (may be NULL).
- *                        Products are exact, accumulation is fp32 on the tensor cores.
+ *                        Exact integer sums of the encoded activations (see Conventions).
  *   act = TERN_ACT_INT8: x_dev = int8[K] from tern_quantize_act, x_scale_dev = &s_x (device).
  *                        acc = sum t*q in int32 (exact), y = ((float)acc * s_x) * scale with two
  *                        fp32 round-to-nearest multiplies.
- *   y_dev: float[N]. x_dev 16-byte aligned. */
+ *   y_dev: float[N]. x_dev 16-byte aligned.
+ *   acc_i32_dev: optional int32[N] (NULL to skip): int8 mode writes acc itself there; must be NULL
+ *                in bf16 mode (TERN_EINVAL otherwise). */
 tern_status tern_gemv(const tern_matrix* W, tern_act act, const void* x_dev, const float* x_scale_dev,
-                      float* y_dev, tern_stream_t stream);
+                      float* y_dev, int32_t* acc_i32_dev, tern_stream_t stream);
 tern_status tern_gemv_ex(const tern_matrix* W, tern_act act, const void* x_dev, const float* x_scale_dev,
-                         float* y_dev, uint32_t flags, tern_stream_t stream);
+                         float* y_dev, int32_t* acc_i32_dev, uint32_t flags, tern_stream_t stream);
 
 /* One M = 1 GEMV of a batch: y[n] = scale[n] * sum_k t[n][k] * x[k] for matrix W. */
 typedef struct {
@@ -255,7 +276,10 @@ tern_status i8_head_gemv_argmax_ex(const int8_t* W_dev, const uint16_t* scale_f1
  *   - M outside 1..TERN_HEAD_NOALLOC_MAX_M (scratch need above the array's size): TERN_ESHAPE,
  *     nothing launched.
  *   - The first call on a device looks up the array's address (cudaGetSymbolAddress, with that
- *     device current) and keeps it; that first call must come before any stream capture.
+ *     device current) and keeps it; that first call must come before any stream capture. The kept
+ *     address belongs to the device's context: after cudaDeviceReset on that device, this entry
+ *     point must not be called again in the process.
+ *   - Every argument is checked before anything is enqueued, exactly as for i8_head_gemv_argmax.
  *   - Each call clears the scratch bytes it uses (cudaMemsetAsync on `stream`) before the launch;
  *     no call allocates or frees device memory.
  *   - All calls on one device share the array: calls that overlap in time (different streams,
@@ -272,8 +296,10 @@ tern_status tern_read_flag(const int32_t* err_flag_dev, tern_stream_t stream);
 
 /* Synchronise `stream` and report whether any kernel of this library on the current device gave
  * up a bounded wait (an mbarrier that did not complete within seconds) since the last call:
- * TERN_ETIMEOUT if so, else TERN_OK. Reading clears the device's latch. Kernels that give up
- * stop early and leave their outputs incomplete; they never hang or trap. */
+ * TERN_ETIMEOUT if so, else TERN_OK. Reading clears the device's latches (one device word per
+ * kernel family, the library's only device-side state besides the no-allocation head's scratch;
+ * they are shared by every stream and caller of the device). Kernels that give up stop early and
+ * leave their outputs incomplete; they never hang or trap. */
 tern_status tern_device_status(tern_stream_t stream);
 
 #if defined(__GNUC__)

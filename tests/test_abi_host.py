@@ -45,16 +45,18 @@ def test_argument_errors_before_launch(L):
     import bit_gemv_tern_b200 as tg
     fake = 1 << 40                      # never dereferenced: validation fails first
     m = tg._Matrix(64, 100, fake, fake)  # K % 128 != 0
-    assert L.tern_gemv(ctypes.byref(m), 0, fake, None, fake, None) == tg.TERN_ESHAPE
+    assert L.tern_gemv(ctypes.byref(m), 0, fake, None, fake, None, None) == tg.TERN_ESHAPE
     m = tg._Matrix(64, 128, None, fake)
-    assert L.tern_gemv(ctypes.byref(m), 0, fake, None, fake, None) == tg.TERN_EINVAL
+    assert L.tern_gemv(ctypes.byref(m), 0, fake, None, fake, None, None) == tg.TERN_EINVAL
     m = tg._Matrix(64, 128, fake, fake)
-    assert L.tern_gemv(ctypes.byref(m), 7, fake, None, fake, None) == tg.TERN_EINVAL        # bad act
-    assert L.tern_gemv(ctypes.byref(m), 1, fake, None, fake, None) == tg.TERN_EINVAL        # int8 needs s_x
-    assert L.tern_gemv(ctypes.byref(m), 0, fake + 4, None, fake, None) == tg.TERN_EINVAL    # misaligned x
+    assert L.tern_gemv(ctypes.byref(m), 7, fake, None, fake, None, None) == tg.TERN_EINVAL        # bad act
+    assert L.tern_gemv(ctypes.byref(m), 1, fake, None, fake, None, None) == tg.TERN_EINVAL        # int8 needs s_x
+    assert L.tern_gemv(ctypes.byref(m), 0, fake + 4, None, fake, None, None) == tg.TERN_EINVAL    # misaligned x
+    assert L.tern_gemv(ctypes.byref(m), 0, fake, None, fake, fake, None) == tg.TERN_EINVAL        # acc in bf16 mode
+    assert L.tern_gemv(ctypes.byref(m), 1, fake, fake, fake, fake + 2, None) == tg.TERN_EINVAL    # misaligned acc
     assert L.tern_gemm_small_m(ctypes.byref(m), 17, 0, fake, None, fake, None) == tg.TERN_ESHAPE
     assert L.tern_gemm_small_m(ctypes.byref(m), 0, 0, fake, None, fake, None) == tg.TERN_ESHAPE
-    assert L.tern_gemv_ex(ctypes.byref(m), 0, fake, None, fake, 8, None) == tg.TERN_EINVAL   # unknown flag
+    assert L.tern_gemv_ex(ctypes.byref(m), 0, fake, None, fake, None, 8, None) == tg.TERN_EINVAL   # unknown flag
     assert L.tern_pack(0, fake, 4, 96, fake, fake, None) == tg.TERN_ESHAPE
     assert L.tern_pack(5, fake, 4, 128, fake, fake, None) == tg.TERN_EINVAL
     assert L.tern_pack(0, fake, 4, 128, fake, None, None) == tg.TERN_EINVAL

@@ -23,12 +23,15 @@ def _run_bf16(W, x):
     return host(y)
 
 
-def _run_i8(W, x, K):
+def _run_i8(W, x, K, with_acc=False):
     q = torch.empty(K, dtype=torch.int8, device="cuda")
     sx = torch.empty(1, dtype=torch.float32, device="cuda")
     tg.tern_quantize_act(dev(x.view(np.int16)), 1, K, q, sx)
     y = torch.empty(W.N, dtype=torch.float32, device="cuda")
-    tg.tern_gemv(W, tg.TERN_ACT_INT8, q, sx, y)
+    acc = torch.full((W.N,), -7, dtype=torch.int32, device="cuda") if with_acc else None
+    tg.tern_gemv(W, tg.TERN_ACT_INT8, q, sx, y, acc=acc)
+    if with_acc:
+        return host(q), host(sx), host(y), host(acc)
     return host(q), host(sx), host(y)
 
 
@@ -45,10 +48,11 @@ def test_gemv_bf16(N, K):
 def test_gemv_int8_bit_exact(N, K):
     W, t, s = make_matrix(42, N * 13 + K, N, K)
     x = synth.activations(42, K, 1, K)
-    q, sx, y = _run_i8(W, x, K)
+    q, sx, y, acc = _run_i8(W, x, K, with_acc=True)
     q_ref, sx_ref = oracle.quantize_act(x, K)
     assert (q == q_ref[0]).all() and sx[0] == sx_ref[0]
-    _, y_ref = oracle.gemm_i8(oracle.pack(t), s, K, q_ref, sx_ref)
+    acc_ref, y_ref = oracle.gemm_i8(oracle.pack(t), s, K, q_ref, sx_ref)
+    assert (acc == acc_ref[0]).all(), "int32 accumulators"
     assert (y == y_ref[0]).all()
 
 

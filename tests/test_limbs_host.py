@@ -1,57 +1,133 @@
-"""Host checks of the exact three-limb encoding behind the bf16 activation mode (no GPU).
+"""Host checks of the exact four-limb encoding behind the bf16 activation mode (no GPU).
 
-The bf16 paths split each activation x into X = rint(x * 2^(22 - E)), E the exponent of the
-absmax (absmax < 2^E), and X into three int8 limbs L2, L1, L0 with X = L2 * 2^16 + L1 * 2^8 + L0.
-These tests check, over every finite bf16 bit pattern, that the split reconstructs X, that
-|L2| <= 64 (so every limb is a valid s8 tensor-core operand), and that X is exactly x * 2^(22 - E)
-whenever |x| >= 2^(E - 15): the bf16 mantissa has 8 significant bits, so such an x is an integer
-multiple of 2^(E - 22)."""
+The bf16 paths turn a group of activations (an item's row, a K part or a K slice) with absmax
+below 2^E (E from frexp of the absmax) into X = rint(x * 2^(30 - E)) and split X into four int8
+limbs, X = L3 * 2^24 + L2 * 2^16 + L1 * 2^8 + L0. The tensor cores then multiply the limbs by the
+exact ternary weights and sum in int32, so the encoding is the only rounding before the final
+conversion to fp32. These tests check, over every finite bf16 bit pattern:
+  * the split reconstructs X, L0..L2 are int8 and |L3| <= 64 (a valid s8 operand);
+  * X * 2^(E - 30) equals x whenever |x| >= 2^(E - 23) (a bf16 mantissa has 8 significant bits);
+  * the rounding error never exceeds 2^(E - 31);
+  * with that bound, every output of a K <= 12288 product meets the bf16-mode tolerance
+    |err| <= 1e-4 * scale * sum_k |x_k| for any inputs, including an outlier activation next to
+    values just below the cut, where the previous 22-bit three-limb encoding did not.
+The float32 emulation mirrors the kernels' documented arithmetic: one exact power-of-two multiply
+(two when 2^(30 - E) exceeds fp32's range), then round half to even."""
 import numpy as np
 import pytest
 
 pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
 
+F = 30          # fractional bits of the fixed-point value relative to 2^E
+PER_OUT = 1e-4  # the bf16-mode per-output tolerance factor
+
 
 def _all_bf16():
     bits = np.arange(1 << 16, dtype=np.uint32)
-    x = (bits << 16).view(np.float32).astype(np.float64)
+    x = (bits << 16).view(np.float32)
     return x[np.isfinite(x)]
 
 
-def _split(X):
-    L0 = ((X & 0xFF) ^ 0x80) - 0x80                      # sign-extended low byte
-    X1 = (X - L0) >> 8
-    L1 = ((X1 & 0xFF) ^ 0x80) - 0x80
-    L2 = (X1 - L1) >> 8
-    return L2, L1, L0
+def _exponent(a):
+    """E with a < 2^E (and 2^(E-1) <= a for a > 0); 0 for a == 0."""
+    if a == 0:
+        return 0
+    return int(np.frexp(np.float64(a))[1])
 
 
-@pytest.mark.parametrize("E", [-20, -3, 0, 1, 2, 3, 7, 40])
+def _fixed(x32, E, frac=F):
+    """rint(x * 2^(frac - E)) as the kernels form it in fp32."""
+    s = frac - E
+    x32 = np.asarray(x32, np.float32)
+    if s <= 126:
+        v = x32 * np.float32(2.0 ** s)
+    else:
+        v = (x32 * np.float32(2.0 ** 64)) * np.float32(2.0 ** (s - 64))
+    return np.rint(v.astype(np.float64)).astype(np.int64)
+
+
+def _split(X, limbs=4):
+    out = []
+    for _ in range(limbs - 1):
+        lo = ((X & 0xFF) ^ 0x80) - 0x80                   # sign-extended low byte
+        out.append(lo)
+        X = (X - lo) >> 8
+    out.append(X)
+    return out[::-1]                                      # top limb first
+
+
+def _encode(x32, frac=F, limbs=4):
+    """Per-group encoding of an fp32 (bf16-valued) vector: the value each element stands for."""
+    E = _exponent(np.abs(x32).max())
+    X = _fixed(x32, E, frac)
+    parts = _split(X, limbs)
+    Xr = sum(L * (1 << (8 * (limbs - 1 - i))) for i, L in enumerate(parts))
+    return Xr.astype(np.float64) * 2.0 ** (E - frac)
+
+
+@pytest.mark.parametrize("E", [-132, -110, -97, -96, -20, -3, 0, 1, 2, 7, 40, 127, 128])
 def test_limbs_reconstruct_and_fit(E):
     x = _all_bf16()
-    x = x[np.abs(x) < 2.0 ** E]                         # the item's absmax is below 2^E
-    X = np.rint(x * 2.0 ** (22 - E)).astype(np.int64)   # round half to even, like the kernels
-    assert np.abs(X).max() <= 2 ** 22
-    L2, L1, L0 = _split(X)
-    assert (L2 * 65536 + L1 * 256 + L0 == X).all()
-    for L in (L1, L0):
+    x = x[np.abs(x.astype(np.float64)) < 2.0 ** E]       # the group's absmax is below 2^E
+    X = _fixed(x, E)
+    assert np.abs(X).max() <= 2 ** F
+    L3, L2, L1, L0 = _split(X)
+    assert (L3 * 2 ** 24 + L2 * 2 ** 16 + L1 * 2 ** 8 + L0 == X).all()
+    for L in (L2, L1, L0):
         assert L.min() >= -128 and L.max() <= 127
-    assert np.abs(L2).max() <= 64
+    assert np.abs(L3).max() <= 64
 
 
-@pytest.mark.parametrize("E", [-3, 0, 2, 7])
+@pytest.mark.parametrize("E", [-120, -3, 0, 2, 7, 100])
 def test_limbs_exact_above_the_cut(E):
-    x = _all_bf16()
-    x = x[(np.abs(x) < 2.0 ** E) & (np.abs(x) >= 2.0 ** (E - 15))]
-    scaled = x * 2.0 ** (22 - E)                        # exact in fp64 (a power-of-two scaling)
-    assert (scaled == np.rint(scaled)).all()            # already an integer: no rounding happens
+    x = _all_bf16().astype(np.float64)
+    x = x[(np.abs(x) < 2.0 ** E) & (np.abs(x) >= 2.0 ** (E - 23))]
+    scaled = x * 2.0 ** (F - E)                          # exact in fp64 (a power-of-two scaling)
+    assert (scaled == np.rint(scaled)).all()             # already an integer: no rounding happens
 
 
-def test_limbs_round_below_the_cut():
-    """Values below 2^(E - 15) do round (the documented bound), by at most half a unit of 2^(E - 22)."""
-    E = 2
+@pytest.mark.parametrize("E", [-132, -100, -40, -3, 0, 2, 7, 64, 128])
+def test_limbs_error_bound_over_all_bf16(E):
+    """|x - X * 2^(E - 30)| <= 2^(E - 31) for every finite bf16 x below 2^E, and the bound is met
+    with equality somewhere (it is the half unit of the fixed-point grid)."""
     x = _all_bf16()
-    x = x[(np.abs(x) < 2.0 ** (E - 15)) & (x != 0)]
-    scaled = x * 2.0 ** (22 - E)
-    err = np.abs(np.rint(scaled) - scaled)
-    assert err.max() <= 0.5 and (err > 0).any()
+    x = x[np.abs(x.astype(np.float64)) < 2.0 ** E]
+    X = _fixed(x, E)
+    err = np.abs(X.astype(np.float64) * 2.0 ** (E - F) - x.astype(np.float64))
+    assert err.max() <= 2.0 ** (E - F - 1)
+    if E > -100:
+        assert (err == 2.0 ** (E - F - 1)).any()
+
+
+def _worst_output_error(K, frac, limbs, rng):
+    """An all-+1 row against an outlier of 1024 next to K-1 values whose encoding error is as large
+    as the grid allows and of one sign (so nothing cancels): the encoded sum's error and the
+    per-output bound (scale 1)."""
+    E = 11                                              # absmax 1024 < 2^11
+    cut = E - frac - 1                                  # values of exponent cut - 1 round by a half unit
+    m = rng.integers(0, 64, K - 1) * 2 + 1              # odd 7-bit mantissas: a half unit off the grid
+    small = ((1.0 + m / 128.0) * 2.0 ** (cut - 1)).astype(np.float32)
+    x = np.concatenate([np.float32([1024.0]), small])
+    exact = x.astype(np.float64).sum()
+    enc = _encode(x, frac, limbs).sum()
+    return abs(enc - exact), PER_OUT * np.abs(x.astype(np.float64)).sum()
+
+
+@pytest.mark.parametrize("K", [1024, 4096, 12288])
+def test_outlier_next_to_values_below_the_cut_meets_the_bound(K):
+    err, bound = _worst_output_error(K, F, 4, np.random.default_rng(K))
+    assert err <= bound, (err, bound)
+
+
+def test_three_limb_22_bit_encoding_misses_the_bound():
+    """The same input under the earlier encoding (22 fractional bits, three limbs) breaks the
+    bound, so the test above does test something: the per-output check catches this failure."""
+    err, bound = _worst_output_error(4096, 22, 3, np.random.default_rng(1))
+    assert err > 5 * bound
+
+
+def test_bound_holds_up_to_107k():
+    """Per output, the encoding error is at most K * 2^(E-31) <= K * 2^-30 * sum|x| (absmax >= 2^(E-1)):
+    within 1e-4 * sum|x| for every K up to 107,374, beyond the largest K (12288) of the batched path."""
+    assert 12288 * 2.0 ** -F <= PER_OUT
+    assert 107374 * 2.0 ** -F <= PER_OUT < 107375 * 2.0 ** -F
