@@ -36,6 +36,10 @@ def lib() -> ctypes.CDLL:
         L.orc_gemm_i8.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp, vp, i32]; L.orc_gemm_i8.restype = None
         L.orc_head_bf16.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp, vp, i32]; L.orc_head_bf16.restype = None
         L.orc_head_i8.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp, vp, vp, i32]; L.orc_head_i8.restype = None
+        L.orc_round_bf16.argtypes = [ctypes.c_double]; L.orc_round_bf16.restype = ctypes.c_uint16
+        L.orc_rmsnorm.argtypes = [vp, i32, i32, vp, ctypes.c_double, vp]; L.orc_rmsnorm.restype = None
+        L.orc_swiglu.argtypes = [vp, i32, i32, vp]; L.orc_swiglu.restype = None
+        L.orc_verify_accept.argtypes = [vp, vp, i32, vp, vp]; L.orc_verify_accept.restype = None
         _LIB = L
     return _LIB
 
@@ -186,3 +190,43 @@ def head_i8(W: np.ndarray, sh_f16: np.ndarray, q: np.ndarray, sx: np.ndarray, wa
     lg = np.empty((M, V), dtype=np.float32) if want_logits else None
     lib().orc_head_i8(_p(w), _p(sh), V, K, M, _p(qq), _p(sxx), _p(lg), _p(am), _p(mv), nthreads or default_threads())
     return am, mv, lg
+
+
+def round_bf16(v) -> np.ndarray:
+    """fp64 values -> bf16 bit patterns (uint16), round to nearest, ties to even."""
+    a = np.asarray(v, dtype=np.float64)
+    f = lib().orc_round_bf16
+    return np.array([f(float(x)) for x in a.reshape(-1)], dtype=np.uint16).reshape(a.shape)
+
+
+def rmsnorm(x_f32: np.ndarray, gain_bf16: np.ndarray, eps: float) -> np.ndarray:
+    """bf16 bits [M, K] of RMSNorm(x) * gain per row (fp64, one rounding); x fp32 [M, K] or [K]."""
+    K = np.asarray(gain_bf16).size
+    x = _c(x_f32, np.float32).reshape(-1, K)
+    M = x.shape[0]
+    g = _c(gain_bf16, np.uint16)
+    out = np.empty((M, K), dtype=np.uint16)
+    lib().orc_rmsnorm(_p(x), M, K, _p(g), float(eps), _p(out))
+    return out
+
+
+def swiglu(gu_f32: np.ndarray, K: int) -> np.ndarray:
+    """bf16 bits [M, K] of silu(gate) * up per row; gu fp32 [M, 2K] (gate first, then up)."""
+    gu = _c(gu_f32, np.float32).reshape(-1, 2 * K)
+    M = gu.shape[0]
+    out = np.empty((M, K), dtype=np.uint16)
+    lib().orc_swiglu(_p(gu), M, K, _p(out))
+    return out
+
+
+def verify_accept(argmax, draft) -> tuple[int, int]:
+    """(accepted drafts n, next token argmax[n]) for argmax [k+1] and draft [k]."""
+    am = _c(argmax, np.int32).reshape(-1)
+    dr = _c(draft, np.int32).reshape(-1)
+    k = dr.size
+    if am.size != k + 1:
+        raise OracleError("argmax needs k + 1 entries")
+    n = np.zeros(1, np.int32)
+    nt = np.zeros(1, np.int32)
+    lib().orc_verify_accept(_p(am), _p(dr) if k else _p(np.zeros(1, np.int32)), k, _p(n), _p(nt))
+    return int(n[0]), int(nt[0])

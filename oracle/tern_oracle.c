@@ -28,7 +28,14 @@
  *     ([R] "토큰 동일성의 경계: 그리디, float32, 그리고 두 개의 근접 동점");
  *   - the int8 output head with greedy argmax ([R] "3진 계열이라는 이름의 실체": embeddings and
  *     head stay int8; [R] "토큰 동일성의 경계": near ties between implementations); the lowest
- *     index wins an exact tie.
+ *     index wins an exact tie;
+ *   - the steps on either side of the linears in a Qwen3 block ([R] "세 모델과 하나의 컨테이너",
+ *     model table: RMSNorm, SwiGLU): RMSNorm y = x / sqrt(mean(x^2) + eps) * gain, and
+ *     SwiGLU h = silu(gate) * up with silu(z) = z / (1 + e^-z); both computed in fp64 from fp32
+ *     inputs and rounded once to bf16, the activation type of the next linear;
+ *   - the acceptance rule of speculative decoding ([R] "검증된 추측 디코딩: 속도만 바꾸고 답은
+ *     바꾸지 않는다"): the target scores the k drafted positions in one pass and keeps the longest
+ *     prefix of drafts that equal its own greedy choices, then adds its own next token.
  *
  * Packed layout (this library's own definition; the pages' FV5 planes are only partly described):
  *   row n of an N x K matrix (K % 128 == 0) occupies K/16 uint32 words starting at word n*K/16;
@@ -68,6 +75,30 @@ float orc_bf16_to_float(uint16_t b) {
   float f;
   memcpy(&f, &u, 4);
   return f;
+}
+
+/* double -> bfloat16, round to nearest, ties to even, in one step from the format definition
+ * (sign, 8-bit exponent with bias 127, 7 fraction bits; subnormals are multiples of 2^-133). */
+uint16_t orc_round_bf16(double v) {
+  if (isnan(v)) return 0x7FC0;
+  const uint16_t sign = signbit(v) ? 0x8000 : 0;
+  const double a = fabs(v);
+  if (a == 0.0) return sign;
+  if (isinf(a)) return sign | 0x7F80;
+  int ex;
+  frexp(a, &ex);                        /* 2^(ex-1) <= a < 2^ex */
+  int e = ex - 1;                       /* unbiased exponent of a */
+  if (e < -126) e = -126;               /* subnormal range: the quantum stays 2^-133 */
+  const double q = ldexp(1.0, e - 7);   /* spacing of bf16 values with this exponent */
+  const double r = rint(a / q);         /* a / q is exact (power of two); rint: ties to even */
+  /* r * q is the rounded magnitude; r = 256 carries into the next exponent, and a subnormal
+   * that rounds up to 2^-126 (r = 128 at e = -126) lands on the smallest normal: in both cases the
+   * encoding below, exponent field + fraction, gives the right bits. */
+  uint32_t bits;
+  if (r >= 128.0) bits = (uint32_t)(e + 127) * 128u + (uint32_t)(r - 128.0);
+  else bits = (uint32_t)r;              /* subnormal (e == -126): fraction field = r */
+  if (bits >= 0x7F80u) return sign | 0x7F80;   /* overflow to infinity */
+  return sign | (uint16_t)bits;
 }
 
 /* ----------------------------------------------------------------------------------------- */
@@ -358,4 +389,49 @@ void orc_head_i8(const int8_t* W, const uint16_t* SH, int32_t V, int32_t K, int3
     MAXV[m] = L[(size_t)m * V + best];
   }
   if (!LOGITS) free(L);
+}
+
+/* ----------------------------------------------------------------------------------------- */
+/* the steps on either side of the linears                                                     */
+
+/* RMSNorm of each fp32 row x[m][0..K): r = 1 / sqrt(sum_k x_k^2 / K + eps) in fp64, then
+ * out_k = bf16((x_k * r) * gain_k), the products in fp64 and one rounding to bf16. */
+void orc_rmsnorm(const float* X, int32_t M, int32_t K, const uint16_t* gain_bf16, double eps, uint16_t* OUT) {
+  for (int m = 0; m < M; ++m) {
+    const float* x = X + (size_t)m * K;
+    double ss = 0.0;
+    for (int k = 0; k < K; ++k) ss += (double)x[k] * (double)x[k];
+    const double r = 1.0 / sqrt(ss / (double)K + eps);
+    for (int k = 0; k < K; ++k)
+      OUT[(size_t)m * K + k] = orc_round_bf16(((double)x[k] * r) * (double)orc_bf16_to_float(gain_bf16[k]));
+  }
+}
+
+/* SwiGLU of each row of a gate|up output GU[m][0..2K) (gate at k, up at K + k):
+ * out_k = bf16(silu(g_k) * u_k), silu(z) = z / (1 + exp(-z)), all in fp64. */
+void orc_swiglu(const float* GU, int32_t M, int32_t K, uint16_t* OUT) {
+  for (int m = 0; m < M; ++m) {
+    const float* g = GU + (size_t)m * 2 * K;
+    const float* u = g + K;
+    for (int k = 0; k < K; ++k) {
+      const double z = (double)g[k];
+      const double silu = z / (1.0 + exp(-z));
+      OUT[(size_t)m * K + k] = orc_round_bf16(silu * (double)u[k]);
+    }
+  }
+}
+
+/* ----------------------------------------------------------------------------------------- */
+/* speculative-verify acceptance                                                               */
+
+/* The verify pass scores positions 0..k: argmax[j] is the target's greedy token after position
+ * j, and draft[j] the drafted token for position j + 1. The accepted count n is the length of the
+ * longest prefix with draft[j] == argmax[j]; the target then supplies argmax[n], so a round
+ * yields n + 1 tokens. */
+void orc_verify_accept(const int32_t* argmax, const int32_t* draft, int32_t k, int32_t* n_accept,
+                       int32_t* next_token) {
+  int32_t n = 0;
+  while (n < k && draft[n] == argmax[n]) ++n;
+  *n_accept = n;
+  *next_token = argmax[n];
 }
