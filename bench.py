@@ -33,10 +33,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "ternary GEMV HBM GB/s & 8B linear-stack tok/s at M=1 (fraction of HBM peak)"
-# DRAM bytes (read + write) of the stream kernel per full 8B step, from the ncu capture summarised
-# in profiles/k_batch_stream_8b_4layers_bf16.md (4 layers: 203.17 MB read + 6.00 MB written),
-# scaled by the units processed (36 / 4 layers). Set to None whenever that kernel changes.
-STREAM_TRAFFIC_PER_STEP = 9 * (203.17e6 + 6.00e6)
+# DRAM bytes (read + write) of the stream kernel per full 8B step, from an ncu capture of the
+# 4-layer profile case (batch-8b-4layers-bf16) scaled by the units processed (36 / 4 layers).
+# None whenever that kernel has changed since the counters were taken.
+STREAM_TRAFFIC_PER_STEP = None
 SEED = 0x7E2A2026
 L2_BYTES = 126 * 1024 * 1024
 
@@ -159,6 +159,31 @@ class Stack:
                 entries.append((lin.W, xb if mode == "bf16" else q, None if mode == "bf16" else sx, self.y[i]))
             self._batches[mode] = tg.GemvBatch(entries, act)
         return self._batches[mode]
+
+    def int8_fused_batch(self):
+        """The stack's GEMVs in int8 mode with the per-token quantiser fused into the batch's operand
+        preparation (bf16 activations in, s_x written by the prep): no separate quantiser launch."""
+        import torch
+        import bit_gemv_tern_b200 as tg
+        if "int8_fused" not in self._batches:
+            self.sx_fused = torch.empty(len(self.linears) * self.M, dtype=torch.float32, device="cuda")
+            entries, pros = [], []
+            for i, lin in enumerate(self.linears):
+                xb, _, _ = self.xs(i)
+                entries.append((lin.W, None, self.sx_fused[i * self.M:(i + 1) * self.M], self.y[i]))
+                pros.append((tg.TERN_PRO_BF16, xb, None, 0.0))
+            self._batches["int8_fused"] = tg.GemvBatch(entries, tg.TERN_ACT_INT8, M=self.M, prologues=pros)
+        return self._batches["int8_fused"]
+
+    def launch_step_int8_fused(self):
+        """int8-mode decode step with every quantisation inside it: the stack's batch (quantiser fused
+        into its prep launch), then the head input's quantiser and the int8 head."""
+        import bit_gemv_tern_b200 as tg
+        self.int8_fused_batch()()
+        xb, q, sx = self.xs(len(self.linears))
+        tg.tern_quantize_act(xb, self.M, self.d, q, sx)
+        tg.i8_head_gemv_argmax(self.head_W, self.head_s, self.V, self.d, self.M, tg.TERN_ACT_INT8, q, sx,
+                               self.argmax, self.maxval, None, self.ws)
 
     def launch_stack(self, mode="bf16", pdl=False, chained=False):
         """M = 1: one batched launch pair for all linears (their activations are independent
@@ -632,13 +657,27 @@ def extra_rows(stack, torch, tg, hbm_peak, bf16_peak):
     def gbs_of(nbytes, ms):
         return nbytes / (ms / 1000.0) / 1e9
 
-    # int8-activation mode on the same 8B stack
+    # int8-activation mode on the same 8B stack, every quantisation inside the step (the stack's
+    # quantiser fused into its prep launch, one quantiser launch for the head input)
     reps = 50
+    g = capture(lambda i: stack.launch_step_int8_fused(), 10)
+    g.replay()
+    ms = timed_replays([(g, reps // 10)]) / reps
+    nb = stack.stack_bytes + stack.head_bytes
+    out["8b_stack_m1_int8"] = {"tok_s": 1000.0 / ms, "ms": ms, "gbs": gbs_of(nb, ms), "frac": gbs_of(nb, ms) / hbm_peak,
+                               "launches_per_step": 4,
+                               "note": "bf16 activations in; quantiser fused into the batch prep; head input quantised in the step"}
+    # the same with activations quantised once before the timed region (kernel-only comparison)
     g = capture(lambda i: (stack.launch_stack("int8"), stack.launch_head("int8")), 10)
     g.replay()
     ms = timed_replays([(g, reps // 10)]) / reps
     nb = stack.stack_bytes - sum(l.K for l in stack.linears) + stack.head_bytes - stack.d
-    out["8b_stack_m1_int8"] = {"tok_s": 1000.0 / ms, "ms": ms, "gbs": gbs_of(nb, ms), "frac": gbs_of(nb, ms) / hbm_peak}
+    out["8b_stack_m1_int8_prequantised"] = {"tok_s": 1000.0 / ms, "ms": ms, "gbs": gbs_of(nb, ms),
+                                            "frac": gbs_of(nb, ms) / hbm_peak}
+    # a decode chain whose linears depend on one another through their prologues
+    out["8b_decode_chain_m1_bf16"] = chain_row(stack, torch, hbm_peak)
+    # speculative-verify rounds: k drafts + 1 through the stack and the head with on-device acceptance
+    out["verify_round_8b_bf16"] = verify_rows(stack, torch, tg, hbm_peak)
     # decode-chain variant: one launch per fused linear, each waiting for its predecessor (PDL)
     g = capture(lambda i: (stack.launch_stack("bf16", pdl=True, chained=True), stack.launch_head("bf16")), 10)
     g.replay()
@@ -702,6 +741,118 @@ def extra_rows(stack, torch, tg, hbm_peak, bf16_peak):
 
     # base-3 transport unpack of all 8B trits (bit-exact expansion into the planes)
     out["base3_unpack_8b"] = base3_row(stack, torch, tg, hbm_peak)
+    return out
+
+
+class Chain:
+    """One decode token through the 8B stack as a dependent chain: each fused linear's activation is
+    computed from the previous linear's fp32 output by a prologue fused into that linear's launch.
+    Per layer: q|k|v <- RMSNorm(h); o <- cast(q part of the q|k|v output, standing in for attention,
+    which is not a linear); gate|up <- RMSNorm(o output); down <- SwiGLU(gate|up output); the next
+    layer's h = the down output. The head takes the RMSNorm of the last h. No residual adds (not part
+    of the path). Weights are the stack's; gains and the entry h are seeded synthetic inputs."""
+
+    def __init__(self, stack, mode="bf16"):
+        import torch
+        import synth
+        import bit_gemv_tern_b200 as tg
+        self.stack, self.mode = stack, mode
+        act = tg.TERN_ACT_BF16 if mode == "bf16" else tg.TERN_ACT_INT8
+        d = stack.d
+        self.h0 = torch.from_numpy(synth.residual(SEED, 0, 1, d).reshape(-1)).cuda()
+        gains = [torch.from_numpy(synth.norm_gains(SEED, i, d).view(np.int16)).cuda() for i in range(2 * stack.L + 1)]
+        self.gains = gains
+        self.batches = []
+        self.sx = torch.empty(len(stack.linears), dtype=torch.float32, device="cuda")
+        src = self.h0
+        for i, lin in enumerate(stack.linears):
+            layer, grp = divmod(i, 4)
+            if grp == 0:
+                pro = (tg.TERN_PRO_RMSNORM, src, gains[2 * layer], 1e-6)
+            elif grp == 1:
+                pro = (tg.TERN_PRO_CAST, src, None, 0.0)          # first 4096 values of q|k|v: the q part
+            elif grp == 2:
+                pro = (tg.TERN_PRO_RMSNORM, src, gains[2 * layer + 1], 1e-6)
+            else:
+                pro = (tg.TERN_PRO_SWIGLU, src, None, 0.0)
+            entry = (lin.W, None, self.sx[i:i + 1] if act == tg.TERN_ACT_INT8 else None, stack.y[i])
+            self.batches.append(tg.GemvBatch([entry], act, M=1, prologues=[pro]))
+            src = stack.y[i]
+        self.last = src
+        self.x_head = torch.empty(d, dtype=torch.int16, device="cuda")
+        self.q_head = torch.empty(d, dtype=torch.int8, device="cuda")
+        self.sx_head = torch.empty(1, dtype=torch.float32, device="cuda")
+
+    def launch(self):
+        import bit_gemv_tern_b200 as tg
+        st = self.stack
+        for b in self.batches:
+            b(flags=tg.TERN_FLAG_PDL)
+        tg.tern_act_prologue(tg.TERN_PRO_RMSNORM, self.last, self.gains[-1], 1e-6, 1, st.d, self.x_head)
+        if self.mode == "bf16":
+            tg.i8_head_gemv_argmax(st.head_W, st.head_s, st.V, st.d, 1, tg.TERN_ACT_BF16, self.x_head, None,
+                                   st.argmax, st.maxval, None, st.ws)
+        else:
+            tg.tern_quantize_act(self.x_head, 1, st.d, self.q_head, self.sx_head)
+            tg.i8_head_gemv_argmax(st.head_W, st.head_s, st.V, st.d, 1, tg.TERN_ACT_INT8, self.q_head, self.sx_head,
+                                   st.argmax, st.maxval, None, st.ws)
+
+    @property
+    def launches(self):
+        return 2 * len(self.batches) + 2 + (1 if self.mode == "int8" else 0)
+
+
+def chain_row(stack, torch, hbm_peak):
+    import bit_gemv_tern_b200 as tg
+    out = {}
+    for mode in ("bf16", "int8"):
+        ch = Chain(stack, mode)
+        g = capture(lambda i: ch.launch(), 5)
+        g.replay()
+        torch.cuda.synchronize()
+        assert tg.tern_device_status() == tg.TERN_OK
+        ms = timed_replays([(g, 4)]) / 20
+        nb = stack.stack_bytes + stack.head_bytes
+        out[mode] = {"tok_s": 1000.0 / ms, "ms": ms, "gbs": nb / (ms / 1000.0) / 1e9,
+                     "frac": nb / (ms / 1000.0) / 1e9 / hbm_peak, "launches_per_token": ch.launches}
+        del g, ch
+    return out
+
+
+def verify_rows(stack, torch, tg, hbm_peak):
+    """k drafted tokens + 1 through the 8B stack (one small-M batch) and the head with the acceptance
+    count on the device. Drafts equal to the target's own greedy tokens (from a previous pass) give
+    the all-accepted round (k + 1 tokens); drafts that all miss give 1 token."""
+    out = {}
+    for k in (1, 3, 6):
+        M = k + 1
+        sv = StackView(stack, M)
+        accept = torch.empty(2, dtype=torch.int32, device="cuda")
+        draft = torch.empty(k, dtype=torch.int32, device="cuda")
+        sv.launch_stack("bf16")
+        sv.launch_head("bf16")
+        torch.cuda.synchronize()
+        hits = sv.argmax[:k].clone()
+
+        def round_(i):
+            sv.launch_stack("bf16")
+            tg.i8_head_verify(stack.head_W, stack.head_s, sv.V, sv.d, M, tg.TERN_ACT_BF16, sv.x[:M * sv.d], None,
+                              draft, sv.argmax, sv.maxval, accept, sv.ws)
+        row = {}
+        for case, d in (("all_accepted", hits), ("none_accepted", hits + 1)):
+            draft.copy_(d)
+            g = capture(round_, 5)
+            g.replay()
+            torch.cuda.synchronize()
+            n = int(accept[0].item())
+            ms = timed_replays([(g, 4)]) / 20
+            row[case] = {"pass_us": ms * 1000.0, "accepted": n, "tokens_per_round": n + 1,
+                         "tokens_per_s": (n + 1) * 1000.0 / ms}
+            del g
+        nb = sv.stack_bytes + sv.head_bytes
+        row["frac_hbm"] = nb / (row["all_accepted"]["pass_us"] / 1e6) / 1e9 / hbm_peak
+        out[f"k{k}"] = row
+        del sv
     return out
 
 

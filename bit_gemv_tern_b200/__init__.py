@@ -23,7 +23,9 @@ __all__ = [
     "i8_head_workspace_bytes", "i8_head_gemv_argmax", "i8_head_gemv_argmax_noalloc",
     "TERN_HEAD_NOALLOC_MAX_M", "tern_read_flag", "tern_device_status",
     "GemvBatch", "tern_gemv_batch", "tern_gemv_batch_workspace_bytes", "tern_gemm_batch",
-    "tern_gemm_batch_workspace_bytes",
+    "tern_gemm_batch_workspace_bytes", "tern_gemm_batch_pro", "tern_act_prologue",
+    "i8_head_verify", "tern_verify_accept",
+    "TERN_PRO_NONE", "TERN_PRO_BF16", "TERN_PRO_CAST", "TERN_PRO_RMSNORM", "TERN_PRO_SWIGLU",
     "tern_status_string",
 ]
 
@@ -32,6 +34,7 @@ TERN_ACT_BF16, TERN_ACT_INT8 = 0, 1
 TERN_SRC_INT8_TRITS, TERN_SRC_BASE3 = 0, 1
 TERN_FLAG_PDL = 1
 TERN_HEAD_NOALLOC_MAX_M = 16
+TERN_PRO_NONE, TERN_PRO_BF16, TERN_PRO_CAST, TERN_PRO_RMSNORM, TERN_PRO_SWIGLU = range(5)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libterngemv.so")
@@ -82,6 +85,10 @@ def lib() -> ctypes.CDLL:
             "tern_gemv_batch": ([vp, i32, i32, vp, sz, u32, vp], i32),
             "tern_gemm_batch_workspace_bytes": ([vp, i32, i32, i32], sz),
             "tern_gemm_batch": ([vp, i32, i32, i32, vp, sz, u32, vp], i32),
+            "tern_gemm_batch_pro": ([vp, vp, i32, i32, i32, vp, sz, u32, vp], i32),
+            "tern_act_prologue": ([vp, i32, i32, vp, vp], i32),
+            "i8_head_verify": ([vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+            "tern_verify_accept": ([vp, vp, i32, vp, vp], i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -113,6 +120,23 @@ def _stream(stream) -> int:
 class _Item(ctypes.Structure):
     _fields_ = [("W", _Matrix), ("x_dev", ctypes.c_void_p), ("x_scale_dev", ctypes.c_void_p),
                 ("y_dev", ctypes.c_void_p)]
+
+
+class _Prologue(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("eps", ctypes.c_float), ("src_dev", ctypes.c_void_p),
+                ("gain_dev", ctypes.c_void_p)]
+
+
+def _prologues(pros):
+    """pros: list of None or (kind, src tensor, gain tensor or None, eps)."""
+    arr = (_Prologue * len(pros))()
+    for i, pr in enumerate(pros):
+        if pr is None:
+            arr[i].kind = TERN_PRO_NONE
+            continue
+        kind, src, gain, eps = pr
+        arr[i].kind, arr[i].src_dev, arr[i].gain_dev, arr[i].eps = int(kind), _ptr(src), _ptr(gain), float(eps)
+    return arr
 
 
 class TernMatrix:
@@ -210,6 +234,19 @@ def i8_head_gemv_argmax_noalloc(W, scale_f16, V: int, K: int, M: int, act: int, 
            "i8_head_gemv_argmax_noalloc")
 
 
+def i8_head_verify(W, scale_f16, V: int, K: int, M: int, act: int, X, x_scale, draft, argmax, maxval, accept,
+                   workspace, stream=None) -> None:
+    """The head over the k + 1 = M verify rows plus the on-device acceptance count: accept[0] = accepted
+    drafts n, accept[1] = the target's token argmax[n]."""
+    _check(lib().i8_head_verify(_ptr(W), _ptr(scale_f16), V, K, M, act, _ptr(X), _ptr(x_scale), _ptr(draft),
+                                _ptr(argmax), _ptr(maxval), _ptr(accept), _ptr(workspace),
+                                int(workspace.numel() * workspace.element_size()), _stream(stream)), "i8_head_verify")
+
+
+def tern_verify_accept(argmax, draft, k: int, accept, stream=None) -> None:
+    _check(lib().tern_verify_accept(_ptr(argmax), _ptr(draft), k, _ptr(accept), _stream(stream)), "tern_verify_accept")
+
+
 def tern_read_flag(err_flag, stream=None) -> int:
     """Synchronise the stream and return TERN_OK or TERN_EBADCODE from a device error flag."""
     st = lib().tern_read_flag(_ptr(err_flag), _stream(stream))
@@ -259,20 +296,42 @@ def tern_gemm_batch(entries, M: int, act: int, workspace, flags: int = 0, stream
            "tern_gemm_batch")
 
 
+def tern_gemm_batch_pro(entries, prologues, M: int, act: int, workspace, flags: int = 0, stream=None) -> None:
+    """tern_gemm_batch with a prologue per entry: prologues[i] is None or (kind, src, gain, eps); for a
+    prologue entry, X is an optional output (or None) and x_scale (int8 mode) the output s_x."""
+    arr, pro = _items(entries), _prologues(prologues)
+    _check(lib().tern_gemm_batch_pro(arr, pro, len(entries), M, act, _ptr(workspace),
+                                     int(workspace.numel() * workspace.element_size()), flags, _stream(stream)),
+           "tern_gemm_batch_pro")
+
+
+def tern_act_prologue(kind: int, src, gain, eps: float, M: int, K: int, out, stream=None) -> None:
+    """The prologue alone: M rows of K bf16 activations (bit patterns) into out."""
+    pro = _prologues([(kind, src, gain, eps)])
+    _check(lib().tern_act_prologue(pro, M, K, _ptr(out), _stream(stream)), "tern_act_prologue")
+
+
 class GemvBatch:
     """A fixed list of GEMVs (M = 1) or small-M GEMMs with its descriptor array and workspace,
     launched repeatedly (e.g. inside a captured CUDA graph). entries: list of (TernMatrix, X,
-    x_scale or None, Y) with X [M][K] and Y [M][N]."""
+    x_scale or None, Y) with X [M][K] and Y [M][N]; prologues: optional list (one per entry) of
+    None or (kind, src, gain, eps), see tern_gemm_batch_pro."""
 
-    def __init__(self, entries, act: int, M: int = 1, device="cuda"):
+    def __init__(self, entries, act: int, M: int = 1, device="cuda", prologues=None):
         import torch
         self.entries, self.act, self.M = list(entries), act, int(M)
         self._arr = _items(self.entries)
+        self._pro = _prologues(prologues) if prologues is not None else None
         nbytes = int(lib().tern_gemm_batch_workspace_bytes(self._arr, len(self.entries), self.M, act))
         if nbytes == 0:
             raise TernError(TERN_ESHAPE, "tern_gemm_batch_workspace_bytes")
         self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
 
     def __call__(self, flags: int = 0, stream=None) -> None:
+        if self._pro is not None:
+            _check(lib().tern_gemm_batch_pro(self._arr, self._pro, len(self.entries), self.M, self.act,
+                                             _ptr(self.workspace), int(self.workspace.numel()), flags,
+                                             _stream(stream)), "tern_gemm_batch_pro")
+            return
         _check(lib().tern_gemm_batch(self._arr, len(self.entries), self.M, self.act, _ptr(self.workspace),
                                      int(self.workspace.numel()), flags, _stream(stream)), "tern_gemm_batch")

@@ -264,8 +264,10 @@ tern_status tern_gemv(const tern_matrix* W, tern_act act, const void* x_dev, con
 
 namespace {
 
-tern_status fill_batch(const tern_gemv_item* items, int32_t count, int32_t M, tern_act act,
-                       tern::BatchParams& bp, size_t& smem, size_t& ws) {
+// Validates a list (and its prologues, if any) and plans both launches. With check_ptrs false
+// only the shapes and modes are checked (the workspace query).
+tern_status fill_batch(const tern_gemv_item* items, const tern_prologue* pro, int32_t count, int32_t M, tern_act act,
+                       bool check_ptrs, tern::BatchParams& bp, tern::PrepParams& pp, size_t& smem, size_t& ws) {
   if (!items) return TERN_EINVAL;
   if (act != TERN_ACT_BF16 && act != TERN_ACT_INT8) return TERN_EINVAL;
   if (count < 1 || count > TERN_BATCH_MAX_ITEMS || M < 1 || M > 16) return TERN_ESHAPE;
@@ -275,32 +277,86 @@ tern_status fill_batch(const tern_gemv_item* items, int32_t count, int32_t M, te
   const uint32_t* planes[TERN_BATCH_MAX_ITEMS];
   for (int i = 0; i < count; ++i) {
     const tern_gemv_item& in = items[i];
-    tern_status st = check_matrix(&in.W);
-    if (st != TERN_OK) return st;
+    const int kind = pro ? pro[i].kind : TERN_PRO_NONE;
+    if (kind < TERN_PRO_NONE || kind > TERN_PRO_SWIGLU) return TERN_EINVAL;
+    if (check_ptrs) {
+      tern_status st = check_matrix(&in.W);
+      if (st != TERN_OK) return st;
+    } else if (!valid_shape(in.W.N, in.W.K)) {
+      return TERN_ESHAPE;
+    }
     if (in.W.K > 12288) return TERN_ESHAPE;
-    if (!in.x_dev || !in.y_dev || !aligned(in.x_dev, 16) || !aligned(in.y_dev, 4)) return TERN_EINVAL;
-    if (act == TERN_ACT_INT8 && (!in.x_scale_dev || !aligned(in.x_scale_dev, 4))) return TERN_EINVAL;
+    if (check_ptrs) {
+      if (!in.y_dev || !aligned(in.y_dev, 4)) return TERN_EINVAL;
+      if (kind == TERN_PRO_NONE) {
+        if (!in.x_dev || !aligned(in.x_dev, 16)) return TERN_EINVAL;
+        if (act == TERN_ACT_INT8 && (!in.x_scale_dev || !aligned(in.x_scale_dev, 4))) return TERN_EINVAL;
+      } else {
+        const tern_prologue& pr = pro[i];
+        if (!pr.src_dev || !aligned(pr.src_dev, 16)) return TERN_EINVAL;
+        if (kind == TERN_PRO_RMSNORM && (!pr.gain_dev || !aligned(pr.gain_dev, 16) || !(pr.eps >= 0.0f) ||
+                                         pr.eps > 3.0e38f))
+          return TERN_EINVAL;
+        if (in.x_dev && !aligned(in.x_dev, 16)) return TERN_EINVAL;       // optional copy of the activation
+        if (act == TERN_ACT_INT8 && (!in.x_scale_dev || !aligned(in.x_scale_dev, 4))) return TERN_EINVAL;
+      }
+    }
     tern::BatchItem& it = bp.items[i];
     planes[i] = in.W.planes;
     it.scale = in.W.scale_f16;
     it.y = in.y_dev;
-    it.x = in.x_dev;
     it.sx = in.x_scale_dev;
     it.N = in.W.N;
     it.K = in.W.K;
+    tern::PrepItem& q = pp.items[i];
+    q.kind = kind;
+    if (kind == TERN_PRO_NONE) {
+      q.x = in.x_dev;
+      q.gain = nullptr;
+      q.xout = nullptr;
+      q.sx_out = nullptr;
+      q.eps = 0.0f;
+    } else {
+      q.x = pro[i].src_dev;
+      q.gain = pro[i].gain_dev;
+      q.xout = const_cast<void*>(in.x_dev);
+      q.sx_out = const_cast<float*>(in.x_scale_dev);
+      q.eps = pro[i].eps;
+    }
   }
   if (!tern::plan_batch(bp, planes, smem, ws)) return TERN_ESHAPE;
   return TERN_OK;
+}
+
+tern_status run_batch(const tern_gemv_item* items, const tern_prologue* pro, int32_t count, int32_t M, tern_act act,
+                      void* workspace_dev, size_t workspace_bytes, uint32_t flags, tern_stream_t stream) {
+  if (flags & ~TERN_FLAG_PDL) return TERN_EINVAL;
+  if (!workspace_dev || !aligned(workspace_dev, 16)) return TERN_EINVAL;
+  tern::BatchParams* bp = new (std::nothrow) tern::BatchParams();
+  tern::PrepParams* pp = new (std::nothrow) tern::PrepParams();
+  tern_status st = (bp && pp) ? TERN_OK : TERN_EINVAL;
+  size_t smem = 0, ws = 0;
+  if (st == TERN_OK) st = fill_batch(items, pro, count, M, act, true, *bp, *pp, smem, ws);
+  if (st == TERN_OK && workspace_bytes < ws) st = TERN_EINVAL;
+  if (st == TERN_OK) {
+    bp->xprep = static_cast<uint8_t*>(workspace_dev);
+    tern::plan_prep(*bp, *pp);
+    st = from_cuda(tern::launch_batch(*bp, *pp, smem, (flags & TERN_FLAG_PDL) != 0, cs(stream)));
+  }
+  delete bp;
+  delete pp;
+  return st;
 }
 
 }  // namespace
 
 size_t tern_gemm_batch_workspace_bytes(const tern_gemv_item* items, int32_t count, int32_t M, tern_act act) {
   tern::BatchParams* bp = new (std::nothrow) tern::BatchParams();
-  if (!bp) return 0;
+  tern::PrepParams* pp = new (std::nothrow) tern::PrepParams();
   size_t smem = 0, ws = 0;
-  const tern_status st = fill_batch(items, count, M, act, *bp, smem, ws);
+  const tern_status st = (bp && pp) ? fill_batch(items, nullptr, count, M, act, false, *bp, *pp, smem, ws) : TERN_EINVAL;
   delete bp;
+  delete pp;
   return st == TERN_OK ? ws : 0;
 }
 
@@ -310,24 +366,32 @@ size_t tern_gemv_batch_workspace_bytes(const tern_gemv_item* items, int32_t coun
 
 tern_status tern_gemm_batch(const tern_gemv_item* items, int32_t count, int32_t M, tern_act act,
                             void* workspace_dev, size_t workspace_bytes, uint32_t flags, tern_stream_t stream) {
-  if (flags & ~TERN_FLAG_PDL) return TERN_EINVAL;
-  if (!workspace_dev || !aligned(workspace_dev, 16)) return TERN_EINVAL;
-  tern::BatchParams* bp = new (std::nothrow) tern::BatchParams();
-  if (!bp) return TERN_EINVAL;
-  size_t smem = 0, ws = 0;
-  tern_status st = fill_batch(items, count, M, act, *bp, smem, ws);
-  if (st == TERN_OK && workspace_bytes < ws) st = TERN_EINVAL;
-  if (st == TERN_OK) {
-    bp->xprep = static_cast<uint8_t*>(workspace_dev);
-    st = from_cuda(tern::launch_batch(*bp, smem, (flags & TERN_FLAG_PDL) != 0, cs(stream)));
-  }
-  delete bp;
-  return st;
+  return run_batch(items, nullptr, count, M, act, workspace_dev, workspace_bytes, flags, stream);
+}
+
+tern_status tern_gemm_batch_pro(const tern_gemv_item* items, const tern_prologue* prologues, int32_t count, int32_t M,
+                                tern_act act, void* workspace_dev, size_t workspace_bytes, uint32_t flags,
+                                tern_stream_t stream) {
+  if (!prologues) return TERN_EINVAL;
+  return run_batch(items, prologues, count, M, act, workspace_dev, workspace_bytes, flags, stream);
 }
 
 tern_status tern_gemv_batch(const tern_gemv_item* items, int32_t count, tern_act act, void* workspace_dev,
                             size_t workspace_bytes, uint32_t flags, tern_stream_t stream) {
   return tern_gemm_batch(items, count, 1, act, workspace_dev, workspace_bytes, flags, stream);
+}
+
+tern_status tern_act_prologue(const tern_prologue* pro, int32_t M, int32_t K, uint16_t* x_bf16_dev,
+                              tern_stream_t stream) {
+  if (!pro || !pro->src_dev || !x_bf16_dev) return TERN_EINVAL;
+  if (pro->kind < TERN_PRO_BF16 || pro->kind > TERN_PRO_SWIGLU) return TERN_EINVAL;
+  if (M < 1 || M > 65536 || !valid_shape(1, K)) return TERN_ESHAPE;
+  if (!aligned(pro->src_dev, 16) || !aligned(x_bf16_dev, 16)) return TERN_EINVAL;
+  if (pro->kind == TERN_PRO_RMSNORM &&
+      (!pro->gain_dev || !aligned(pro->gain_dev, 16) || !(pro->eps >= 0.0f) || pro->eps > 3.0e38f))
+    return TERN_EINVAL;
+  return from_cuda(tern::launch_prologue(pro->kind, pro->src_dev, pro->gain_dev, pro->eps, M, K, x_bf16_dev,
+                                         cs(stream)));
 }
 
 size_t i8_head_workspace_bytes(int32_t V, int32_t M) {
@@ -345,6 +409,29 @@ tern_status i8_head_gemv_argmax_ex(const int8_t* W_dev, const uint16_t* scale_f1
                                               maxval_dev, logits_dev, workspace_dev, workspace_bytes, flags, p);
   if (st != TERN_OK) return st;
   return from_cuda(tern::launch_head(p, (flags & TERN_FLAG_PDL) != 0, cs(stream)));
+}
+
+tern_status i8_head_verify(const int8_t* W_dev, const uint16_t* scale_f16_dev, int32_t V, int32_t K, int32_t M,
+                           tern_act act, const void* X_dev, const float* x_scale_dev, const int32_t* draft_dev,
+                           int32_t* argmax_dev, float* maxval_dev, int32_t* accept_dev, void* workspace_dev,
+                           size_t workspace_bytes, tern_stream_t stream) {
+  if (!accept_dev || !aligned(accept_dev, 4)) return TERN_EINVAL;
+  if (M > 1 && (!draft_dev || !aligned(draft_dev, 4))) return TERN_EINVAL;
+  tern::HeadParams p = {};
+  const tern_status st = tern::plan_head_call(W_dev, scale_f16_dev, V, K, M, act, X_dev, x_scale_dev, argmax_dev,
+                                              maxval_dev, nullptr, workspace_dev, workspace_bytes, 0u, p);
+  if (st != TERN_OK) return st;
+  p.draft = draft_dev;
+  p.accept = accept_dev;
+  return from_cuda(tern::launch_head(p, false, cs(stream)));
+}
+
+tern_status tern_verify_accept(const int32_t* argmax_dev, const int32_t* draft_dev, int32_t k, int32_t* accept_dev,
+                               tern_stream_t stream) {
+  if (!argmax_dev || !accept_dev || (k > 0 && !draft_dev)) return TERN_EINVAL;
+  if (!aligned(argmax_dev, 4) || !aligned(accept_dev, 4) || (draft_dev && !aligned(draft_dev, 4))) return TERN_EINVAL;
+  if (k < 0 || k > 65535) return TERN_ESHAPE;
+  return from_cuda(tern::launch_verify_accept(argmax_dev, draft_dev, k, accept_dev, cs(stream)));
 }
 
 tern_status i8_head_gemv_argmax(const int8_t* W_dev, const uint16_t* scale_f16_dev, int32_t V, int32_t K, int32_t M,

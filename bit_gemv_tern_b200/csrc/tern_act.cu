@@ -8,6 +8,7 @@
 
 #include "tern_device.cuh"
 #include "tern_kernels.h"
+#include "tern_prologue.cuh"
 
 namespace tern {
 namespace {
@@ -57,7 +58,30 @@ __global__ void __launch_bounds__(256) k_quantize(const uint16_t* __restrict__ x
   pdl_launch_dependents();
 }
 
+// One CTA per row: the prologue's bf16 row (tern_prologue.cuh), as the batched launch computes it
+// inside its operand preparation.
+constexpr int kProThreads = 256;
+__global__ void __launch_bounds__(kProThreads) k_prologue(int32_t kind, const void* src, const uint16_t* gain,
+                                                         float eps, int32_t K, uint16_t* out) {
+  __shared__ double red[kProThreads / 32];
+  const int64_t row = blockIdx.x;
+  const int64_t row_elems = (int64_t)K * (kind == kProSwiGLU ? 2 : 1);
+  const void* s = kind == kProBF16 ? static_cast<const void*>(static_cast<const uint16_t*>(src) + row * K)
+                                   : static_cast<const void*>(static_cast<const float*>(src) + row * row_elems);
+  pdl_wait();
+  const double r = kind == kProRMSNorm ? rmsnorm_r<kProThreads>(static_cast<const float*>(s), K, eps, red) : 1.0;
+  for (int k = threadIdx.x * 8; k < K; k += kProThreads * 8)
+    *reinterpret_cast<uint4*>(out + row * K + k) = prologue8(kind, s, gain, K, k, r);
+  pdl_launch_dependents();
+}
+
 }  // namespace
+
+cudaError_t launch_prologue(int32_t kind, const void* src, const uint16_t* gain, float eps, int32_t M, int32_t K,
+                            uint16_t* out, cudaStream_t st) {
+  k_prologue<<<M, kProThreads, 0, st>>>(kind, src, gain, eps, K, out);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_quantize(const uint16_t* x, int32_t M, int32_t K, int8_t* q, float* sx, cudaStream_t st) {
   k_quantize<<<M, 256, 0, st>>>(x, K, q, sx);

@@ -36,6 +36,7 @@
 
 #include "tern_device.cuh"
 #include "tern_kernels.h"
+#include "tern_prologue.cuh"
 
 namespace tern {
 
@@ -130,22 +131,29 @@ __host__ __device__ constexpr int seg_words(int mode, int mp) {
 
 // prep: one CTA of kPrepThreads per (item, token slot), wide enough that each pass over an
 // activation of up to 8192 (int8: 16384) elements is a single round of loads. Block layout: kp
-// segments of seg_bytes.
+// segments of seg_bytes. An item with a prologue first computes its bf16 row into shared memory
+// (tern_prologue.cuh), then encodes from there; int8 mode quantises that row per token here, so no
+// separate quantiser launch runs.
 constexpr int kPrepThreads = 1024;
-__global__ void __launch_bounds__(kPrepThreads) k_batch_prep(const __grid_constant__ BatchParams p) {
-  const BatchItem& it = p.items[blockIdx.x];
+constexpr int kPrepMaxK = 12288;
+__global__ void __launch_bounds__(kPrepThreads) k_batch_prep(const __grid_constant__ PrepParams p) {
+  const PrepItem& it = p.items[blockIdx.x];
   const int m = blockIdx.y;                          // token slot (< mp)
   uint32_t* blk = reinterpret_cast<uint32_t*>(p.xprep + it.xoff);
   const int K = it.K, KP = it.kp, mp = p.mp;
   const int ncols = seg_cols(p.mode, mp);
   const int segw = p.seg_bytes / 4;
   const int nl = p.mode == 0 ? kLimbs : 1;           // columns of this token
+  const bool pro = it.kind != kProNone;
   int colof[kLimbs];
   for (int l = 0; l < kLimbs; ++l) colof[l] = mp == 1 ? l : l * mp + m;
   const bool live = m < p.M;
   __shared__ float red[kPrepThreads / 32];
+  __shared__ double dred[kPrepThreads / 32];
   __shared__ int sums[kLimbs];
   __shared__ int Esh;
+  __shared__ float ssh;
+  __shared__ __align__(16) uint16_t xs[kPrepMaxK];  // a prologue item's prepared bf16 row
   pdl_wait();
   {
     // the split-block sums and counters of the stream start at zero
@@ -166,41 +174,78 @@ __global__ void __launch_bounds__(kPrepThreads) k_batch_prep(const __grid_consta
     }
   }
   if (threadIdx.x < kLimbs) sums[threadIdx.x] = 0;
-  if (threadIdx.x == 0) Esh = 0;
-  if (p.mode == 0 && live) {
-    const uint16_t* xb = static_cast<const uint16_t*>(it.x) + (size_t)m * K;
-    float amax = 0.0f;
-    for (int k = threadIdx.x * 8; k < K; k += blockDim.x * 8) {
-      const uint4 v = ld_nc(xb + k);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        amax = fmaxf(amax, fmaxf(fabsf(bf16_bits_to_float(w[e] & 0xFFFFu)), fabsf(bf16_bits_to_float(w[e] >> 16))));
+  if (threadIdx.x == 0) { Esh = 0; ssh = 0.0f; }
+  // the bf16 row of a prologue item, into shared memory (and the optional bf16 copy)
+  float amax = 0.0f;
+  if (live && pro) {
+    const size_t row_elems = (size_t)K * (it.kind == kProSwiGLU ? 2 : 1);
+    const void* src = it.kind == kProBF16 ? static_cast<const void*>(static_cast<const uint16_t*>(it.x) + (size_t)m * K)
+                                          : static_cast<const void*>(static_cast<const float*>(it.x) + (size_t)m * row_elems);
+    const double r = it.kind == kProRMSNorm ? rmsnorm_r<kPrepThreads>(static_cast<const float*>(src), K, it.eps, dred) : 1.0;
+    uint16_t* xo = (p.mode == 0 && it.xout) ? static_cast<uint16_t*>(it.xout) + (size_t)m * K : nullptr;
+    for (int k = threadIdx.x * 8; k < K; k += kPrepThreads * 8) {
+      const uint4 v = prologue8(it.kind, src, it.gain, K, k, r);
+      *reinterpret_cast<uint4*>(xs + k) = v;
+      if (xo) *reinterpret_cast<uint4*>(xo + k) = v;
+      amax = fmaxf(amax, absmax8(v));
     }
+  } else if (live && p.mode == 0) {
+    const uint16_t* xb = static_cast<const uint16_t*>(it.x) + (size_t)m * K;
+    for (int k = threadIdx.x * 8; k < K; k += kPrepThreads * 8) amax = fmaxf(amax, absmax8(ld_nc(xb + k)));
+  }
+  if (live && (p.mode == 0 || pro)) {
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
     __syncthreads();
     if (threadIdx.x == 0) {
       float mx = red[0];
       for (int i = 1; i < kPrepThreads / 32; ++i) mx = fmaxf(mx, red[i]);
-      Esh = limb_exponent(mx);
+      if (p.mode == 0) {
+        Esh = limb_exponent(mx);
+      } else {
+        const float sx = __fdiv_rn(mx, 127.0f);     // the per-token quantiser's scale
+        ssh = sx;
+        it.sx_out[m] = sx;
+      }
     }
   }
   __syncthreads();
   const int E = Esh;
+  const float sq = ssh;
+  int8_t* qo = (p.mode == 1 && pro && it.xout) ? static_cast<int8_t*>(it.xout) + (size_t)m * K : nullptr;
   // one 16-element half of a 32-trit word per thread iteration
   int ls[kLimbs] = {0, 0, 0, 0};
   for (int v = threadIdx.x; live && v < K / 16; v += blockDim.x) {
     const int word = v >> 1, h = v & 1;              // global word index and half
     const int part = word >> 4, w = word & 15;
     uint32_t* seg = blk + part * segw + part_slot(w);
+    uint4 a, b;                                      // 16 bf16 values of this half (bf16 sources)
+    if (pro) {
+      a = *reinterpret_cast<const uint4*>(xs + 16 * v);
+      b = *reinterpret_cast<const uint4*>(xs + 16 * v + 8);
+    } else if (p.mode == 0) {
+      const uint16_t* xb = static_cast<const uint16_t*>(it.x) + (size_t)m * K + 16 * v;
+      a = ld_nc(xb);
+      b = ld_nc(xb + 8);
+    }
     if (p.mode == 1) {
-      const uint4 q = ld_nc(static_cast<const int8_t*>(it.x) + (size_t)m * K + 16 * v);
+      uint4 q;
+      if (pro) {
+        const uint32_t wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        uint32_t qw[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const uint32_t bits = (e & 1) ? (wv[e >> 1] >> 16) : (wv[e >> 1] & 0xFFFFu);
+          qw[e >> 2] |= (uint32_t)(uint8_t)(int8_t)quant_i8(bf16_bits_to_float(bits), sq) << (8 * (e & 3));
+        }
+        q = make_uint4(qw[0], qw[1], qw[2], qw[3]);
+        if (qo) *reinterpret_cast<uint4*>(qo + 16 * v) = q;
+      } else {
+        q = ld_nc(static_cast<const int8_t*>(it.x) + (size_t)m * K + 16 * v);
+      }
       ls[0] += bsum(q.x) + bsum(q.y) + bsum(q.z) + bsum(q.w);
       store_operand_half(seg + colof[0] * kColWords, h, permute_i8_half(q));
     } else {
-      const uint16_t* xb = static_cast<const uint16_t*>(it.x) + (size_t)m * K + 16 * v;
-      const uint4 a = ld_nc(xb), b = ld_nc(xb + 8);
       const uint32_t wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
       uint32_t l[kLimbs][4] = {};
 #pragma unroll
@@ -835,7 +880,23 @@ cudaError_t read_and_clear_batch_latch(int* out) {
   return cudaMemcpyToSymbol(g_batch_latch, &zero, sizeof(int));
 }
 
-cudaError_t launch_batch(const BatchParams& p, size_t smem, bool pdl, cudaStream_t st) {
+void plan_prep(const BatchParams& b, PrepParams& q) {
+  q.count = b.count;
+  q.mode = b.mode;
+  q.M = b.M;
+  q.mp = b.mp;
+  q.seg_bytes = b.seg_bytes;
+  q.xprep = b.xprep;
+  q.scratch_off = b.scratch_off;
+  q.scratch_words = b.scratch_words;
+  for (int i = 0; i < b.count; ++i) {
+    q.items[i].K = b.items[i].K;
+    q.items[i].kp = b.items[i].kp;
+    q.items[i].xoff = b.items[i].xoff;
+  }
+}
+
+cudaError_t launch_batch(const BatchParams& p, const PrepParams& q, size_t smem, bool pdl, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   int na = 0;
@@ -851,7 +912,7 @@ cudaError_t launch_batch(const BatchParams& p, size_t smem, bool pdl, cudaStream
   cfg.gridDim = dim3(p.count, p.mp, 1);
   cfg.blockDim = dim3(kPrepThreads, 1, 1);
   cfg.dynamicSmemBytes = 0;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, k_batch_prep, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, k_batch_prep, q);
   if (e != cudaSuccess) return e;
   // 2. the stream (always programmatically dependent on the prep launch)
   cudaLaunchAttribute attr2[1];

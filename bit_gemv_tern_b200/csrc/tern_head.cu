@@ -215,10 +215,34 @@ __global__ void __launch_bounds__(kThreads, 2) k_head(const HeadParams p) {
     __threadfence();
     if (threadIdx.x < p.M) {
       const unsigned long long key = atomicExch(&p.keys[threadIdx.x], 0ull);
-      p.argmax[threadIdx.x] = (int32_t)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull));
+      const int32_t idx = (int32_t)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull));
+      p.argmax[threadIdx.x] = idx;
       p.maxval[threadIdx.x] = float_from_order_key((uint32_t)(key >> 32));
+      expo[threadIdx.x] = idx;                       // the winners, for the verify round below
     }
     if (threadIdx.x == 0) atomicExch(p.counter, 0u);
+    if (p.accept) {
+      // verify round: the longest prefix of drafts equal to the greedy tokens, then the target's
+      // own next token (PyTorchKR review, section "검증된 추측 디코딩")
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        int n = 0;
+        while (n < p.M - 1 && p.draft[n] == expo[n]) ++n;
+        p.accept[0] = n;
+        p.accept[1] = expo[n];
+      }
+    }
+  }
+}
+
+// The acceptance rule alone, on argmax indices already on the device (one thread).
+__global__ void k_verify_accept(const int32_t* argmax, const int32_t* draft, int32_t k, int32_t* accept) {
+  pdl_wait();
+  if (threadIdx.x == 0) {
+    int n = 0;
+    while (n < k && draft[n] == argmax[n]) ++n;
+    accept[0] = n;
+    accept[1] = argmax[n];
   }
 }
 
@@ -269,6 +293,12 @@ cudaError_t launch_mode(const HeadParams& p, int ng, size_t smem, bool pdl, cuda
 }  // namespace
 
 size_t head_workspace_bytes(int M) { return 16 + 8 * (size_t)M; }
+
+cudaError_t launch_verify_accept(const int32_t* argmax, const int32_t* draft, int32_t k, int32_t* accept,
+                                 cudaStream_t st) {
+  k_verify_accept<<<1, 32, 0, st>>>(argmax, draft, k, accept);
+  return cudaGetLastError();
+}
 
 size_t head_smem_bytes(int mode, int M, int kr) {
   const int ncols = mode == 0 ? 4 * M : M;

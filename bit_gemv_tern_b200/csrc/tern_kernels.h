@@ -100,8 +100,7 @@ cudaError_t read_and_clear_error_latch(int* out, cudaStream_t st);
 struct BatchItem {
   const uint16_t* scale;
   float* y;               // [M][N]
-  const void* x;          // bf16 bits [M][K] or int8 [M][K]
-  const float* sx;        // int8 mode: [M]
+  const float* sx;        // int8 mode: s_x [M] (written by the prep launch for prologue items)
   int32_t N, K;
   int32_t kp;             // 512-trit K parts (the last may be partial): stages per row block
   int32_t unit0;          // first global unit (row block) of the item
@@ -137,9 +136,33 @@ struct BatchParams {
   int32_t scratch_words;  // words to zero before the stream (sums and counters)
 };
 static_assert(sizeof(BatchParams) <= 32764, "kernel parameter limit");
+// The operand preparation of one item (the prep launch): where its activation comes from and the
+// prologue that turns it into the linear's bf16 (or int8) activation (tern_prologue.cuh).
+struct PrepItem {
+  const void* x;          // kProNone: bf16 [M][K] (bf16 mode) or int8 q [M][K]; kProBF16: bf16 [M][K];
+                          // kProCast, kProRMSNorm: fp32 [M][K]; kProSwiGLU: fp32 [M][2K] (gate | up)
+  const uint16_t* gain;   // kProRMSNorm: bf16 [K]
+  void* xout;             // prologue items, optional: the prepared activation (bf16, or int8 q) [M][K]
+  float* sx_out;          // prologue items in int8 mode: s_x [M]
+  float eps;              // kProRMSNorm
+  int32_t kind;           // kProNone .. kProSwiGLU
+  int32_t K, kp;
+  uint32_t xoff;          // byte offset of the item's operand block in the workspace
+};
+struct PrepParams {
+  PrepItem items[kBatchMaxItems];
+  int32_t count, mode, M, mp, seg_bytes;
+  uint8_t* xprep;
+  uint32_t scratch_off;
+  int32_t scratch_words;
+};
+static_assert(sizeof(PrepParams) <= 32764, "kernel parameter limit");
 // Host: fills tmap/kp/units/xoff, the stage ring and the CTA split; fails on unsupported shapes.
 bool plan_batch(BatchParams& p, const uint32_t* const* planes, size_t& smem, size_t& workspace);
-cudaError_t launch_batch(const BatchParams& p, size_t smem, bool pdl, cudaStream_t st);
+// Copies the plan's per-item fields (K, kp, xoff, mode, workspace layout) into the prep parameters,
+// whose activation sources and prologues the caller has filled.
+void plan_prep(const BatchParams& b, PrepParams& q);
+cudaError_t launch_batch(const BatchParams& p, const PrepParams& q, size_t smem, bool pdl, cudaStream_t st);
 cudaError_t read_and_clear_batch_latch(int* out);
 
 // Prefill dense contraction on tcgen05 (tern_prefill.cu).
@@ -169,6 +192,8 @@ struct HeadParams {
   float* logits;          // optional [M][V]
   unsigned long long* keys;  // workspace: M packed (value key, index) maxima
   unsigned int* counter;     // workspace: CTAs finished
+  const int32_t* draft;      // verify round, optional: M - 1 drafted tokens
+  int32_t* accept;           // verify round: {accepted drafts n, next token argmax[n]}
   int32_t kr, ksplit;
   int32_t nrb;            // row blocks of 128 rows
   int32_t nby;            // CTAs along the row-block axis (persistent loop)
@@ -176,6 +201,8 @@ struct HeadParams {
 size_t head_workspace_bytes(int M);
 size_t head_smem_bytes(int mode, int M, int kr);
 cudaError_t launch_head(const HeadParams& p, bool pdl, cudaStream_t st);
+cudaError_t launch_verify_accept(const int32_t* argmax, const int32_t* draft, int32_t k, int32_t* accept,
+                                 cudaStream_t st);
 // Every argument check of i8_head_gemv_argmax_ex and its launch plan (tern_abi.cu); enqueues nothing.
 tern_status plan_head_call(const int8_t* W_dev, const uint16_t* scale_f16_dev, int32_t V, int32_t K, int32_t M,
                            tern_act act, const void* X_dev, const float* x_scale_dev, int32_t* argmax_dev,
@@ -210,7 +237,9 @@ cudaError_t launch_encode_base3(const int8_t* src, int32_t N, int32_t K, uint8_t
                                 cudaStream_t st);
 cudaError_t launch_occupancy(const uint32_t* planes, int32_t N, int32_t K, int64_t* counts, cudaStream_t st);
 
-// Activation quantiser (tern_act.cu).
+// Activation quantiser and standalone prologue (tern_act.cu).
 cudaError_t launch_quantize(const uint16_t* x, int32_t M, int32_t K, int8_t* q, float* sx, cudaStream_t st);
+cudaError_t launch_prologue(int32_t kind, const void* src, const uint16_t* gain, float eps, int32_t M, int32_t K,
+                            uint16_t* out, cudaStream_t st);
 
 }  // namespace tern

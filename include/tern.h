@@ -45,8 +45,9 @@
  *   - tern_pack takes no scale argument: the per-row fp16 scales stay a separate caller array
  *     that a tern_matrix points to; packing would only copy it.
  *   - The launch flags of the *_ex entry points, the batched entry points (tern_pack_batch,
- *     tern_gemv_batch, tern_gemm_batch), tern_base3_encode, tern_occupancy, tern_quantize_act and
- *     i8_head_gemv_argmax_noalloc are additions.
+ *     tern_gemv_batch, tern_gemm_batch), tern_base3_encode, tern_occupancy, tern_quantize_act,
+ *     the prologues (tern_gemm_batch_pro, tern_act_prologue), the verify round (i8_head_verify,
+ *     tern_verify_accept) and i8_head_gemv_argmax_noalloc are additions.
  *
  * Packed layout (this library's own; the pages' FV5 bit-planes are only partly described)
  *   Matrix N x K, K a multiple of 128. Row n occupies K/16 uint32 words at word offset n*K/16:
@@ -213,6 +214,7 @@ tern_status tern_gemv_batch(const tern_gemv_item* items, int32_t count, tern_act
 
 /* Workspace bytes tern_gemm_batch needs for these items and M activation rows (0 if invalid). */
 size_t tern_gemm_batch_workspace_bytes(const tern_gemv_item* items, int32_t count, int32_t M, tern_act act);
+/* (Only the items' shapes are read: activation and output pointers may be NULL in this query.) */
 
 /* tern_gemv_batch for M activation rows per item (the draft-verify pass of speculative decoding
  * over a whole layer list, [R] "검증된 추측 디코딩"): for every item,
@@ -223,6 +225,47 @@ size_t tern_gemm_batch_workspace_bytes(const tern_gemv_item* items, int32_t coun
  * call equals this one with M = 1). */
 tern_status tern_gemm_batch(const tern_gemv_item* items, int32_t count, int32_t M, tern_act act,
                             void* workspace_dev, size_t workspace_bytes, uint32_t flags, tern_stream_t stream);
+
+/* Activation prologues: the step before a linear in the Qwen3 block of the Neutrino-1 models
+ * ([R] "세 모델과 하나의 컨테이너", model table: RMSNorm before q|k|v and gate|up, SwiGLU before
+ * down), computed where the linear's operands are prepared, so it costs no launch of its own. Each
+ * kind turns source rows into the bf16 activation the linear consumes, in fp64 with one rounding
+ * to nearest (ties to even) to bf16:
+ *   TERN_PRO_BF16:    x = the bf16 source row as given (int8 mode then quantises it in place of a
+ *                     tern_quantize_act launch)
+ *   TERN_PRO_CAST:    x_k = bf16(s_k) of an fp32 row
+ *   TERN_PRO_RMSNORM: x_k = bf16((s_k * r) * gain_k), r = 1 / sqrt(sum_k s_k^2 / K + eps)
+ *   TERN_PRO_SWIGLU:  x_k = bf16(silu(s_k) * s_(K+k)), silu(z) = z / (1 + e^-z), of a gate|up row of
+ *                     2K fp32 values (gate first, as tern_gemm_batch writes a fused gate|up output)
+ * In int8 mode the bf16 row is then quantised exactly as tern_quantize_act does. */
+typedef enum {
+  TERN_PRO_NONE = 0, TERN_PRO_BF16 = 1, TERN_PRO_CAST = 2, TERN_PRO_RMSNORM = 3, TERN_PRO_SWIGLU = 4
+} tern_prologue_kind;
+
+typedef struct {
+  int32_t kind;               /* tern_prologue_kind                                              */
+  float eps;                  /* TERN_PRO_RMSNORM: added to the mean square, finite and >= 0     */
+  const void* src_dev;        /* source rows, 16-byte aligned: bf16 [M][K] (BF16), fp32 [M][K]
+                                 (CAST, RMSNORM) or fp32 [M][2K] (SWIGLU)                         */
+  const uint16_t* gain_dev;   /* TERN_PRO_RMSNORM: bf16 [K] gains, 16-byte aligned               */
+} tern_prologue;
+
+/* tern_gemm_batch with a prologue per item: prologues[i] (host array of `count`) prepares item i's
+ * activation from its source rows inside the batch's operand-preparation launch. For an item with
+ * kind TERN_PRO_NONE the item is read as for tern_gemm_batch. For any other kind:
+ *   x_dev        optional output (NULL to skip): the prepared activation, bf16 [M][K] (bf16 mode)
+ *                or the quantised int8 q [M][K] (int8 mode), 16-byte aligned;
+ *   x_scale_dev  int8 mode, required output: s_x [M] of the per-token quantiser.
+ * Results are bit-identical to tern_act_prologue, then (int8 mode) tern_quantize_act, then
+ * tern_gemm_batch on the prepared rows. Workspace: tern_gemm_batch_workspace_bytes of the items. */
+tern_status tern_gemm_batch_pro(const tern_gemv_item* items, const tern_prologue* prologues, int32_t count,
+                                int32_t M, tern_act act, void* workspace_dev, size_t workspace_bytes,
+                                uint32_t flags, tern_stream_t stream);
+
+/* The prologue alone: M rows of K (K % 128 == 0) bf16 activations into x_bf16_dev [M][K]
+ * (16-byte aligned). Kind TERN_PRO_NONE is invalid here. */
+tern_status tern_act_prologue(const tern_prologue* pro, int32_t M, int32_t K, uint16_t* x_bf16_dev,
+                              tern_stream_t stream);
 
 /* Small-M GEMM for the draft-verify pass of speculative decoding ([R] "검증된 추측 디코딩": the
  * 8B scores up to seven drafted positions in one batched forward pass):
@@ -268,6 +311,25 @@ tern_status i8_head_gemv_argmax_ex(const int8_t* W_dev, const uint16_t* scale_f1
                                    const float* x_scale_dev, int32_t* argmax_dev, float* maxval_dev,
                                    float* logits_dev, void* workspace_dev, size_t workspace_bytes,
                                    uint32_t flags, tern_stream_t stream);
+
+/* The verify round of speculative decoding on the device ([R] "검증된 추측 디코딩: 속도만 바꾸고
+ * 답은 바꾸지 않는다": the target scores the drafted positions in one batched pass and keeps the
+ * longest prefix of drafts that equal its own greedy tokens). i8_head_gemv_argmax over the
+ * M = k + 1 activation rows of the verify pass (row j: the position after which draft[j] was
+ * proposed; row k: after the last draft), then, in the same launch, the acceptance count:
+ *   n = the largest j <= k with draft[i] == argmax[i] for every i < j,
+ *   accept_dev[0] = n, accept_dev[1] = argmax[n]   (the round yields n + 1 tokens)
+ * draft_dev: int32 [M - 1] (may be NULL when M = 1); accept_dev: int32 [2]. Other arguments as
+ * for i8_head_gemv_argmax (no logits output, no flags). */
+tern_status i8_head_verify(const int8_t* W_dev, const uint16_t* scale_f16_dev, int32_t V, int32_t K, int32_t M,
+                           tern_act act, const void* X_dev, const float* x_scale_dev, const int32_t* draft_dev,
+                           int32_t* argmax_dev, float* maxval_dev, int32_t* accept_dev, void* workspace_dev,
+                           size_t workspace_bytes, tern_stream_t stream);
+
+/* The acceptance rule alone on k + 1 argmax indices already on the device (argmax_dev int32
+ * [k + 1], draft_dev int32 [k], accept_dev int32 [2] as above; 0 <= k <= 65535). */
+tern_status tern_verify_accept(const int32_t* argmax_dev, const int32_t* draft_dev, int32_t k, int32_t* accept_dev,
+                               tern_stream_t stream);
 
 /* No-allocation variant of i8_head_gemv_argmax. The source pages describe no counterpart: it is
  * an interface convenience of this library. Same arguments, results and error codes as

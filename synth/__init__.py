@@ -149,6 +149,18 @@ def activations(seed: int, tid: int, M: int, K: int) -> np.ndarray:
     return f32_to_bf16_bits(z.astype(np.float32)).reshape(M, K)
 
 
+def norm_gains(seed: int, tid: int, K: int) -> np.ndarray:
+    """bf16 bit patterns uint16[K] of RMSNorm gains: 1 + N(0,1) / 8, drawn from the activation
+    stream family with tensor ids of their own (the pages give no gain statistics)."""
+    z = bf16_bits_to_f32(activations(seed, 1_000_000 + tid, 1, K)[0]).astype(np.float64)
+    return f32_to_bf16_bits((1.0 + z / 8.0).astype(np.float32))
+
+
+def residual(seed: int, tid: int, M: int, K: int) -> np.ndarray:
+    """fp32 [M, K] rows of N(0,1) draws: the residual stream entering a decode chain."""
+    return bf16_bits_to_f32(activations(seed, 2_000_000 + tid, M, K)).astype(np.float32)
+
+
 def head_weights(seed: int, tid: int, V: int, K: int, rows: np.ndarray | None = None,
                  chunk_rows: int = 4096) -> np.ndarray:
     """int8[V or len(rows), K] uniform in [-127, 127]: (u mod 255) - 127."""

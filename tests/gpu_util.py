@@ -49,18 +49,20 @@ def make_matrix(seed: int, tid: int, N: int, K: int, p=synth.P_DEFAULT, host_tri
 
 
 def check_bf16(y: np.ndarray, y_ref: np.ndarray, x_bf16: np.ndarray, scale_f16: np.ndarray,
-               rel_l2: bool = True) -> None:
+               rel_l2=True) -> None:
     """y, y_ref: [M, N]; x_bf16: [M, K] bits; scale_f16: [N] bits (or for sampled rows, the rows' scales).
-    rel_l2=False checks only the per-output bound: for inputs whose every output is made of
-    activations far below the absmax (a single nonzero weight per row against sub-grid values), the
-    relative L2 error is not bounded by any fixed-precision arithmetic, while the per-output bound
-    still holds for every input."""
+    The per-output bound is always checked. rel_l2: True checks relative L2 <= 1e-5; a float checks
+    it against that limit instead; False skips it (for inputs whose every output is made of
+    activations far below the absmax -- a single nonzero weight per row against sub-grid values --
+    the relative L2 error is not bounded by any fixed-precision arithmetic, while the per-output
+    bound still holds for every input)."""
     y = np.asarray(y, np.float64)
     err = y - y_ref
-    rel = np.linalg.norm(err) / max(np.linalg.norm(y_ref), 1e-300)
-    if rel_l2:
-        assert rel <= REL_L2, f"rel-L2 {rel:.3e} > {REL_L2}"
     absx = np.abs(synth.bf16_bits_to_f32(x_bf16).astype(np.float64)).sum(1)       # [M]
     sc = scale_f16.view(np.float16).astype(np.float64)                             # [N]
     bound = PER_OUT * absx[:, None] * sc[None, :]
     assert (np.abs(err) <= bound).all(), f"max |err|/bound = {(np.abs(err) / bound).max():.3e}"
+    rel = np.linalg.norm(err) / max(np.linalg.norm(y_ref), 1e-300)
+    if rel_l2 is not False:
+        limit = REL_L2 if rel_l2 is True else float(rel_l2)
+        assert rel <= limit, f"rel-L2 {rel:.3e} > {limit} (max |err|/bound {(np.abs(err) / bound).max():.3e})"
