@@ -40,6 +40,9 @@ def lib() -> ctypes.CDLL:
         L.orc_rmsnorm.argtypes = [vp, i32, i32, vp, ctypes.c_double, vp]; L.orc_rmsnorm.restype = None
         L.orc_swiglu.argtypes = [vp, i32, i32, vp]; L.orc_swiglu.restype = None
         L.orc_verify_accept.argtypes = [vp, vp, i32, vp, vp]; L.orc_verify_accept.restype = None
+        L.orc_rans_freqs.argtypes = [vp, i64, vp]; L.orc_rans_freqs.restype = None
+        L.orc_rans_encode.argtypes = [vp, i32, i32, vp, vp, vp, i64]; L.orc_rans_encode.restype = i64
+        L.orc_rans_decode.argtypes = [vp, vp, i32, i32, vp, vp]; L.orc_rans_decode.restype = i32
         _LIB = L
     return _LIB
 
@@ -230,3 +233,34 @@ def verify_accept(argmax, draft) -> tuple[int, int]:
     nt = np.zeros(1, np.int32)
     lib().orc_verify_accept(_p(am), _p(dr) if k else _p(np.zeros(1, np.int32)), k, _p(n), _p(nt))
     return int(n[0]), int(nt[0])
+
+
+def rans_freqs(trits: np.ndarray) -> np.ndarray:
+    """Quantised frequencies (uint16[3], order t = 0, +1, -1, sum 4096) of a tensor's trits."""
+    t = _c(trits, np.int8).reshape(-1)
+    f = np.empty(3, np.uint16)
+    lib().orc_rans_freqs(_p(t), t.size, _p(f))
+    return f
+
+
+def rans_encode(trits: np.ndarray, freq: np.ndarray | None = None):
+    """Order-0 rANS transport of an int8 [N, K] trit tensor: (freq uint16[3], row_end uint32[N],
+    payload uint8[...]). freq defaults to the tensor's own quantised frequencies."""
+    t = _c(trits, np.int8)
+    N, K = t.shape
+    f = rans_freqs(t) if freq is None else _c(freq, np.uint16)
+    row_end = np.empty(N, np.uint32)
+    cap = N * (2 * K + 8)
+    out = np.empty(cap, np.uint8)
+    n = lib().orc_rans_encode(_p(t), N, K, _p(f), _p(row_end), _p(out), cap)
+    if n < 0:
+        raise OracleError("rans_encode: not a trit tensor")
+    return f, row_end, out[:n].copy()
+
+
+def rans_decode(freq: np.ndarray, row_end: np.ndarray, payload: np.ndarray, N: int, K: int):
+    """(trits int8[N, K], ok): ok is False if any row's stream is invalid."""
+    t = np.empty((N, K), np.int8)
+    st = lib().orc_rans_decode(_p(_c(payload, np.uint8)), _p(_c(row_end, np.uint32)), N, K,
+                               _p(_c(freq, np.uint16)), _p(t))
+    return t, st == 0
