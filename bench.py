@@ -34,9 +34,10 @@ sys.path.insert(0, ROOT)
 
 METRIC = "ternary GEMV HBM GB/s & 8B linear-stack tok/s at M=1 (fraction of HBM peak)"
 # DRAM bytes (read + write) of the stream kernel per full 8B step, from an ncu capture of the
-# 4-layer profile case (batch-8b-4layers-bf16) scaled by the units processed (36 / 4 layers).
-# None whenever that kernel has changed since the counters were taken.
-STREAM_TRAFFIC_PER_STEP = None
+# 4-layer profile case (batch-8b-4layers-bf16: 203.27 MB read + 6.39 MB written) scaled by the
+# units processed (36 / 4 layers). None whenever that kernel has changed since the counters were
+# taken.
+STREAM_TRAFFIC_PER_STEP = 9 * (203.27e6 + 6.39e6)
 SEED = 0x7E2A2026
 L2_BYTES = 126 * 1024 * 1024
 
@@ -741,6 +742,8 @@ def extra_rows(stack, torch, tg, hbm_peak, bf16_peak):
 
     # base-3 transport unpack of all 8B trits (bit-exact expansion into the planes)
     out["base3_unpack_8b"] = base3_row(stack, torch, tg, hbm_peak)
+    # order-0 rANS transport of all 8B trits: decode into the planes in one launch
+    out["rans_decode_8b"] = rans_row(torch, tg, hbm_peak)
     return out
 
 
@@ -984,6 +987,48 @@ def base3_row(stack, torch, tg, hbm_peak):
     out = {"ms": ms, "gbs": nb / (ms / 1000.0) / 1e9, "frac": nb / (ms / 1000.0) / 1e9 / hbm_peak,
            "trits": trits, "bytes": nb, "tensors": len(items), "launches": 1}
     del items
+    return out
+
+
+def rans_row(torch, tg, hbm_peak):
+    """All 252 ternary tensors of the 8B coded by the device encoder (order-0 rANS, one stream per
+    row), then decoded into their planes by one tern_rans_decode call (one launch). Bytes = payload
+    + row ends read, planes written."""
+    import synth
+    import synth.cuda as sc
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    L = synth.GEOMETRY["8b"]["layers"]
+    shapes = synth.linear_shapes("8b")
+    Nmax = max(N for _, N, _ in shapes)
+    Kmax = max(K for _, _, K in shapes)
+    bound = max(tg.tern_rans_payload_bound(N, K) for _, N, K in shapes)
+    ws = torch.empty(max(tg.tern_rans_workspace_bytes(N, K) for _, N, K in shapes), dtype=torch.uint8, device="cuda")
+    buf = torch.empty(bound, dtype=torch.uint8, device="cuda")
+    t = torch.empty(Nmax * Kmax, dtype=torch.int8, device="cuda")
+    entries, payload_bytes, trits = [], 0, 0
+    for layer in range(L):
+        for p, N, K in shapes:
+            sc.trits_into(t[:N * K], SEED, synth.tensor_id(layer, p), K, synth.trit_probs("8b", layer, p))
+            freq = torch.empty(3, dtype=torch.int16, device="cuda")
+            row_end = torch.empty(N, dtype=torch.int32, device="cuda")
+            tg.tern_rans_encode(t[:N * K], N, K, freq, row_end, buf, ws, flag)
+            assert tg.tern_read_flag(flag) == 0
+            n = int(row_end[-1].item()) & 0xFFFFFFFF
+            payload = buf[:n].clone()
+            entries.append((freq, row_end, payload, N, K, torch.empty(N * K // 16, dtype=torch.int32, device="cuda")))
+            payload_bytes += n + 4 * N
+            trits += N * K
+    del t, ws, buf
+    g = capture(lambda i: tg.tern_rans_decode(entries, flag), 1)
+    g.replay()
+    reps = 3
+    ms = timed_replays([(g, reps)]) / reps
+    assert tg.tern_read_flag(flag) == 0
+    nb = payload_bytes + trits // 4
+    out = {"ms": ms, "gbs": nb / (ms / 1000.0) / 1e9, "frac": nb / (ms / 1000.0) / 1e9 / hbm_peak,
+           "trits": trits, "transport_bytes": payload_bytes, "bits_per_trit": 8.0 * payload_bytes / trits,
+           "tensors": len(entries), "launches": 1}
+    del entries
     return out
 
 

@@ -25,6 +25,7 @@ __all__ = [
     "GemvBatch", "tern_gemv_batch", "tern_gemv_batch_workspace_bytes", "tern_gemm_batch",
     "tern_gemm_batch_workspace_bytes", "tern_gemm_batch_pro", "tern_act_prologue",
     "i8_head_verify", "tern_verify_accept",
+    "tern_rans_payload_bound", "tern_rans_workspace_bytes", "tern_rans_encode", "tern_rans_decode",
     "TERN_PRO_NONE", "TERN_PRO_BF16", "TERN_PRO_CAST", "TERN_PRO_RMSNORM", "TERN_PRO_SWIGLU",
     "tern_status_string",
 ]
@@ -89,6 +90,10 @@ def lib() -> ctypes.CDLL:
             "tern_act_prologue": ([vp, i32, i32, vp, vp], i32),
             "i8_head_verify": ([vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
             "tern_verify_accept": ([vp, vp, i32, vp, vp], i32),
+            "tern_rans_payload_bound": ([i32, i32], sz),
+            "tern_rans_workspace_bytes": ([i32, i32], sz),
+            "tern_rans_encode": ([vp, i32, i32, vp, vp, vp, sz, vp, sz, vp, vp], i32),
+            "tern_rans_decode": ([vp, i32, vp, vp], i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -245,6 +250,38 @@ def i8_head_verify(W, scale_f16, V: int, K: int, M: int, act: int, X, x_scale, d
 
 def tern_verify_accept(argmax, draft, k: int, accept, stream=None) -> None:
     _check(lib().tern_verify_accept(_ptr(argmax), _ptr(draft), k, _ptr(accept), _stream(stream)), "tern_verify_accept")
+
+
+class _RansItem(ctypes.Structure):
+    _fields_ = [("freq_dev", ctypes.c_void_p), ("row_end_dev", ctypes.c_void_p), ("payload_dev", ctypes.c_void_p),
+                ("payload_bytes", ctypes.c_size_t), ("N", ctypes.c_int32), ("K", ctypes.c_int32),
+                ("planes_dev", ctypes.c_void_p)]
+
+
+def tern_rans_payload_bound(N: int, K: int) -> int:
+    return int(lib().tern_rans_payload_bound(N, K))
+
+
+def tern_rans_workspace_bytes(N: int, K: int) -> int:
+    return int(lib().tern_rans_workspace_bytes(N, K))
+
+
+def tern_rans_encode(trits, N: int, K: int, freq, row_end, payload, workspace, err_flag, stream=None) -> None:
+    """int8 trits [N*K] -> order-0 rANS transport: freq (3 x int16), row_end (N x int32), payload (uint8)."""
+    _check(lib().tern_rans_encode(_ptr(trits), N, K, _ptr(freq), _ptr(row_end), _ptr(payload),
+                                  int(payload.numel() * payload.element_size()), _ptr(workspace),
+                                  int(workspace.numel() * workspace.element_size()), _ptr(err_flag),
+                                  _stream(stream)), "tern_rans_encode")
+
+
+def tern_rans_decode(entries, err_flag, stream=None) -> None:
+    """entries: list of (freq, row_end, payload, N, K, planes); one launch for all."""
+    arr = (_RansItem * len(entries))()
+    for i, (freq, row_end, payload, N, K, planes) in enumerate(entries):
+        arr[i].freq_dev, arr[i].row_end_dev, arr[i].payload_dev = _ptr(freq), _ptr(row_end), _ptr(payload)
+        arr[i].payload_bytes = int(payload.numel() * payload.element_size())
+        arr[i].N, arr[i].K, arr[i].planes_dev = int(N), int(K), _ptr(planes)
+    _check(lib().tern_rans_decode(arr, len(entries), _ptr(err_flag), _stream(stream)), "tern_rans_decode")
 
 
 def tern_read_flag(err_flag, stream=None) -> int:

@@ -172,6 +172,56 @@ tern_status tern_pack_batch(tern_src src, const tern_pack_item* items, int32_t c
   return from_cuda(e);
 }
 
+size_t tern_rans_payload_bound(int32_t N, int32_t K) {
+  return valid_shape(N, K) ? (size_t)N * (tern::rans_slot_bytes(K)) : 0;
+}
+
+size_t tern_rans_workspace_bytes(int32_t N, int32_t K) {
+  return valid_shape(N, K) ? tern::rans_workspace_bytes(N, K) : 0;
+}
+
+tern_status tern_rans_encode(const int8_t* trits_dev, int32_t N, int32_t K, uint16_t* freq_dev, uint32_t* row_end_dev,
+                             uint8_t* payload_dev, size_t payload_capacity, void* workspace_dev, size_t workspace_bytes,
+                             int32_t* err_flag_dev, tern_stream_t stream) {
+  if (!trits_dev || !freq_dev || !row_end_dev || !payload_dev || !workspace_dev || !err_flag_dev) return TERN_EINVAL;
+  if (!valid_shape(N, K)) return TERN_ESHAPE;
+  if (!aligned(trits_dev, 16) || !aligned(freq_dev, 2) || !aligned(row_end_dev, 4) || !aligned(workspace_dev, 16) ||
+      !aligned(err_flag_dev, 4))
+    return TERN_EINVAL;
+  if (workspace_bytes < tern::rans_workspace_bytes(N, K)) return TERN_EINVAL;
+  if (cudaMemsetAsync(err_flag_dev, 0, sizeof(int32_t), cs(stream)) != cudaSuccess) return TERN_ECUDA;
+  return from_cuda(tern::launch_rans_encode(trits_dev, N, K, freq_dev, row_end_dev, payload_dev, payload_capacity,
+                                            workspace_dev, err_flag_dev, cs(stream)));
+}
+
+tern_status tern_rans_decode(const tern_rans_item* items, int32_t count, int32_t* err_flag_dev, tern_stream_t stream) {
+  if (!items || !err_flag_dev || !aligned(err_flag_dev, 4)) return TERN_EINVAL;
+  if (count < 1 || count > TERN_PACK_MAX_ITEMS) return TERN_ESHAPE;
+  for (int i = 0; i < count; ++i) {
+    const tern_rans_item& it = items[i];
+    if (!it.freq_dev || !it.row_end_dev || !it.payload_dev || !it.planes_dev) return TERN_EINVAL;
+    if (!valid_shape(it.N, it.K)) return TERN_ESHAPE;
+    if (!aligned(it.freq_dev, 2) || !aligned(it.row_end_dev, 4) || !aligned(it.planes_dev, 16)) return TERN_EINVAL;
+  }
+  tern::RansBatch* b = new (std::nothrow) tern::RansBatch();
+  if (!b) return TERN_EINVAL;
+  b->count = count;
+  for (int i = 0; i < count; ++i) {
+    b->items[i].freq = items[i].freq_dev;
+    b->items[i].row_end = items[i].row_end_dev;
+    b->items[i].payload = items[i].payload_dev;
+    b->items[i].payload_bytes = items[i].payload_bytes;
+    b->items[i].N = items[i].N;
+    b->items[i].K = items[i].K;
+    b->items[i].planes = items[i].planes_dev;
+  }
+  tern_status st = TERN_OK;
+  if (cudaMemsetAsync(err_flag_dev, 0, sizeof(int32_t), cs(stream)) != cudaSuccess) st = TERN_ECUDA;
+  if (st == TERN_OK) st = from_cuda(tern::launch_rans_decode(*b, err_flag_dev, cs(stream)));
+  delete b;
+  return st;
+}
+
 tern_status tern_base3_encode(const int8_t* trits_dev, int32_t N, int32_t K, uint8_t* out_dev,
                               int32_t* err_flag_dev, tern_stream_t stream) {
   if (!trits_dev || !out_dev || !err_flag_dev) return TERN_EINVAL;

@@ -237,6 +237,27 @@ cudaError_t launch_encode_base3(const int8_t* src, int32_t N, int32_t K, uint8_t
                                 cudaStream_t st);
 cudaError_t launch_occupancy(const uint32_t* planes, int32_t N, int32_t K, int64_t* counts, cudaStream_t st);
 
+// Order-0 rANS transport (tern_rans.cu).
+struct RansItem {
+  const uint16_t* freq;       // device: the tensor's three 12-bit frequencies (t = 0, +1, -1)
+  const uint32_t* row_end;    // device: end byte of each row's stream in the payload [N]
+  const uint8_t* payload;     // device: the rows' streams back to back
+  uint64_t payload_bytes;     // bytes of the payload buffer (reads never go past it)
+  int32_t N, K;
+  uint32_t* planes;           // output: packed planes, N * K / 16 words
+};
+struct RansBatch {
+  RansItem items[kPackMaxItems];
+  int64_t row0[kPackMaxItems];  // first global row of each item (set by the launcher)
+  int64_t rows_total;
+  int32_t count;
+};
+size_t rans_slot_bytes(int32_t K);
+size_t rans_workspace_bytes(int32_t N, int32_t K);
+cudaError_t launch_rans_encode(const int8_t* trits, int32_t N, int32_t K, uint16_t* freq, uint32_t* row_end,
+                               uint8_t* payload, uint64_t capacity, void* workspace, int32_t* flag, cudaStream_t st);
+cudaError_t launch_rans_decode(RansBatch& p, int32_t* flag, cudaStream_t st);
+
 // Activation quantiser and standalone prologue (tern_act.cu).
 cudaError_t launch_quantize(const uint16_t* x, int32_t M, int32_t K, int8_t* q, float* sx, cudaStream_t st);
 cudaError_t launch_prologue(int32_t kind, const void* src, const uint16_t* gain, float eps, int32_t M, int32_t K,

@@ -45,7 +45,8 @@
  *   - tern_pack takes no scale argument: the per-row fp16 scales stay a separate caller array
  *     that a tern_matrix points to; packing would only copy it.
  *   - The launch flags of the *_ex entry points, the batched entry points (tern_pack_batch,
- *     tern_gemv_batch, tern_gemm_batch), tern_base3_encode, tern_occupancy, tern_quantize_act,
+ *     tern_gemv_batch, tern_gemm_batch), tern_base3_encode, the rANS transport (tern_rans_*),
+ *     tern_occupancy, tern_quantize_act,
  *     the prologues (tern_gemm_batch_pro, tern_act_prologue), the verify round (i8_head_verify,
  *     tern_verify_accept) and i8_head_gemv_argmax_noalloc are additions.
  *
@@ -154,6 +155,51 @@ tern_status tern_pack_batch(tern_src src, const tern_pack_item* items, int32_t c
  * tern_pack with TERN_SRC_BASE3). err_flag_dev as for tern_pack. */
 tern_status tern_base3_encode(const int8_t* trits_dev, int32_t N, int32_t K, uint8_t* out_dev,
                               int32_t* err_flag_dev, tern_stream_t stream);
+
+/* Order-0 entropy-coded transport of a ternary tensor (rANS). The pages code the transport close
+ * to its order-0 coding bound ([R] "3진 계열이라는 이름의 실체": within 0.007% of it for the 0.6B)
+ * without naming the coder; this library's coder is byte-wise range asymmetric numeral systems
+ * (J. Duda, 2013), one static 12-bit frequency table per tensor and one stream per row:
+ *   - symbols s = 0 (t = 0), 1 (t = +1), 2 (t = -1); freq[s] >= 1, freq[0] + freq[1] + freq[2] =
+ *     4096; cum = (0, freq[0], freq[0] + freq[1]); the table of a tensor is
+ *     f_s = max(1, floor(4096 c_s / (N*K))) of its trit counts c_s, with 4096 - sum f added to the
+ *     most frequent symbol (the lowest s on ties);
+ *   - a row is encoded from its last trit to its first, from x = 2^23: while x >= 2^19 freq[s],
+ *     the low byte of x is emitted and shifted out; x = (x / freq[s]) * 4096 + x % freq[s] +
+ *     cum[s]; then the final x, low byte first. The row's stream is every emitted byte in reverse
+ *     order (it starts with the final state, most significant byte first);
+ *   - row n's stream occupies payload bytes [row_end[n-1], row_end[n]) (row_end[-1] = 0).
+ * Size: the order-0 entropy of the tensor plus 24..32 bits per row (about 1.334 bits per trit at
+ * the 8B geometry's distribution, against 1.6 for the base-3 transport). */
+typedef struct {
+  const uint16_t* freq_dev;     /* device, 3 frequencies                                        */
+  const uint32_t* row_end_dev;  /* device, N end offsets                                        */
+  const uint8_t* payload_dev;   /* device, the streams                                          */
+  size_t payload_bytes;         /* size of the payload buffer: no read goes past it            */
+  int32_t N, K;                 /* shape, K % 128 == 0                                          */
+  uint32_t* planes_dev;         /* output planes, N*K/16 words, 16-byte aligned                 */
+} tern_rans_item;
+
+/* Payload bytes to provide to tern_rans_encode (an upper bound of any tensor's stream). */
+size_t tern_rans_payload_bound(int32_t N, int32_t K);
+/* Scratch bytes tern_rans_encode needs. */
+size_t tern_rans_workspace_bytes(int32_t N, int32_t K);
+
+/* Encodes int8 trits [N][K] (16-byte aligned) into the transport: freq_dev (3 x uint16),
+ * row_end_dev (N x uint32) and payload_dev (payload_capacity bytes, at least
+ * tern_rans_payload_bound; the stream's size is row_end[N-1]). err_flag_dev is cleared, then set if
+ * a value is not a trit or the payload does not fit (outputs then unspecified). workspace_dev:
+ * tern_rans_workspace_bytes(N, K) bytes, 16-byte aligned, contents need no initialisation. */
+tern_status tern_rans_encode(const int8_t* trits_dev, int32_t N, int32_t K, uint16_t* freq_dev, uint32_t* row_end_dev,
+                             uint8_t* payload_dev, size_t payload_capacity, void* workspace_dev, size_t workspace_bytes,
+                             int32_t* err_flag_dev, tern_stream_t stream);
+
+/* Decodes a list of transports (1..TERN_PACK_MAX_ITEMS, e.g. a whole model at load time) into
+ * their packed planes in one launch, bit-exactly (the planes equal tern_pack of the same trits).
+ * err_flag_dev is cleared, then set if any row is not a valid stream (frequencies not summing to
+ * 4096, a row range outside the payload, a row that does not end in the initial state with all of
+ * its bytes read); that row's planes are then unspecified. No read leaves a row's byte range. */
+tern_status tern_rans_decode(const tern_rans_item* items, int32_t count, int32_t* err_flag_dev, tern_stream_t stream);
 
 /* Per-row occupancy of a packed matrix ([R] "출하된 컨테이너를 직접 읽기": zero / +1 / -1
  * fractions of each tensor). counts_dev: int64[N][3] = {zeros, plus_ones, minus_ones}. */

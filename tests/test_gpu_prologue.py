@@ -67,10 +67,11 @@ def test_standalone_prologue_matches_oracle(kind, K):
     _assert_bits(host(out).view(np.uint16).reshape(M, K), want, exact)
 
 
-@pytest.mark.parametrize("gain_scale", [2.0 ** -125, 2.0 ** 120])
+@pytest.mark.parametrize("gain_scale", [2.0 ** -125, 2.0 ** 126])
 def test_rmsnorm_prologue_subnormal_and_overflow(gain_scale):
-    """Gains of 2^-125 put the outputs into bf16's subnormal range, 2^120 past its largest value
-    (infinity): the one-step fp64 -> bf16 rounding on the device matches the oracle there too."""
+    """Gains of 2^-125 put the outputs into bf16's subnormal range; gains of 2^126 push the larger
+    normalised values (|x| r > 2) past bf16's largest value, to infinity: the one-step fp64 -> bf16
+    rounding on the device matches the oracle there too."""
     M, K = 2, 1024
     src, gain, eps, want, exact = _source("rmsnorm", M, K, 11, gain_scale)
     out = torch.empty(M * K, dtype=torch.int16, device="cuda")
