@@ -43,6 +43,11 @@ def lib() -> ctypes.CDLL:
         L.orc_rans_freqs.argtypes = [vp, i64, vp]; L.orc_rans_freqs.restype = None
         L.orc_rans_encode.argtypes = [vp, i32, i32, vp, vp, vp, i64]; L.orc_rans_encode.restype = i64
         L.orc_rans_decode.argtypes = [vp, vp, i32, i32, vp, vp]; L.orc_rans_decode.restype = i32
+        L.orc_fv5_pack.argtypes = [vp, i32, i32, vp]; L.orc_fv5_pack.restype = i64
+        L.orc_fv5_unpack.argtypes = [vp, i32, i32, vp]; L.orc_fv5_unpack.restype = None
+        L.orc_fv5_gemm_bf16.argtypes = [vp, vp, i32, i32, i32, vp, vp, i32]; L.orc_fv5_gemm_bf16.restype = None
+        L.orc_fv5_gemm_i8.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp, i32]; L.orc_fv5_gemm_i8.restype = None
+        L.orc_fv5b_head.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp, vp, vp]; L.orc_fv5b_head.restype = None
         _LIB = L
     return _LIB
 
@@ -261,6 +266,64 @@ def rans_encode(trits: np.ndarray, freq: np.ndarray | None = None):
 def rans_decode(freq: np.ndarray, row_end: np.ndarray, payload: np.ndarray, N: int, K: int):
     """(trits int8[N, K], ok): ok is False if any row's stream is invalid."""
     t = np.empty((N, K), np.int8)
-    st = lib().orc_rans_decode(_p(_c(payload, np.uint8)), _p(_c(row_end, np.uint32)), N, K,
-                               _p(_c(freq, np.uint16)), _p(t))
+    pl, re, f = _c(payload, np.uint8), _c(row_end, np.uint32), _c(freq, np.uint16)
+    st = lib().orc_rans_decode(_p(pl), _p(re), N, K, _p(f), _p(t))
     return t, st == 0
+
+
+def fv5_pack(codes: np.ndarray) -> np.ndarray:
+    """Five-valued codes int8 [N, K] (values -2..2, K % 256 == 0) -> planes uint32 [N, 3K/32]."""
+    c = _c(codes, np.int8)
+    N, K = c.shape
+    if K % 512:
+        raise OracleError("fv5_pack: K must be a multiple of 512")
+    planes = np.empty((N, 3 * K // 32), np.uint32)
+    if lib().orc_fv5_pack(_p(c), N, K, _p(planes)) != 0:
+        raise OracleError("fv5_pack: code outside -2..2")
+    return planes
+
+
+def fv5_unpack(planes: np.ndarray, K: int) -> np.ndarray:
+    pl = _c(planes, np.uint32)
+    N = pl.size // (3 * K // 32)
+    out = np.empty((N, K), np.int8)
+    lib().orc_fv5_unpack(_p(pl), N, K, _p(out))
+    return out
+
+
+def fv5_gemm_bf16(planes, scales, K: int, x_bf16, nthreads: int | None = None) -> np.ndarray:
+    """fp64 Y[M, N] of the five-valued weights (scales fp32 [N, K/256, 2]) times bf16 x [M, K]."""
+    pl = _c(planes, np.uint32)
+    N = pl.size // (3 * K // 32)
+    x = _c(x_bf16, np.uint16).reshape(-1, K)
+    sc = _c(scales, np.float32)
+    y = np.empty((x.shape[0], N), np.float64)
+    lib().orc_fv5_gemm_bf16(_p(pl), _p(sc), N, K, x.shape[0], _p(x), _p(y), nthreads or default_threads())
+    return y
+
+
+def fv5_gemm_i8(planes, scales, K: int, q, sx, nthreads: int | None = None) -> np.ndarray:
+    pl = _c(planes, np.uint32)
+    N = pl.size // (3 * K // 32)
+    qq = _c(q, np.int8).reshape(-1, K)
+    sc, sxx = _c(scales, np.float32), _c(sx, np.float32)
+    y = np.empty((qq.shape[0], N), np.float32)
+    lib().orc_fv5_gemm_i8(_p(pl), _p(sc), N, K, qq.shape[0], _p(qq), _p(sxx), _p(y), nthreads or default_threads())
+    return y
+
+
+def fv5b_head(W, S, x_bf16=None, q=None, sx=None):
+    """(argmax int32[M], logits float64[M, V]) of the block-scaled int8 head; bf16 x or int8 q + s_x."""
+    w = _c(W, np.int8)
+    V, K = w.shape
+    if q is not None:
+        qq = _c(q, np.int8).reshape(-1, K)
+        M, X, Q, SX = qq.shape[0], None, qq, _c(sx, np.float32)
+    else:
+        X = _c(x_bf16, np.uint16).reshape(-1, K)
+        M, Q, SX = X.shape[0], None, None
+    ss = _c(S, np.float32)
+    lg = np.empty((M, V), np.float64)
+    am = np.empty(M, np.int32)
+    lib().orc_fv5b_head(_p(w), _p(ss), V, K, M, _p(X), _p(Q), _p(SX), _p(lg), _p(am))
+    return am, lg

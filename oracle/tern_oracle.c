@@ -538,3 +538,157 @@ int32_t orc_rans_decode(const uint8_t* payload, const uint32_t* row_end, int32_t
   }
   return status;
 }
+
+/* ----------------------------------------------------------------------------------------- */
+/* five-valued blocks (FV5-style) and the block-scaled int8 head (FV5B-style)                  */
+/*
+ * The pages' shipped formats ([R] "FV5와 FV5B: llama.cpp 포크가 공개한 블록 구조", table): FV5
+ * stores 256 weights per block as three 32-byte bitplanes plus fp32 s_lo and s_hi (3.25 bits per
+ * weight), read as sign and zero plus two magnitude steps -- five states; FV5B stores 256 int8
+ * weights per block with one fp32 scale. The pages do not give the plane semantics; this
+ * library's reading:
+ *   - a five-valued code c in {-2, -1, 0, +1, +2}; block b = weights 256b .. 256b + 255 of a row;
+ *     weight w = 0 (c = 0), sign(c) * s_lo[b] (|c| = 1), sign(c) * s_hi[b] (|c| = 2);
+ *   - planes of a row: mask (c != 0), sign (c < 0), magnitude (|c| = 2), each K/32 words with the
+ *     ternary layout's bit order (mask and magnitude bit of in-word trit j at p(j), sign bit at
+ *     (p(j) + 1) % 32); inside each group of 16 words (512 trits) of a plane, logical word
+ *     w = 4e + t is stored at position 4t + e; row n = [mask | sign | magnitude], 3K/32 words;
+ *   - scales: fp32 [N][K/256][2] = (s_lo, s_hi) per row and block; FV5B head: fp32 [V][K/256];
+ *   - K is a multiple of 512 (whole groups of 16 words).
+ * Products: bf16 mode in fp64 (the plain definition). int8 mode: per block the exact integer sums
+ * A_lo, A_hi of sign * q over the block's |c| = 1 and |c| = 2 weights, then
+ * y = fp32(s_x * sum_b (s_lo[b] A_lo[b] + s_hi[b] A_hi[b])), the sum in fp64 in block order, one
+ * rounding to fp32.
+ */
+
+static int fv5_storage_word(int w) {          /* logical word w of a row plane -> stored word */
+  const int g = w / 16, i = w % 16;
+  return 16 * g + 4 * (i % 4) + i / 4;
+}
+
+int64_t orc_fv5_pack(const int8_t* codes, int32_t N, int32_t K, uint32_t* planes) {
+  const int KW = K / 32;
+  int64_t bad = 0;
+  if (K % 512) return -1;
+  memset(planes, 0, sizeof(uint32_t) * (size_t)N * 3 * KW);
+  for (int32_t n = 0; n < N; ++n) {
+    uint32_t* row = planes + (size_t)n * 3 * KW;
+    for (int32_t k = 0; k < K; ++k) {
+      const int c = codes[(size_t)n * K + k];
+      if (c < -2 || c > 2) { ++bad; continue; }
+      const int w = fv5_storage_word(k / 32);
+      if (c != 0) row[w] |= 1u << mask_bit(k);
+      if (c < 0) row[KW + w] |= 1u << sign_bit(k);
+      if (c == 2 || c == -2) row[2 * KW + w] |= 1u << mask_bit(k);
+    }
+  }
+  return bad;
+}
+
+void orc_fv5_unpack(const uint32_t* planes, int32_t N, int32_t K, int8_t* codes) {
+  const int KW = K / 32;
+  for (int32_t n = 0; n < N; ++n) {
+    const uint32_t* row = planes + (size_t)n * 3 * KW;
+    for (int32_t k = 0; k < K; ++k) {
+      const int w = fv5_storage_word(k / 32);
+      const int m = (row[w] >> mask_bit(k)) & 1, s = (row[KW + w] >> sign_bit(k)) & 1;
+      const int g = (row[2 * KW + w] >> mask_bit(k)) & 1;
+      codes[(size_t)n * K + k] = (int8_t)(m ? (s ? -1 : 1) * (g ? 2 : 1) : 0);
+    }
+  }
+}
+
+typedef struct {
+  const uint32_t* planes; const float* scales; int32_t N, K, M; const uint16_t* X; double* Y;
+} fv5_bf16_ctx;
+
+static void fv5_bf16_rows(void* p, int64_t b, int64_t e) {
+  fv5_bf16_ctx* c = (fv5_bf16_ctx*)p;
+  int8_t* code = (int8_t*)malloc((size_t)c->K);
+  for (int64_t n = b; n < e; ++n) {
+    orc_fv5_unpack(c->planes + (size_t)n * 3 * (c->K / 32), 1, c->K, code);
+    const float* sc = c->scales + (size_t)n * (c->K / 256) * 2;
+    for (int m = 0; m < c->M; ++m) {
+      const uint16_t* x = c->X + (size_t)m * c->K;
+      double acc = 0.0;
+      for (int k = 0; k < c->K; ++k) {
+        const int cc = code[k];
+        if (!cc) continue;
+        const double w = (cc > 0 ? 1.0 : -1.0) * (double)sc[2 * (k / 256) + (cc == 2 || cc == -2)];
+        acc += w * (double)orc_bf16_to_float(x[k]);
+      }
+      c->Y[(size_t)m * c->N + n] = acc;
+    }
+  }
+  free(code);
+}
+
+void orc_fv5_gemm_bf16(const uint32_t* planes, const float* scales, int32_t N, int32_t K, int32_t M,
+                       const uint16_t* X, double* Y, int32_t nthreads) {
+  fv5_bf16_ctx c = {planes, scales, N, K, M, X, Y};
+  parallel_for(N, nthreads, fv5_bf16_rows, &c);
+}
+
+typedef struct {
+  const uint32_t* planes; const float* scales; int32_t N, K, M; const int8_t* Q; const float* SX; float* Y;
+} fv5_i8_ctx;
+
+static void fv5_i8_rows(void* p, int64_t b, int64_t e) {
+  fv5_i8_ctx* c = (fv5_i8_ctx*)p;
+  int8_t* code = (int8_t*)malloc((size_t)c->K);
+  for (int64_t n = b; n < e; ++n) {
+    orc_fv5_unpack(c->planes + (size_t)n * 3 * (c->K / 32), 1, c->K, code);
+    const float* sc = c->scales + (size_t)n * (c->K / 256) * 2;
+    for (int m = 0; m < c->M; ++m) {
+      const int8_t* q = c->Q + (size_t)m * c->K;
+      double tot = 0.0;
+      for (int blk = 0; blk < c->K / 256; ++blk) {
+        int64_t lo = 0, hi = 0;
+        for (int k = 256 * blk; k < 256 * blk + 256; ++k) {
+          const int cc = code[k];
+          if (cc == 1) lo += q[k]; else if (cc == -1) lo -= q[k];
+          else if (cc == 2) hi += q[k]; else if (cc == -2) hi -= q[k];
+        }
+        tot += (double)sc[2 * blk] * (double)lo + (double)sc[2 * blk + 1] * (double)hi;
+      }
+      c->Y[(size_t)m * c->N + n] = (float)((double)c->SX[m] * tot);
+    }
+  }
+  free(code);
+}
+
+void orc_fv5_gemm_i8(const uint32_t* planes, const float* scales, int32_t N, int32_t K, int32_t M,
+                     const int8_t* Q, const float* SX, float* Y, int32_t nthreads) {
+  fv5_i8_ctx c = {planes, scales, N, K, M, Q, SX, Y};
+  parallel_for(N, nthreads, fv5_i8_rows, &c);
+}
+
+/* FV5B-style head: logits[m][v] = sum_b s[v][b] * sum_{k in b} W[v][k] x[m][k]; argmax, lowest
+ * index on exact ties. bf16 mode in fp64; int8 mode fp32(s_x * sum_b s_b A_b), fp64 sum in order. */
+void orc_fv5b_head(const int8_t* W, const float* S, int32_t V, int32_t K, int32_t M, const uint16_t* X,
+                   const int8_t* Q, const float* SX, double* LOGITS, int32_t* ARGMAX) {
+  const int nb = K / 256;
+  for (int m = 0; m < M; ++m) {
+    for (int32_t v = 0; v < V; ++v) {
+      const int8_t* w = W + (size_t)v * K;
+      double tot = 0.0;
+      for (int blk = 0; blk < nb; ++blk) {
+        if (Q) {
+          int64_t a = 0;
+          for (int k = 256 * blk; k < 256 * blk + 256; ++k) a += (int64_t)w[k] * Q[(size_t)m * K + k];
+          tot += (double)S[(size_t)v * nb + blk] * (double)a;
+        } else {
+          double a = 0.0;
+          for (int k = 256 * blk; k < 256 * blk + 256; ++k)
+            a += (double)w[k] * (double)orc_bf16_to_float(X[(size_t)m * K + k]);
+          tot += (double)S[(size_t)v * nb + blk] * a;
+        }
+      }
+      LOGITS[(size_t)m * V + v] = Q ? (double)(float)((double)SX[m] * tot) : tot;
+    }
+    int32_t best = 0;
+    for (int32_t v = 1; v < V; ++v)
+      if (LOGITS[(size_t)m * V + v] > LOGITS[(size_t)m * V + best]) best = v;
+    ARGMAX[m] = best;
+  }
+}
