@@ -744,6 +744,8 @@ def extra_rows(stack, torch, tg, hbm_peak, bf16_peak):
     out["base3_unpack_8b"] = base3_row(stack, torch, tg, hbm_peak)
     # order-0 rANS transport of all 8B trits: decode into the planes in one launch
     out["rans_decode_8b"] = rans_row(torch, tg, hbm_peak)
+    # five-valued (FV5-style) weights and the block-scaled (FV5B-style) head
+    out["fv5_8b"] = fv5_rows(stack, torch, tg, hbm_peak)
     return out
 
 
@@ -1029,6 +1031,64 @@ def rans_row(torch, tg, hbm_peak):
            "trits": trits, "transport_bytes": payload_bytes, "bits_per_trit": 8.0 * payload_bytes / trits,
            "tensors": len(entries), "launches": 1}
     del entries
+    return out
+
+
+def fv5_rows(stack, torch, tg, hbm_peak):
+    """Three 8B layers' seven linears (21 launches, 235 MB > L2) as five-valued weights at M = 1
+    (codes: the 8B trits, magnitude 2 where a second trit stream draws +1; fp32 s_lo in
+    [0.01, 0.05), s_hi = 2..3 x s_lo, seeded), then the FV5B-style head 151936 x 4096 (the stack's
+    int8 head weights with one fp32 scale per 256-weight block). bf16 activations."""
+    import synth
+    import synth.cuda as sc
+    gen = torch.Generator(device="cuda").manual_seed(SEED)
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    mats, xs, ys, nbytes = [], {}, [], 0
+    for layer in range(1, 4):
+        for p, N, K in synth.linear_shapes("8b"):
+            t = torch.empty(N * K, dtype=torch.int8, device="cuda")
+            h = torch.empty(N * K, dtype=torch.int8, device="cuda")
+            sc.trits_into(t, SEED, synth.tensor_id(layer, p), K, synth.trit_probs("8b", layer, p))
+            sc.trits_into(h, SEED + 1, synth.tensor_id(layer, p), K)
+            codes = t * (1 + (h == 1).to(torch.int8))
+            del t, h
+            planes = torch.empty(N * 3 * K // 32, dtype=torch.int32, device="cuda")
+            tg.tern_fv5_pack(codes, N, K, planes, flag)
+            del codes
+            lo = 0.01 + 0.04 * torch.rand(N * (K // 256), device="cuda", generator=gen)
+            hi = lo * (2 + torch.rand(N * (K // 256), device="cuda", generator=gen))
+            scales = torch.stack([lo, hi], 1).contiguous()
+            mats.append(tg.Fv5Matrix(planes, scales, N, K))
+            if K not in xs:
+                xs[K] = torch.from_numpy(synth.activations(SEED, 8000 + K, 1, K).view(np.int16)).cuda()
+            ys.append(torch.empty(N, dtype=torch.float32, device="cuda"))
+            nbytes += N * K * 3 // 8 + N * (K // 256) * 8 + 2 * K + 4 * N
+    assert tg.tern_read_flag(flag) == 0
+
+    def pass_(i):
+        for W, y in zip(mats, ys):
+            tg.tern_fv5_gemm(W, 1, tg.TERN_ACT_BF16, xs[W.K], None, y)
+    g = capture(pass_, 2)
+    g.replay()
+    torch.cuda.synchronize()
+    ms = timed_replays([(g, 5)]) / 10
+    out = {"linears_3_layers_m1_bf16": {"ms": ms, "gbs": nbytes / (ms / 1000.0) / 1e9,
+                                        "frac": nbytes / (ms / 1000.0) / 1e9 / hbm_peak, "bytes": nbytes,
+                                        "launches": len(mats), "bits_per_weight": 3.25}}
+    del mats, g
+    V, d = stack.V, stack.d
+    S = (0.001 + 0.02 * torch.rand(V * (d // 256), device="cuda", generator=gen)).contiguous()
+    xb = torch.from_numpy(synth.activations(SEED, 8100, 1, d).view(np.int16)).cuda()
+    am = torch.empty(1, dtype=torch.int32, device="cuda")
+    mv = torch.empty(1, dtype=torch.float32, device="cuda")
+    g = capture(lambda i: tg.fv5b_head_gemv_argmax(stack.head_W, S, V, d, 1, tg.TERN_ACT_BF16, xb, None, am, mv,
+                                                    None, stack.ws), 5)
+    g.replay()
+    torch.cuda.synchronize()
+    ms = timed_replays([(g, 4)]) / 20
+    hb = V * d + V * (d // 256) * 4 + 2 * d + 8
+    out["fv5b_head_151936x4096_m1_bf16"] = {"us": ms * 1000.0, "gbs": hb / (ms / 1000.0) / 1e9,
+                                            "frac": hb / (ms / 1000.0) / 1e9 / hbm_peak}
     return out
 
 

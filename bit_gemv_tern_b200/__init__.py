@@ -25,6 +25,7 @@ __all__ = [
     "GemvBatch", "tern_gemv_batch", "tern_gemv_batch_workspace_bytes", "tern_gemm_batch",
     "tern_gemm_batch_workspace_bytes", "tern_gemm_batch_pro", "tern_act_prologue",
     "i8_head_verify", "tern_verify_accept",
+    "Fv5Matrix", "tern_fv5_packed_bytes", "tern_fv5_pack", "tern_fv5_gemm", "fv5b_head_gemv_argmax",
     "tern_rans_payload_bound", "tern_rans_workspace_bytes", "tern_rans_encode", "tern_rans_decode",
     "TERN_PRO_NONE", "TERN_PRO_BF16", "TERN_PRO_CAST", "TERN_PRO_RMSNORM", "TERN_PRO_SWIGLU",
     "tern_status_string",
@@ -90,6 +91,10 @@ def lib() -> ctypes.CDLL:
             "tern_act_prologue": ([vp, i32, i32, vp, vp], i32),
             "i8_head_verify": ([vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
             "tern_verify_accept": ([vp, vp, i32, vp, vp], i32),
+            "tern_fv5_packed_bytes": ([i32, i32], sz),
+            "tern_fv5_pack": ([vp, i32, i32, vp, vp, vp], i32),
+            "tern_fv5_gemm": ([vp, i32, i32, vp, vp, vp, vp], i32),
+            "fv5b_head_gemv_argmax": ([vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp], i32),
             "tern_rans_payload_bound": ([i32, i32], sz),
             "tern_rans_workspace_bytes": ([i32, i32], sz),
             "tern_rans_encode": ([vp, i32, i32, vp, vp, vp, sz, vp, sz, vp, vp], i32),
@@ -250,6 +255,41 @@ def i8_head_verify(W, scale_f16, V: int, K: int, M: int, act: int, X, x_scale, d
 
 def tern_verify_accept(argmax, draft, k: int, accept, stream=None) -> None:
     _check(lib().tern_verify_accept(_ptr(argmax), _ptr(draft), k, _ptr(accept), _stream(stream)), "tern_verify_accept")
+
+
+class _Fv5Matrix(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int32), ("K", ctypes.c_int32), ("planes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
+class Fv5Matrix:
+    """Five-valued weights: planes (int32 tensor of N*3K/32 words) and fp32 scales [N, K/256, 2]."""
+
+    def __init__(self, planes, scales, N: int, K: int):
+        self.planes, self.scales, self.N, self.K = planes, scales, int(N), int(K)
+        self._c = _Fv5Matrix(self.N, self.K, _ptr(planes), _ptr(scales))
+
+    def ref(self):
+        return ctypes.byref(self._c)
+
+
+def tern_fv5_packed_bytes(N: int, K: int) -> int:
+    return int(lib().tern_fv5_packed_bytes(N, K))
+
+
+def tern_fv5_pack(codes, N: int, K: int, planes, err_flag, stream=None) -> None:
+    _check(lib().tern_fv5_pack(_ptr(codes), N, K, _ptr(planes), _ptr(err_flag), _stream(stream)), "tern_fv5_pack")
+
+
+def tern_fv5_gemm(W: Fv5Matrix, M: int, act: int, X, x_scale, Y, stream=None) -> None:
+    _check(lib().tern_fv5_gemm(W.ref(), M, act, _ptr(X), _ptr(x_scale), _ptr(Y), _stream(stream)), "tern_fv5_gemm")
+
+
+def fv5b_head_gemv_argmax(W, block_scale, V: int, K: int, M: int, act: int, X, x_scale, argmax, maxval, logits,
+                          workspace, stream=None) -> None:
+    _check(lib().fv5b_head_gemv_argmax(_ptr(W), _ptr(block_scale), V, K, M, act, _ptr(X), _ptr(x_scale),
+                                       _ptr(argmax), _ptr(maxval), _ptr(logits), _ptr(workspace),
+                                       int(workspace.numel() * workspace.element_size()), _stream(stream)),
+           "fv5b_head_gemv_argmax")
 
 
 class _RansItem(ctypes.Structure):

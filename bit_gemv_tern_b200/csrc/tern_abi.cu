@@ -50,12 +50,15 @@ namespace tern {
 tern_status plan_head_call(const int8_t* W_dev, const uint16_t* scale_f16_dev, int32_t V, int32_t K, int32_t M,
                            tern_act act, const void* X_dev, const float* x_scale_dev, int32_t* argmax_dev,
                            float* maxval_dev, float* logits_dev, void* workspace_dev, size_t workspace_bytes,
-                           uint32_t flags, HeadParams& p) {
-  if (!W_dev || !scale_f16_dev || !X_dev || !argmax_dev || !maxval_dev || !workspace_dev) return TERN_EINVAL;
+                           uint32_t flags, HeadParams& p, const float* block_scale_dev) {
+  const bool bs = block_scale_dev != nullptr;
+  if (!W_dev || (!bs && !scale_f16_dev) || !X_dev || !argmax_dev || !maxval_dev || !workspace_dev) return TERN_EINVAL;
   if (act != TERN_ACT_BF16 && act != TERN_ACT_INT8) return TERN_EINVAL;
   if (flags & ~TERN_FLAG_PDL) return TERN_EINVAL;
   if (!valid_shape(V, K) || M < 1 || M > 16) return TERN_ESHAPE;
-  if (!aligned(W_dev, 16) || !aligned(X_dev, 16) || !aligned(workspace_dev, 16) || !aligned(scale_f16_dev, 2))
+  if (bs && (K % 256 || (act == TERN_ACT_BF16 && M > 8))) return TERN_ESHAPE;
+  if (!aligned(W_dev, 16) || !aligned(X_dev, 16) || !aligned(workspace_dev, 16) ||
+      (!bs && !aligned(scale_f16_dev, 2)) || (bs && !aligned(block_scale_dev, 4)))
     return TERN_EINVAL;
   if (!aligned(argmax_dev, 4) || !aligned(maxval_dev, 4) || (logits_dev && !aligned(logits_dev, 4)))
     return TERN_EINVAL;
@@ -75,10 +78,11 @@ tern_status plan_head_call(const int8_t* W_dev, const uint16_t* scale_f16_dev, i
   p.logits = logits_dev;
   p.counter = static_cast<unsigned int*>(workspace_dev);
   p.keys = reinterpret_cast<unsigned long long*>(static_cast<char*>(workspace_dev) + 16);
-  const int units = K / 128;
+  p.bscale = block_scale_dev;
+  const int units = K / (bs ? 256 : 128);            // a K slice holds whole units
   int ks = 1;
-  while (head_smem_bytes(p.mode, M, K / ks) > kHeadSmemCap && ks < 8 && units % (2 * ks) == 0) ks *= 2;
-  if (head_smem_bytes(p.mode, M, K / ks) > kHeadSmemCap) return TERN_ESHAPE;
+  while (head_smem_bytes(p.mode, M, K / ks, bs) > kHeadSmemCap && ks < 8 && units % (2 * ks) == 0) ks *= 2;
+  if (head_smem_bytes(p.mode, M, K / ks, bs) > kHeadSmemCap) return TERN_ESHAPE;
   p.ksplit = ks;
   p.kr = K / ks;
   p.nrb = (V + 127) / 128;
@@ -456,7 +460,8 @@ tern_status i8_head_gemv_argmax_ex(const int8_t* W_dev, const uint16_t* scale_f1
                                    tern_stream_t stream) {
   tern::HeadParams p = {};
   const tern_status st = tern::plan_head_call(W_dev, scale_f16_dev, V, K, M, act, X_dev, x_scale_dev, argmax_dev,
-                                              maxval_dev, logits_dev, workspace_dev, workspace_bytes, flags, p);
+                                              maxval_dev, logits_dev, workspace_dev, workspace_bytes, flags, p,
+                                              nullptr);
   if (st != TERN_OK) return st;
   return from_cuda(tern::launch_head(p, (flags & TERN_FLAG_PDL) != 0, cs(stream)));
 }
@@ -469,7 +474,7 @@ tern_status i8_head_verify(const int8_t* W_dev, const uint16_t* scale_f16_dev, i
   if (M > 1 && (!draft_dev || !aligned(draft_dev, 4))) return TERN_EINVAL;
   tern::HeadParams p = {};
   const tern_status st = tern::plan_head_call(W_dev, scale_f16_dev, V, K, M, act, X_dev, x_scale_dev, argmax_dev,
-                                              maxval_dev, nullptr, workspace_dev, workspace_bytes, 0u, p);
+                                              maxval_dev, nullptr, workspace_dev, workspace_bytes, 0u, p, nullptr);
   if (st != TERN_OK) return st;
   p.draft = draft_dev;
   p.accept = accept_dev;
@@ -490,6 +495,63 @@ tern_status i8_head_gemv_argmax(const int8_t* W_dev, const uint16_t* scale_f16_d
                                 tern_stream_t stream) {
   return i8_head_gemv_argmax_ex(W_dev, scale_f16_dev, V, K, M, act, X_dev, x_scale_dev, argmax_dev, maxval_dev,
                                 logits_dev, workspace_dev, workspace_bytes, 0u, stream);
+}
+
+size_t tern_fv5_packed_bytes(int32_t N, int32_t K) {
+  return (N > 0 && K > 0 && K % 512 == 0) ? (size_t)N * (size_t)K * 3 / 8 : 0;
+}
+
+tern_status tern_fv5_pack(const int8_t* codes_dev, int32_t N, int32_t K, uint32_t* planes_dev, int32_t* err_flag_dev,
+                          tern_stream_t stream) {
+  if (!codes_dev || !planes_dev || !err_flag_dev) return TERN_EINVAL;
+  if (N <= 0 || K <= 0 || K % 512) return TERN_ESHAPE;
+  if (!aligned(codes_dev, 16) || !aligned(planes_dev, 16) || !aligned(err_flag_dev, 4)) return TERN_EINVAL;
+  if (cudaMemsetAsync(err_flag_dev, 0, sizeof(int32_t), cs(stream)) != cudaSuccess) return TERN_ECUDA;
+  return from_cuda(tern::launch_fv5_pack(codes_dev, N, K, planes_dev, err_flag_dev, cs(stream)));
+}
+
+tern_status tern_fv5_gemm(const tern_fv5_matrix* W, int32_t M, tern_act act, const void* X_dev, const float* x_scale_dev,
+                          float* Y_dev, tern_stream_t stream) {
+  if (!W || !W->planes || !W->scales) return TERN_EINVAL;
+  if (W->N <= 0 || W->K <= 0 || W->K % 512) return TERN_ESHAPE;
+  if (act != TERN_ACT_BF16 && act != TERN_ACT_INT8) return TERN_EINVAL;
+  if (M < 1 || M > (act == TERN_ACT_BF16 ? 8 : 16)) return TERN_ESHAPE;
+  if (!aligned(W->planes, 16) || !aligned(W->scales, 8)) return TERN_EINVAL;
+  if (!X_dev || !Y_dev || !aligned(X_dev, 16) || !aligned(Y_dev, 4)) return TERN_EINVAL;
+  if (act == TERN_ACT_INT8 && (!x_scale_dev || !aligned(x_scale_dev, 4))) return TERN_EINVAL;
+  tern::Fv5Params p = {};
+  p.planes = W->planes;
+  p.scales = W->scales;
+  p.N = W->N;
+  p.K = W->K;
+  p.x = X_dev;
+  p.sx = x_scale_dev;
+  p.y = Y_dev;
+  p.M = M;
+  p.mode = act == TERN_ACT_BF16 ? 0 : 1;
+  // split K over a cluster of up to 8 CTAs (whole 512-trit groups per slice) to cover the SMs
+  const int row_blocks = (p.N + tern::fv5_rows_per_cta() - 1) / tern::fv5_rows_per_cta();
+  const int units = p.K / 512;
+  const int sms = tern::device_sm_count();
+  int ks = 1;
+  while (ks < 8 && row_blocks * ks < 2 * sms && units % (2 * ks) == 0) ks *= 2;
+  while (tern::fv5_smem_bytes(p.mode, M, p.K / ks) > kGemmSmemCap && ks < 8 && units % (2 * ks) == 0) ks *= 2;
+  if (tern::fv5_smem_bytes(p.mode, M, p.K / ks) > kGemmSmemCap) return TERN_ESHAPE;
+  p.ksplit = ks;
+  p.kr = p.K / ks;
+  return from_cuda(tern::launch_fv5_gemm(p, cs(stream)));
+}
+
+tern_status fv5b_head_gemv_argmax(const int8_t* W_dev, const float* block_scale_dev, int32_t V, int32_t K, int32_t M,
+                                  tern_act act, const void* X_dev, const float* x_scale_dev, int32_t* argmax_dev,
+                                  float* maxval_dev, float* logits_dev, void* workspace_dev, size_t workspace_bytes,
+                                  tern_stream_t stream) {
+  if (!block_scale_dev) return TERN_EINVAL;
+  tern::HeadParams p = {};
+  const tern_status st = tern::plan_head_call(W_dev, nullptr, V, K, M, act, X_dev, x_scale_dev, argmax_dev, maxval_dev,
+                                              logits_dev, workspace_dev, workspace_bytes, 0u, p, block_scale_dev);
+  if (st != TERN_OK) return st;
+  return from_cuda(tern::launch_head(p, false, cs(stream)));
 }
 
 tern_status tern_read_flag(const int32_t* err_flag_dev, tern_stream_t stream) {

@@ -1,0 +1,328 @@
+// Five-valued weights in 256-weight blocks (FV5-style): packing and the GEMV / small-M product.
+//
+// The pages' shipped linear format (PyTorchKR review "Fermion Research, 3진 계열 포맷으로 직접
+// 학습한 Neutrino-1 모델군 3종 공개", section "FV5와 FV5B: llama.cpp 포크가 공개한 블록 구조")
+// stores 256 weights per block as three bitplanes and two fp32 scales, s_lo and s_hi: sign and
+// zero plus two magnitude steps. This library's reading (include/tern.h): a code c in -2..2 per
+// weight, w = sign(c) * (|c| == 2 ? s_hi : s_lo) of its row and block, planes mask / sign / high
+// magnitude in the ternary layout's bit order, words transposed inside each 512-trit group so that
+// lane t of a quad reads logical words t, 4 + t, 8 + t, 12 + t as one 128-bit load.
+//
+//   Y[m][n] = sum_b ( s_lo[n][b] * sum_{k in b, |c| = 1} sign * X[m][k]
+//                   + s_hi[n][b] * sum_{k in b, |c| = 2} sign * X[m][k] )
+//
+// Kernel: as the ternary small-M kernel (tern_gemv.cu): 16-row warp tiles, the K slice of the
+// activations staged once as int8 operand columns (q, or four exact limbs per token), CTAs splitting
+// K form a cluster. Each word is split into its low- and high-magnitude ternary parts (mask & ~g,
+// sign & ~g; mask & g, sign & g), each decoded to 64 * t bytes and multiplied exactly by the
+// tensor cores into its own int32 accumulators. Step e of a 512-trit chunk covers logical words
+// 4e .. 4e + 3 of all four quad lanes, i.e. trits 128e .. 128e + 127, so steps 0-1 and 2-3 are the
+// chunk's two blocks: after each block the exact sums are scaled by the block's s_lo and s_hi and
+// added into fp64 accumulators, which the epilogue rounds once to fp32 (int8 mode after * s_x).
+#include <atomic>
+#include <cooperative_groups.h>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "tern_device.cuh"
+#include "tern_kernels.h"
+
+namespace cg = cooperative_groups;
+
+namespace tern {
+namespace {
+
+constexpr int kRows = 128;  // rows per CTA: 8 warps x 16 rows
+
+__device__ __forceinline__ uint32_t u4get(const uint4& v, int e) {
+  return e == 0 ? v.x : (e == 1 ? v.y : (e == 2 ? v.z : v.w));
+}
+__device__ __forceinline__ int fv5_cols(int mode, int M) { return mode == 0 ? 4 * M : M; }
+__device__ __forceinline__ int col_words(int kr) { return kr / 4 + 16; }
+__device__ __forceinline__ int half_ofs(int v) { return 4 * (v ^ ((v >> 3) & 3)); }
+
+// ---- pack -------------------------------------------------------------------------------------------
+// One thread per (row, logical 32-trit word): 32 codes in, the three plane words out at the word's
+// stored position.
+__global__ void k_fv5_pack(const int8_t* __restrict__ codes, int64_t words, int32_t KW, uint32_t* __restrict__ planes,
+                           int32_t* flag) {
+  bool bad = false;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < words; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = i / KW;
+    const int w = (int)(i - row * KW);
+    const int8_t* c = codes + i * 32;
+    const uint4 v0 = ld_stream(c), v1 = ld_stream(c + 16);
+    const uint32_t b[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    uint32_t m = 0u, s = 0u, g = 0u;                        // natural order: bit j = trit j of the word
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int x = (int8_t)(b[j >> 2] >> (8 * (j & 3)));
+      bad |= x < -2 || x > 2;
+      m |= (uint32_t)(x != 0) << j;
+      s |= (uint32_t)(x < 0) << j;
+      g |= (uint32_t)(x == 2 || x == -2) << j;
+    }
+    // natural order -> the layout's order p(j) (swap bits 0 and 4 of j)
+    auto order = [](uint32_t x) {
+      const uint32_t t = lop3<0x28u>(x >> 15, x, 0x0000AAAAu);
+      return lop3<0x96u>(x, t, t << 15);
+    };
+    const int grp = w >> 4, li = w & 15;
+    const int sw = 16 * grp + 4 * (li & 3) + (li >> 2);     // stored position of logical word w
+    uint32_t* rp = planes + row * 3 * (int64_t)KW;
+    const uint32_t sp = order(s);
+    rp[sw] = order(m);
+    rp[KW + sw] = (sp << 1) | (sp >> 31);
+    rp[2 * KW + sw] = order(g);
+  }
+  if (__any_sync(0xFFFFFFFFu, bad) && (threadIdx.x & 31) == 0) atomicExch(flag, 1);
+}
+
+// ---- product ----------------------------------------------------------------------------------------
+template <int MODE, int NG>
+__global__ void __launch_bounds__(kThreads) k_fv5_gemm(const Fv5Params p) {
+  extern __shared__ __align__(16) uint32_t smem[];
+  __shared__ int expo[16];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int ks = blockIdx.x;
+  const int k0 = ks * p.kr;
+  const int row0 = blockIdx.y * kRows + warp * 16;
+  const int KM = p.K >> 5;
+  const int nw = p.kr >> 5;                                // multiple of 16
+  const int nchunks = nw >> 4;
+  const bool warp_live = row0 < p.N;
+  const int ra = min(row0 + g, p.N - 1), rb = min(row0 + g + 8, p.N - 1);
+  const uint32_t* pa = p.planes + (size_t)ra * (3 * KM) + (k0 >> 5);
+  const uint32_t* pb = p.planes + (size_t)rb * (3 * KM) + (k0 >> 5);
+  const int nblk = p.K >> 8;
+  const float2* sca = reinterpret_cast<const float2*>(p.scales) + (size_t)ra * nblk + (k0 >> 8);
+  const float2* scb = reinterpret_cast<const float2*>(p.scales) + (size_t)rb * nblk + (k0 >> 8);
+  const int ncols = fv5_cols(MODE, p.M);
+  const int RS = col_words(p.kr);
+
+  // chunk c: stored words [16c + 4t, 16c + 4t + 4) of the three planes of rows ra, rb
+  auto load_chunk = [&](int c, uint4 (&w)[6]) {
+    const int off = 16 * c + 4 * t;
+    if (warp_live && c < nchunks) {
+      w[0] = ld_stream(pa + off);
+      w[1] = ld_stream(pb + off);
+      w[2] = ld_stream(pa + KM + off);
+      w[3] = ld_stream(pb + KM + off);
+      w[4] = ld_stream(pa + 2 * KM + off);
+      w[5] = ld_stream(pb + 2 * KM + off);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 6; ++i) w[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  uint4 cur[6], nxt[6];
+  load_chunk(0, cur);
+  load_chunk(1, nxt);
+  pdl_wait();
+
+  // ---- stage the activation slice as int8 operand columns (as tern_gemv.cu) ----------------------
+  const int per_row = p.kr >> 4;
+  if (MODE == 1) {
+    const int8_t* xs = static_cast<const int8_t*>(p.x);
+    for (int i = threadIdx.x; i < p.M * per_row; i += kThreads) {
+      const int m = i / per_row, v = i - m * per_row;
+      *reinterpret_cast<uint4*>(smem + m * RS + half_ofs(v)) = permute_i8_half(ld_nc(xs + (size_t)m * p.K + k0 + 16 * v));
+    }
+  } else {
+    const uint16_t* xs = static_cast<const uint16_t*>(p.x);
+    for (int m = warp; m < p.M; m += kThreads / 32) {
+      float amax = 0.0f;
+      for (int k = lane * 8; k < p.kr; k += 256) {
+        const uint4 v = ld_nc(xs + (size_t)m * p.K + k0 + k);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          amax = fmaxf(amax, fmaxf(fabsf(bf16_bits_to_float(w[e] & 0xFFFFu)), fabsf(bf16_bits_to_float(w[e] >> 16))));
+      }
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+      if (lane == 0) expo[m] = limb_exponent(amax);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < p.M * per_row; i += kThreads) {
+      const int m = i / per_row, v = i - m * per_row;
+      const int E = expo[m];
+      const uint16_t* xb = xs + (size_t)m * p.K + k0 + 16 * v;
+      const uint4 a = ld_nc(xb), b = ld_nc(xb + 8);
+      const uint32_t wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      uint32_t l[4][4] = {};
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const uint32_t bits = (e & 1) ? (wv[e >> 1] >> 16) : (wv[e >> 1] & 0xFFFFu);
+        int L[4];
+        limbs_of(limb_fixed(bf16_bits_to_float(bits), E), L);
+        const int sh = 8 * (e & 3);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) l[c][e >> 2] |= (uint32_t)(uint8_t)L[c] << sh;
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        *reinterpret_cast<uint4*>(smem + (4 * m + c) * RS + half_ofs(v)) =
+            permute_i8_half(make_uint4(l[c][0], l[c][1], l[c][2], l[c][3]));
+    }
+  }
+  __syncthreads();
+
+  double Y[NG][4];
+#pragma unroll
+  for (int n = 0; n < NG; ++n) Y[n][0] = Y[n][1] = Y[n][2] = Y[n][3] = 0.0;
+
+  for (int c = 0; c < nchunks; ++c) {
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {                 // the chunk's two 256-weight blocks
+      int accL[NG][4], accH[NG][4];
+#pragma unroll
+      for (int n = 0; n < NG; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) accL[n][i] = accH[n][i] = 0;
+#pragma unroll
+      for (int ee = 0; ee < 2; ++ee) {
+        const int e = 2 * half + ee;
+        const int w = 16 * c + 4 * e + t;                  // logical word of this lane
+        const uint32_t ga = u4get(cur[4], e), gb = u4get(cur[5], e);
+        uint32_t la0, lb0, la1, lb1, ha0, hb0, ha1, hb1;
+        merge_planes(u4get(cur[0], e) & ~ga, u4get(cur[2], e) & ~(ga << 1 | ga >> 31), la0, lb0);
+        merge_planes(u4get(cur[1], e) & ~gb, u4get(cur[3], e) & ~(gb << 1 | gb >> 31), la1, lb1);
+        merge_planes(u4get(cur[0], e) & ga, u4get(cur[2], e) & (ga << 1 | ga >> 31), ha0, hb0);
+        merge_planes(u4get(cur[1], e) & gb, u4get(cur[3], e) & (gb << 1 | gb >> 31), ha1, hb1);
+        const uint32_t AL[8][2] = {
+            {dec_i8<0>(la0, lb0), dec_i8<0>(la1, lb1)}, {dec_i8<1>(la0, lb0), dec_i8<1>(la1, lb1)},
+            {dec_i8<2>(la0, lb0), dec_i8<2>(la1, lb1)}, {dec_i8<3>(la0, lb0), dec_i8<3>(la1, lb1)},
+            {dec_i8<4>(la0, lb0), dec_i8<4>(la1, lb1)}, {dec_i8<5>(la0, lb0), dec_i8<5>(la1, lb1)},
+            {dec_i8<6>(la0, lb0), dec_i8<6>(la1, lb1)}, {dec_i8<7>(la0, lb0), dec_i8<7>(la1, lb1)}};
+        const uint32_t AH[8][2] = {
+            {dec_i8<0>(ha0, hb0), dec_i8<0>(ha1, hb1)}, {dec_i8<1>(ha0, hb0), dec_i8<1>(ha1, hb1)},
+            {dec_i8<2>(ha0, hb0), dec_i8<2>(ha1, hb1)}, {dec_i8<3>(ha0, hb0), dec_i8<3>(ha1, hb1)},
+            {dec_i8<4>(ha0, hb0), dec_i8<4>(ha1, hb1)}, {dec_i8<5>(ha0, hb0), dec_i8<5>(ha1, hb1)},
+            {dec_i8<6>(ha0, hb0), dec_i8<6>(ha1, hb1)}, {dec_i8<7>(ha0, hb0), dec_i8<7>(ha1, hb1)}};
+#pragma unroll
+        for (int n = 0; n < NG; ++n) {
+          const int col = 8 * n + g;
+          uint32_t xb[8];
+          if (col < ncols) {
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const uint4 v = *reinterpret_cast<const uint4*>(smem + col * RS + half_ofs(2 * w + q));
+              xb[4 * q] = v.x; xb[4 * q + 1] = v.y; xb[4 * q + 2] = v.z; xb[4 * q + 3] = v.w;
+            }
+          } else {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) xb[q] = 0u;
+          }
+#pragma unroll
+          for (int r = 0; r < 8; r += 2) {
+            mma_s8(accL[n], AL[r][0], AL[r][1], AL[r + 1][0], AL[r + 1][1], xb[r], xb[r + 1]);
+            mma_s8(accH[n], AH[r][0], AH[r][1], AH[r + 1][0], AH[r + 1][1], xb[r], xb[r + 1]);
+          }
+        }
+      }
+      // the block's exact sums (acc = 64 * sum), scaled by its s_lo and s_hi, into fp64
+      const int blk = 2 * c + half;
+      const float2 sa = warp_live ? __ldg(sca + blk) : make_float2(0.f, 0.f);
+      const float2 sb = warp_live ? __ldg(scb + blk) : make_float2(0.f, 0.f);
+#pragma unroll
+      for (int n = 0; n < NG; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 s2 = (i >> 1) ? sb : sa;
+          Y[n][i] += (double)s2.x * (double)(accL[n][i] >> 6) + (double)s2.y * (double)(accH[n][i] >> 6);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 6; ++i) cur[i] = nxt[i];
+    load_chunk(c + 2, nxt);
+  }
+  pdl_launch_dependents();
+
+  // ---- epilogue: partial tile [kRows][8 * NG] doubles, then (split K) a cluster-wide sum ----------
+  constexpr int kCols = 8 * NG;
+  double* part = reinterpret_cast<double*>(smem + ncols * RS + (ncols * RS & 1));
+#pragma unroll
+  for (int n = 0; n < NG; ++n)
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      part[(warp * 16 + g + 8 * (i >> 1)) * kCols + 8 * n + 2 * t + (i & 1)] = Y[n][i];
+  cg::cluster_group cluster = cg::this_cluster();
+  if (p.ksplit > 1) cluster.sync(); else __syncthreads();
+  const int rows_per_rank = kRows / p.ksplit;
+  for (int i = threadIdx.x; i < rows_per_rank * p.M; i += kThreads) {
+    const int lrow = ks * rows_per_rank + i / p.M, m = i % p.M;
+    const int row = blockIdx.y * kRows + lrow;
+    if (row >= p.N) continue;
+    double tot = 0.0;
+    for (int r = 0; r < p.ksplit; ++r) {
+      const double* rp = (p.ksplit > 1 ? cluster.map_shared_rank(part, r) : part) + lrow * kCols;
+      if (MODE == 1) {
+        tot += rp[m];
+      } else {
+        const int E = (p.ksplit > 1 ? cluster.map_shared_rank(expo, r) : expo)[m];
+        const double* l = rp + 4 * m;
+        tot += ldexp(((l[0] * 256.0 + l[1]) * 256.0 + l[2]) * 256.0 + l[3], E - kLimbFrac);
+      }
+    }
+    p.y[(size_t)m * p.N + row] = MODE == 1 ? (float)((double)p.sx[m] * tot) : (float)tot;
+  }
+  if (p.ksplit > 1) cluster.sync();
+}
+
+template <int MODE, int NG>
+cudaError_t launch_fv5_one(const Fv5Params& p, size_t smem, cudaStream_t st) {
+  auto kern = k_fv5_gemm<MODE, NG>;
+  static std::atomic<unsigned long long> smem_raised{0};
+  cudaError_t e = allow_max_dynamic_smem(kern, smem_raised);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.ksplit, (p.N + kRows - 1) / kRows, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  int na = 0;
+  if (p.ksplit > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = p.ksplit;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+}  // namespace
+
+size_t fv5_smem_bytes(int mode, int M, int kr) {
+  const int ncols = mode == 0 ? 4 * M : M;
+  const int ng = (ncols + 7) / 8;
+  return (size_t)ncols * (kr / 4 + 16) * 4 + 8 + (size_t)kRows * 8 * ng * 8;
+}
+
+int fv5_rows_per_cta() { return kRows; }
+
+cudaError_t launch_fv5_gemm(const Fv5Params& p, cudaStream_t st) {
+  const int ng = ((p.mode == 0 ? 4 * p.M : p.M) + 7) / 8;
+  const size_t smem = fv5_smem_bytes(p.mode, p.M, p.kr);
+  if (p.mode == 1) return ng == 1 ? launch_fv5_one<1, 1>(p, smem, st) : launch_fv5_one<1, 2>(p, smem, st);
+  switch (ng) {
+    case 1: return launch_fv5_one<0, 1>(p, smem, st);
+    case 2: return launch_fv5_one<0, 2>(p, smem, st);
+    case 3: return launch_fv5_one<0, 3>(p, smem, st);
+    default: return launch_fv5_one<0, 4>(p, smem, st);
+  }
+}
+
+cudaError_t launch_fv5_pack(const int8_t* codes, int32_t N, int32_t K, uint32_t* planes, int32_t* flag,
+                            cudaStream_t st) {
+  const int64_t words = (int64_t)N * (K / 32);
+  const int64_t cap = (int64_t)device_sm_count() * 16;
+  const int64_t blocks = (words + 255) / 256;
+  k_fv5_pack<<<(unsigned)(blocks < cap ? blocks : cap), 256, 0, st>>>(codes, words, K / 32, planes, flag);
+  return cudaGetLastError();
+}
+
+}  // namespace tern

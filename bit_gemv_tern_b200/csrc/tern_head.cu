@@ -19,8 +19,10 @@
 // kept as a packed (order-preserving value key, inverted index) 64-bit word, reduced with
 // shared-memory and then global atomicMax; the last CTA to finish publishes the result and
 // zero-fills the workspace again.
+#include <atomic>
 #include <cooperative_groups.h>
 #include <cstdint>
+#include <type_traits>
 #include <cuda_runtime.h>
 
 #include "tern_device.cuh"
@@ -33,7 +35,9 @@ namespace {
 
 constexpr int kHeadRows = 128;   // rows per row block: 8 warps x 16 rows
 
-template <int MODE, int NG>
+// BS: block-scaled weights (FV5B-style): one fp32 scale per row and 256-weight block instead of the
+// fp16 row scale; the exact int32 sums of each block are scaled into fp64 accumulators.
+template <int MODE, int NG, bool BS>
 __global__ void __launch_bounds__(kThreads, 2) k_head(const HeadParams p) {
   extern __shared__ __align__(16) uint32_t smem[];
   __shared__ unsigned long long best[16];
@@ -125,13 +129,19 @@ __global__ void __launch_bounds__(kThreads, 2) k_head(const HeadParams p) {
   // Let the next kernel of the chain get resident and start its own weight prefetch.
   pdl_launch_dependents();
   constexpr int kCols = 8 * NG;
-  int* part = reinterpret_cast<int*>(smem + ncols * RS);
+  using PT = typename std::conditional<BS, double, int>::type;
+  PT* part = reinterpret_cast<PT*>(smem + ncols * RS + (BS ? ((ncols * RS) & 1) : 0));
   cg::cluster_group cluster = cg::this_cluster();
   const int rows_per_rank = kHeadRows / p.ksplit;
+  const int nblk = p.K >> 8;
   for (; rb < p.nrb; rb += p.nby) {
     int acc[NG][4];
 #pragma unroll
     for (int n = 0; n < NG; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0;
+    double Yb[BS ? NG : 1][4];
+#pragma unroll
+    for (int n = 0; n < (BS ? NG : 1); ++n) Yb[n][0] = Yb[n][1] = Yb[n][2] = Yb[n][3] = 0.0;
+    const int brow0 = min(rb * kHeadRows + warp * 16 + g, p.V - 1), brow1 = min(rb * kHeadRows + warp * 16 + g + 8, p.V - 1);
 
     for (int c = 0; c < nch; ++c) {
 #pragma unroll
@@ -148,6 +158,19 @@ __global__ void __launch_bounds__(kThreads, 2) k_head(const HeadParams p) {
         mma_s8(acc[n], cur[0].z, cur[2].z, cur[0].w, cur[2].w, b0.z, b0.w);
         mma_s8(acc[n], cur[1].x, cur[3].x, cur[1].y, cur[3].y, b1.x, b1.y);
         mma_s8(acc[n], cur[1].z, cur[3].z, cur[1].w, cur[3].w, b1.z, b1.w);
+      }
+      if (BS && (c & 1)) {
+        // a whole 256-weight block: its exact sums times the block's scale, into fp64
+        const int blk = ((k0 + 128 * c) >> 8);
+        const double s0 = (double)__ldg(p.bscale + (size_t)brow0 * nblk + blk);
+        const double s1 = (double)__ldg(p.bscale + (size_t)brow1 * nblk + blk);
+#pragma unroll
+        for (int n = 0; n < (BS ? NG : 1); ++n)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            Yb[n][i] += ((i >> 1) ? s1 : s0) * (double)acc[n][i];
+            acc[n][i] = 0;
+          }
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -169,26 +192,43 @@ __global__ void __launch_bounds__(kThreads, 2) k_head(const HeadParams p) {
     for (int n = 0; n < NG; ++n)
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        part[(warp * 16 + g + 8 * (i >> 1)) * kCols + 8 * n + 2 * t + (i & 1)] = acc[n][i];
+        part[(warp * 16 + g + 8 * (i >> 1)) * kCols + 8 * n + 2 * t + (i & 1)] =
+            BS ? (PT)Yb[BS ? n : 0][i] : (PT)acc[n][i];
     if (p.ksplit > 1) cluster.sync(); else __syncthreads();
 
     for (int i = threadIdx.x; i < rows_per_rank * p.M; i += kThreads) {
       const int lrow = ks * rows_per_rank + i / p.M, m = i % p.M;
       const int row = rb * kHeadRows + lrow;
       if (row >= p.V) continue;
-      const float shv = f16_bits_to_float(p.sh[row]);
       float logit;
-      if (MODE == 1) {
-        int a = 0;
-        for (int r = 0; r < p.ksplit; ++r)
-          a += (p.ksplit > 1 ? cluster.map_shared_rank(part, r) : part)[lrow * kCols + m];
-        logit = __fmul_rn(__fmul_rn(__int2float_rn(a), p.sx[m]), shv);
-      } else {
+      if (BS) {
+        // the fp64 block-scaled sums of every K slice, then one rounding (int8 mode after * s_x)
         double tot = 0.0;
         for (int r = 0; r < p.ksplit; ++r) {
-          const int* rp = (p.ksplit > 1 ? cluster.map_shared_rank(part, r) : part) + lrow * kCols + 4 * m;
+          const PT* rp = (p.ksplit > 1 ? cluster.map_shared_rank(part, r) : part) + lrow * kCols;
+          if (MODE == 1) {
+            tot += (double)rp[m];
+          } else {
+            const int E = (p.ksplit > 1 ? cluster.map_shared_rank(expo, r) : expo)[m];
+            const PT* l = rp + 4 * m;
+            tot += ldexp((((double)l[0] * 256.0 + (double)l[1]) * 256.0 + (double)l[2]) * 256.0 + (double)l[3],
+                         E - kLimbFrac);
+          }
+        }
+        logit = MODE == 1 ? (float)((double)p.sx[m] * tot) : (float)tot;
+      } else if (MODE == 1) {
+        const float shv = f16_bits_to_float(p.sh[row]);
+        int a = 0;
+        for (int r = 0; r < p.ksplit; ++r)
+          a += (int)(p.ksplit > 1 ? cluster.map_shared_rank(part, r) : part)[lrow * kCols + m];
+        logit = __fmul_rn(__fmul_rn(__int2float_rn(a), p.sx[m]), shv);
+      } else {
+        const float shv = f16_bits_to_float(p.sh[row]);
+        double tot = 0.0;
+        for (int r = 0; r < p.ksplit; ++r) {
+          const PT* rp = (p.ksplit > 1 ? cluster.map_shared_rank(part, r) : part) + lrow * kCols + 4 * m;
           const int E = (p.ksplit > 1 ? cluster.map_shared_rank(expo, r) : expo)[m];
-          const long long D = limb_combine(rp[0], rp[1], rp[2], rp[3]);
+          const long long D = limb_combine((long long)rp[0], (long long)rp[1], (long long)rp[2], (long long)rp[3]);
           tot += ldexp((double)D, E - kLimbFrac);
         }
         logit = (float)(tot * (double)shv);
@@ -246,9 +286,9 @@ __global__ void k_verify_accept(const int32_t* argmax, const int32_t* draft, int
   }
 }
 
-template <int MODE, int NG>
+template <int MODE, int NG, bool BS>
 cudaError_t launch_ng(const HeadParams& p, size_t smem, bool pdl, cudaStream_t st) {
-  auto kern = k_head<MODE, NG>;
+  auto kern = k_head<MODE, NG, BS>;
   static std::atomic<unsigned long long> smem_raised{0};
   cudaError_t e = allow_max_dynamic_smem(kern, smem_raised);
   if (e != cudaSuccess) return e;
@@ -278,15 +318,23 @@ cudaError_t launch_ng(const HeadParams& p, size_t smem, bool pdl, cudaStream_t s
 
 template <int MODE>
 cudaError_t launch_mode(const HeadParams& p, int ng, size_t smem, bool pdl, cudaStream_t st) {
+  if (p.bscale) {
+    switch (ng) {
+      case 1: return launch_ng<MODE, 1, true>(p, smem, pdl, st);
+      case 2: return launch_ng<MODE, 2, true>(p, smem, pdl, st);
+      case 3: return launch_ng<MODE, 3, true>(p, smem, pdl, st);
+      default: return launch_ng<MODE, 4, true>(p, smem, pdl, st);
+    }
+  }
   switch (ng) {
-    case 1: return launch_ng<MODE, 1>(p, smem, pdl, st);
-    case 2: return launch_ng<MODE, 2>(p, smem, pdl, st);
-    case 3: return launch_ng<MODE, 3>(p, smem, pdl, st);
-    case 4: return launch_ng<MODE, 4>(p, smem, pdl, st);
-    case 5: return launch_ng<MODE, 5>(p, smem, pdl, st);
-    case 6: return launch_ng<MODE, 6>(p, smem, pdl, st);
-    case 7: return launch_ng<MODE, 7>(p, smem, pdl, st);
-    default: return launch_ng<MODE, 8>(p, smem, pdl, st);
+    case 1: return launch_ng<MODE, 1, false>(p, smem, pdl, st);
+    case 2: return launch_ng<MODE, 2, false>(p, smem, pdl, st);
+    case 3: return launch_ng<MODE, 3, false>(p, smem, pdl, st);
+    case 4: return launch_ng<MODE, 4, false>(p, smem, pdl, st);
+    case 5: return launch_ng<MODE, 5, false>(p, smem, pdl, st);
+    case 6: return launch_ng<MODE, 6, false>(p, smem, pdl, st);
+    case 7: return launch_ng<MODE, 7, false>(p, smem, pdl, st);
+    default: return launch_ng<MODE, 8, false>(p, smem, pdl, st);
   }
 }
 
@@ -300,16 +348,17 @@ cudaError_t launch_verify_accept(const int32_t* argmax, const int32_t* draft, in
   return cudaGetLastError();
 }
 
-size_t head_smem_bytes(int mode, int M, int kr) {
+size_t head_smem_bytes(int mode, int M, int kr, bool block_scaled) {
   const int ncols = mode == 0 ? 4 * M : M;
   const int ng = (ncols + 7) / 8;
-  return (size_t)ncols * (kr / 4 + 4) * 4 + (size_t)kHeadRows * 8 * ng * 4;
+  return (size_t)ncols * (kr / 4 + 4) * 4 + (block_scaled ? 8 : 0) +
+         (size_t)kHeadRows * 8 * ng * (block_scaled ? 8 : 4);
 }
 
 cudaError_t launch_head(const HeadParams& p, bool pdl, cudaStream_t st) {
   const int ncols = p.mode == 0 ? 4 * p.M : p.M;
   const int ng = (ncols + 7) / 8;
-  const size_t smem = head_smem_bytes(p.mode, p.M, p.kr);
+  const size_t smem = head_smem_bytes(p.mode, p.M, p.kr, p.bscale != nullptr);
   return p.mode == 0 ? launch_mode<0>(p, ng, smem, pdl, st) : launch_mode<1>(p, ng, smem, pdl, st);
 }
 

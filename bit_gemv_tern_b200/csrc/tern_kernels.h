@@ -192,6 +192,7 @@ struct HeadParams {
   float* logits;          // optional [M][V]
   unsigned long long* keys;  // workspace: M packed (value key, index) maxima
   unsigned int* counter;     // workspace: CTAs finished
+  const float* bscale;       // block-scaled head (FV5B-style), optional: fp32 [V][K / 256]
   const int32_t* draft;      // verify round, optional: M - 1 drafted tokens
   int32_t* accept;           // verify round: {accepted drafts n, next token argmax[n]}
   int32_t kr, ksplit;
@@ -199,7 +200,7 @@ struct HeadParams {
   int32_t nby;            // CTAs along the row-block axis (persistent loop)
 };
 size_t head_workspace_bytes(int M);
-size_t head_smem_bytes(int mode, int M, int kr);
+size_t head_smem_bytes(int mode, int M, int kr, bool block_scaled);
 cudaError_t launch_head(const HeadParams& p, bool pdl, cudaStream_t st);
 cudaError_t launch_verify_accept(const int32_t* argmax, const int32_t* draft, int32_t k, int32_t* accept,
                                  cudaStream_t st);
@@ -207,7 +208,7 @@ cudaError_t launch_verify_accept(const int32_t* argmax, const int32_t* draft, in
 tern_status plan_head_call(const int8_t* W_dev, const uint16_t* scale_f16_dev, int32_t V, int32_t K, int32_t M,
                            tern_act act, const void* X_dev, const float* x_scale_dev, int32_t* argmax_dev,
                            float* maxval_dev, float* logits_dev, void* workspace_dev, size_t workspace_bytes,
-                           uint32_t flags, HeadParams& p);
+                           uint32_t flags, HeadParams& p, const float* block_scale_dev);
 
 // Loader kernels (tern_pack.cu).
 constexpr int kPackMaxItems = 256;
@@ -236,6 +237,22 @@ cudaError_t launch_unpack_base3(const uint8_t* src, int32_t N, int32_t K, uint32
 cudaError_t launch_encode_base3(const int8_t* src, int32_t N, int32_t K, uint8_t* out, int32_t* flag,
                                 cudaStream_t st);
 cudaError_t launch_occupancy(const uint32_t* planes, int32_t N, int32_t K, int64_t* counts, cudaStream_t st);
+
+// Five-valued weights (tern_fv5.cu).
+struct Fv5Params {
+  const uint32_t* planes;     // [N][3 K / 32]: mask, sign, magnitude planes (words transposed per 512 trits)
+  const float* scales;        // [N][K / 256][2]: s_lo, s_hi
+  int32_t N, K;
+  const void* x;              // bf16 [M][K] or int8 [M][K]
+  const float* sx;            // int8 mode: [M]
+  float* y;                   // [M][N]
+  int32_t M, mode, kr, ksplit;
+};
+size_t fv5_smem_bytes(int mode, int M, int kr);
+int fv5_rows_per_cta();
+cudaError_t launch_fv5_gemm(const Fv5Params& p, cudaStream_t st);
+cudaError_t launch_fv5_pack(const int8_t* codes, int32_t N, int32_t K, uint32_t* planes, int32_t* flag,
+                            cudaStream_t st);
 
 // Order-0 rANS transport (tern_rans.cu).
 struct RansItem {

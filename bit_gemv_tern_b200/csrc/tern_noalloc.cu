@@ -56,7 +56,7 @@ tern_status i8_head_gemv_argmax_noalloc(const int8_t* W_dev, const uint16_t* sca
   if (st != TERN_OK) return st;
   tern::HeadParams p = {};
   st = tern::plan_head_call(W_dev, scale_f16_dev, V, K, M, act, X_dev, x_scale_dev, argmax_dev, maxval_dev,
-                            logits_dev, ws, kScratchBytes, 0u, p);
+                            logits_dev, ws, kScratchBytes, 0u, p, nullptr);
   if (st != TERN_OK) return st;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(ws, 0, need, s) != cudaSuccess) return TERN_ECUDA;

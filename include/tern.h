@@ -48,7 +48,8 @@
  *     tern_gemv_batch, tern_gemm_batch), tern_base3_encode, the rANS transport (tern_rans_*),
  *     tern_occupancy, tern_quantize_act,
  *     the prologues (tern_gemm_batch_pro, tern_act_prologue), the verify round (i8_head_verify,
- *     tern_verify_accept) and i8_head_gemv_argmax_noalloc are additions.
+ *     tern_verify_accept), the five-valued blocks (tern_fv5_*, fv5b_head_gemv_argmax) and
+ *     i8_head_gemv_argmax_noalloc are additions.
  *
  * Packed layout (this library's own; the pages' FV5 bit-planes are only partly described)
  *   Matrix N x K, K a multiple of 128. Row n occupies K/16 uint32 words at word offset n*K/16:
@@ -398,6 +399,49 @@ tern_status i8_head_gemv_argmax_noalloc(const int8_t* W_dev, const uint16_t* sca
                                         int32_t K, int32_t M, tern_act act, const void* X_dev,
                                         const float* x_scale_dev, int32_t* argmax_dev, float* maxval_dev,
                                         float* logits_dev, tern_stream_t stream);
+
+/* Five-valued weights in 256-weight blocks and the block-scaled int8 head: this library's reading of
+ * the pages' shipped FV5 and FV5B types ([R] "FV5와 FV5B: llama.cpp 포크가 공개한 블록 구조":
+ * 256 weights per block, three bitplanes plus fp32 s_lo and s_hi, 3.25 bits per weight; FV5B: int8
+ * with one fp32 scale per block, used for the embedding and output head).
+ *   - A weight is a code c in {-2, -1, 0, +1, +2}: w = 0, sign(c) * s_lo[b] (|c| = 1) or
+ *     sign(c) * s_hi[b] (|c| = 2), b = the weight's 256-weight block of its row. K % 512 == 0.
+ *   - Planes of a row: mask (c != 0), sign (c < 0), high magnitude (|c| = 2), K/32 words each, in
+ *     the ternary layout's bit order (mask and magnitude bit of in-word trit j at p(j), sign bit at
+ *     (p(j) + 1) % 32); inside each group of 16 words (512 trits) of a plane, logical word
+ *     w = 4e + t is stored at position 4t + e. Row n = [mask | sign | magnitude], 3K/32 words.
+ *   - Scales: fp32 [N][K/256][2] = (s_lo, s_hi) of each row and block.
+ *   - Products: exact integer sums per block, scaled per block in fp64 and rounded once to fp32
+ *     (int8 mode: fp32(s_x * sum_b (s_lo A_lo + s_hi A_hi))). bf16 mode keeps the per-output bound
+ *     of the bf16 mode with max(s_lo, s_hi) of the row in place of the row scale. */
+typedef struct {
+  int32_t N, K;                 /* rows, K % 512 == 0                                           */
+  const uint32_t* planes;       /* device, N * 3K/32 words, 16-byte aligned                     */
+  const float* scales;          /* device, N * K/256 * 2 fp32 (s_lo, s_hi), 8-byte aligned      */
+} tern_fv5_matrix;
+
+/* Bytes of FV5 planes for N x K (3NK/8); 0 if the shape is invalid. */
+size_t tern_fv5_packed_bytes(int32_t N, int32_t K);
+
+/* Packs codes int8 [N][K] (values -2..2, 16-byte aligned) into planes_dev (N * 3K/32 words);
+ * err_flag_dev is cleared, then set if a code is outside -2..2. */
+tern_status tern_fv5_pack(const int8_t* codes_dev, int32_t N, int32_t K, uint32_t* planes_dev, int32_t* err_flag_dev,
+                          tern_stream_t stream);
+
+/* Y[m][n] = sum_k w[n][k] X[m][k] for 1 <= M <= 8 (bf16) or 16 (int8) activation rows; X, x_scale
+ * and Y as for tern_gemm_small_m. */
+tern_status tern_fv5_gemm(const tern_fv5_matrix* W, int32_t M, tern_act act, const void* X_dev, const float* x_scale_dev,
+                          float* Y_dev, tern_stream_t stream);
+
+/* The int8 head with one fp32 scale per row and 256-weight block (block_scale_dev: fp32
+ * [V][K/256], 4-byte aligned; K % 256 == 0) instead of the fp16 row scale:
+ *   logits[m][v] = sum_b block_scale[v][b] * sum_{k in b} W[v][k] x[m][k],
+ * argmax with the lowest index on exact ties. bf16 mode M <= 8, int8 mode M <= 16; other
+ * arguments and the workspace as for i8_head_gemv_argmax. */
+tern_status fv5b_head_gemv_argmax(const int8_t* W_dev, const float* block_scale_dev, int32_t V, int32_t K, int32_t M,
+                                  tern_act act, const void* X_dev, const float* x_scale_dev, int32_t* argmax_dev,
+                                  float* maxval_dev, float* logits_dev, void* workspace_dev, size_t workspace_bytes,
+                                  tern_stream_t stream);
 
 /* Synchronise `stream`, read *err_flag_dev and map it: 0 -> TERN_OK, nonzero -> TERN_EBADCODE. */
 tern_status tern_read_flag(const int32_t* err_flag_dev, tern_stream_t stream);
