@@ -65,7 +65,10 @@ class Linear:
         return self.N * self.K // 4 + 2 * self.N + 2 * self.K + 4 * self.N
 
 
-def build_linear(model, layer, projs, seed=SEED):
+def build_linear(model, layer, projs, seed=SEED, interleave=False):
+    """interleave (two projections of equal shape, e.g. gate and up): rows in groups of eight,
+    16j .. 16j + 7 from the first projection's rows 8j .. 8j + 7, then the second's (the layout of
+    the dependent chain's SwiGLU epilogue)."""
     import torch
     import bit_gemv_tern_b200 as tg
     import synth
@@ -81,8 +84,13 @@ def build_linear(model, layer, projs, seed=SEED):
         sc.trits_into(tr[r * K:(r + n) * K], seed, tid, K, synth.trit_probs(model, layer, p))
         scales.append(synth.row_scales(seed, tid, n))
         r += n
+    scale = np.concatenate(scales)
+    if interleave:
+        n = N // 2
+        tr = tr.view(2, n // 8, 8, K).transpose(0, 1).contiguous().view(-1)
+        scale = scale.reshape(2, n // 8, 8).transpose(1, 0, 2).reshape(-1).copy()
     W = tg.TernMatrix.empty(N, K)
-    W.scale.copy_(torch.from_numpy(np.concatenate(scales).view(np.float16)))
+    W.scale.copy_(torch.from_numpy(scale.view(np.float16)))
     flag = torch.zeros(1, dtype=torch.int32, device="cuda")
     tg.tern_pack(tg.TERN_SRC_INT8_TRITS, tr, N, K, W.planes, flag)
     assert tg.tern_read_flag(flag) == 0
@@ -104,7 +112,9 @@ class Stack:
         self.linears, self.x_tid = [], []
         for layer in range(self.L):
             for grp, projs in synth.FUSED_GROUPS:
-                self.linears.append(build_linear(model, layer, projs, seed))
+                # gate|up rows interleaved by eight (the dependent chain fuses SwiGLU into its epilogue;
+                # the independent batches only see the outputs in another order)
+                self.linears.append(build_linear(model, layer, projs, seed, interleave=grp == "gate_up"))
                 self.x_tid.append(synth.act_tensor_id(model, layer, grp))
         htid = synth.head_tensor_id(model)
         self.head_W = torch.empty(self.V * self.d, dtype=torch.int8, device="cuda")
@@ -676,7 +686,7 @@ def extra_rows(stack, torch, tg, hbm_peak, bf16_peak):
     out["8b_stack_m1_int8_prequantised"] = {"tok_s": 1000.0 / ms, "ms": ms, "gbs": gbs_of(nb, ms),
                                             "frac": gbs_of(nb, ms) / hbm_peak}
     # a decode chain whose linears depend on one another through their prologues
-    out["8b_decode_chain_m1_bf16"] = chain_row(stack, torch, hbm_peak)
+    out["8b_decode_chain_m1"] = chain_row(stack, torch, hbm_peak)
     # speculative-verify rounds: k drafts + 1 through the stack and the head with on-device acceptance
     out["verify_round_8b_bf16"] = verify_rows(stack, torch, tg, hbm_peak)
     # decode-chain variant: one launch per fused linear, each waiting for its predecessor (PDL)
@@ -750,12 +760,14 @@ def extra_rows(stack, torch, tg, hbm_peak, bf16_peak):
 
 
 class Chain:
-    """One decode token through the 8B stack as a dependent chain: each fused linear's activation is
-    computed from the previous linear's fp32 output by a prologue fused into that linear's launch.
-    Per layer: q|k|v <- RMSNorm(h); o <- cast(q part of the q|k|v output, standing in for attention,
-    which is not a linear); gate|up <- RMSNorm(o output); down <- SwiGLU(gate|up output); the next
-    layer's h = the down output. The head takes the RMSNorm of the last h. No residual adds (not part
-    of the path). Weights are the stack's; gains and the entry h are seeded synthetic inputs."""
+    """One decode token through the 8B stack as a dependent chain in one cooperative launch
+    (tern_chain_run): each fused linear's activation is computed from an earlier linear's output.
+    Per layer: q|k|v <- RMSNorm(h); o <- cast of the q part of the q|k|v output (standing in for
+    attention, which is not a linear); gate|up <- RMSNorm(o output), its SwiGLU fused into its
+    epilogue (gate and up rows interleaved); down <- that SwiGLU; the next layer's h = the down
+    output. No residual adds (not part of the path). Then the head on the RMSNorm of the last h (a
+    prologue launch and the head launch). Weights are the stack's; gains and the entry h are seeded
+    synthetic inputs."""
 
     def __init__(self, stack, mode="bf16"):
         import torch
@@ -765,25 +777,27 @@ class Chain:
         act = tg.TERN_ACT_BF16 if mode == "bf16" else tg.TERN_ACT_INT8
         d = stack.d
         self.h0 = torch.from_numpy(synth.residual(SEED, 0, 1, d).reshape(-1)).cuda()
-        gains = [torch.from_numpy(synth.norm_gains(SEED, i, d).view(np.int16)).cuda() for i in range(2 * stack.L + 1)]
-        self.gains = gains
-        self.batches = []
+        self.gains = [torch.from_numpy(synth.norm_gains(SEED, i, d).view(np.int16)).cuda() for i in range(2 * stack.L + 1)]
+        self.h = {}
         self.sx = torch.empty(len(stack.linears), dtype=torch.float32, device="cuda")
-        src = self.h0
+        items = []
         for i, lin in enumerate(stack.linears):
             layer, grp = divmod(i, 4)
+            sx = self.sx[i:i + 1] if act == tg.TERN_ACT_INT8 else None
             if grp == 0:
-                pro = (tg.TERN_PRO_RMSNORM, src, gains[2 * layer], 1e-6)
+                it = tg.ChainItem(lin.W, tg.TERN_PRO_RMSNORM, stack.y[i], src_item=i - 1 if i else -1,
+                                  src=None if i else self.h0, gain=self.gains[2 * layer], eps=1e-6, x_scale=sx)
             elif grp == 1:
-                pro = (tg.TERN_PRO_CAST, src, None, 0.0)          # first 4096 values of q|k|v: the q part
+                it = tg.ChainItem(lin.W, tg.TERN_PRO_CAST, stack.y[i], src_item=i - 1, x_scale=sx)
             elif grp == 2:
-                pro = (tg.TERN_PRO_RMSNORM, src, gains[2 * layer + 1], 1e-6)
+                self.h[i] = torch.empty(lin.N // 2, dtype=torch.int16, device="cuda")
+                it = tg.ChainItem(lin.W, tg.TERN_PRO_RMSNORM, stack.y[i], src_item=i - 1, gain=self.gains[2 * layer + 1],
+                                  eps=1e-6, swiglu_out=True, h=self.h[i], x_scale=sx)
             else:
-                pro = (tg.TERN_PRO_SWIGLU, src, None, 0.0)
-            entry = (lin.W, None, self.sx[i:i + 1] if act == tg.TERN_ACT_INT8 else None, stack.y[i])
-            self.batches.append(tg.GemvBatch([entry], act, M=1, prologues=[pro]))
-            src = stack.y[i]
-        self.last = src
+                it = tg.ChainItem(lin.W, tg.TERN_PRO_BF16, stack.y[i], src_item=i - 1, src_h=True, x_scale=sx)
+            items.append(it)
+        self.chain = tg.Chain(items, act)
+        self.last = stack.y[len(stack.linears) - 1]
         self.x_head = torch.empty(d, dtype=torch.int16, device="cuda")
         self.q_head = torch.empty(d, dtype=torch.int8, device="cuda")
         self.sx_head = torch.empty(1, dtype=torch.float32, device="cuda")
@@ -791,8 +805,7 @@ class Chain:
     def launch(self):
         import bit_gemv_tern_b200 as tg
         st = self.stack
-        for b in self.batches:
-            b(flags=tg.TERN_FLAG_PDL)
+        self.chain()
         tg.tern_act_prologue(tg.TERN_PRO_RMSNORM, self.last, self.gains[-1], 1e-6, 1, st.d, self.x_head)
         if self.mode == "bf16":
             tg.i8_head_gemv_argmax(st.head_W, st.head_s, st.V, st.d, 1, tg.TERN_ACT_BF16, self.x_head, None,
@@ -804,23 +817,54 @@ class Chain:
 
     @property
     def launches(self):
-        return 2 * len(self.batches) + 2 + (1 if self.mode == "int8" else 0)
+        return 3 + (1 if self.mode == "int8" else 0)
+
+
+def _timed_direct(fn, n):
+    """fn() launched n times between two events on the current stream; returns elapsed ms."""
+    import torch
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(n):
+        fn()
+    b.record()
+    b.synchronize()
+    return a.elapsed_time(b)
 
 
 def chain_row(stack, torch, hbm_peak):
+    """The dependent decode chain, timed as direct launches (the chain kernel is a cooperative launch;
+    a CUDA graph of it is tried too and reported when capture succeeds)."""
     import bit_gemv_tern_b200 as tg
     out = {}
     for mode in ("bf16", "int8"):
         ch = Chain(stack, mode)
-        g = capture(lambda i: ch.launch(), 5)
-        g.replay()
+        for _ in range(3):
+            ch.launch()
         torch.cuda.synchronize()
         assert tg.tern_device_status() == tg.TERN_OK
-        ms = timed_replays([(g, 4)]) / 20
+        ms = _timed_direct(ch.launch, 50) / 50
+        mc = _timed_direct(ch.chain, 50) / 50
+        assert tg.tern_device_status() == tg.TERN_OK
         nb = stack.stack_bytes + stack.head_bytes
-        out[mode] = {"tok_s": 1000.0 / ms, "ms": ms, "gbs": nb / (ms / 1000.0) / 1e9,
-                     "frac": nb / (ms / 1000.0) / 1e9 / hbm_peak, "launches_per_token": ch.launches}
-        del g, ch
+        row = {"tok_s": 1000.0 / ms, "ms": ms, "gbs": nb / (ms / 1000.0) / 1e9,
+               "frac": nb / (ms / 1000.0) / 1e9 / hbm_peak, "launches_per_token": ch.launches,
+               "chain_kernel_ms": mc, "chain_kernel_frac": stack.stack_bytes / (mc / 1000.0) / 1e9 / hbm_peak,
+               "timing": "direct launches"}
+        try:
+            g = capture(lambda i: ch.launch(), 10)
+            g.replay()
+            torch.cuda.synchronize()
+            mg = timed_replays([(g, 5)]) / 50
+            row["graph_ms"], row["graph_tok_s"] = mg, 1000.0 / mg
+            del g
+        except Exception as e:                    # capture of a cooperative launch refused
+            row["graph"] = "capture failed: %s" % str(e).splitlines()[0][:120]
+            torch.cuda.synchronize()
+        out[mode] = row
+        del ch
     return out
 
 

@@ -25,6 +25,7 @@ __all__ = [
     "GemvBatch", "tern_gemv_batch", "tern_gemv_batch_workspace_bytes", "tern_gemm_batch",
     "tern_gemm_batch_workspace_bytes", "tern_gemm_batch_pro", "tern_act_prologue",
     "i8_head_verify", "tern_verify_accept",
+    "ChainItem", "Chain",
     "Fv5Matrix", "tern_fv5_packed_bytes", "tern_fv5_pack", "tern_fv5_gemm", "fv5b_head_gemv_argmax",
     "tern_rans_payload_bound", "tern_rans_workspace_bytes", "tern_rans_encode", "tern_rans_decode",
     "TERN_PRO_NONE", "TERN_PRO_BF16", "TERN_PRO_CAST", "TERN_PRO_RMSNORM", "TERN_PRO_SWIGLU",
@@ -91,6 +92,9 @@ def lib() -> ctypes.CDLL:
             "tern_act_prologue": ([vp, i32, i32, vp, vp], i32),
             "i8_head_verify": ([vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
             "tern_verify_accept": ([vp, vp, i32, vp, vp], i32),
+            "tern_chain_workspace_bytes": ([vp, i32, i32], sz),
+            "tern_chain_plan": ([vp, i32, i32, vp, sz, vp], i32),
+            "tern_chain_run": ([vp, vp], i32),
             "tern_fv5_packed_bytes": ([i32, i32], sz),
             "tern_fv5_pack": ([vp, i32, i32, vp, vp, vp], i32),
             "tern_fv5_gemm": ([vp, i32, i32, vp, vp, vp, vp], i32),
@@ -255,6 +259,56 @@ def i8_head_verify(W, scale_f16, V: int, K: int, M: int, act: int, X, x_scale, d
 
 def tern_verify_accept(argmax, draft, k: int, accept, stream=None) -> None:
     _check(lib().tern_verify_accept(_ptr(argmax), _ptr(draft), k, _ptr(accept), _stream(stream)), "tern_verify_accept")
+
+
+class _ChainItem(ctypes.Structure):
+    _fields_ = [("W", _Matrix), ("kind", ctypes.c_int32), ("src_item", ctypes.c_int32), ("src_h", ctypes.c_int32),
+                ("swiglu_out", ctypes.c_int32), ("eps", ctypes.c_float), ("src_dev", ctypes.c_void_p),
+                ("gain_dev", ctypes.c_void_p), ("y_dev", ctypes.c_void_p), ("h_dev", ctypes.c_void_p),
+                ("x_scale_dev", ctypes.c_void_p)]
+
+
+class _ChainHandle(ctypes.Structure):
+    _fields_ = [("workspace_dev", ctypes.c_void_p), ("count", ctypes.c_int32), ("mode", ctypes.c_int32),
+                ("grid", ctypes.c_int32), ("stages", ctypes.c_int32), ("smem_bytes", ctypes.c_size_t)]
+
+
+class ChainItem:
+    """One linear of a dependent chain (see tern_chain_item in include/tern.h)."""
+
+    def __init__(self, W: TernMatrix, kind: int, y, src_item: int = -1, src=None, gain=None, eps: float = 0.0,
+                 src_h: bool = False, swiglu_out: bool = False, h=None, x_scale=None):
+        self.W, self.kind, self.y, self.src_item, self.src, self.gain = W, kind, y, src_item, src, gain
+        self.eps, self.src_h, self.swiglu_out, self.h, self.x_scale = eps, src_h, swiglu_out, h, x_scale
+
+
+class Chain:
+    """A planned chain: its workspace and host handle; call() runs it (one cooperative launch)."""
+
+    def __init__(self, items, act: int, device="cuda"):
+        import torch
+        self.items = list(items)
+        arr = (_ChainItem * len(self.items))()
+        for i, it in enumerate(self.items):
+            a = arr[i]
+            a.W = it.W._c
+            a.kind, a.src_item, a.src_h, a.swiglu_out = int(it.kind), int(it.src_item), int(it.src_h), int(it.swiglu_out)
+            a.eps = float(it.eps)
+            a.src_dev, a.gain_dev, a.y_dev = _ptr(it.src), _ptr(it.gain), _ptr(it.y)
+            a.h_dev, a.x_scale_dev = _ptr(it.h), _ptr(it.x_scale)
+        self._arr = arr
+        n = int(lib().tern_chain_workspace_bytes(arr, len(self.items), act))
+        if n == 0:
+            raise TernError(TERN_ESHAPE, "tern_chain_workspace_bytes")
+        self.workspace = torch.empty(n + 64, dtype=torch.uint8, device=device)
+        base = self.workspace.data_ptr()
+        off = (-base) % 64
+        self.handle = _ChainHandle()
+        _check(lib().tern_chain_plan(arr, len(self.items), act, base + off, n, ctypes.byref(self.handle)),
+               "tern_chain_plan")
+
+    def __call__(self, stream=None) -> None:
+        _check(lib().tern_chain_run(ctypes.byref(self.handle), _stream(stream)), "tern_chain_run")
 
 
 class _Fv5Matrix(ctypes.Structure):

@@ -554,6 +554,138 @@ tern_status fv5b_head_gemv_argmax(const int8_t* W_dev, const float* block_scale_
   return from_cuda(tern::launch_head(p, false, cs(stream)));
 }
 
+namespace {
+
+// Workspace layout of a chain: [items (64-byte aligned)][done counters][finished][scratch].
+struct ChainWs {
+  size_t items, done, finished, scratch, total;
+};
+ChainWs chain_ws(int count, size_t scratch_words) {
+  ChainWs w;
+  w.items = 0;
+  w.done = ((size_t)count * sizeof(tern::ChainItem) + 63) & ~(size_t)63;
+  w.finished = w.done + (((size_t)count * 4 + 63) & ~(size_t)63);
+  w.scratch = w.finished + 64;
+  w.total = w.scratch + scratch_words * 4;
+  return w;
+}
+
+// Checks and converts the items (check_ptrs false: shapes and sources only).
+tern_status chain_items(const tern_chain_item* items, int32_t count, tern_act act, bool check_ptrs, tern::ChainItem* out,
+                        const uint32_t** planes) {
+  if (!items) return TERN_EINVAL;
+  if (act != TERN_ACT_BF16 && act != TERN_ACT_INT8) return TERN_EINVAL;
+  if (count < 1 || count > TERN_CHAIN_MAX_ITEMS) return TERN_ESHAPE;
+  for (int i = 0; i < count; ++i) {
+    const tern_chain_item& in = items[i];
+    if (check_ptrs) {
+      tern_status st = check_matrix(&in.W);
+      if (st != TERN_OK) return st;
+    } else if (!valid_shape(in.W.N, in.W.K)) {
+      return TERN_ESHAPE;
+    }
+    if (in.W.K > 12288) return TERN_ESHAPE;
+    if (in.kind != TERN_PRO_BF16 && in.kind != TERN_PRO_CAST && in.kind != TERN_PRO_RMSNORM) return TERN_EINVAL;
+    if (in.src_item >= i || in.src_item < -1) return TERN_EINVAL;
+    if (in.swiglu_out && in.W.N % 16) return TERN_ESHAPE;
+    if (in.src_item >= 0) {
+      const tern_chain_item& d = items[in.src_item];
+      if (in.src_h) {
+        if (!d.swiglu_out || in.kind != TERN_PRO_BF16) return TERN_EINVAL;
+        if (d.W.N / 2 < in.W.K) return TERN_ESHAPE;
+      } else {
+        if (in.kind == TERN_PRO_BF16) return TERN_EINVAL;          // a y source is fp32
+        if (d.W.N < in.W.K) return TERN_ESHAPE;
+      }
+    }
+    if (check_ptrs) {
+      if (in.src_item < 0 && (!in.src_dev || !aligned(in.src_dev, 16))) return TERN_EINVAL;
+      if (in.kind == TERN_PRO_RMSNORM &&
+          (!in.gain_dev || !aligned(in.gain_dev, 16) || !(in.eps >= 0.0f) || in.eps > 3.0e38f))
+        return TERN_EINVAL;
+      if (!in.y_dev || !aligned(in.y_dev, 16)) return TERN_EINVAL;
+      if (in.swiglu_out && (!in.h_dev || !aligned(in.h_dev, 16))) return TERN_EINVAL;
+      if (in.x_scale_dev && !aligned(in.x_scale_dev, 4)) return TERN_EINVAL;
+    }
+    if (out) {
+      tern::ChainItem& c = out[i];
+      c = tern::ChainItem{};
+      planes[i] = in.W.planes;
+      c.scale = in.W.scale_f16;
+      c.y = in.y_dev;
+      c.hout = in.swiglu_out ? in.h_dev : nullptr;
+      c.sx_out = act == TERN_ACT_INT8 ? in.x_scale_dev : nullptr;
+      c.src = in.src_item < 0 ? in.src_dev
+                              : (in.src_h ? static_cast<const void*>(items[in.src_item].h_dev)
+                                          : static_cast<const void*>(items[in.src_item].y_dev));
+      c.gain = in.gain_dev;
+      c.eps = in.eps;
+      c.kind = in.kind;
+      c.dep = in.src_item;
+      c.N = in.W.N;
+      c.K = in.W.K;
+    }
+  }
+  return TERN_OK;
+}
+
+}  // namespace
+
+size_t tern_chain_workspace_bytes(const tern_chain_item* items, int32_t count, tern_act act) {
+  if (chain_items(items, count, act, false, nullptr, nullptr) != TERN_OK) return 0;
+  size_t scratch = 0;
+  for (int i = 0; i < count; ++i) {
+    const int units = (items[i].W.N + 383) / 384;
+    scratch += (size_t)units * 384 * 8 + (size_t)units * 12;
+  }
+  return chain_ws(count, scratch).total;
+}
+
+tern_status tern_chain_plan(const tern_chain_item* items, int32_t count, tern_act act, void* workspace_dev,
+                            size_t workspace_bytes, tern_chain* chain) {
+  if (!chain || !workspace_dev || !aligned(workspace_dev, 64)) return TERN_EINVAL;
+  tern::ChainItem* host = new (std::nothrow) tern::ChainItem[count > 0 && count <= TERN_CHAIN_MAX_ITEMS ? count : 1];
+  const uint32_t** planes = new (std::nothrow) const uint32_t*[count > 0 && count <= TERN_CHAIN_MAX_ITEMS ? count : 1];
+  tern_status st = (host && planes) ? chain_items(items, count, act, true, host, planes) : TERN_EINVAL;
+  tern::ChainLayout L = {};
+  if (st == TERN_OK && !tern::plan_chain(host, count, act == TERN_ACT_BF16 ? 0 : 1, planes, L)) st = TERN_ESHAPE;
+  ChainWs w = chain_ws(count > 0 ? count : 1, L.scratch_words);
+  if (st == TERN_OK && workspace_bytes < w.total) st = TERN_EINVAL;
+  if (st == TERN_OK) {
+    uint8_t* ws = static_cast<uint8_t*>(workspace_dev);
+    if (cudaMemcpy(ws + w.items, host, (size_t)count * sizeof(tern::ChainItem), cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemset(ws + w.done, 0, w.total - w.done) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
+      st = TERN_ECUDA;
+  }
+  if (st == TERN_OK) {
+    chain->workspace_dev = workspace_dev;
+    chain->count = count;
+    chain->mode = act == TERN_ACT_BF16 ? 0 : 1;
+    chain->grid = tern::chain_grid();
+    chain->stages = L.stages;
+    chain->smem_bytes = L.smem;
+  }
+  delete[] host;
+  delete[] planes;
+  return st;
+}
+
+tern_status tern_chain_run(const tern_chain* chain, tern_stream_t stream) {
+  if (!chain || !chain->workspace_dev || chain->count < 1 || chain->grid < 1 || chain->stages < 2) return TERN_EINVAL;
+  const ChainWs w = chain_ws(chain->count, 0);
+  uint8_t* ws = static_cast<uint8_t*>(chain->workspace_dev);
+  tern::ChainParams p = {};
+  p.items = reinterpret_cast<const tern::ChainItem*>(ws + w.items);
+  p.count = chain->count;
+  p.mode = chain->mode;
+  p.grid = chain->grid;
+  p.stages = chain->stages;
+  p.done = reinterpret_cast<int32_t*>(ws + w.done);
+  p.finished = reinterpret_cast<int32_t*>(ws + w.finished);
+  p.scratch = reinterpret_cast<int32_t*>(ws + w.scratch);
+  return from_cuda(tern::launch_chain(p, chain->smem_bytes, cs(stream)));
+}
+
 tern_status tern_read_flag(const int32_t* err_flag_dev, tern_stream_t stream) {
   if (!err_flag_dev) return TERN_EINVAL;
   if (cudaStreamSynchronize(cs(stream)) != cudaSuccess) return TERN_ECUDA;
@@ -563,11 +695,12 @@ tern_status tern_read_flag(const int32_t* err_flag_dev, tern_stream_t stream) {
 }
 
 tern_status tern_device_status(tern_stream_t stream) {
-  int v = 0, w = 0, x = 0;
+  int v = 0, w = 0, x = 0, c = 0;
   if (tern::read_and_clear_error_latch(&v, cs(stream)) != cudaSuccess) return TERN_ECUDA;
   if (tern::read_and_clear_batch_latch(&w) != cudaSuccess) return TERN_ECUDA;
   if (tern::read_and_clear_prefill_latch(&x) != cudaSuccess) return TERN_ECUDA;
-  return (v == 0 && w == 0 && x == 0) ? TERN_OK : TERN_ETIMEOUT;
+  if (tern::read_and_clear_chain_latch(&c) != cudaSuccess) return TERN_ECUDA;
+  return (v == 0 && w == 0 && x == 0 && c == 0) ? TERN_OK : TERN_ETIMEOUT;
 }
 
 tern_status tern_gemm_prefill(const tern_matrix* W, int32_t M, const uint16_t* X_bf16_dev, float* Y_dev,

@@ -238,6 +238,40 @@ cudaError_t launch_encode_base3(const int8_t* src, int32_t N, int32_t K, uint8_t
                                 cudaStream_t st);
 cudaError_t launch_occupancy(const uint32_t* planes, int32_t N, int32_t K, int64_t* counts, cudaStream_t st);
 
+// Dependent decode chain in one cooperative launch (tern_chain.cu). The plan (this array) lives in
+// device memory; tensor maps need 64-byte alignment there.
+struct alignas(64) ChainItem {
+  CUtensorMap tmap;           // planes as [plane 2][row N][word K/32]
+  const uint16_t* scale;      // fp16 [N]
+  float* y;                   // fp32 [N]
+  uint16_t* hout;             // SwiGLU output bf16 [N / 2] (rows interleave gate and up by 8), or null
+  float* sx_out;              // int8 mode: s_x of this linear's activation, or null
+  const void* src;            // the activation's source: bf16 [K] (kProBF16) or fp32 [K]
+  const uint16_t* gain;       // kProRMSNorm: bf16 [K]
+  float eps;
+  int32_t kind;               // kProBF16, kProCast or kProRMSNorm
+  int32_t dep;                // linear whose outputs src holds (-1: written before the launch)
+  int32_t N, K, kp, units;
+  uint32_t scratch_off;       // int32 words: split-block sums [units][384][8]
+  uint32_t counter_off;       // int32 words: split-block counters [units][12]
+};
+struct ChainParams {
+  const ChainItem* items;     // device
+  int32_t count, mode, grid, stages;
+  int32_t* done;              // device: completion counter of each linear [count]
+  int32_t* finished;          // device: CTAs finished with the whole chain
+  int32_t* scratch;           // device: split-block sums and counters
+};
+struct ChainLayout {
+  int stages;
+  size_t smem;
+  size_t scratch_words;
+};
+bool plan_chain(ChainItem* items, int count, int mode, const uint32_t* const* planes, ChainLayout& L);
+cudaError_t launch_chain(const ChainParams& p, size_t smem, cudaStream_t st);
+int chain_grid();
+cudaError_t read_and_clear_chain_latch(int* out);
+
 // Five-valued weights (tern_fv5.cu).
 struct Fv5Params {
   const uint32_t* planes;     // [N][3 K / 32]: mask, sign, magnitude planes (words transposed per 512 trits)

@@ -48,8 +48,8 @@
  *     tern_gemv_batch, tern_gemm_batch), tern_base3_encode, the rANS transport (tern_rans_*),
  *     tern_occupancy, tern_quantize_act,
  *     the prologues (tern_gemm_batch_pro, tern_act_prologue), the verify round (i8_head_verify,
- *     tern_verify_accept), the five-valued blocks (tern_fv5_*, fv5b_head_gemv_argmax) and
- *     i8_head_gemv_argmax_noalloc are additions.
+ *     tern_verify_accept), the five-valued blocks (tern_fv5_*, fv5b_head_gemv_argmax), the dependent chain
+ *     (tern_chain_*) and i8_head_gemv_argmax_noalloc are additions.
  *
  * Packed layout (this library's own; the pages' FV5 bit-planes are only partly described)
  *   Matrix N x K, K a multiple of 128. Row n occupies K/16 uint32 words at word offset n*K/16:
@@ -399,6 +399,56 @@ tern_status i8_head_gemv_argmax_noalloc(const int8_t* W_dev, const uint16_t* sca
                                         int32_t K, int32_t M, tern_act act, const void* X_dev,
                                         const float* x_scale_dev, int32_t* argmax_dev, float* maxval_dev,
                                         float* logits_dev, tern_stream_t stream);
+
+/* A decode step's chain of dependent linear layers in one cooperative launch (M = 1). The pages put
+ * the time above a decode step's DRAM floor in the dependency chains between its ~120 kernels
+ * ([R] "뉴트리노 엔진: 토큰 하나의 시간은 어디로 가는가"); here every linear of the chain runs in one
+ * persistent kernel whose weight stream continues across the linears while each linear waits for
+ * the one it reads. Item i's activation is its prologue (as for tern_gemm_batch_pro) applied to:
+ *   src_item < 0:  src_dev, written before the launch;
+ *   src_item = j:  item j's fp32 output y (kinds TERN_PRO_CAST, TERN_PRO_RMSNORM: its first K
+ *                  values), or, with src_h = 1 (kind TERN_PRO_BF16), item j's SwiGLU output h.
+ * An item with swiglu_out = 1 has its rows interleaved in groups of eight: rows 16j .. 16j + 7 are
+ * gate rows 8j .. 8j + 7 and rows 16j + 8 .. 16j + 15 the matching up rows (N % 16 == 0); besides y it
+ * writes h[8j + i] = bf16(silu(y[16j + i]) * y[16j + 8 + i]) (silu(z) = z / (1 + e^-z), fp64, one
+ * rounding) -- the SwiGLU of the gate|up output, fused into its epilogue.
+ * Outputs equal tern_gemm_batch_pro's for the same prologue and source, bit for bit, in both modes. */
+typedef struct {
+  tern_matrix W;                /* K <= 12288                                                     */
+  int32_t kind;                 /* TERN_PRO_BF16, TERN_PRO_CAST or TERN_PRO_RMSNORM              */
+  int32_t src_item;             /* an earlier item, or -1                                         */
+  int32_t src_h;                /* 1: the source is item src_item's SwiGLU output h               */
+  int32_t swiglu_out;           /* 1: interleaved gate|up rows; h_dev receives the SwiGLU        */
+  float eps;                    /* TERN_PRO_RMSNORM                                               */
+  const void* src_dev;          /* src_item < 0: bf16 [K] (BF16) or fp32 [K], 16-byte aligned     */
+  const uint16_t* gain_dev;     /* TERN_PRO_RMSNORM: bf16 [K], 16-byte aligned                   */
+  float* y_dev;                 /* fp32 [N], 16-byte aligned                                      */
+  uint16_t* h_dev;              /* swiglu_out: bf16 [N / 2], 16-byte aligned                      */
+  float* x_scale_dev;           /* int8 mode, optional output: s_x of this item's activation      */
+} tern_chain_item;
+
+/* Host handle of a planned chain (filled by tern_chain_plan; owned by the caller). */
+typedef struct {
+  void* workspace_dev;
+  int32_t count, mode, grid, stages;
+  size_t smem_bytes;
+} tern_chain;
+
+#define TERN_CHAIN_MAX_ITEMS 4096
+
+/* Workspace bytes of a chain (0 if the list is invalid; pointers are not checked). */
+size_t tern_chain_workspace_bytes(const tern_chain_item* items, int32_t count, tern_act act);
+
+/* Checks the items, writes the chain's plan (tensor maps, per-linear shapes and sources) into
+ * workspace_dev (64-byte aligned, at least tern_chain_workspace_bytes) and clears its counters and
+ * scratch. Synchronous (blocking copies): call it once, before any stream capture. */
+tern_status tern_chain_plan(const tern_chain_item* items, int32_t count, tern_act act, void* workspace_dev,
+                            size_t workspace_bytes, tern_chain* chain);
+
+/* Runs the planned chain on `stream` (one cooperative launch: one CTA per SM, all resident). The
+ * workspace is left ready for the next run; two runs of one workspace must not overlap in time. A
+ * wait that gives up latches TERN_ETIMEOUT (tern_device_status) and the outputs are incomplete. */
+tern_status tern_chain_run(const tern_chain* chain, tern_stream_t stream);
 
 /* Five-valued weights in 256-weight blocks and the block-scaled int8 head: this library's reading of
  * the pages' shipped FV5 and FV5B types ([R] "FV5와 FV5B: llama.cpp 포크가 공개한 블록 구조":
