@@ -314,31 +314,32 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------------------------
-def _oracle_sample(rows=256):
-    """Inputs for the CPU oracle: `rows` rows of each fused 8B launch and 4x as many head rows."""
+def _oracle_sample(rows=256, model="8b"):
+    """Inputs for the CPU oracle: `rows` rows of each fused launch of `model` and 4x as many head
+    rows."""
     import oracle
     import synth
-    shapes = {p: (N, K) for p, N, K in synth.linear_shapes("8b")}
+    shapes = {p: (N, K) for p, N, K in synth.linear_shapes(model)}
     fused = [(grp, sum(shapes[p][0] for p in projs), shapes[projs[0]][1]) for grp, projs in synth.FUSED_GROUPS]
     mats = []
     for grp, N, K in fused:
         t = synth.trits(SEED, 9000 + K, rows, K)
         mats.append((grp, N, K, oracle.pack(t), synth.row_scales(SEED, 9000 + K, rows),
                      synth.activations(SEED, 9000 + K, 1, K)))
-    d = synth.GEOMETRY["8b"]["d"]
+    d = synth.GEOMETRY[model]["d"]
     head = (synth.head_weights(SEED, 9999, 4 * rows, d), synth.head_scales(SEED, 9999, 4 * rows),
             synth.activations(SEED, 9999, 1, d))
-    return mats, head, rows
+    return mats, head, rows, model
 
 
 def _oracle_token_seconds(sample, threads, budget_s):
     """Time the oracle on the sample (repeating calls until budget_s is spent) and scale by rows to
-    one 8B token: 36 layers x 4 fused launches + the 151936-row head. Returns (s/token, s measured)."""
+    one token of the sample's model: layers x 4 fused launches + the vocabulary-row head.
+    Returns (s/token, s measured)."""
     import oracle
     import synth
-    mats, head, rows = sample
-    L, V = synth.GEOMETRY["8b"]["layers"], synth.GEOMETRY["8b"]["vocab"]
-    per_row = {}
+    mats, head, rows, model = sample
+    L, V = synth.GEOMETRY[model]["layers"], synth.GEOMETRY[model]["vocab"]
     spent, reps = 0.0, 0
     tot = {}
     while True:
@@ -361,15 +362,60 @@ def _oracle_token_seconds(sample, threads, budget_s):
     return t_token, spent
 
 
+def token_bytes(model):
+    """Algorithmic bytes of one M = 1 token of `model`: per fused linear the packed planes N*K/4,
+    the fp16 scales 2N, the bf16 activation 2K and the fp32 outputs 4N; the int8 head V*d + 2V
+    (+ its activation and result)."""
+    import synth
+    g = synth.GEOMETRY[model]
+    shapes = {p: (N, K) for p, N, K in synth.linear_shapes(model)}
+    b = 0
+    for _, projs in synth.FUSED_GROUPS:
+        N, K = sum(shapes[p][0] for p in projs), shapes[projs[0]][1]
+        b += N * K // 4 + 2 * N + 2 * K + 4 * N
+    return g["layers"] * b + g["vocab"] * g["d"] + 2 * g["vocab"] + 2 * g["d"] + 8
+
+
+def _oracle_gemv_seconds(threads, budget_s):
+    """The oracle on the whole single-GEMV workload (N = 3072, K = 1024, M = 1), repeated until
+    budget_s is spent; returns s per GEMV."""
+    import oracle
+    import synth
+    N, K = 3072, 1024
+    pl = oracle.pack(synth.trits(SEED, 1, N, K))
+    s, x = synth.row_scales(SEED, 1, N), synth.activations(SEED, 1, 1, K)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.gemm_bf16(pl, s, K, x, nthreads=threads)
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    return (time.perf_counter() - t0) / reps
+
+
 def cpu_baseline(budget_s=12.0):
-    """The oracle on this host's cores on a bounded sample of the 8B token, scaled to tok/s."""
+    """The oracle on this host's cores on a bounded sample of the 8B token, scaled to tok/s; with
+    the same on one thread and the oracle's GB/s (the workload's algorithmic bytes over its time)
+    for the single GEMV, the 0.6B token and the 8B token."""
     threads = os.cpu_count() or 1
     sample = _oracle_sample()
     t_token, spent = _oracle_token_seconds(sample, threads, budget_s)
+    t_token_1, spent_1 = _oracle_token_seconds(sample, 1, budget_s / 3)
+    t_06, spent_06 = _oracle_token_seconds(_oracle_sample(model="0.6b"), threads, budget_s / 4)
+    t_gemv = _oracle_gemv_seconds(threads, 1.0)
+    gemv_bytes = 3072 * 1024 // 4 + 2 * 3072 + 2 * 1024 + 4 * 3072
+    per_config = {
+        "gemv_3072x1024_m1": {"gbs": gemv_bytes / t_gemv / 1e9, "us_per_call": t_gemv * 1e6},
+        "0.6b_token_m1": {"gbs": token_bytes("0.6b") / t_06 / 1e9, "tok_s": 1.0 / t_06},
+        "8b_token_m1": {"gbs": token_bytes("8b") / t_token / 1e9, "tok_s": 1.0 / t_token,
+                        "gbs_1thread": token_bytes("8b") / t_token_1 / 1e9, "tok_s_1thread": 1.0 / t_token_1},
+    }
     return {"value": 1.0 / t_token, "unit": "tok/s", "cores": threads, "kind": "oracle",
+            "value_1thread": 1.0 / t_token_1, "per_config": per_config,
             "sample": f"{sample[2]} rows of each fused 8B launch (q|k|v, o, gate|up, down; full K) and "
-                      f"{4 * sample[2]} head rows (K=4096), fp64 oracle, calls repeated for {spent:.1f} s, "
-                      f"per-row time scaled to 36 layers + the 151936-row head"}
+                      f"{4 * sample[2]} head rows (K=4096), fp64 oracle, calls repeated for {spent:.1f} s "
+                      f"({spent_1:.1f} s on 1 thread), per-row time scaled to 36 layers + the 151936-row head; "
+                      f"0.6B the same at its widths ({spent_06:.1f} s); the single GEMV whole"}
 
 
 # ---------------------------------------------------------------------------------------------

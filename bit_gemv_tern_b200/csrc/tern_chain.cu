@@ -113,6 +113,17 @@ __device__ __forceinline__ int part_slot(int w) { return ((w & 3) * 4 + (w >> 2)
 // CTA range of a linear with P units over G CTAs: [P c / G, P (c + 1) / G); the CTA owning unit p.
 __device__ __forceinline__ int range_start(int P, int G, int c) { return (int)((long long)P * c / G); }
 __device__ __forceinline__ int owner(int P, int G, int p) { return (int)(((long long)(p + 1) * G - 1) / P); }
+// Number of CTAs that own units of [b0, b1): owners are nondecreasing in the unit index, but with
+// fewer units than CTAs the CTAs between two owners own none, so count the distinct owners.
+__device__ __forceinline__ int contributors(int P, int G, int b0, int b1) {
+  int n = 1, o = owner(P, G, b0);
+  for (int u = b0 + 1; u < b1; ++u) {
+    const int v = owner(P, G, u);
+    n += v != o;
+    o = v;
+  }
+  return n;
+}
 
 // 8 bf16 values (k .. k+7) of the linear's activation row, computed from its source with the
 // prologue's arithmetic; sources written during the launch are read through L2.
@@ -261,7 +272,7 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 1) k_chain(const ChainParams p
         sh_E = limb_exponent(mx);
       } else {
         sh_sx = __fdiv_rn(mx, 127.0f);
-        if (c == 0 && it.sx_out) it.sx_out[0] = sh_sx;
+        if (p0 == 0 && it.sx_out) it.sx_out[0] = sh_sx;     // the CTA holding unit 0
       }
     }
     consumers_sync();
@@ -315,7 +326,7 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 1) k_chain(const ChainParams p
     for (int u = p0; u < p1 && ok;) {
       const int rb = u / kp;
       const int pend = min(p1, (rb + 1) * kp);                  // this CTA's parts of the block: [u, pend)
-      const int need = owner(P, G, (rb + 1) * kp - 1) - owner(P, G, rb * kp) + 1;
+      const int need = contributors(P, G, rb * kp, (rb + 1) * kp);
       const int row_base = rb * kStageRows + warp * 16;
       int acc[kTPW][4];
 #pragma unroll

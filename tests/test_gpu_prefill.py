@@ -36,13 +36,14 @@ def test_prefill_full(N, K, M):
 
 @pytest.mark.parametrize("proj", ["q", "k", "o", "gate", "down"])
 def test_prefill_8b_shapes_sampled_tokens(proj):
-    """M = 4096 tokens through an 8B linear shape; 24 sampled tokens checked against every row."""
+    """M = 4096 tokens through an 8B linear shape; 64 sampled tokens (the first and the last among
+    them) checked against every row."""
     N, K = {p: (n, k) for p, n, k in synth.linear_shapes("8b")}[proj]
     M = 4096
     W, t, s = make_matrix(52, 7000 + N + K, N, K, host_trits=False)
     X = synth.activations(52, N + K, M, K)
     Y = _prefill(W, X)
-    toks = np.sort(np.random.default_rng(N + K).choice(M, 24, replace=False))
+    toks = np.sort(np.random.default_rng(N + K).choice(M, 64, replace=False))
     toks[0], toks[-1] = 0, M - 1
     tr = synth.trits(52, 7000 + N + K, N, K)
     check_bf16(Y[toks], oracle.gemm_bf16(oracle.pack(tr), s, K, X[toks]), X[toks], s)
