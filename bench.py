@@ -778,17 +778,7 @@ def extra_rows(stack, torch, tg, hbm_peak, bf16_peak):
     del s06
 
     # small-M sweep on the 8B stack + head (speculative verify)
-    sweep = {}
-    for M in (1, 2, 4, 7, 8, 16):
-        sm = stack if M == 1 else StackView(stack, M)
-        g = capture(lambda i: (sm.launch_stack("bf16"), sm.launch_head("bf16")), 5)
-        g.replay()
-        ms = timed_replays([(g, 4)]) / 20
-        nb = sm.stack_bytes + sm.head_bytes
-        sweep[str(M)] = {"pass_us": ms * 1000.0, "tokens_per_s": M * 1000.0 / ms, "gbs": gbs_of(nb, ms),
-                         "frac": gbs_of(nb, ms) / hbm_peak, "launches_per_pass": 3}
-        del g
-    out["small_m_8b_bf16"] = sweep
+    out["small_m_8b_bf16"] = small_m_sweep(stack, hbm_peak)
 
     # prefill: M = 4096 tokens through each of the 7 distinct 8B linear shapes (tcgen05)
     out["prefill_8b_m4096"] = prefill_row(torch, tg, bf16_peak)
@@ -914,6 +904,33 @@ def chain_row(stack, torch, hbm_peak):
     return out
 
 
+def small_m_sweep(stack, hbm_peak, Ms=(1, 2, 3, 4, 5, 7, 8, 12, 16)):
+    """One pass of M rows through the 8B stack + head per M. From bf16 M >= 3 the stack runs on the
+    tcgen05 kernels; the same pass on the mma.sync kernels is timed beside it."""
+    out = {}
+    for M in Ms:
+        sm = stack if M == 1 else StackView(stack, M)
+        row = {}
+        for name, mma_sync in (("", False), ("mma_sync_", True)):
+            if mma_sync and M < 3:
+                continue
+            if M == 1:
+                g = capture(lambda i: (sm.launch_stack("bf16"), sm.launch_head("bf16")), 5)
+            else:
+                g = capture(lambda i: (sm.launch_stack("bf16", mma_sync=mma_sync), sm.launch_head("bf16")), 5)
+            g.replay()
+            ms = timed_replays([(g, 4)]) / 20
+            nb = sm.stack_bytes + sm.head_bytes
+            row[name + "pass_us"] = ms * 1000.0
+            row[name + "frac"] = gbs_of(nb, ms) / hbm_peak
+            if not name:
+                row.update({"tokens_per_s": M * 1000.0 / ms, "gbs": gbs_of(nb, ms), "launches_per_pass": 3,
+                            "kernel": "tcgen05" if M >= 3 else "mma.sync"})
+            del g
+        out[str(M)] = row
+    return out
+
+
 def verify_rows(stack, torch, tg, hbm_peak):
     """k drafted tokens + 1 through the 8B stack (one small-M batch) and the head with the acceptance
     count on the device. Drafts equal to the target's own greedy tokens (from a previous pass) give
@@ -1013,13 +1030,14 @@ class StackView:
     stack_bytes = Stack.stack_bytes
     head_bytes = Stack.head_bytes
 
-    def launch_stack(self, mode="bf16", pdl=False):
-        """All 144 fused linears as one batched small-M launch pair (each reads its X [M][K])."""
+    def launch_stack(self, mode="bf16", pdl=False, mma_sync=False):
+        """All 144 fused linears as one batched small-M launch pair (each reads its X [M][K]);
+        mma_sync: the warp-level MMA kernels instead of the tcgen05 ones."""
         import bit_gemv_tern_b200 as tg
         if not hasattr(self, "_batch"):
             entries = [(lin.W, self.x[:self.M * lin.K], None, self.y[i]) for i, lin in enumerate(self.linears)]
             self._batch = tg.GemvBatch(entries, tg.TERN_ACT_BF16, M=self.M)
-        self._batch(flags=tg.TERN_FLAG_PDL if pdl else 0)
+        self._batch(flags=(tg.TERN_FLAG_PDL if pdl else 0) | (tg.TERN_FLAG_MMA_SYNC if mma_sync else 0))
 
     def launch_head(self, mode="bf16", pdl=False):
         import bit_gemv_tern_b200 as tg

@@ -320,14 +320,25 @@ namespace {
 
 // Validates a list (and its prologues, if any) and plans both launches. With check_ptrs false
 // only the shapes and modes are checked (the workspace query).
+// The tensor-core (tcgen05) small-M kernels take lists of M rows from these sizes on, without
+// prologues, unless the caller asks for the mma.sync kernels.
+bool use_tc(const tern_prologue* pro, int32_t count, int32_t M, tern_act act, uint32_t flags) {
+  if (flags & TERN_FLAG_MMA_SYNC) return false;
+  if (pro)
+    for (int i = 0; i < count; ++i)
+      if (pro[i].kind != TERN_PRO_NONE) return false;
+  return act == TERN_ACT_BF16 ? M >= 3 : M >= 5;
+}
+
 tern_status fill_batch(const tern_gemv_item* items, const tern_prologue* pro, int32_t count, int32_t M, tern_act act,
-                       bool check_ptrs, tern::BatchParams& bp, tern::PrepParams& pp, size_t& smem, size_t& ws) {
+                       bool check_ptrs, bool tc, tern::BatchParams& bp, tern::PrepParams& pp, size_t& smem, size_t& ws) {
   if (!items) return TERN_EINVAL;
   if (act != TERN_ACT_BF16 && act != TERN_ACT_INT8) return TERN_EINVAL;
   if (count < 1 || count > TERN_BATCH_MAX_ITEMS || M < 1 || M > 16) return TERN_ESHAPE;
   bp.count = count;
   bp.M = M;
   bp.mode = act == TERN_ACT_BF16 ? 0 : 1;
+  bp.tc = tc ? 1 : 0;
   const uint32_t* planes[TERN_BATCH_MAX_ITEMS];
   for (int i = 0; i < count; ++i) {
     const tern_gemv_item& in = items[i];
@@ -384,13 +395,14 @@ tern_status fill_batch(const tern_gemv_item* items, const tern_prologue* pro, in
 
 tern_status run_batch(const tern_gemv_item* items, const tern_prologue* pro, int32_t count, int32_t M, tern_act act,
                       void* workspace_dev, size_t workspace_bytes, uint32_t flags, tern_stream_t stream) {
-  if (flags & ~TERN_FLAG_PDL) return TERN_EINVAL;
+  if (flags & ~(TERN_FLAG_PDL | TERN_FLAG_MMA_SYNC)) return TERN_EINVAL;
   if (!workspace_dev || !aligned(workspace_dev, 16)) return TERN_EINVAL;
   tern::BatchParams* bp = new (std::nothrow) tern::BatchParams();
   tern::PrepParams* pp = new (std::nothrow) tern::PrepParams();
   tern_status st = (bp && pp) ? TERN_OK : TERN_EINVAL;
   size_t smem = 0, ws = 0;
-  if (st == TERN_OK) st = fill_batch(items, pro, count, M, act, true, *bp, *pp, smem, ws);
+  if (st == TERN_OK)
+    st = fill_batch(items, pro, count, M, act, true, use_tc(pro, count, M, act, flags), *bp, *pp, smem, ws);
   if (st == TERN_OK && workspace_bytes < ws) st = TERN_EINVAL;
   if (st == TERN_OK) {
     bp->xprep = static_cast<uint8_t*>(workspace_dev);
@@ -407,11 +419,16 @@ tern_status run_batch(const tern_gemv_item* items, const tern_prologue* pro, int
 size_t tern_gemm_batch_workspace_bytes(const tern_gemv_item* items, int32_t count, int32_t M, tern_act act) {
   tern::BatchParams* bp = new (std::nothrow) tern::BatchParams();
   tern::PrepParams* pp = new (std::nothrow) tern::PrepParams();
-  size_t smem = 0, ws = 0;
-  const tern_status st = (bp && pp) ? fill_batch(items, nullptr, count, M, act, false, *bp, *pp, smem, ws) : TERN_EINVAL;
+  // enough for either kernel family (the launch flags choose between them)
+  size_t smem = 0, ws = 0, ws_tc = 0;
+  tern_status st = (bp && pp) ? fill_batch(items, nullptr, count, M, act, false, false, *bp, *pp, smem, ws) : TERN_EINVAL;
+  if (st == TERN_OK && use_tc(nullptr, count, M, act, 0u)) {
+    *bp = tern::BatchParams();
+    st = fill_batch(items, nullptr, count, M, act, false, true, *bp, *pp, smem, ws_tc);
+  }
   delete bp;
   delete pp;
-  return st == TERN_OK ? ws : 0;
+  return st == TERN_OK ? (ws > ws_tc ? ws : ws_tc) : 0;
 }
 
 size_t tern_gemv_batch_workspace_bytes(const tern_gemv_item* items, int32_t count, tern_act act) {
@@ -695,12 +712,13 @@ tern_status tern_read_flag(const int32_t* err_flag_dev, tern_stream_t stream) {
 }
 
 tern_status tern_device_status(tern_stream_t stream) {
-  int v = 0, w = 0, x = 0, c = 0;
+  int v = 0, w = 0, x = 0, c = 0, t = 0;
   if (tern::read_and_clear_error_latch(&v, cs(stream)) != cudaSuccess) return TERN_ECUDA;
   if (tern::read_and_clear_batch_latch(&w) != cudaSuccess) return TERN_ECUDA;
   if (tern::read_and_clear_prefill_latch(&x) != cudaSuccess) return TERN_ECUDA;
   if (tern::read_and_clear_chain_latch(&c) != cudaSuccess) return TERN_ECUDA;
-  return (v == 0 && w == 0 && x == 0 && c == 0) ? TERN_OK : TERN_ETIMEOUT;
+  if (tern::read_and_clear_tc_latch(&t) != cudaSuccess) return TERN_ECUDA;
+  return (v == 0 && w == 0 && x == 0 && c == 0 && t == 0) ? TERN_OK : TERN_ETIMEOUT;
 }
 
 tern_status tern_gemm_prefill(const tern_matrix* W, int32_t M, const uint16_t* X_bf16_dev, float* Y_dev,

@@ -754,15 +754,24 @@ cudaError_t launch_stream_kernel(cudaLaunchConfig_t& cfg, const BatchParams& p) 
 bool plan_batch(BatchParams& p, const uint32_t* const* planes, size_t& smem, size_t& workspace) {
   if (p.M < 1 || p.M > 16) return false;
   int mp = 1, tpw = 2, cw = 12;
-  batch_shape(p.mode, p.M, mp, tpw, cw);
+  if (p.tc) {
+    // tensor-core path (tern_tc.cu): 8 decoder warps own the 128 rows of a box (one TMEM lane
+    // each), two boxes per 256-row block; B segments of tc_cols x 512 bytes per part
+    if (p.M < 2) return false;
+    mp = tc_token_slots(p.mode, p.M);
+    cw = tc_consumer_warps();
+    tpw = tc_stage_rows() / box_rows(cw);
+  } else {
+    batch_shape(p.mode, p.M, mp, tpw, cw);
+  }
   p.mp = mp;
   p.tpw = tpw;
   p.cw = cw;
   const int kBoxRows = box_rows(cw), kBoxBytes = box_bytes(cw);
-  p.nc = seg_cols(p.mode, mp);
-  p.seg_bytes = seg_words(p.mode, mp) * 4;
+  p.nc = p.tc ? (p.mode == 0 ? 4 * mp : mp) : seg_cols(p.mode, mp);
+  p.seg_bytes = p.tc ? tc_segment_bytes(p.mode, mp) : seg_words(p.mode, mp) * 4;
   const int stage_rows = kBoxRows * tpw;
-  const int ncolp = 8 * ((seg_cols(p.mode, mp) + 7) / 8); // scratch columns: 8 per MMA group
+  const int ncolp = 8 * ((p.nc + 7) / 8);                 // scratch columns: 8 per MMA group
   PFN_cuTensorMapEncodeTiled_v12000 encode = encode_fn();
   if (!encode) return false;
   long long total_cost = 0;
@@ -788,8 +797,9 @@ bool plan_batch(BatchParams& p, const uint32_t* const* planes, size_t& smem, siz
     const cuuint32_t box[3] = {(cuuint32_t)kPartWords, (cuuint32_t)kBoxRows, 2};
     const cuuint32_t estr[3] = {1, 1, 1};
     if (encode(&p.tmap[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t*>(planes[i]), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               p.tc ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE,   // tc: conflict-free row reads
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return false;
   }
   p.total_units = units;
@@ -858,18 +868,23 @@ bool plan_batch(BatchParams& p, const uint32_t* const* planes, size_t& smem, siz
     p.cta_split[c] = code;
   }
   p.nslots = nslots;
-  // workspace: operand segments, then the split sums [slot][rows][ncolp] and counters [slot][cw]
+  // workspace: operand segments, (tc) the token exponents [count][16], then the split sums
+  // [slot][rows][ncolp] and counters [slot][cw]
   xoff = (xoff + 15) & ~(size_t)15;
+  p.meta_off = (uint32_t)xoff;
+  if (p.tc) xoff += (size_t)p.count * 16 * 4;
   p.scratch_off = (uint32_t)xoff;
   p.scratch_words = nslots * (stage_rows * ncolp + cw);
   workspace = xoff + (size_t)p.scratch_words * 4 + 16;
+  if (workspace > 0xFFFFFFFFull) return false;
   p.stage_slot_bytes = (tpw * kBoxBytes + p.seg_bytes + 1023) & ~1023;
   const size_t budget = 227 * 1024;
-  int stages = (int)((budget - 1024) / (size_t)p.stage_slot_bytes);
+  const size_t fixed = p.tc ? tc_smem_bytes(0, 0) : 1024;
+  int stages = (int)((budget - fixed) / (size_t)p.stage_slot_bytes);
   if (stages > 8) stages = 8;
   if (stages < 2) return false;
   p.stages = stages;
-  smem = 1024 + (size_t)stages * p.stage_slot_bytes;
+  smem = p.tc ? tc_smem_bytes(stages, p.stage_slot_bytes) : 1024 + (size_t)stages * p.stage_slot_bytes;
   return true;
 }
 
@@ -889,6 +904,7 @@ void plan_prep(const BatchParams& b, PrepParams& q) {
   q.xprep = b.xprep;
   q.scratch_off = b.scratch_off;
   q.scratch_words = b.scratch_words;
+  q.meta_off = b.meta_off;
   for (int i = 0; i < b.count; ++i) {
     q.items[i].K = b.items[i].K;
     q.items[i].kp = b.items[i].kp;
@@ -897,6 +913,7 @@ void plan_prep(const BatchParams& b, PrepParams& q) {
 }
 
 cudaError_t launch_batch(const BatchParams& p, const PrepParams& q, size_t smem, bool pdl, cudaStream_t st) {
+  if (p.tc) return launch_tc(p, q, smem, pdl, st);
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   int na = 0;

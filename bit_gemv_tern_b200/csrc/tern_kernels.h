@@ -134,6 +134,8 @@ struct BatchParams {
   int32_t nslots;
   uint32_t scratch_off;   // workspace byte offset: [nslots][rows][8 * groups] int32, then counters
   int32_t scratch_words;  // words to zero before the stream (sums and counters)
+  int32_t tc;             // 1: the tensor-core (tcgen05) small-M kernels of tern_tc.cu
+  uint32_t meta_off;      // tc: workspace byte offset of the token exponents E [count][16] int32
 };
 static_assert(sizeof(BatchParams) <= 32764, "kernel parameter limit");
 // The operand preparation of one item (the prep launch): where its activation comes from and the
@@ -155,6 +157,7 @@ struct PrepParams {
   uint8_t* xprep;
   uint32_t scratch_off;
   int32_t scratch_words;
+  uint32_t meta_off;      // tc: token exponents E [count][16] int32
 };
 static_assert(sizeof(PrepParams) <= 32764, "kernel parameter limit");
 // Host: fills tmap/kp/units/xoff, the stage ring and the CTA split; fails on unsupported shapes.
@@ -164,6 +167,15 @@ bool plan_batch(BatchParams& p, const uint32_t* const* planes, size_t& smem, siz
 void plan_prep(const BatchParams& b, PrepParams& q);
 cudaError_t launch_batch(const BatchParams& p, const PrepParams& q, size_t smem, bool pdl, cudaStream_t st);
 cudaError_t read_and_clear_batch_latch(int* out);
+// Small-M lists on tcgen05 (tern_tc.cu): the shape of the plan when BatchParams::tc is set, and the
+// launch pair (operand preparation, stream) that replaces launch_batch's.
+int tc_token_slots(int mode, int M);
+int tc_segment_bytes(int mode, int mp);
+int tc_stage_rows();
+int tc_consumer_warps();
+size_t tc_smem_bytes(int stages, int slot_bytes);
+cudaError_t launch_tc(const BatchParams& p, const PrepParams& q, size_t smem, bool pdl, cudaStream_t st);
+cudaError_t read_and_clear_tc_latch(int* out);
 
 // Prefill dense contraction on tcgen05 (tern_prefill.cu).
 struct PrefillParams {

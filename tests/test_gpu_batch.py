@@ -161,6 +161,32 @@ def test_gemm_batch_small_m_matches_oracle(mode, M):
             assert (yy == y_ref).all(), (N, K, M)
 
 
+@pytest.mark.parametrize("M", [3, 4, 5, 7, 8, 9, 12, 16])
+@pytest.mark.parametrize("mode", ["bf16", "int8"])
+def test_gemm_batch_tensor_core_equals_mma_sync(mode, M):
+    """The tcgen05 kernels (chosen from bf16 M >= 3 and int8 M >= 5) and the mma.sync kernels
+    (TERN_FLAG_MMA_SYNC) give the same bits for every output: every sum is an exact integer and the
+    final roundings are the same. Ragged N (37, 200, 1000 rows: partial row blocks and boxes),
+    K = 128 and 640 (partial 512-trit parts), and lists whose row blocks are split between CTAs;
+    twice in a row (split-block scratch left clean) and with PDL."""
+    act = tg.TERN_ACT_BF16 if mode == "bf16" else tg.TERN_ACT_INT8
+    shapes = SHAPES_M + [(1000, 128), (6144, 4096)]
+    items, _ = _build_m(95 + M, shapes, M, act)
+    batch = tg.GemvBatch(items, act, M=M)
+    batch(flags=tg.TERN_FLAG_MMA_SYNC)
+    torch.cuda.synchronize()
+    assert tg.tern_device_status() == tg.TERN_OK
+    want = [host(Y).copy() for (_, _, _, Y) in items]
+    for flags in (0, 0, tg.TERN_FLAG_PDL):
+        for (_, _, _, Y) in items:
+            Y.fill_(float("nan"))
+        batch(flags=flags)
+        torch.cuda.synchronize()
+        assert tg.tern_device_status() == tg.TERN_OK
+        for (W, _, _, Y), a in zip(items, want):
+            assert (host(Y).view(np.uint32) == a.view(np.uint32)).all(), (mode, M, W.N, W.K, flags)
+
+
 def test_gemm_batch_int8_equals_small_m_entry():
     """The batched small-M path and tern_gemm_small_m agree bit for bit in int8 mode."""
     M = 7
