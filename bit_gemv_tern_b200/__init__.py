@@ -271,7 +271,8 @@ class _ChainItem(ctypes.Structure):
 
 class _ChainHandle(ctypes.Structure):
     _fields_ = [("workspace_dev", ctypes.c_void_p), ("count", ctypes.c_int32), ("mode", ctypes.c_int32),
-                ("grid", ctypes.c_int32), ("stages", ctypes.c_int32), ("smem_bytes", ctypes.c_size_t)]
+                ("grid", ctypes.c_int32), ("stages", ctypes.c_int32), ("seg_parts", ctypes.c_int32),
+                ("smem_bytes", ctypes.c_size_t)]
 
 
 class ChainItem:

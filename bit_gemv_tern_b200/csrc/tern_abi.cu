@@ -320,13 +320,10 @@ namespace {
 
 // Validates a list (and its prologues, if any) and plans both launches. With check_ptrs false
 // only the shapes and modes are checked (the workspace query).
-// The tensor-core (tcgen05) small-M kernels take lists of M rows from these sizes on, without
-// prologues, unless the caller asks for the mma.sync kernels.
-bool use_tc(const tern_prologue* pro, int32_t count, int32_t M, tern_act act, uint32_t flags) {
+// The tensor-core (tcgen05) small-M kernels take lists of M rows from these sizes on, unless the
+// caller asks for the mma.sync kernels (which exist for bf16 lists of at most 4 rows and for int8).
+bool use_tc(int32_t M, tern_act act, uint32_t flags) {
   if (flags & TERN_FLAG_MMA_SYNC) return false;
-  if (pro)
-    for (int i = 0; i < count; ++i)
-      if (pro[i].kind != TERN_PRO_NONE) return false;
   return act == TERN_ACT_BF16 ? M >= 3 : M >= 5;
 }
 
@@ -396,13 +393,14 @@ tern_status fill_batch(const tern_gemv_item* items, const tern_prologue* pro, in
 tern_status run_batch(const tern_gemv_item* items, const tern_prologue* pro, int32_t count, int32_t M, tern_act act,
                       void* workspace_dev, size_t workspace_bytes, uint32_t flags, tern_stream_t stream) {
   if (flags & ~(TERN_FLAG_PDL | TERN_FLAG_MMA_SYNC)) return TERN_EINVAL;
+  if ((flags & TERN_FLAG_MMA_SYNC) && act == TERN_ACT_BF16 && M > 4) return TERN_EINVAL;   // tensor cores only
   if (!workspace_dev || !aligned(workspace_dev, 16)) return TERN_EINVAL;
   tern::BatchParams* bp = new (std::nothrow) tern::BatchParams();
   tern::PrepParams* pp = new (std::nothrow) tern::PrepParams();
   tern_status st = (bp && pp) ? TERN_OK : TERN_EINVAL;
   size_t smem = 0, ws = 0;
   if (st == TERN_OK)
-    st = fill_batch(items, pro, count, M, act, true, use_tc(pro, count, M, act, flags), *bp, *pp, smem, ws);
+    st = fill_batch(items, pro, count, M, act, true, use_tc(M, act, flags), *bp, *pp, smem, ws);
   if (st == TERN_OK && workspace_bytes < ws) st = TERN_EINVAL;
   if (st == TERN_OK) {
     bp->xprep = static_cast<uint8_t*>(workspace_dev);
@@ -419,10 +417,12 @@ tern_status run_batch(const tern_gemv_item* items, const tern_prologue* pro, int
 size_t tern_gemm_batch_workspace_bytes(const tern_gemv_item* items, int32_t count, int32_t M, tern_act act) {
   tern::BatchParams* bp = new (std::nothrow) tern::BatchParams();
   tern::PrepParams* pp = new (std::nothrow) tern::PrepParams();
-  // enough for either kernel family (the launch flags choose between them)
+  // enough for either kernel family the launch flags can choose
   size_t smem = 0, ws = 0, ws_tc = 0;
-  tern_status st = (bp && pp) ? fill_batch(items, nullptr, count, M, act, false, false, *bp, *pp, smem, ws) : TERN_EINVAL;
-  if (st == TERN_OK && use_tc(nullptr, count, M, act, 0u)) {
+  const bool legacy = act != TERN_ACT_BF16 || M <= 4;
+  tern_status st = (bp && pp) ? TERN_OK : TERN_EINVAL;
+  if (st == TERN_OK && legacy) st = fill_batch(items, nullptr, count, M, act, false, false, *bp, *pp, smem, ws);
+  if (st == TERN_OK && use_tc(M, act, 0u)) {
     *bp = tern::BatchParams();
     st = fill_batch(items, nullptr, count, M, act, false, true, *bp, *pp, smem, ws_tc);
   }
@@ -573,7 +573,7 @@ tern_status fv5b_head_gemv_argmax(const int8_t* W_dev, const float* block_scale_
 
 namespace {
 
-// Workspace layout of a chain: [items (64-byte aligned)][done counters][finished][scratch].
+// Workspace layout of a chain: [items (64-byte aligned)][done counters][finished] (no scratch).
 struct ChainWs {
   size_t items, done, finished, scratch, total;
 };
@@ -650,12 +650,7 @@ tern_status chain_items(const tern_chain_item* items, int32_t count, tern_act ac
 
 size_t tern_chain_workspace_bytes(const tern_chain_item* items, int32_t count, tern_act act) {
   if (chain_items(items, count, act, false, nullptr, nullptr) != TERN_OK) return 0;
-  size_t scratch = 0;
-  for (int i = 0; i < count; ++i) {
-    const int units = (items[i].W.N + 383) / 384;
-    scratch += (size_t)units * 384 * 8 + (size_t)units * 12;
-  }
-  return chain_ws(count, scratch).total;
+  return chain_ws(count, 0).total;                              // every output is one CTA's: no scratch
 }
 
 tern_status tern_chain_plan(const tern_chain_item* items, int32_t count, tern_act act, void* workspace_dev,
@@ -665,7 +660,8 @@ tern_status tern_chain_plan(const tern_chain_item* items, int32_t count, tern_ac
   const uint32_t** planes = new (std::nothrow) const uint32_t*[count > 0 && count <= TERN_CHAIN_MAX_ITEMS ? count : 1];
   tern_status st = (host && planes) ? chain_items(items, count, act, true, host, planes) : TERN_EINVAL;
   tern::ChainLayout L = {};
-  if (st == TERN_OK && !tern::plan_chain(host, count, act == TERN_ACT_BF16 ? 0 : 1, planes, L)) st = TERN_ESHAPE;
+  const int grid = tern::chain_grid();
+  if (st == TERN_OK && !tern::plan_chain(host, count, act == TERN_ACT_BF16 ? 0 : 1, grid, planes, L)) st = TERN_ESHAPE;
   ChainWs w = chain_ws(count > 0 ? count : 1, L.scratch_words);
   if (st == TERN_OK && workspace_bytes < w.total) st = TERN_EINVAL;
   if (st == TERN_OK) {
@@ -678,8 +674,9 @@ tern_status tern_chain_plan(const tern_chain_item* items, int32_t count, tern_ac
     chain->workspace_dev = workspace_dev;
     chain->count = count;
     chain->mode = act == TERN_ACT_BF16 ? 0 : 1;
-    chain->grid = tern::chain_grid();
+    chain->grid = grid;
     chain->stages = L.stages;
+    chain->seg_parts = L.seg_parts;
     chain->smem_bytes = L.smem;
   }
   delete[] host;
@@ -688,7 +685,9 @@ tern_status tern_chain_plan(const tern_chain_item* items, int32_t count, tern_ac
 }
 
 tern_status tern_chain_run(const tern_chain* chain, tern_stream_t stream) {
-  if (!chain || !chain->workspace_dev || chain->count < 1 || chain->grid < 1 || chain->stages < 2) return TERN_EINVAL;
+  if (!chain || !chain->workspace_dev || chain->count < 1 || chain->grid < 1 || chain->stages < 2 ||
+      chain->seg_parts < 1)
+    return TERN_EINVAL;
   const ChainWs w = chain_ws(chain->count, 0);
   uint8_t* ws = static_cast<uint8_t*>(chain->workspace_dev);
   tern::ChainParams p = {};
@@ -697,6 +696,7 @@ tern_status tern_chain_run(const tern_chain* chain, tern_stream_t stream) {
   p.mode = chain->mode;
   p.grid = chain->grid;
   p.stages = chain->stages;
+  p.seg_parts = chain->seg_parts;
   p.done = reinterpret_cast<int32_t*>(ws + w.done);
   p.finished = reinterpret_cast<int32_t*>(ws + w.finished);
   p.scratch = reinterpret_cast<int32_t*>(ws + w.scratch);

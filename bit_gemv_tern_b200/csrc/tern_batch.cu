@@ -22,9 +22,8 @@
 //      consumer warps walk the stages in order; warp w owns kTPW tiles of 16 rows of the block,
 //      decodes them (one AND per operand register, see tern_device.cuh) into mma.sync u8 x s8
 //      products, and keeps the sums in registers across all parts of the block, so a tile's
-//      outputs are written once, at its end. Shapes with many operand columns (bf16 mode, 8 or 16
-//      token slots) decode to signed 64 * t bytes instead (shift and AND) and keep one accumulator
-//      per column group rather than four.
+//      outputs are written once, at its end. (bf16 lists of 5..16 rows run on the tensor-core
+//      kernels of tern_tc.cu instead.)
 // All sums are exact integers; int8 mode ends with y = ((float)acc * s_x) * scale (two fp32
 // round-to-nearest multiplies), bf16 mode with one fp64 -> fp32 rounding. Every mbarrier wait is
 // bounded and latches TERN_ETIMEOUT on give-up.
@@ -281,10 +280,9 @@ __global__ void __launch_bounds__(kPrepThreads) k_batch_prep(const __grid_consta
 
 // ---------------------------------------------------------------------------------------------
 // MODE: 0 bf16 / 1 int8 activations; MP: token slots (1, 2, 4, 8 or 16; 2 and 4 in bf16 mode
-// only); TPW: tiles per consumer warp; CW: consumer warps; SGN: signed decode (bytes 64 * t, one
-// accumulator per column group, no offset to remove) instead of the offset decode (bytes
-// 4^i * (t + 2), four field accumulators per group).
-template <int MODE, int MP, int TPW, int CW, bool SGN>
+// only); TPW: tiles per consumer warp; CW: consumer warps. The decode is the offset decode (bytes
+// 4^i * (t + 2), four field accumulators per column group, the offset removed with the column sums).
+template <int MODE, int MP, int TPW, int CW>
 __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_constant__ BatchParams p) {
   constexpr int kCW = CW;
   constexpr int kBoxRows = box_rows(CW);
@@ -391,7 +389,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
   }
 
   // ====================== consumers ======================
-  constexpr int NF = SGN ? 1 : 4;                           // accumulators per column group
+  constexpr int NF = 4;                                      // accumulators per column group
   const int g = lane >> 2, t = lane & 3;
   // operand column of group j this lane feeds: M = 1: the lane's limb (rows g >= nc repeat column 0)
   // columns past NCOL (M = 1, PACK) repeat a real column; their sums are never read
@@ -491,27 +489,15 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
 #pragma unroll
         for (int a = 0; a < TPW; ++a) {
           uint32_t wa0, wb0, wa1, wb1;
-          if (SGN) {
-            merge_planes(u4get(ma[a], e), u4get(sa[a], e), wa0, wb0);
-            merge_planes(u4get(mb[a], e), u4get(sb[a], e), wa1, wb1);
-          } else {
-            merge_planes_offset(u4get(ma[a], e), u4get(sa[a], e), wa0, wb0);
-            merge_planes_offset(u4get(mb[a], e), u4get(sb[a], e), wa1, wb1);
-          }
+          merge_planes_offset(u4get(ma[a], e), u4get(sa[a], e), wa0, wb0);
+          merge_planes_offset(u4get(mb[a], e), u4get(sb[a], e), wa1, wb1);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            if (SGN) {                                      // field i of every byte -> 64 * t
-              A[a][i][0] = (wa0 << (6 - 2 * i)) & 0xC0C0C0C0u;
-              A[a][i][1] = (wa1 << (6 - 2 * i)) & 0xC0C0C0C0u;
-              A[a][i][2] = (wb0 << (6 - 2 * i)) & 0xC0C0C0C0u;
-              A[a][i][3] = (wb1 << (6 - 2 * i)) & 0xC0C0C0C0u;
-            } else {                                        // field i in place -> 4^i * (t + 2)
-              const uint32_t msk = 0x03030303u << (2 * i);
-              A[a][i][0] = wa0 & msk;
-              A[a][i][1] = wa1 & msk;
-              A[a][i][2] = wb0 & msk;
-              A[a][i][3] = wb1 & msk;
-            }
+          for (int i = 0; i < 4; ++i) {                     // field i in place -> 4^i * (t + 2)
+            const uint32_t msk = 0x03030303u << (2 * i);
+            A[a][i][0] = wa0 & msk;
+            A[a][i][1] = wa1 & msk;
+            A[a][i][2] = wb0 & msk;
+            A[a][i][3] = wb1 & msk;
           }
         }
 #pragma unroll
@@ -528,10 +514,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
             for (int i = 0; i < 4; ++i) {
               const uint32_t b0 = i < 2 ? u4get(x01, 2 * i) : u4get(x23, 2 * i - 4);
               const uint32_t b1 = i < 2 ? u4get(x01, 2 * i + 1) : u4get(x23, 2 * i - 3);
-              if (SGN)
-                mma_s8(acc[a][j][0], A[a][i][0], A[a][i][1], A[a][i][2], A[a][i][3], b0, b1);
-              else
-                mma_u8s8(acc[a][j][i], A[a][i][0], A[a][i][1], A[a][i][2], A[a][i][3], b0, b1);
+              mma_u8s8(acc[a][j][i], A[a][i][0], A[a][i][1], A[a][i][2], A[a][i][3], b0, b1);
             }
         }
       }
@@ -555,9 +538,8 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
 #pragma unroll
             for (int b = 0; b < 2; ++b) {
               const int m = 8 * jj + 2 * t + b;
-              if (!SGN)
 #pragma unroll
-                for (int l = 0; l < NL; ++l) tot[jj][l][b] = lds32(st + mofs + 4u * (uint32_t)(l * MP + m));
+              for (int l = 0; l < NL; ++l) tot[jj][l][b] = lds32(st + mofs + 4u * (uint32_t)(l * MP + m));
               if (MODE == 0) Etok[jj][b] = lds32(st + mofs + 4u * (uint32_t)(NCOL + m));
             }
         }
@@ -577,9 +559,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
       for (int j = 0; j < G; ++j)
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          V[a][j][q] = SGN ? (acc[a][j][0][q] >> 6)
-                           : acc[a][j][0][q] + (acc[a][j][NF > 1 ? 1 : 0][q] >> 2) +
-                                 (acc[a][j][NF > 2 ? 2 : 0][q] >> 4) + (acc[a][j][NF > 3 ? 3 : 0][q] >> 6);
+          V[a][j][q] = acc[a][j][0][q] + (acc[a][j][1][q] >> 2) + (acc[a][j][2][q] >> 4) + (acc[a][j][3][q] >> 6);
     bool emit = true;
     if (slot >= 0) {
       // a block split between CTAs: add this CTA's part sums; the last contributor (per warp)
@@ -735,18 +715,18 @@ void batch_shape(int mode, int M, int& mp, int& tpw, int& cw) {
     cw = 11;
     return;
   }
-  mp = M <= 8 ? 8 : 16;                         // bf16: 4 or 8 groups, signed decode
-  tpw = mode == 0 ? 1 : 2;
+  mp = M <= 8 ? 8 : 16;                         // int8: one or two groups (bf16 lists of 5..16 rows
+  tpw = 2;                                      // run on the tensor-core kernels, tern_tc.cu)
   cw = 11;
 }
 
-template <int MODE, int MP, int TPW, int CW, bool SGN = false>
+template <int MODE, int MP, int TPW, int CW>
 cudaError_t launch_stream_kernel(cudaLaunchConfig_t& cfg, const BatchParams& p) {
   static std::atomic<unsigned long long> smem_raised{0};
-  cudaError_t e = allow_max_dynamic_smem(k_batch_stream<MODE, MP, TPW, CW, SGN>, smem_raised);
+  cudaError_t e = allow_max_dynamic_smem(k_batch_stream<MODE, MP, TPW, CW>, smem_raised);
   if (e != cudaSuccess) return e;
   cfg.blockDim = dim3((CW + 1) * 32, 1, 1);
-  return cudaLaunchKernelEx(&cfg, k_batch_stream<MODE, MP, TPW, CW, SGN>, p);
+  return cudaLaunchKernelEx(&cfg, k_batch_stream<MODE, MP, TPW, CW>, p);
 }
 
 }  // namespace
@@ -762,6 +742,7 @@ bool plan_batch(BatchParams& p, const uint32_t* const* planes, size_t& smem, siz
     cw = tc_consumer_warps();
     tpw = tc_stage_rows() / box_rows(cw);
   } else {
+    if (p.mode == 0 && p.M > 4) return false;           // bf16 lists of 5..16 rows: tensor cores only
     batch_shape(p.mode, p.M, mp, tpw, cw);
   }
   p.mp = mp;
@@ -943,8 +924,7 @@ cudaError_t launch_batch(const BatchParams& p, const PrepParams& q, size_t smem,
     if (p.mp == 1) return launch_stream_kernel<0, 1, 2, 12>(cfg, p);
     if (p.mp == 2) return launch_stream_kernel<0, 2, 2, 12>(cfg, p);
     if (p.mp == 4) return launch_stream_kernel<0, 4, 2, 11>(cfg, p);
-    if (p.mp == 8) return launch_stream_kernel<0, 8, 1, 11, true>(cfg, p);
-    return launch_stream_kernel<0, 16, 1, 11, true>(cfg, p);
+    return cudaErrorInvalidValue;
   }
   if (p.mp == 1) return launch_stream_kernel<1, 1, 2, 12>(cfg, p);
   if (p.mp == 8) return launch_stream_kernel<1, 8, 2, 11>(cfg, p);

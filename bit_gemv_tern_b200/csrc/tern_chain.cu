@@ -4,23 +4,26 @@
 // between and inside the ~120 kernels of a step (PyTorchKR review "Fermion Research, 3진 계열
 // 포맷으로 직접 학습한 Neutrino-1 모델군 3종 공개", section "뉴트리노 엔진: 토큰 하나의 시간은 어디로
 // 가는가"). Here the chain of a step's linears runs as one cooperative kernel, one CTA per SM:
+//   * every linear's rows are cut into chunks of R rows (R a multiple of 16, about N / CTAs), and
+//     CTA c owns chunks c, c + G, ... over the whole of K, so no output needs a sum from another CTA;
 //   * a producer lane streams the weights of every linear, one after the other, through a ring of
-//     shared-memory stages (tensor TMA of the row-major planes, no multicast). Weights do not
-//     depend on activations, so the ring keeps filling while the consumers wait for the previous
-//     linear's outputs: the weight stream does not stop at a linear's boundary;
-//   * the consumer warps of every CTA take an even share of each linear's (row block, 512-trit part)
-//     units. Before a linear, they wait (bounded) until every CTA has finished the linear it reads,
-//     then compute its activation from that output -- RMSNorm, an fp32 cast, or a bf16 row such as
-//     the SwiGLU output -- exactly as the batched prologues do (tern_prologue.cuh), encode the parts
-//     they need as int8 operands (four exact limbs of the row's 30-bit fixed point, or the int8
-//     quantiser's q) and run the signed decode (64 * t bytes) through mma.sync s8 x s8;
+//     shared-memory stages (tensor TMA of the row-major planes, no multicast): a stage holds the
+//     chunk's rows for ps consecutive 512-trit parts. Weights do not depend on activations, so the
+//     ring keeps filling while the consumers wait for the previous linear's outputs: the weight
+//     stream does not stop at a linear's boundary;
+//   * before a linear the consumer warps wait (bounded) until every CTA has finished the linear it
+//     reads, then compute its activation from that output -- RMSNorm, an fp32 cast, or a bf16 row
+//     such as the SwiGLU output -- exactly as the batched prologues do (tern_prologue.cuh), and
+//     encode every 512-trit part as int8 operands (four exact limbs of the row's 30-bit fixed
+//     point, or the int8 quantiser's q);
+//   * the 12 consumer warps split a chunk's 16-row tiles, and the parts of a stage between the warps
+//     of one tile; each runs the signed decode (64 * t bytes) through mma.sync s8 x s8, and the warps
+//     of a tile add their exact sums through shared memory before one of them writes the outputs;
 //   * a gate|up linear whose rows interleave gate and up in groups of eight writes, besides its
 //     fp32 outputs, the SwiGLU activation bf16(silu(gate) * up) of each pair: a lane holds rows r
 //     and r + 8 of its tile, i.e. the gate and the up row of one feature (the SwiGLU epilogue);
-//   * a row block split between CTAs adds exact partial sums in a workspace slot; its last
-//     contributor writes the outputs and clears the slot for the next call; a CTA that has finished
-//     its share of a linear bumps that linear's completion counter (release); the last CTA of the
-//     launch clears the counters.
+//   * a CTA that has written its chunks of a linear bumps that linear's completion counter
+//     (release); the last CTA of the launch clears the counters for the next call.
 // All sums are exact integers and the prologues are the batched path's arithmetic, so every output
 // equals tern_gemm_batch_pro's with the same prologue, bit for bit. Every wait is bounded and latches
 // TERN_ETIMEOUT on give-up.
@@ -42,14 +45,16 @@ __device__ int g_chain_latch = 0;
 namespace {
 
 constexpr int kCW = 12;                          // consumer warps
-constexpr int kTPW = 2;                          // tiles of 16 rows per consumer warp
-constexpr int kBoxRows = kCW * 16;               // rows of one TMA box
-constexpr int kStageRows = kBoxRows * kTPW;      // rows of a row block (384)
+constexpr int kMaxRows = kCW * 16;               // rows of a chunk at most: one 16-row tile per warp
 constexpr int kPartWords = 16;                   // words per plane and row in a 512-trit part
-constexpr int kBoxBytes = 2 * kBoxRows * kPartWords * 4;
-constexpr int kStageBytes = kTPW * kBoxBytes;    // 49152
+constexpr int kStageBytes = 24576;               // one ring stage: 2 planes x R rows x ps parts x 64 B
 constexpr int kColWords = 132;                   // operand words per column and part (128 + skew)
 constexpr int kConsumers = kCW * 32;
+constexpr int kMaxK = 12288;
+constexpr int kJE = kMaxK / (4 * kConsumers);   // float4 activation elements per consumer thread
+static_assert(kJE * 4 * kConsumers == kMaxK, "activation row split");
+constexpr int kRedBytes = kCW * 32 * 4 * 4;      // cross-warp sums: [warp][lane][4] int32
+
 constexpr uint32_t kWaitTries = 1u << 13;
 constexpr long long kSpinNs = 4000000000LL;      // dependency waits give up after ~4 s
 
@@ -104,50 +109,10 @@ __device__ __forceinline__ bool consumers_all(bool v) {
 }
 // L2 loads of data other CTAs wrote during this launch (no stale L1 lines)
 __device__ __forceinline__ float4 ldcg4(const float* p) { return __ldcg(reinterpret_cast<const float4*>(p)); }
-__device__ __forceinline__ uint4 ldcg16(const uint16_t* p) { return __ldcg(reinterpret_cast<const uint4*>(p)); }
 
 // Operand words of word w (0..15) of a part, as in the batched kernel: lane t = w / 4 reads the eight
 // words of its word e = w % 4 at ((e * 4) + t) * 8.
 __device__ __forceinline__ int part_slot(int w) { return ((w & 3) * 4 + (w >> 2)) * 8; }
-
-// CTA range of a linear with P units over G CTAs: [P c / G, P (c + 1) / G); the CTA owning unit p.
-__device__ __forceinline__ int range_start(int P, int G, int c) { return (int)((long long)P * c / G); }
-__device__ __forceinline__ int owner(int P, int G, int p) { return (int)(((long long)(p + 1) * G - 1) / P); }
-// Number of CTAs that own units of [b0, b1): owners are nondecreasing in the unit index, but with
-// fewer units than CTAs the CTAs between two owners own none, so count the distinct owners.
-__device__ __forceinline__ int contributors(int P, int G, int b0, int b1) {
-  int n = 1, o = owner(P, G, b0);
-  for (int u = b0 + 1; u < b1; ++u) {
-    const int v = owner(P, G, u);
-    n += v != o;
-    o = v;
-  }
-  return n;
-}
-
-// 8 bf16 values (k .. k+7) of the linear's activation row, computed from its source with the
-// prologue's arithmetic; sources written during the launch are read through L2.
-__device__ __forceinline__ uint4 act8(const ChainItem& it, int k, double r) {
-  if (it.kind == kProBF16) return ldcg16(static_cast<const uint16_t*>(it.src) + k);
-  const float* s = static_cast<const float*>(it.src);
-  const float4 a0 = ldcg4(s + k), a1 = ldcg4(s + k + 4);
-  const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-  uint16_t h[8];
-  if (it.kind == kProRMSNorm) {
-    const uint4 gw = ld_nc(it.gain + k);
-    const uint32_t g[4] = {gw.x, gw.y, gw.z, gw.w};
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const double ge = (double)bf16_bits_to_float((e & 1) ? (g[e >> 1] >> 16) : (g[e >> 1] & 0xFFFFu));
-      h[e] = bf16_rn(((double)a[e] * r) * ge);
-    }
-  } else {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) h[e] = bf16_rn((double)a[e]);
-  }
-  return make_uint4(h[0] | ((uint32_t)h[1] << 16), h[2] | ((uint32_t)h[3] << 16), h[4] | ((uint32_t)h[5] << 16),
-                    h[6] | ((uint32_t)h[7] << 16));
-}
 
 // Bounded wait until every participating CTA has finished linear `dep` (acquire).
 __device__ bool wait_done(const int* done, int dep, int need) {
@@ -169,8 +134,12 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 1) k_chain(const ChainParams p
   const int S = p.stages;
   const uint32_t full0 = smem_u32(smem), empty0 = full0 + 8 * S;
   const uint32_t ring = smem_u32(smem + 1024);
-  uint32_t* segbuf = reinterpret_cast<uint32_t*>(smem + 1024 + (size_t)S * kStageBytes);   // [kp][NCOL * kColWords]
+  // after the ring: operand segments [seg_parts][NCOL * kColWords] words, the cross-warp sums,
+  // then the linear's bf16 activation row [K]
+  uint32_t* segbuf = reinterpret_cast<uint32_t*>(smem + 1024 + (size_t)S * kStageBytes);
   const uint32_t seg0 = smem_u32(segbuf);
+  int* red = reinterpret_cast<int*>(segbuf + (size_t)p.seg_parts * NCOL * kColWords);
+  uint16_t* xs = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(red) + kRedBytes);
   __shared__ double dred[kCW];
   __shared__ float fred[kCW];
   __shared__ int sh_E;
@@ -198,21 +167,18 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 1) k_chain(const ChainParams p
     bool ok = true;
     for (int i = 0; i < p.count && ok; ++i) {
       const ChainItem& it = items[i];
-      const int P = it.units * it.kp;
       // the tensor map was written to global memory by the host: order it before its TMA use
       asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(&it.tmap) : "memory");
-      for (int u = range_start(P, G, c); u < range_start(P, G, c + 1) && ok; ++u) {
-        const int rb = u / it.kp, part = u - rb * it.kp;
-        if (q >= S && !(ok = mbar_wait(empty0 + 8 * s, ph ^ 1u))) break;
-        int boxes = 0;
-        for (int b = 0; b < kTPW; ++b) boxes += (rb * kStageRows + b * kBoxRows < it.N) ? 1 : 0;
-        const uint32_t bar = full0 + 8 * s, dst = ring + (uint32_t)s * kStageBytes;
-        mbar_arrive_expect_tx(bar, (uint32_t)(boxes * kBoxBytes));
-        for (int b = 0; b < boxes; ++b)
-          tma_load_3d(dst + b * kBoxBytes, &it.tmap, part * kPartWords, rb * kStageRows + b * kBoxRows, 0, bar);
-        ++q;
-        if (++s == S) { s = 0; ph ^= 1u; }
-      }
+      const uint32_t bytes = (uint32_t)(it.rows * it.ps * 128);
+      for (int ch = c; ch < it.chunks && ok; ch += G)
+        for (int st = 0; st < it.nst; ++st) {
+          if (q >= S && !(ok = mbar_wait(empty0 + 8 * s, ph ^ 1u))) break;
+          const uint32_t bar = full0 + 8 * s;
+          mbar_arrive_expect_tx(bar, bytes);
+          tma_load_3d(ring + (uint32_t)s * kStageBytes, &it.tmap, st * it.ps * kPartWords, ch * it.rows, 0, bar);
+          ++q;
+          if (++s == S) { s = 0; ph ^= 1u; }
+        }
     }
     if (!ok) atomicExch(&g_chain_latch, 5);
     // do not exit with copies in flight: wait for the stages issued last
@@ -225,43 +191,82 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 1) k_chain(const ChainParams p
   const int g = lane >> 2, t = lane & 3;
   const int tid = threadIdx.x;                                  // 0 .. kConsumers-1
   const bool live0 = MODE == 0 ? g < NCOL : g == 0;             // lanes whose MMA column carries data
-  const uint32_t wofs = (uint32_t)((warp * 16 + g) * kPartWords * 4 + t * 16);
   int s = 0;
   uint32_t ph = 0;
   bool ok = true;
   for (int i = 0; i < p.count && ok; ++i) {
     const ChainItem& it = items[i];
-    const int K = it.K, kp = it.kp;
-    const int P = it.units * kp;
-    const int p0 = range_start(P, G, c), p1 = range_start(P, G, c + 1);
-    if (p0 >= p1) continue;                                     // no share of this linear
-    // ---- 1. the linear's activation: wait for its source, statistics over the whole row ----------
+    // the next linear's descriptor into L1 (its gains follow into L2 once this linear is done):
+    // neither depends on this linear
+    const bool has_next = i + 1 < p.count;
+    if (has_next && tid == 0)
+      asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<const uint8_t*>(items + i + 1) + 128));
+    const uint16_t* next_gain = has_next ? items[i + 1].gain : nullptr;
+    const int next_k = has_next ? items[i + 1].K : 0;
+    if (c >= it.chunks) continue;                               // no rows of this linear
+    const int K = it.K, kp = it.kp, kind = it.kind;
+    const void* src = it.src;
+    const uint16_t* gain = it.gain;
+    // the gains do not depend on the source either: load them before the wait
+    uint2 gv[kJE];
+#pragma unroll
+    for (int j = 0; j < kJE; ++j) {
+      const int k = 4 * (tid + j * kConsumers);
+      gv[j] = (k < K && kind == kProRMSNorm) ? __ldg(reinterpret_cast<const uint2*>(gain + k)) : make_uint2(0u, 0u);
+    }
+    // ---- 1. wait for the source ----------------------------------------------------------------
     if (it.dep >= 0) {
       bool got = true;
-      if (tid == 0) {
-        const ChainItem& d = items[it.dep];
-        const int Pd = d.units * d.kp;
-        got = wait_done(p.done, it.dep, Pd < G ? Pd : G);
-      }
+      if (tid == 0) got = wait_done(p.done, it.dep, it.dep_need);
       if (!consumers_all(got)) { ok = false; break; }          // uniform: every consumer breaks
     }
+    // ---- 2. the activation row, each thread's elements k = 4 (tid + j kConsumers) in registers:
+    //         sum of squares (RMSNorm), then the bf16 values into shared memory and their absmax ----
+    float4 av[kJE];
     double r = 1.0;
-    if (it.kind == kProRMSNorm) {
+    if (kind != kProBF16) {
       double ss = 0.0;
-      const float* src = static_cast<const float*>(it.src);
-      for (int k = tid * 4; k < K; k += kConsumers * 4) {
-        const float4 v = ldcg4(src + k);
-        ss += (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
+#pragma unroll
+      for (int j = 0; j < kJE; ++j) {
+        const int k = 4 * (tid + j * kConsumers);
+        av[j] = k < K ? ldcg4(static_cast<const float*>(src) + k) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        ss += (double)av[j].x * av[j].x + (double)av[j].y * av[j].y + (double)av[j].z * av[j].z +
+              (double)av[j].w * av[j].w;
       }
-      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
-      if (lane == 0) dred[warp] = ss;
-      consumers_sync();
-      double tot = 0.0;
-      for (int w = 0; w < kCW; ++w) tot += dred[w];
-      r = 1.0 / sqrt(tot / (double)K + (double)it.eps);
+      if (kind == kProRMSNorm) {
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+        if (lane == 0) dred[warp] = ss;
+        consumers_sync();
+        double tot = 0.0;
+        for (int w = 0; w < kCW; ++w) tot += dred[w];
+        r = 1.0 / sqrt(tot / (double)K + (double)it.eps);
+      }
     }
     float amax = 0.0f;
-    for (int k = tid * 8; k < K; k += kConsumers * 8) amax = fmaxf(amax, absmax8(act8(it, k, r)));
+#pragma unroll
+    for (int j = 0; j < kJE; ++j) {
+      const int k = 4 * (tid + j * kConsumers);
+      if (k < K) {
+        uint32_t h[4];
+        if (kind == kProBF16) {
+          const uint2 v = __ldcg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(src) + k));
+          h[0] = v.x & 0xFFFFu; h[1] = v.x >> 16; h[2] = v.y & 0xFFFFu; h[3] = v.y >> 16;
+        } else {
+          const float a[4] = {av[j].x, av[j].y, av[j].z, av[j].w};
+          if (kind == kProRMSNorm) {
+            const uint32_t gg[4] = {gv[j].x & 0xFFFFu, gv[j].x >> 16, gv[j].y & 0xFFFFu, gv[j].y >> 16};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) h[e] = bf16_rn(((double)a[e] * r) * (double)bf16_bits_to_float(gg[e]));
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) h[e] = bf16_rn((double)a[e]);
+          }
+        }
+        *reinterpret_cast<uint2*>(xs + k) = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
+#pragma unroll
+        for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(bf16_bits_to_float(h[e])));
+      }
+    }
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
     if (lane == 0) fred[warp] = amax;
     consumers_sync();
@@ -272,103 +277,91 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 1) k_chain(const ChainParams p
         sh_E = limb_exponent(mx);
       } else {
         sh_sx = __fdiv_rn(mx, 127.0f);
-        if (p0 == 0 && it.sx_out) it.sx_out[0] = sh_sx;     // the CTA holding unit 0
+        if (c == 0 && it.sx_out) it.sx_out[0] = sh_sx;      // CTA 0 owns chunk 0
       }
     }
     consumers_sync();
     const int E = sh_E;
     const float sxv = sh_sx;
-    // ---- 2. operand segments of the parts this CTA streams (all parts when it covers a row block) ---
-    {
-      const bool all = p1 - p0 >= kp;
-      const int first = p0 % kp, cnt = all ? kp : p1 - p0;
-      // one 16-element half of a 32-trit word per thread iteration; parts first .. first + cnt - 1 (mod kp)
-      for (int v = tid; v < cnt * 32; v += kConsumers) {
-        const int part = (first + v / 32) % kp, wh = v % 32, w = wh >> 1, h = wh & 1;
-        const int k = part * 512 + 32 * w + 16 * h;
-        uint32_t* seg = segbuf + (size_t)part * (NCOL * kColWords) + part_slot(w);
-        if (k >= K) {                                           // past the row: zero operands
-          for (int col = 0; col < NCOL; ++col) {
-            uint32_t* d = seg + col * kColWords;
-            d[0 + h] = d[2 + h] = d[4 + h] = d[6 + h] = 0u;
-          }
-          continue;
-        }
-        const uint4 a = act8(it, k, r), b = act8(it, k + 8, r);
-        const uint32_t wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-        uint32_t l[NCOL][4] = {};
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float xf = bf16_bits_to_float((e & 1) ? (wv[e >> 1] >> 16) : (wv[e >> 1] & 0xFFFFu));
-          const int sh = 8 * (e & 3);
-          if (MODE == 0) {
-            int L[4];
-            limbs_of(limb_fixed(xf, E), L);
-#pragma unroll
-            for (int col = 0; col < NCOL; ++col) l[col][e >> 2] |= (uint32_t)(uint8_t)L[col] << sh;
-          } else {
-            l[0][e >> 2] |= (uint32_t)(uint8_t)(int8_t)quant_i8(xf, sxv) << sh;
-          }
-        }
-#pragma unroll
+    // ---- 3. operand segments of every part, from the shared-memory row --------------------------
+    for (int v = tid; v < kp * 32; v += kConsumers) {
+      const int part = v >> 5, w = (v & 31) >> 1, h = v & 1;   // one 16-element half of a word
+      const int k = part * 512 + 32 * w + 16 * h;
+      uint32_t* seg = segbuf + (size_t)part * (NCOL * kColWords) + part_slot(w);
+      if (k >= K) {                                             // past the row: zero operands
         for (int col = 0; col < NCOL; ++col) {
-          const uint4 pv = permute_i8_half(make_uint4(l[col][0], l[col][1], l[col][2], l[col][3]));
           uint32_t* d = seg + col * kColWords;
-          d[0 + h] = pv.x;
-          d[2 + h] = pv.y;
-          d[4 + h] = pv.z;
-          d[6 + h] = pv.w;
+          d[0 + h] = d[2 + h] = d[4 + h] = d[6 + h] = 0u;
         }
+        continue;
+      }
+      const uint4 a = *reinterpret_cast<const uint4*>(xs + k), b = *reinterpret_cast<const uint4*>(xs + k + 8);
+      const uint32_t wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      uint32_t l[NCOL][4] = {};
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float xf = bf16_bits_to_float((e & 1) ? (wv[e >> 1] >> 16) : (wv[e >> 1] & 0xFFFFu));
+        const int sh = 8 * (e & 3);
+        if (MODE == 0) {
+          int L[4];
+          limbs_of(limb_fixed(xf, E), L);
+#pragma unroll
+          for (int col = 0; col < NCOL; ++col) l[col][e >> 2] |= (uint32_t)(uint8_t)L[col] << sh;
+        } else {
+          l[0][e >> 2] |= (uint32_t)(uint8_t)(int8_t)quant_i8(xf, sxv) << sh;
+        }
+      }
+#pragma unroll
+      for (int col = 0; col < NCOL; ++col) {
+        const uint4 pv = permute_i8_half(make_uint4(l[col][0], l[col][1], l[col][2], l[col][3]));
+        uint32_t* d = seg + col * kColWords;
+        d[0 + h] = pv.x;
+        d[2 + h] = pv.y;
+        d[4 + h] = pv.z;
+        d[6 + h] = pv.w;
       }
     }
     consumers_sync();
-    // ---- 3. stream this CTA's share, row block by row block ----------------------------------------
-    for (int u = p0; u < p1 && ok;) {
-      const int rb = u / kp;
-      const int pend = min(p1, (rb + 1) * kp);                  // this CTA's parts of the block: [u, pend)
-      const int need = contributors(P, G, rb * kp, (rb + 1) * kp);
-      const int row_base = rb * kStageRows + warp * 16;
-      int acc[kTPW][4];
+    // ---- 4. this CTA's chunks: warps split the 16-row tiles, then a stage's parts -----------------
+    const int T = it.rows >> 4;                                 // tiles of a chunk (<= kCW)
+    const int wpt = kCW / T;                                    // warps per tile
+    const bool active = warp < T * wpt;
+    const int tile = warp % T, lg = warp / T;
+    const int rstride = 64 * it.ps;                             // bytes of one row of a plane in a stage
+    for (int ch = c; ch < it.chunks && ok; ch += G) {
+      const int r0 = ch * it.rows + tile * 16 + g;              // rows r0 (q = 0, 1) and r0 + 8 (q = 2, 3)
+      uint16_t sc_bits[2];
 #pragma unroll
-      for (int a = 0; a < kTPW; ++a) acc[a][0] = acc[a][1] = acc[a][2] = acc[a][3] = 0;
-      uint16_t sc_bits[kTPW][2];
-#pragma unroll
-      for (int a = 0; a < kTPW; ++a)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int row = row_base + a * kBoxRows + g + 8 * h;
-          sc_bits[a][h] = (t == 0 && row < it.N) ? it.scale[row] : (uint16_t)0;
-        }
-      for (int uu = u; uu < pend; ++uu) {
+      for (int h = 0; h < 2; ++h)
+        sc_bits[h] = (active && lg == 0 && t == 0 && r0 + 8 * h < it.N) ? it.scale[r0 + 8 * h] : (uint16_t)0;
+      int acc4[4][4] = {};                                      // one chain per decode field f
+      for (int st = 0; st < it.nst; ++st) {
         if (!(ok = mbar_wait(full0 + 8 * s, ph))) break;
-        const int part = uu % kp;
-        const uint32_t st = ring + (uint32_t)s * kStageBytes;
-        const uint32_t xo = seg0 + (uint32_t)(part * NCOL * kColWords + (live0 ? g : 0) * kColWords + t * 8) * 4;
-        uint4 ma[kTPW], mb[kTPW], sa[kTPW], sb[kTPW];
+        if (active) {
+          const uint32_t rowa = ring + (uint32_t)s * kStageBytes + (uint32_t)((tile * 16 + g) * rstride + t * 16);
+          const uint32_t planeb = (uint32_t)(it.rows * rstride);
+          for (int pp = lg; pp < it.ps; pp += wpt) {
+            const int part = st * it.ps + pp;
+            if (part >= kp) break;
+            const uint32_t ra = rowa + pp * 64;
+            const uint4 ma = lds128(ra), mb = lds128(ra + 8 * rstride);
+            const uint4 sa = lds128(ra + planeb), sb = lds128(ra + planeb + 8 * rstride);
+            const uint32_t xo = seg0 + (uint32_t)(part * NCOL * kColWords + (live0 ? g : 0) * kColWords + t * 8) * 4;
 #pragma unroll
-        for (int a = 0; a < kTPW; ++a) {
-          const uint32_t rr = st + a * kBoxBytes + wofs;
-          ma[a] = lds128(rr);
-          mb[a] = lds128(rr + 8 * kPartWords * 4);
-          sa[a] = lds128(rr + kBoxRows * kPartWords * 4);
-          sb[a] = lds128(rr + (kBoxRows + 8) * kPartWords * 4);
-        }
+            for (int e = 0; e < 4; ++e) {
+              const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+              const uint4 x01 = live0 ? lds128(xo + e * 128) : zero;
+              const uint4 x23 = live0 ? lds128(xo + e * 128 + 16) : zero;
+              uint32_t wa0, wb0, wa1, wb1;
+              merge_planes(u4get(ma, e), u4get(sa, e), wa0, wb0);
+              merge_planes(u4get(mb, e), u4get(sb, e), wa1, wb1);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-          const uint4 x01 = live0 ? lds128(xo + e * 128) : zero;
-          const uint4 x23 = live0 ? lds128(xo + e * 128 + 16) : zero;
-#pragma unroll
-          for (int a = 0; a < kTPW; ++a) {
-            uint32_t wa0, wb0, wa1, wb1;
-            merge_planes(u4get(ma[a], e), u4get(sa[a], e), wa0, wb0);
-            merge_planes(u4get(mb[a], e), u4get(sb[a], e), wa1, wb1);
-#pragma unroll
-            for (int f = 0; f < 4; ++f) {
-              const uint32_t b0 = f < 2 ? u4get(x01, 2 * f) : u4get(x23, 2 * f - 4);
-              const uint32_t b1 = f < 2 ? u4get(x01, 2 * f + 1) : u4get(x23, 2 * f - 3);
-              mma_s8(acc[a], (wa0 << (6 - 2 * f)) & 0xC0C0C0C0u, (wa1 << (6 - 2 * f)) & 0xC0C0C0C0u,
-                     (wb0 << (6 - 2 * f)) & 0xC0C0C0C0u, (wb1 << (6 - 2 * f)) & 0xC0C0C0C0u, b0, b1);
+              for (int f = 0; f < 4; ++f) {
+                const uint32_t b0 = f < 2 ? u4get(x01, 2 * f) : u4get(x23, 2 * f - 4);
+                const uint32_t b1 = f < 2 ? u4get(x01, 2 * f + 1) : u4get(x23, 2 * f - 3);
+                mma_s8(acc4[f], (wa0 << (6 - 2 * f)) & 0xC0C0C0C0u, (wa1 << (6 - 2 * f)) & 0xC0C0C0C0u,
+                       (wb0 << (6 - 2 * f)) & 0xC0C0C0C0u, (wb1 << (6 - 2 * f)) & 0xC0C0C0C0u, b0, b1);
+              }
             }
           }
         }
@@ -376,66 +369,39 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 1) k_chain(const ChainParams p
         if (lane == 0) mbar_arrive(empty0 + 8 * s);
         if (++s == S) { s = 0; ph ^= 1u; }
       }
-      if (!ok) break;                                         // to the CTA-uniform check of step 4
-      // exact sums of this CTA's parts (acc = 64 * sum)
-      int V[kTPW][4];
+      // the tile's exact sums: the warps of a tile add theirs through shared memory (acc = 64 * sum)
+      int acc[4];
 #pragma unroll
-      for (int a = 0; a < kTPW; ++a)
+      for (int q = 0; q < 4; ++q) acc[q] = acc4[0][q] + acc4[1][q] + acc4[2][q] + acc4[3][q];
+      if (!consumers_all(ok)) { ok = false; break; }
+      if (wpt > 1) {
+        if (active && lg > 0) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) V[a][q] = acc[a][q] >> 6;
-      bool emit = true;
-      if (need > 1) {
-        // the block is split between CTAs: add into its slot; the last contributor (per warp) reads
-        // the totals back, writes the outputs and clears the slot and counter for the next call
-        int* sums = p.scratch + it.scratch_off + (size_t)rb * kStageRows * 8;
-        int* counter = p.scratch + it.counter_off + rb * kCW + warp;
-#pragma unroll
-        for (int a = 0; a < kTPW; ++a)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int col = 2 * t + (q & 1);
-            if (col < NCOL) atomicAdd(&sums[(a * kBoxRows + warp * 16 + g + 8 * (q >> 1)) * 8 + col], V[a][q]);
-          }
-        __threadfence();
-        __syncwarp();
-        int last = 0;
-        if (lane == 0) last = atomicAdd(counter, 1) == need - 1;
-        last = __shfl_sync(0xFFFFFFFFu, last, 0);
-        if (last) {
-          __threadfence();
-#pragma unroll
-          for (int a = 0; a < kTPW; ++a)
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int col = 2 * t + (q & 1);
-              if (col < NCOL) {
-                int* e = &sums[(a * kBoxRows + warp * 16 + g + 8 * (q >> 1)) * 8 + col];
-                V[a][q] = __ldcg(e);
-                *e = 0;
-              }
-            }
-          if (lane == 0) *counter = 0;
-        } else {
-          emit = false;
+          for (int q = 0; q < 4; ++q) red[(warp * 32 + lane) * 4 + q] = acc[q];
         }
-      }
+        consumers_sync();
+        if (active && lg == 0)
+          for (int l = 1; l < wpt; ++l)
 #pragma unroll
-      for (int a = 0; a < kTPW && emit; ++a) {
-        const int r0 = row_base + a * kBoxRows + g;             // rows r0 (q = 0, 1) and r0 + 8 (q = 2, 3)
+            for (int q = 0; q < 4; ++q) acc[q] += red[((warp + l * T) * 32 + lane) * 4 + q];
+      }
+      if (active && lg == 0) {
+        int V[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) V[q] = acc[q] >> 6;
         float y[2] = {0.0f, 0.0f};
         if (MODE == 1) {
 #pragma unroll
-          for (int h = 0; h < 2; ++h)
-            y[h] = __fmul_rn(__fmul_rn(__int2float_rn(V[a][2 * h]), sxv), f16_bits_to_float(sc_bits[a][h]));
+          for (int h = 0; h < 2; ++h) y[h] = __fmul_rn(__fmul_rn(__int2float_rn(V[2 * h]), sxv), f16_bits_to_float(sc_bits[h]));
         } else {
           // lane t = 0 holds columns 0 (L3) and 1 (L2), lane t = 1 columns 2 (L1) and 3 (L0)
           int w[4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) w[q] = __shfl_down_sync(0xFFFFFFFFu, V[a][q], 1);
+          for (int q = 0; q < 4; ++q) w[q] = __shfl_down_sync(0xFFFFFFFFu, V[q], 1);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const long long D = limb_combine(V[a][2 * h], V[a][2 * h + 1], w[2 * h], w[2 * h + 1]);
-            y[h] = (float)((double)D * exp2_i(E - kLimbFrac) * (double)f16_bits_to_float(sc_bits[a][h]));
+            const long long D = limb_combine(V[2 * h], V[2 * h + 1], w[2 * h], w[2 * h + 1]);
+            y[h] = (float)((double)D * exp2_i(E - kLimbFrac) * (double)f16_bits_to_float(sc_bits[h]));
           }
         }
         if (t == 0) {
@@ -449,9 +415,9 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 1) k_chain(const ChainParams p
           }
         }
       }
-      u = pend;
     }
-    // ---- 4. this CTA's share of the linear is written: release it --------------------------------
+    if (next_gain && tid * 64 < next_k) asm volatile("prefetch.global.L2 [%0];" ::"l"(next_gain + tid * 64));
+    // ---- 5. this CTA's chunks of the linear are written: release them ----------------------------
     // (a warp whose bounded wait gave up still arrives here, so the decision is CTA-uniform)
     ok = consumers_all(ok);
     if (!ok) break;
@@ -486,41 +452,56 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 }  // namespace
 
-// Host plan of a chain: tensor maps, per-linear units and parts, scratch offsets, the stage ring.
-bool plan_chain(ChainItem* items, int count, int mode, const uint32_t* const* planes, ChainLayout& L) {
+// Host plan of a chain: per linear the chunk rows R (a multiple of 16, at most 192), the parts per
+// stage, the tensor map (boxes of 16 ps words x R rows x 2 planes), and the shared-memory layout.
+bool plan_chain(ChainItem* items, int count, int mode, int grid, const uint32_t* const* planes, ChainLayout& L) {
   PFN_cuTensorMapEncodeTiled_v12000 encode = encode_fn();
-  if (!encode) return false;
+  if (!encode || grid < 1) return false;
   const int ncol = mode == 0 ? 4 : 1;
-  size_t scratch = 0;                                            // int32 words
-  int kp_max = 1;
+  int kp_max = 1, kmax = 128;
   for (int i = 0; i < count; ++i) {
     ChainItem& it = items[i];
-    if (it.K % 128 || it.K <= 0 || it.N <= 0 || it.K > 12288) return false;
+    if (it.K % 128 || it.K <= 0 || it.N <= 0 || it.K > kMaxK) return false;
     it.kp = (it.K + 511) / 512;
-    it.units = (it.N + kStageRows - 1) / kStageRows;
+    long long R = ((long long)it.N + grid - 1) / grid;
+    R = (R + 15) / 16 * 16;
+    if (R > kMaxRows) R = kMaxRows;
+    it.rows = (int)R;
+    it.chunks = (int)(((long long)it.N + R - 1) / R);
+    int ps = kStageBytes / (it.rows * 128);
+    if (ps > it.kp) ps = it.kp;
+    if (ps > 16) ps = 16;
+    if (ps < 1) return false;
+    it.ps = ps;
+    it.nst = (it.kp + ps - 1) / ps;
     if (it.kp > kp_max) kp_max = it.kp;
-    it.scratch_off = (uint32_t)scratch;
-    scratch += (size_t)it.units * kStageRows * 8;
-    it.counter_off = (uint32_t)scratch;
-    scratch += (size_t)it.units * kCW;
-    if (scratch > 0x7FFFFFFF) return false;
+    if (it.K > kmax) kmax = it.K;
+    it.dep_need = 0;
+    if (it.dep >= 0) {
+      if (it.dep >= i) return false;
+      it.dep_need = items[it.dep].chunks < grid ? items[it.dep].chunks : grid;
+    }
     const cuuint64_t dims[3] = {(cuuint64_t)(it.K / 32), (cuuint64_t)it.N, 2};
     const cuuint64_t strides[2] = {(cuuint64_t)it.K / 4, (cuuint64_t)it.K / 8};
-    const cuuint32_t box[3] = {(cuuint32_t)kPartWords, (cuuint32_t)kBoxRows, 2};
+    const cuuint32_t box[3] = {(cuuint32_t)(kPartWords * ps), (cuuint32_t)it.rows, 2};
     const cuuint32_t estr[3] = {1, 1, 1};
     if (encode(&it.tmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t*>(planes[i]), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return false;
   }
+  // shared memory: barriers (1 KB), the stage ring, the operand segments, the cross-warp sums, the
+  // activation row
   const size_t seg_bytes = (size_t)kp_max * ncol * kColWords * 4;
+  const size_t fixed = 1024 + seg_bytes + kRedBytes + (size_t)kmax * 2;
   const size_t budget = 226 * 1024;                              // dynamic: the opt-in limit less 1 KB static
-  if (1024 + seg_bytes + 2 * (size_t)kStageBytes > budget) return false;
-  int stages = (int)((budget - 1024 - seg_bytes) / kStageBytes);
-  if (stages > 4) stages = 4;
+  if (fixed + 2 * (size_t)kStageBytes > budget) return false;
+  int stages = (int)((budget - fixed) / kStageBytes);
+  if (stages > 8) stages = 8;
   L.stages = stages;
-  L.smem = 1024 + (size_t)stages * kStageBytes + seg_bytes;
-  L.scratch_words = scratch;
+  L.seg_parts = kp_max;
+  L.smem = fixed + (size_t)stages * kStageBytes;
+  L.scratch_words = 0;
   return true;
 }
 

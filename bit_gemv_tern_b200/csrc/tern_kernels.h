@@ -263,23 +263,29 @@ struct alignas(64) ChainItem {
   float eps;
   int32_t kind;               // kProBF16, kProCast or kProRMSNorm
   int32_t dep;                // linear whose outputs src holds (-1: written before the launch)
-  int32_t N, K, kp, units;
-  uint32_t scratch_off;       // int32 words: split-block sums [units][384][8]
-  uint32_t counter_off;       // int32 words: split-block counters [units][12]
+  int32_t N, K, kp;
+  int32_t rows;               // rows of a chunk (a multiple of 16, <= 192); CTA c owns chunks c, c + grid, ...
+  int32_t chunks;             // ceil(N / rows)
+  int32_t ps;                 // 512-trit parts per ring stage
+  int32_t nst;                // stages per chunk: ceil(kp / ps)
+  int32_t dep_need;           // CTAs that release the linear dep: min(its chunks, grid)
 };
 struct ChainParams {
   const ChainItem* items;     // device
   int32_t count, mode, grid, stages;
+  int32_t seg_parts;          // operand segment slots in shared memory (parts a CTA streams per linear)
   int32_t* done;              // device: completion counter of each linear [count]
   int32_t* finished;          // device: CTAs finished with the whole chain
-  int32_t* scratch;           // device: split-block sums and counters
+  int32_t* scratch;           // unused (no output needs another CTA's sums)
 };
 struct ChainLayout {
   int stages;
+  int seg_parts;
   size_t smem;
   size_t scratch_words;
 };
-bool plan_chain(ChainItem* items, int count, int mode, const uint32_t* const* planes, ChainLayout& L);
+// grid: the launch's CTAs (chain_grid()), which fixes how many parts a CTA prepares per linear.
+bool plan_chain(ChainItem* items, int count, int mode, int grid, const uint32_t* const* planes, ChainLayout& L);
 cudaError_t launch_chain(const ChainParams& p, size_t smem, cudaStream_t st);
 int chain_grid();
 cudaError_t read_and_clear_chain_latch(int* out);

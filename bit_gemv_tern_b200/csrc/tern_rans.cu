@@ -210,31 +210,39 @@ __global__ void __launch_bounds__(kRansThreads) k_rans_decode(const __grid_const
   uint32_t ahead = 0u;
 #pragma unroll
   for (int b = 0; b < 4; ++b) ahead = (ahead << 8) | (p0 + b < end ? (uint32_t)__ldg(s + p0 + b) : 0u);
-  const int KW = I.K / 32;
+  const int KW = I.K / 32;                             // a multiple of 4 (K % 128 == 0)
   uint32_t* rowp = I.planes + (int64_t)row * 2 * KW;
   bool ok = true;
-  for (int w = 0; w < KW && ok; ++w) {
-    uint32_t m = 0u, sg = 0u;
+  // four words (128 trits) per plane at a time, written as one 16-byte store each: every thread
+  // writes its own row, so word-sized stores would each touch a sector of their own
+  for (int w0 = 0; w0 < KW && ok; w0 += 4) {
+    uint32_t mw[4], sw[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      uint32_t m = 0u, sg = 0u;
 #pragma unroll 8
-    for (int j = 0; j < 32; ++j) {
-      const uint32_t slot = x & 4095u;
-      const uint32_t sym = (slot >= c1) + (slot >= c2);
-      const uint32_t fs = sym == 0 ? f[0] : (sym == 1 ? f[1] : f[2]);
-      const uint32_t cs = sym == 0 ? 0u : (sym == 1 ? c1 : c2);
-      m |= (uint32_t)(sym != 0) << j;
-      sg |= (uint32_t)(sym == 2) << j;
-      x = fs * (x >> 12) + slot - cs;
+      for (int j = 0; j < 32; ++j) {
+        const uint32_t slot = x & 4095u;
+        const uint32_t sym = (slot >= c1) + (slot >= c2);
+        const uint32_t fs = sym == 0 ? f[0] : (sym == 1 ? f[1] : f[2]);
+        const uint32_t cs = sym == 0 ? 0u : (sym == 1 ? c1 : c2);
+        m |= (uint32_t)(sym != 0) << j;
+        sg |= (uint32_t)(sym == 2) << j;
+        x = fs * (x >> 12) + slot - cs;
 #pragma unroll 1
-      for (int r = 0; r < 2 && x < kRansL; ++r) {     // at most two bytes per trit (x >= 2^11 here)
-        x = (x << 8) | (ahead >> 24);
-        const uint32_t q = p0 + 4;
-        ahead = (ahead << 8) | (q < end ? (uint32_t)__ldg(s + q) : 0u);
-        ++p0;
+        for (int r = 0; r < 2 && x < kRansL; ++r) {   // at most two bytes per trit (x >= 2^11 here)
+          x = (x << 8) | (ahead >> 24);
+          const uint32_t q = p0 + 4;
+          ahead = (ahead << 8) | (q < end ? (uint32_t)__ldg(s + q) : 0u);
+          ++p0;
+        }
       }
+      mw[u] = to_layout_order(m);
+      const uint32_t sp = to_layout_order(sg);
+      sw[u] = (sp << 1) | (sp >> 31);                  // the sign bit sits one above its mask bit
     }
-    rowp[w] = to_layout_order(m);
-    const uint32_t sp = to_layout_order(sg);
-    rowp[KW + w] = (sp << 1) | (sp >> 31);           // the sign bit sits one above its mask bit
+    *reinterpret_cast<uint4*>(rowp + w0) = make_uint4(mw[0], mw[1], mw[2], mw[3]);
+    *reinterpret_cast<uint4*>(rowp + KW + w0) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
     ok = p0 <= end;
   }
   if (!ok || x != kRansL || p0 != end) set_flag(flag);

@@ -36,6 +36,7 @@
 
 #include "tern_device.cuh"
 #include "tern_kernels.h"
+#include "tern_prologue.cuh"
 
 namespace tern {
 
@@ -151,48 +152,71 @@ __host__ __device__ constexpr int tc_cols(int mode, int mp) { return mode == 0 ?
 // ---------------------------------------------------------------------------------------------
 // Operand preparation: one CTA per (item, token slot m). Writes the slot's columns of every part's
 // B segment (zeros past K and for slots m >= M), the token's exponent E (bf16 mode) into the
-// metadata, and clears the split-block scratch.
+// metadata, and clears the split-block scratch. An item with a prologue first computes its bf16 row
+// into shared memory (tern_prologue.cuh, the arithmetic and thread count of tern_act_prologue), then
+// encodes from there; int8 mode quantises that row here (tern_quantize_act's quantiser), writing s_x
+// and, if asked, the prepared activation.
 constexpr int kTcPrepThreads = 256;
+constexpr int kTcPrepMaxK = 12288;
 __global__ void __launch_bounds__(kTcPrepThreads) k_tc_prep(const __grid_constant__ PrepParams p) {
   const PrepItem& it = p.items[blockIdx.x];
   const int m = blockIdx.y;
   const int K = it.K, KP = it.kp;
   const int nc = tc_cols(p.mode, p.mp);
   const bool live = m < p.M;
+  const bool pro = it.kind != kProNone;
   uint8_t* blk = p.xprep + it.xoff;
   __shared__ float red[kTcPrepThreads / 32];
+  __shared__ double dred[kTcPrepThreads / 32];
   __shared__ int Esh;
+  __shared__ float ssh;
+  __shared__ __align__(16) uint16_t xs[kTcPrepMaxK];         // a prologue item's prepared bf16 row
   pdl_wait();
   {
     uint32_t* scr = reinterpret_cast<uint32_t*>(p.xprep + p.scratch_off);
     const int nct = gridDim.x * gridDim.y, ct = blockIdx.y * gridDim.x + blockIdx.x;
     for (int i = ct * blockDim.x + threadIdx.x; i < p.scratch_words; i += nct * blockDim.x) scr[i] = 0u;
   }
-  int E = 0;
-  if (p.mode == 0) {
-    float amax = 0.0f;
-    if (live) {
-      const uint16_t* xb = static_cast<const uint16_t*>(it.x) + (size_t)m * K;
-      for (int k = threadIdx.x * 8; k < K; k += kTcPrepThreads * 8) {
-        const uint4 v = ld_nc(xb + k);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          amax = fmaxf(amax, fmaxf(fabsf(bf16_bits_to_float(w[e] & 0xFFFFu)), fabsf(bf16_bits_to_float(w[e] >> 16))));
-      }
+  float amax = 0.0f;
+  if (live && pro) {
+    const size_t row_elems = (size_t)K * (it.kind == kProSwiGLU ? 2 : 1);
+    const void* src = it.kind == kProBF16 ? static_cast<const void*>(static_cast<const uint16_t*>(it.x) + (size_t)m * K)
+                                          : static_cast<const void*>(static_cast<const float*>(it.x) + (size_t)m * row_elems);
+    const double r =
+        it.kind == kProRMSNorm ? rmsnorm_r<kTcPrepThreads>(static_cast<const float*>(src), K, it.eps, dred) : 1.0;
+    uint16_t* xo = (p.mode == 0 && it.xout) ? static_cast<uint16_t*>(it.xout) + (size_t)m * K : nullptr;
+    for (int k = threadIdx.x * 8; k < K; k += kTcPrepThreads * 8) {
+      const uint4 v = prologue8(it.kind, src, it.gain, K, k, r);
+      *reinterpret_cast<uint4*>(xs + k) = v;
+      if (xo) *reinterpret_cast<uint4*>(xo + k) = v;
+      amax = fmaxf(amax, absmax8(v));
     }
+  } else if (live && p.mode == 0) {
+    const uint16_t* xb = static_cast<const uint16_t*>(it.x) + (size_t)m * K;
+    for (int k = threadIdx.x * 8; k < K; k += kTcPrepThreads * 8) amax = fmaxf(amax, absmax8(ld_nc(xb + k)));
+  }
+  int E = 0;
+  float sq = 0.0f;
+  if (p.mode == 0 || pro) {
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
     __syncthreads();
     if (threadIdx.x == 0) {
       float mx = red[0];
       for (int i = 1; i < kTcPrepThreads / 32; ++i) mx = fmaxf(mx, red[i]);
-      Esh = limb_exponent(mx);
-      reinterpret_cast<int*>(p.xprep + p.meta_off)[blockIdx.x * 16 + m] = Esh;
+      if (p.mode == 0) {
+        Esh = limb_exponent(mx);
+        reinterpret_cast<int*>(p.xprep + p.meta_off)[blockIdx.x * 16 + m] = Esh;
+      } else {
+        ssh = __fdiv_rn(mx, 127.0f);                          // the per-token quantiser's scale
+        if (live) it.sx_out[m] = ssh;
+      }
     }
     __syncthreads();
     E = Esh;
+    sq = ssh;
   }
+  int8_t* qo = (p.mode == 1 && pro && live && it.xout) ? static_cast<int8_t*>(it.xout) + (size_t)m * K : nullptr;
   // one 16-element half of a 32-trit word per iteration, over every part (past K: zeros)
   const size_t part_bytes = (size_t)4 * nc * 128;
   for (int v = threadIdx.x; v < KP * 32; v += kTcPrepThreads) {
@@ -201,17 +225,36 @@ __global__ void __launch_bounds__(kTcPrepThreads) k_tc_prep(const __grid_constan
     const int chunk = w >> 2, u = 2 * (w & 3) + h;      // 16-byte unit of the 128-byte row
     uint8_t* base = blk + part * part_bytes + (size_t)chunk * nc * 128;
     const bool have = live && k < K;
+    // the 16 bf16 values (prologue row or bf16 input) of this half
+    uint32_t wv[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    if (have && (pro || p.mode == 0)) {
+      const uint16_t* xb = pro ? xs + k : static_cast<const uint16_t*>(it.x) + (size_t)m * K + k;
+      const uint4 a = pro ? *reinterpret_cast<const uint4*>(xb) : ld_nc(xb);
+      const uint4 b = pro ? *reinterpret_cast<const uint4*>(xb + 8) : ld_nc(xb + 8);
+      wv[0] = a.x; wv[1] = a.y; wv[2] = a.z; wv[3] = a.w; wv[4] = b.x; wv[5] = b.y; wv[6] = b.z; wv[7] = b.w;
+    }
     if (p.mode == 1) {
       uint4 q = make_uint4(0u, 0u, 0u, 0u);
-      if (have) q = permute_i8_half(ld_nc(static_cast<const int8_t*>(it.x) + (size_t)m * K + k));
+      if (have) {
+        if (pro) {
+          uint32_t qw[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const uint32_t bits = (e & 1) ? (wv[e >> 1] >> 16) : (wv[e >> 1] & 0xFFFFu);
+            qw[e >> 2] |= (uint32_t)(uint8_t)(int8_t)quant_i8(bf16_bits_to_float(bits), sq) << (8 * (e & 3));
+          }
+          q = make_uint4(qw[0], qw[1], qw[2], qw[3]);
+          if (qo) *reinterpret_cast<uint4*>(qo + k) = q;
+        } else {
+          q = ld_nc(static_cast<const int8_t*>(it.x) + (size_t)m * K + k);
+        }
+        q = permute_i8_half(q);
+      }
       const int n = m;
       *reinterpret_cast<uint4*>(base + n * 128 + ((u ^ (n & 7)) << 4)) = q;
     } else {
       uint32_t l[4][4] = {};
       if (have) {
-        const uint16_t* xb = static_cast<const uint16_t*>(it.x) + (size_t)m * K + k;
-        const uint4 a = ld_nc(xb), b = ld_nc(xb + 8);
-        const uint32_t wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const uint32_t bits = (e & 1) ? (wv[e >> 1] >> 16) : (wv[e >> 1] & 0xFFFFu);

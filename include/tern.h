@@ -109,8 +109,8 @@ typedef enum { TERN_SRC_INT8_TRITS = 0, TERN_SRC_BASE3 = 1 } tern_src;
 #define TERN_FLAG_PDL 1u
 /* TERN_FLAG_MMA_SYNC (tern_gemm_batch / tern_gemm_batch_pro only): run a small-M list on the
  *   warp-level mma.sync kernels even where the tensor-core (tcgen05) kernels would be chosen
- *   (bf16 mode M >= 3, int8 mode M >= 5, no prologues). Both give bit-identical results; the flag
- *   exists to compare them. */
+ *   (bf16 mode M >= 3, int8 mode M >= 5). Both give bit-identical results; the flag exists to
+ *   compare them. bf16 lists of 5..16 rows have no mma.sync kernel: TERN_EINVAL. */
 #define TERN_FLAG_MMA_SYNC 2u
 
 /* A packed ternary matrix: views of caller-owned device memory. */
@@ -277,7 +277,7 @@ size_t tern_gemm_batch_workspace_bytes(const tern_gemv_item* items, int32_t coun
  * call equals this one with M = 1), plus TERN_FLAG_MMA_SYNC. From bf16 mode M >= 3 and int8 mode
  * M >= 5 the product runs on the 5th-generation tensor cores (tcgen05: the decoded weights are the
  * MMA's A operand in tensor memory, the activation columns its B operand in shared memory), with
- * results bit-identical to the mma.sync kernels'. */
+ * results bit-identical to the mma.sync kernels' where both exist. */
 tern_status tern_gemm_batch(const tern_gemv_item* items, int32_t count, int32_t M, tern_act act,
                             void* workspace_dev, size_t workspace_bytes, uint32_t flags, tern_stream_t stream);
 
@@ -439,6 +439,7 @@ typedef struct {
 typedef struct {
   void* workspace_dev;
   int32_t count, mode, grid, stages;
+  int32_t seg_parts;            /* operand segments a CTA prepares per linear (plan detail)       */
   size_t smem_bytes;
 } tern_chain;
 

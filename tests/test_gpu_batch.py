@@ -161,8 +161,7 @@ def test_gemm_batch_small_m_matches_oracle(mode, M):
             assert (yy == y_ref).all(), (N, K, M)
 
 
-@pytest.mark.parametrize("M", [3, 4, 5, 7, 8, 9, 12, 16])
-@pytest.mark.parametrize("mode", ["bf16", "int8"])
+@pytest.mark.parametrize("mode,M", [("bf16", 3), ("bf16", 4)] + [("int8", M) for M in (5, 7, 8, 9, 12, 16)])
 def test_gemm_batch_tensor_core_equals_mma_sync(mode, M):
     """The tcgen05 kernels (chosen from bf16 M >= 3 and int8 M >= 5) and the mma.sync kernels
     (TERN_FLAG_MMA_SYNC) give the same bits for every output: every sum is an exact integer and the
@@ -185,6 +184,46 @@ def test_gemm_batch_tensor_core_equals_mma_sync(mode, M):
         assert tg.tern_device_status() == tg.TERN_OK
         for (W, _, _, Y), a in zip(items, want):
             assert (host(Y).view(np.uint32) == a.view(np.uint32)).all(), (mode, M, W.N, W.K, flags)
+
+
+def _on_grid(X: np.ndarray) -> np.ndarray:
+    """bf16 activations with every nonzero |x| >= 2^-12 (tiny values moved to +-2^-12): far above the
+    fixed-point grid 2^(E-30) of the four-limb encoding for these rows (absmax < 2^5), so the device
+    sums are the exact sums and the result equals the oracle's single rounding bit for bit."""
+    X = X.copy()
+    mag = X & 0x7FFF
+    tiny = (mag != 0) & (mag < 0x3980)
+    X[tiny] = (X[tiny] & 0x8000) | 0x3980
+    return X
+
+
+@pytest.mark.parametrize("M", [5, 8, 16])
+def test_gemm_batch_bf16_tensor_core_exact(M):
+    """bf16 lists of 5..16 rows run on tcgen05 only. On activations with no element below the limb
+    grid every output equals the oracle's bit for bit (exact integer sums, the same final rounding),
+    twice in a row, on ragged and split shapes; TERN_FLAG_MMA_SYNC is refused for these lists."""
+    shapes = [(200, 640), (1000, 128), (4096, 12288), (24576, 4096), (6144, 4096)]
+    items, refs = [], []
+    for i, (N, K) in enumerate(shapes):
+        W, t, s = make_matrix(131 + M, 300 + i, N, K, host_trits=False)
+        X = _on_grid(synth.activations(131 + M, 400 + i, M, K))
+        Y = torch.full((M * N,), float("nan"), dtype=torch.float32, device="cuda")
+        items.append((W, dev(X.view(np.int16)), None, Y))
+        refs.append((s, X, i))
+    batch = tg.GemvBatch(items, tg.TERN_ACT_BF16, M=M)
+    for _ in range(2):
+        batch()
+        torch.cuda.synchronize()
+        assert tg.tern_device_status() == tg.TERN_OK
+        for (W, _, _, Y), (s, X, i) in zip(items, refs):
+            N, K = W.N, W.K
+            rows = _rows(N, i)
+            tr = synth.trits(131 + M, 300 + i, N, K, rows=rows)
+            want = oracle.gemm_bf16(oracle.pack(tr), s[rows], K, X)
+            got = host(Y).reshape(M, N)[:, rows]
+            assert (got.astype(np.float32).view(np.uint32) == np.asarray(want, np.float32).view(np.uint32)).all(), (M, N, K)
+    with pytest.raises(tg.TernError):
+        batch(flags=tg.TERN_FLAG_MMA_SYNC)
 
 
 def test_gemm_batch_int8_equals_small_m_entry():

@@ -113,10 +113,12 @@ def _batch(kind, mode, M, shapes, seed):
     return act, fused, plain, pros, refs
 
 
-@pytest.mark.parametrize("M", [1, 4])
+@pytest.mark.parametrize("M", [1, 4, 8])
 @pytest.mark.parametrize("mode", ["bf16", "int8"])
 @pytest.mark.parametrize("kind", list(KINDS))
 def test_fused_prologue_equals_two_step_and_oracle(kind, mode, M):
+    """M = 1 and int8 M = 4 run the mma.sync lists, bf16 M = 4 and both modes at M = 8 the tcgen05
+    lists (whose operand preparation computes the prologue itself)."""
     shapes = [(640, 4096), (300, 1024), (256, 12288)]
     act, fused, plain, pros, refs = _batch(kind, mode, M, shapes, 31)
     tg.GemvBatch(plain, act, M=M)()
