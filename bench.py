@@ -630,6 +630,14 @@ def _profile_batch(mode):
     return run
 
 
+def _profile_smallm(M):
+    def run():
+        st = Stack("8b", M=1, layers=4)
+        sv = StackView(st, M)
+        return lambda: sv.launch_stack("bf16")
+    return run
+
+
 def _profile_head(mode):
     def run():
         st = Stack("8b", M=1, layers=0)
@@ -689,6 +697,7 @@ PROFILE_CASES = {
     "batch-8b-4layers-bf16": _profile_batch("bf16"),
     "batch-8b-4layers-int8": _profile_batch("int8"),
     "head-8b-bf16": _profile_head("bf16"),
+    "smallm-8b-4layers-m8-bf16": _profile_smallm(8),
     "prefill-8b-gate-m4096": _profile_prefill("gate"),
     "base3-8b-1layer": _profile_base3(),
     "pack-8b-1layer": _profile_pack(),
@@ -707,12 +716,13 @@ def run_profile_case(name):
     return 0 if st == tg.TERN_OK else 1
 
 
+def gbs_of(nbytes, ms):
+    return nbytes / (ms / 1000.0) / 1e9
+
+
 def extra_rows(stack, torch, tg, hbm_peak, bf16_peak):
     """The other scope rows, each timed with CUDA events over graph replays."""
     out = {}
-
-    def gbs_of(nbytes, ms):
-        return nbytes / (ms / 1000.0) / 1e9
 
     # int8-activation mode on the same 8B stack, every quantisation inside the step (the stack's
     # quantiser fused into its prep launch, one quantiser launch for the head input)
@@ -905,29 +915,33 @@ def chain_row(stack, torch, hbm_peak):
 
 
 def small_m_sweep(stack, hbm_peak, Ms=(1, 2, 3, 4, 5, 7, 8, 12, 16)):
-    """One pass of M rows through the 8B stack + head per M. From bf16 M >= 3 the stack runs on the
-    tcgen05 kernels; the same pass on the mma.sync kernels is timed beside it."""
+    """One pass of M rows through the 8B stack + head per M (bf16): mma.sync kernels up to M = 4,
+    tcgen05 from M = 5. Then the stack alone in int8 mode at M = 5, 8, 16 on both kernel families
+    (activations quantised once)."""
     out = {}
     for M in Ms:
         sm = stack if M == 1 else StackView(stack, M)
+        g = capture(lambda i: (sm.launch_stack("bf16"), sm.launch_head("bf16")), 5)
+        g.replay()
+        ms = timed_replays([(g, 4)]) / 20
+        nb = sm.stack_bytes + sm.head_bytes
+        out[str(M)] = {"pass_us": ms * 1000.0, "frac": gbs_of(nb, ms) / hbm_peak, "tokens_per_s": M * 1000.0 / ms,
+                       "gbs": gbs_of(nb, ms), "launches_per_pass": 3, "kernel": "tcgen05" if M >= 5 else "mma.sync"}
+        del g
+    int8 = {}
+    for M in (5, 8, 16):
+        sm = StackView(stack, M)
         row = {}
-        for name, mma_sync in (("", False), ("mma_sync_", True)):
-            if mma_sync and M < 3:
-                continue
-            if M == 1:
-                g = capture(lambda i: (sm.launch_stack("bf16"), sm.launch_head("bf16")), 5)
-            else:
-                g = capture(lambda i: (sm.launch_stack("bf16", mma_sync=mma_sync), sm.launch_head("bf16")), 5)
+        for name, tc in (("tcgen05", True), ("mma_sync", False)):
+            g = capture(lambda i: sm.launch_stack("int8", tc=tc), 5)
             g.replay()
             ms = timed_replays([(g, 4)]) / 20
-            nb = sm.stack_bytes + sm.head_bytes
-            row[name + "pass_us"] = ms * 1000.0
-            row[name + "frac"] = gbs_of(nb, ms) / hbm_peak
-            if not name:
-                row.update({"tokens_per_s": M * 1000.0 / ms, "gbs": gbs_of(nb, ms), "launches_per_pass": 3,
-                            "kernel": "tcgen05" if M >= 3 else "mma.sync"})
+            nb = sm.stack_bytes - sum(l.K for l in sm.linears) * M
+            row[name + "_pass_us"] = ms * 1000.0
+            row[name + "_frac"] = gbs_of(nb, ms) / hbm_peak
             del g
-        out[str(M)] = row
+        int8[str(M)] = row
+    out["int8_stack_only"] = int8
     return out
 
 
@@ -1030,14 +1044,32 @@ class StackView:
     stack_bytes = Stack.stack_bytes
     head_bytes = Stack.head_bytes
 
-    def launch_stack(self, mode="bf16", pdl=False, mma_sync=False):
-        """All 144 fused linears as one batched small-M launch pair (each reads its X [M][K]);
-        mma_sync: the warp-level MMA kernels instead of the tcgen05 ones."""
+    def launch_stack(self, mode="bf16", pdl=False, tc=False):
+        """All 144 fused linears as one batched small-M launch pair (each reads its X [M][K]; int8
+        mode: q [M][K] and s_x [M], quantised once); tc: the tcgen05 kernels where the mma.sync
+        ones are the default (every list but bf16 of 5..16 rows)."""
+        import torch
         import bit_gemv_tern_b200 as tg
-        if not hasattr(self, "_batch"):
-            entries = [(lin.W, self.x[:self.M * lin.K], None, self.y[i]) for i, lin in enumerate(self.linears)]
-            self._batch = tg.GemvBatch(entries, tg.TERN_ACT_BF16, M=self.M)
-        self._batch(flags=(tg.TERN_FLAG_PDL if pdl else 0) | (tg.TERN_FLAG_MMA_SYNC if mma_sync else 0))
+        key = "_batch_" + mode
+        if not hasattr(self, key):
+            if mode == "bf16":
+                entries = [(lin.W, self.x[:self.M * lin.K], None, self.y[i]) for i, lin in enumerate(self.linears)]
+                setattr(self, key, tg.GemvBatch(entries, tg.TERN_ACT_BF16, M=self.M))
+            else:
+                self.q = torch.empty(self.M * 12288, dtype=torch.int8, device="cuda")
+                self.sxq = torch.empty(self.M, dtype=torch.float32, device="cuda")
+                self.qk = {}
+                entries = []
+                for i, lin in enumerate(self.linears):
+                    if lin.K not in self.qk:
+                        q = torch.empty(self.M * lin.K, dtype=torch.int8, device="cuda")
+                        sx = torch.empty(self.M, dtype=torch.float32, device="cuda")
+                        tg.tern_quantize_act(self.x[:self.M * lin.K], self.M, lin.K, q, sx)
+                        self.qk[lin.K] = (q, sx)
+                    q, sx = self.qk[lin.K]
+                    entries.append((lin.W, q, sx, self.y[i]))
+                setattr(self, key, tg.GemvBatch(entries, tg.TERN_ACT_INT8, M=self.M))
+        getattr(self, key)(flags=(tg.TERN_FLAG_PDL if pdl else 0) | (tg.TERN_FLAG_TCGEN05 if tc else 0))
 
     def launch_head(self, mode="bf16", pdl=False):
         import bit_gemv_tern_b200 as tg

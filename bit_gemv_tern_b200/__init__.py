@@ -17,7 +17,7 @@ import os
 
 __all__ = [
     "TernError", "TernMatrix", "lib", "library_path",
-    "TERN_ACT_BF16", "TERN_ACT_INT8", "TERN_SRC_INT8_TRITS", "TERN_SRC_BASE3", "TERN_FLAG_PDL", "TERN_FLAG_MMA_SYNC",
+    "TERN_ACT_BF16", "TERN_ACT_INT8", "TERN_SRC_INT8_TRITS", "TERN_SRC_BASE3", "TERN_FLAG_PDL", "TERN_FLAG_TCGEN05",
     "tern_packed_bytes", "tern_base3_bytes", "tern_pack", "tern_pack_batch", "tern_base3_encode", "tern_occupancy",
     "tern_quantize_act", "tern_gemv", "tern_gemm_small_m", "tern_gemm_prefill",
     "i8_head_workspace_bytes", "i8_head_gemv_argmax", "i8_head_gemv_argmax_noalloc",
@@ -36,7 +36,7 @@ TERN_OK, TERN_EINVAL, TERN_ESHAPE, TERN_EBADCODE, TERN_ECUDA, TERN_ETIMEOUT = ra
 TERN_ACT_BF16, TERN_ACT_INT8 = 0, 1
 TERN_SRC_INT8_TRITS, TERN_SRC_BASE3 = 0, 1
 TERN_FLAG_PDL = 1
-TERN_FLAG_MMA_SYNC = 2
+TERN_FLAG_TCGEN05 = 2
 TERN_HEAD_NOALLOC_MAX_M = 16
 TERN_PRO_NONE, TERN_PRO_BF16, TERN_PRO_CAST, TERN_PRO_RMSNORM, TERN_PRO_SWIGLU = range(5)
 

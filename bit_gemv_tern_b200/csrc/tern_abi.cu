@@ -320,11 +320,13 @@ namespace {
 
 // Validates a list (and its prologues, if any) and plans both launches. With check_ptrs false
 // only the shapes and modes are checked (the workspace query).
-// The tensor-core (tcgen05) small-M kernels take lists of M rows from these sizes on, unless the
-// caller asks for the mma.sync kernels (which exist for bf16 lists of at most 4 rows and for int8).
+// Which small-M kernels run a list: the tensor-core (tcgen05) ones for bf16 lists of 5..16 rows
+// (the only kernels there) and wherever the caller asks for them (M >= 2); the mma.sync ones for
+// everything else (measured faster wherever both exist).
 bool use_tc(int32_t M, tern_act act, uint32_t flags) {
-  if (flags & TERN_FLAG_MMA_SYNC) return false;
-  return act == TERN_ACT_BF16 ? M >= 3 : M >= 5;
+  if (M < 2) return false;
+  if (flags & TERN_FLAG_TCGEN05) return true;
+  return act == TERN_ACT_BF16 && M >= 5;
 }
 
 tern_status fill_batch(const tern_gemv_item* items, const tern_prologue* pro, int32_t count, int32_t M, tern_act act,
@@ -392,8 +394,8 @@ tern_status fill_batch(const tern_gemv_item* items, const tern_prologue* pro, in
 
 tern_status run_batch(const tern_gemv_item* items, const tern_prologue* pro, int32_t count, int32_t M, tern_act act,
                       void* workspace_dev, size_t workspace_bytes, uint32_t flags, tern_stream_t stream) {
-  if (flags & ~(TERN_FLAG_PDL | TERN_FLAG_MMA_SYNC)) return TERN_EINVAL;
-  if ((flags & TERN_FLAG_MMA_SYNC) && act == TERN_ACT_BF16 && M > 4) return TERN_EINVAL;   // tensor cores only
+  if (flags & ~(TERN_FLAG_PDL | TERN_FLAG_TCGEN05)) return TERN_EINVAL;
+  if ((flags & TERN_FLAG_TCGEN05) && M < 2) return TERN_EINVAL;                    // no tcgen05 kernel at M = 1
   if (!workspace_dev || !aligned(workspace_dev, 16)) return TERN_EINVAL;
   tern::BatchParams* bp = new (std::nothrow) tern::BatchParams();
   tern::PrepParams* pp = new (std::nothrow) tern::PrepParams();
@@ -422,7 +424,7 @@ size_t tern_gemm_batch_workspace_bytes(const tern_gemv_item* items, int32_t coun
   const bool legacy = act != TERN_ACT_BF16 || M <= 4;
   tern_status st = (bp && pp) ? TERN_OK : TERN_EINVAL;
   if (st == TERN_OK && legacy) st = fill_batch(items, nullptr, count, M, act, false, false, *bp, *pp, smem, ws);
-  if (st == TERN_OK && use_tc(M, act, 0u)) {
+  if (st == TERN_OK && M >= 2) {
     *bp = tern::BatchParams();
     st = fill_batch(items, nullptr, count, M, act, false, true, *bp, *pp, smem, ws_tc);
   }

@@ -180,28 +180,21 @@ __device__ __forceinline__ float float_from_order_key(uint32_t k) {
 }
 
 // ---- activation prologues ------------------------------------------------------------------------
-// fp64 -> bf16 bit pattern, round to nearest, ties to even, in one step: the value keeps 8
-// significant bits (7 below the leading one) on the grid of its binade, 2^(e - 7), or on the
-// subnormal grid 2^-133 below 2^-126; a carry out of the significand moves to the next binade and
-// the largest finite bf16 rounds up to infinity. NaN maps to the canonical quiet NaN.
+// fp64 -> bf16 bit pattern, round to nearest, ties to even, as one correctly rounded step (never
+// a double rounding): the value keeps 8 significant bits on the grid of its binade, or the
+// subnormal grid 2^-133 below 2^-126, and values from halfway past the largest finite bf16 on
+// become infinity. NaN maps to the canonical quiet NaN. Done through fp32 by rounding to odd
+// (Boldo and Melquiond, "Emulation of FMA and correctly rounded sums: proved algorithms using
+// rounding to odd", IEEE TC 2008): truncate to fp32 and set the last bit when the truncation was
+// inexact, then round that to nearest even at bf16's last bit; fp32 carries 16 more bits than bf16
+// and the same exponent range (subnormals included), so the result is the correctly rounded one.
 __device__ __forceinline__ uint16_t bf16_rn(double v) {
-  const unsigned long long u = (unsigned long long)__double_as_longlong(v);
-  const uint32_t sign = (uint32_t)(u >> 48) & 0x8000u;
-  const unsigned long long a = u & 0x7FFFFFFFFFFFFFFFull;
-  if (a > 0x7FF0000000000000ull) return 0x7FC0;                // NaN
-  const int e = (int)(a >> 52) - 1023;                          // binade of |v| (double subnormals: -1023)
-  if (e < -134) return (uint16_t)sign;                          // below half the smallest subnormal
-  if (e > 127) return (uint16_t)(sign | 0x7F80u);               // at or above 2^128 (and infinity)
-  const unsigned long long m = (a & 0xFFFFFFFFFFFFFull) | (1ull << 52);   // |v| = m * 2^(e - 52)
-  const int eb = e < -126 ? -126 : e;                           // binade of the bf16 grid
-  const int shift = 45 + (eb - e);                              // low bits of m below the grid (45..53)
-  unsigned long long r = m >> shift;
-  const unsigned long long rem = m & ((1ull << shift) - 1ull), half = 1ull << (shift - 1);
-  if (rem > half || (rem == half && (r & 1ull))) ++r;
-  // r = rounded |v| in grid units: a normal value has r in [128, 256] and bits (eb + 126) * 128 + r
-  // (r = 256 carries into the exponent field); the subnormal binade has eb = -126 and bits r.
-  const uint32_t bits = (uint32_t)(eb + 126) * 128u + (uint32_t)r;
-  return (uint16_t)(sign | (bits >= 0x7F80u ? 0x7F80u : bits));
+  if (v != v) return 0x7FC0;
+  const float f = __double2float_rz(v);                          // toward zero (fp32 max on overflow)
+  uint32_t b = __float_as_uint(f);
+  if ((double)f != v) b |= 1u;                                  // round to odd: the sticky bit
+  b += 0x7FFFu + ((b >> 16) & 1u);                              // nearest even at bit 16
+  return (uint16_t)(b >> 16);
 }
 
 // The int8 quantiser of one activation: clamp(rint(x / s), -127, 127), fp32 round-to-nearest

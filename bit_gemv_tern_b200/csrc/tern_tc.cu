@@ -48,11 +48,13 @@ constexpr int kRG = 2;                           // row groups of 128 per row bl
 constexpr int kRows = 128 * kRG;                 // rows of a row block (one stage)
 constexpr int kBox = 2 * 128 * 64;               // bytes of one row group's box: 2 planes x 128 rows x 64 B
 constexpr int kNA = 4;                           // TMEM A slots (one 128-trit chunk of both row groups)
-constexpr int kDecWarps = 8;
+constexpr int kEpiWarps = 8;                     // one per (row group, TMEM lane quarter): the epilogue
+constexpr int kDecWarps = 2 * kEpiWarps;         // decoders: the same, once per chunk parity
 constexpr int kTcThreads = (2 + kDecWarps) * 32;
 constexpr int kTmemCols = 512;
 constexpr int kDCol = 0;                         // accumulators: row group g at columns 64 g ..
-constexpr int kACol = 128;                       // A slots: slot a, row group g at 128 + 32 (2 a + g)
+constexpr int kACol = 64 * kRG;                  // A slots: slot a, row group g at kACol + 32 (kRG a + g)
+static_assert(kACol + 32 * kRG * kNA <= 512, "TMEM columns");
 constexpr uint32_t kWaitTries = 1u << 13;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
@@ -64,6 +66,21 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 }
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+// Spin (no suspension) until the phase completes: for the single MMA-issuing thread, whose waits
+// are short and on the critical path. Bounded like mbar_wait.
+__device__ __forceinline__ bool mbar_spin(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  for (uint32_t i = 0;; ++i) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if ((i & 1023u) == 1023u && clock64() - t0 > 8000000000LL) return false;   // ~4 s
+  }
 }
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   for (uint32_t i = 0; i < kWaitTries; ++i) {
@@ -302,7 +319,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_stream(const __grid_consta
       mbar_init(empty0 + 8 * i, 1);
     }
     for (int a = 0; a < kNA; ++a) {
-      mbar_init(afull0 + 8 * a, kDecWarps);
+      mbar_init(afull0 + 8 * a, kEpiWarps);                 // the decoder warps of the chunk it holds
       mbar_init(aempty0 + 8 * a, 1);
     }
     mbar_init(dfull, 1);
@@ -389,11 +406,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_stream(const __grid_consta
       for (int q = 0; q < n_stages && ok; ++q) {
         const BatchItem& B = p.items[it];
         const bool last_of_block = (part == B.kp - 1) || (q == n_stages - 1);
-        if (!(ok = mbar_wait(full0 + 8 * s, ph))) break;
+        if (!(ok = mbar_spin(full0 + 8 * s, ph))) break;
         const uint32_t seg = ring + (uint32_t)s * slot_bytes + kRG * kBox;
         for (int c = 0; c < 4 && ok; ++c, ++ac) {
           const int a = ac % kNA;
-          if (!(ok = mbar_wait(afull0 + 8 * a, (uint32_t)((ac / kNA) & 1)))) break;
+          if (!(ok = mbar_spin(afull0 + 8 * a, (uint32_t)((ac / kNA) & 1)))) break;
           tc_fence_after();
 #pragma unroll
           for (int g = 0; g < kRG; ++g)
@@ -420,8 +437,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_stream(const __grid_consta
     }
   } else {
     // ====================== decoders / epilogue ======================
-    const int d = warp - 2;                                // 0 .. 7
-    const int g = d >> 2;                                  // row group
+    const int d = warp - 2;                                // 0 .. 15
+    const int g = (d >> 2) & 1;                            // row group
+    const int cp = d >> 3;                                 // chunks cp and cp + 2 of every stage
+    const int de = d & 7;                                  // epilogue warp index (cp == 0 warps)
     const int quarter = warp & 3;                          // TMEM lanes 32 quarter .. + 31
     const int r = 32 * quarter + lane;                     // row within the group
     const uint32_t lane_addr = (uint32_t)(32 * quarter) << 16;
@@ -430,7 +449,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_stream(const __grid_consta
     const int slot_last = (int)((split >> 16) & 0xFFu) - 1, need_last = (int)(split >> 24);
     constexpr int NCOLP = N;
     int it = first_item, rb = first_rb, part = first_part;
-    int s = 0, ac = 0, blk = 0;
+    int s = 0, blk = 0;
     uint32_t ph = 0;
     int gq = g0;                                           // global part of the block's first stage
     int pstart = first_part;
@@ -439,9 +458,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_stream(const __grid_consta
       const bool last_of_block = (part == B.kp - 1) || (q == n_stages - 1);
       if (!(ok = mbar_wait(full0 + 8 * s, ph))) break;
       const uint32_t box = ring + (uint32_t)s * slot_bytes + (uint32_t)(g * kBox);
-      for (int c = 0; c < 4 && ok; ++c, ++ac) {
-        const int a = ac % kNA;
-        if (ac >= kNA && !(ok = mbar_wait(aempty0 + 8 * a, (uint32_t)(((ac / kNA) - 1) & 1)))) break;
+      for (int c = cp; c < 4 && ok; c += 2) {
+        const int ac = 4 * q + c, a = ac % kNA, use = ac / kNA;   // chunks fill the A slots in turn
+        if (use > 0) {
+          if (!(ok = mbar_wait(aempty0 + 8 * a, (uint32_t)((use - 1) & 1)))) break;
+          tc_fence_after();                                 // the MMAs that read the slot are done
+        }
         // words 4c .. 4c + 3 of this row: 16-byte chunk c of its 64-byte row, 64-byte swizzle
         const uint32_t off = (uint32_t)(r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
         const uint4 mw = lds128(box + off), sw = lds128(box + 128 * 64 + off);
@@ -468,58 +490,60 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_stream(const __grid_consta
       }
       if (!ok) break;
       if (last_of_block) {
-        // ---- the block's outputs: this thread's row, all N accumulator columns ----
-        if (!(ok = mbar_wait(dfull, (uint32_t)(blk & 1)))) break;
-        tc_fence_after();
-        const int row = rb * kRows + g * 128 + r;
-        const int pend = part + 1;                          // this CTA's parts of the block: [pstart, pend)
-        int slot = -1, need = 0;
-        if (gq == g0) { slot = slot_first; need = need_first; }
-        if (gq + (pend - pstart) == g1 && slot_last >= 0) { slot = slot_last; need = need_last; }
-        int V[N];
+        const int pend = part + 1;                            // this CTA's parts of the block: [pstart, pend)
+        if (cp == 0) {
+          // ---- the block's outputs: this thread's row, all N accumulator columns ----
+          if (!(ok = mbar_wait(dfull, (uint32_t)(blk & 1)))) break;
+          tc_fence_after();
+          const int row = rb * kRows + g * 128 + r;
+          int slot = -1, need = 0;
+          if (gq == g0) { slot = slot_first; need = need_first; }
+          if (gq + (pend - pstart) == g1 && slot_last >= 0) { slot = slot_last; need = need_last; }
+          int V[N];
 #pragma unroll
-        for (int c8 = 0; c8 < N / 8; ++c8) {
-          int t8[8];
-          tmem_ld8(tmem + lane_addr + (uint32_t)(kDCol + 64 * g + 8 * c8), t8);
+          for (int c8 = 0; c8 < N / 8; ++c8) {
+            int t8[8];
+            tmem_ld8(tmem + lane_addr + (uint32_t)(kDCol + 64 * g + 8 * c8), t8);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) V[8 * c8 + j] = t8[j] >> 6;      // exact: every term is 64 * t * x
-        }
-        tc_fence_before();
-        bool emit = true;
-        if (slot >= 0) {
-          int* sums = reinterpret_cast<int*>(p.xprep + p.scratch_off) + (size_t)slot * kRows * NCOLP;
-          int* counter = reinterpret_cast<int*>(p.xprep + p.scratch_off) + (size_t)p.nslots * kRows * NCOLP +
-                         slot * kDecWarps + d;
-          int* mine = sums + (size_t)(g * 128 + r) * NCOLP;
-#pragma unroll
-          for (int j = 0; j < N; ++j) atomicAdd(mine + j, V[j]);
-          __threadfence();
-          __syncwarp();
-          int last = 0;
-          if (lane == 0) last = atomicAdd(counter, 1) == need - 1;
-          last = __shfl_sync(0xFFFFFFFFu, last, 0);
-          if (last) {
-            __threadfence();
-#pragma unroll
-            for (int j = 0; j < N; ++j) V[j] = __ldcg(mine + j);
-          } else {
-            emit = false;
+            for (int j = 0; j < 8; ++j) V[8 * c8 + j] = t8[j] >> 6;      // exact: every term is 64 * t * x
           }
-        }
-        if (emit && row < B.N) {
-          const double sc = (double)f16_bits_to_float(B.scale[row]);
-          if (MODE == 1) {
+          tc_fence_before();
+          bool emit = true;
+          if (slot >= 0) {
+            int* sums = reinterpret_cast<int*>(p.xprep + p.scratch_off) + (size_t)slot * kRows * NCOLP;
+            int* counter = reinterpret_cast<int*>(p.xprep + p.scratch_off) + (size_t)p.nslots * kRows * NCOLP +
+                           slot * kEpiWarps + de;
+            int* mine = sums + (size_t)(g * 128 + r) * NCOLP;
 #pragma unroll
-            for (int m = 0; m < MP; ++m)
-              if (m < p.M) B.y[(size_t)m * B.N + row] = __fmul_rn(__fmul_rn(__int2float_rn(V[m]), B.sx[m]), (float)sc);
-          } else {
-            const int* Em = reinterpret_cast<const int*>(p.xprep + p.meta_off) + it * 16;
+            for (int j = 0; j < N; ++j) atomicAdd(mine + j, V[j]);
+            __threadfence();
+            __syncwarp();
+            int last = 0;
+            if (lane == 0) last = atomicAdd(counter, 1) == need - 1;
+            last = __shfl_sync(0xFFFFFFFFu, last, 0);
+            if (last) {
+              __threadfence();
 #pragma unroll
-            for (int m = 0; m < MP; ++m)
-              if (m < p.M) {
-                const long long D = limb_combine(V[4 * m], V[4 * m + 1], V[4 * m + 2], V[4 * m + 3]);
-                B.y[(size_t)m * B.N + row] = (float)((double)D * exp2_i(Em[m] - kLimbFrac) * sc);
-              }
+              for (int j = 0; j < N; ++j) V[j] = __ldcg(mine + j);
+            } else {
+              emit = false;
+            }
+          }
+          if (emit && row < B.N) {
+            const double sc = (double)f16_bits_to_float(B.scale[row]);
+            if (MODE == 1) {
+#pragma unroll
+              for (int m = 0; m < MP; ++m)
+                if (m < p.M) B.y[(size_t)m * B.N + row] = __fmul_rn(__fmul_rn(__int2float_rn(V[m]), B.sx[m]), (float)sc);
+            } else {
+              const int* Em = reinterpret_cast<const int*>(p.xprep + p.meta_off) + it * 16;
+#pragma unroll
+              for (int m = 0; m < MP; ++m)
+                if (m < p.M) {
+                  const long long D = limb_combine(V[4 * m], V[4 * m + 1], V[4 * m + 2], V[4 * m + 3]);
+                  B.y[(size_t)m * B.N + row] = (float)((double)D * exp2_i(Em[m] - kLimbFrac) * sc);
+                }
+            }
           }
         }
         ++blk;
@@ -559,8 +583,13 @@ int tc_token_slots(int mode, int M) {
 }
 int tc_segment_bytes(int mode, int mp) { return tc_cols(mode, mp) * 512; }
 int tc_stage_rows() { return kRows; }
-int tc_consumer_warps() { return kDecWarps; }
-size_t tc_smem_bytes(int stages, int slot_bytes) { return 1024 + (size_t)stages * slot_bytes + 256; }
+// The plan's warps per TMA box (box_rows = 16 per warp: 128 rows) and split counters per slot (the
+// kernel uses kEpiWarps of them).
+int tc_consumer_warps() { return 8; }   // 8 x 16 = 128 rows per box
+// 1 KB of alignment slack, the ring, then the barriers (16 per stage, 16 per A slot, 20 more)
+constexpr int kBarBytes = 512;
+static_assert(16 * 8 + 16 * kNA + 20 <= kBarBytes, "barrier area");
+size_t tc_smem_bytes(int stages, int slot_bytes) { return 1024 + (size_t)stages * slot_bytes + kBarBytes; }
 
 cudaError_t launch_tc(const BatchParams& p, const PrepParams& q, size_t smem, bool pdl, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};

@@ -107,11 +107,11 @@ typedef enum { TERN_SRC_INT8_TRITS = 0, TERN_SRC_BASE3 = 1 } tern_src;
  *   kernel, and reads activations / writes outputs only after. Only valid when the weight
  *   buffers are not written by work still in flight on the stream (true in a decode loop). */
 #define TERN_FLAG_PDL 1u
-/* TERN_FLAG_MMA_SYNC (tern_gemm_batch / tern_gemm_batch_pro only): run a small-M list on the
- *   warp-level mma.sync kernels even where the tensor-core (tcgen05) kernels would be chosen
- *   (bf16 mode M >= 3, int8 mode M >= 5). Both give bit-identical results; the flag exists to
- *   compare them. bf16 lists of 5..16 rows have no mma.sync kernel: TERN_EINVAL. */
-#define TERN_FLAG_MMA_SYNC 2u
+/* TERN_FLAG_TCGEN05 (tern_gemm_batch / tern_gemm_batch_pro only, M >= 2): run the list on the
+ *   tensor-core (tcgen05) small-M kernels, which otherwise take only bf16 lists of 5..16 rows (the
+ *   warp-level mma.sync kernels, bit-identical, run everything else and are faster wherever both
+ *   exist). For comparisons. */
+#define TERN_FLAG_TCGEN05 2u
 
 /* A packed ternary matrix: views of caller-owned device memory. */
 typedef struct {
@@ -274,10 +274,10 @@ size_t tern_gemm_batch_workspace_bytes(const tern_gemv_item* items, int32_t coun
  * with each item's x_dev = X: bf16[M][K] or int8[M][K] row-major, x_scale_dev = float[M] (int8
  * mode), y_dev = Y: float[M][N]. Each decoded weight word feeds all M rows; the weights stream
  * once. Arithmetic, determinism, aliasing rule, workspace and flags as for tern_gemv_batch (whose
- * call equals this one with M = 1), plus TERN_FLAG_MMA_SYNC. From bf16 mode M >= 3 and int8 mode
- * M >= 5 the product runs on the 5th-generation tensor cores (tcgen05: the decoded weights are the
- * MMA's A operand in tensor memory, the activation columns its B operand in shared memory), with
- * results bit-identical to the mma.sync kernels' where both exist. */
+ * call equals this one with M = 1), plus TERN_FLAG_TCGEN05. bf16 lists of 5..16 rows run on the
+ * 5th-generation tensor cores (tcgen05: the decoded weights are the MMA's A operand in tensor
+ * memory, the activation columns (four limbs per row) its B operand in shared memory); every other
+ * list on warp-level mma.sync. Results are bit-identical wherever both exist. */
 tern_status tern_gemm_batch(const tern_gemv_item* items, int32_t count, int32_t M, tern_act act,
                             void* workspace_dev, size_t workspace_bytes, uint32_t flags, tern_stream_t stream);
 
