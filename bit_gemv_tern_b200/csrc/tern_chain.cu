@@ -51,8 +51,8 @@ constexpr int kStageBytes = 24576;               // one ring stage: 2 planes x R
 constexpr int kColWords = 132;                   // operand words per column and part (128 + skew)
 constexpr int kConsumers = kCW * 32;
 constexpr int kMaxK = 12288;
-constexpr int kJE = kMaxK / (4 * kConsumers);   // float4 activation elements per consumer thread
-static_assert(kJE * 4 * kConsumers == kMaxK, "activation row split");
+constexpr int kJH = kMaxK / (16 * kConsumers);  // 16-element halves of the activation per consumer thread
+static_assert(kJH * 16 * kConsumers == kMaxK, "activation row split");
 constexpr int kRedBytes = kCW * 32 * 4 * 4;      // cross-warp sums: [warp][lane][4] int32
 
 constexpr uint32_t kWaitTries = 1u << 13;
@@ -134,12 +134,10 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 1) k_chain(const ChainParams p
   const int S = p.stages;
   const uint32_t full0 = smem_u32(smem), empty0 = full0 + 8 * S;
   const uint32_t ring = smem_u32(smem + 1024);
-  // after the ring: operand segments [seg_parts][NCOL * kColWords] words, the cross-warp sums,
-  // then the linear's bf16 activation row [K]
+  // after the ring: operand segments [seg_parts][NCOL * kColWords] words, the cross-warp sums
   uint32_t* segbuf = reinterpret_cast<uint32_t*>(smem + 1024 + (size_t)S * kStageBytes);
   const uint32_t seg0 = smem_u32(segbuf);
   int* red = reinterpret_cast<int*>(segbuf + (size_t)p.seg_parts * NCOL * kColWords);
-  uint16_t* xs = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(red) + kRedBytes);
   __shared__ double dred[kCW];
   __shared__ float fred[kCW];
   __shared__ int sh_E;
@@ -207,12 +205,17 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 1) k_chain(const ChainParams p
     const int K = it.K, kp = it.kp, kind = it.kind;
     const void* src = it.src;
     const uint16_t* gain = it.gain;
-    // the gains do not depend on the source either: load them before the wait
-    uint2 gv[kJE];
+    // each thread's 16-element halves of the activation row -- v = tid + j kConsumers, elements
+    // 16 v .. 16 v + 15: one unit of the operand layout -- stay in registers from the loads to the
+    // operands. The gains do not depend on the source: load them before the wait.
+    const int nh = kp * 32;                                     // halves of the row's parts (zeros past K)
+    uint4 gw[kJH][2];
 #pragma unroll
-    for (int j = 0; j < kJE; ++j) {
-      const int k = 4 * (tid + j * kConsumers);
-      gv[j] = (k < K && kind == kProRMSNorm) ? __ldg(reinterpret_cast<const uint2*>(gain + k)) : make_uint2(0u, 0u);
+    for (int j = 0; j < kJH; ++j) {
+      const int k = 16 * (tid + j * kConsumers);
+      const bool in = k < K && kind == kProRMSNorm;
+      gw[j][0] = in ? __ldg(reinterpret_cast<const uint4*>(gain + k)) : make_uint4(0u, 0u, 0u, 0u);
+      gw[j][1] = in ? __ldg(reinterpret_cast<const uint4*>(gain + k + 8)) : make_uint4(0u, 0u, 0u, 0u);
     }
     // ---- 1. wait for the source ----------------------------------------------------------------
     if (it.dep >= 0) {
@@ -220,18 +223,20 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 1) k_chain(const ChainParams p
       if (tid == 0) got = wait_done(p.done, it.dep, it.dep_need);
       if (!consumers_all(got)) { ok = false; break; }          // uniform: every consumer breaks
     }
-    // ---- 2. the activation row, each thread's elements k = 4 (tid + j kConsumers) in registers:
-    //         sum of squares (RMSNorm), then the bf16 values into shared memory and their absmax ----
-    float4 av[kJE];
+    // ---- 2. the activation: sum of squares (RMSNorm), the bf16 values and their absmax ----------
+    float4 av[kJH][4];
     double r = 1.0;
     if (kind != kProBF16) {
       double ss = 0.0;
 #pragma unroll
-      for (int j = 0; j < kJE; ++j) {
-        const int k = 4 * (tid + j * kConsumers);
-        av[j] = k < K ? ldcg4(static_cast<const float*>(src) + k) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        ss += (double)av[j].x * av[j].x + (double)av[j].y * av[j].y + (double)av[j].z * av[j].z +
-              (double)av[j].w * av[j].w;
+      for (int j = 0; j < kJH; ++j) {
+        const int k = 16 * (tid + j * kConsumers);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          av[j][u] = k < K ? ldcg4(static_cast<const float*>(src) + k + 4 * u) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          ss += (double)av[j][u].x * av[j][u].x + (double)av[j][u].y * av[j][u].y + (double)av[j][u].z * av[j][u].z +
+                (double)av[j][u].w * av[j][u].w;
+        }
       }
       if (kind == kProRMSNorm) {
         for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
@@ -242,29 +247,38 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 1) k_chain(const ChainParams p
         r = 1.0 / sqrt(tot / (double)K + (double)it.eps);
       }
     }
+    uint32_t hv[kJH][8];                                        // the bf16 values, two per word
     float amax = 0.0f;
 #pragma unroll
-    for (int j = 0; j < kJE; ++j) {
-      const int k = 4 * (tid + j * kConsumers);
+    for (int j = 0; j < kJH; ++j) {
+      const int k = 16 * (tid + j * kConsumers);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) hv[j][e] = 0u;
       if (k < K) {
-        uint32_t h[4];
         if (kind == kProBF16) {
-          const uint2 v = __ldcg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(src) + k));
-          h[0] = v.x & 0xFFFFu; h[1] = v.x >> 16; h[2] = v.y & 0xFFFFu; h[3] = v.y >> 16;
+          const uint4 x0 = __ldcg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(src) + k));
+          const uint4 x1 = __ldcg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(src) + k + 8));
+          hv[j][0] = x0.x; hv[j][1] = x0.y; hv[j][2] = x0.z; hv[j][3] = x0.w;
+          hv[j][4] = x1.x; hv[j][5] = x1.y; hv[j][6] = x1.z; hv[j][7] = x1.w;
         } else {
-          const float a[4] = {av[j].x, av[j].y, av[j].z, av[j].w};
-          if (kind == kProRMSNorm) {
-            const uint32_t gg[4] = {gv[j].x & 0xFFFFu, gv[j].x >> 16, gv[j].y & 0xFFFFu, gv[j].y >> 16};
+          const uint32_t gg[8] = {gw[j][0].x, gw[j][0].y, gw[j][0].z, gw[j][0].w, gw[j][1].x, gw[j][1].y, gw[j][1].z, gw[j][1].w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) h[e] = bf16_rn(((double)a[e] * r) * (double)bf16_bits_to_float(gg[e]));
-          } else {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) h[e] = bf16_rn((double)a[e]);
+          for (int e = 0; e < 16; ++e) {
+            const float4 q4 = av[j][e >> 2];
+            const float a = (e & 3) == 0 ? q4.x : ((e & 3) == 1 ? q4.y : ((e & 3) == 2 ? q4.z : q4.w));
+            uint32_t h;
+            if (kind == kProRMSNorm) {
+              const uint32_t gb = (e & 1) ? (gg[e >> 1] >> 16) : (gg[e >> 1] & 0xFFFFu);
+              h = bf16_rn(((double)a * r) * (double)bf16_bits_to_float(gb));
+            } else {
+              h = bf16_rn((double)a);
+            }
+            hv[j][e >> 1] |= h << (16 * (e & 1));
           }
         }
-        *reinterpret_cast<uint2*>(xs + k) = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
 #pragma unroll
-        for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(bf16_bits_to_float(h[e])));
+        for (int e = 0; e < 8; ++e)
+          amax = fmaxf(amax, fmaxf(fabsf(bf16_bits_to_float(hv[j][e] & 0xFFFFu)), fabsf(bf16_bits_to_float(hv[j][e] >> 16))));
       }
     }
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
@@ -283,24 +297,17 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 1) k_chain(const ChainParams p
     consumers_sync();
     const int E = sh_E;
     const float sxv = sh_sx;
-    // ---- 3. operand segments of every part, from the shared-memory row --------------------------
-    for (int v = tid; v < kp * 32; v += kConsumers) {
-      const int part = v >> 5, w = (v & 31) >> 1, h = v & 1;   // one 16-element half of a word
-      const int k = part * 512 + 32 * w + 16 * h;
+    // ---- 3. operand segments of every part, from the registers ------------------------------------
+#pragma unroll
+    for (int j = 0; j < kJH; ++j) {
+      const int v = tid + j * kConsumers;
+      if (v >= nh) continue;
+      const int part = v >> 5, w = (v & 31) >> 1, h = v & 1;
       uint32_t* seg = segbuf + (size_t)part * (NCOL * kColWords) + part_slot(w);
-      if (k >= K) {                                             // past the row: zero operands
-        for (int col = 0; col < NCOL; ++col) {
-          uint32_t* d = seg + col * kColWords;
-          d[0 + h] = d[2 + h] = d[4 + h] = d[6 + h] = 0u;
-        }
-        continue;
-      }
-      const uint4 a = *reinterpret_cast<const uint4*>(xs + k), b = *reinterpret_cast<const uint4*>(xs + k + 8);
-      const uint32_t wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-      uint32_t l[NCOL][4] = {};
+      uint32_t l[NCOL][4] = {};                                // zeros past K
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
-        const float xf = bf16_bits_to_float((e & 1) ? (wv[e >> 1] >> 16) : (wv[e >> 1] & 0xFFFFu));
+        const float xf = bf16_bits_to_float((e & 1) ? (hv[j][e >> 1] >> 16) : (hv[j][e >> 1] & 0xFFFFu));
         const int sh = 8 * (e & 3);
         if (MODE == 0) {
           int L[4];
@@ -458,7 +465,7 @@ bool plan_chain(ChainItem* items, int count, int mode, int grid, const uint32_t*
   PFN_cuTensorMapEncodeTiled_v12000 encode = encode_fn();
   if (!encode || grid < 1) return false;
   const int ncol = mode == 0 ? 4 : 1;
-  int kp_max = 1, kmax = 128;
+  int kp_max = 1;
   for (int i = 0; i < count; ++i) {
     ChainItem& it = items[i];
     if (it.K % 128 || it.K <= 0 || it.N <= 0 || it.K > kMaxK) return false;
@@ -475,7 +482,6 @@ bool plan_chain(ChainItem* items, int count, int mode, int grid, const uint32_t*
     it.ps = ps;
     it.nst = (it.kp + ps - 1) / ps;
     if (it.kp > kp_max) kp_max = it.kp;
-    if (it.K > kmax) kmax = it.K;
     it.dep_need = 0;
     if (it.dep >= 0) {
       if (it.dep >= i) return false;
@@ -490,10 +496,9 @@ bool plan_chain(ChainItem* items, int count, int mode, int grid, const uint32_t*
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return false;
   }
-  // shared memory: barriers (1 KB), the stage ring, the operand segments, the cross-warp sums, the
-  // activation row
+  // shared memory: barriers (1 KB), the stage ring, the operand segments, the cross-warp sums
   const size_t seg_bytes = (size_t)kp_max * ncol * kColWords * 4;
-  const size_t fixed = 1024 + seg_bytes + kRedBytes + (size_t)kmax * 2;
+  const size_t fixed = 1024 + seg_bytes + kRedBytes;
   const size_t budget = 226 * 1024;                              // dynamic: the opt-in limit less 1 KB static
   if (fixed + 2 * (size_t)kStageBytes > budget) return false;
   int stages = (int)((budget - fixed) / kStageBytes);
