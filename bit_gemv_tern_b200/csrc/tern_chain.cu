@@ -202,7 +202,14 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 1) k_chain(const ChainParams p
     const uint16_t* next_gain = has_next ? items[i + 1].gain : nullptr;
     const int next_k = has_next ? items[i + 1].K : 0;
     if (c >= it.chunks) continue;                               // no rows of this linear
-    const int K = it.K, kp = it.kp, kind = it.kind;
+    // every field this linear needs, into registers now: the descriptor line may have left L1
+    const int K = it.K, kp = it.kp, kind = it.kind, N = it.N, rows = it.rows, chunks = it.chunks;
+    const int ps = it.ps, nst = it.nst, dep = it.dep, dep_need = it.dep_need;
+    const float eps = it.eps;
+    const uint16_t* scale = it.scale;
+    float* yout = it.y;
+    uint16_t* hout = it.hout;
+    float* sx_out = it.sx_out;
     const void* src = it.src;
     const uint16_t* gain = it.gain;
     // each thread's 16-element halves of the activation row -- v = tid + j kConsumers, elements
@@ -218,9 +225,9 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 1) k_chain(const ChainParams p
       gw[j][1] = in ? __ldg(reinterpret_cast<const uint4*>(gain + k + 8)) : make_uint4(0u, 0u, 0u, 0u);
     }
     // ---- 1. wait for the source ----------------------------------------------------------------
-    if (it.dep >= 0) {
+    if (dep >= 0) {
       bool got = true;
-      if (tid == 0) got = wait_done(p.done, it.dep, it.dep_need);
+      if (tid == 0) got = wait_done(p.done, dep, dep_need);
       if (!consumers_all(got)) { ok = false; break; }          // uniform: every consumer breaks
     }
     // ---- 2. the activation: sum of squares (RMSNorm), the bf16 values and their absmax ----------
@@ -244,7 +251,7 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 1) k_chain(const ChainParams p
         consumers_sync();
         double tot = 0.0;
         for (int w = 0; w < kCW; ++w) tot += dred[w];
-        r = 1.0 / sqrt(tot / (double)K + (double)it.eps);
+        r = 1.0 / sqrt(tot / (double)K + (double)eps);
       }
     }
     uint32_t hv[kJH][8];                                        // the bf16 values, two per word
@@ -291,7 +298,7 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 1) k_chain(const ChainParams p
         sh_E = limb_exponent(mx);
       } else {
         sh_sx = __fdiv_rn(mx, 127.0f);
-        if (c == 0 && it.sx_out) it.sx_out[0] = sh_sx;      // CTA 0 owns chunk 0
+        if (c == 0 && sx_out) sx_out[0] = sh_sx;      // CTA 0 owns chunk 0
       }
     }
     consumers_sync();
@@ -306,16 +313,21 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 1) k_chain(const ChainParams p
       uint32_t* seg = segbuf + (size_t)part * (NCOL * kColWords) + part_slot(w);
       uint32_t l[NCOL][4] = {};                                // zeros past K
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const float xf = bf16_bits_to_float((e & 1) ? (hv[j][e >> 1] >> 16) : (hv[j][e >> 1] & 0xFFFFu));
-        const int sh = 8 * (e & 3);
-        if (MODE == 0) {
-          int L[4];
-          limbs_of(limb_fixed(xf, E), L);
+      for (int g4 = 0; g4 < 4; ++g4) {                          // elements 4 g4 .. 4 g4 + 3
+        int X[4];
 #pragma unroll
-          for (int col = 0; col < NCOL; ++col) l[col][e >> 2] |= (uint32_t)(uint8_t)L[col] << sh;
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t w2 = hv[j][2 * g4 + (e >> 1)];
+          const float xf = bf16_bits_to_float((e & 1) ? (w2 >> 16) : (w2 & 0xFFFFu));
+          X[e] = MODE == 0 ? limb_fixed(xf, E) : quant_i8(xf, sxv);
+        }
+        if (MODE == 0) {
+          uint32_t o[4];
+          limbs4_of(X, o);
+#pragma unroll
+          for (int col = 0; col < NCOL; ++col) l[col][g4] = o[col];
         } else {
-          l[0][e >> 2] |= (uint32_t)(uint8_t)(int8_t)quant_i8(xf, sxv) << sh;
+          l[0][g4] = (X[0] & 0xFF) | ((X[1] & 0xFF) << 8) | ((X[2] & 0xFF) << 16) | ((uint32_t)X[3] << 24);
         }
       }
 #pragma unroll
@@ -330,25 +342,25 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 1) k_chain(const ChainParams p
     }
     consumers_sync();
     // ---- 4. this CTA's chunks: warps split the 16-row tiles, then a stage's parts -----------------
-    const int T = it.rows >> 4;                                 // tiles of a chunk (<= kCW)
+    const int T = rows >> 4;                                 // tiles of a chunk (<= kCW)
     const int wpt = kCW / T;                                    // warps per tile
     const bool active = warp < T * wpt;
     const int tile = warp % T, lg = warp / T;
-    const int rstride = 64 * it.ps;                             // bytes of one row of a plane in a stage
-    for (int ch = c; ch < it.chunks && ok; ch += G) {
-      const int r0 = ch * it.rows + tile * 16 + g;              // rows r0 (q = 0, 1) and r0 + 8 (q = 2, 3)
+    const int rstride = 64 * ps;                             // bytes of one row of a plane in a stage
+    for (int ch = c; ch < chunks && ok; ch += G) {
+      const int r0 = ch * rows + tile * 16 + g;              // rows r0 (q = 0, 1) and r0 + 8 (q = 2, 3)
       uint16_t sc_bits[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h)
-        sc_bits[h] = (active && lg == 0 && t == 0 && r0 + 8 * h < it.N) ? it.scale[r0 + 8 * h] : (uint16_t)0;
+        sc_bits[h] = (active && lg == 0 && t == 0 && r0 + 8 * h < N) ? scale[r0 + 8 * h] : (uint16_t)0;
       int acc4[4][4] = {};                                      // one chain per decode field f
-      for (int st = 0; st < it.nst; ++st) {
+      for (int st = 0; st < nst; ++st) {
         if (!(ok = mbar_wait(full0 + 8 * s, ph))) break;
         if (active) {
           const uint32_t rowa = ring + (uint32_t)s * kStageBytes + (uint32_t)((tile * 16 + g) * rstride + t * 16);
-          const uint32_t planeb = (uint32_t)(it.rows * rstride);
-          for (int pp = lg; pp < it.ps; pp += wpt) {
-            const int part = st * it.ps + pp;
+          const uint32_t planeb = (uint32_t)(rows * rstride);
+          for (int pp = lg; pp < ps; pp += wpt) {
+            const int part = st * ps + pp;
             if (part >= kp) break;
             const uint32_t ra = rowa + pp * 64;
             const uint4 ma = lds128(ra), mb = lds128(ra + 8 * rstride);
@@ -414,11 +426,11 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 1) k_chain(const ChainParams p
         if (t == 0) {
 #pragma unroll
           for (int h = 0; h < 2; ++h)
-            if (r0 + 8 * h < it.N) it.y[r0 + 8 * h] = y[h];
-          if (it.hout && r0 + 8 < it.N) {
+            if (r0 + 8 * h < N) yout[r0 + 8 * h] = y[h];
+          if (hout && r0 + 8 < N) {
             // SwiGLU epilogue: rows r0 (gate) and r0 + 8 (up) of the interleaved tile are one feature
             const double z = (double)y[0];
-            it.hout[(r0 - g) / 2 + g] = bf16_rn((z / (1.0 + exp(-z))) * (double)y[1]);
+            hout[(r0 - g) / 2 + g] = bf16_rn((z / (1.0 + exp(-z))) * (double)y[1]);
           }
         }
       }

@@ -164,6 +164,21 @@ __device__ __forceinline__ void limbs_of(int X, int (&L)[4]) {
   L[1] = (int)(int8_t)(X & 0xFF);
   L[0] = (X - L[1]) >> 8;                 // |L[0]| <= 64
 }
+// The limbs of four values at once, as four operand registers: out[c] holds limb c (top first) of
+// X[0..3] in bytes 0..3, the bytes limbs_of gives one value at a time. Balanced base-256 digits:
+// with Y = X + 0x808080 each of Y's three low bytes is its digit plus 128 and Y's top byte is the
+// top digit (|top| <= 64), so a 4 x 4 byte transpose of the Y's and a flip of bit 7 of the three
+// low digits make the operands.
+__device__ __forceinline__ void limbs4_of(const int (&X)[4], uint32_t (&out)[4]) {
+  const uint32_t y0 = (uint32_t)X[0] + 0x00808080u, y1 = (uint32_t)X[1] + 0x00808080u;
+  const uint32_t y2 = (uint32_t)X[2] + 0x00808080u, y3 = (uint32_t)X[3] + 0x00808080u;
+  const uint32_t a = __byte_perm(y0, y1, 0x5140), b = __byte_perm(y0, y1, 0x7362);   // bytes 0,1 | 2,3
+  const uint32_t c = __byte_perm(y2, y3, 0x5140), d = __byte_perm(y2, y3, 0x7362);
+  out[3] = __byte_perm(a, c, 0x5410) ^ 0x80808080u;            // byte 0 of each: the lowest limb
+  out[2] = __byte_perm(a, c, 0x7632) ^ 0x80808080u;
+  out[1] = __byte_perm(b, d, 0x5410) ^ 0x80808080u;
+  out[0] = __byte_perm(b, d, 0x7632);                           // byte 3: the top limb
+}
 // Exact recombination of the four limb sums S[0] (top) .. S[3]: fits int64 for K < 2^24.
 __device__ __forceinline__ long long limb_combine(long long s3, long long s2, long long s1, long long s0) {
   return s3 * 16777216LL + s2 * 65536LL + s1 * 256LL + s0;
