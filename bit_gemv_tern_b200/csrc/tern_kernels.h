@@ -113,7 +113,7 @@ struct BatchParams {
   CUtensorMap tmap[kBatchMaxItems];  // per item: planes viewed as [2 planes][N rows][K/32 words]
   BatchItem items[kBatchMaxItems];
   int32_t count;
-  int32_t mode;           // 0 = bf16 activations (three int8 limbs), 1 = int8
+  int32_t mode;           // 0 = bf16 activations (four int8 limbs), 1 = int8
   int32_t nc;             // operand columns of a segment
   int32_t M;              // activation rows (tokens), 1..16
   int32_t mp;             // token slots: 1, 2 / 4 (bf16 mode), 8 or 16

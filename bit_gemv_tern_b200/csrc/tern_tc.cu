@@ -12,7 +12,8 @@
 //   * the operand preparation (k_tc_prep, one CTA per item and token slot) writes each item's
 //     activation columns (four limbs per token, or the int8 q) as the MMA's B operand: per 512-trit
 //     part, four 128-trit chunks of N rows x 128 bytes in the 128-byte-swizzled K-major layout the
-//     tensor core reads from shared memory, in the decode's k order (permute_i8_half);
+//     tensor core reads from shared memory, in the decode's k order (permute_i8_half); an item
+//     with a prologue (tern_prologue.cuh) computes its activation first;
 //   * k_tc_stream (one CTA per SM) walks the same balanced (row block, part) sequence as the
 //     mma.sync stream, with row blocks of 256 rows (two groups of 128):
 //       warp 0      producer: per stage, the block's mask and sign words (tensor TMA, 64-byte
@@ -20,11 +21,13 @@
 //       warp 1      allocates 512 TMEM columns; one lane issues tcgen05.mma kind::i8 with A (the
 //                   weights) in TMEM and B in shared memory: M = 128 rows, N = the operand
 //                   columns, K = 32 per instruction, int32 accumulators in TMEM;
-//       warps 2..9  each thread owns one weight row (a TMEM lane): it decodes the row's 32-trit
-//                   words into signed bytes 64 * t (one shift and one AND per register, the signed
-//                   decode of tern_device.cuh) and stores them into TMEM with tcgen05.st, one
-//                   128-trit chunk at a time through four A slots; at the end of a row block the
-//                   same threads read their row's accumulators (tcgen05.ld) and write the outputs.
+//       warps 2..17 sixteen decoders, two per (row group, TMEM lane quarter): each thread owns one
+//                   weight row (a TMEM lane) and, for alternate 128-trit chunks of a stage,
+//                   decodes the row's 32-trit words into signed bytes 64 * t (one shift and one
+//                   AND per register, the signed decode of tern_device.cuh) and stores them into
+//                   TMEM with tcgen05.st through four A slots; at the end of a row block the
+//                   decoders of even chunks read their row's accumulators (tcgen05.ld) and write
+//                   the outputs.
 // Every sum is an exact integer (|64 t L| <= 2^13 per product, K <= 12288), so the outputs equal
 // the mma.sync path's bit for bit: int8 mode y = ((float)acc * s_x) * scale with two fp32
 // roundings, bf16 mode one fp64 -> fp32 rounding of the recombined limb sums. Every wait is bounded;
