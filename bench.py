@@ -638,6 +638,14 @@ def _profile_smallm(M):
     return run
 
 
+def _profile_chain(mode):
+    def run():
+        st = Stack("8b", M=1, layers=4)
+        ch = Chain(st, mode)
+        return ch.chain
+    return run
+
+
 def _profile_head(mode):
     def run():
         st = Stack("8b", M=1, layers=0)
@@ -698,6 +706,7 @@ PROFILE_CASES = {
     "batch-8b-4layers-int8": _profile_batch("int8"),
     "head-8b-bf16": _profile_head("bf16"),
     "smallm-8b-4layers-m8-bf16": _profile_smallm(8),
+    "chain-8b-4layers-bf16": _profile_chain("bf16"),
     "prefill-8b-gate-m4096": _profile_prefill("gate"),
     "base3-8b-1layer": _profile_base3(),
     "pack-8b-1layer": _profile_pack(),
@@ -1023,7 +1032,7 @@ def prefill_row(torch, tg, bf16_peak):
         m1 = timed_replays([(g1, reps)]) / reps
         per["x".join(map(str, (lin.N, lin.K)))] = {"ms": m1, "tflops": 2.0 * ps.M * lin.N * lin.K / (m1 / 1000.0) / 1e12}
     del ps
-    return {"ms_per_set": ms, "tflops": tf, "frac": tf / bf16_peak, "peak": "measured bf16 dense (burst)",
+    return {"ms_per_set": ms, "tflops": tf, "frac": tf / bf16_peak, "peak": f"{peaks()[3]} bf16 dense (burst)",
             "flops_per_set": 1.5805e12, "status": st, "shapes": per}
 
 
