@@ -140,8 +140,6 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 1) k_chain(const ChainParams p
   int* red = reinterpret_cast<int*>(segbuf + (size_t)p.seg_parts * NCOL * kColWords);
   __shared__ double dred[kCW];
   __shared__ float fred[kCW];
-  __shared__ int sh_E;
-  __shared__ float sh_sx;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = gridDim.x, c = blockIdx.x;
   const ChainItem* items = p.items;
@@ -291,19 +289,14 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 1) k_chain(const ChainParams p
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
     if (lane == 0) fred[warp] = amax;
     consumers_sync();
-    if (tid == 0) {
-      float mx = fred[0];
-      for (int w = 1; w < kCW; ++w) mx = fmaxf(mx, fred[w]);
-      if (MODE == 0) {
-        sh_E = limb_exponent(mx);
-      } else {
-        sh_sx = __fdiv_rn(mx, 127.0f);
-        if (c == 0 && sx_out) sx_out[0] = sh_sx;      // CTA 0 owns chunk 0
-      }
-    }
-    consumers_sync();
-    const int E = sh_E;
-    const float sxv = sh_sx;
+    // every thread reduces the warp maxima itself (one barrier instead of two); fred is next
+    // written after the operand build's barrier
+    float mx = fred[0];
+#pragma unroll
+    for (int w = 1; w < kCW; ++w) mx = fmaxf(mx, fred[w]);
+    const int E = MODE == 0 ? limb_exponent(mx) : 0;
+    const float sxv = MODE == 1 ? __fdiv_rn(mx, 127.0f) : 0.0f;
+    if (MODE == 1 && tid == 0 && c == 0 && sx_out) sx_out[0] = sxv;   // CTA 0 owns chunk 0
     // ---- 3. operand segments of every part, from the registers ------------------------------------
 #pragma unroll
     for (int j = 0; j < kJH; ++j) {
