@@ -410,20 +410,28 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_stream(const __grid_consta
         const BatchItem& B = p.items[it];
         const bool last_of_block = (part == B.kp - 1) || (q == n_stages - 1);
         if (!(ok = mbar_spin(full0 + 8 * s, ph))) break;
-        const uint32_t seg = ring + (uint32_t)s * slot_bytes + kRG * kBox;
-        for (int c = 0; c < 4 && ok; ++c, ++ac) {
-          const int a = ac % kNA;
-          if (!(ok = mbar_spin(afull0 + 8 * a, (uint32_t)((ac / kNA) & 1)))) break;
-          tc_fence_after();
+        // the stage's four chunks fill A slots 0..3 in order (kNA == 4), so every slot index, TMEM
+        // address and descriptor offset below is a constant of the unrolled code: a straight run of
+        // MMAs issues at the tensor core's own pace, a rolled loop around them costs far more
+        static_assert(kNA == 4, "one A slot per chunk of a stage");
+        const uint32_t aph = (uint32_t)((ac / kNA) & 1);
+        const uint64_t b0 = smem_desc_sw128(ring + (uint32_t)s * slot_bytes + kRG * kBox);
+        const uint32_t acc0 = first_of_block ? 0u : 1u;
 #pragma unroll
-          for (int g = 0; g < kRG; ++g)
+        for (int c = 0; c < 4; ++c) {
+          if (ok) ok = mbar_spin(afull0 + 8 * c, aph);
+          if (ok) {
+            tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-              mma_i8_ts(tmem + (uint32_t)(kDCol + 64 * g), tmem + (uint32_t)(kACol + 32 * (kRG * a + g) + 8 * ks),
-                        smem_desc_sw128(seg + (uint32_t)(c * N * 128 + 32 * ks)), kIdesc,
-                        (first_of_block && c == 0 && ks == 0) ? 0u : 1u);
-          mma_commit(aempty0 + 8 * a);                    // the A slot is free once these MMAs are done
+            for (int g = 0; g < kRG; ++g)
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks)
+                mma_i8_ts(tmem + (uint32_t)(kDCol + 64 * g), tmem + (uint32_t)(kACol + 32 * (kRG * c + g) + 8 * ks),
+                          b0 + (uint64_t)((c * N * 128 + 32 * ks) >> 4), kIdesc, (c == 0 && ks == 0) ? acc0 : 1u);
+            mma_commit(aempty0 + 8 * c);                  // the A slot is free once these MMAs are done
+          }
         }
+        ac += 4;
         if (!ok) break;
         mma_commit(empty0 + 8 * s);                       // the stage too (B read, planes decoded)
         if (last_of_block) mma_commit(dfull);             // the block's accumulators are complete

@@ -144,3 +144,23 @@ def test_chain_argument_errors():
                   tg.ChainItem(W, tg.TERN_PRO_BF16, y, src_item=0, src_h=True)], tg.TERN_ACT_BF16)
     with pytest.raises(tg.TernError):                   # RMSNorm needs a gain
         tg.Chain([tg.ChainItem(W, tg.TERN_PRO_RMSNORM, y, src=y)], tg.TERN_ACT_BF16)
+
+
+def test_chain_runs_read_only_their_own_outputs():
+    """Each run of one workspace reads only the outputs of that run: two entry vectors A and B run
+    as A, B, A, B give the first two runs' bits again (a linear that read a stale source would
+    mix the runs)."""
+    mats, items, ys, hs, sxs, specs, h0 = _build(52)
+    chain = tg.Chain(items, tg.TERN_ACT_BF16)
+    a = h0.clone()
+    b = dev(synth.residual(53, 0, 1, D).reshape(-1))
+    runs = []
+    for src in (a, b, a, b):
+        h0.copy_(src)
+        chain()
+        torch.cuda.synchronize()
+        assert tg.tern_device_status() == tg.TERN_OK
+        runs.append([host(y).view(np.uint32).copy() for y in ys] + [host(hs[2]).copy()])
+    for i in range(len(runs[0])):
+        assert (runs[0][i] == runs[2][i]).all() and (runs[1][i] == runs[3][i]).all(), i
+        assert not (runs[0][i] == runs[1][i]).all(), i
