@@ -192,6 +192,9 @@ __global__ void __launch_bounds__(kTcPrepThreads) k_tc_prep(const __grid_constan
   __shared__ float ssh;
   __shared__ __align__(16) uint16_t xs[kTcPrepMaxK];         // a prologue item's prepared bf16 row
   pdl_wait();
+  // the stream kernel may get resident now: its producer prefetches weights, and it waits for this
+  // grid's completion before it reads a segment
+  pdl_launch_dependents();
   {
     uint32_t* scr = reinterpret_cast<uint32_t*>(p.xprep + p.scratch_off);
     const int nct = gridDim.x * gridDim.y, ct = blockIdx.y * gridDim.x + blockIdx.x;
@@ -292,7 +295,6 @@ __global__ void __launch_bounds__(kTcPrepThreads) k_tc_prep(const __grid_constan
       }
     }
   }
-  pdl_launch_dependents();
 }
 
 // ---------------------------------------------------------------------------------------------
