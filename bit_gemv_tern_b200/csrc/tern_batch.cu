@@ -128,14 +128,22 @@ __host__ __device__ constexpr int seg_words(int mode, int mp) {
   return (seg_cols(mode, mp) * kColWords + seg_cols(mode, mp) + mp + 3) & ~3;
 }
 
-// prep: one CTA of kPrepThreads per (item, token slot), wide enough that each pass over an
-// activation of up to 8192 (int8: 16384) elements is a single round of loads. Block layout: kp
-// segments of seg_bytes. An item with a prologue first computes its bf16 row into shared memory
-// (tern_prologue.cuh), then encodes from there; int8 mode quantises that row per token here, so no
-// separate quantiser launch runs.
+// prep: one CTA of NT threads per (item, token slot). Block layout: kp segments of seg_bytes. An
+// item with a prologue first computes its bf16 row into shared memory (tern_prologue.cuh), then
+// encodes from there; int8 mode quantises that row per token here, so no separate quantiser launch
+// runs. Two shapes:
+//   PRO: lists with prologue items, 1024 threads (each pass over a row of up to 8192 elements is a
+//        single round of loads) and the row buffer in shared memory;
+//   !PRO: plain lists, 256 threads with at most 48 registers and no row buffer, so that a CTA fits
+//        on an SM next to a stream CTA (128 registers x 416 threads, ~205 KB of shared memory): the
+//        stream kernel, released at this kernel's entry, then gets resident on every SM at once
+//        instead of waiting for the prep CTAs to leave (measured: the 0.6B stack's stream CTAs
+//        started over a 2-12 us window behind 1024-thread prep CTAs).
 constexpr int kPrepThreads = 1024;
+constexpr int kPrepThreadsPlain = 256;
 constexpr int kPrepMaxK = 12288;
-__global__ void __launch_bounds__(kPrepThreads) k_batch_prep(const __grid_constant__ PrepParams p) {
+template <int NT, bool PRO>
+__global__ void __launch_bounds__(NT, PRO ? 1 : 5) k_batch_prep(const __grid_constant__ PrepParams p) {
   const PrepItem& it = p.items[blockIdx.x];
   const int m = blockIdx.y;                          // token slot (< mp)
   uint32_t* blk = reinterpret_cast<uint32_t*>(p.xprep + it.xoff);
@@ -143,16 +151,16 @@ __global__ void __launch_bounds__(kPrepThreads) k_batch_prep(const __grid_consta
   const int ncols = seg_cols(p.mode, mp);
   const int segw = p.seg_bytes / 4;
   const int nl = p.mode == 0 ? kLimbs : 1;           // columns of this token
-  const bool pro = it.kind != kProNone;
+  const bool pro = PRO && it.kind != kProNone;
   int colof[kLimbs];
   for (int l = 0; l < kLimbs; ++l) colof[l] = mp == 1 ? l : l * mp + m;
   const bool live = m < p.M;
-  __shared__ float red[kPrepThreads / 32];
-  __shared__ double dred[kPrepThreads / 32];
+  __shared__ float red[NT / 32];
+  __shared__ double dred[NT / 32];
   __shared__ int sums[kLimbs];
   __shared__ int Esh;
   __shared__ float ssh;
-  __shared__ __align__(16) uint16_t xs[kPrepMaxK];  // a prologue item's prepared bf16 row
+  __shared__ __align__(16) uint16_t xs[PRO ? kPrepMaxK : 8];  // a prologue item's prepared bf16 row
   pdl_wait();
   // let the stream kernel get resident now: its producer prefetches weights, which do not depend
   // on this kernel, and its consumers wait for this grid's completion before reading segments
@@ -183,9 +191,9 @@ __global__ void __launch_bounds__(kPrepThreads) k_batch_prep(const __grid_consta
     const size_t row_elems = (size_t)K * (it.kind == kProSwiGLU ? 2 : 1);
     const void* src = it.kind == kProBF16 ? static_cast<const void*>(static_cast<const uint16_t*>(it.x) + (size_t)m * K)
                                           : static_cast<const void*>(static_cast<const float*>(it.x) + (size_t)m * row_elems);
-    const double r = it.kind == kProRMSNorm ? rmsnorm_r<kPrepThreads>(static_cast<const float*>(src), K, it.eps, dred) : 1.0;
+    const double r = it.kind == kProRMSNorm ? rmsnorm_r<NT>(static_cast<const float*>(src), K, it.eps, dred) : 1.0;
     uint16_t* xo = (p.mode == 0 && it.xout) ? static_cast<uint16_t*>(it.xout) + (size_t)m * K : nullptr;
-    for (int k = threadIdx.x * 8; k < K; k += kPrepThreads * 8) {
+    for (int k = threadIdx.x * 8; k < K; k += NT * 8) {
       const uint4 v = prologue8(it.kind, src, it.gain, K, k, r);
       *reinterpret_cast<uint4*>(xs + k) = v;
       if (xo) *reinterpret_cast<uint4*>(xo + k) = v;
@@ -193,7 +201,7 @@ __global__ void __launch_bounds__(kPrepThreads) k_batch_prep(const __grid_consta
     }
   } else if (live && p.mode == 0) {
     const uint16_t* xb = static_cast<const uint16_t*>(it.x) + (size_t)m * K;
-    for (int k = threadIdx.x * 8; k < K; k += kPrepThreads * 8) amax = fmaxf(amax, absmax8(ld_nc(xb + k)));
+    for (int k = threadIdx.x * 8; k < K; k += NT * 8) amax = fmaxf(amax, absmax8(ld_nc(xb + k)));
   }
   if (live && (p.mode == 0 || pro)) {
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
@@ -201,7 +209,7 @@ __global__ void __launch_bounds__(kPrepThreads) k_batch_prep(const __grid_consta
     __syncthreads();
     if (threadIdx.x == 0) {
       float mx = red[0];
-      for (int i = 1; i < kPrepThreads / 32; ++i) mx = fmaxf(mx, red[i]);
+      for (int i = 1; i < NT / 32; ++i) mx = fmaxf(mx, red[i]);
       if (p.mode == 0) {
         Esh = limb_exponent(mx);
       } else {
@@ -324,8 +332,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
   if (g1 <= g0) return;
 
   // item, row block and part of the first stage
-  int first_item = 0;
-  while (first_item + 1 < p.count && p.items[first_item + 1].part0 <= g0) ++first_item;
+  const int first_item = p.cta_item[blockIdx.x];
   const int first_rb = (g0 - p.items[first_item].part0) / p.items[first_item].kp;
   const int first_part = (g0 - p.items[first_item].part0) - first_rb * p.items[first_item].kp;
 
@@ -820,6 +827,15 @@ bool plan_batch(BatchParams& p, const uint32_t* const* planes, size_t& smem, siz
     for (; c <= grid; ++c) p.cta_part[c] = parts;
     p.cta_part[grid] = parts;
   }
+  // each CTA's first item: a scan of items[] (kernel parameters, read through the constant cache)
+  // at the kernel's entry cost the last CTAs of a 112-item list up to 10 us before their first load
+  {
+    int i = 0;
+    for (int c = 0; c < grid; ++c) {
+      while (i + 1 < p.count && p.items[i + 1].part0 <= p.cta_part[c]) ++i;
+      p.cta_item[c] = (int16_t)i;
+    }
+  }
   // blocks shared by several CTAs: one scratch slot each, with its contributor count
   auto unit_of = [&](int gpart, int& ustart, int& uend) {
     int i = 0;
@@ -918,10 +934,19 @@ cudaError_t launch_batch(const BatchParams& p, const PrepParams& q, size_t smem,
   cfg.numAttrs = na;
   cfg.stream = st;
   // 1. operand segments: one CTA per (item, token slot)
+  bool any_pro = false;
+  for (int i = 0; i < q.count; ++i) any_pro = any_pro || q.items[i].kind != kProNone;
   cfg.gridDim = dim3(p.count, p.mp, 1);
-  cfg.blockDim = dim3(kPrepThreads, 1, 1);
+  cfg.blockDim = dim3(any_pro ? kPrepThreads : kPrepThreadsPlain, 1, 1);
   cfg.dynamicSmemBytes = 0;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, k_batch_prep, q);
+  cudaError_t e = cudaSuccess;
+  if (any_pro) {
+    e = cudaLaunchKernelEx(&cfg, k_batch_prep<kPrepThreads, true>, q);
+  } else {
+    static std::atomic<unsigned long long> carveout_set{0};
+    e = prefer_max_shared_carveout(k_batch_prep<kPrepThreadsPlain, false>, carveout_set);
+    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, k_batch_prep<kPrepThreadsPlain, false>, q);
+  }
   if (e != cudaSuccess) return e;
   // 2. the stream (always programmatically dependent on the prep launch)
   cudaLaunchAttribute attr2[1];

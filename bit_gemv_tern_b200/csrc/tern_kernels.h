@@ -54,6 +54,22 @@ cudaError_t allow_max_dynamic_smem(F* kern, std::atomic<unsigned long long>& don
   return e;
 }
 
+// Prefer the largest shared-memory carveout for a kernel that runs just before (and overlaps) a
+// kernel using nearly all of an SM's shared memory: an SM whose L1/shared split must change waits
+// until its resident CTAs have left, so a small kernel at the default carveout would hold the big
+// one off its SM. Set up once per device, as above.
+template <typename F>
+cudaError_t prefer_max_shared_carveout(F* kern, std::atomic<unsigned long long>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = (dev >= 0 && dev < 64) ? 1ull << dev : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
 // Ternary GEMV / small-M GEMM (tern_gemv.cu).
 struct GemmParams {
   const uint32_t* planes;
@@ -126,6 +142,7 @@ struct BatchParams {
   int32_t seg_bytes;      // operand bytes of one 512-trit part (all columns + sums + exponent)
   uint8_t* xprep;         // workspace: operand blocks
   int32_t cta_part[kMaxGridCTAs + 1];  // CTA c handles global parts [cta_part[c], cta_part[c + 1])
+  int16_t cta_item[kMaxGridCTAs];      // the item holding CTA c's first part (no scan of items[] at entry)
   // Row blocks split between CTAs: each contributor adds exact partial sums into a workspace
   // slot; the last one (per warp, by counter) writes the outputs.
   // per CTA, 8 bits each: slot of its first block + 1, that block's contributors, slot of its

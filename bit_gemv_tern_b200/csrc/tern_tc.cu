@@ -345,10 +345,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_stream(const __grid_consta
   bool ok = true;
 
   // item, row block and part of the first stage
-  int first_item = 0;
-  if (g1 > g0) {
-    while (first_item + 1 < p.count && p.items[first_item + 1].part0 <= g0) ++first_item;
-  }
+  const int first_item = g1 > g0 ? p.cta_item[blockIdx.x] : 0;
   const int fkp = p.items[first_item].kp;
   const int first_rb = g1 > g0 ? (g0 - p.items[first_item].part0) / fkp : 0;
   const int first_part = g1 > g0 ? (g0 - p.items[first_item].part0) - first_rb * fkp : 0;
