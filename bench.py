@@ -34,10 +34,10 @@ sys.path.insert(0, ROOT)
 
 METRIC = "ternary GEMV HBM GB/s & 8B linear-stack tok/s at M=1 (fraction of HBM peak)"
 # DRAM bytes (read + write) of the stream kernel per full 8B step, from an ncu capture of the
-# 4-layer profile case (batch-8b-4layers-bf16: 203.27 MB read + 6.39 MB written) scaled by the
+# 4-layer profile case (batch-8b-4layers-bf16: 195.43 MB read + 5.26 MB written) scaled by the
 # units processed (36 / 4 layers). None whenever that kernel has changed since the counters were
 # taken.
-STREAM_TRAFFIC_PER_STEP = 9 * (203.27e6 + 6.39e6)
+STREAM_TRAFFIC_PER_STEP = 9 * (195.43e6 + 5.26e6)
 SEED = 0x7E2A2026
 L2_BYTES = 126 * 1024 * 1024
 
