@@ -256,16 +256,8 @@ __global__ void __launch_bounds__(NT, PRO ? 1 : 5) k_batch_prep(const __grid_con
       store_operand_half(seg + colof[0] * kColWords, h, permute_i8_half(q));
     } else {
       const uint32_t wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-      uint32_t l[kLimbs][4] = {};
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const uint32_t bits = (e & 1) ? (wv[e >> 1] >> 16) : (wv[e >> 1] & 0xFFFFu);
-        int L[kLimbs];
-        limbs_of(limb_fixed(bf16_bits_to_float(bits), E), L);
-        const int sh = 8 * (e & 3);
-#pragma unroll
-        for (int c = 0; c < kLimbs; ++c) l[c][e >> 2] |= (uint32_t)(uint8_t)L[c] << sh;
-      }
+      uint32_t l[kLimbs][4];
+      limbs_of_bf16<4>(wv, E, l);
 #pragma unroll
       for (int c = 0; c < kLimbs; ++c) {
         ls[c] += bsum(l[c][0]) + bsum(l[c][1]) + bsum(l[c][2]) + bsum(l[c][3]);

@@ -179,6 +179,24 @@ __device__ __forceinline__ void limbs4_of(const int (&X)[4], uint32_t (&out)[4])
   out[1] = __byte_perm(b, d, 0x5410) ^ 0x80808080u;
   out[0] = __byte_perm(b, d, 0x7632);                           // byte 3: the top limb
 }
+// The limbs of 4·G bf16 values (packed two per word in wv, element 2i in the low half of word i)
+// relative to 2^E: l[c][g] holds limb c (top first) of elements 4g .. 4g + 3, one per byte.
+template <int G>
+__device__ __forceinline__ void limbs_of_bf16(const uint32_t (&wv)[2 * G], int E, uint32_t (&l)[4][G]) {
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    int X[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t w2 = wv[2 * g + (e >> 1)];
+      X[e] = limb_fixed(bf16_bits_to_float((e & 1) ? (w2 >> 16) : (w2 & 0xFFFFu)), E);
+    }
+    uint32_t o[4];
+    limbs4_of(X, o);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) l[c][g] = o[c];
+  }
+}
 // Exact recombination of the four limb sums S[0] (top) .. S[3]: fits int64 for K < 2^24.
 __device__ __forceinline__ long long limb_combine(long long s3, long long s2, long long s1, long long s0) {
   return s3 * 16777216LL + s2 * 65536LL + s1 * 256LL + s0;

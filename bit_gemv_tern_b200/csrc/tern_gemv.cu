@@ -116,16 +116,8 @@ __global__ void __launch_bounds__(kThreads) k_tern_gemm(const GemmParams p) {
       const uint16_t* xb = xs + (size_t)m * p.K + k0 + 16 * v;
       const uint4 a = ld_nc(xb), b = ld_nc(xb + 8);
       const uint32_t wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-      uint32_t l[4][4] = {};
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const uint32_t bits = (e & 1) ? (wv[e >> 1] >> 16) : (wv[e >> 1] & 0xFFFFu);
-        int L[4];
-        limbs_of(limb_fixed(bf16_bits_to_float(bits), E), L);
-        const int sh = 8 * (e & 3);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) l[c][e >> 2] |= (uint32_t)(uint8_t)L[c] << sh;
-      }
+      uint32_t l[4][4];
+      limbs_of_bf16<4>(wv, E, l);
 #pragma unroll
       for (int c = 0; c < 4; ++c)
         *reinterpret_cast<uint4*>(smem + (4 * m + c) * RS + gemm_half_ofs(v)) =

@@ -112,16 +112,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_head(const HeadParams p) {
       const int E = expo[m];
       const uint4 val = ld_nc(xb + (size_t)m * p.K + k0 + 8 * v);
       const uint32_t w[4] = {val.x, val.y, val.z, val.w};
-      uint32_t l[4][2] = {};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const uint32_t bits = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
-        int L[4];
-        limbs_of(limb_fixed(bf16_bits_to_float(bits), E), L);
-        const int sh = 8 * (e & 3);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) l[c][e >> 2] |= (uint32_t)(uint8_t)L[c] << sh;
-      }
+      uint32_t l[4][2];
+      limbs_of_bf16<2>(w, E, l);
 #pragma unroll
       for (int c = 0; c < 4; ++c) *reinterpret_cast<uint2*>(smem + (4 * m + c) * RS + 2 * v) = make_uint2(l[c][0], l[c][1]);
     }

@@ -195,20 +195,8 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_tern_stream(const StreamPa
       uint4 a2 = a, b2 = b;
       if (!(mine && v == lane)) { a2 = ld_nc(xb + 16 * v); b2 = ld_nc(xb + 16 * v + 8); }
       const uint32_t wv[8] = {a2.x, a2.y, a2.z, a2.w, b2.x, b2.y, b2.z, b2.w};
-      uint32_t l[NC][4];
-#pragma unroll
-      for (int g4 = 0; g4 < 4; ++g4) {               // four values at a time: one byte transpose
-        int X[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t w2 = wv[2 * g4 + (e >> 1)];
-          X[e] = limb_fixed(bf16_bits_to_float((e & 1) ? (w2 >> 16) : (w2 & 0xFFFFu)), E);
-        }
-        uint32_t o[4];
-        limbs4_of(X, o);
-#pragma unroll
-        for (int c = 0; c < NC; ++c) l[c][g4] = o[c];
-      }
+      uint32_t l[4][4];
+      limbs_of_bf16<4>(wv, E, l);
       const int o = slot_of(v);
 #pragma unroll
       for (int c = 0; c < NC; ++c) {

@@ -277,16 +277,7 @@ __global__ void __launch_bounds__(kTcPrepThreads) k_tc_prep(const __grid_constan
       *reinterpret_cast<uint4*>(base + n * 128 + ((u ^ (n & 7)) << 4)) = q;
     } else {
       uint32_t l[4][4] = {};
-      if (have) {
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const uint32_t bits = (e & 1) ? (wv[e >> 1] >> 16) : (wv[e >> 1] & 0xFFFFu);
-          int L[4];
-          limbs_of(limb_fixed(bf16_bits_to_float(bits), E), L);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) l[c][e >> 2] |= (uint32_t)(uint8_t)L[c] << (8 * (e & 3));
-        }
-      }
+      if (have) limbs_of_bf16<4>(wv, E, l);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int n = 4 * m + c;
