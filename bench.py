@@ -679,6 +679,33 @@ def _profile_base3():
     return run
 
 
+def _profile_fv5():
+    def run():
+        import torch
+        import synth
+        import synth.cuda as sc
+        import bit_gemv_tern_b200 as tg
+        gen = torch.Generator(device="cuda").manual_seed(SEED)
+        flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+        entries = []
+        for p, N, K in synth.linear_shapes("8b"):
+            t = torch.empty(N * K, dtype=torch.int8, device="cuda")
+            h = torch.empty(N * K, dtype=torch.int8, device="cuda")
+            sc.trits_into(t, SEED, synth.tensor_id(1, p), K)
+            sc.trits_into(h, SEED + 1, synth.tensor_id(1, p), K)
+            codes = t * (1 + (h == 1).to(torch.int8))
+            del t, h
+            planes = torch.empty(N * 3 * K // 32, dtype=torch.int32, device="cuda")
+            tg.tern_fv5_pack(codes, N, K, planes, flag)
+            del codes
+            lo = 0.01 + 0.04 * torch.rand(N * (K // 256), device="cuda", generator=gen)
+            scales = torch.stack([lo, lo * (2 + torch.rand(N * (K // 256), device="cuda", generator=gen))], 1).contiguous()
+            x = torch.from_numpy(synth.activations(SEED, 8000 + K, 1, K).view(np.int16)).cuda()
+            entries.append((tg.Fv5Matrix(planes, scales, N, K), x, None, torch.empty(N, dtype=torch.float32, device="cuda")))
+        return lambda: tg.tern_fv5_gemv_batch(entries, tg.TERN_ACT_BF16)
+    return run
+
+
 def _profile_pack():
     def run():
         import torch
@@ -700,6 +727,8 @@ def _profile_pack():
 #   head-8b-*:          the int8 head 151936 x 4096 (622 MB)
 #   prefill-8b-gate-*:  one 12288 x 4096 linear at M = 4096 tokens (tcgen05 prefill)
 #   base3-8b-1layer:    the transport of one 8B layer's seven tensors (86.9 MB) in one batched call
+#   fv5-8b-1layer-batched: one 8B layer's seven linears as five-valued weights (78.6 MB), M = 1, bf16,
+#                       in one tern_fv5_gemv_batch call
 #   pack-8b-1layer:     the int8 trits of one 8B layer's seven tensors (193 MB) in one batched call
 PROFILE_CASES = {
     "batch-8b-4layers-bf16": _profile_batch("bf16"),
@@ -709,6 +738,7 @@ PROFILE_CASES = {
     "chain-8b-4layers-bf16": _profile_chain("bf16"),
     "prefill-8b-gate-m4096": _profile_prefill("gate"),
     "base3-8b-1layer": _profile_base3(),
+    "fv5-8b-1layer-batched": _profile_fv5(),
     "pack-8b-1layer": _profile_pack(),
 }
 
@@ -1224,7 +1254,16 @@ def fv5_rows(stack, torch, tg, hbm_peak):
     out = {"linears_3_layers_m1_bf16": {"ms": ms, "gbs": nbytes / (ms / 1000.0) / 1e9,
                                         "frac": nbytes / (ms / 1000.0) / 1e9 / hbm_peak, "bytes": nbytes,
                                         "launches": len(mats), "bits_per_weight": 3.25}}
-    del mats, g
+    del g
+    # the same 21 linears as one tern_fv5_gemv_batch call (one persistent launch)
+    entries = [(W, xs[W.K], None, y) for W, y in zip(mats, ys)]
+    g = capture(lambda i: tg.tern_fv5_gemv_batch(entries, tg.TERN_ACT_BF16), 2)
+    g.replay()
+    torch.cuda.synchronize()
+    ms = timed_replays([(g, 5)]) / 10
+    out["linears_3_layers_m1_bf16_batched"] = {"ms": ms, "gbs": nbytes / (ms / 1000.0) / 1e9,
+                                               "frac": nbytes / (ms / 1000.0) / 1e9 / hbm_peak, "launches": 1}
+    del mats, g, entries
     V, d = stack.V, stack.d
     S = (0.001 + 0.02 * torch.rand(V * (d // 256), device="cuda", generator=gen)).contiguous()
     xb = torch.from_numpy(synth.activations(SEED, 8100, 1, d).view(np.int16)).cuda()

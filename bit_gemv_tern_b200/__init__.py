@@ -26,7 +26,8 @@ __all__ = [
     "tern_gemm_batch_workspace_bytes", "tern_gemm_batch_pro", "tern_act_prologue",
     "i8_head_verify", "tern_verify_accept",
     "ChainItem", "Chain",
-    "Fv5Matrix", "tern_fv5_packed_bytes", "tern_fv5_pack", "tern_fv5_gemm", "fv5b_head_gemv_argmax",
+    "Fv5Matrix", "tern_fv5_packed_bytes", "tern_fv5_pack", "tern_fv5_gemm", "tern_fv5_gemv_batch",
+    "fv5b_head_gemv_argmax",
     "tern_rans_payload_bound", "tern_rans_workspace_bytes", "tern_rans_encode", "tern_rans_decode",
     "TERN_PRO_NONE", "TERN_PRO_BF16", "TERN_PRO_CAST", "TERN_PRO_RMSNORM", "TERN_PRO_SWIGLU",
     "tern_status_string",
@@ -99,6 +100,7 @@ def lib() -> ctypes.CDLL:
             "tern_fv5_packed_bytes": ([i32, i32], sz),
             "tern_fv5_pack": ([vp, i32, i32, vp, vp, vp], i32),
             "tern_fv5_gemm": ([vp, i32, i32, vp, vp, vp, vp], i32),
+            "tern_fv5_gemv_batch": ([vp, i32, i32, vp], i32),
             "fv5b_head_gemv_argmax": ([vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp], i32),
             "tern_rans_payload_bound": ([i32, i32], sz),
             "tern_rans_workspace_bytes": ([i32, i32], sz),
@@ -338,6 +340,18 @@ def tern_fv5_pack(codes, N: int, K: int, planes, err_flag, stream=None) -> None:
 
 def tern_fv5_gemm(W: Fv5Matrix, M: int, act: int, X, x_scale, Y, stream=None) -> None:
     _check(lib().tern_fv5_gemm(W.ref(), M, act, _ptr(X), _ptr(x_scale), _ptr(Y), _stream(stream)), "tern_fv5_gemm")
+
+
+class _Fv5BatchItem(ctypes.Structure):
+    _fields_ = [("W", _Fv5Matrix), ("x", ctypes.c_void_p), ("x_scale", ctypes.c_void_p), ("y", ctypes.c_void_p)]
+
+
+def tern_fv5_gemv_batch(entries, act: int, stream=None) -> None:
+    """entries: list of (Fv5Matrix, x, x_scale or None, y) at M = 1, run in one launch."""
+    arr = (_Fv5BatchItem * len(entries))()
+    for i, (W, x, sx, y) in enumerate(entries):
+        arr[i] = _Fv5BatchItem(W._c, _ptr(x), _ptr(sx), _ptr(y))
+    _check(lib().tern_fv5_gemv_batch(arr, len(entries), act, _stream(stream)), "tern_fv5_gemv_batch")
 
 
 def fv5b_head_gemv_argmax(W, block_scale, V: int, K: int, M: int, act: int, X, x_scale, argmax, maxval, logits,

@@ -561,6 +561,40 @@ tern_status tern_fv5_gemm(const tern_fv5_matrix* W, int32_t M, tern_act act, con
   return from_cuda(tern::launch_fv5_gemm(p, cs(stream)));
 }
 
+tern_status tern_fv5_gemv_batch(const tern_fv5_batch_item* items, int32_t count, tern_act act, tern_stream_t stream) {
+  if (!items) return TERN_EINVAL;
+  if (act != TERN_ACT_BF16 && act != TERN_ACT_INT8) return TERN_EINVAL;
+  if (count < 1 || count > TERN_FV5_BATCH_MAX_ITEMS || count > tern::kBatchMaxItems) return TERN_ESHAPE;
+  tern::Fv5BatchParams* p = new (std::nothrow) tern::Fv5BatchParams();
+  if (!p) return TERN_EINVAL;
+  tern_status st = TERN_OK;
+  for (int i = 0; i < count && st == TERN_OK; ++i) {
+    const tern_fv5_batch_item& in = items[i];
+    if (!in.W.planes || !in.W.scales || !in.x_dev || !in.y_dev) st = TERN_EINVAL;
+    else if (in.W.N <= 0 || in.W.K <= 0 || in.W.K % 512 || in.W.K > 12288) st = TERN_ESHAPE;
+    else if (!aligned(in.W.planes, 16) || !aligned(in.W.scales, 8) || !aligned(in.x_dev, 16) || !aligned(in.y_dev, 4))
+      st = TERN_EINVAL;
+    else if (act == TERN_ACT_INT8 && (!in.x_scale_dev || !aligned(in.x_scale_dev, 4))) st = TERN_EINVAL;
+    else {
+      tern::Fv5BatchItem& it = p->items[i];
+      it.planes = in.W.planes;
+      it.scales = in.W.scales;
+      it.x = in.x_dev;
+      it.sx = act == TERN_ACT_INT8 ? in.x_scale_dev : nullptr;
+      it.y = in.y_dev;
+      it.N = in.W.N;
+      it.K = in.W.K;
+    }
+  }
+  if (st == TERN_OK) {
+    p->count = count;
+    p->mode = act == TERN_ACT_BF16 ? 0 : 1;
+    st = from_cuda(tern::launch_fv5_batch(*p, cs(stream)));
+  }
+  delete p;
+  return st;
+}
+
 tern_status fv5b_head_gemv_argmax(const int8_t* W_dev, const float* block_scale_dev, int32_t V, int32_t K, int32_t M,
                                   tern_act act, const void* X_dev, const float* x_scale_dev, int32_t* argmax_dev,
                                   float* maxval_dev, float* logits_dev, void* workspace_dev, size_t workspace_bytes,

@@ -261,6 +261,215 @@ __global__ void __launch_bounds__(kThreads) k_fv5_gemm(const Fv5Params p) {
   if (p.ksplit > 1) cluster.sync();
 }
 
+// ---- a list of linears at M = 1 in one persistent launch ---------------------------------------------
+// Work units are tiles of 16 rows of one item over the whole of K; CTA c takes a contiguous,
+// cost-balanced range of them. It walks its range one item at a time: the CTA stages the item's
+// activation (as above, all K), then its warps take the item's tiles in turn, each streaming its 16
+// rows with two chunks in flight (a warp's next tile is fetched while it forms this one's outputs),
+// with the same block-by-block products and fp64 sums as k_fv5_gemm, and writing its rows' outputs
+// itself: with K whole in the warp no other warp's partial sums are needed.
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 2) k_fv5_batch(const __grid_constant__ Fv5BatchParams p) {
+  extern __shared__ __align__(16) uint32_t smem[];         // the current item's activation columns
+  __shared__ float fred[kThreads / 32];
+  __shared__ int expo_s;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int u0 = p.cta_unit[blockIdx.x], u1 = p.cta_unit[blockIdx.x + 1];
+  if (u0 >= u1) return;
+  constexpr int NC = MODE == 0 ? 4 : 1;
+  // the tile being fetched: its rows and plane pointers of this lane's rows ra, rb
+  int f_KM = 0, f_nchunks = 0, f_row0 = 0, f_u = -1;           // f_u: the tile fetched, or -1
+  bool f_live = false;
+  const uint32_t *pa = nullptr, *pb = nullptr;
+  auto set_tile = [&](int item, int u) {
+    const Fv5BatchItem& I = p.items[item];
+    f_u = u;
+    f_row0 = (u - p.unit0[item]) * 16;
+    f_KM = I.K >> 5;
+    f_nchunks = I.K >> 9;
+    f_live = true;
+    const int ra = min(f_row0 + g, I.N - 1), rb = min(f_row0 + g + 8, I.N - 1);
+    pa = I.planes + (size_t)ra * (3 * f_KM);
+    pb = I.planes + (size_t)rb * (3 * f_KM);
+  };
+  auto load_chunk = [&](int c, uint4 (&w)[6]) {
+    const int off = 16 * c + 4 * t;
+    if (f_live && c < f_nchunks) {
+      w[0] = ld_stream(pa + off);
+      w[1] = ld_stream(pb + off);
+      w[2] = ld_stream(pa + f_KM + off);
+      w[3] = ld_stream(pb + f_KM + off);
+      w[4] = ld_stream(pa + 2 * f_KM + off);
+      w[5] = ld_stream(pb + 2 * f_KM + off);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 6; ++i) w[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  uint4 cur[6], nxt[6];
+  int item = p.cta_item[blockIdx.x];
+  // this warp's first tile of the first segment, fetched before the dependency wait
+  {
+    const int s1 = min(u1, p.unit0[item + 1]);
+    if (u0 + warp < s1) {
+      set_tile(item, u0 + warp);
+      load_chunk(0, cur);
+      load_chunk(1, nxt);
+    }
+  }
+  pdl_wait();
+  for (int s0 = u0; s0 < u1; ++item) {
+    while (p.unit0[item + 1] <= s0) ++item;                 // the item of this segment
+    const int s1 = min(u1, p.unit0[item + 1]);               // tiles [s0, s1) of this item
+    const Fv5BatchItem& I = p.items[item];
+    const int K = I.K, RS = col_words(K), nblk = K >> 8;
+    // ---- stage the item's activation as int8 operand columns --------------------------------------
+    __syncthreads();                                         // the previous item's columns are read
+    const int per_row = K >> 4;
+    if (MODE == 1) {
+      const int8_t* xs = static_cast<const int8_t*>(I.x);
+      for (int v = threadIdx.x; v < per_row; v += kThreads)
+        *reinterpret_cast<uint4*>(smem + half_ofs(v)) = permute_i8_half(ld_nc(xs + 16 * v));
+    } else {
+      const uint16_t* xs = static_cast<const uint16_t*>(I.x);
+      float amax = 0.0f;
+      for (int k = threadIdx.x * 8; k < K; k += kThreads * 8) {
+        const uint4 v = ld_nc(xs + k);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          amax = fmaxf(amax, fmaxf(fabsf(bf16_bits_to_float(w[e] & 0xFFFFu)), fabsf(bf16_bits_to_float(w[e] >> 16))));
+      }
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+      if (lane == 0) fred[warp] = amax;
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        float mx = fred[0];
+        for (int i = 1; i < kThreads / 32; ++i) mx = fmaxf(mx, fred[i]);
+        expo_s = limb_exponent(mx);
+      }
+      __syncthreads();
+      const int E = expo_s;
+      for (int v = threadIdx.x; v < per_row; v += kThreads) {
+        const uint16_t* xb = xs + 16 * v;
+        const uint4 a = ld_nc(xb), b = ld_nc(xb + 8);
+        const uint32_t wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        uint32_t l[4][4];
+        limbs_of_bf16<4>(wv, E, l);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(smem + c * RS + half_ofs(v)) =
+              permute_i8_half(make_uint4(l[c][0], l[c][1], l[c][2], l[c][3]));
+      }
+    }
+    __syncthreads();
+    // a warp that had no tile in the previous segment has not fetched its first one of this segment
+    if (s0 + warp < s1 && f_u != s0 + warp) {
+      set_tile(item, s0 + warp);
+      load_chunk(0, cur);
+      load_chunk(1, nxt);
+    }
+    // ---- this warp's tiles of the segment: s0 + warp, s0 + warp + 8, ... -----------------------------
+    for (int u = s0 + warp; u < s1; u += kThreads / 32) {
+      const int row0 = f_row0, nchunks = f_nchunks;
+      const int ra = min(row0 + g, I.N - 1), rb = min(row0 + g + 8, I.N - 1);
+      const float2* sca = reinterpret_cast<const float2*>(I.scales) + (size_t)ra * nblk;
+      const float2* scb = reinterpret_cast<const float2*>(I.scales) + (size_t)rb * nblk;
+      double Y[4] = {0.0, 0.0, 0.0, 0.0};
+      for (int c = 0; c < nchunks; ++c) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {               // the chunk's two 256-weight blocks
+          int accL[4] = {0, 0, 0, 0}, accH[4] = {0, 0, 0, 0};
+#pragma unroll
+          for (int ee = 0; ee < 2; ++ee) {
+            const int e = 2 * half + ee;
+            const int w = 16 * c + 4 * e + t;                // logical word of this lane
+            const uint32_t ga = u4get(cur[4], e), gb = u4get(cur[5], e);
+            uint32_t la0, lb0, la1, lb1, ha0, hb0, ha1, hb1;
+            merge_planes(u4get(cur[0], e) & ~ga, u4get(cur[2], e) & ~(ga << 1 | ga >> 31), la0, lb0);
+            merge_planes(u4get(cur[1], e) & ~gb, u4get(cur[3], e) & ~(gb << 1 | gb >> 31), la1, lb1);
+            merge_planes(u4get(cur[0], e) & ga, u4get(cur[2], e) & (ga << 1 | ga >> 31), ha0, hb0);
+            merge_planes(u4get(cur[1], e) & gb, u4get(cur[3], e) & (gb << 1 | gb >> 31), ha1, hb1);
+            const uint32_t AL[8][2] = {
+                {dec_i8<0>(la0, lb0), dec_i8<0>(la1, lb1)}, {dec_i8<1>(la0, lb0), dec_i8<1>(la1, lb1)},
+                {dec_i8<2>(la0, lb0), dec_i8<2>(la1, lb1)}, {dec_i8<3>(la0, lb0), dec_i8<3>(la1, lb1)},
+                {dec_i8<4>(la0, lb0), dec_i8<4>(la1, lb1)}, {dec_i8<5>(la0, lb0), dec_i8<5>(la1, lb1)},
+                {dec_i8<6>(la0, lb0), dec_i8<6>(la1, lb1)}, {dec_i8<7>(la0, lb0), dec_i8<7>(la1, lb1)}};
+            const uint32_t AH[8][2] = {
+                {dec_i8<0>(ha0, hb0), dec_i8<0>(ha1, hb1)}, {dec_i8<1>(ha0, hb0), dec_i8<1>(ha1, hb1)},
+                {dec_i8<2>(ha0, hb0), dec_i8<2>(ha1, hb1)}, {dec_i8<3>(ha0, hb0), dec_i8<3>(ha1, hb1)},
+                {dec_i8<4>(ha0, hb0), dec_i8<4>(ha1, hb1)}, {dec_i8<5>(ha0, hb0), dec_i8<5>(ha1, hb1)},
+                {dec_i8<6>(ha0, hb0), dec_i8<6>(ha1, hb1)}, {dec_i8<7>(ha0, hb0), dec_i8<7>(ha1, hb1)}};
+            uint32_t xb[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+            if (g < NC) {
+#pragma unroll
+              for (int q = 0; q < 2; ++q) {
+                const uint4 v = *reinterpret_cast<const uint4*>(smem + g * RS + half_ofs(2 * w + q));
+                xb[4 * q] = v.x; xb[4 * q + 1] = v.y; xb[4 * q + 2] = v.z; xb[4 * q + 3] = v.w;
+              }
+            }
+#pragma unroll
+            for (int r = 0; r < 8; r += 2) {
+              mma_s8(accL, AL[r][0], AL[r][1], AL[r + 1][0], AL[r + 1][1], xb[r], xb[r + 1]);
+              mma_s8(accH, AH[r][0], AH[r][1], AH[r + 1][0], AH[r + 1][1], xb[r], xb[r + 1]);
+            }
+          }
+          // the block's exact sums (acc = 64 * sum), scaled by its s_lo and s_hi, into fp64
+          const int blk = 2 * c + half;
+          const float2 sa = __ldg(sca + blk), sb = __ldg(scb + blk);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 s2 = (i >> 1) ? sb : sa;
+            Y[i] += (double)s2.x * (double)(accL[i] >> 6) + (double)s2.y * (double)(accH[i] >> 6);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 6; ++i) cur[i] = nxt[i];
+        load_chunk(c + 2, nxt);
+      }
+      // this warp's next tile streams in while this tile's outputs are formed: the next of this
+      // segment, else its first of the next segment (whose item is staged after the barrier)
+      {
+        int nu = u + kThreads / 32, nitem = item;
+        if (nu >= s1 && s1 < u1) {
+          nitem = item + 1;
+          while (p.unit0[nitem + 1] <= s1) ++nitem;
+          nu = s1 + warp;
+          if (nu >= min(u1, p.unit0[nitem + 1])) nu = u1;    // no tile for this warp there
+        }
+        if (nu < u1 && (nu < s1 || nitem != item)) {
+          set_tile(nitem, nu);
+          load_chunk(0, cur);
+          load_chunk(1, nxt);
+        } else {
+          f_live = false;
+          f_u = -1;
+        }
+      }
+      // ---- outputs: lane t = 0 holds columns 0, 1 of rows g and g + 8, lane t = 1 columns 2, 3 -----
+      double w2[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) w2[i] = __shfl_down_sync(0xFFFFFFFFu, Y[i], 1);
+      if (t == 0) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int row = row0 + g + 8 * h;
+          if (row >= I.N) continue;
+          float yv;
+          if (MODE == 1) {
+            yv = (float)((double)I.sx[0] * Y[2 * h]);
+          } else {
+            yv = (float)ldexp(((Y[2 * h] * 256.0 + Y[2 * h + 1]) * 256.0 + w2[2 * h]) * 256.0 + w2[2 * h + 1],
+                              expo_s - kLimbFrac);
+          }
+          I.y[row] = yv;
+        }
+      }
+    }
+    s0 = s1;
+  }
+}
+
 template <int MODE, int NG>
 cudaError_t launch_fv5_one(const Fv5Params& p, size_t smem, cudaStream_t st) {
   auto kern = k_fv5_gemm<MODE, NG>;
@@ -306,6 +515,59 @@ cudaError_t launch_fv5_gemm(const Fv5Params& p, cudaStream_t st) {
     case 3: return launch_fv5_one<0, 3>(p, smem, st);
     default: return launch_fv5_one<0, 4>(p, smem, st);
   }
+}
+
+cudaError_t launch_fv5_batch(Fv5BatchParams& p, cudaStream_t st) {
+  // units and their costs (rows x K), then contiguous cost-balanced ranges, one per CTA
+  int64_t units = 0, total = 0;
+  p.kmax = 0;
+  for (int i = 0; i < p.count; ++i) {
+    p.unit0[i] = (int32_t)units;
+    units += (p.items[i].N + 15) / 16;
+    total += (int64_t)p.items[i].N * p.items[i].K;
+    if (p.items[i].K > p.kmax) p.kmax = p.items[i].K;
+  }
+  if (units > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  p.unit0[p.count] = (int32_t)units;
+  // two CTAs per SM (16 warps: the decode and MMA chains of one CTA's 8 warps leave the SM idle)
+  long long g2 = 2LL * device_sm_count();
+  if (g2 > kFv5MaxCTAs) g2 = kFv5MaxCTAs;
+  if (g2 > units) g2 = units;
+  const int grid = (int)(g2 < 1 ? 1 : g2);
+  p.grid = grid;
+  {
+    int c = 1, it = 0;
+    int64_t acc = 0;
+    p.cta_unit[0] = 0;
+    for (int64_t u = 0; u < units && c < grid; ++u) {
+      while (it + 1 < p.count && p.unit0[it + 1] <= u) ++it;
+      const int rows = p.items[it].N - (int)(u - p.unit0[it]) * 16;
+      acc += (int64_t)(rows < 16 ? rows : 16) * p.items[it].K;
+      while (c < grid && acc * grid >= total * c) p.cta_unit[c++] = (int32_t)(u + 1);
+    }
+    for (; c <= grid; ++c) p.cta_unit[c] = (int32_t)units;
+    int i = 0;
+    for (c = 0; c < grid; ++c) {
+      while (i + 1 < p.count && p.unit0[i + 1] <= p.cta_unit[c]) ++i;
+      p.cta_item[c] = (int16_t)i;
+    }
+  }
+  const size_t smem = (size_t)(p.mode == 0 ? 4 : 1) * (p.kmax / 4 + 16) * 4;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  if (p.mode == 0) {
+    static std::atomic<unsigned long long> raised{0};
+    cudaError_t e = allow_max_dynamic_smem(k_fv5_batch<0>, raised);
+    if (e != cudaSuccess) return e;
+    return cudaLaunchKernelEx(&cfg, k_fv5_batch<0>, p);
+  }
+  static std::atomic<unsigned long long> raised1{0};
+  cudaError_t e = allow_max_dynamic_smem(k_fv5_batch<1>, raised1);
+  if (e != cudaSuccess) return e;
+  return cudaLaunchKernelEx(&cfg, k_fv5_batch<1>, p);
 }
 
 cudaError_t launch_fv5_pack(const int8_t* codes, int32_t N, int32_t K, uint32_t* planes, int32_t* flag,

@@ -317,6 +317,25 @@ struct Fv5Params {
   float* y;                   // [M][N]
   int32_t M, mode, kr, ksplit;
 };
+// A list of five-valued linears at M = 1 in one persistent launch (tern_fv5.cu): units of 128 rows
+// of one item over the whole of K, cut into contiguous, cost-balanced ranges per CTA.
+struct Fv5BatchItem {
+  const uint32_t* planes;
+  const float* scales;
+  const void* x;              // bf16 [K] or int8 [K]
+  const float* sx;            // int8 mode: [1]
+  float* y;                   // [N]
+  int32_t N, K;
+};
+constexpr int kFv5MaxCTAs = 2 * kMaxGridCTAs;   // two CTAs per SM
+struct Fv5BatchParams {
+  Fv5BatchItem items[kBatchMaxItems];
+  int32_t unit0[kBatchMaxItems + 1];   // first unit of each item; unit0[count] = all units
+  int32_t cta_unit[kFv5MaxCTAs + 1];   // CTA c takes units [cta_unit[c], cta_unit[c + 1])
+  int16_t cta_item[kFv5MaxCTAs];       // the item of CTA c's first unit
+  int32_t count, mode, grid, kmax;
+};
+cudaError_t launch_fv5_batch(Fv5BatchParams& p, cudaStream_t st);
 size_t fv5_smem_bytes(int mode, int M, int kr);
 int fv5_rows_per_cta();
 cudaError_t launch_fv5_gemm(const Fv5Params& p, cudaStream_t st);

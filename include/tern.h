@@ -492,6 +492,21 @@ tern_status tern_fv5_pack(const int8_t* codes_dev, int32_t N, int32_t K, uint32_
 tern_status tern_fv5_gemm(const tern_fv5_matrix* W, int32_t M, tern_act act, const void* X_dev, const float* x_scale_dev,
                           float* Y_dev, tern_stream_t stream);
 
+/* A list of five-valued linears at M = 1 in one persistent launch (the batched counterpart of
+ * tern_fv5_gemm for a decode step: no launch per linear). Item i: y_i[n] = sum_k w_i[n][k] x_i[k],
+ * x_i bf16 [K] or int8 [K] with x_scale_i [1] (int8 mode), y_i fp32 [N]; the same products and
+ * rounding as tern_fv5_gemm at M = 1, the block sums added in block order. 1 <= count <= 160;
+ * W, x (16-byte aligned), x_scale (int8 mode, 4-byte aligned) and y (4-byte aligned) device
+ * pointers, caller-owned; no workspace. Argument errors return before anything is enqueued. */
+typedef struct {
+  tern_fv5_matrix W;
+  const void* x_dev;
+  const float* x_scale_dev;
+  float* y_dev;
+} tern_fv5_batch_item;
+#define TERN_FV5_BATCH_MAX_ITEMS 160
+tern_status tern_fv5_gemv_batch(const tern_fv5_batch_item* items, int32_t count, tern_act act, tern_stream_t stream);
+
 /* The int8 head with one fp32 scale per row and 256-weight block (block_scale_dev: fp32
  * [V][K/256], 4-byte aligned; K % 256 == 0) instead of the fp16 row scale:
  *   logits[m][v] = sum_b block_scale[v][b] * sum_{k in b} W[v][k] x[m][k],

@@ -167,3 +167,71 @@ def test_fv5_invalid_codes_and_arguments():
     y = torch.zeros(9 * N, dtype=torch.float32, device="cuda")
     with pytest.raises(tg.TernError):
         tg.tern_fv5_gemm(W, 9, tg.TERN_ACT_BF16, x, None, y)             # bf16 mode M <= 8
+
+
+BATCH_SHAPES = [(37, 512), (300, 1024), (1024, 4096), (200, 12288), (129, 4096), (4096, 4096)]
+
+
+@pytest.mark.parametrize("mode", ["bf16", "int8"])
+def test_gemv_batch_matches_oracle(mode):
+    """tern_fv5_gemv_batch: a list of ragged shapes (N not a multiple of 128, K up to 12288) in one
+    launch against the oracle: int8 mode bit for bit (the block sums are added in block order, as the
+    oracle adds them), bf16 mode within the per-output bound; twice on the same outputs."""
+    act = tg.TERN_ACT_BF16 if mode == "bf16" else tg.TERN_ACT_INT8
+    entries, refs, bounds = [], [], []
+    for i, (N, K) in enumerate(BATCH_SHAPES):
+        W, c, s = _matrix(41 + i, N, K)
+        X = synth.activations(42 + i, 1, 1, K)
+        y = torch.full((N,), float("nan"), dtype=torch.float32, device="cuda")
+        if mode == "bf16":
+            entries.append((W, dev(X.view(np.int16)), None, y))
+            refs.append(oracle.fv5_gemm_bf16(oracle.fv5_pack(c), s, K, X)[0])
+            absx = np.abs(synth.bf16_bits_to_f32(X).astype(np.float64)).sum()
+            bounds.append(PER_OUT * absx * s.reshape(N, -1).max(1).astype(np.float64))
+        else:
+            q = torch.empty(K, dtype=torch.int8, device="cuda")
+            sx = torch.empty(1, dtype=torch.float32, device="cuda")
+            tg.tern_quantize_act(dev(X.view(np.int16)), 1, K, q, sx)
+            entries.append((W, q, sx, y))
+            refs.append(oracle.fv5_gemm_i8(oracle.fv5_pack(c), s, K, host(q).reshape(1, K), host(sx))[0])
+    for _ in range(2):
+        for (_, _, _, y) in entries:
+            y.fill_(float("nan"))
+        tg.tern_fv5_gemv_batch(entries, act)
+        torch.cuda.synchronize()
+        for i, (W, _, _, y) in enumerate(entries):
+            got = host(y)
+            if mode == "int8":
+                assert (got.view(np.uint32) == refs[i].astype(np.float32).view(np.uint32)).all(), BATCH_SHAPES[i]
+            else:
+                err = got.astype(np.float64) - refs[i]
+                assert (np.abs(err) <= bounds[i]).all(), BATCH_SHAPES[i]
+                assert np.linalg.norm(err) / np.linalg.norm(refs[i]) <= REL_L2
+
+
+def test_gemv_batch_equals_single_entry_bf16():
+    """bf16 mode: each item equals tern_fv5_gemm at M = 1 on K values one 512-weight slice long (a
+    single K slice there too, so the fp64 order is the same)."""
+    entries, singles = [], []
+    for i, N in enumerate([64, 300, 1000]):
+        W, c, s = _matrix(61 + i, N, 512)
+        X = dev(synth.activations(62 + i, 1, 1, 512).view(np.int16))
+        y = torch.empty(N, dtype=torch.float32, device="cuda")
+        y1 = torch.empty(N, dtype=torch.float32, device="cuda")
+        tg.tern_fv5_gemm(W, 1, tg.TERN_ACT_BF16, X, None, y1)
+        entries.append((W, X, None, y))
+        singles.append(y1)
+    tg.tern_fv5_gemv_batch(entries, tg.TERN_ACT_BF16)
+    torch.cuda.synchronize()
+    for (_, _, _, y), y1 in zip(entries, singles):
+        assert (host(y).view(np.uint32) == host(y1).view(np.uint32)).all()
+
+
+def test_gemv_batch_argument_errors():
+    W, c, s = _matrix(71, 64, 512)
+    x = torch.zeros(512, dtype=torch.int16, device="cuda")
+    y = torch.zeros(64, dtype=torch.float32, device="cuda")
+    with pytest.raises(tg.TernError):                 # int8 mode needs x_scale
+        tg.tern_fv5_gemv_batch([(W, x, None, y)], tg.TERN_ACT_INT8)
+    with pytest.raises(tg.TernError):                 # empty list
+        tg.tern_fv5_gemv_batch([], tg.TERN_ACT_BF16)
