@@ -264,10 +264,16 @@ __global__ void __launch_bounds__(kThreads) k_fv5_gemm(const Fv5Params p) {
 // ---- a list of linears at M = 1 in one persistent launch ---------------------------------------------
 // Work units are tiles of 16 rows of one item over the whole of K; CTA c takes a contiguous,
 // cost-balanced range of them. It walks its range one item at a time: the CTA stages the item's
-// activation (as above, all K), then its warps take the item's tiles in turn, each streaming its 16
-// rows with two chunks in flight (a warp's next tile is fetched while it forms this one's outputs),
-// with the same block-by-block products and fp64 sums as k_fv5_gemm, and writing its rows' outputs
-// itself: with K whole in the warp no other warp's partial sums are needed.
+// activation (all K) as the batched stream's operand words (tern_batch.cu: eight words per 32-trit
+// word, in natural word order here since the planes' word transposition already gives each quad
+// lane its word) together with each 256-weight block's column sums; then its warps take the item's
+// tiles in turn, each streaming its 16 rows with two chunks in flight (a warp's next tile is fetched
+// while it forms this one's outputs). A word's low- and high-magnitude parts take the offset decode
+// of the batched stream (one AND per operand register: field i in place reads 4^i (t + 2)), each
+// into its own four field accumulators; at a block's end the exact sums (the offset removed with
+// the block's column sums) are scaled by s_lo and s_hi into fp64, as in k_fv5_gemm, and each warp
+// writes its rows' outputs itself: with K whole in the warp no other warp's partial sums are
+// needed.
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 2) k_fv5_batch(const __grid_constant__ Fv5BatchParams p) {
   extern __shared__ __align__(16) uint32_t smem[];         // the current item's activation columns
@@ -322,15 +328,16 @@ __global__ void __launch_bounds__(kThreads, 2) k_fv5_batch(const __grid_constant
     while (p.unit0[item + 1] <= s0) ++item;                 // the item of this segment
     const int s1 = min(u1, p.unit0[item + 1]);               // tiles [s0, s1) of this item
     const Fv5BatchItem& I = p.items[item];
-    const int K = I.K, RS = col_words(K), nblk = K >> 8;
-    // ---- stage the item's activation as int8 operand columns --------------------------------------
+    const int K = I.K, nblk = K >> 8;
+    // ---- stage the item's activation: operand words and per-block column sums --------------------
+    const int RS = K / 4 + 4;                                // words per column (+4: the quarter-warp's
+                                                             // two columns' 128-bit reads miss each other)
+    int* bsum = reinterpret_cast<int*>(smem + NC * (p.kmax / 4 + 4));   // [NC][K / 256]
     __syncthreads();                                         // the previous item's columns are read
-    const int per_row = K >> 4;
-    if (MODE == 1) {
-      const int8_t* xs = static_cast<const int8_t*>(I.x);
-      for (int v = threadIdx.x; v < per_row; v += kThreads)
-        *reinterpret_cast<uint4*>(smem + half_ofs(v)) = permute_i8_half(ld_nc(xs + 16 * v));
-    } else {
+    for (int i = threadIdx.x; i < NC * nblk; i += kThreads) bsum[i] = 0;
+    const int per_row = K >> 4;                              // 16-element halves
+    int E = 0;
+    if (MODE == 0) {
       const uint16_t* xs = static_cast<const uint16_t*>(I.x);
       float amax = 0.0f;
       for (int k = threadIdx.x * 8; k < K; k += kThreads * 8) {
@@ -349,17 +356,33 @@ __global__ void __launch_bounds__(kThreads, 2) k_fv5_batch(const __grid_constant
         expo_s = limb_exponent(mx);
       }
       __syncthreads();
-      const int E = expo_s;
-      for (int v = threadIdx.x; v < per_row; v += kThreads) {
-        const uint16_t* xb = xs + 16 * v;
+      E = expo_s;
+    } else {
+      __syncthreads();                                       // bsum zeroed
+    }
+    for (int v = threadIdx.x; v < per_row; v += kThreads) {
+      const int w = v >> 1, h = v & 1, blk = v >> 4;
+      if (MODE == 1) {
+        const uint4 q = ld_nc(static_cast<const int8_t*>(I.x) + 16 * v);
+        atomicAdd(&bsum[blk], __dp4a((int)q.x, 0x01010101, 0) + __dp4a((int)q.y, 0x01010101, 0) +
+                                  __dp4a((int)q.z, 0x01010101, 0) + __dp4a((int)q.w, 0x01010101, 0));
+        const uint4 o = permute_i8_half(q);
+        uint32_t* slot = smem + w * 8;
+        slot[0 + h] = o.x; slot[2 + h] = o.y; slot[4 + h] = o.z; slot[6 + h] = o.w;
+      } else {
+        const uint16_t* xb = static_cast<const uint16_t*>(I.x) + 16 * v;
         const uint4 a = ld_nc(xb), b = ld_nc(xb + 8);
         const uint32_t wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
         uint32_t l[4][4];
         limbs_of_bf16<4>(wv, E, l);
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4*>(smem + c * RS + half_ofs(v)) =
-              permute_i8_half(make_uint4(l[c][0], l[c][1], l[c][2], l[c][3]));
+        for (int c = 0; c < 4; ++c) {
+          atomicAdd(&bsum[c * nblk + blk], __dp4a((int)l[c][0], 0x01010101, 0) + __dp4a((int)l[c][1], 0x01010101, 0) +
+                                               __dp4a((int)l[c][2], 0x01010101, 0) + __dp4a((int)l[c][3], 0x01010101, 0));
+          const uint4 o = permute_i8_half(make_uint4(l[c][0], l[c][1], l[c][2], l[c][3]));
+          uint32_t* slot = smem + c * RS + w * 8;
+          slot[0 + h] = o.x; slot[2 + h] = o.y; slot[4 + h] = o.z; slot[6 + h] = o.w;
+        }
       }
     }
     __syncthreads();
@@ -376,51 +399,52 @@ __global__ void __launch_bounds__(kThreads, 2) k_fv5_batch(const __grid_constant
       const float2* sca = reinterpret_cast<const float2*>(I.scales) + (size_t)ra * nblk;
       const float2* scb = reinterpret_cast<const float2*>(I.scales) + (size_t)rb * nblk;
       double Y[4] = {0.0, 0.0, 0.0, 0.0};
+      // accumulator register q holds row g + 8 (q >> 1), column 2t + (q & 1)
+      const int colq0 = 2 * t, colq1 = 2 * t + 1;
       for (int c = 0; c < nchunks; ++c) {
 #pragma unroll
         for (int half = 0; half < 2; ++half) {               // the chunk's two 256-weight blocks
-          int accL[4] = {0, 0, 0, 0}, accH[4] = {0, 0, 0, 0};
+          const int blk = 2 * c + half;
+          const int cs0 = colq0 < NC ? bsum[colq0 * nblk + blk] : 0;
+          const int cs1 = colq1 < NC ? bsum[colq1 * nblk + blk] : 0;
+          int v[2][4];                                       // [lo, hi] exact block sums
 #pragma unroll
-          for (int ee = 0; ee < 2; ++ee) {
-            const int e = 2 * half + ee;
-            const int w = 16 * c + 4 * e + t;                // logical word of this lane
-            const uint32_t ga = u4get(cur[4], e), gb = u4get(cur[5], e);
-            uint32_t la0, lb0, la1, lb1, ha0, hb0, ha1, hb1;
-            merge_planes(u4get(cur[0], e) & ~ga, u4get(cur[2], e) & ~(ga << 1 | ga >> 31), la0, lb0);
-            merge_planes(u4get(cur[1], e) & ~gb, u4get(cur[3], e) & ~(gb << 1 | gb >> 31), la1, lb1);
-            merge_planes(u4get(cur[0], e) & ga, u4get(cur[2], e) & (ga << 1 | ga >> 31), ha0, hb0);
-            merge_planes(u4get(cur[1], e) & gb, u4get(cur[3], e) & (gb << 1 | gb >> 31), ha1, hb1);
-            const uint32_t AL[8][2] = {
-                {dec_i8<0>(la0, lb0), dec_i8<0>(la1, lb1)}, {dec_i8<1>(la0, lb0), dec_i8<1>(la1, lb1)},
-                {dec_i8<2>(la0, lb0), dec_i8<2>(la1, lb1)}, {dec_i8<3>(la0, lb0), dec_i8<3>(la1, lb1)},
-                {dec_i8<4>(la0, lb0), dec_i8<4>(la1, lb1)}, {dec_i8<5>(la0, lb0), dec_i8<5>(la1, lb1)},
-                {dec_i8<6>(la0, lb0), dec_i8<6>(la1, lb1)}, {dec_i8<7>(la0, lb0), dec_i8<7>(la1, lb1)}};
-            const uint32_t AH[8][2] = {
-                {dec_i8<0>(ha0, hb0), dec_i8<0>(ha1, hb1)}, {dec_i8<1>(ha0, hb0), dec_i8<1>(ha1, hb1)},
-                {dec_i8<2>(ha0, hb0), dec_i8<2>(ha1, hb1)}, {dec_i8<3>(ha0, hb0), dec_i8<3>(ha1, hb1)},
-                {dec_i8<4>(ha0, hb0), dec_i8<4>(ha1, hb1)}, {dec_i8<5>(ha0, hb0), dec_i8<5>(ha1, hb1)},
-                {dec_i8<6>(ha0, hb0), dec_i8<6>(ha1, hb1)}, {dec_i8<7>(ha0, hb0), dec_i8<7>(ha1, hb1)}};
-            uint32_t xb[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-            if (g < NC) {
+          for (int part = 0; part < 2; ++part) {             // low magnitudes, then high: one set
+            int acc[4][4] = {};                              // of field accumulators live at a time
 #pragma unroll
-              for (int q = 0; q < 2; ++q) {
-                const uint4 v = *reinterpret_cast<const uint4*>(smem + g * RS + half_ofs(2 * w + q));
-                xb[4 * q] = v.x; xb[4 * q + 1] = v.y; xb[4 * q + 2] = v.z; xb[4 * q + 3] = v.w;
+            for (int ee = 0; ee < 2; ++ee) {
+              const int e = 2 * half + ee;
+              const int w = 16 * c + 4 * e + t;              // logical word of this lane
+              const uint32_t ga = u4get(cur[4], e), gb = u4get(cur[5], e);
+              const uint32_t ka = part ? ga : ~ga, kb = part ? gb : ~gb;
+              uint32_t a0, b0, a1, b1;
+              merge_planes_offset(u4get(cur[0], e) & ka, u4get(cur[2], e) & __funnelshift_l(ka, ka, 1), a0, b0);
+              merge_planes_offset(u4get(cur[1], e) & kb, u4get(cur[3], e) & __funnelshift_l(kb, kb, 1), a1, b1);
+              uint4 x01 = make_uint4(0u, 0u, 0u, 0u), x23 = x01;
+              if (g < NC) {
+                const uint32_t* xo = smem + g * RS + w * 8;
+                x01 = *reinterpret_cast<const uint4*>(xo);
+                x23 = *reinterpret_cast<const uint4*>(xo + 4);
+              }
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {                  // field i in place -> 4^i * (t + 2)
+                const uint32_t msk = 0x03030303u << (2 * i);
+                const uint32_t x0 = i < 2 ? u4get(x01, 2 * i) : u4get(x23, 2 * i - 4);
+                const uint32_t x1 = i < 2 ? u4get(x01, 2 * i + 1) : u4get(x23, 2 * i - 3);
+                mma_u8s8(acc[i], a0 & msk, a1 & msk, b0 & msk, b1 & msk, x0, x1);
               }
             }
+            // the offset 2 per weight removed with the block's column sums
 #pragma unroll
-            for (int r = 0; r < 8; r += 2) {
-              mma_s8(accL, AL[r][0], AL[r][1], AL[r + 1][0], AL[r + 1][1], xb[r], xb[r + 1]);
-              mma_s8(accH, AH[r][0], AH[r][1], AH[r + 1][0], AH[r + 1][1], xb[r], xb[r + 1]);
-            }
+            for (int q = 0; q < 4; ++q)
+              v[part][q] = acc[0][q] + (acc[1][q] >> 2) + (acc[2][q] >> 4) + (acc[3][q] >> 6) - 2 * ((q & 1) ? cs1 : cs0);
           }
-          // the block's exact sums (acc = 64 * sum), scaled by its s_lo and s_hi, into fp64
-          const int blk = 2 * c + half;
+          // scaled by the block's s_lo and s_hi, into fp64
           const float2 sa = __ldg(sca + blk), sb = __ldg(scb + blk);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float2 s2 = (i >> 1) ? sb : sa;
-            Y[i] += (double)s2.x * (double)(accL[i] >> 6) + (double)s2.y * (double)(accH[i] >> 6);
+          for (int q = 0; q < 4; ++q) {
+            const float2 s2 = (q >> 1) ? sb : sa;
+            Y[q] += (double)s2.x * (double)v[0][q] + (double)s2.y * (double)v[1][q];
           }
         }
 #pragma unroll
@@ -552,7 +576,8 @@ cudaError_t launch_fv5_batch(Fv5BatchParams& p, cudaStream_t st) {
       p.cta_item[c] = (int16_t)i;
     }
   }
-  const size_t smem = (size_t)(p.mode == 0 ? 4 : 1) * (p.kmax / 4 + 16) * 4;
+  const int nc = p.mode == 0 ? 4 : 1;
+  const size_t smem = (size_t)nc * (p.kmax / 4 + 4) * 4 + (size_t)nc * (p.kmax / 256) * 4;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
