@@ -748,13 +748,14 @@ tern_status tern_read_flag(const int32_t* err_flag_dev, tern_stream_t stream) {
 }
 
 tern_status tern_device_status(tern_stream_t stream) {
-  int v = 0, w = 0, x = 0, c = 0, t = 0;
+  int v = 0, w = 0, x = 0, c = 0, t = 0, f = 0;
   if (tern::read_and_clear_error_latch(&v, cs(stream)) != cudaSuccess) return TERN_ECUDA;
   if (tern::read_and_clear_batch_latch(&w) != cudaSuccess) return TERN_ECUDA;
   if (tern::read_and_clear_prefill_latch(&x) != cudaSuccess) return TERN_ECUDA;
   if (tern::read_and_clear_chain_latch(&c) != cudaSuccess) return TERN_ECUDA;
   if (tern::read_and_clear_tc_latch(&t) != cudaSuccess) return TERN_ECUDA;
-  return (v == 0 && w == 0 && x == 0 && c == 0 && t == 0) ? TERN_OK : TERN_ETIMEOUT;
+  if (tern::read_and_clear_fv5_latch(&f) != cudaSuccess) return TERN_ECUDA;
+  return (v == 0 && w == 0 && x == 0 && c == 0 && t == 0 && f == 0) ? TERN_OK : TERN_ETIMEOUT;
 }
 
 tern_status tern_gemm_prefill(const tern_matrix* W, int32_t M, const uint16_t* X_bf16_dev, float* Y_dev,

@@ -40,6 +40,7 @@ __device__ __forceinline__ uint32_t u4get(const uint4& v, int e) {
 __device__ __forceinline__ int fv5_cols(int mode, int M) { return mode == 0 ? 4 * M : M; }
 __device__ __forceinline__ int col_words(int kr) { return kr / 4 + 16; }
 __device__ __forceinline__ int half_ofs(int v) { return 4 * (v ^ ((v >> 3) & 3)); }
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
 
 // ---- pack -------------------------------------------------------------------------------------------
 // One thread per (row, logical 32-trit word): 32 codes in, the three plane words out at the word's
@@ -262,117 +263,168 @@ __global__ void __launch_bounds__(kThreads) k_fv5_gemm(const Fv5Params p) {
 }
 
 // ---- a list of linears at M = 1 in one persistent launch ---------------------------------------------
-// Work units are tiles of 16 rows of one item over the whole of K; CTA c takes a contiguous,
-// cost-balanced range of them. It walks its range one item at a time: the CTA stages the item's
-// activation (all K) as the batched stream's operand words (tern_batch.cu: eight words per 32-trit
-// word, in natural word order here since the planes' word transposition already gives each quad
-// lane its word) together with each 256-weight block's column sums; then its warps take the item's
-// tiles in turn, each streaming its 16 rows with two chunks in flight (a warp's next tile is fetched
-// while it forms this one's outputs). A word's low- and high-magnitude parts take the offset decode
-// of the batched stream (one AND per operand register: field i in place reads 4^i (t + 2)), each
-// into its own four field accumulators; at a block's end the exact sums (the offset removed with
-// the block's column sums) are scaled by s_lo and s_hi into fp64, as in k_fv5_gemm, and each warp
-// writes its rows' outputs itself: with K whole in the warp no other warp's partial sums are
-// needed.
+// Work units are 16-row tiles of one item over the whole of K; the host cuts the list into
+// contiguous ranges of tiles with equal numbers of 512-trit chunks, one per CTA, two CTAs per SM
+// (a range also closes where its items' staged activations would outgrow the shared-memory budget).
+// A CTA stages the activations of all of its range's items at once (all K) as the batched stream's
+// operand words (tern_batch.cu: eight words per 32-trit word, in natural word order here since the
+// planes' word transposition already gives each quad lane its word) together with each 256-weight
+// block's column sums. Its chunks are then cut into eight equal contiguous parts, one per warp, so a
+// tile may be split between two warps (or, for a tile longer than a part, several). The blocks of a
+// tile must still be added in order, so the fp64 partial sums of a tile's first part are handed to
+// the owner of its next part: a warp takes the head of its last tile first (publishing its partial
+// sums in shared memory at once), then its whole tiles, and the tail of its first tile last (taking
+// the partial sums published by the previous part's owner, long since ready). Each wait is bounded.
+// A word's low- and high-magnitude parts take the offset decode of the batched stream (one AND per
+// operand register: field i in place reads 4^i (t + 2)) in turn, each into one set of four field
+// accumulators; at a block's end the exact sums (the offset removed with the block's column sums)
+// are scaled by s_lo and s_hi into fp64, as in k_fv5_gemm, and the owner of a tile's last part
+// writes its rows' outputs.
+constexpr int kWarps = kThreads / 32;
+constexpr long long kHandSpin = 4000000000LL;               // clock64 cycles (~2 s) before a wait gives up
+__device__ int g_fv5_latch = 0;
+
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 2) k_fv5_batch(const __grid_constant__ Fv5BatchParams p) {
-  extern __shared__ __align__(16) uint32_t smem[];         // the current item's activation columns
-  __shared__ float fred[kThreads / 32];
-  __shared__ int expo_s;
+  extern __shared__ __align__(16) uint32_t smem[];         // the range's items' activations, back to back
+  __shared__ double hand[kWarps][4][32];                    // partial sums handed to warp w
+  __shared__ int hflag[kWarps];
+  __shared__ float fredw[kFv5MaxItemsPerCTA][kWarps];       // per item, per warp absmax (bf16 mode)
+  __shared__ int offs[kFv5MaxItemsPerCTA], expo[kFv5MaxItemsPerCTA];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int u0 = p.cta_unit[blockIdx.x], u1 = p.cta_unit[blockIdx.x + 1];
   if (u0 >= u1) return;
   constexpr int NC = MODE == 0 ? 4 : 1;
-  // the tile being fetched: its rows and plane pointers of this lane's rows ra, rb
-  int f_KM = 0, f_nchunks = 0, f_row0 = 0, f_u = -1;           // f_u: the tile fetched, or -1
-  bool f_live = false;
+  const int i0 = p.cta_item[blockIdx.x];
+  int iend = i0 + 1;                                        // items [i0, iend) meet the range
+  while (iend < p.count && p.unit0[iend] < u1) ++iend;
+  auto tiles_of = [&](int j) { return min(u1, p.unit0[j + 1]) - max(u0, p.unit0[j]); };
+  // this warp's chunks [a, b) of the range's Wc
+  int Wc = 0;
+  for (int j = i0; j < iend; ++j) Wc += tiles_of(j) * (p.items[j].K >> 9);
+  const int a = (int)((long long)Wc * warp / kWarps), b = (int)((long long)Wc * (warp + 1) / kWarps);
+  // chunk x of the range -> item, tile, chunk of the tile
+  auto locate = [&](int x, int& item, int& u, int& c) {
+    int j = i0;
+    while (true) {
+      const int nch = p.items[j].K >> 9, cj = tiles_of(j) * nch;
+      if (x < cj || j + 1 >= iend) {
+        item = j;
+        u = max(u0, p.unit0[j]) + x / nch;
+        c = x % nch;
+        return;
+      }
+      x -= cj;
+      ++j;
+    }
+  };
+  int iA = 0, uA = 0, cA = 0, iB = 0, uB = 0, cBe = 0, npieces = 0;
+  if (a < b) {
+    locate(a, iA, uA, cA);
+    locate(b - 1, iB, uB, cBe);
+    ++cBe;
+    npieces = uA == uB ? 1 : uB - uA + 1;
+  }
+  const bool headB = cBe < (p.items[iB].K >> 9);
+  // piece k in the order taken: the head of the last tile (if split), the whole tiles, the first tile
+  auto piece = [&](int k, int& item, int& u, int& ca, int& cb) {
+    if (uA == uB) { item = iA; u = uA; ca = cA; cb = cBe; return; }
+    if (k == uB - uA) { item = iA; u = uA; ca = cA; cb = p.items[iA].K >> 9; return; }
+    if (headB && k == 0) { item = iB; u = uB; ca = 0; cb = cBe; return; }
+    u = headB ? uA + k : uA + 1 + k;
+    int j = iA;
+    while (p.unit0[j + 1] <= u) ++j;
+    item = j;
+    ca = 0;
+    cb = p.items[j].K >> 9;
+  };
+  // the fetch side runs two chunks ahead of the products, across pieces
+  int fk = 0, f_u = 0, f_c = 0, f_cb = 0, f_KM = 0;
   const uint32_t *pa = nullptr, *pb = nullptr;
-  auto set_tile = [&](int item, int u) {
+  auto fetch_setup = [&](int k) {
+    int item;
+    piece(k, item, f_u, f_c, f_cb);
     const Fv5BatchItem& I = p.items[item];
-    f_u = u;
-    f_row0 = (u - p.unit0[item]) * 16;
     f_KM = I.K >> 5;
-    f_nchunks = I.K >> 9;
-    f_live = true;
-    const int ra = min(f_row0 + g, I.N - 1), rb = min(f_row0 + g + 8, I.N - 1);
+    const int row0 = (f_u - p.unit0[item]) * 16;
+    const int ra = min(row0 + g, I.N - 1), rb = min(row0 + g + 8, I.N - 1);
     pa = I.planes + (size_t)ra * (3 * f_KM);
     pb = I.planes + (size_t)rb * (3 * f_KM);
   };
-  auto load_chunk = [&](int c, uint4 (&w)[6]) {
-    const int off = 16 * c + 4 * t;
-    if (f_live && c < f_nchunks) {
+  auto fetch_next = [&](uint4 (&w)[6]) {
+    if (fk < npieces) {
+      const int off = 16 * f_c + 4 * t;
       w[0] = ld_stream(pa + off);
       w[1] = ld_stream(pb + off);
       w[2] = ld_stream(pa + f_KM + off);
       w[3] = ld_stream(pb + f_KM + off);
       w[4] = ld_stream(pa + 2 * f_KM + off);
       w[5] = ld_stream(pb + 2 * f_KM + off);
+      if (++f_c == f_cb && ++fk < npieces) fetch_setup(fk);
     } else {
 #pragma unroll
       for (int i = 0; i < 6; ++i) w[i] = make_uint4(0u, 0u, 0u, 0u);
     }
   };
   uint4 cur[6], nxt[6];
-  int item = p.cta_item[blockIdx.x];
-  // this warp's first tile of the first segment, fetched before the dependency wait
+  if (npieces > 0) fetch_setup(0);
+  fetch_next(cur);                                          // weights: before the dependency wait
+  fetch_next(nxt);
+  pdl_wait();
+
+  // ---- stage the range's activations: operand words and per-block column sums --------------------
+  if (threadIdx.x < kWarps) hflag[threadIdx.x] = 0;
   {
-    const int s1 = min(u1, p.unit0[item + 1]);
-    if (u0 + warp < s1) {
-      set_tile(item, u0 + warp);
-      load_chunk(0, cur);
-      load_chunk(1, nxt);
+    int off = 0;
+    for (int j = i0; j < iend; ++j) {
+      const Fv5BatchItem& I = p.items[j];
+      const int K = I.K, nblk = K >> 8, jj = j - i0;
+      int* bsum = reinterpret_cast<int*>(smem + off + NC * (K / 4 + 4));
+      for (int i = threadIdx.x; i < NC * nblk; i += kThreads) bsum[i] = 0;
+      if (threadIdx.x == 0) offs[jj] = off;
+      if (MODE == 0) {
+        const uint16_t* xs = static_cast<const uint16_t*>(I.x);
+        float amax = 0.0f;
+        for (int k = threadIdx.x * 8; k < K; k += kThreads * 8) {
+          const uint4 v = ld_nc(xs + k);
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            amax = fmaxf(amax, fmaxf(fabsf(bf16_bits_to_float(w[e] & 0xFFFFu)), fabsf(bf16_bits_to_float(w[e] >> 16))));
+        }
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+        if (lane == 0) fredw[jj][warp] = amax;
+      }
+      off += fv5_stage_words(NC, K);
     }
   }
-  pdl_wait();
-  for (int s0 = u0; s0 < u1; ++item) {
-    while (p.unit0[item + 1] <= s0) ++item;                 // the item of this segment
-    const int s1 = min(u1, p.unit0[item + 1]);               // tiles [s0, s1) of this item
-    const Fv5BatchItem& I = p.items[item];
-    const int K = I.K, nblk = K >> 8;
-    // ---- stage the item's activation: operand words and per-block column sums --------------------
-    const int RS = K / 4 + 4;                                // words per column (+4: the quarter-warp's
-                                                             // two columns' 128-bit reads miss each other)
-    int* bsum = reinterpret_cast<int*>(smem + NC * (p.kmax / 4 + 4));   // [NC][K / 256]
-    __syncthreads();                                         // the previous item's columns are read
-    for (int i = threadIdx.x; i < NC * nblk; i += kThreads) bsum[i] = 0;
-    const int per_row = K >> 4;                              // 16-element halves
+  __syncthreads();                                          // absmax partials, zeroed sums, offsets
+  for (int j = i0; j < iend; ++j) {
+    const Fv5BatchItem& I = p.items[j];
+    const int K = I.K, nblk = K >> 8, jj = j - i0, RS = K / 4 + 4;
+    uint32_t* xb = smem + offs[jj];
+    int* bsum = reinterpret_cast<int*>(xb + NC * RS);
     int E = 0;
     if (MODE == 0) {
-      const uint16_t* xs = static_cast<const uint16_t*>(I.x);
-      float amax = 0.0f;
-      for (int k = threadIdx.x * 8; k < K; k += kThreads * 8) {
-        const uint4 v = ld_nc(xs + k);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      float mx = fredw[jj][0];
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          amax = fmaxf(amax, fmaxf(fabsf(bf16_bits_to_float(w[e] & 0xFFFFu)), fabsf(bf16_bits_to_float(w[e] >> 16))));
-      }
-      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-      if (lane == 0) fred[warp] = amax;
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        float mx = fred[0];
-        for (int i = 1; i < kThreads / 32; ++i) mx = fmaxf(mx, fred[i]);
-        expo_s = limb_exponent(mx);
-      }
-      __syncthreads();
-      E = expo_s;
-    } else {
-      __syncthreads();                                       // bsum zeroed
+      for (int i = 1; i < kWarps; ++i) mx = fmaxf(mx, fredw[jj][i]);
+      E = limb_exponent(mx);
+      if (threadIdx.x == 0) expo[jj] = E;
     }
-    for (int v = threadIdx.x; v < per_row; v += kThreads) {
+    for (int v = threadIdx.x; v < (K >> 4); v += kThreads) {  // 16-element halves
       const int w = v >> 1, h = v & 1, blk = v >> 4;
       if (MODE == 1) {
         const uint4 q = ld_nc(static_cast<const int8_t*>(I.x) + 16 * v);
         atomicAdd(&bsum[blk], __dp4a((int)q.x, 0x01010101, 0) + __dp4a((int)q.y, 0x01010101, 0) +
                                   __dp4a((int)q.z, 0x01010101, 0) + __dp4a((int)q.w, 0x01010101, 0));
         const uint4 o = permute_i8_half(q);
-        uint32_t* slot = smem + w * 8;
+        uint32_t* slot = xb + w * 8;
         slot[0 + h] = o.x; slot[2 + h] = o.y; slot[4 + h] = o.z; slot[6 + h] = o.w;
       } else {
-        const uint16_t* xb = static_cast<const uint16_t*>(I.x) + 16 * v;
-        const uint4 a = ld_nc(xb), b = ld_nc(xb + 8);
-        const uint32_t wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        const uint16_t* xe = static_cast<const uint16_t*>(I.x) + 16 * v;
+        const uint4 lo = ld_nc(xe), hi = ld_nc(xe + 8);
+        const uint32_t wv[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
         uint32_t l[4][4];
         limbs_of_bf16<4>(wv, E, l);
 #pragma unroll
@@ -380,117 +432,129 @@ __global__ void __launch_bounds__(kThreads, 2) k_fv5_batch(const __grid_constant
           atomicAdd(&bsum[c * nblk + blk], __dp4a((int)l[c][0], 0x01010101, 0) + __dp4a((int)l[c][1], 0x01010101, 0) +
                                                __dp4a((int)l[c][2], 0x01010101, 0) + __dp4a((int)l[c][3], 0x01010101, 0));
           const uint4 o = permute_i8_half(make_uint4(l[c][0], l[c][1], l[c][2], l[c][3]));
-          uint32_t* slot = smem + c * RS + w * 8;
+          uint32_t* slot = xb + c * RS + w * 8;
           slot[0 + h] = o.x; slot[2 + h] = o.y; slot[4 + h] = o.z; slot[6 + h] = o.w;
         }
       }
     }
-    __syncthreads();
-    // a warp that had no tile in the previous segment has not fetched its first one of this segment
-    if (s0 + warp < s1 && f_u != s0 + warp) {
-      set_tile(item, s0 + warp);
-      load_chunk(0, cur);
-      load_chunk(1, nxt);
+  }
+  __syncthreads();
+
+  // ---- this warp's pieces ---------------------------------------------------------------------------
+  // accumulator register q holds row g + 8 (q >> 1), column 2t + (q & 1)
+  const int colq0 = 2 * t, colq1 = 2 * t + 1;
+  for (int k = 0; k < npieces; ++k) {
+    int item, u, ca, cb;
+    piece(k, item, u, ca, cb);
+    const Fv5BatchItem& I = p.items[item];
+    const int K = I.K, nblk = K >> 8, nch = K >> 9, RS = K / 4 + 4, jj = item - i0;
+    const uint32_t* xb = smem + offs[jj];
+    const int* bsum = reinterpret_cast<const int*>(xb + NC * RS);
+    const int row0 = (u - p.unit0[item]) * 16;
+    const int ra = min(row0 + g, I.N - 1), rb = min(row0 + g + 8, I.N - 1);
+    const float2* sca = reinterpret_cast<const float2*>(I.scales) + (size_t)ra * nblk;
+    const float2* scb = reinterpret_cast<const float2*>(I.scales) + (size_t)rb * nblk;
+    double Y[4] = {0.0, 0.0, 0.0, 0.0};
+    if (ca > 0) {                                           // the tile's earlier blocks: their sums
+      bool ok = true;
+      if (lane == 0) {
+        const long long t0 = clock64();
+        int v = 0, spins = 0;
+        while (true) {
+          asm volatile("ld.acquire.cta.shared.s32 %0, [%1];" : "=r"(v) : "r"(smem_u32(&hflag[warp])) : "memory");
+          if (v) break;
+          if (++spins > 32) __nanosleep(100);
+          if (clock64() - t0 > kHandSpin) { ok = false; break; }
+        }
+        if (!ok) atomicExch(&g_fv5_latch, 5);
+      }
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (ok) {
+        int v;
+        asm volatile("ld.acquire.cta.shared.s32 %0, [%1];" : "=r"(v) : "r"(smem_u32(&hflag[warp])) : "memory");
+#pragma unroll
+        for (int q = 0; q < 4; ++q) Y[q] = hand[warp][q][lane];
+      }
     }
-    // ---- this warp's tiles of the segment: s0 + warp, s0 + warp + 8, ... -----------------------------
-    for (int u = s0 + warp; u < s1; u += kThreads / 32) {
-      const int row0 = f_row0, nchunks = f_nchunks;
-      const int ra = min(row0 + g, I.N - 1), rb = min(row0 + g + 8, I.N - 1);
-      const float2* sca = reinterpret_cast<const float2*>(I.scales) + (size_t)ra * nblk;
-      const float2* scb = reinterpret_cast<const float2*>(I.scales) + (size_t)rb * nblk;
-      double Y[4] = {0.0, 0.0, 0.0, 0.0};
-      // accumulator register q holds row g + 8 (q >> 1), column 2t + (q & 1)
-      const int colq0 = 2 * t, colq1 = 2 * t + 1;
-      for (int c = 0; c < nchunks; ++c) {
+    for (int c = ca; c < cb; ++c) {
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {               // the chunk's two 256-weight blocks
-          const int blk = 2 * c + half;
-          const int cs0 = colq0 < NC ? bsum[colq0 * nblk + blk] : 0;
-          const int cs1 = colq1 < NC ? bsum[colq1 * nblk + blk] : 0;
-          int v[2][4];                                       // [lo, hi] exact block sums
+      for (int half = 0; half < 2; ++half) {                // the chunk's two 256-weight blocks
+        const int blk = 2 * c + half;
+        const int cs0 = colq0 < NC ? bsum[colq0 * nblk + blk] : 0;
+        const int cs1 = colq1 < NC ? bsum[colq1 * nblk + blk] : 0;
+        int vv[2][4];                                       // [lo, hi] exact block sums
 #pragma unroll
-          for (int part = 0; part < 2; ++part) {             // low magnitudes, then high: one set
-            int acc[4][4] = {};                              // of field accumulators live at a time
+        for (int part = 0; part < 2; ++part) {              // low magnitudes, then high: one set
+          int acc[4][4] = {};                               // of field accumulators live at a time
 #pragma unroll
-            for (int ee = 0; ee < 2; ++ee) {
-              const int e = 2 * half + ee;
-              const int w = 16 * c + 4 * e + t;              // logical word of this lane
-              const uint32_t ga = u4get(cur[4], e), gb = u4get(cur[5], e);
-              const uint32_t ka = part ? ga : ~ga, kb = part ? gb : ~gb;
-              uint32_t a0, b0, a1, b1;
-              merge_planes_offset(u4get(cur[0], e) & ka, u4get(cur[2], e) & __funnelshift_l(ka, ka, 1), a0, b0);
-              merge_planes_offset(u4get(cur[1], e) & kb, u4get(cur[3], e) & __funnelshift_l(kb, kb, 1), a1, b1);
-              uint4 x01 = make_uint4(0u, 0u, 0u, 0u), x23 = x01;
-              if (g < NC) {
-                const uint32_t* xo = smem + g * RS + w * 8;
-                x01 = *reinterpret_cast<const uint4*>(xo);
-                x23 = *reinterpret_cast<const uint4*>(xo + 4);
-              }
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {                  // field i in place -> 4^i * (t + 2)
-                const uint32_t msk = 0x03030303u << (2 * i);
-                const uint32_t x0 = i < 2 ? u4get(x01, 2 * i) : u4get(x23, 2 * i - 4);
-                const uint32_t x1 = i < 2 ? u4get(x01, 2 * i + 1) : u4get(x23, 2 * i - 3);
-                mma_u8s8(acc[i], a0 & msk, a1 & msk, b0 & msk, b1 & msk, x0, x1);
-              }
+          for (int ee = 0; ee < 2; ++ee) {
+            const int e = 2 * half + ee;
+            const int w = 16 * c + 4 * e + t;               // logical word of this lane
+            const uint32_t ga = u4get(cur[4], e), gb = u4get(cur[5], e);
+            const uint32_t ka = part ? ga : ~ga, kb = part ? gb : ~gb;
+            uint32_t a0, b0, a1, b1;
+            merge_planes_offset(u4get(cur[0], e) & ka, u4get(cur[2], e) & __funnelshift_l(ka, ka, 1), a0, b0);
+            merge_planes_offset(u4get(cur[1], e) & kb, u4get(cur[3], e) & __funnelshift_l(kb, kb, 1), a1, b1);
+            uint4 x01 = make_uint4(0u, 0u, 0u, 0u), x23 = x01;
+            if (g < NC) {
+              const uint32_t* xo = xb + g * RS + w * 8;
+              x01 = *reinterpret_cast<const uint4*>(xo);
+              x23 = *reinterpret_cast<const uint4*>(xo + 4);
             }
-            // the offset 2 per weight removed with the block's column sums
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              v[part][q] = acc[0][q] + (acc[1][q] >> 2) + (acc[2][q] >> 4) + (acc[3][q] >> 6) - 2 * ((q & 1) ? cs1 : cs0);
+            for (int i = 0; i < 4; ++i) {                   // field i in place -> 4^i * (t + 2)
+              const uint32_t msk = 0x03030303u << (2 * i);
+              const uint32_t x0 = i < 2 ? u4get(x01, 2 * i) : u4get(x23, 2 * i - 4);
+              const uint32_t x1 = i < 2 ? u4get(x01, 2 * i + 1) : u4get(x23, 2 * i - 3);
+              mma_u8s8(acc[i], a0 & msk, a1 & msk, b0 & msk, b1 & msk, x0, x1);
+            }
           }
-          // scaled by the block's s_lo and s_hi, into fp64
-          const float2 sa = __ldg(sca + blk), sb = __ldg(scb + blk);
+          // the offset 2 per weight removed with the block's column sums
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float2 s2 = (q >> 1) ? sb : sa;
-            Y[q] += (double)s2.x * (double)v[0][q] + (double)s2.y * (double)v[1][q];
-          }
+          for (int q = 0; q < 4; ++q)
+            vv[part][q] = acc[0][q] + (acc[1][q] >> 2) + (acc[2][q] >> 4) + (acc[3][q] >> 6) - 2 * ((q & 1) ? cs1 : cs0);
         }
+        // scaled by the block's s_lo and s_hi, into fp64
+        const float2 sa = __ldg(sca + blk), sb = __ldg(scb + blk);
 #pragma unroll
-        for (int i = 0; i < 6; ++i) cur[i] = nxt[i];
-        load_chunk(c + 2, nxt);
+        for (int q = 0; q < 4; ++q) {
+          const float2 s2 = (q >> 1) ? sb : sa;
+          Y[q] += (double)s2.x * (double)vv[0][q] + (double)s2.y * (double)vv[1][q];
+        }
       }
-      // this warp's next tile streams in while this tile's outputs are formed: the next of this
-      // segment, else its first of the next segment (whose item is staged after the barrier)
-      {
-        int nu = u + kThreads / 32, nitem = item;
-        if (nu >= s1 && s1 < u1) {
-          nitem = item + 1;
-          while (p.unit0[nitem + 1] <= s1) ++nitem;
-          nu = s1 + warp;
-          if (nu >= min(u1, p.unit0[nitem + 1])) nu = u1;    // no tile for this warp there
-        }
-        if (nu < u1 && (nu < s1 || nitem != item)) {
-          set_tile(nitem, nu);
-          load_chunk(0, cur);
-          load_chunk(1, nxt);
+#pragma unroll
+      for (int i = 0; i < 6; ++i) cur[i] = nxt[i];
+      fetch_next(nxt);
+    }
+    if (cb < nch) {                                         // hand the sums to the next part's owner
+      const int dst = (int)((8LL * b + 7) / Wc);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) hand[dst][q][lane] = Y[q];
+      __threadfence_block();
+      __syncwarp();
+      if (lane == 0)
+        asm volatile("st.release.cta.shared.s32 [%0], %1;" :: "r"(smem_u32(&hflag[dst])), "r"(1) : "memory");
+      continue;
+    }
+    // ---- outputs: lane t = 0 holds columns 0, 1 of rows g and g + 8, lane t = 1 columns 2, 3 -----
+    double w2[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w2[i] = __shfl_down_sync(0xFFFFFFFFu, Y[i], 1);
+    if (t == 0) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int row = row0 + g + 8 * h;
+        if (row >= I.N) continue;
+        float yv;
+        if (MODE == 1) {
+          yv = (float)((double)I.sx[0] * Y[2 * h]);
         } else {
-          f_live = false;
-          f_u = -1;
+          yv = (float)ldexp(((Y[2 * h] * 256.0 + Y[2 * h + 1]) * 256.0 + w2[2 * h]) * 256.0 + w2[2 * h + 1],
+                            expo[jj] - kLimbFrac);
         }
-      }
-      // ---- outputs: lane t = 0 holds columns 0, 1 of rows g and g + 8, lane t = 1 columns 2, 3 -----
-      double w2[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) w2[i] = __shfl_down_sync(0xFFFFFFFFu, Y[i], 1);
-      if (t == 0) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int row = row0 + g + 8 * h;
-          if (row >= I.N) continue;
-          float yv;
-          if (MODE == 1) {
-            yv = (float)((double)I.sx[0] * Y[2 * h]);
-          } else {
-            yv = (float)ldexp(((Y[2 * h] * 256.0 + Y[2 * h + 1]) * 256.0 + w2[2 * h]) * 256.0 + w2[2 * h + 1],
-                              expo_s - kLimbFrac);
-          }
-          I.y[row] = yv;
-        }
+        I.y[row] = yv;
       }
     }
-    s0 = s1;
   }
 }
 
@@ -542,46 +606,65 @@ cudaError_t launch_fv5_gemm(const Fv5Params& p, cudaStream_t st) {
 }
 
 cudaError_t launch_fv5_batch(Fv5BatchParams& p, cudaStream_t st) {
-  // units and their costs (rows x K), then contiguous cost-balanced ranges, one per CTA
+  // units (16-row tiles) and their costs (512-trit chunks), then contiguous ranges of equal cost,
+  // one per CTA, each closed early where its items' staged activations would outgrow the budget
+  const int nc = p.mode == 0 ? 4 : 1;
   int64_t units = 0, total = 0;
   p.kmax = 0;
   for (int i = 0; i < p.count; ++i) {
     p.unit0[i] = (int32_t)units;
     units += (p.items[i].N + 15) / 16;
-    total += (int64_t)p.items[i].N * p.items[i].K;
+    total += (int64_t)((p.items[i].N + 15) / 16) * (p.items[i].K / 512);
     if (p.items[i].K > p.kmax) p.kmax = p.items[i].K;
+    if (fv5_stage_words(nc, p.items[i].K) > kFv5StageBudgetWords) return cudaErrorInvalidValue;
   }
-  if (units > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  if (units > 0x7FFFFFFF || total > 0x7FFFFFFF) return cudaErrorInvalidValue;
   p.unit0[p.count] = (int32_t)units;
   // two CTAs per SM (16 warps: the decode and MMA chains of one CTA's 8 warps leave the SM idle)
-  long long g2 = 2LL * device_sm_count();
-  if (g2 > kFv5MaxCTAs) g2 = kFv5MaxCTAs;
-  if (g2 > units) g2 = units;
-  const int grid = (int)(g2 < 1 ? 1 : g2);
-  p.grid = grid;
-  {
-    int c = 1, it = 0;
-    int64_t acc = 0;
-    p.cta_unit[0] = 0;
-    for (int64_t u = 0; u < units && c < grid; ++u) {
-      while (it + 1 < p.count && p.unit0[it + 1] <= u) ++it;
-      const int rows = p.items[it].N - (int)(u - p.unit0[it]) * 16;
-      acc += (int64_t)(rows < 16 ? rows : 16) * p.items[it].K;
-      while (c < grid && acc * grid >= total * c) p.cta_unit[c++] = (int32_t)(u + 1);
+  long long G = 2LL * device_sm_count();
+  if (G > units) G = units;
+  if (G < 1) G = 1;
+  int c = 0, it = 0, last = -1, nitems = 0, words = 0, max_words = 0;
+  int64_t acc = 0, q = 1;
+  p.cta_unit[0] = 0;
+  for (int64_t u = 0; u < units; ++u) {
+    while (it + 1 < p.count && p.unit0[it + 1] <= u) ++it;
+    if (it != last) {                                      // the range meets a new item
+      const int need = fv5_stage_words(nc, p.items[it].K);
+      if (nitems > 0 && (words + need > kFv5StageBudgetWords || nitems == kFv5MaxItemsPerCTA)) {
+        if (c + 1 >= kFv5MaxCTAs) return cudaErrorInvalidValue;
+        p.cta_unit[++c] = (int32_t)u;
+        words = 0;
+        nitems = 0;
+      }
+      words += need;
+      ++nitems;
+      last = it;
+      if (words > max_words) max_words = words;
     }
-    for (; c <= grid; ++c) p.cta_unit[c] = (int32_t)units;
-    int i = 0;
-    for (c = 0; c < grid; ++c) {
-      while (i + 1 < p.count && p.unit0[i + 1] <= p.cta_unit[c]) ++i;
-      p.cta_item[c] = (int16_t)i;
+    acc += p.items[it].K / 512;
+    if (q < G && acc * G >= total * q) {                   // a quantile of the cost: close the range
+      while (q < G && acc * G >= total * q) ++q;
+      if (u + 1 < units) {
+        if (c + 1 >= kFv5MaxCTAs) return cudaErrorInvalidValue;
+        p.cta_unit[++c] = (int32_t)(u + 1);
+        words = 0;
+        nitems = 0;
+        last = -1;
+      }
     }
   }
-  const int nc = p.mode == 0 ? 4 : 1;
-  const size_t smem = (size_t)nc * (p.kmax / 4 + 4) * 4 + (size_t)nc * (p.kmax / 256) * 4;
+  const int grid = c + 1;
+  p.cta_unit[grid] = (int32_t)units;
+  p.grid = grid;
+  for (int k = 0, i = 0; k < grid; ++k) {
+    while (i + 1 < p.count && p.unit0[i + 1] <= p.cta_unit[k]) ++i;
+    p.cta_item[k] = (int16_t)i;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = (size_t)max_words * 4;
   cfg.stream = st;
   if (p.mode == 0) {
     static std::atomic<unsigned long long> raised{0};
@@ -593,6 +676,13 @@ cudaError_t launch_fv5_batch(Fv5BatchParams& p, cudaStream_t st) {
   cudaError_t e = allow_max_dynamic_smem(k_fv5_batch<1>, raised1);
   if (e != cudaSuccess) return e;
   return cudaLaunchKernelEx(&cfg, k_fv5_batch<1>, p);
+}
+
+cudaError_t read_and_clear_fv5_latch(int* out) {
+  cudaError_t e = cudaMemcpyFromSymbol(out, g_fv5_latch, sizeof(int));
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_fv5_latch, &zero, sizeof(int));
 }
 
 cudaError_t launch_fv5_pack(const int8_t* codes, int32_t N, int32_t K, uint32_t* planes, int32_t* flag,

@@ -327,7 +327,14 @@ struct Fv5BatchItem {
   float* y;                   // [N]
   int32_t N, K;
 };
-constexpr int kFv5MaxCTAs = 2 * kMaxGridCTAs;   // two CTAs per SM
+// Two CTAs per SM, plus one extra range per item at most (a range closes early where its items'
+// staged activations would outgrow the budget below).
+constexpr int kFv5MaxCTAs = 2 * kMaxGridCTAs + kBatchMaxItems;
+constexpr int kFv5MaxItemsPerCTA = 32;
+constexpr int kFv5StageBudgetWords = 24576;   // 96 KB of staged activations per CTA
+// Words one item's staged activation takes: nc operand columns of K / 4 + 4 words, then nc column
+// sums per 256-weight block; rounded up to four words (16-byte aligned columns).
+__host__ __device__ inline int fv5_stage_words(int nc, int K) { return (nc * (K / 4 + 4) + nc * (K / 256) + 3) & ~3; }
 struct Fv5BatchParams {
   Fv5BatchItem items[kBatchMaxItems];
   int32_t unit0[kBatchMaxItems + 1];   // first unit of each item; unit0[count] = all units
@@ -336,6 +343,7 @@ struct Fv5BatchParams {
   int32_t count, mode, grid, kmax;
 };
 cudaError_t launch_fv5_batch(Fv5BatchParams& p, cudaStream_t st);
+cudaError_t read_and_clear_fv5_latch(int* out);
 size_t fv5_smem_bytes(int mode, int M, int kr);
 int fv5_rows_per_cta();
 cudaError_t launch_fv5_gemm(const Fv5Params& p, cudaStream_t st);

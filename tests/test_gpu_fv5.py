@@ -170,16 +170,35 @@ def test_fv5_invalid_codes_and_arguments():
 
 
 BATCH_SHAPES = [(37, 512), (300, 1024), (1024, 4096), (200, 12288), (129, 4096), (4096, 4096)]
+_rs = np.random.default_rng(7)
+BATCH_SETS = {
+    # ragged shapes, K up to 12288: tiles split between two warps of a CTA
+    "ragged": BATCH_SHAPES,
+    # one 16-row tile over K = 12288: its 24 chunks cut among all eight warps of one CTA, each part
+    # taking the partial sums of the one before
+    "one_tile": [(16, 12288)],
+    # many small items of mixed K
+    "many_items": [(int(_rs.integers(1, 49)), 512 * int(_rs.integers(1, 9))) for _ in range(120)],
+    # one long item, then 150 one-tile items: a range's share of the chunks holds more than the
+    # 32 items a CTA stages, so ranges close at that limit
+    "item_limit": [(200000, 512)] + [(1 + i % 16, 512) for i in range(150)],
+    # K = 12288 items of a few tiles: in bf16 mode a second one would outgrow a CTA's staging
+    # budget, so ranges close at each item
+    "staging_budget": [(40 + 8 * i, 12288) for i in range(12)],
+}
 
 
 @pytest.mark.parametrize("mode", ["bf16", "int8"])
-def test_gemv_batch_matches_oracle(mode):
-    """tern_fv5_gemv_batch: a list of ragged shapes (N not a multiple of 128, K up to 12288) in one
-    launch against the oracle: int8 mode bit for bit (the block sums are added in block order, as the
-    oracle adds them), bf16 mode within the per-output bound; twice on the same outputs."""
+@pytest.mark.parametrize("shapes", sorted(BATCH_SETS))
+def test_gemv_batch_matches_oracle(mode, shapes):
+    """tern_fv5_gemv_batch: a list of shapes in one launch against the oracle: int8 mode bit for bit
+    (the block sums are added in block order, as the oracle adds them, also where a tile's blocks
+    are split among warps), bf16 mode within the per-output bound; twice on the same outputs, with
+    no device-side wait giving up."""
     act = tg.TERN_ACT_BF16 if mode == "bf16" else tg.TERN_ACT_INT8
+    shape_list = BATCH_SETS[shapes]
     entries, refs, bounds = [], [], []
-    for i, (N, K) in enumerate(BATCH_SHAPES):
+    for i, (N, K) in enumerate(shape_list):
         W, c, s = _matrix(41 + i, N, K)
         X = synth.activations(42 + i, 1, 1, K)
         y = torch.full((N,), float("nan"), dtype=torch.float32, device="cuda")
@@ -199,13 +218,14 @@ def test_gemv_batch_matches_oracle(mode):
             y.fill_(float("nan"))
         tg.tern_fv5_gemv_batch(entries, act)
         torch.cuda.synchronize()
+        assert tg.tern_device_status() == tg.TERN_OK
         for i, (W, _, _, y) in enumerate(entries):
             got = host(y)
             if mode == "int8":
-                assert (got.view(np.uint32) == refs[i].astype(np.float32).view(np.uint32)).all(), BATCH_SHAPES[i]
+                assert (got.view(np.uint32) == refs[i].astype(np.float32).view(np.uint32)).all(), shape_list[i]
             else:
                 err = got.astype(np.float64) - refs[i]
-                assert (np.abs(err) <= bounds[i]).all(), BATCH_SHAPES[i]
+                assert (np.abs(err) <= bounds[i]).all(), shape_list[i]
                 assert np.linalg.norm(err) / np.linalg.norm(refs[i]) <= REL_L2
 
 
