@@ -367,6 +367,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_fv5_batch(const __grid_constant
     }
   };
   uint4 cur[6], nxt[6];
+  int par = 0;                                              // the buffer of the next chunk to take
   if (npieces > 0) fetch_setup(0);
   fetch_next(cur);                                          // weights: before the dependency wait
   fetch_next(nxt);
@@ -476,55 +477,75 @@ __global__ void __launch_bounds__(kThreads, 2) k_fv5_batch(const __grid_constant
         for (int q = 0; q < 4; ++q) Y[q] = hand[warp][q][lane];
       }
     }
-    for (int c = ca; c < cb; ++c) {
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {                // the chunk's two 256-weight blocks
-        const int blk = 2 * c + half;
-        const int cs0 = colq0 < NC ? bsum[colq0 * nblk + blk] : 0;
-        const int cs1 = colq1 < NC ? bsum[colq1 * nblk + blk] : 0;
-        int vv[2][4];                                       // [lo, hi] exact block sums
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {              // low magnitudes, then high: one set
-          int acc[4][4] = {};                               // of field accumulators live at a time
-#pragma unroll
-          for (int ee = 0; ee < 2; ++ee) {
-            const int e = 2 * half + ee;
-            const int w = 16 * c + 4 * e + t;               // logical word of this lane
-            const uint32_t ga = u4get(cur[4], e), gb = u4get(cur[5], e);
-            const uint32_t ka = part ? ga : ~ga, kb = part ? gb : ~gb;
-            uint32_t a0, b0, a1, b1;
-            merge_planes_offset(u4get(cur[0], e) & ka, u4get(cur[2], e) & __funnelshift_l(ka, ka, 1), a0, b0);
-            merge_planes_offset(u4get(cur[1], e) & kb, u4get(cur[3], e) & __funnelshift_l(kb, kb, 1), a1, b1);
-            uint4 x01 = make_uint4(0u, 0u, 0u, 0u), x23 = x01;
-            if (g < NC) {
-              const uint32_t* xo = xb + g * RS + w * 8;
-              x01 = *reinterpret_cast<const uint4*>(xo);
-              x23 = *reinterpret_cast<const uint4*>(xo + 4);
+    // the chunk at step s of this warp sits in buffer s & 1 and is refilled, once used, with the
+    // chunk two steps on: the two buffers alternate without register copies
+    auto chunk = [&](const uint4 (&cw)[6], int c) {
+  #pragma unroll
+        for (int half = 0; half < 2; ++half) {                // the chunk's two 256-weight blocks
+          const int blk = 2 * c + half;
+          const int cs0 = colq0 < NC ? bsum[colq0 * nblk + blk] : 0;
+          const int cs1 = colq1 < NC ? bsum[colq1 * nblk + blk] : 0;
+          int R[2][4];                                        // offset sums: all nonzero weights, high magnitudes
+  #pragma unroll
+          for (int part = 0; part < 2; ++part) {              // all nonzero weights, then the high magnitudes:
+            int acc[4][4] = {};                               // one set of field accumulators live at a time
+  #pragma unroll
+            for (int ee = 0; ee < 2; ++ee) {
+              const int e = 2 * half + ee;
+              const int w = 16 * c + 4 * e + t;               // logical word of this lane
+              uint32_t ma = u4get(cw[0], e), mb = u4get(cw[1], e), sa = u4get(cw[2], e), sb = u4get(cw[3], e);
+              if (part) {
+                const uint32_t ga = u4get(cw[4], e), gb = u4get(cw[5], e);
+                ma &= ga;
+                mb &= gb;
+                sa &= __funnelshift_l(ga, ga, 1);
+                sb &= __funnelshift_l(gb, gb, 1);
+              }
+              uint32_t a0, b0, a1, b1;
+              merge_planes_offset(ma, sa, a0, b0);
+              merge_planes_offset(mb, sb, a1, b1);
+              uint4 x01 = make_uint4(0u, 0u, 0u, 0u), x23 = x01;
+              if (g < NC) {
+                const uint32_t* xo = xb + g * RS + w * 8;
+                x01 = *reinterpret_cast<const uint4*>(xo);
+                x23 = *reinterpret_cast<const uint4*>(xo + 4);
+              }
+  #pragma unroll
+              for (int i = 0; i < 4; ++i) {                   // field i in place -> 4^i * (t + 2)
+                const uint32_t msk = 0x03030303u << (2 * i);
+                const uint32_t x0 = i < 2 ? u4get(x01, 2 * i) : u4get(x23, 2 * i - 4);
+                const uint32_t x1 = i < 2 ? u4get(x01, 2 * i + 1) : u4get(x23, 2 * i - 3);
+                mma_u8s8(acc[i], a0 & msk, a1 & msk, b0 & msk, b1 & msk, x0, x1);
+              }
             }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {                   // field i in place -> 4^i * (t + 2)
-              const uint32_t msk = 0x03030303u << (2 * i);
-              const uint32_t x0 = i < 2 ? u4get(x01, 2 * i) : u4get(x23, 2 * i - 4);
-              const uint32_t x1 = i < 2 ? u4get(x01, 2 * i + 1) : u4get(x23, 2 * i - 3);
-              mma_u8s8(acc[i], a0 & msk, a1 & msk, b0 & msk, b1 & msk, x0, x1);
-            }
+  #pragma unroll
+            for (int q = 0; q < 4; ++q) R[part][q] = acc[0][q] + (acc[1][q] >> 2) + (acc[2][q] >> 4) + (acc[3][q] >> 6);
           }
-          // the offset 2 per weight removed with the block's column sums
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            vv[part][q] = acc[0][q] + (acc[1][q] >> 2) + (acc[2][q] >> 4) + (acc[3][q] >> 6) - 2 * ((q & 1) ? cs1 : cs0);
+          // low magnitudes = all - high (the offsets cancel); the high part's offset 2 per weight
+          // removed with the block's column sums
+          int vv[2][4];
+  #pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            vv[0][q] = R[0][q] - R[1][q];
+            vv[1][q] = R[1][q] - 2 * ((q & 1) ? cs1 : cs0);
+          }
+          // scaled by the block's s_lo and s_hi, into fp64
+          const float2 sa = __ldg(sca + blk), sb = __ldg(scb + blk);
+  #pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 s2 = (q >> 1) ? sb : sa;
+            Y[q] += (double)s2.x * (double)vv[0][q] + (double)s2.y * (double)vv[1][q];
+          }
         }
-        // scaled by the block's s_lo and s_hi, into fp64
-        const float2 sa = __ldg(sca + blk), sb = __ldg(scb + blk);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 s2 = (q >> 1) ? sb : sa;
-          Y[q] += (double)s2.x * (double)vv[0][q] + (double)s2.y * (double)vv[1][q];
-        }
+    };
+    for (int c = ca; c < cb; ++c, par ^= 1) {
+      if (par == 0) {
+        chunk(cur, c);
+        fetch_next(cur);
+      } else {
+        chunk(nxt, c);
+        fetch_next(nxt);
       }
-#pragma unroll
-      for (int i = 0; i < 6; ++i) cur[i] = nxt[i];
-      fetch_next(nxt);
     }
     if (cb < nch) {                                         // hand the sums to the next part's owner
       const int dst = (int)((8LL * b + 7) / Wc);
