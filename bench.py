@@ -965,7 +965,7 @@ def small_m_sweep(stack, hbm_peak, Ms=(1, 2, 3, 4, 5, 7, 8, 12, 16)):
         ms = timed_replays([(g, 4)]) / 20
         nb = sm.stack_bytes + sm.head_bytes
         out[str(M)] = {"pass_us": ms * 1000.0, "frac": gbs_of(nb, ms) / hbm_peak, "tokens_per_s": M * 1000.0 / ms,
-                       "gbs": gbs_of(nb, ms), "launches_per_pass": 3, "kernel": "tcgen05" if M >= 5 else "mma.sync"}
+                       "gbs": gbs_of(nb, ms), "launches_per_pass": 3, "kernel": "tcgen05" if M >= 9 else "mma.sync"}
         del g
     int8 = {}
     for M in (5, 8, 16):
@@ -1086,7 +1086,7 @@ class StackView:
     def launch_stack(self, mode="bf16", pdl=False, tc=False):
         """All 144 fused linears as one batched small-M launch pair (each reads its X [M][K]; int8
         mode: q [M][K] and s_x [M], quantised once); tc: the tcgen05 kernels where the mma.sync
-        ones are the default (every list but bf16 of 5..16 rows)."""
+        ones are the default (every list but bf16 of 9..16 rows)."""
         import torch
         import bit_gemv_tern_b200 as tg
         key = "_batch_" + mode

@@ -320,13 +320,13 @@ namespace {
 
 // Validates a list (and its prologues, if any) and plans both launches. With check_ptrs false
 // only the shapes and modes are checked (the workspace query).
-// Which small-M kernels run a list: the tensor-core (tcgen05) ones for bf16 lists of 5..16 rows
+// Which small-M kernels run a list: the tensor-core (tcgen05) ones for bf16 lists of 9..16 rows
 // (the only kernels there) and wherever the caller asks for them (M >= 2); the mma.sync ones for
 // everything else (measured faster wherever both exist).
 bool use_tc(int32_t M, tern_act act, uint32_t flags) {
   if (M < 2) return false;
   if (flags & TERN_FLAG_TCGEN05) return true;
-  return act == TERN_ACT_BF16 && M >= 5;
+  return act == TERN_ACT_BF16 && M >= 9;
 }
 
 tern_status fill_batch(const tern_gemv_item* items, const tern_prologue* pro, int32_t count, int32_t M, tern_act act,
@@ -421,7 +421,7 @@ size_t tern_gemm_batch_workspace_bytes(const tern_gemv_item* items, int32_t coun
   tern::PrepParams* pp = new (std::nothrow) tern::PrepParams();
   // enough for either kernel family the launch flags can choose
   size_t smem = 0, ws = 0, ws_tc = 0;
-  const bool legacy = act != TERN_ACT_BF16 || M <= 4;
+  const bool legacy = act != TERN_ACT_BF16 || M <= 8;
   tern_status st = (bp && pp) ? TERN_OK : TERN_EINVAL;
   if (st == TERN_OK && legacy) st = fill_batch(items, nullptr, count, M, act, false, false, *bp, *pp, smem, ws);
   if (st == TERN_OK && M >= 2) {

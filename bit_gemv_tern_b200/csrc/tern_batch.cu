@@ -22,7 +22,7 @@
 //      consumer warps walk the stages in order; warp w owns kTPW tiles of 16 rows of the block,
 //      decodes them (one AND per operand register, see tern_device.cuh) into mma.sync u8 x s8
 //      products, and keeps the sums in registers across all parts of the block, so a tile's
-//      outputs are written once, at its end. (bf16 lists of 5..16 rows run on the tensor-core
+//      outputs are written once, at its end. (bf16 lists of 9..16 rows run on the tensor-core
 //      kernels of tern_tc.cu instead.)
 // All sums are exact integers; int8 mode ends with y = ((float)acc * s_x) * scale (two fp32
 // round-to-nearest multiplies), bf16 mode with one fp64 -> fp32 rounding. Every mbarrier wait is
@@ -715,9 +715,9 @@ void batch_shape(int mode, int M, int& mp, int& tpw, int& cw) {
     cw = 11;
     return;
   }
-  mp = M <= 8 ? 8 : 16;                         // int8: one or two groups (bf16 lists of 5..16 rows
-  tpw = 2;                                      // run on the tensor-core kernels, tern_tc.cu)
-  cw = 11;
+  mp = M <= 8 ? 8 : 16;                         // int8: one or two groups; bf16 (5..8 rows): four
+  tpw = mode == 0 ? 1 : 2;                      // groups, one per limb, so one tile per warp (bf16
+  cw = 11;                                      // lists of 9..16 rows run on tern_tc.cu's kernels)
 }
 
 template <int MODE, int MP, int TPW, int CW>
@@ -742,7 +742,7 @@ bool plan_batch(BatchParams& p, const uint32_t* const* planes, size_t& smem, siz
     cw = tc_consumer_warps();
     tpw = tc_stage_rows() / box_rows(cw);
   } else {
-    if (p.mode == 0 && p.M > 4) return false;           // bf16 lists of 5..16 rows: tensor cores only
+    if (p.mode == 0 && p.M > 8) return false;           // bf16 lists of 9..16 rows: tensor cores only
     batch_shape(p.mode, p.M, mp, tpw, cw);
   }
   p.mp = mp;
@@ -953,6 +953,7 @@ cudaError_t launch_batch(const BatchParams& p, const PrepParams& q, size_t smem,
     if (p.mp == 1) return launch_stream_kernel<0, 1, 2, 12>(cfg, p);
     if (p.mp == 2) return launch_stream_kernel<0, 2, 2, 12>(cfg, p);
     if (p.mp == 4) return launch_stream_kernel<0, 4, 2, 11>(cfg, p);
+    if (p.mp == 8) return launch_stream_kernel<0, 8, 1, 11>(cfg, p);
     return cudaErrorInvalidValue;
   }
   if (p.mp == 1) return launch_stream_kernel<1, 1, 2, 12>(cfg, p);

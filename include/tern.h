@@ -108,7 +108,7 @@ typedef enum { TERN_SRC_INT8_TRITS = 0, TERN_SRC_BASE3 = 1 } tern_src;
  *   buffers are not written by work still in flight on the stream (true in a decode loop). */
 #define TERN_FLAG_PDL 1u
 /* TERN_FLAG_TCGEN05 (tern_gemm_batch / tern_gemm_batch_pro only, M >= 2): run the list on the
- *   tensor-core (tcgen05) small-M kernels, which otherwise take only bf16 lists of 5..16 rows (the
+ *   tensor-core (tcgen05) small-M kernels, which otherwise take only bf16 lists of 9..16 rows (the
  *   warp-level mma.sync kernels, bit-identical, run everything else and are faster wherever both
  *   exist). For comparisons. */
 #define TERN_FLAG_TCGEN05 2u
@@ -274,7 +274,7 @@ size_t tern_gemm_batch_workspace_bytes(const tern_gemv_item* items, int32_t coun
  * with each item's x_dev = X: bf16[M][K] or int8[M][K] row-major, x_scale_dev = float[M] (int8
  * mode), y_dev = Y: float[M][N]. Each decoded weight word feeds all M rows; the weights stream
  * once. Arithmetic, determinism, aliasing rule, workspace and flags as for tern_gemv_batch (whose
- * call equals this one with M = 1), plus TERN_FLAG_TCGEN05. bf16 lists of 5..16 rows run on the
+ * call equals this one with M = 1), plus TERN_FLAG_TCGEN05. bf16 lists of 9..16 rows run on the
  * 5th-generation tensor cores (tcgen05: the decoded weights are the MMA's A operand in tensor
  * memory, the activation columns (four limbs per row) its B operand in shared memory); every other
  * list on warp-level mma.sync. Results are bit-identical wherever both exist. */

@@ -161,22 +161,23 @@ def test_gemm_batch_small_m_matches_oracle(mode, M):
             assert (yy == y_ref).all(), (N, K, M)
 
 
-@pytest.mark.parametrize("mode,M", [("bf16", 2), ("bf16", 3), ("bf16", 4)] + [("int8", M) for M in (2, 5, 7, 8, 9, 12, 16)])
+@pytest.mark.parametrize("mode,M", [("bf16", M) for M in (2, 3, 4, 5, 7, 8)] + [("int8", M) for M in (2, 5, 7, 8, 9, 12, 16)])
 def test_gemm_batch_tensor_core_equals_mma_sync(mode, M):
     """The tcgen05 kernels (TERN_FLAG_TCGEN05) and the mma.sync kernels (the default at these sizes)
     give the same bits for every output: every sum is an exact integer and the final roundings are
     the same. Ragged N (37, 200, 1000 rows: partial row blocks and boxes), K = 128 and 640 (partial
-    512-trit parts), and lists whose row blocks are split between CTAs; twice in a row (split-block
-    scratch left clean) and with PDL."""
+    512-trit parts), and lists whose row blocks are split between CTAs. The tcgen05 result is the
+    reference; the mma.sync kernels run four times against it (split-block scratch left clean
+    between runs), the last two with PDL, then tcgen05 once more."""
     act = tg.TERN_ACT_BF16 if mode == "bf16" else tg.TERN_ACT_INT8
     shapes = SHAPES_M + [(1000, 128), (6144, 4096)]
     items, _ = _build_m(95 + M, shapes, M, act)
     batch = tg.GemvBatch(items, act, M=M)
-    batch()
+    batch(flags=tg.TERN_FLAG_TCGEN05)
     torch.cuda.synchronize()
     assert tg.tern_device_status() == tg.TERN_OK
     want = [host(Y).copy() for (_, _, _, Y) in items]
-    for flags in (tg.TERN_FLAG_TCGEN05, tg.TERN_FLAG_TCGEN05, tg.TERN_FLAG_TCGEN05 | tg.TERN_FLAG_PDL):
+    for flags in (0, 0, tg.TERN_FLAG_PDL, tg.TERN_FLAG_PDL, tg.TERN_FLAG_TCGEN05 | tg.TERN_FLAG_PDL):
         for (_, _, _, Y) in items:
             Y.fill_(float("nan"))
         batch(flags=flags)
@@ -197,11 +198,13 @@ def _on_grid(X: np.ndarray) -> np.ndarray:
     return X
 
 
+@pytest.mark.parametrize("flags", [0, 2])
 @pytest.mark.parametrize("M", [5, 8, 16])
-def test_gemm_batch_bf16_tensor_core_exact(M):
-    """bf16 lists of 5..16 rows run on tcgen05 only. On activations with no element below the limb
-    grid every output equals the oracle's bit for bit (exact integer sums, the same final rounding),
-    twice in a row, on ragged and split shapes."""
+def test_gemm_batch_bf16_tensor_core_exact(M, flags):
+    """bf16 lists of 5..16 rows, on the default kernels (mma.sync up to 8 rows, tcgen05 above) and on
+    tcgen05 (flags = TERN_FLAG_TCGEN05). On activations with no element below the limb grid every
+    output equals the oracle's bit for bit (exact integer sums, the same final rounding), twice in a
+    row, on ragged and split shapes."""
     shapes = [(200, 640), (1000, 128), (4096, 12288), (24576, 4096), (6144, 4096)]
     items, refs = [], []
     for i, (N, K) in enumerate(shapes):
@@ -211,8 +214,11 @@ def test_gemm_batch_bf16_tensor_core_exact(M):
         items.append((W, dev(X.view(np.int16)), None, Y))
         refs.append((s, X, i))
     batch = tg.GemvBatch(items, tg.TERN_ACT_BF16, M=M)
+    assert flags in (0, tg.TERN_FLAG_TCGEN05)
     for _ in range(2):
-        batch()
+        for (_, _, _, Y) in items:
+            Y.fill_(float("nan"))
+        batch(flags=flags)
         torch.cuda.synchronize()
         assert tg.tern_device_status() == tg.TERN_OK
         for (W, _, _, Y), (s, X, i) in zip(items, refs):
@@ -222,7 +228,6 @@ def test_gemm_batch_bf16_tensor_core_exact(M):
             want = oracle.gemm_bf16(oracle.pack(tr), s[rows], K, X)
             got = host(Y).reshape(M, N)[:, rows]
             assert (got.astype(np.float32).view(np.uint32) == np.asarray(want, np.float32).view(np.uint32)).all(), (M, N, K)
-    batch(flags=tg.TERN_FLAG_TCGEN05)                           # the same kernels: accepted
 
 
 def test_gemm_batch_int8_equals_small_m_entry():
