@@ -289,9 +289,9 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
   constexpr int kBoxRows = box_rows(CW);
   constexpr int kBoxBytes = box_bytes(CW);
   extern __shared__ __align__(1024) uint8_t smem[];
-  // PACK: bf16 mode with 2 or 4 token slots, whose 3 * MP limb columns share one or two MMA
-  // groups (a lane then holds limbs of several tokens; the epilogue gathers them by shuffles)
-  constexpr bool PACK = MP == 2 || MP == 4;
+  // PACK: bf16 mode with 2, 4 or 6 token slots, whose 4 * MP limb columns share one, two or three
+  // MMA groups (a lane then holds limbs of several tokens; the epilogue gathers them by shuffles)
+  constexpr bool PACK = MP == 2 || MP == 4 || MP == 6;
   static_assert(!PACK || MODE == 0, "packed token slots are a bf16-mode shape");
   constexpr int NCOL = seg_cols(MODE, MP);
   constexpr int G = MP == 1 ? 1 : (NCOL + 7) / 8;           // MMA column groups
@@ -394,7 +394,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
   // operand column of group j this lane feeds: M = 1: the lane's limb (rows g >= nc repeat column 0)
   // columns past NCOL (M = 1, PACK) repeat a real column; their sums are never read
   const int col0 = (MP == 1 || PACK) ? (g < NCOL ? g : 0) : g;
-  const int col1 = 8 + g < NCOL ? 8 + g : 8;                // PACK, MP = 4: group 1
+  const int col1 = 8 + g < NCOL ? 8 + g : 8;                // PACK, MP >= 4: group 1
   // lanes whose column of group 0 / group 1 exists (M = 1, PACK); the others feed zeros, so the
   // tensor cores multiply no real data into the accumulators that are never read
   const bool live0 = (MP == 1 || PACK) ? g < NCOL : true;
@@ -527,11 +527,14 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
           tot[0][3][0] = (int)m4.w;
           if (MODE == 0) Etok[0][0] = lds32(st + mofs + 4u * NCOL);
         } else if (PACK) {
-          // lane t reads token t: its column sums and E
-          const int m = t < MP ? t : 0;
+          // lane t reads tokens t and (MP = 6) t + 4: their column sums and E
 #pragma unroll
-          for (int l = 0; l < kLimbs; ++l) tot[0][l][0] = lds32(st + mofs + 4u * (uint32_t)(l * MP + m));
-          Etok[0][0] = lds32(st + mofs + 4u * (uint32_t)(NCOL + m));
+          for (int b = 0; b < (MP > 4 ? 2 : 1); ++b) {
+            const int m = t + 4 * b < MP ? t + 4 * b : 0;
+#pragma unroll
+            for (int l = 0; l < kLimbs; ++l) tot[0][l][b] = lds32(st + mofs + 4u * (uint32_t)(l * MP + m));
+            Etok[0][b] = lds32(st + mofs + 4u * (uint32_t)(NCOL + m));
+          }
         } else {
 #pragma unroll
           for (int jj = 0; jj < JJ; ++jj)
@@ -635,7 +638,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
         }
       } else if (PACK) {
         // limb l of token m sits in column c = l * MP + m: group c / 8, held by quad lane
-        // (c % 8) / 2 as half c % 2 of its row pair; lane t = m gathers its token's limbs
+        // (c % 8) / 2 as half c % 2 of its row pair; lane t = m % 4 gathers its token's limbs
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int row = r0 + 8 * h;
@@ -646,12 +649,12 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) k_batch_stream(const __grid_
             for (int l = 0; l < kLimbs; ++l) {
               const int c = l * MP + m;
               L[l] = __shfl_sync(0xFFFFFFFFu, V[a][c >> 3][2 * h + (c & 1)], (lane & ~3) | ((c & 7) >> 1)) -
-                     2LL * tot[0][l][0];
+                     2LL * tot[0][l][m >> 2];
             }
-            if (t == m && m < M && row < B.N) {
+            if (t == (m & 3) && m < M && row < B.N) {
               const long long D = limb_combine(L[0], L[1], L[2], L[3]);
               B.y[(size_t)m * B.N + row] =
-                  (float)((double)D * exp2_i(Etok[0][0] - kLimbFrac) * (double)f16_bits_to_float(sc_bits[a][h]));
+                  (float)((double)D * exp2_i(Etok[0][m >> 2] - kLimbFrac) * (double)f16_bits_to_float(sc_bits[a][h]));
             }
           }
         }
@@ -712,6 +715,12 @@ void batch_shape(int mode, int M, int& mp, int& tpw, int& cw) {
   if (mode == 0 && M <= 4) {                    // 4 x 4 limbs in two groups
     mp = 4;
     tpw = 2;
+    cw = 11;
+    return;
+  }
+  if (mode == 0 && M <= 6) {                    // 4 x 6 limbs in three groups
+    mp = 6;
+    tpw = 1;
     cw = 11;
     return;
   }
@@ -953,6 +962,7 @@ cudaError_t launch_batch(const BatchParams& p, const PrepParams& q, size_t smem,
     if (p.mp == 1) return launch_stream_kernel<0, 1, 2, 12>(cfg, p);
     if (p.mp == 2) return launch_stream_kernel<0, 2, 2, 12>(cfg, p);
     if (p.mp == 4) return launch_stream_kernel<0, 4, 2, 11>(cfg, p);
+    if (p.mp == 6) return launch_stream_kernel<0, 6, 1, 11>(cfg, p);
     if (p.mp == 8) return launch_stream_kernel<0, 8, 1, 11>(cfg, p);
     return cudaErrorInvalidValue;
   }

@@ -138,7 +138,7 @@ def _build_m(seed, shapes, M, act):
 SHAPES_M = [(37, 384), (200, 640), (3072, 1024), (1024, 3072), (4096, 12288), (24576, 4096)]
 
 
-@pytest.mark.parametrize("M", [2, 3, 4, 5, 7, 8, 9, 16])
+@pytest.mark.parametrize("M", [2, 3, 4, 5, 6, 7, 8, 9, 16])
 @pytest.mark.parametrize("mode", ["bf16", "int8"])
 def test_gemm_batch_small_m_matches_oracle(mode, M):
     """Every token row of every item: int8 bit-exact, bf16 within the tolerance (sampled rows of
@@ -161,7 +161,7 @@ def test_gemm_batch_small_m_matches_oracle(mode, M):
             assert (yy == y_ref).all(), (N, K, M)
 
 
-@pytest.mark.parametrize("mode,M", [("bf16", M) for M in (2, 3, 4, 5, 7, 8)] + [("int8", M) for M in (2, 5, 7, 8, 9, 12, 16)])
+@pytest.mark.parametrize("mode,M", [("bf16", M) for M in (2, 3, 4, 5, 6, 7, 8)] + [("int8", M) for M in (2, 5, 7, 8, 9, 12, 16)])
 def test_gemm_batch_tensor_core_equals_mma_sync(mode, M):
     """The tcgen05 kernels (TERN_FLAG_TCGEN05) and the mma.sync kernels (the default at these sizes)
     give the same bits for every output: every sum is an exact integer and the final roundings are
@@ -199,7 +199,7 @@ def _on_grid(X: np.ndarray) -> np.ndarray:
 
 
 @pytest.mark.parametrize("flags", [0, 2])
-@pytest.mark.parametrize("M", [5, 8, 16])
+@pytest.mark.parametrize("M", [5, 6, 8, 16])
 def test_gemm_batch_bf16_tensor_core_exact(M, flags):
     """bf16 lists of 5..16 rows, on the default kernels (mma.sync up to 8 rows, tcgen05 above) and on
     tcgen05 (flags = TERN_FLAG_TCGEN05). On activations with no element below the limb grid every
