@@ -495,9 +495,13 @@ tern_status tern_fv5_gemm(const tern_fv5_matrix* W, int32_t M, tern_act act, con
 /* A list of five-valued linears at M = 1 in one persistent launch (the batched counterpart of
  * tern_fv5_gemm for a decode step: no launch per linear). Item i: y_i[n] = sum_k w_i[n][k] x_i[k],
  * x_i bf16 [K] or int8 [K] with x_scale_i [1] (int8 mode), y_i fp32 [N]; the same products and
- * rounding as tern_fv5_gemm at M = 1, the block sums added in block order. 1 <= count <= 160;
- * W, x (16-byte aligned), x_scale (int8 mode, 4-byte aligned) and y (4-byte aligned) device
- * pointers, caller-owned; no workspace. Argument errors return before anything is enqueued. */
+ * rounding as tern_fv5_gemm at M = 1, the block sums added in block order (a 16-row tile split
+ * between warps hands its partial sums on in that order, so int8 mode stays bit-identical).
+ * 1 <= count <= 160, K % 512 == 0 and K <= 12288 per item; W, x (16-byte aligned), x_scale (int8
+ * mode, 4-byte aligned) and y (4-byte aligned) device pointers, caller-owned; no workspace; y
+ * must not overlap any item's x. Argument errors return before anything is enqueued. The hand-off
+ * between warps is a bounded wait: if it gives up, TERN_ETIMEOUT latches (tern_device_status) and
+ * the outputs are incomplete. */
 typedef struct {
   tern_fv5_matrix W;
   const void* x_dev;
