@@ -117,8 +117,12 @@ __global__ void __launch_bounds__(kThreads) k_fv5_gemm(const Fv5Params p) {
     }
   };
   uint4 cur[6], nxt[6];
-  load_chunk(0, cur);
-  load_chunk(1, nxt);
+  // the first two chunks' weights: int8 mode before the dependency wait, bf16 mode after its
+  // two-pass staging of the activations (issued first, they would hold up its reads)
+  if (MODE == 1) {
+    load_chunk(0, cur);
+    load_chunk(1, nxt);
+  }
   pdl_wait();
 
   // ---- stage the activation slice as int8 operand columns (as tern_gemv.cu) ----------------------
@@ -157,6 +161,8 @@ __global__ void __launch_bounds__(kThreads) k_fv5_gemm(const Fv5Params p) {
         *reinterpret_cast<uint4*>(smem + (4 * m + c) * RS + half_ofs(v)) =
             permute_i8_half(make_uint4(l[c][0], l[c][1], l[c][2], l[c][3]));
     }
+    load_chunk(0, cur);
+    load_chunk(1, nxt);
   }
   __syncthreads();
 
