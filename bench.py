@@ -953,9 +953,9 @@ def chain_row(stack, torch, hbm_peak):
     return out
 
 
-def small_m_sweep(stack, hbm_peak, Ms=(1, 2, 3, 4, 5, 7, 8, 12, 16)):
-    """One pass of M rows through the 8B stack + head per M (bf16): mma.sync kernels up to M = 4,
-    tcgen05 from M = 5. Then the stack alone in int8 mode at M = 5, 8, 16 on both kernel families
+def small_m_sweep(stack, hbm_peak, Ms=(1, 2, 3, 4, 5, 6, 7, 8, 12, 16)):
+    """One pass of M rows through the 8B stack + head per M (bf16): mma.sync kernels up to M = 8,
+    tcgen05 from M = 9. Then the stack alone in int8 mode at M = 5, 8, 16 on both kernel families
     (activations quantised once)."""
     out = {}
     for M in Ms:
