@@ -114,3 +114,28 @@ def test_list_and_prefill_argument_errors_before_launch(L):
     assert L.tern_gemm_prefill(ctypes.byref(m), 128, fake + 8, fake, None) == tg.TERN_EINVAL    # misaligned X
     assert L.tern_gemm_prefill(ctypes.byref(m), 128, fake, fake + 2, None) == tg.TERN_EINVAL    # misaligned Y
     assert L.tern_gemm_prefill(ctypes.byref(m), 128, None, fake, None) == tg.TERN_EINVAL
+
+
+def test_fv5_batch_argument_errors_before_launch(L):
+    """tern_fv5_gemv_batch rejects a bad list before it plans or launches anything."""
+    import bit_gemv_tern_b200 as tg
+    fake = 1 << 40                                      # never dereferenced: validation fails first
+    items = (tg._Fv5BatchItem * 2)()
+    for it in items:
+        it.W = tg._Fv5Matrix(64, 4096, fake, fake)
+        it.x, it.x_scale, it.y = fake, None, fake
+    assert L.tern_fv5_gemv_batch(None, 2, 0, None) == tg.TERN_EINVAL
+    assert L.tern_fv5_gemv_batch(items, 0, 0, None) == tg.TERN_ESHAPE                  # empty list
+    assert L.tern_fv5_gemv_batch(items, 161, 0, None) == tg.TERN_ESHAPE                # > 160 items
+    assert L.tern_fv5_gemv_batch(items, 2, 9, None) == tg.TERN_EINVAL                  # bad act
+    assert L.tern_fv5_gemv_batch(items, 2, 1, None) == tg.TERN_EINVAL                  # int8 needs x_scale
+    for bad in ((64, 4000), (64, 12800), (0, 4096)):                                   # K % 512, K > 12288, N < 1
+        items[1].W = tg._Fv5Matrix(bad[0], bad[1], fake, fake)
+        assert L.tern_fv5_gemv_batch(items, 2, 0, None) == tg.TERN_ESHAPE, bad
+    items[1].W = tg._Fv5Matrix(64, 4096, fake + 4, fake)                               # planes not 16-aligned
+    assert L.tern_fv5_gemv_batch(items, 2, 0, None) == tg.TERN_EINVAL
+    items[1].W = tg._Fv5Matrix(64, 4096, fake, fake)
+    items[1].x = fake + 4                                                              # x not 16-aligned
+    assert L.tern_fv5_gemv_batch(items, 2, 0, None) == tg.TERN_EINVAL
+    items[1].x, items[1].y = fake, None                                                # no output
+    assert L.tern_fv5_gemv_batch(items, 2, 0, None) == tg.TERN_EINVAL
