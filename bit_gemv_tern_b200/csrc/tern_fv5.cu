@@ -1,4 +1,5 @@
-// Five-valued weights in 256-weight blocks (FV5-style): packing and the GEMV / small-M product.
+// Five-valued weights in 256-weight blocks (FV5-style): packing, the GEMV / small-M product of one
+// matrix, and a list of matrices at M = 1 in one persistent launch (k_fv5_batch, below).
 //
 // The pages' shipped linear format (PyTorchKR review "Fermion Research, 3진 계열 포맷으로 직접
 // 학습한 Neutrino-1 모델군 3종 공개", section "FV5와 FV5B: llama.cpp 포크가 공개한 블록 구조")
