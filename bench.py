@@ -630,11 +630,11 @@ def _profile_batch(mode):
     return run
 
 
-def _profile_smallm(M):
+def _profile_smallm(M, tc=False):
     def run():
         st = Stack("8b", M=1, layers=4)
         sv = StackView(st, M)
-        return lambda: sv.launch_stack("bf16")
+        return lambda: sv.launch_stack("bf16", tc=tc)
     return run
 
 
@@ -730,11 +730,14 @@ def _profile_pack():
 #   fv5-8b-1layer-batched: one 8B layer's seven linears as five-valued weights (78.6 MB), M = 1, bf16,
 #                       in one tern_fv5_gemv_batch call
 #   pack-8b-1layer:     the int8 trits of one 8B layer's seven tensors (193 MB) in one batched call
+#   smallm-8b-4layers-m8-bf16(-tc): the 16 fused GEMVs of 4 layers at M = 8 in bf16 mode, on the
+#                       default (mma.sync) kernels or, with -tc, on the tcgen05 ones
 PROFILE_CASES = {
     "batch-8b-4layers-bf16": _profile_batch("bf16"),
     "batch-8b-4layers-int8": _profile_batch("int8"),
     "head-8b-bf16": _profile_head("bf16"),
     "smallm-8b-4layers-m8-bf16": _profile_smallm(8),
+    "smallm-8b-4layers-m8-bf16-tc": _profile_smallm(8, tc=True),
     "chain-8b-4layers-bf16": _profile_chain("bf16"),
     "prefill-8b-gate-m4096": _profile_prefill("gate"),
     "base3-8b-1layer": _profile_base3(),
